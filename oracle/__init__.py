@@ -1,0 +1,179 @@
+"""fp64 CPU oracle of the selective scan (S6) -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never loads it, and it imports nothing from them.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision, OpenMP over
+independent channels).  This module only compiles it with gcc and passes
+numpy float64 arrays to it.  Which page and section each step follows is
+stated in ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_HDR = os.path.join(_HERE, "oracle.h")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+_lock = threading.Lock()
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+
+def build(force: bool = False, src: str | None = None, out: str | None = None,
+          openmp: bool = True) -> str:
+    """Compile the oracle into a shared library with gcc; returns its path.
+
+    ``src``/``out`` let a test compile a modified copy of the source.
+    """
+    src = src or _SRC
+    out = out or _LIB_PATH
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= max(os.path.getmtime(src),
+                                             os.path.getmtime(_HDR))):
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-I", _HERE,
+           "-fno-fast-math", "-ffp-contract=off"]
+    if openmp:
+        cmd.append("-fopenmp")
+    tmp = out + f".tmp{os.getpid()}"
+    cmd += [src, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _bind(lib):
+    lib.oracle_combine_f64.argtypes = [ctypes.c_double] * 4 + [_D, _D]
+    lib.oracle_combine_f64.restype = None
+    lib.oracle_softplus_f64.argtypes = [ctypes.c_double]
+    lib.oracle_softplus_f64.restype = ctypes.c_double
+    lib.oracle_silu_f64.argtypes = [ctypes.c_double]
+    lib.oracle_silu_f64.restype = ctypes.c_double
+    lib.oracle_selective_scan_f64.argtypes = (
+        [_I64] * 4 + [_D] * 8 + [ctypes.c_int, _D, _D, _D])
+    lib.oracle_selective_scan_f64.restype = ctypes.c_int
+    lib.oracle_selective_state_update_f64.argtypes = (
+        [_I64] * 3 + [_D] * 9 + [ctypes.c_int, _D])
+    lib.oracle_selective_state_update_f64.restype = ctypes.c_int
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def load(path: str | None = None):
+    """Load (building if needed) the oracle library.  ``path`` loads another
+    compiled copy (used by the planted-mistake tests)."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(_D)
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def combine(a1, b1, a2, b2, lib=None):
+    """(a1, b1) then (a2, b2) -> (a1 a2, a2 b1 + b2)."""
+    lib = lib or load()
+    a = ctypes.c_double()
+    b = ctypes.c_double()
+    lib.oracle_combine_f64(a1, b1, a2, b2, ctypes.byref(a), ctypes.byref(b))
+    return a.value, b.value
+
+
+def softplus(x, lib=None):
+    lib = lib or load()
+    return lib.oracle_softplus_f64(float(x))
+
+
+def silu(z, lib=None):
+    lib = lib or load()
+    return lib.oracle_silu_f64(float(z))
+
+
+def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                   delta_softplus=True, h0=None, return_last_state=False,
+                   lib=None):
+    """Sequential fp64 selective scan.
+
+    u, delta, z: (batch, dim, L); B, C: (batch, N, L); A: (dim, N);
+    D, delta_bias: (dim,); h0: (batch, dim, N).  Returns y (batch, dim, L)
+    float64, and the final state when ``return_last_state``.
+    """
+    lib = lib or load()
+    u = _f64(u)
+    delta = _f64(delta)
+    A = _f64(A)
+    B = _f64(B)
+    C = _f64(C)
+    D = _f64(D)
+    z = _f64(z)
+    delta_bias = _f64(delta_bias)
+    h0 = _f64(h0)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    assert delta.shape == u.shape and A.shape == (dim, N)
+    assert B.shape == (batch, N, L) and C.shape == (batch, N, L)
+    y = np.empty((batch, dim, L), dtype=np.float64)
+    last = (np.empty((batch, dim, N), dtype=np.float64)
+            if return_last_state else None)
+    rc = lib.oracle_selective_scan_f64(
+        batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+        _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)),
+        _ptr(h0), _ptr(y), _ptr(last))
+    if rc != 0:
+        raise ValueError("oracle_selective_scan_f64 rejected the sizes")
+    return (y, last) if return_last_state else y
+
+
+def selective_state_update(state, x, dt, A, B, C, D=None, z=None,
+                           dt_bias=None, dt_softplus=True, lib=None):
+    """One fp64 decode step.  Returns (new_state, y); ``state`` is not
+    modified (a copy is updated)."""
+    lib = lib or load()
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    x = _f64(x)
+    dt = _f64(dt)
+    A = _f64(A)
+    B = _f64(B)
+    C = _f64(C)
+    D = _f64(D)
+    z = _f64(z)
+    dt_bias = _f64(dt_bias)
+    batch, dim, N = st.shape
+    y = np.empty((batch, dim), dtype=np.float64)
+    rc = lib.oracle_selective_state_update_f64(
+        batch, dim, N, _ptr(st), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)),
+        _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle_selective_state_update_f64 rejected sizes")
+    return st, y
+
+
+def num_threads(lib=None) -> int:
+    lib = lib or load()
+    return int(lib.oracle_num_threads())

@@ -1,0 +1,74 @@
+/*
+ * oracle.h -- fp64 CPU reference of the selective scan (S6).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link,
+ * load or call this code: only tests/, __graft_entry__.smoke() and the CPU
+ * baseline leg of bench.py use it.  It shares no header, helper, table or
+ * constant with the CUDA library and imports nothing from it.
+ *
+ * Every function computes the plain definition, in the order the sources
+ * state it, in double precision.  Layouts (all row-major, contiguous):
+ *   u, delta, z, y        (batch, dim, seqlen)
+ *   B, C                  (batch, dstate, seqlen)   shared by all channels
+ *   A                     (dim, dstate)
+ *   D, delta_bias         (dim)
+ *   h0, last_state        (batch, dim, dstate)
+ * Optional pointers may be NULL (D, z, delta_bias, h0 -> treated as 0 /
+ * "no gate"; last_state -> not written).
+ */
+#ifndef SSS48_ORACLE_H
+#define SSS48_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Composition of two fade-and-add steps, "step 1 then step 2":
+ * (a1, b1) then (a2, b2) = (a1*a2, a2*b1 + b2).
+ * Page "Mamba is attention... part 2", section "The relay". */
+void oracle_combine_f64(double a1, double b1, double a2, double b2,
+                        double *a_out, double *b_out);
+
+/* softplus(x) = log(1 + exp(x)), evaluated as max(x,0) + log1p(exp(-|x|)). */
+double oracle_softplus_f64(double x);
+
+/* silu(z) = z / (1 + exp(-z)). */
+double oracle_silu_f64(double z);
+
+/* Full selective scan, sequential over t (the recurrence as defined):
+ *   Delta_t = softplus(delta_t + delta_bias[d])   (or delta_t + delta_bias[d]
+ *                                                    when delta_softplus == 0)
+ *   h_t[n]  = exp(Delta_t * A[d,n]) * h_{t-1}[n] + Delta_t * B_t[n] * u_t
+ *   y_t     = sum_n C_t[n] * h_t[n] + D[d] * u_t
+ *   y_t    *= silu(z_t)                            (when z != NULL)
+ * with h_{-1} = h0 (or 0).  Returns 0, or -1 on a bad size. */
+int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
+                              int64_t seqlen, const double *u,
+                              const double *delta, const double *A,
+                              const double *B, const double *C,
+                              const double *D, const double *z,
+                              const double *delta_bias, int delta_softplus,
+                              const double *h0, double *y,
+                              double *last_state);
+
+/* One decode step (the same recurrence for a single t), state updated in
+ * place.  x, dt, z, y: (batch, dim); B, C: (batch, dstate);
+ * state: (batch, dim, dstate).  Returns 0, or -1 on a bad size. */
+int oracle_selective_state_update_f64(int64_t batch, int64_t dim,
+                                      int64_t dstate, double *state,
+                                      const double *x, const double *dt,
+                                      const double *A, const double *B,
+                                      const double *C, const double *D,
+                                      const double *z, const double *dt_bias,
+                                      int dt_softplus, double *y);
+
+/* Number of OpenMP threads the scan uses (1 when built without OpenMP). */
+int oracle_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif

@@ -1,0 +1,64 @@
+"""Planted mistakes in a copy of the oracle must each fail a pin.
+
+Each mutation below is a plausible slip in writing the recurrence (a wrong
+sign, a dropped term, a transposed operand, a wrong index).  The test
+compiles a mutated copy of oracle.c into a temporary library and checks that
+at least one pin in tests/pins.py rejects it.  The real oracle is untouched.
+"""
+import os
+import tempfile
+
+import pytest
+
+import oracle
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTATIONS = {
+    "combine_transposed": ("*b_out = a2 * b1 + b2;", "*b_out = a1 * b2 + b1;"),
+    "fade_applied_to_input": ("hp[n] = abar * hp[n] + bbar_u;",
+                              "hp[n] = hp[n] + abar * bbar_u;"),
+    "readout_uses_B": ("acc += Cb[n * seqlen + t] * hp[n];",
+                       "acc += Bb[n * seqlen + t] * hp[n];"),
+    "skip_dropped": ("double yt = acc + dskip * ut;", "double yt = acc;"),
+    "decay_sign": ("exp(dt * A[d * dstate + n])", "exp(-dt * A[d * dstate + n])"),
+    "B_index_transposed": ("dt * Bb[n * seqlen + t] * ut",
+                           "dt * Bb[t * dstate + n] * ut"),
+    "softplus_sign": ("log1p(exp(-ax))", "log1p(exp(ax))"),
+    "softplus_no_max": ("(x > 0.0 ? x : 0.0) + log1p", "0.0 + log1p"),
+    "silu_sign": ("z / (1.0 + exp(-z))", "z / (1.0 + exp(z))"),
+    "bias_ignored": ("double x = delta + bias;", "double x = delta;"),
+    "h0_ignored": ("hp[n] = h0 ? h0[(b * dim + d) * dstate + n] : 0.0;",
+                   "hp[n] = 0.0;"),
+    "input_without_step": ("const double bbar_u = dt * Bb[n * seqlen + t] * ut;",
+                           "const double bbar_u = Bb[n * seqlen + t] * ut;"),
+    "gate_before_skip": ("double yt = acc + dskip * ut;\n      if (zrow) yt *= oracle_silu_f64(zrow[t]);",
+                         "double yt = acc;\n      if (zrow) yt *= oracle_silu_f64(zrow[t]);\n      yt += dskip * ut;"),
+    "readout_before_update": (
+        "        hp[n] = abar * hp[n] + bbar_u;\n        /* [eq]: y_t = C_t h_t, with the state after the update. */\n        acc += Cb[n * seqlen + t] * hp[n];",
+        "        acc += Cb[n * seqlen + t] * hp[n];\n        hp[n] = abar * hp[n] + bbar_u;"),
+    "update_step_uses_input_twice": (
+        "step * B[b * dstate + n] * x[ch];", "step * B[b * dstate + n] * x[ch] * x[ch];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique/found"
+    with tempfile.TemporaryDirectory() as tmp:
+        path = os.path.join(tmp, "mutant.c")
+        with open(path, "w") as f:
+            f.write(src.replace(old, new))
+        so = oracle.build(force=True, src=path,
+                          out=os.path.join(tmp, "libmutant.so"), openmp=False)
+        lib = oracle.load(path=so)
+        failed = []
+        for pin in pins.ALL_PINS:
+            try:
+                pin(lib)
+            except AssertionError:
+                failed.append(pin.__name__)
+        assert failed, f"no pin caught the planted mistake {name}"
