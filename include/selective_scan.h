@@ -1,0 +1,168 @@
+/*
+ * selective_scan.h -- C ABI of the B200 selective-scan (S6) library
+ * (libsss48.so).
+ *
+ * What it computes.  For every batch row b, channel d in [0, dim) and state
+ * n in [0, dstate), over time t in [0, seqlen):
+ *
+ *   Delta_t = softplus(delta[b,d,t] + delta_bias[d])      (softplus optional)
+ *   h_t[n]  = exp(Delta_t * A[d,n]) * h_{t-1}[n] + Delta_t * B[b,n,t] * u[b,d,t]
+ *   y[b,d,t]= (sum_n C[b,n,t] * h_t[n] + D[d] * u[b,d,t]) * silu(z[b,d,t])
+ *
+ * with h_{-1} = h0 (or 0), silu(z) = z / (1 + e^-z), and the gate omitted
+ * when z is NULL.  Sources, by page and section:
+ *  - the recurrence and readout h_t = Abar h_{t-1} + Bbar u_t, y = C h + D u:
+ *    "The State That Must Remember Everything", Part 2, "The Equation";
+ *  - Abar = exp(Delta A), Bbar = Delta B (exponential-Euler discretisation):
+ *    same page, Part 7 "Mamba-3";
+ *  - Delta, B, C chosen per token: "State Space Models and the
+ *    Post-Transformer Era", section "The Selection Mechanism";
+ *  - the scan over time by composing fade-and-add pairs
+ *    (a1,b1) then (a2,b2) = (a1 a2, a2 b1 + b2): "Mamba is attention all you
+ *    really need, part 2", section "The relay";
+ *  - discretisation, scan and readout in one kernel, the state kept on chip
+ *    and only y written back: same page, "Keeping the pad on the desk", and
+ *    "The State That Must Remember Everything", "The Hardware-Aware Way Out";
+ *  - decode as a single state update: "Mamba: The State Space Models
+ *    Challenging the Transformer", section "What a state space model
+ *    actually is".
+ * The softplus step size, delta_bias and the silu(z) gate are not written
+ * out on the pages; they follow the standard Mamba parameterisation.
+ *
+ * Memory and ownership.  Every pointer is a device pointer owned by the
+ * caller.  The library never allocates or frees device or host memory.  All
+ * tensors are dense and row-major (C order) with the shapes given below.
+ * Work is enqueued on the caller's stream (a cudaStream_t passed as void*,
+ * NULL = legacy default stream) and is never synchronised, except in
+ * mss_scan_status().
+ *
+ * Errors.  Argument checks happen before any launch; a failing check returns
+ * MSS_ERR_INVALID_ARG or MSS_ERR_UNSUPPORTED and enqueues nothing.  A CUDA
+ * launch error returns MSS_ERR_CUDA.  Errors detected on the device (a
+ * bounded wait that ran out) are written to a status word inside the
+ * workspace and reported by mss_scan_status().
+ */
+#ifndef SSS48_SELECTIVE_SCAN_H
+#define SSS48_SELECTIVE_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MSS_ABI_VERSION 1
+
+typedef enum {
+  MSS_OK = 0,
+  MSS_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or dtype   */
+  MSS_ERR_UNSUPPORTED = 2, /* valid request this build does not implement   */
+  MSS_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed          */
+  MSS_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out            */
+  MSS_ERR_WORKSPACE = 5    /* workspace missing or smaller than required    */
+} mss_status;
+
+typedef enum { MSS_F32 = 0, MSS_BF16 = 1 } mss_dtype;
+
+/* Test-only flags (mss_scan_args.test_flags); 0 in production. */
+#define MSS_TESTFLAG_DROP_PUBLISH 0x1u /* one sequence chunk never publishes
+                                          its carry, so its successor's
+                                          bounded wait must run out         */
+
+/* Arguments of one forward scan.  Shapes:
+ *   u, delta, z, y   (batch, dim, seqlen)   in_dtype (y: out_dtype)
+ *   B, C             (batch, dstate, seqlen) in_dtype, shared by all channels
+ *   A                (dim, dstate)          fp32, expected <= 0
+ *   D, delta_bias    (dim)                  fp32
+ *   h0, last_state   (batch, dim, dstate)   fp32
+ * Optional (may be NULL): D (-> 0), z (-> no gate), delta_bias (-> 0),
+ * h0 (-> zero initial state), last_state (-> not written).
+ * Alignment: every pointer must be aligned to its element size; 16-byte
+ * alignment of u, delta, z, B, C, y with seqlen * element size a multiple
+ * of 16 enables the vectorised load path (otherwise a scalar path runs).
+ * h0 may alias last_state. */
+typedef struct mss_scan_args {
+  int64_t batch;   /* >= 1 */
+  int64_t dim;     /* >= 1, channels D */
+  int64_t dstate;  /* 1..16, states N per channel */
+  int64_t seqlen;  /* >= 1, sequence length L */
+  mss_dtype in_dtype;
+  mss_dtype out_dtype;
+  const void *u;
+  const void *delta;
+  const float *A;
+  const void *B;
+  const void *C;
+  const float *D;
+  const void *z;
+  const float *delta_bias;
+  int delta_softplus; /* 1: Delta = softplus(delta + bias); 0: delta + bias */
+  const float *h0;
+  void *y;
+  float *last_state;
+  void *workspace;        /* device, >= mss_scan_workspace_size() bytes,
+                             256-byte aligned; may be NULL if that is 0 */
+  size_t workspace_bytes;
+  int plan_splits;        /* 0 = automatic; > 0 forces the number of
+                             sequence chunks (tests use it to check that
+                             the result does not depend on the grouping) */
+  int plan_chunk_steps;   /* reserved, must be 0 */
+  unsigned test_flags;    /* 0 in production */
+  int64_t spin_timeout_ns;/* bound of each device-side wait; 0 = 1 s */
+} mss_scan_args;
+
+/* Bytes of device workspace the scan needs for these arguments (0 when the
+ * sequence is not split).  Reads only sizes, dtypes and plan fields. */
+mss_status mss_scan_workspace_size(const mss_scan_args *args, size_t *bytes);
+
+/* Forward selective scan: validates, plans the launch (sequence split,
+ * chunk length), clears the workspace flags with cudaMemsetAsync and
+ * launches on `stream`.  Writes y and, if requested, last_state. */
+mss_status mamba_selective_scan_fwd(const mss_scan_args *args, void *stream);
+
+/* Synchronises `stream`, then reports the device-side status of the last
+ * scan that used args->workspace (MSS_OK when the scan needed none). */
+mss_status mss_scan_status(const mss_scan_args *args, void *stream);
+
+/* Arguments of one decode step.  Shapes:
+ *   state            (batch, dim, dstate) fp32, updated in place
+ *   x, dt, z, y      (batch, dim)         in_dtype (y: out_dtype)
+ *   B, C             (batch, dstate)      in_dtype
+ *   A                (dim, dstate)        fp32
+ *   D, dt_bias       (dim)                fp32, optional
+ */
+typedef struct mss_update_args {
+  int64_t batch;
+  int64_t dim;
+  int64_t dstate; /* 1..16 */
+  mss_dtype in_dtype;
+  mss_dtype out_dtype;
+  float *state;
+  const void *x;
+  const void *dt;
+  const float *A;
+  const void *B;
+  const void *C;
+  const float *D;
+  const void *z;
+  const float *dt_bias;
+  int dt_softplus;
+  void *y;
+} mss_update_args;
+
+/* Single-token state update (decode): one step of the recurrence above for
+ * every (batch, channel), state updated in place, y written. */
+mss_status selective_state_update(const mss_update_args *args, void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *mss_status_string(mss_status status);
+
+/* MSS_ABI_VERSION of the loaded library. */
+int mss_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif

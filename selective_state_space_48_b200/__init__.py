@@ -1,0 +1,312 @@
+"""Python binding of the B200 selective-scan (S6) library.
+
+Argument marshalling only: torch tensors supply device memory and the
+current CUDA stream; every step of the computation runs in the CUDA kernels
+of ``_lib/libsss48.so`` behind the C ABI declared in
+``include/selective_scan.h``.  There is no CPU fallback: if the library is
+missing or no CUDA device is present, the calls raise.
+
+Functions mirror the C entry points:
+  mamba_selective_scan_fwd  -> selective_scan_fwd(...)
+  selective_state_update    -> selective_state_update(...)
+  mss_scan_workspace_size   -> scan_workspace_size(...)
+  mss_scan_status           -> scan_status(...)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import builder as _build
+
+LIB_PATH = _build.LIB_PATH
+
+MSS_OK = 0
+MSS_ERR_INVALID_ARG = 1
+MSS_ERR_UNSUPPORTED = 2
+MSS_ERR_CUDA = 3
+MSS_ERR_TIMEOUT = 4
+MSS_ERR_WORKSPACE = 5
+MSS_F32 = 0
+MSS_BF16 = 1
+MSS_TESTFLAG_DROP_PUBLISH = 0x1
+
+# every symbol include/selective_scan.h declares
+EXPORTED_SYMBOLS = (
+    "mss_scan_workspace_size",
+    "mamba_selective_scan_fwd",
+    "mss_scan_status",
+    "selective_state_update",
+    "mss_status_string",
+    "mss_abi_version",
+)
+
+
+class ScanArgs(ctypes.Structure):
+    """Mirror of ``mss_scan_args``."""
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("dim", ctypes.c_int64),
+        ("dstate", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("in_dtype", ctypes.c_int),
+        ("out_dtype", ctypes.c_int),
+        ("u", ctypes.c_void_p),
+        ("delta", ctypes.c_void_p),
+        ("A", ctypes.c_void_p),
+        ("B", ctypes.c_void_p),
+        ("C", ctypes.c_void_p),
+        ("D", ctypes.c_void_p),
+        ("z", ctypes.c_void_p),
+        ("delta_bias", ctypes.c_void_p),
+        ("delta_softplus", ctypes.c_int),
+        ("h0", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("last_state", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("plan_splits", ctypes.c_int),
+        ("plan_chunk_steps", ctypes.c_int),
+        ("test_flags", ctypes.c_uint),
+        ("spin_timeout_ns", ctypes.c_int64),
+    ]
+
+
+class UpdateArgs(ctypes.Structure):
+    """Mirror of ``mss_update_args``."""
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("dim", ctypes.c_int64),
+        ("dstate", ctypes.c_int64),
+        ("in_dtype", ctypes.c_int),
+        ("out_dtype", ctypes.c_int),
+        ("state", ctypes.c_void_p),
+        ("x", ctypes.c_void_p),
+        ("dt", ctypes.c_void_p),
+        ("A", ctypes.c_void_p),
+        ("B", ctypes.c_void_p),
+        ("C", ctypes.c_void_p),
+        ("D", ctypes.c_void_p),
+        ("z", ctypes.c_void_p),
+        ("dt_bias", ctypes.c_void_p),
+        ("dt_softplus", ctypes.c_int),
+        ("y", ctypes.c_void_p),
+    ]
+
+
+class MssError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library():
+    """Load libsss48.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"CUDA library {LIB_PATH} is missing; build it with "
+                    "`python -m selective_state_space_48_b200.builder`")
+            lib = ctypes.CDLL(LIB_PATH)
+            P = ctypes.POINTER
+            lib.mss_scan_workspace_size.argtypes = [P(ScanArgs), P(ctypes.c_size_t)]
+            lib.mss_scan_workspace_size.restype = ctypes.c_int
+            lib.mamba_selective_scan_fwd.argtypes = [P(ScanArgs), ctypes.c_void_p]
+            lib.mamba_selective_scan_fwd.restype = ctypes.c_int
+            lib.mss_scan_status.argtypes = [P(ScanArgs), ctypes.c_void_p]
+            lib.mss_scan_status.restype = ctypes.c_int
+            lib.selective_state_update.argtypes = [P(UpdateArgs), ctypes.c_void_p]
+            lib.selective_state_update.restype = ctypes.c_int
+            lib.mss_status_string.argtypes = [ctypes.c_int]
+            lib.mss_status_string.restype = ctypes.c_char_p
+            lib.mss_abi_version.argtypes = []
+            lib.mss_abi_version.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load_library().mss_status_string(int(code)).decode()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return MSS_F32
+    if t == torch.bfloat16:
+        return MSS_BF16
+    raise TypeError(f"unsupported dtype {t}; use float32 or bfloat16")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_cuda(name, t, dtype=None, shape=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                   delta_softplus=True, h0=None, y=None, last_state=None,
+                   workspace=None, plan_splits=0, test_flags=0,
+                   spin_timeout_ns=0) -> ScanArgs:
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    ind = u.dtype
+    _check_cuda("u", u, ind)
+    _check_cuda("delta", delta, ind, (batch, dim, L))
+    _check_cuda("A", A, torch.float32, (dim, N))
+    _check_cuda("B", B, ind, (batch, N, L))
+    _check_cuda("C", C, ind, (batch, N, L))
+    _check_cuda("D", D, torch.float32, (dim,))
+    _check_cuda("z", z, ind, (batch, dim, L))
+    _check_cuda("delta_bias", delta_bias, torch.float32, (dim,))
+    _check_cuda("h0", h0, torch.float32, (batch, dim, N))
+    _check_cuda("last_state", last_state, torch.float32, (batch, dim, N))
+    if y is not None:
+        _check_cuda("y", y, None, (batch, dim, L))
+    a = ScanArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = batch, dim, N, L
+    a.in_dtype = _dtype_code(ind)
+    a.out_dtype = _dtype_code(y.dtype) if y is not None else MSS_F32
+    a.u, a.delta, a.A, a.B, a.C = (_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C))
+    a.D, a.z, a.delta_bias = _ptr(D), _ptr(z), _ptr(delta_bias)
+    a.delta_softplus = 1 if delta_softplus else 0
+    a.h0, a.y, a.last_state = _ptr(h0), _ptr(y), _ptr(last_state)
+    if workspace is not None:
+        a.workspace = workspace.data_ptr()
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a.plan_splits = int(plan_splits)
+    a.plan_chunk_steps = 0
+    a.test_flags = int(test_flags)
+    a.spin_timeout_ns = int(spin_timeout_ns)
+    return a
+
+
+def scan_workspace_size(args: ScanArgs) -> int:
+    n = ctypes.c_size_t(0)
+    rc = load_library().mss_scan_workspace_size(ctypes.byref(args), ctypes.byref(n))
+    if rc != MSS_OK:
+        raise MssError(rc, "mss_scan_workspace_size")
+    return int(n.value)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    # torch allocations are 512-byte aligned, above the 256 the ABI needs
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                       delta_softplus=True, h0=None, return_last_state=False,
+                       out_dtype=torch.float32, y=None, last_state=None,
+                       workspace=None, stream=None, plan_splits=0,
+                       test_flags=0, spin_timeout_ns=0, check_status=False):
+    """Forward selective scan through ``mamba_selective_scan_fwd``.
+
+    u, delta, z: (batch, dim, L); B, C: (batch, N, L) (float32 or bfloat16,
+    all the same dtype); A: (dim, N), D, delta_bias: (dim,), h0:
+    (batch, dim, N) float32.  Returns y (batch, dim, L) in ``out_dtype``
+    (and the final state when ``return_last_state``).
+    """
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    if y is None:
+        y = torch.empty((batch, dim, L), dtype=out_dtype, device=u.device)
+    if return_last_state and last_state is None:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32,
+                                 device=u.device)
+    args = make_scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus,
+                          h0, y, last_state, None, plan_splits, test_flags,
+                          spin_timeout_ns)
+    if workspace is None:
+        workspace = alloc_workspace(scan_workspace_size(args), u.device)
+    if workspace is not None:
+        args.workspace = workspace.data_ptr()
+        args.workspace_bytes = workspace.numel() * workspace.element_size()
+    lib = load_library()
+    rc = lib.mamba_selective_scan_fwd(ctypes.byref(args), _stream_handle(stream))
+    if rc != MSS_OK:
+        raise MssError(rc, "mamba_selective_scan_fwd")
+    if check_status:
+        rc = lib.mss_scan_status(ctypes.byref(args), _stream_handle(stream))
+        if rc != MSS_OK:
+            raise MssError(rc, "mss_scan_status")
+    # keep the workspace alive until the stream has used it
+    if workspace is not None:
+        workspace.record_stream(stream or torch.cuda.current_stream())
+    return (y, last_state) if return_last_state else y
+
+
+def scan_status(args: ScanArgs, stream=None) -> int:
+    """Raw status code of the last scan that used ``args.workspace``."""
+    return load_library().mss_scan_status(ctypes.byref(args), _stream_handle(stream))
+
+
+def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                           dt_softplus=True, out_dtype=torch.float32, y=None,
+                           stream=None):
+    """One decode step through ``selective_state_update``; ``state``
+    (batch, dim, N) float32 is updated in place.  x, dt, z: (batch, dim);
+    B, C: (batch, N).  Returns y (batch, dim)."""
+    batch, dim, N = state.shape
+    ind = x.dtype
+    _check_cuda("state", state, torch.float32)
+    _check_cuda("x", x, ind, (batch, dim))
+    _check_cuda("dt", dt, ind, (batch, dim))
+    _check_cuda("A", A, torch.float32, (dim, N))
+    _check_cuda("B", B, ind, (batch, N))
+    _check_cuda("C", C, ind, (batch, N))
+    _check_cuda("D", D, torch.float32, (dim,))
+    _check_cuda("z", z, ind, (batch, dim))
+    _check_cuda("dt_bias", dt_bias, torch.float32, (dim,))
+    if y is None:
+        y = torch.empty((batch, dim), dtype=out_dtype, device=state.device)
+    _check_cuda("y", y, None, (batch, dim))
+    a = UpdateArgs()
+    a.batch, a.dim, a.dstate = batch, dim, N
+    a.in_dtype, a.out_dtype = _dtype_code(ind), _dtype_code(y.dtype)
+    a.state, a.x, a.dt = _ptr(state), _ptr(x), _ptr(dt)
+    a.A, a.B, a.C, a.D, a.z = _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z)
+    a.dt_bias = _ptr(dt_bias)
+    a.dt_softplus = 1 if dt_softplus else 0
+    a.y = _ptr(y)
+    rc = load_library().selective_state_update(ctypes.byref(a), _stream_handle(stream))
+    if rc != MSS_OK:
+        raise MssError(rc, "selective_state_update")
+    return y
+
+
+def build(force: bool = False) -> str:
+    return _build.build(force=force)
+
+
+__all__ = [
+    "selective_scan_fwd", "selective_state_update", "scan_workspace_size",
+    "scan_status", "make_scan_args", "load_library", "status_string",
+    "MssError", "ScanArgs", "UpdateArgs", "EXPORTED_SYMBOLS", "build",
+]

@@ -1,0 +1,251 @@
+// api.cu -- C ABI of the selective-scan library: argument checks, launch
+// planning and dispatch.  Declarations and their documentation are in
+// include/selective_scan.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "scan_fwd.cuh"
+#include "selective_scan.h"
+
+using namespace sss48;
+
+namespace {
+
+constexpr int64_t kMinChunk = 1024;  // shortest automatic sequence chunk
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void *p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+size_t esize(mss_dtype t) { return t == MSS_BF16 ? 2 : 4; }
+
+bool valid_dtype(mss_dtype t) { return t == MSS_F32 || t == MSS_BF16; }
+
+struct Plan {
+  int groups;
+  int ch_tiles;
+  int64_t tiles;
+  int splits;
+  int64_t chunk;
+  size_t workspace;
+};
+
+int device_sms(int dev) {
+  static int cache[kMaxDevices] = {0};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess ||
+        n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+int blocks_per_sm(int dev, int in_bf16, int out_bf16, int groups) {
+  static int cache[kMaxDevices][2][2][5] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= kMaxDevices) return 1;
+  int &c = cache[dev][in_bf16][out_bf16][groups];
+  if (c == 0) c = scan_blocks_per_sm(in_bf16, out_bf16, 1, groups, 0);
+  return c;
+}
+
+mss_status check_scan_args(const mss_scan_args *a) {
+  if (!a) return MSS_ERR_INVALID_ARG;
+  if (a->batch < 1 || a->dim < 1 || a->seqlen < 1 || a->dstate < 1)
+    return MSS_ERR_INVALID_ARG;
+  if (a->dstate > kMaxStates) return MSS_ERR_UNSUPPORTED;
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
+    return MSS_ERR_INVALID_ARG;
+  if (a->plan_splits < 0 || a->plan_chunk_steps != 0 || a->spin_timeout_ns < 0)
+    return MSS_ERR_INVALID_ARG;
+  // sizes whose element counts or grid would overflow
+  const int64_t lim = int64_t(1) << 40;
+  if (a->batch > lim / a->dim || a->batch * a->dim > lim / a->seqlen)
+    return MSS_ERR_UNSUPPORTED;
+  if (!a->u || !a->delta || !a->A || !a->B || !a->C || !a->y)
+    return MSS_ERR_INVALID_ARG;
+  const size_t ei = esize(a->in_dtype), eo = esize(a->out_dtype);
+  if (!aligned(a->u, ei) || !aligned(a->delta, ei) || !aligned(a->B, ei) ||
+      !aligned(a->C, ei) || (a->z && !aligned(a->z, ei)) ||
+      !aligned(a->y, eo) || !aligned(a->A, 4) || (a->D && !aligned(a->D, 4)) ||
+      (a->delta_bias && !aligned(a->delta_bias, 4)) ||
+      (a->h0 && !aligned(a->h0, 4)) ||
+      (a->last_state && !aligned(a->last_state, 4)))
+    return MSS_ERR_INVALID_ARG;
+  return MSS_OK;
+}
+
+mss_status make_plan(const mss_scan_args *a, Plan *pl) {
+  pl->groups = static_cast<int>((a->dstate + 3) / 4);
+  pl->ch_tiles = static_cast<int>((a->dim + kChannelsPerBlock - 1) /
+                                  kChannelsPerBlock);
+  pl->tiles = a->batch * pl->ch_tiles;
+  int64_t want = a->plan_splits;
+  if (want == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MSS_ERR_CUDA;
+    const int64_t target =
+        int64_t(device_sms(dev)) *
+        blocks_per_sm(dev, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16,
+                      pl->groups);
+    if (pl->tiles * 4 >= target * 3) {
+      want = 1;
+    } else {
+      want = (target + pl->tiles - 1) / pl->tiles;
+      want = std::min<int64_t>(want, std::max<int64_t>(1, a->seqlen / kMinChunk));
+    }
+  }
+  want = std::max<int64_t>(1, std::min<int64_t>(want, a->seqlen));
+  int64_t chunk = (a->seqlen + want - 1) / want;
+  chunk = ((chunk + kTimeBlock - 1) / kTimeBlock) * kTimeBlock;
+  pl->chunk = chunk;
+  pl->splits = static_cast<int>((a->seqlen + chunk - 1) / chunk);
+  if (pl->tiles * pl->splits > int64_t(INT32_MAX)) return MSS_ERR_UNSUPPORTED;
+  pl->workspace = scan_workspace_bytes(pl->tiles, pl->splits, pl->groups);
+  return MSS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mss_status mss_scan_workspace_size(const mss_scan_args *args, size_t *bytes) {
+  if (!bytes) return MSS_ERR_INVALID_ARG;
+  mss_status st = check_scan_args(args);
+  if (st != MSS_OK) return st;
+  Plan pl;
+  st = make_plan(args, &pl);
+  if (st != MSS_OK) return st;
+  *bytes = pl.workspace;
+  return MSS_OK;
+}
+
+mss_status mamba_selective_scan_fwd(const mss_scan_args *a, void *stream) {
+  mss_status st = check_scan_args(a);
+  if (st != MSS_OK) return st;
+  Plan pl;
+  st = make_plan(a, &pl);
+  if (st != MSS_OK) return st;
+  if (pl.workspace > 0 &&
+      (!a->workspace || a->workspace_bytes < pl.workspace ||
+       !aligned(a->workspace, 256)))
+    return MSS_ERR_WORKSPACE;
+
+  ScanParams p{};
+  p.batch = a->batch;
+  p.dim = a->dim;
+  p.dstate = a->dstate;
+  p.seqlen = a->seqlen;
+  p.u = a->u;
+  p.delta = a->delta;
+  p.A = a->A;
+  p.B = a->B;
+  p.C = a->C;
+  p.D = a->D;
+  p.z = a->z;
+  p.delta_bias = a->delta_bias;
+  p.softplus = a->delta_softplus ? 1 : 0;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.last_state = a->last_state;
+  p.chunk = pl.chunk;
+  p.splits = pl.splits;
+  p.ch_tiles = pl.ch_tiles;
+  p.tiles = pl.tiles;
+  p.test_flags = a->test_flags;
+  p.spin_timeout_ns = a->spin_timeout_ns;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pl.splits > 1) {
+    scan_bind_workspace(p, a->workspace, pl.groups);
+    if (cudaMemsetAsync(a->workspace, 0,
+                        scan_workspace_clear_bytes(pl.tiles, pl.splits),
+                        s) != cudaSuccess)
+      return MSS_ERR_CUDA;
+  }
+  if (launch_scan_fwd(p, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16,
+                      a->z != nullptr, s) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  return MSS_OK;
+}
+
+mss_status mss_scan_status(const mss_scan_args *a, void *stream) {
+  mss_status st = check_scan_args(a);
+  if (st != MSS_OK) return st;
+  Plan pl;
+  st = make_plan(a, &pl);
+  if (st != MSS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MSS_ERR_CUDA;
+  if (pl.splits <= 1) return MSS_OK;
+  if (!a->workspace || a->workspace_bytes < pl.workspace)
+    return MSS_ERR_WORKSPACE;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, a->workspace, sizeof(word), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return MSS_ERR_CUDA;
+  if (word & kStatusTimeout) return MSS_ERR_TIMEOUT;
+  return MSS_OK;
+}
+
+mss_status selective_state_update(const mss_update_args *a, void *stream) {
+  if (!a) return MSS_ERR_INVALID_ARG;
+  if (a->batch < 1 || a->dim < 1 || a->dstate < 1) return MSS_ERR_INVALID_ARG;
+  if (a->dstate > kMaxStates) return MSS_ERR_UNSUPPORTED;
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
+    return MSS_ERR_INVALID_ARG;
+  if (a->batch > (int64_t(1) << 40) / a->dim) return MSS_ERR_UNSUPPORTED;
+  if (!a->state || !a->x || !a->dt || !a->A || !a->B || !a->C || !a->y)
+    return MSS_ERR_INVALID_ARG;
+  const size_t ei = esize(a->in_dtype), eo = esize(a->out_dtype);
+  if (!aligned(a->state, 4) || !aligned(a->x, ei) || !aligned(a->dt, ei) ||
+      !aligned(a->B, ei) || !aligned(a->C, ei) || (a->z && !aligned(a->z, ei)) ||
+      !aligned(a->y, eo) || !aligned(a->A, 4) || (a->D && !aligned(a->D, 4)) ||
+      (a->dt_bias && !aligned(a->dt_bias, 4)))
+    return MSS_ERR_INVALID_ARG;
+  UpdateParams p{};
+  p.batch = a->batch;
+  p.dim = a->dim;
+  p.dstate = a->dstate;
+  p.state = a->state;
+  p.x = a->x;
+  p.dt = a->dt;
+  p.A = a->A;
+  p.B = a->B;
+  p.C = a->C;
+  p.D = a->D;
+  p.z = a->z;
+  p.dt_bias = a->dt_bias;
+  p.softplus = a->dt_softplus ? 1 : 0;
+  p.y = a->y;
+  if (launch_state_update(p, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16,
+                          static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  return MSS_OK;
+}
+
+const char *mss_status_string(mss_status s) {
+  switch (s) {
+    case MSS_OK: return "MSS_OK";
+    case MSS_ERR_INVALID_ARG: return "MSS_ERR_INVALID_ARG";
+    case MSS_ERR_UNSUPPORTED: return "MSS_ERR_UNSUPPORTED";
+    case MSS_ERR_CUDA: return "MSS_ERR_CUDA";
+    case MSS_ERR_TIMEOUT: return "MSS_ERR_TIMEOUT";
+    case MSS_ERR_WORKSPACE: return "MSS_ERR_WORKSPACE";
+  }
+  return "MSS_ERR_UNKNOWN";
+}
+
+int mss_abi_version(void) { return MSS_ABI_VERSION; }
+
+}  // extern "C"

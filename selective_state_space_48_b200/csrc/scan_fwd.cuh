@@ -1,0 +1,81 @@
+// scan_fwd.cuh -- launch interface between the C ABI layer and the
+// forward-scan / state-update kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sss48 {
+
+// Channels per thread block (one per lane) and states per lane.  A block has
+// one warp per group of kStatesPerLane states, so every lane of a warp owns
+// the same state indices and reads B_t[n], C_t[n] at warp-uniform addresses.
+constexpr int kChannelsPerBlock = 32;
+constexpr int kStatesPerLane = 4;
+constexpr int kMaxStates = 16;
+constexpr int kTimeBlock = 32;  // timesteps staged in shared memory at once
+
+struct ScanParams {
+  int64_t batch, dim, dstate, seqlen;
+  const void *u, *delta;
+  const float *A;
+  const void *B, *C;
+  const float *D;
+  const void *z;
+  const float *delta_bias;
+  int softplus;
+  const float *h0;
+  void *y;
+  float *last_state;
+  // launch plan
+  int64_t chunk;   // timesteps per sequence chunk (multiple of kTimeBlock)
+  int splits;      // number of sequence chunks
+  int ch_tiles;    // ceil(dim / kChannelsPerBlock)
+  int64_t tiles;   // batch * ch_tiles
+  // split-mode workspace
+  unsigned *status;
+  unsigned *ticket;
+  unsigned *flags;
+  float *agg;      // per item: decay product P then local end state e
+  float *incl;     // per item: true state at the end of the chunk
+  unsigned test_flags;
+  int64_t spin_timeout_ns;
+};
+
+// Workspace bytes for `splits` chunks over `tiles` tiles with `groups`
+// state groups (0 when splits == 1).
+size_t scan_workspace_bytes(int64_t tiles, int splits, int groups);
+
+// Carves the workspace into the fields of `p`.
+void scan_bind_workspace(ScanParams &p, void *ws, int groups);
+
+// Bytes of the header + flag region that must be zero before a launch.
+size_t scan_workspace_clear_bytes(int64_t tiles, int splits);
+
+// Thread blocks of the scan kernel that fit on one SM (for planning).
+int scan_blocks_per_sm(int in_bf16, int out_bf16, int has_z, int groups,
+                       int split);
+
+cudaError_t launch_scan_fwd(const ScanParams &p, int in_bf16, int out_bf16,
+                            int has_z, cudaStream_t stream);
+
+struct UpdateParams {
+  int64_t batch, dim, dstate;
+  float *state;
+  const void *x, *dt;
+  const float *A;
+  const void *B, *C;
+  const float *D;
+  const void *z;
+  const float *dt_bias;
+  int softplus;
+  void *y;
+};
+
+cudaError_t launch_state_update(const UpdateParams &p, int in_bf16,
+                                int out_bf16, cudaStream_t stream);
+
+constexpr unsigned kStatusTimeout = 1u;
+
+}  // namespace sss48

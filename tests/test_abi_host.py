@@ -1,0 +1,158 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute launched).
+
+* the library builds and loads, and exports every function the header
+  declares;
+* the ctypes mirrors of the argument structs have the C layout;
+* argument checks reject bad calls before touching the device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import selective_state_space_48_b200 as sss
+from selective_state_space_48_b200 import builder as sbuild
+
+HEADER_DIR = sbuild.INCLUDE
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sbuild.build()
+    return sss.load_library()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(HEADER_DIR):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b([A-Za-z_]\w*)\s*\([^;{]*\)\s*;",
+                             text, flags=re.M):
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for sym in sss.EXPORTED_SYMBOLS:
+        assert sym in names
+    assert set(names) == set(sss.EXPORTED_SYMBOLS), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", sbuild.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for sym in declared_functions():
+        assert sym in exported, sym
+        assert getattr(lib, sym) is not None
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.mss_abi_version() == 1
+    for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
+                       (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
+                       (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
+        assert sss.status_string(code) == name
+
+
+def test_struct_layout_matches_c():
+    """Compile a C program that prints sizeof/offsetof of both structs."""
+    fields_scan = [f[0] for f in sss.ScanArgs._fields_]
+    fields_upd = [f[0] for f in sss.UpdateArgs._fields_]
+    src = ['#include <stdio.h>', '#include <stddef.h>', '#include "selective_scan.h"',
+           'int main(void) {',
+           'printf("%zu\\n", sizeof(mss_scan_args));']
+    src += [f'printf("%zu\\n", offsetof(mss_scan_args, {f}));' for f in fields_scan]
+    src += ['printf("%zu\\n", sizeof(mss_update_args));']
+    src += [f'printf("%zu\\n", offsetof(mss_update_args, {f}));' for f in fields_upd]
+    src += ['return 0; }']
+    with tempfile.TemporaryDirectory() as tmp:
+        c = os.path.join(tmp, "layout.c")
+        exe = os.path.join(tmp, "layout")
+        open(c, "w").write("\n".join(src))
+        subprocess.run(["gcc", "-I", HEADER_DIR, c, "-o", exe], check=True)
+        vals = [int(v) for v in subprocess.run([exe], capture_output=True, text=True,
+                                               check=True).stdout.split()]
+    want = [ctypes.sizeof(sss.ScanArgs)] + [getattr(sss.ScanArgs, f).offset for f in fields_scan]
+    want += [ctypes.sizeof(sss.UpdateArgs)] + [getattr(sss.UpdateArgs, f).offset for f in fields_upd]
+    assert vals == want
+
+
+def _args(**kw):
+    a = sss.ScanArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = 2, 40, 16, 4096
+    a.in_dtype, a.out_dtype = sss.MSS_BF16, sss.MSS_F32
+    fake = 0x10000
+    a.u = a.delta = a.A = a.B = a.C = a.y = fake
+    a.plan_splits = 4
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _ws(lib, a):
+    n = ctypes.c_size_t(123)
+    rc = lib.mss_scan_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_follows_plan(lib):
+    rc, n = _ws(lib, _args(plan_splits=1))
+    assert rc == sss.MSS_OK and n == 0
+    rc, n4 = _ws(lib, _args(plan_splits=4))
+    assert rc == sss.MSS_OK and n4 > 0
+    rc, n8 = _ws(lib, _args(plan_splits=8))
+    assert rc == sss.MSS_OK and n8 > n4
+    # 2 batch rows x 2 channel tiles x 8 chunks, each with (P, e) and the
+    # inclusive state for 32 channels x 16 states
+    items = 2 * 2 * 8
+    assert n8 >= items * 32 * 16 * 3 * 4
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(dim=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(seqlen=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(dstate=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(dstate=17), sss.MSS_ERR_UNSUPPORTED),
+    (dict(in_dtype=7), sss.MSS_ERR_INVALID_ARG),
+    (dict(out_dtype=-1), sss.MSS_ERR_INVALID_ARG),
+    (dict(u=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(y=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(A=0x10002), sss.MSS_ERR_INVALID_ARG),      # fp32 A misaligned
+    (dict(u=0x10001), sss.MSS_ERR_INVALID_ARG),      # bf16 u misaligned
+    (dict(plan_splits=-1), sss.MSS_ERR_INVALID_ARG),
+    (dict(plan_chunk_steps=64), sss.MSS_ERR_INVALID_ARG),
+    (dict(spin_timeout_ns=-5), sss.MSS_ERR_INVALID_ARG),
+])
+def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
+    a = _args(**kw)
+    rc, _ = _ws(lib, a)
+    assert rc == code
+    # the forward call applies the same checks and launches nothing
+    assert lib.mamba_selective_scan_fwd(ctypes.byref(a), None) == code
+
+
+def test_missing_workspace_is_reported(lib):
+    a = _args(plan_splits=4)
+    assert lib.mamba_selective_scan_fwd(ctypes.byref(a), None) == sss.MSS_ERR_WORKSPACE
+    a.workspace = 0x10000
+    a.workspace_bytes = 16
+    assert lib.mamba_selective_scan_fwd(ctypes.byref(a), None) == sss.MSS_ERR_WORKSPACE
+
+
+def test_null_args_rejected(lib):
+    n = ctypes.c_size_t()
+    assert lib.mss_scan_workspace_size(None, ctypes.byref(n)) == sss.MSS_ERR_INVALID_ARG
+    assert lib.mamba_selective_scan_fwd(None, None) == sss.MSS_ERR_INVALID_ARG
+    assert lib.selective_state_update(None, None) == sss.MSS_ERR_INVALID_ARG
+    u = sss.UpdateArgs()
+    u.batch, u.dim, u.dstate = 1, 1, 17
+    assert lib.selective_state_update(ctypes.byref(u), None) == sss.MSS_ERR_UNSUPPORTED
