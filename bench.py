@@ -1,0 +1,480 @@
+#!/usr/bin/env python
+"""Benchmark of the forward selective scan (S6) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one full forward scan (softplus step size, discretisation,
+recurrence, C readout, D skip, silu(z) gate) over one batch of the
+Mamba-130M-shaped layer workload (batch 8, D 1536, N 16, L 2048, bf16
+inputs, fp32 state and output) with inputs resident in HBM.  W untimed steps,
+then exactly K steps bracketed by a barrier and a device synchronise on both
+sides, timed with CUDA events on the launching stream; the time is the max
+over ranks.  The working set (253 MB of inputs and outputs) is larger than
+the 126 MB L2, so no step finds the previous step's data in L2.
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+workload on its own GPU (the scan needs no exchange between GPUs) and
+``value`` is the bytes moved by all ranks divided by the slowest rank's time.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+instead (the only other place the bench runs it), on a bounded sample of the
+same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import faulthandler
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = ("selective-scan HBM GB/s (fraction of B200 peak); "
+          "B·D·L·N state-updates/s")
+DEFAULT_WORKLOAD = "mamba130m-layer"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+
+REASON_BITS = [
+    (0x1, "gpu_idle"), (0x2, "applications_clocks_setting"),
+    (0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x10, "sync_boost"),
+    (0x20, "sw_thermal_slowdown"), (0x40, "hw_thermal_slowdown"),
+    (0x80, "hw_power_brake_slowdown"), (0x100, "display_clock_setting"),
+]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=[w.name for w in workloads.WORKLOADS])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU work of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- helpers
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_48_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(csrc, "*.cu")) +
+                    glob.glob(os.path.join(csrc, "*.cuh"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when
+    the kernels changed since the counters were taken."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("kernel_source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def workload_config(w) -> dict:
+    return {"workload": w.name, "batch": w.batch, "dim": w.dim,
+            "dstate": w.dstate, "seqlen": w.seqlen, "in_dtype": w.in_dtype,
+            "out_dtype": "f32", "gate": "silu(z)" if w.has_z else "none",
+            "l2": (f"inputs+outputs {w.algorithmic_bytes() / 1e6:.0f} MB per "
+                   "step, larger than the 126 MB L2; no flush")}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, cuda_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            handle = None
+            uuid = getattr(torch.cuda.get_device_properties(cuda_index), "uuid", None)
+            if isinstance(uuid, str) and uuid:
+                # NVML wants the "GPU-" prefixed form; only a str is passed on
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(
+                        uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+                except Exception:
+                    handle = None
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(int(cuda_index))
+            self._handle = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self._handle, n.NVML_CLOCK_SM)
+                reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": [name for bit, name in REASON_BITS if bits & bit],
+                "samples": len(self.samples)}
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max over ranks (all ranks call this in the same order)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def whole_job_gbs(bytes_per_step: int, steps: int, world: int,
+                  max_ms: float) -> float:
+    return bytes_per_step * steps * world / (max_ms * 1e-3) / 1e9
+
+
+# ------------------------------------------------------- oracle (CPU) legs
+
+
+def _oracle_sample_inputs(inp: dict, channels: int, w):
+    """First `channels` channels in (b, d) order, as float64 host arrays,
+    grouped per batch row (contiguous d ranges)."""
+    groups = []
+    left = channels
+    b = 0
+    while left > 0 and b < w.batch:
+        nd = min(left, w.dim)
+        sl = lambda t: None if t is None else t[b:b + 1, :nd].detach().cpu().double().numpy()
+        pd = lambda t: None if t is None else t[:nd].detach().cpu().double().numpy()
+        groups.append(dict(u=sl(inp["u"]), delta=sl(inp["delta"]), z=sl(inp["z"]),
+                           B=inp["B"][b:b + 1].detach().cpu().double().numpy(),
+                           C=inp["C"][b:b + 1].detach().cpu().double().numpy(),
+                           A=inp["A"][:nd].detach().cpu().double().numpy(),
+                           D=pd(inp["D"]), delta_bias=pd(inp["delta_bias"])))
+        left -= nd
+        b += 1
+    return groups
+
+
+def _run_oracle_groups(groups, w):
+    import oracle
+    for g in groups:
+        oracle.selective_scan(g["u"], g["delta"], g["A"], g["B"], g["C"],
+                              D=g["D"], z=g["z"], delta_bias=g["delta_bias"],
+                              delta_softplus=w.softplus)
+
+
+def _calibrate_oracle(inp, w) -> float:
+    """Seconds of wall time per channel with all oracle threads busy."""
+    import oracle
+    threads = oracle.num_threads()
+    probe = max(1, min(threads, w.batch * w.dim))
+    groups = _oracle_sample_inputs(inp, probe, w)
+    t0 = time.perf_counter()
+    _run_oracle_groups(groups, w)
+    dt = time.perf_counter() - t0
+    return dt / probe
+
+
+def oracle_timing(inp, w, seconds: float, steps: int = 1, warmup: int = 0):
+    """Time the oracle on a bounded sample; returns (GB/s, updates/s,
+    channels per step, threads, total seconds)."""
+    import oracle
+    threads = oracle.num_threads()
+    per_ch = _calibrate_oracle(inp, w)
+    per_step = seconds / max(1, steps + warmup)
+    ch = int(max(1, min(w.batch * w.dim, round(per_step / per_ch))))
+    groups = _oracle_sample_inputs(inp, ch, w)
+    for _ in range(warmup):
+        _run_oracle_groups(groups, w)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        _run_oracle_groups(groups, w)
+    total = time.perf_counter() - t0
+    share = ch / (w.batch * w.dim)
+    gbs = w.algorithmic_bytes() * share * steps / total / 1e9
+    ups = w.state_updates * share * steps / total
+    return gbs, ups, ch, threads, total
+
+
+# ------------------------------------------------------------- our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import selective_state_space_48_b200 as sss
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.BY_NAME[args.workload]
+    inp = workloads.make_inputs(w, device=dev)
+    y = torch.empty((w.batch, w.dim, w.seqlen), dtype=torch.float32, device=dev)
+    sargs = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"],
+                               inp["C"], D=inp["D"], z=inp["z"],
+                               delta_bias=inp["delta_bias"],
+                               delta_softplus=w.softplus, y=y)
+    ws_bytes = sss.scan_workspace_size(sargs)
+    ws = sss.alloc_workspace(ws_bytes, dev)
+    if ws is not None:
+        sargs.workspace = ws.data_ptr()
+        sargs.workspace_bytes = ws_bytes
+    lib = sss.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    argp = ctypes.byref(sargs)
+
+    def step():
+        rc = lib.mamba_selective_scan_fwd(argp, sh)
+        if rc != 0:
+            raise sss.MssError(rc, "mamba_selective_scan_fwd")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if lib.mss_scan_status(argp, sh) != 0:
+        raise RuntimeError("device-side status error during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(world)
+    local_ms = t_start.elapsed_time(t_end)
+    kernel_ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    max_ms = reduce_max(local_ms, world)
+    max_kernel_ms = reduce_max(kernel_ms, world)
+    if lib.mss_scan_status(argp, sh) != 0:
+        raise RuntimeError("device-side status error in the timed region")
+
+    bytes_step = w.algorithmic_bytes()
+    value = whole_job_gbs(bytes_step, K, world, max_ms)
+    updates = w.state_updates * K * world / (max_ms * 1e-3)
+
+    # ---- end to end through the public API with host buffers
+    names = ["u", "delta", "z", "B", "C", "A", "D", "delta_bias"]
+    host = {k: inp[k].detach().cpu().pin_memory() for k in names if inp[k] is not None}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = y.numel() * y.element_size()
+    Ke = max(1, args.e2e_steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(Ke):
+        for k, t in host.items():
+            inp[k].copy_(t, non_blocking=True)
+        sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"],
+                               inp["C"], D=inp["D"], z=inp["z"],
+                               delta_bias=inp["delta_bias"],
+                               delta_softplus=w.softplus, y=y, workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), world)
+    e2e_value = whole_job_gbs(bytes_step, Ke, world, e2e_ms)
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, ups, ch, threads, total = oracle_timing(inp, w, args.cpu_seconds)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "state_updates_per_s": ups,
+               "sample": (f"{ch} of {w.batch * w.dim} channels, full length "
+                          f"L={w.seqlen}, one pass, {total:.1f} s wall, "
+                          "fp64 C oracle with OpenMP over channels; GB/s = the "
+                          "sample's share of the step's algorithmic bytes / time")}
+
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_step / (max_kernel_ms * 1e-3) / 1e9
+    clk = clocks.summary()
+    sm_mhz = clk.get("sm_mhz") or 1965.0
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": max_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": workload_config(w),
+        "state_updates_per_s": updates,
+        "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
+        "frac_of_measured_hbm": value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": peak_kind,
+                     "traffic": profiled_traffic(w.name),
+                     "algorithmic_bytes_per_launch": bytes_step,
+                     "kernel_ms": max_kernel_ms},
+        "exp_unit": {"bound": "alu",
+                     "achieved_gexp_s": w.state_updates / (max_kernel_ms * 1e-3) / 1e9,
+                     "mufu_peak_gexp_s": 16 * 148 * sm_mhz / 1e3,
+                     "note": "one exp per state update; MUFU ex2 16/clk/SM"},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke},
+        "gpu_launches": K,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                   "reasons": clk["reasons"], "samples": clk["samples"]},
+        "kernel_source_hash": kernel_source_hash(),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
+# -------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    """The fp64 oracle as it stands, on this host's cores, each step a
+    bounded sample (a share of the channels, full length) of the workload."""
+    w = workloads.BY_NAME[args.workload]
+    inp = workloads.make_inputs(w, device="cpu")
+    budget = min(120.0, max(20.0, 3.0 * (args.steps + args.warmup)))
+    gbs, ups, ch, threads, total = oracle_timing(inp, w, budget, steps=args.steps,
+                                                 warmup=args.warmup)
+    sample = (f"{ch} of {w.batch * w.dim} channels per step, full length "
+              f"L={w.seqlen}; fp64 C oracle, OpenMP over channels")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": gbs,
+        "unit": "GB/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total * 1e3 / max(1, args.steps),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(w),
+        "state_updates_per_s": ups,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    faulthandler.enable()
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

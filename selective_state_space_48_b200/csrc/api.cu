@@ -56,7 +56,7 @@ int blocks_per_sm(int dev, int in_bf16, int out_bf16, int groups) {
   std::lock_guard<std::mutex> lock(mu);
   if (dev < 0 || dev >= kMaxDevices) return 1;
   int &c = cache[dev][in_bf16][out_bf16][groups];
-  if (c == 0) c = scan_blocks_per_sm(in_bf16, out_bf16, 1, groups, 0);
+  if (c == 0) c = scan_blocks_per_sm(in_bf16, out_bf16, groups);
   return c;
 }
 
@@ -93,13 +93,17 @@ mss_status make_plan(const mss_scan_args *a, Plan *pl) {
   pl->tiles = a->batch * pl->ch_tiles;
   int64_t want = a->plan_splits;
   if (want == 0) {
+    // Split the sequence only when there are fewer channel tiles than SMs:
+    // a chunk that does not start the sequence pays a carry correction whose
+    // length grows with the state's memory, so whole-sequence tiles are
+    // preferred whenever they can occupy the chip.
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MSS_ERR_CUDA;
+    const int64_t sms = device_sms(dev);
     const int64_t target =
-        int64_t(device_sms(dev)) *
-        blocks_per_sm(dev, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16,
-                      pl->groups);
-    if (pl->tiles * 4 >= target * 3) {
+        sms * blocks_per_sm(dev, a->in_dtype == MSS_BF16,
+                            a->out_dtype == MSS_BF16, pl->groups);
+    if (pl->tiles >= sms) {
       want = 1;
     } else {
       want = (target + pl->tiles - 1) / pl->tiles;
@@ -172,9 +176,12 @@ mss_status mamba_selective_scan_fwd(const mss_scan_args *a, void *stream) {
                         scan_workspace_clear_bytes(pl.tiles, pl.splits),
                         s) != cudaSuccess)
       return MSS_ERR_CUDA;
+  } else {
+    p.status = scan_status_word();
+    if (!p.status) return MSS_ERR_CUDA;
   }
   if (launch_scan_fwd(p, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16,
-                      a->z != nullptr, s) != cudaSuccess)
+                      s) != cudaSuccess)
     return MSS_ERR_CUDA;
   return MSS_OK;
 }
@@ -187,13 +194,22 @@ mss_status mss_scan_status(const mss_scan_args *a, void *stream) {
   if (st != MSS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return MSS_ERR_CUDA;
-  if (pl.splits <= 1) return MSS_OK;
-  if (!a->workspace || a->workspace_bytes < pl.workspace)
-    return MSS_ERR_WORKSPACE;
   unsigned word = 0;
-  if (cudaMemcpy(&word, a->workspace, sizeof(word), cudaMemcpyDeviceToHost) !=
-      cudaSuccess)
-    return MSS_ERR_CUDA;
+  if (pl.splits <= 1) {
+    // scans without workspace report into the library's own word, which is
+    // read and cleared here
+    unsigned *w = scan_status_word();
+    if (!w) return MSS_ERR_CUDA;
+    if (cudaMemcpy(&word, w, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(w, 0, sizeof(word)) != cudaSuccess)
+      return MSS_ERR_CUDA;
+  } else {
+    if (!a->workspace || a->workspace_bytes < pl.workspace)
+      return MSS_ERR_WORKSPACE;
+    if (cudaMemcpy(&word, a->workspace, sizeof(word), cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+      return MSS_ERR_CUDA;
+  }
   if (word & kStatusTimeout) return MSS_ERR_TIMEOUT;
   return MSS_OK;
 }

@@ -1,12 +1,10 @@
-// device_math.cuh -- small device helpers of the selective-scan kernels.
-//
-// Only the arithmetic the scan needs: the base-2 exponential used for the
-// decay exp(Delta*A), the softplus step size and the silu gate.  The decay
-// uses the MUFU ex2 unit; fp32 accuracy of the scan is checked by the parity
-// tests against the fp64 oracle.
+// device_math.cuh -- device helpers of the selective-scan kernels: the
+// special-function arithmetic of the step size, decay and gate, and the
+// PTX wrappers for TMA loads, mbarriers and release/acquire flags.
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 namespace sss48 {
@@ -14,21 +12,37 @@ namespace sss48 {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// 2^x on the special-function unit (flushes subnormal results to zero).
+// 2^x on the special-function unit (subnormal results flush to zero).
 __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-// softplus(x) = log(1 + e^x).  Above 15 it equals x to fp32 precision.
+__device__ __forceinline__ float lg2_mufu(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// softplus(x) = log(1 + e^x).  With e = e^x: below e = 1/32 the alternating
+// series e - e^2/2 + e^3/3 - e^4/4 + e^5/5 (truncation < e^6/6, i.e. under
+// 2e-9 relative); above, ln2 * log2(1 + e), whose argument is then >= 1.03 so
+// the base-2 logarithm's absolute error stays a few 1e-6 relative; above
+// x = 15, softplus(x) = x to fp32 precision.
 __device__ __forceinline__ float softplus_f(float x) {
-  return x > 15.0f ? x : log1pf(__expf(x));
+  const float e = ex2_mufu(x * kLog2e);
+  const float series =
+      e * fmaf(e, fmaf(e, fmaf(e, fmaf(e, 0.2f, -0.25f), 1.0f / 3.0f), -0.5f),
+               1.0f);
+  const float logv = lg2_mufu(1.0f + e) * kLn2;
+  const float r = e < 0.03125f ? series : logv;
+  return x > 15.0f ? x : r;
 }
 
 // silu(z) = z / (1 + e^-z); e^-z overflowing to inf gives -0, as it should.
 __device__ __forceinline__ float silu_f(float z) {
-  return __fdividef(z, 1.0f + __expf(-z));
+  return __fdividef(z, 1.0f + ex2_mufu(-z * kLog2e));
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);
@@ -57,6 +71,65 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
 
 __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---- mbarrier + TMA (no clusters: every CTA is its own cluster of one)
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of `bar` to complete, giving up after
+// `limit_ns` nanoseconds (returns false then).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t start = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 63u && global_timer_ns() - start > limit_ns) return false;
+  }
+}
+
+// 3-D tiled TMA load of box {c0 (innermost), c1, c2} into shared memory,
+// completing `bar`'s transaction count.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map,
+                                            int c0, int c1, int c2,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2),
+      "r"(smem_addr(bar))
+      : "memory");
 }
 
 }  // namespace sss48

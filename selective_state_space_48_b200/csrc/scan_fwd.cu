@@ -4,17 +4,20 @@
 // a chunk of the sequence.  Lane l of warp g owns channel d0 + l and the
 // states n = 4g .. 4g+3, whose fp32 values h[n] stay in registers for the
 // whole chunk ("Keeping the pad on the desk": the state never goes back to
-// HBM; only y is written).  Time is walked in blocks of 32 steps:
+// HBM; only y is written).  Time is walked in blocks of 32 steps through a
+// two-stage ring of raw input tiles in shared memory, filled by TMA (one
+// elected thread issues five 3-D tensor copies per block and the block waits
+// on an mbarrier, each wait bounded) while the previous block is computed:
 //
-//   prep   every (channel, t) of the block computes, once,
-//          Delta = softplus(delta + delta_bias), Delta*u, D*u and silu(z),
-//          and B_t[n], C_t[n] are widened to fp32 -- all into shared memory;
-//   scan   each lane runs h = exp(Delta A) h + Delta B u over the 32 steps
-//          for its 4 states and forms its share of y_t = sum_n C_t[n] h_t[n]
-//          (page "The State That Must Remember Everything", "The Equation",
-//          with the exponential-Euler discretisation of its Part 7);
+//   prep     every (channel, t) of the block computes, once,
+//            Delta = softplus(delta + delta_bias) and Delta*u, and B_t[n],
+//            C_t[n] are widened to fp32, into shared memory;
+//   scan     each lane runs h = exp(Delta A) h + Delta B u over the 32 steps
+//            for its 4 states and forms its share of y_t = sum_n C_t[n] h_t[n]
+//            (page "The State That Must Remember Everything", "The Equation",
+//            with the exponential-Euler discretisation of its Part 7);
 //   epilogue the shares of the state groups are summed, the D*u skip added,
-//          the silu(z) gate applied and y stored, coalesced along t.
+//            the silu(z) gate applied and y stored, coalesced along t.
 //
 // Long sequences with few channels are split into chunks that run in
 // parallel ("The relay": fade-and-add steps compose associatively, so a
@@ -25,154 +28,225 @@
 // then adds the missing term sum_n C_t[n] exp(A[n] sigma_t) h_in[n] to the
 // outputs it has written, until that term has decayed below 2^-64 of h_in
 // (sigma_t is the running sum of Delta from the chunk start).
+//
+// Shapes whose rows TMA cannot address (a row of seqlen elements that is
+// not a multiple of 16 bytes, or unaligned pointers) take the same kernel
+// with the tiles filled by plain coalesced loads instead.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
-#include <algorithm>
 #include <cstdint>
+#include <cstring>
+#include <mutex>
 
 #include "device_math.cuh"
 #include "scan_fwd.cuh"
 
 namespace sss48 {
+
+__device__ unsigned g_scan_status;  // status of scans run without workspace
+
 namespace {
 
 constexpr int CH = kChannelsPerBlock;
 constexpr int TB = kTimeBlock;
-constexpr int ROW = TB + 4;  // padded row: lanes reading float4 at row l hit
-                             // distinct bank groups
+constexpr int ROW = TB + 4;  // padded fp32 row: float4 reads of 32 lanes at
+                             // rows l spread over all bank groups
+constexpr int STAGES = 2;
 constexpr float kCutoffLog2 = -64.0f;
+constexpr uint64_t kTmaWaitNs = 2000000000ull;
+
+constexpr int align128(int x) { return (x + 127) / 128 * 128; }
+
+template <typename InT, int G>
+struct Layout {
+  static constexpr int NP = 4 * G;
+  static constexpr int tileU = align128(CH * TB * static_cast<int>(sizeof(InT)));
+  static constexpr int tileB = align128(NP * TB * static_cast<int>(sizeof(InT)));
+  static constexpr int stage = 3 * tileU + 2 * tileB;  // u, delta, z, B, C
+  static constexpr int raw = 0;
+  static constexpr int delta = raw + STAGES * stage;   // fp32 [CH][ROW]
+  static constexpr int du = delta + CH * ROW * 4;      // fp32 [CH][ROW]
+  static constexpr int sB = du + CH * ROW * 4;         // fp32 [NP][TB]
+  static constexpr int sC = sB + NP * TB * 4;          // fp32 [NP][TB]
+  static constexpr int part = sC + NP * TB * 4;        // fp32 [G][CH][ROW]
+  static constexpr int bias = part + G * CH * ROW * 4; // fp32 [CH]
+  static constexpr int dskip = bias + CH * 4;          // fp32 [CH]
+  static constexpr int bars = dskip + CH * 4;          // u64 [STAGES]
+  static constexpr int misc = bars + STAGES * 8;       // int [4]
+  static constexpr int bytes = misc + 16;
+};
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) {
   return a < b ? a : b;
 }
 
-struct Smem {
-  // offsets in floats into dynamic shared memory
-  static constexpr int delta = 0;
-  static constexpr int du = delta + CH * ROW;
-  static constexpr int skip = du + CH * ROW;
-  static constexpr int gate = skip + CH * ROW;
-  static constexpr int part = gate + CH * ROW;
-  // followed by part[G][CH][ROW], then sB[NP][TB], sC[NP][TB]
-  static constexpr int bytes(int G) {
-    return (part + G * CH * ROW + 2 * 4 * G * TB) * 4;
+template <typename InT, typename OutT, int G, bool TMA>
+struct Scan {
+  using Lay = Layout<InT, G>;
+  static constexpr int NT = 32 * G;
+  static constexpr int NP = 4 * G;
+
+  const ScanParams &p;
+  const TmaMaps &maps;
+  unsigned char *smem;
+  int64_t b, d0;
+  bool has_z;
+
+  __device__ Scan(const ScanParams &p_, const TmaMaps &m_, unsigned char *s_)
+      : p(p_), maps(m_), smem(s_), b(0), d0(0), has_z(p_.z != nullptr) {}
+
+  __device__ float *f32(int off) const { return reinterpret_cast<float *>(smem + off); }
+  __device__ InT *raw(int stage, int which) const {
+    const int off = Lay::raw + stage * Lay::stage +
+                    (which < 3 ? which * Lay::tileU : 3 * Lay::tileU + (which - 3) * Lay::tileB);
+    return reinterpret_cast<InT *>(smem + off);
   }
-};
+  __device__ uint64_t *bar(int stage) const {
+    return reinterpret_cast<uint64_t *>(smem + Lay::bars) + stage;
+  }
 
-template <typename InT>
-__device__ __forceinline__ float ld_in(const void *base, int64_t idx) {
-  return to_f32<InT>(reinterpret_cast<const InT *>(base)[idx]);
-}
+  // thread 0: start the TMA copies of the block at t0 into `stage`
+  __device__ void issue(int stage, int64_t t0) const {
+    const uint32_t bytes = static_cast<uint32_t>(
+        (2 + (has_z ? 1 : 0)) * CH * TB * sizeof(InT) + 2 * NP * TB * sizeof(InT));
+    uint64_t *bb = bar(stage);
+    mbar_expect_tx(bb, bytes);
+    const int x = static_cast<int>(t0), yd = static_cast<int>(d0), zb = static_cast<int>(b);
+    tma_load_3d(raw(stage, 0), &maps.u, x, yd, zb, bb);
+    tma_load_3d(raw(stage, 1), &maps.delta, x, yd, zb, bb);
+    if (has_z) tma_load_3d(raw(stage, 2), &maps.z, x, yd, zb, bb);
+    tma_load_3d(raw(stage, 3), &maps.B, x, 0, zb, bb);
+    tma_load_3d(raw(stage, 4), &maps.C, x, 0, zb, bb);
+  }
 
-// Fill the shared-memory tiles of one time block [t0, t0 + nt).
-template <typename InT, int G, bool HAS_Z>
-__device__ __forceinline__ void prep_block(const ScanParams &p, float *sm,
-                                           int64_t b, int64_t d0, int64_t t0,
-                                           int nt, bool with_skip) {
-  constexpr int NT = 32 * G;
-  constexpr int NP = 4 * G;
-  const int tid = threadIdx.x;
-  float *sDelta = sm + Smem::delta;
-  float *sDu = sm + Smem::du;
-  float *sSkip = sm + Smem::skip;
-  float *sGate = sm + Smem::gate;
-  float *sB = sm + Smem::part + G * CH * ROW;
-  float *sC = sB + NP * TB;
-#pragma unroll 4
-  for (int idx = tid; idx < CH * TB; idx += NT) {
-    const int c = idx / TB;
-    const int t = idx % TB;
-    const int64_t d = d0 + c;
-    float dl = 0.f, u = 0.f, g = 1.f, dskip = 0.f;
-    if (d < p.dim && t < nt) {
-      const int64_t off = (b * p.dim + d) * p.seqlen + t0 + t;
-      u = ld_in<InT>(p.u, off);
-      float x = ld_in<InT>(p.delta, off);
-      if (p.delta_bias) x += p.delta_bias[d];
-      dl = p.softplus ? softplus_f(x) : x;
-      if (HAS_Z) g = silu_f(ld_in<InT>(p.z, off));
-      if (p.D) dskip = p.D[d];
+  // all threads: fill `stage` with plain loads (zero outside the tensors)
+  __device__ void load_plain(int stage, int64_t t0, int nt) const {
+    const InT zero = from_f32<InT>(0.f);
+    const InT *gu = static_cast<const InT *>(p.u);
+    const InT *gd = static_cast<const InT *>(p.delta);
+    const InT *gz = static_cast<const InT *>(p.z);
+    InT *ru = raw(stage, 0), *rd = raw(stage, 1), *rz = raw(stage, 2);
+    for (int idx = threadIdx.x; idx < CH * TB; idx += NT) {
+      const int c = idx / TB, t = idx % TB;
+      const bool ok = d0 + c < p.dim && t < nt;
+      const int64_t off = (b * p.dim + d0 + c) * p.seqlen + t0 + t;
+      ru[idx] = ok ? gu[off] : zero;
+      rd[idx] = ok ? gd[off] : zero;
+      if (has_z) rz[idx] = ok ? gz[off] : zero;
     }
-    sDelta[c * ROW + t] = dl;
-    sDu[c * ROW + t] = dl * u;
-    if (with_skip) sSkip[c * ROW + t] = dskip * u;
-    if (HAS_Z) sGate[c * ROW + t] = g;
-  }
-#pragma unroll 4
-  for (int idx = tid; idx < NP * TB; idx += NT) {
-    const int n = idx / TB;
-    const int t = idx % TB;
-    float bv = 0.f, cv = 0.f;
-    if (n < p.dstate && t < nt) {
+    const InT *gb = static_cast<const InT *>(p.B);
+    const InT *gc = static_cast<const InT *>(p.C);
+    InT *rb = raw(stage, 3), *rc = raw(stage, 4);
+    for (int idx = threadIdx.x; idx < NP * TB; idx += NT) {
+      const int n = idx / TB, t = idx % TB;
+      const bool ok = n < p.dstate && t < nt;
       const int64_t off = (b * p.dstate + n) * p.seqlen + t0 + t;
-      bv = ld_in<InT>(p.B, off);
-      cv = ld_in<InT>(p.C, off);
+      rb[idx] = ok ? gb[off] : zero;
+      rc[idx] = ok ? gc[off] : zero;
     }
-    sB[n * TB + t] = bv;
-    sC[n * TB + t] = cv;
   }
-}
 
-// Sum the state-group shares of y for the block and store (or accumulate
-// into) y.
-template <typename OutT, int G, bool HAS_Z, bool ACCUMULATE>
-__device__ __forceinline__ void epilogue_block(const ScanParams &p, float *sm,
-                                               int64_t b, int64_t d0,
-                                               int64_t t0, int nt) {
-  constexpr int NT = 32 * G;
-  const float *sPart = sm + Smem::part;
-  const float *sSkip = sm + Smem::skip;
-  const float *sGate = sm + Smem::gate;
-  OutT *y = reinterpret_cast<OutT *>(p.y);
-  for (int idx = threadIdx.x; idx < CH * TB; idx += NT) {
-    const int c = idx / TB;
-    const int t = idx % TB;
-    const int64_t d = d0 + c;
-    if (d >= p.dim || t >= nt) continue;
-    float s = 0.f;
+  // Make the block at t0 available in `stage`; false if a TMA wait ran out.
+  __device__ bool acquire(int stage, uint32_t &phase, int64_t t0, int nt) const {
+    if (TMA) {
+      const bool ok = mbar_wait_bounded(bar(stage), (phase >> stage) & 1u, kTmaWaitNs);
+      phase ^= 1u << stage;
+      return __syncthreads_and(ok);
+    }
+    load_plain(stage, t0, nt);
+    __syncthreads();
+    return true;
+  }
+
+  // Delta, Delta*u (and B, C when `with_b`) of one block into fp32 tiles.
+  // Steps past the end of the chunk get Delta = 0: exp(0 * A) = 1 and no
+  // input, so they leave the state unchanged.
+  __device__ void prep(int stage, int nt, bool with_b) const {
+    const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
+    float *sDelta = f32(Lay::delta), *sDu = f32(Lay::du);
+    const float *sBias = f32(Lay::bias);
+    for (int idx = threadIdx.x; idx < CH * TB; idx += NT) {
+      const int c = idx / TB, t = idx % TB;
+      float dl = 0.f, du = 0.f;
+      if (t < nt) {
+        const float x = to_f32<InT>(rd[idx]) + sBias[c];
+        dl = p.softplus ? softplus_f(x) : x;
+        du = dl * to_f32<InT>(ru[idx]);
+      }
+      sDelta[c * ROW + t] = dl;
+      sDu[c * ROW + t] = du;
+    }
+    const InT *rb = raw(stage, 3), *rc = raw(stage, 4);
+    float *sB = f32(Lay::sB), *sC = f32(Lay::sC);
+    for (int idx = threadIdx.x; idx < NP * TB; idx += NT) {
+      if (with_b) sB[idx] = to_f32<InT>(rb[idx]);
+      sC[idx] = to_f32<InT>(rc[idx]);
+    }
+  }
+
+  // y = (sum of state-group shares + D u) * silu(z), or y += shares * silu(z)
+  __device__ void epilogue(int stage, int64_t t0, int nt, bool accumulate) const {
+    const InT *ru = raw(stage, 0), *rz = raw(stage, 2);
+    const float *sPart = f32(Lay::part), *sD = f32(Lay::dskip);
+    OutT *y = static_cast<OutT *>(p.y);
+    for (int idx = threadIdx.x; idx < CH * TB; idx += NT) {
+      const int c = idx / TB, t = idx % TB;
+      if (d0 + c >= p.dim || t >= nt) continue;
+      float s = 0.f;
 #pragma unroll
-    for (int g = 0; g < G; ++g) s += sPart[(g * CH + c) * ROW + t];
-    const int64_t off = (b * p.dim + d) * p.seqlen + t0 + t;
-    if (ACCUMULATE) {
-      if (HAS_Z) s *= sGate[c * ROW + t];
-      y[off] = from_f32<OutT>(to_f32<OutT>(y[off]) + s);
-    } else {
-      s += sSkip[c * ROW + t];
-      if (HAS_Z) s *= sGate[c * ROW + t];
+      for (int g = 0; g < G; ++g) s += sPart[(g * CH + c) * ROW + t];
+      const int64_t off = (b * p.dim + d0 + c) * p.seqlen + t0 + t;
+      if (!accumulate) s = fmaf(sD[c], to_f32<InT>(ru[idx]), s);
+      if (has_z) s *= silu_f(to_f32<InT>(rz[idx]));
+      if (accumulate) s += to_f32<OutT>(y[off]);
       y[off] = from_f32<OutT>(s);
     }
   }
-}
+};
 
-template <typename InT, typename OutT, int G, bool HAS_Z, bool SPLIT>
+template <typename InT, typename OutT, int G, bool TMA>
 __global__ void __launch_bounds__(32 * G)
-    scan_fwd_kernel(const ScanParams p) {
-  extern __shared__ __align__(16) float sm[];
+    scan_fwd_kernel(const ScanParams p, const __grid_constant__ TmaMaps maps) {
+  using S = Scan<InT, OutT, G, TMA>;
+  using Lay = typename S::Lay;
   constexpr int NP = 4 * G;
-  __shared__ int s_item;
-  __shared__ unsigned s_flag;
+  extern __shared__ __align__(128) unsigned char smem[];
+  S sc(p, maps, smem);
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int g = tid >> 5;  // state group of this warp
+  const bool split = p.splits > 1;
+  int *misc = reinterpret_cast<int *>(smem + Lay::misc);
 
-  int64_t item;
-  if (SPLIT) {
-    if (tid == 0) s_item = static_cast<int>(atomicAdd(p.ticket, 1u));
-    __syncthreads();
-    item = s_item;
-  } else {
-    item = blockIdx.x;
+  if (tid == 0) {
+    misc[0] = split ? static_cast<int>(atomicAdd(p.ticket, 1u))
+                    : static_cast<int>(blockIdx.x);
+    if (TMA) {
+      for (int s = 0; s < STAGES; ++s) mbar_init(sc.bar(s), 1);
+      fence_mbar_init();
+    }
   }
+  __syncthreads();
+  const int64_t item = misc[0];
   const int64_t k = item / p.tiles;  // sequence chunk (chunk-major order)
   const int64_t tile = item % p.tiles;
-  const int64_t b = tile / p.ch_tiles;
-  const int64_t d0 = (tile % p.ch_tiles) * CH;
+  sc.b = tile / p.ch_tiles;
+  sc.d0 = (tile % p.ch_tiles) * CH;
+  const int64_t b = sc.b, d0 = sc.d0;
   const int64_t d = d0 + lane;
   const bool dvalid = d < p.dim;
   const int64_t t_begin = k * p.chunk;
   const int64_t t_end = min64(t_begin + p.chunk, p.seqlen);
+  const int nblk = static_cast<int>((t_end - t_begin + TB - 1) / TB);
+  if (tid < CH) {
+    const bool ok = d0 + tid < p.dim;
+    sc.f32(Lay::bias)[tid] = (ok && p.delta_bias) ? p.delta_bias[d0 + tid] : 0.f;
+    sc.f32(Lay::dskip)[tid] = (ok && p.D) ? p.D[d0 + tid] : 0.f;
+  }
 
   float alpha[4], h[4];
   bool live[4];
@@ -181,21 +255,29 @@ __global__ void __launch_bounds__(32 * G)
     const int n = 4 * g + i;
     live[i] = dvalid && n < p.dstate;
     alpha[i] = live[i] ? p.A[d * p.dstate + n] * kLog2e : 0.f;
-    h[i] = (live[i] && k == 0 && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n]
-                                       : 0.f;
+    h[i] = (live[i] && k == 0 && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
   }
   float dsum = 0.f;
 
-  const float *sDelta = sm + Smem::delta;
-  const float *sDu = sm + Smem::du;
-  float *sPart = sm + Smem::part;
-  const float *sB = sm + Smem::part + G * CH * ROW;
-  const float *sC = sB + NP * TB;
+  const float *sDelta = sc.f32(Lay::delta);
+  const float *sDu = sc.f32(Lay::du);
+  float *sPart = sc.f32(Lay::part);
+  const float *sB = sc.f32(Lay::sB);
+  const float *sC = sc.f32(Lay::sC);
+  uint32_t phase = 0;
 
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += TB) {
+  // ------------------------------------------------------------ main pass
+  if (TMA && tid == 0) sc.issue(0, t_begin);
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int s = blk & 1;
+    const int64_t t0 = t_begin + static_cast<int64_t>(blk) * TB;
     const int nt = static_cast<int>(min64(TB, t_end - t0));
-    __syncthreads();
-    prep_block<InT, G, HAS_Z>(p, sm, b, d0, t0, nt, true);
+    if (!sc.acquire(s, phase, t0, nt)) {
+      if (tid == 0) atomicOr(p.status, kStatusTimeout);
+      return;
+    }
+    if (TMA && tid == 0 && blk + 1 < nblk) sc.issue(s ^ 1, t0 + TB);
+    sc.prep(s, nt, true);
     __syncthreads();
     const int nq = (nt + 3) >> 2;
     for (int q = 0; q < nq; ++q) {
@@ -220,13 +302,13 @@ __global__ void __launch_bounds__(32 * G)
       }
       *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
           make_float4(part[0], part[1], part[2], part[3]);
-      if (SPLIT) dsum += (dls[0] + dls[1]) + (dls[2] + dls[3]);
+      if (split) dsum += (dls[0] + dls[1]) + (dls[2] + dls[3]);
     }
     __syncthreads();
-    epilogue_block<OutT, G, HAS_Z, false>(p, sm, b, d0, t0, nt);
+    sc.epilogue(s, t0, nt, false);
   }
 
-  if (!SPLIT) {
+  if (!split) {
     if (p.last_state) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -276,10 +358,10 @@ __global__ void __launch_bounds__(32 * G)
           __nanosleep(128);
           f = ld_acquire_gpu(&p.flags[pred]);
         }
-        s_flag = f;
+        misc[1] = static_cast<int>(f);
       }
       __syncthreads();
-      const unsigned f = s_flag;
+      const unsigned f = static_cast<unsigned>(misc[1]);
       bool done = true;
       if (f == 2u) {
         const float *pi = p.incl + pred * static_cast<int64_t>(CH * NP);
@@ -297,7 +379,6 @@ __global__ void __launch_bounds__(32 * G)
       }
       if (__syncthreads_and(done)) break;
     }
-    // the true state at the end of this chunk: P * h_in + e
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       h[i] = fmaf(P[i], h_in[i], h[i]);
@@ -316,16 +397,24 @@ __global__ void __launch_bounds__(32 * G)
   }
   if (k == 0) return;
 
-  // correction: y_t += silu(z_t) * sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n]
-  float sigma = 0.f;
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += TB) {
-    bool need = false;
+  // ------------------------------------------------------ correction pass
+  // y_t += silu(z_t) * sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n]
+  bool need = false;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      need |= live[i] && h_in[i] != 0.f && !(alpha[i] * sigma < kCutoffLog2);
-    if (!__syncthreads_or(need)) break;
+  for (int i = 0; i < 4; ++i) need |= live[i] && h_in[i] != 0.f;
+  if (!__syncthreads_or(need)) return;
+  float sigma = 0.f;
+  if (TMA && tid == 0) sc.issue(0, t_begin);
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int s = blk & 1;
+    const int64_t t0 = t_begin + static_cast<int64_t>(blk) * TB;
     const int nt = static_cast<int>(min64(TB, t_end - t0));
-    prep_block<InT, G, HAS_Z>(p, sm, b, d0, t0, nt, false);
+    if (!sc.acquire(s, phase, t0, nt)) {
+      if (tid == 0) atomicOr(p.status, kStatusTimeout);
+      return;
+    }
+    if (TMA && tid == 0 && blk + 1 < nblk) sc.issue(s ^ 1, t0 + TB);
+    sc.prep(s, nt, false);
     __syncthreads();
     const int nq = (nt + 3) >> 2;
     for (int q = 0; q < nq; ++q) {
@@ -351,59 +440,132 @@ __global__ void __launch_bounds__(32 * G)
           make_float4(part[0], part[1], part[2], part[3]);
     }
     __syncthreads();
-    epilogue_block<OutT, G, HAS_Z, true>(p, sm, b, d0, t0, nt);
-    __syncthreads();
+    sc.epilogue(s, t0, nt, true);
+    need = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      need |= live[i] && h_in[i] != 0.f && !(alpha[i] * sigma < kCutoffLog2);
+    if (!__syncthreads_or(need)) {
+      // the copy of the next block may be in flight: let it land first
+      if (TMA && blk + 1 < nblk) {
+        const bool ok = mbar_wait_bounded(sc.bar(s ^ 1), (phase >> (s ^ 1)) & 1u,
+                                          kTmaWaitNs);
+        if (!ok && tid == 0) atomicOr(p.status, kStatusTimeout);
+      }
+      return;
+    }
   }
 }
 
-template <typename InT, typename OutT, int G, bool HAS_Z, bool SPLIT>
-cudaError_t launch_typed(const ScanParams &p, cudaStream_t stream) {
-  auto kern = scan_fwd_kernel<InT, OutT, G, HAS_Z, SPLIT>;
-  const int smem = Smem::bytes(G);
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+// ------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool encode_3d(CUtensorMap *m, const void *ptr, bool bf16, uint64_t len,
+               uint64_t rows, uint64_t batch, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const uint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {len, rows, batch};
+  cuuint64_t strides[2] = {len * es, len * rows * es};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(TB), box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+             3, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tma_eligible(const ScanParams &p, int in_bf16) {
+  const uint64_t es = in_bf16 ? 2 : 4;
+  auto al = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  if ((p.seqlen * es) % 16 != 0) return false;
+  if (p.seqlen >= (int64_t(1) << 31) || p.dim >= (int64_t(1) << 31) ||
+      p.batch >= (int64_t(1) << 31))
+    return false;
+  if (!al(p.u) || !al(p.delta) || !al(p.B) || !al(p.C) || (p.z && !al(p.z)))
+    return false;
+  return tensor_map_encoder() != nullptr;
+}
+
+bool build_maps(const ScanParams &p, int in_bf16, int groups, TmaMaps *m) {
+  const uint32_t np = 4 * groups;
+  const uint64_t L = p.seqlen, D = p.dim, N = p.dstate, Bt = p.batch;
+  if (!encode_3d(&m->u, p.u, in_bf16, L, D, Bt, CH)) return false;
+  if (!encode_3d(&m->delta, p.delta, in_bf16, L, D, Bt, CH)) return false;
+  if (p.z && !encode_3d(&m->z, p.z, in_bf16, L, D, Bt, CH)) return false;
+  if (!encode_3d(&m->B, p.B, in_bf16, L, N, Bt, np)) return false;
+  if (!encode_3d(&m->C, p.C, in_bf16, L, N, Bt, np)) return false;
+  return true;
+}
+
+template <typename InT, typename OutT, int G, bool TMA>
+cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t s) {
+  auto kern = scan_fwd_kernel<InT, OutT, G, TMA>;
+  const int smem = Layout<InT, G>::bytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.tiles * p.splits;
-  kern<<<static_cast<unsigned>(grid), 32 * G, smem, stream>>>(p);
+  kern<<<static_cast<unsigned>(grid), 32 * G, smem, s>>>(p, maps);
   return cudaGetLastError();
 }
 
-template <typename InT, typename OutT, int G>
-cudaError_t dispatch_z(const ScanParams &p, int has_z, cudaStream_t s) {
-  const bool split = p.splits > 1;
-  if (has_z)
-    return split ? launch_typed<InT, OutT, G, true, true>(p, s)
-                 : launch_typed<InT, OutT, G, true, false>(p, s);
-  return split ? launch_typed<InT, OutT, G, false, true>(p, s)
-               : launch_typed<InT, OutT, G, false, false>(p, s);
-}
-
 template <typename InT, typename OutT>
-cudaError_t dispatch_g(const ScanParams &p, int has_z, cudaStream_t s) {
+cudaError_t dispatch(const ScanParams &p, bool tma, const TmaMaps &maps, cudaStream_t s) {
   const int G = static_cast<int>((p.dstate + 3) / 4);
+  if (tma) {
+    switch (G) {
+      case 1: return launch_typed<InT, OutT, 1, true>(p, maps, s);
+      case 2: return launch_typed<InT, OutT, 2, true>(p, maps, s);
+      default: return launch_typed<InT, OutT, 4, true>(p, maps, s);
+    }
+  }
   switch (G) {
-    case 1: return dispatch_z<InT, OutT, 1>(p, has_z, s);
-    case 2: return dispatch_z<InT, OutT, 2>(p, has_z, s);
-    case 3: return dispatch_z<InT, OutT, 3>(p, has_z, s);
-    default: return dispatch_z<InT, OutT, 4>(p, has_z, s);
+    case 1: return launch_typed<InT, OutT, 1, false>(p, maps, s);
+    case 2: return launch_typed<InT, OutT, 2, false>(p, maps, s);
+    default: return launch_typed<InT, OutT, 4, false>(p, maps, s);
   }
 }
 
-template <typename InT, typename OutT, int G, bool HAS_Z, bool SPLIT>
+template <typename InT, typename OutT, int G>
 int occupancy_typed() {
   int n = 0;
-  auto kern = scan_fwd_kernel<InT, OutT, G, HAS_Z, SPLIT>;
-  const int smem = Smem::bytes(G);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * G, smem) !=
+  auto kern = scan_fwd_kernel<InT, OutT, G, true>;
+  const int smem = Layout<InT, G>::bytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return 1;
-  return std::max(n, 1);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * G, smem) != cudaSuccess)
+    return 1;
+  return n > 0 ? n : 1;
+}
+
+template <typename InT, typename OutT>
+int occupancy_g(int groups) {
+  switch (groups) {
+    case 1: return occupancy_typed<InT, OutT, 1>();
+    case 2: return occupancy_typed<InT, OutT, 2>();
+    default: return occupancy_typed<InT, OutT, 4>();
+  }
 }
 
 }  // namespace
+
+// groups 3 runs on the 4-group kernel (the fourth group's states are padding)
+static int kernel_groups(int groups) { return groups == 3 ? 4 : groups; }
 
 size_t scan_workspace_clear_bytes(int64_t tiles, int splits) {
   const size_t items = static_cast<size_t>(tiles) * splits;
@@ -413,7 +575,7 @@ size_t scan_workspace_clear_bytes(int64_t tiles, int splits) {
 size_t scan_workspace_bytes(int64_t tiles, int splits, int groups) {
   if (splits <= 1) return 0;
   const size_t items = static_cast<size_t>(tiles) * splits;
-  const size_t np = 4 * static_cast<size_t>(groups);
+  const size_t np = 4 * static_cast<size_t>(kernel_groups(groups));
   const size_t agg = items * 2 * CH * np * sizeof(float);
   const size_t incl = items * CH * np * sizeof(float);
   return scan_workspace_clear_bytes(tiles, splits) + ((agg + 255) / 256) * 256 +
@@ -423,7 +585,7 @@ size_t scan_workspace_bytes(int64_t tiles, int splits, int groups) {
 void scan_bind_workspace(ScanParams &p, void *ws, int groups) {
   char *base = static_cast<char *>(ws);
   const size_t items = static_cast<size_t>(p.tiles) * p.splits;
-  const size_t np = 4 * static_cast<size_t>(groups);
+  const size_t np = 4 * static_cast<size_t>(kernel_groups(groups));
   p.status = reinterpret_cast<unsigned *>(base);
   p.ticket = reinterpret_cast<unsigned *>(base + 4);
   p.flags = reinterpret_cast<unsigned *>(base + 256);
@@ -433,44 +595,35 @@ void scan_bind_workspace(ScanParams &p, void *ws, int groups) {
   p.incl = reinterpret_cast<float *>(base + clear + agg);
 }
 
-int scan_blocks_per_sm(int in_bf16, int out_bf16, int has_z, int groups,
-                       int split) {
-  // Occupancy depends on registers and shared memory only; the z / split
-  // variants are close enough that the z = true, split = false kernel
-  // stands in for all of them.
-  (void)has_z;
-  (void)split;
+unsigned *scan_status_word() {
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_scan_status) != cudaSuccess) return nullptr;
+  return static_cast<unsigned *>(ptr);
+}
+
+int scan_blocks_per_sm(int in_bf16, int out_bf16, int groups) {
   using BF = __nv_bfloat16;
+  const int G = kernel_groups(groups);
   switch ((in_bf16 ? 2 : 0) + (out_bf16 ? 1 : 0)) {
-    case 0:
-      switch (groups) {
-        case 1: return occupancy_typed<float, float, 1, true, false>();
-        case 2: return occupancy_typed<float, float, 2, true, false>();
-        case 3: return occupancy_typed<float, float, 3, true, false>();
-        default: return occupancy_typed<float, float, 4, true, false>();
-      }
-    case 1:
-      return occupancy_typed<float, BF, 4, true, false>();
-    case 2:
-      switch (groups) {
-        case 1: return occupancy_typed<BF, float, 1, true, false>();
-        case 2: return occupancy_typed<BF, float, 2, true, false>();
-        case 3: return occupancy_typed<BF, float, 3, true, false>();
-        default: return occupancy_typed<BF, float, 4, true, false>();
-      }
-    default:
-      return occupancy_typed<BF, BF, 4, true, false>();
+    case 0: return occupancy_g<float, float>(G);
+    case 1: return occupancy_g<float, BF>(G);
+    case 2: return occupancy_g<BF, float>(G);
+    default: return occupancy_g<BF, BF>(G);
   }
 }
 
 cudaError_t launch_scan_fwd(const ScanParams &p, int in_bf16, int out_bf16,
-                            int has_z, cudaStream_t stream) {
+                            cudaStream_t stream) {
   using BF = __nv_bfloat16;
+  TmaMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int groups = kernel_groups(static_cast<int>((p.dstate + 3) / 4));
+  const bool tma = tma_eligible(p, in_bf16) && build_maps(p, in_bf16, groups, &maps);
   if (in_bf16)
-    return out_bf16 ? dispatch_g<BF, BF>(p, has_z, stream)
-                    : dispatch_g<BF, float>(p, has_z, stream);
-  return out_bf16 ? dispatch_g<float, BF>(p, has_z, stream)
-                  : dispatch_g<float, float>(p, has_z, stream);
+    return out_bf16 ? dispatch<BF, BF>(p, tma, maps, stream)
+                    : dispatch<BF, float>(p, tma, maps, stream);
+  return out_bf16 ? dispatch<float, BF>(p, tma, maps, stream)
+                  : dispatch<float, float>(p, tma, maps, stream);
 }
 
 }  // namespace sss48

@@ -2,9 +2,11 @@
 // forward-scan / state-update kernels.
 #pragma once
 
+#include <cuda.h>
+#include <cuda_runtime.h>
+
 #include <cstddef>
 #include <cstdint>
-#include <cuda_runtime.h>
 
 namespace sss48 {
 
@@ -33,14 +35,20 @@ struct ScanParams {
   int splits;      // number of sequence chunks
   int ch_tiles;    // ceil(dim / kChannelsPerBlock)
   int64_t tiles;   // batch * ch_tiles
-  // split-mode workspace
+  // device-side status word (workspace when split, library word otherwise)
   unsigned *status;
+  // split-mode workspace
   unsigned *ticket;
   unsigned *flags;
   float *agg;      // per item: decay product P then local end state e
   float *incl;     // per item: true state at the end of the chunk
   unsigned test_flags;
   int64_t spin_timeout_ns;
+};
+
+// TMA descriptors of the five streamed inputs (z unused without a gate).
+struct TmaMaps {
+  CUtensorMap u, delta, z, B, C;
 };
 
 // Workspace bytes for `splits` chunks over `tiles` tiles with `groups`
@@ -53,12 +61,15 @@ void scan_bind_workspace(ScanParams &p, void *ws, int groups);
 // Bytes of the header + flag region that must be zero before a launch.
 size_t scan_workspace_clear_bytes(int64_t tiles, int splits);
 
+// Device address of the library's own status word (used when a scan has no
+// workspace); nullptr on failure.
+unsigned *scan_status_word();
+
 // Thread blocks of the scan kernel that fit on one SM (for planning).
-int scan_blocks_per_sm(int in_bf16, int out_bf16, int has_z, int groups,
-                       int split);
+int scan_blocks_per_sm(int in_bf16, int out_bf16, int groups);
 
 cudaError_t launch_scan_fwd(const ScanParams &p, int in_bf16, int out_bf16,
-                            int has_z, cudaStream_t stream);
+                            cudaStream_t stream);
 
 struct UpdateParams {
   int64_t batch, dim, dstate;
