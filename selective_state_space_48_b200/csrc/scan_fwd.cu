@@ -161,48 +161,83 @@ struct Scan {
     return true;
   }
 
-  // Delta, Delta*u (and B, C when `with_b`) of one block into fp32 tiles.
-  // Steps past the end of the chunk get Delta = 0: exp(0 * A) = 1 and no
-  // input, so they leave the state unchanged.
+  // Delta, Delta*u (and B, C when `with_b`) of one block into fp32 tiles,
+  // two timesteps per thread and iteration.  Steps past the end of the chunk
+  // get Delta = 0: exp(0 * A) = 1 and no input, so they leave the state
+  // unchanged.
   __device__ void prep(int stage, int nt, bool with_b) const {
     const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
     float *sDelta = f32(Lay::delta), *sDu = f32(Lay::du);
     const float *sBias = f32(Lay::bias);
-    for (int idx = threadIdx.x; idx < CH * TB; idx += NT) {
-      const int c = idx / TB, t = idx % TB;
-      float dl = 0.f, du = 0.f;
-      if (t < nt) {
-        const float x = to_f32<InT>(rd[idx]) + sBias[c];
-        dl = p.softplus ? softplus_f(x) : x;
-        du = dl * to_f32<InT>(ru[idx]);
+    constexpr int HT = TB / 2;
+#pragma unroll 2
+    for (int idx = threadIdx.x; idx < CH * HT; idx += NT) {
+      const int c = idx / HT, t = 2 * (idx % HT);
+      const float2 u = load2_f32(ru + c * TB + t);
+      const float2 dd = load2_f32(rd + c * TB + t);
+      const float bias = sBias[c];
+      float2 dl;
+      if (p.softplus) {
+        dl.x = softplus_f(dd.x + bias);
+        dl.y = softplus_f(dd.y + bias);
+      } else {
+        dl.x = dd.x + bias;
+        dl.y = dd.y + bias;
       }
-      sDelta[c * ROW + t] = dl;
-      sDu[c * ROW + t] = du;
+      if (t >= nt) dl.x = 0.f;
+      if (t + 1 >= nt) dl.y = 0.f;
+      *reinterpret_cast<float2 *>(sDelta + c * ROW + t) = dl;
+      *reinterpret_cast<float2 *>(sDu + c * ROW + t) = __fmul2_rn(dl, u);
     }
     const InT *rb = raw(stage, 3), *rc = raw(stage, 4);
     float *sB = f32(Lay::sB), *sC = f32(Lay::sC);
-    for (int idx = threadIdx.x; idx < NP * TB; idx += NT) {
-      if (with_b) sB[idx] = to_f32<InT>(rb[idx]);
-      sC[idx] = to_f32<InT>(rc[idx]);
+    for (int idx = 4 * threadIdx.x; idx < NP * TB; idx += 4 * NT) {
+      if (with_b) store4(sB + idx, load4_f32(rb + idx));
+      store4(sC + idx, load4_f32(rc + idx));
     }
   }
 
-  // y = (sum of state-group shares + D u) * silu(z), or y += shares * silu(z)
+  // y = (sum of state-group shares + D u) * silu(z), or y += shares * silu(z);
+  // four timesteps per thread and iteration, stored with one 16-byte (fp32)
+  // or 8-byte (bf16) store when the row allows it.
   __device__ void epilogue(int stage, int64_t t0, int nt, bool accumulate) const {
     const InT *ru = raw(stage, 0), *rz = raw(stage, 2);
     const float *sPart = f32(Lay::part), *sD = f32(Lay::dskip);
     OutT *y = static_cast<OutT *>(p.y);
-    for (int idx = threadIdx.x; idx < CH * TB; idx += NT) {
-      const int c = idx / TB, t = idx % TB;
+    constexpr int QT = TB / 4;
+    for (int idx = threadIdx.x; idx < CH * QT; idx += NT) {
+      const int c = idx / QT, t = 4 * (idx % QT);
       if (d0 + c >= p.dim || t >= nt) continue;
-      float s = 0.f;
+      float4 s = *reinterpret_cast<const float4 *>(sPart + c * ROW + t);
 #pragma unroll
-      for (int g = 0; g < G; ++g) s += sPart[(g * CH + c) * ROW + t];
-      const int64_t off = (b * p.dim + d0 + c) * p.seqlen + t0 + t;
-      if (!accumulate) s = fmaf(sD[c], to_f32<InT>(ru[idx]), s);
-      if (has_z) s *= silu_f(to_f32<InT>(rz[idx]));
-      if (accumulate) s += to_f32<OutT>(y[off]);
-      y[off] = from_f32<OutT>(s);
+      for (int g = 1; g < G; ++g) {
+        const float4 v = *reinterpret_cast<const float4 *>(sPart + (g * CH + c) * ROW + t);
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      if (!accumulate) {
+        const float4 u = load4_f32(ru + c * TB + t);
+        const float dk = sD[c];
+        s.x = fmaf(dk, u.x, s.x); s.y = fmaf(dk, u.y, s.y);
+        s.z = fmaf(dk, u.z, s.z); s.w = fmaf(dk, u.w, s.w);
+      }
+      if (has_z) {
+        const float4 z = load4_f32(rz + c * TB + t);
+        s.x *= silu_f(z.x); s.y *= silu_f(z.y);
+        s.z *= silu_f(z.z); s.w *= silu_f(z.w);
+      }
+      OutT *yr = y + (b * p.dim + d0 + c) * p.seqlen + t0 + t;
+      if (p.y_vec && t + 4 <= nt) {
+        if (accumulate) {
+          const float4 o = make_float4(to_f32<OutT>(yr[0]), to_f32<OutT>(yr[1]),
+                                       to_f32<OutT>(yr[2]), to_f32<OutT>(yr[3]));
+          s.x += o.x; s.y += o.y; s.z += o.z; s.w += o.w;
+        }
+        store4(yr, s);
+      } else {
+        const float sv[4] = {s.x, s.y, s.z, s.w};
+        for (int j = 0; j < 4 && t + j < nt; ++j)
+          yr[j] = from_f32<OutT>(accumulate ? sv[j] + to_f32<OutT>(yr[j]) : sv[j]);
+      }
     }
   }
 };
@@ -258,6 +293,9 @@ __global__ void __launch_bounds__(32 * G)
     h[i] = (live[i] && k == 0 && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
   }
   float dsum = 0.f;
+  float2 al2[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) al2[i] = make_float2(alpha[i], alpha[i]);
 
   const float *sDelta = sc.f32(Lay::delta);
   const float *sDu = sc.f32(Lay::du);
@@ -279,30 +317,36 @@ __global__ void __launch_bounds__(32 * G)
     if (TMA && tid == 0 && blk + 1 < nblk) sc.issue(s ^ 1, t0 + TB);
     sc.prep(s, nt, true);
     __syncthreads();
-    const int nq = (nt + 3) >> 2;
-    for (int q = 0; q < nq; ++q) {
+    // all 8 groups of 4 steps (padding steps past the chunk are identities)
+#pragma unroll
+    for (int q = 0; q < TB / 4; ++q) {
       const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
       const float4 du = *reinterpret_cast<const float4 *>(&sDu[lane * ROW + 4 * q]);
-      const float dls[4] = {dl.x, dl.y, dl.z, dl.w};
-      const float dus[4] = {du.x, du.y, du.z, du.w};
-      float part[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 dl01 = make_float2(dl.x, dl.y), dl23 = make_float2(dl.z, dl.w);
+      const float2 du01 = make_float2(du.x, du.y), du23 = make_float2(du.z, du.w);
+      float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int n = 4 * g + i;
         const float4 bq = *reinterpret_cast<const float4 *>(&sB[n * TB + 4 * q]);
         const float4 cq = *reinterpret_cast<const float4 *>(&sC[n * TB + 4 * q]);
-        const float bs[4] = {bq.x, bq.y, bq.z, bq.w};
-        const float cs[4] = {cq.x, cq.y, cq.z, cq.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float a = ex2_mufu(dls[j] * alpha[i]);
-          h[i] = fmaf(a, h[i], dus[j] * bs[j]);
-          part[j] = fmaf(cs[j], h[i], part[j]);
-        }
+        // exponents and inputs of steps (t, t+1) in one paired instruction
+        const float2 x01 = __fmul2_rn(dl01, al2[i]);
+        const float2 x23 = __fmul2_rn(dl23, al2[i]);
+        const float2 b01 = __fmul2_rn(du01, make_float2(bq.x, bq.y));
+        const float2 b23 = __fmul2_rn(du23, make_float2(bq.z, bq.w));
+        float2 h01, h23;
+        h01.x = fmaf(ex2_mufu(x01.x), h[i], b01.x);
+        h01.y = fmaf(ex2_mufu(x01.y), h01.x, b01.y);
+        h23.x = fmaf(ex2_mufu(x23.x), h01.y, b23.x);
+        h23.y = fmaf(ex2_mufu(x23.y), h23.x, b23.y);
+        h[i] = h23.y;
+        p01 = __ffma2_rn(make_float2(cq.x, cq.y), h01, p01);
+        p23 = __ffma2_rn(make_float2(cq.z, cq.w), h23, p23);
       }
       *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
-          make_float4(part[0], part[1], part[2], part[3]);
-      if (split) dsum += (dls[0] + dls[1]) + (dls[2] + dls[3]);
+          make_float4(p01.x, p01.y, p23.x, p23.y);
+      if (split) dsum += (dl.x + dl.y) + (dl.z + dl.w);
     }
     __syncthreads();
     sc.epilogue(s, t0, nt, false);
@@ -612,9 +656,12 @@ int scan_blocks_per_sm(int in_bf16, int out_bf16, int groups) {
   }
 }
 
-cudaError_t launch_scan_fwd(const ScanParams &p, int in_bf16, int out_bf16,
+cudaError_t launch_scan_fwd(const ScanParams &params, int in_bf16, int out_bf16,
                             cudaStream_t stream) {
   using BF = __nv_bfloat16;
+  ScanParams p = params;
+  const uintptr_t yv = 4 * (out_bf16 ? 2 : 4);
+  p.y_vec = (p.seqlen % 4 == 0) && (reinterpret_cast<uintptr_t>(p.y) % yv == 0);
   TmaMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const int groups = kernel_groups(static_cast<int>((p.dstate + 3) / 4));

@@ -30,6 +30,7 @@ struct ScanParams {
   const float *h0;
   void *y;
   float *last_state;
+  int y_vec;       // rows of y allow 4-element vector stores (set at launch)
   // launch plan
   int64_t chunk;   // timesteps per sequence chunk (multiple of kTimeBlock)
   int splits;      // number of sequence chunks
