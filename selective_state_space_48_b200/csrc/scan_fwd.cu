@@ -4,20 +4,27 @@
 // a chunk of the sequence.  Lane l of warp g owns channel d0 + l and the
 // states n = 4g .. 4g+3, whose fp32 values h[n] stay in registers for the
 // whole chunk ("Keeping the pad on the desk": the state never goes back to
-// HBM; only y is written).  Time is walked in blocks of 32 steps through a
-// two-stage ring of raw input tiles in shared memory, filled by TMA (one
-// elected thread issues five 3-D tensor copies per block and the block waits
-// on an mbarrier, each wait bounded) while the previous block is computed:
+// HBM; only y is written).  Time is walked in blocks of 16 steps.  Raw input
+// tiles (u, delta, z, B, C) arrive in a five-stage shared-memory ring filled
+// by TMA three blocks ahead (one thread issues five 3-D tensor copies per
+// block; every wait on the ring's mbarriers is bounded).  Each block passes
+// three phases:
 //
 //   prep     every (channel, t) of the block computes, once,
 //            Delta = softplus(delta + delta_bias) and Delta*u, and B_t[n],
 //            C_t[n] are widened to fp32, into shared memory;
-//   scan     each lane runs h = exp(Delta A) h + Delta B u over the 32 steps
+//   scan     each lane runs h = exp(Delta A) h + Delta B u over the 16 steps
 //            for its 4 states and forms its share of y_t = sum_n C_t[n] h_t[n]
 //            (page "The State That Must Remember Everything", "The Equation",
 //            with the exponential-Euler discretisation of its Part 7);
 //   epilogue the shares of the state groups are summed, the D*u skip added,
 //            the silu(z) gate applied and y stored, coalesced along t.
+//
+// The phases run in different warps at the same time: the scan warps (one
+// per group of 4 states) do nothing but the recurrence, while four auxiliary
+// warps issue the copies, prep block i+2 and finish block i.  Tiles and y
+// shares are double buffered and handed over through named barriers, so the
+// special-function work of prep and epilogue overlaps the recurrence.
 //
 // Long sequences with few channels are split into chunks that run in
 // parallel ("The relay": fade-and-add steps compose associatively, so a
@@ -53,9 +60,14 @@ namespace {
 constexpr int CH = kChannelsPerBlock;
 constexpr int TB = kTimeBlock;
 constexpr int ROW = TB + 4;  // padded fp32 row: float4 reads of 32 lanes at
-                             // rows l spread over all bank groups
-constexpr int STAGES = 2;
+                             // rows l spread over the bank groups
+constexpr int STAGES = 5;    // raw tile ring: blocks i-1 .. i+3 alive at once
+constexpr int PREFETCH = 3;  // block i+3 is requested while block i is scanned
 constexpr float kCutoffLog2 = -64.0f;
+// States per lane (of 4) whose decay exp(Delta A) is evaluated by the
+// FMA-pipe polynomial instead of the special-function unit; balances the
+// two pipes (the unit's 16 results per clock per SM bound the scan).
+constexpr int kPolyStates = 0;
 constexpr uint64_t kTmaWaitNs = 2000000000ull;
 
 constexpr int align128(int x) { return (x + 127) / 128 * 128; }
@@ -65,17 +77,23 @@ struct Layout {
   static constexpr int NP = 4 * G;
   static constexpr int tileU = align128(CH * TB * static_cast<int>(sizeof(InT)));
   static constexpr int tileB = align128(NP * TB * static_cast<int>(sizeof(InT)));
-  static constexpr int stage = 3 * tileU + 2 * tileB;  // u, delta, z, B, C
+  static constexpr int stage = 3 * tileU + 2 * tileB;   // u, delta, z, B, C
   static constexpr int raw = 0;
-  static constexpr int delta = raw + STAGES * stage;   // fp32 [CH][ROW]
-  static constexpr int du = delta + CH * ROW * 4;      // fp32 [CH][ROW]
-  static constexpr int sB = du + CH * ROW * 4;         // fp32 [NP][TB]
-  static constexpr int sC = sB + NP * TB * 4;          // fp32 [NP][TB]
-  static constexpr int part = sC + NP * TB * 4;        // fp32 [G][CH][ROW]
-  static constexpr int bias = part + G * CH * ROW * 4; // fp32 [CH]
-  static constexpr int dskip = bias + CH * 4;          // fp32 [CH]
-  static constexpr int bars = dskip + CH * 4;          // u64 [STAGES]
-  static constexpr int misc = bars + STAGES * 8;       // int [4]
+  // two sets of fp32 tiles: Delta, Delta*u [CH][ROW]; B, C [NP][TB]
+  static constexpr int set0 = raw + STAGES * stage;
+  static constexpr int oDelta = 0;
+  static constexpr int oDu = CH * ROW * 4;
+  static constexpr int oB = 2 * CH * ROW * 4;
+  static constexpr int oC = oB + NP * TB * 4;
+  static constexpr int set = oC + NP * TB * 4;
+  // two sets of state-group shares of y: [G][CH][ROW]
+  static constexpr int part0 = set0 + 2 * set;
+  static constexpr int part = G * CH * ROW * 4;
+  static constexpr int bias = part0 + 2 * part;          // fp32 [CH]
+  static constexpr int dskip = bias + CH * 4;            // fp32 [CH]
+  static constexpr int bars = dskip + CH * 4;            // u64 [STAGES]
+  static constexpr int hand = bars + STAGES * 8;         // u64 [8] handoffs
+  static constexpr int misc = hand + 8 * 8;              // int [4]
   static constexpr int bytes = misc + 16;
 };
 
@@ -92,13 +110,18 @@ struct Scan {
   const ScanParams &p;
   const TmaMaps &maps;
   unsigned char *smem;
-  int64_t b, d0;
+  int64_t b, d0, t_begin, t_end;
   bool has_z;
 
   __device__ Scan(const ScanParams &p_, const TmaMaps &m_, unsigned char *s_)
-      : p(p_), maps(m_), smem(s_), b(0), d0(0), has_z(p_.z != nullptr) {}
+      : p(p_), maps(m_), smem(s_), b(0), d0(0), t_begin(0), t_end(0),
+        has_z(p_.z != nullptr) {}
 
   __device__ float *f32(int off) const { return reinterpret_cast<float *>(smem + off); }
+  __device__ float *fset(int set, int off) const {
+    return f32(Lay::set0 + set * Lay::set + off);
+  }
+  __device__ float *fpart(int set) const { return f32(Lay::part0 + set * Lay::part); }
   __device__ InT *raw(int stage, int which) const {
     const int off = Lay::raw + stage * Lay::stage +
                     (which < 3 ? which * Lay::tileU : 3 * Lay::tileU + (which - 3) * Lay::tileB);
@@ -107,14 +130,24 @@ struct Scan {
   __device__ uint64_t *bar(int stage) const {
     return reinterpret_cast<uint64_t *>(smem + Lay::bars) + stage;
   }
+  // handoff barrier `kind` (0 tiles ready, 1 tiles free, 2 shares ready,
+  // 3 shares free) of buffer set `set`
+  __device__ uint64_t *hand(int kind, int set) const {
+    return reinterpret_cast<uint64_t *>(smem + Lay::hand) + 2 * kind + set;
+  }
+  __device__ int64_t t0_of(int blk) const { return t_begin + static_cast<int64_t>(blk) * TB; }
+  __device__ int nt_of(int blk) const {
+    return static_cast<int>(min64(TB, t_end - t0_of(blk)));
+  }
 
-  // thread 0: start the TMA copies of the block at t0 into `stage`
-  __device__ void issue(int stage, int64_t t0) const {
+  // thread 0: start the TMA copies of block `blk` into `stage`
+  __device__ void issue(int stage, int blk) const {
     const uint32_t bytes = static_cast<uint32_t>(
         (2 + (has_z ? 1 : 0)) * CH * TB * sizeof(InT) + 2 * NP * TB * sizeof(InT));
     uint64_t *bb = bar(stage);
     mbar_expect_tx(bb, bytes);
-    const int x = static_cast<int>(t0), yd = static_cast<int>(d0), zb = static_cast<int>(b);
+    const int x = static_cast<int>(t0_of(blk)), yd = static_cast<int>(d0),
+              zb = static_cast<int>(b);
     tma_load_3d(raw(stage, 0), &maps.u, x, yd, zb, bb);
     tma_load_3d(raw(stage, 1), &maps.delta, x, yd, zb, bb);
     if (has_z) tma_load_3d(raw(stage, 2), &maps.z, x, yd, zb, bb);
@@ -122,14 +155,17 @@ struct Scan {
     tma_load_3d(raw(stage, 4), &maps.C, x, 0, zb, bb);
   }
 
-  // all threads: fill `stage` with plain loads (zero outside the tensors)
-  __device__ void load_plain(int stage, int64_t t0, int nt) const {
+  // all threads: fill `stage` with block `blk` by plain loads (zero outside
+  // the tensors); visible to other threads after the next barrier
+  __device__ void load_plain(int stage, int blk, int ti, int nth) const {
+    const int64_t t0 = t0_of(blk);
+    const int nt = nt_of(blk);
     const InT zero = from_f32<InT>(0.f);
     const InT *gu = static_cast<const InT *>(p.u);
     const InT *gd = static_cast<const InT *>(p.delta);
     const InT *gz = static_cast<const InT *>(p.z);
     InT *ru = raw(stage, 0), *rd = raw(stage, 1), *rz = raw(stage, 2);
-    for (int idx = threadIdx.x; idx < CH * TB; idx += NT) {
+    for (int idx = ti; idx < CH * TB; idx += nth) {
       const int c = idx / TB, t = idx % TB;
       const bool ok = d0 + c < p.dim && t < nt;
       const int64_t off = (b * p.dim + d0 + c) * p.seqlen + t0 + t;
@@ -140,7 +176,7 @@ struct Scan {
     const InT *gb = static_cast<const InT *>(p.B);
     const InT *gc = static_cast<const InT *>(p.C);
     InT *rb = raw(stage, 3), *rc = raw(stage, 4);
-    for (int idx = threadIdx.x; idx < NP * TB; idx += NT) {
+    for (int idx = ti; idx < NP * TB; idx += nth) {
       const int n = idx / TB, t = idx % TB;
       const bool ok = n < p.dstate && t < nt;
       const int64_t off = (b * p.dstate + n) * p.seqlen + t0 + t;
@@ -149,63 +185,100 @@ struct Scan {
     }
   }
 
-  // Make the block at t0 available in `stage`; false if a TMA wait ran out.
-  __device__ bool acquire(int stage, uint32_t &phase, int64_t t0, int nt) const {
+  // Fill the raw stage of block `blk` (blocks past the chunk: nothing).
+  // TMA: thread ti == 0 starts the copies, which complete the stage's
+  // mbarrier.  Plain: the group of nth threads loads and each thread then
+  // arrives on the mbarrier, whose arrival count is that group's size.
+  __device__ void produce(int blk, int nblk, int ti, int nth) const {
+    if (blk >= nblk) return;
+    const int stage = blk % STAGES;
     if (TMA) {
-      const bool ok = mbar_wait_bounded(bar(stage), (phase >> stage) & 1u, kTmaWaitNs);
-      phase ^= 1u << stage;
-      return __syncthreads_and(ok);
+      if (ti == 0) issue(stage, blk);
+    } else {
+      load_plain(stage, blk, ti, nth);
+      mbar_arrive(bar(stage));
     }
-    load_plain(stage, t0, nt);
-    __syncthreads();
-    return true;
   }
 
-  // Delta, Delta*u (and B, C when `with_b`) of one block into fp32 tiles,
-  // two timesteps per thread and iteration.  Steps past the end of the chunk
-  // get Delta = 0: exp(0 * A) = 1 and no input, so they leave the state
-  // unchanged.
-  __device__ void prep(int stage, int nt, bool with_b) const {
+  // Wait (bounded) until the raw stage of block `blk` is complete; true
+  // when it is.  Every thread that waits tracks the stage phases itself.
+  __device__ bool wait_raw(int blk, int stage_base, uint32_t &phase) const {
+    const int stage = (stage_base + blk) % STAGES;
+    const bool ok = mbar_wait_bounded(bar(stage), (phase >> stage) & 1u, kTmaWaitNs);
+    phase ^= 1u << stage;
+    return ok;
+  }
+
+  // Correction pass (all threads of the block): TMA copies or plain loads
+  // by everyone, completed by the next barrier.
+  __device__ void request(int blk, int nblk, int stage_base, int ti, int nth) const {
+    if (blk >= nblk) return;
+    const int stage = (stage_base + blk) % STAGES;
+    if (TMA) {
+      if (ti == 0) issue(stage, blk);
+    } else {
+      load_plain(stage, blk, ti, nth);
+    }
+  }
+
+  __device__ bool land(int blk, int nblk, int stage_base, uint32_t &phase) const {
+    if (!TMA || blk >= nblk) return true;
+    return wait_raw(blk, stage_base, phase);
+  }
+
+  // Delta, Delta*u (and B, C when `with_b`) of one block into fp32 set
+  // `set`, two timesteps per thread and iteration.  Steps past the end of
+  // the chunk get Delta = 0: exp(0 * A) = 1 and no input, so they leave the
+  // state unchanged.
+  __device__ void prep(int stage, int set, int nt, bool with_b, int ti, int nth) const {
     const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
-    float *sDelta = f32(Lay::delta), *sDu = f32(Lay::du);
+    float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
     const float *sBias = f32(Lay::bias);
-    constexpr int HT = TB / 2;
-#pragma unroll 2
-    for (int idx = threadIdx.x; idx < CH * HT; idx += NT) {
-      const int c = idx / HT, t = 2 * (idx % HT);
-      const float2 u = load2_f32(ru + c * TB + t);
-      const float2 dd = load2_f32(rd + c * TB + t);
+    constexpr int QT = TB / 4;
+    // four timesteps per thread: four independent softplus chains
+    for (int idx = ti; idx < CH * QT; idx += nth) {
+      const int c = idx / QT, t = 4 * (idx % QT);
+      const float4 u = load4_f32(ru + c * TB + t);
+      const float4 dd = load4_f32(rd + c * TB + t);
       const float bias = sBias[c];
-      float2 dl;
+      float4 dl = make_float4(dd.x + bias, dd.y + bias, dd.z + bias, dd.w + bias);
       if (p.softplus) {
-        dl.x = softplus_f(dd.x + bias);
-        dl.y = softplus_f(dd.y + bias);
-      } else {
-        dl.x = dd.x + bias;
-        dl.y = dd.y + bias;
+        dl.x = softplus_f(dl.x); dl.y = softplus_f(dl.y);
+        dl.z = softplus_f(dl.z); dl.w = softplus_f(dl.w);
       }
-      if (t >= nt) dl.x = 0.f;
-      if (t + 1 >= nt) dl.y = 0.f;
-      *reinterpret_cast<float2 *>(sDelta + c * ROW + t) = dl;
-      *reinterpret_cast<float2 *>(sDu + c * ROW + t) = __fmul2_rn(dl, u);
+      if (t + 4 > nt) {
+        if (t >= nt) dl.x = 0.f;
+        if (t + 1 >= nt) dl.y = 0.f;
+        if (t + 2 >= nt) dl.z = 0.f;
+        if (t + 3 >= nt) dl.w = 0.f;
+      }
+      *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
+      *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
+          make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
     }
     const InT *rb = raw(stage, 3), *rc = raw(stage, 4);
-    float *sB = f32(Lay::sB), *sC = f32(Lay::sC);
-    for (int idx = 4 * threadIdx.x; idx < NP * TB; idx += 4 * NT) {
-      if (with_b) store4(sB + idx, load4_f32(rb + idx));
-      store4(sC + idx, load4_f32(rc + idx));
+    float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
+    for (int idx = 4 * ti; idx < 2 * NP * TB; idx += 4 * nth) {
+      if (idx < NP * TB) {
+        if (with_b) store4(sB + idx, load4_f32(rb + idx));
+      } else {
+        store4(sC + idx - NP * TB, load4_f32(rc + idx - NP * TB));
+      }
     }
   }
 
   // y = (sum of state-group shares + D u) * silu(z), or y += shares * silu(z);
   // four timesteps per thread and iteration, stored with one 16-byte (fp32)
   // or 8-byte (bf16) store when the row allows it.
-  __device__ void epilogue(int stage, int64_t t0, int nt, bool accumulate) const {
+  __device__ void epilogue(int stage, int set, int blk, bool accumulate, int ti,
+                           int nth) const {
+    const int64_t t0 = t0_of(blk);
+    const int nt = nt_of(blk);
     const InT *ru = raw(stage, 0), *rz = raw(stage, 2);
-    const float *sPart = f32(Lay::part), *sD = f32(Lay::dskip);
+    const float *sPart = fpart(set), *sD = f32(Lay::dskip);
     OutT *y = static_cast<OutT *>(p.y);
     constexpr int QT = TB / 4;
-    for (int idx = threadIdx.x; idx < CH * QT; idx += NT) {
+    for (int idx = ti; idx < CH * QT; idx += nth) {
       const int c = idx / QT, t = 4 * (idx % QT);
       if (d0 + c >= p.dim || t >= nt) continue;
       float4 s = *reinterpret_cast<const float4 *>(sPart + c * ROW + t);
@@ -228,9 +301,8 @@ struct Scan {
       OutT *yr = y + (b * p.dim + d0 + c) * p.seqlen + t0 + t;
       if (p.y_vec && t + 4 <= nt) {
         if (accumulate) {
-          const float4 o = make_float4(to_f32<OutT>(yr[0]), to_f32<OutT>(yr[1]),
-                                       to_f32<OutT>(yr[2]), to_f32<OutT>(yr[3]));
-          s.x += o.x; s.y += o.y; s.z += o.z; s.w += o.w;
+          s.x += to_f32<OutT>(yr[0]); s.y += to_f32<OutT>(yr[1]);
+          s.z += to_f32<OutT>(yr[2]); s.w += to_f32<OutT>(yr[3]);
         }
         store4(yr, s);
       } else {
@@ -240,30 +312,141 @@ struct Scan {
       }
     }
   }
+
+  // The recurrence over one block for this lane's channel and 4 states:
+  // h = exp(Delta A) h + Delta B u, with this warp's share of
+  // y_t = sum_n C_t[n] h_t[n] written to part set `set`.  Exponents and
+  // inputs of steps (t, t+1) go through one paired f32x2 instruction, as do
+  // the shares of y.
+  __device__ void scan(int set, int g, int lane, float (&h)[4],
+                       const float2 (&al2)[4], float &dsum, bool split) const {
+    const float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
+    const float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
+    float *sPart = fpart(set);
+#pragma unroll
+    for (int q = 0; q < TB / 4; ++q) {
+      const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
+      const float4 du = *reinterpret_cast<const float4 *>(&sDu[lane * ROW + 4 * q]);
+      const float2 dl01 = make_float2(dl.x, dl.y), dl23 = make_float2(dl.z, dl.w);
+      const float2 du01 = make_float2(du.x, du.y), du23 = make_float2(du.z, du.w);
+      float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int n = 4 * g + i;
+        const float4 bq = *reinterpret_cast<const float4 *>(&sB[n * TB + 4 * q]);
+        const float4 cq = *reinterpret_cast<const float4 *>(&sC[n * TB + 4 * q]);
+        const float2 x01 = __fmul2_rn(dl01, al2[i]);
+        const float2 x23 = __fmul2_rn(dl23, al2[i]);
+        const float2 b01 = __fmul2_rn(du01, make_float2(bq.x, bq.y));
+        const float2 b23 = __fmul2_rn(du23, make_float2(bq.z, bq.w));
+        // the last kPolyStates states of the group take their decays from
+        // the FMA-pipe polynomial, the others from the special-function unit
+        float2 e01, e23;
+        if (i >= 4 - kPolyStates) {
+          e01 = exp2_poly2(x01);
+          e23 = exp2_poly2(x23);
+        } else {
+          e01 = make_float2(ex2_mufu(x01.x), ex2_mufu(x01.y));
+          e23 = make_float2(ex2_mufu(x23.x), ex2_mufu(x23.y));
+        }
+        float2 h01, h23;
+        h01.x = fmaf(e01.x, h[i], b01.x);
+        h01.y = fmaf(e01.y, h01.x, b01.y);
+        h23.x = fmaf(e23.x, h01.y, b23.x);
+        h23.y = fmaf(e23.y, h23.x, b23.y);
+        h[i] = h23.y;
+        p01 = __ffma2_rn(make_float2(cq.x, cq.y), h01, p01);
+        p23 = __ffma2_rn(make_float2(cq.z, cq.w), h23, p23);
+      }
+      *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
+          make_float4(p01.x, p01.y, p23.x, p23.y);
+      if (split) dsum += (dl.x + dl.y) + (dl.z + dl.w);
+    }
+  }
+
+  // The carried-state term of the correction pass for one block:
+  // share of sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n].
+  __device__ void scan_carry(int set, int g, int lane, const float (&alpha)[4],
+                             const float (&h_in)[4], float &sigma) const {
+    const float *sDelta = fset(set, Lay::oDelta), *sC = fset(set, Lay::oC);
+    float *sPart = fpart(set);
+#pragma unroll
+    for (int q = 0; q < TB / 4; ++q) {
+      const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
+      const float dls[4] = {dl.x, dl.y, dl.z, dl.w};
+      float part[4] = {0.f, 0.f, 0.f, 0.f};
+      float sig[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        sigma += dls[j];
+        sig[j] = sigma;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int n = 4 * g + i;
+        const float4 cq = *reinterpret_cast<const float4 *>(&sC[n * TB + 4 * q]);
+        const float cs[4] = {cq.x, cq.y, cq.z, cq.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          part[j] = fmaf(cs[j] * ex2_mufu(alpha[i] * sig[j]), h_in[i], part[j]);
+      }
+      *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
+          make_float4(part[0], part[1], part[2], part[3]);
+    }
+  }
 };
 
+// Warp roles of one block: G scan warps (one per group of 4 states), two
+// prep warps and two epilogue warps.  They hand tiles and y shares over
+// through mbarriers in shared memory (one per kind and buffer set), so each
+// warp waits only for the data it needs and never for its siblings; every
+// wait is bounded.
+constexpr int kPrepWarps = 2;
+constexpr int kEpiWarps = 2;
+constexpr int kAuxWarps = kPrepWarps + kEpiWarps;
+constexpr int kTilesReady = 0;  // prep -> scan: fp32 tiles of a block written
+constexpr int kTilesFree = 1;   // scan -> prep: tiles of a block consumed
+constexpr int kPartReady = 2;   // scan -> epi: y shares of a block written
+constexpr int kPartFree = 3;    // epi -> scan: y shares of a block consumed
+constexpr int kBarEpi = 1;      // named barrier of the epilogue warps only
+constexpr uint64_t kHandoffWaitNs = 2000000000ull;
+
 template <typename InT, typename OutT, int G, bool TMA>
-__global__ void __launch_bounds__(32 * G)
+__global__ void __launch_bounds__(32 * (G + kAuxWarps))
     scan_fwd_kernel(const ScanParams p, const __grid_constant__ TmaMaps maps) {
   using S = Scan<InT, OutT, G, TMA>;
   using Lay = typename S::Lay;
   constexpr int NP = 4 * G;
+  constexpr int NSCAN = 32 * G;
+  constexpr int NPREP = 32 * kPrepWarps;
+  constexpr int NEPI = 32 * kEpiWarps;
+  constexpr int NALL = NSCAN + NPREP + NEPI;
   extern __shared__ __align__(128) unsigned char smem[];
   S sc(p, maps, smem);
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
-  const int g = tid >> 5;  // state group of this warp
+  const bool is_scan = tid < NSCAN;
+  const int g = is_scan ? (tid >> 5) : 0;  // state group of a scan warp
+  const bool is_prep = !is_scan && tid < NSCAN + NPREP;
+  const int tp = tid - NSCAN;              // index within the prep warps
+  const int te = tid - NSCAN - NPREP;      // index within the epilogue warps
   const bool split = p.splits > 1;
   int *misc = reinterpret_cast<int *>(smem + Lay::misc);
 
   if (tid == 0) {
     misc[0] = split ? static_cast<int>(atomicAdd(p.ticket, 1u))
                     : static_cast<int>(blockIdx.x);
-    if (TMA) {
-      for (int s = 0; s < STAGES; ++s) mbar_init(sc.bar(s), 1);
-      fence_mbar_init();
+    // a raw stage completes when its TMA bytes land (one arrival) or when
+    // every epilogue thread has stored its share of the plain loads
+    for (int s = 0; s < STAGES; ++s) mbar_init(sc.bar(s), TMA ? 1 : NEPI);
+    for (int set = 0; set < 2; ++set) {
+      mbar_init(sc.hand(kTilesReady, set), NPREP);
+      mbar_init(sc.hand(kTilesFree, set), NSCAN);
+      mbar_init(sc.hand(kPartReady, set), NSCAN);
+      mbar_init(sc.hand(kPartFree, set), NEPI);
     }
+    fence_mbar_init();
   }
   __syncthreads();
   const int64_t item = misc[0];
@@ -271,12 +454,12 @@ __global__ void __launch_bounds__(32 * G)
   const int64_t tile = item % p.tiles;
   sc.b = tile / p.ch_tiles;
   sc.d0 = (tile % p.ch_tiles) * CH;
+  sc.t_begin = k * p.chunk;
+  sc.t_end = min64(sc.t_begin + p.chunk, p.seqlen);
   const int64_t b = sc.b, d0 = sc.d0;
   const int64_t d = d0 + lane;
-  const bool dvalid = d < p.dim;
-  const int64_t t_begin = k * p.chunk;
-  const int64_t t_end = min64(t_begin + p.chunk, p.seqlen);
-  const int nblk = static_cast<int>((t_end - t_begin + TB - 1) / TB);
+  const bool dvalid = is_scan && d < p.dim;
+  const int nblk = static_cast<int>((sc.t_end - sc.t_begin + TB - 1) / TB);
   if (tid < CH) {
     const bool ok = d0 + tid < p.dim;
     sc.f32(Lay::bias)[tid] = (ok && p.delta_bias) ? p.delta_bias[d0 + tid] : 0.f;
@@ -296,61 +479,57 @@ __global__ void __launch_bounds__(32 * G)
   float2 al2[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) al2[i] = make_float2(alpha[i], alpha[i]);
-
-  const float *sDelta = sc.f32(Lay::delta);
-  const float *sDu = sc.f32(Lay::du);
-  float *sPart = sc.f32(Lay::part);
-  const float *sB = sc.f32(Lay::sB);
-  const float *sC = sc.f32(Lay::sC);
   uint32_t phase = 0;
 
   // ------------------------------------------------------------ main pass
-  if (TMA && tid == 0) sc.issue(0, t_begin);
-  for (int blk = 0; blk < nblk; ++blk) {
-    const int s = blk & 1;
-    const int64_t t0 = t_begin + static_cast<int64_t>(blk) * TB;
-    const int nt = static_cast<int>(min64(TB, t_end - t0));
-    if (!sc.acquire(s, phase, t0, nt)) {
-      if (tid == 0) atomicOr(p.status, kStatusTimeout);
-      return;
+  // Scan warps only run the recurrence.  Prep warps turn raw block i+2 into
+  // fp32 tiles while block i is scanned; epilogue warps write the outputs of
+  // block i and then refill its raw stage with block i+STAGES.  Tiles and y
+  // shares are double buffered (set = block & 1).  A wait that runs out is
+  // recorded and the pipeline carries on, so no warp is ever left waiting.
+  __syncthreads();  // bias / D tiles, barrier initialisation
+  bool ok = true;
+  uint32_t hp = 0;  // parities of the handoff barriers this thread waits on
+  auto wait_hand = [&](int kind, int set) {
+    const int bit = 2 * kind + set;
+    ok &= mbar_wait_bounded(sc.hand(kind, set), (hp >> bit) & 1u, kHandoffWaitNs);
+    hp ^= 1u << bit;
+  };
+  if (is_scan) {
+    for (int i = 0; i < nblk; ++i) {
+      const int s = i & 1;
+      wait_hand(kTilesReady, s);
+      if (i >= 2) wait_hand(kPartFree, s);
+      sc.scan(s, g, lane, h, al2, dsum, split);
+      if (i + 2 < nblk) mbar_arrive(sc.hand(kTilesFree, s));
+      mbar_arrive(sc.hand(kPartReady, s));
     }
-    if (TMA && tid == 0 && blk + 1 < nblk) sc.issue(s ^ 1, t0 + TB);
-    sc.prep(s, nt, true);
-    __syncthreads();
-    // all 8 groups of 4 steps (padding steps past the chunk are identities)
-#pragma unroll
-    for (int q = 0; q < TB / 4; ++q) {
-      const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
-      const float4 du = *reinterpret_cast<const float4 *>(&sDu[lane * ROW + 4 * q]);
-      const float2 dl01 = make_float2(dl.x, dl.y), dl23 = make_float2(dl.z, dl.w);
-      const float2 du01 = make_float2(du.x, du.y), du23 = make_float2(du.z, du.w);
-      float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int n = 4 * g + i;
-        const float4 bq = *reinterpret_cast<const float4 *>(&sB[n * TB + 4 * q]);
-        const float4 cq = *reinterpret_cast<const float4 *>(&sC[n * TB + 4 * q]);
-        // exponents and inputs of steps (t, t+1) in one paired instruction
-        const float2 x01 = __fmul2_rn(dl01, al2[i]);
-        const float2 x23 = __fmul2_rn(dl23, al2[i]);
-        const float2 b01 = __fmul2_rn(du01, make_float2(bq.x, bq.y));
-        const float2 b23 = __fmul2_rn(du23, make_float2(bq.z, bq.w));
-        float2 h01, h23;
-        h01.x = fmaf(ex2_mufu(x01.x), h[i], b01.x);
-        h01.y = fmaf(ex2_mufu(x01.y), h01.x, b01.y);
-        h23.x = fmaf(ex2_mufu(x23.x), h01.y, b23.x);
-        h23.y = fmaf(ex2_mufu(x23.y), h23.x, b23.y);
-        h[i] = h23.y;
-        p01 = __ffma2_rn(make_float2(cq.x, cq.y), h01, p01);
-        p23 = __ffma2_rn(make_float2(cq.z, cq.w), h23, p23);
-      }
-      *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
-          make_float4(p01.x, p01.y, p23.x, p23.y);
-      if (split) dsum += (dl.x + dl.y) + (dl.z + dl.w);
+  } else if (is_prep) {
+    for (int blk = 0; blk < nblk; ++blk) {
+      if (blk >= 2) wait_hand(kTilesFree, blk & 1);
+      ok &= sc.wait_raw(blk, 0, phase);
+      sc.prep(blk % STAGES, blk & 1, sc.nt_of(blk), true, tp, NPREP);
+      mbar_arrive(sc.hand(kTilesReady, blk & 1));
     }
-    __syncthreads();
-    sc.epilogue(s, t0, nt, false);
+    // the prep warps waited on every raw block: their phases seed the
+    // correction pass
+    if (tp == 0) misc[2] = static_cast<int>(phase);
+  } else {
+    for (int j = 0; j < STAGES; ++j) sc.produce(j, nblk, te, NEPI);
+    for (int i = 0; i < nblk; ++i) {
+      const int s = i & 1;
+      wait_hand(kPartReady, s);
+      ok &= sc.wait_raw(i, 0, phase);
+      sc.epilogue(i % STAGES, s, i, false, te, NEPI);
+      if (i + 2 < nblk) mbar_arrive(sc.hand(kPartFree, s));
+      // the raw stage of block i is free once every epilogue thread is done
+      bar_sync(kBarEpi, NEPI);
+      sc.produce(i + STAGES, nblk, te, NEPI);
+    }
   }
+  if (!ok) atomicOr(p.status, kStatusTimeout);
+  __syncthreads();
+  phase = static_cast<uint32_t>(misc[2]);
 
   if (!split) {
     if (p.last_state) {
@@ -370,15 +549,21 @@ __global__ void __launch_bounds__(32 * G)
 #pragma unroll
   for (int i = 0; i < 4; ++i) P[i] = ex2_mufu(alpha[i] * dsum);
 
+  // only the scan warps hold states; the aux warps take part in the
+  // barriers but write nothing
   float h_in[4] = {0.f, 0.f, 0.f, 0.f};
   if (k == 0) {
+    if (is_scan) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) my_incl[(4 * g + i) * CH + lane] = h[i];
+      for (int i = 0; i < 4; ++i) my_incl[(4 * g + i) * CH + lane] = h[i];
+    }
   } else {
+    if (is_scan) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      my_agg[(4 * g + i) * CH + lane] = P[i];
-      my_agg[CH * NP + (4 * g + i) * CH + lane] = h[i];
+      for (int i = 0; i < 4; ++i) {
+        my_agg[(4 * g + i) * CH + lane] = P[i];
+        my_agg[CH * NP + (4 * g + i) * CH + lane] = h[i];
+      }
     }
     __syncthreads();
     if (tid == 0 && !drop) {
@@ -424,9 +609,10 @@ __global__ void __launch_bounds__(32 * G)
       if (__syncthreads_and(done)) break;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      h[i] = fmaf(P[i], h_in[i], h[i]);
-      my_incl[(4 * g + i) * CH + lane] = h[i];
+    for (int i = 0; i < 4; ++i) h[i] = fmaf(P[i], h_in[i], h[i]);
+    if (is_scan) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) my_incl[(4 * g + i) * CH + lane] = h[i];
     }
   }
   __syncthreads();
@@ -434,7 +620,7 @@ __global__ void __launch_bounds__(32 * G)
     __threadfence();
     st_release_gpu(&p.flags[item], 2u);
   }
-  if (p.last_state && t_end == p.seqlen) {
+  if (p.last_state && sc.t_end == p.seqlen) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       if (live[i]) p.last_state[(b * p.dim + d) * p.dstate + 4 * g + i] = h[i];
@@ -442,62 +628,41 @@ __global__ void __launch_bounds__(32 * G)
   if (k == 0) return;
 
   // ------------------------------------------------------ correction pass
-  // y_t += silu(z_t) * sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n]
+  // y_t += silu(z_t) * sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n], block by
+  // block from the chunk start until every carried term has decayed.  The
+  // ring continues at stage nblk so the barrier phases stay consistent.
   bool need = false;
 #pragma unroll
   for (int i = 0; i < 4; ++i) need |= live[i] && h_in[i] != 0.f;
   if (!__syncthreads_or(need)) return;
   float sigma = 0.f;
-  if (TMA && tid == 0) sc.issue(0, t_begin);
-  for (int blk = 0; blk < nblk; ++blk) {
-    const int s = blk & 1;
-    const int64_t t0 = t_begin + static_cast<int64_t>(blk) * TB;
-    const int nt = static_cast<int>(min64(TB, t_end - t0));
-    if (!sc.acquire(s, phase, t0, nt)) {
+  const int base = nblk % STAGES;
+  for (int j = 0; j < PREFETCH; ++j) sc.request(j, nblk, base, tid, NALL);
+  for (int i = 0; i < nblk; ++i) {
+    const bool ok = sc.land(i, nblk, base, phase);
+    if (!__syncthreads_and(ok)) {
       if (tid == 0) atomicOr(p.status, kStatusTimeout);
       return;
     }
-    if (TMA && tid == 0 && blk + 1 < nblk) sc.issue(s ^ 1, t0 + TB);
-    sc.prep(s, nt, false);
+    const int stage = (base + i) % STAGES;
+    sc.prep(stage, 0, sc.nt_of(i), false, tid, NALL);
     __syncthreads();
-    const int nq = (nt + 3) >> 2;
-    for (int q = 0; q < nq; ++q) {
-      const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
-      const float dls[4] = {dl.x, dl.y, dl.z, dl.w};
-      float part[4] = {0.f, 0.f, 0.f, 0.f};
-      float sig[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        sigma += dls[j];
-        sig[j] = sigma;
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int n = 4 * g + i;
-        const float4 cq = *reinterpret_cast<const float4 *>(&sC[n * TB + 4 * q]);
-        const float cs[4] = {cq.x, cq.y, cq.z, cq.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          part[j] = fmaf(cs[j] * ex2_mufu(alpha[i] * sig[j]), h_in[i], part[j]);
-      }
-      *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
-          make_float4(part[0], part[1], part[2], part[3]);
-    }
+    if (is_scan) sc.scan_carry(0, g, lane, alpha, h_in, sigma);
     __syncthreads();
-    sc.epilogue(s, t0, nt, true);
+    sc.epilogue(stage, 0, i, true, tid, NALL);
     need = false;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      need |= live[i] && h_in[i] != 0.f && !(alpha[i] * sigma < kCutoffLog2);
+    for (int q = 0; q < 4; ++q)
+      need |= live[q] && h_in[q] != 0.f && !(alpha[q] * sigma < kCutoffLog2);
     if (!__syncthreads_or(need)) {
-      // the copy of the next block may be in flight: let it land first
-      if (TMA && blk + 1 < nblk) {
-        const bool ok = mbar_wait_bounded(sc.bar(s ^ 1), (phase >> (s ^ 1)) & 1u,
-                                          kTmaWaitNs);
-        if (!ok && tid == 0) atomicOr(p.status, kStatusTimeout);
-      }
+      // copies already requested must land before the block exits
+      bool okd = true;
+      for (int j = i + 1; j < i + PREFETCH && j < nblk; ++j)
+        okd &= sc.land(j, nblk, base, phase);
+      if (!okd && tid == 0) atomicOr(p.status, kStatusTimeout);
       return;
     }
+    sc.request(i + PREFETCH, nblk, base, tid, NALL);
   }
 }
 
@@ -563,7 +728,7 @@ cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.tiles * p.splits;
-  kern<<<static_cast<unsigned>(grid), 32 * G, smem, s>>>(p, maps);
+  kern<<<static_cast<unsigned>(grid), 32 * (G + kAuxWarps), smem, s>>>(p, maps);
   return cudaGetLastError();
 }
 
@@ -592,7 +757,8 @@ int occupancy_typed() {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * G, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * (G + kAuxWarps), smem) !=
+      cudaSuccess)
     return 1;
   return n > 0 ? n : 1;
 }

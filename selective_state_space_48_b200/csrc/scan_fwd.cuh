@@ -16,7 +16,7 @@ namespace sss48 {
 constexpr int kChannelsPerBlock = 32;
 constexpr int kStatesPerLane = 4;
 constexpr int kMaxStates = 16;
-constexpr int kTimeBlock = 32;  // timesteps staged in shared memory at once
+constexpr int kTimeBlock = 16;  // timesteps staged in shared memory at once
 
 struct ScanParams {
   int64_t batch, dim, dstate, seqlen;

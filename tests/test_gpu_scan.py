@@ -61,11 +61,13 @@ def test_odd_shapes_match_oracle(case):
 
 @pytest.mark.parametrize("splits", [2, 3, 7, 64])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_sequence_split_matches_oracle(splits, dt):
+@pytest.mark.parametrize("N,L", [(16, 5000), (5, 4999), (2, 3001)])
+def test_sequence_split_matches_oracle(splits, dt, N, L):
     """Chunks combined by look-back give the sequential result ("The relay":
-    group the steps any way you like)."""
-    w = workloads.custom(2, 40, 16, 5000, in_dtype=dt, has_z=True)
-    inp = gpu_inputs(w, seed=splits, h0=True)
+    group the steps any way you like).  Odd lengths take the plain-load
+    path, N < 16 the kernels with fewer state groups."""
+    w = workloads.custom(2, 40, N, L, in_dtype=dt, has_z=True)
+    inp = gpu_inputs(w, seed=splits + N, h0=True)
     y, last = run_gpu(w, inp, plan_splits=splits, return_last_state=True,
                       check_status=True)
     want, want_last = run_oracle(w, inp, return_last_state=True)
