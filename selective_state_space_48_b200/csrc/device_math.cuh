@@ -71,6 +71,31 @@ __device__ __forceinline__ float silu_f(float z) {
   return __fdividef(z, 1.0f + ex2_mufu(-z * kLog2e));
 }
 
+// softplus of two values with the exponential on the FMA pipe (the
+// logarithm stays on the special-function unit); same formula as softplus_f.
+__device__ __forceinline__ float2 softplus2_f(float2 x) {
+  const float2 e = exp2_poly2(__fmul2_rn(x, make_float2(kLog2e, kLog2e)));
+  float2 r;
+  {
+    const float s = e.x * fmaf(e.x, fmaf(e.x, fmaf(e.x, fmaf(e.x, 0.2f, -0.25f), 1.0f / 3.0f), -0.5f), 1.0f);
+    r.x = e.x < 0.03125f ? s : lg2_mufu(1.0f + e.x) * kLn2;
+  }
+  {
+    const float s = e.y * fmaf(e.y, fmaf(e.y, fmaf(e.y, fmaf(e.y, 0.2f, -0.25f), 1.0f / 3.0f), -0.5f), 1.0f);
+    r.y = e.y < 0.03125f ? s : lg2_mufu(1.0f + e.y) * kLn2;
+  }
+  r.x = x.x > 15.0f ? x.x : r.x;
+  r.y = x.y > 15.0f ? x.y : r.y;
+  return r;
+}
+
+// silu of two values with e^-z on the FMA pipe; the polynomial saturates at
+// 2^127 for z < -88, where silu(z) is -0 to fp32 precision anyway.
+__device__ __forceinline__ float2 silu2_f(float2 z) {
+  const float2 e = exp2_poly2(__fmul2_rn(z, make_float2(-kLog2e, -kLog2e)));
+  return make_float2(__fdividef(z.x, 1.0f + e.x), __fdividef(z.y, 1.0f + e.y));
+}
+
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {

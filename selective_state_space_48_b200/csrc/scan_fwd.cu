@@ -243,8 +243,9 @@ struct Scan {
       const float bias = sBias[c];
       float4 dl = make_float4(dd.x + bias, dd.y + bias, dd.z + bias, dd.w + bias);
       if (p.softplus) {
-        dl.x = softplus_f(dl.x); dl.y = softplus_f(dl.y);
-        dl.z = softplus_f(dl.z); dl.w = softplus_f(dl.w);
+        const float2 a = softplus2_f(make_float2(dl.x, dl.y));
+        const float2 b2 = softplus2_f(make_float2(dl.z, dl.w));
+        dl = make_float4(a.x, a.y, b2.x, b2.y);
       }
       if (t + 4 > nt) {
         if (t >= nt) dl.x = 0.f;
@@ -295,8 +296,9 @@ struct Scan {
       }
       if (has_z) {
         const float4 z = load4_f32(rz + c * TB + t);
-        s.x *= silu_f(z.x); s.y *= silu_f(z.y);
-        s.z *= silu_f(z.z); s.w *= silu_f(z.w);
+        const float2 g01 = silu2_f(make_float2(z.x, z.y));
+        const float2 g23 = silu2_f(make_float2(z.z, z.w));
+        s.x *= g01.x; s.y *= g01.y; s.z *= g23.x; s.w *= g23.y;
       }
       OutT *yr = y + (b * p.dim + d0 + c) * p.seqlen + t0 + t;
       if (p.y_vec && t + 4 <= nt) {
