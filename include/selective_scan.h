@@ -125,6 +125,32 @@ mss_status mamba_selective_scan_fwd(const mss_scan_args *args, void *stream);
  * scan that used args->workspace (MSS_OK when the scan needed none). */
 mss_status mss_scan_status(const mss_scan_args *args, void *stream);
 
+/* The same forward scan for callers that cannot allocate device memory:
+ * plugins and runtimes that are handed only the tensors they own and have no
+ * allocator of their own to call, code running under a memory pool it must
+ * not re-enter, and latency-critical paths where cudaMalloc (which can
+ * synchronise the device) is not allowed.  The pages have no counterpart;
+ * this is a calling convenience of this library.
+ *
+ * A scan whose plan splits the sequence needs workspace
+ * (mss_scan_workspace_size() > 0).  Here it uses an 8 MiB array that the
+ * library keeps in device memory (every device that loads the library holds
+ * it until the process exits) instead of args->workspace, which is ignored.
+ * Inputs and outputs are still the caller's.  Plans needing more than 8 MiB
+ * of workspace are rejected with MSS_ERR_WORKSPACE before anything is
+ * enqueued.  Nothing is allocated or freed, by this call or by any library
+ * it calls.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  All
+ * calls share the one array and its flags are cleared on the caller's stream
+ * at the start of each call: two calls whose work overlaps on the GPU (on
+ * different streams, or from different threads) race and must not be
+ * issued.  A bounded device-side wait that runs out is recorded inside the
+ * array and not reported; results are then unspecified. */
+mss_status mamba_selective_scan_fwd_noalloc(const mss_scan_args *args,
+                                           void *stream);
+
 /* Arguments of one decode step.  Shapes:
  *   state            (batch, dim, dstate) fp32, updated in place
  *   x, dt, z, y      (batch, dim)         in_dtype (y: out_dtype)

@@ -39,6 +39,7 @@ EXPORTED_SYMBOLS = (
     "mss_scan_workspace_size",
     "mamba_selective_scan_fwd",
     "mss_scan_status",
+    "mamba_selective_scan_fwd_noalloc",
     "selective_state_update",
     "mss_status_string",
     "mss_abi_version",
@@ -124,6 +125,8 @@ def load_library():
             lib.mamba_selective_scan_fwd.restype = ctypes.c_int
             lib.mss_scan_status.argtypes = [P(ScanArgs), ctypes.c_void_p]
             lib.mss_scan_status.restype = ctypes.c_int
+            lib.mamba_selective_scan_fwd_noalloc.argtypes = [P(ScanArgs), ctypes.c_void_p]
+            lib.mamba_selective_scan_fwd_noalloc.restype = ctypes.c_int
             lib.selective_state_update.argtypes = [P(UpdateArgs), ctypes.c_void_p]
             lib.selective_state_update.restype = ctypes.c_int
             lib.mss_status_string.argtypes = [ctypes.c_int]

@@ -265,3 +265,87 @@ const char *mss_status_string(mss_status s) {
 int mss_abi_version(void) { return MSS_ABI_VERSION; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Scan without any allocation by the caller or the library: the workspace of
+// a sequence-split scan lives in a fixed array in device memory that this
+// library owns (see the declaration in selective_scan.h).
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+
+// Every device that loads the library holds this array until the process
+// exits.  Host code must not use its name as an address: the device address
+// is looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array on the current device, looked up on the first
+// call per device (nullptr if the lookup fails).
+void *noalloc_scratch_address() {
+  static void *addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = ptr;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" mss_status mamba_selective_scan_fwd_noalloc(const mss_scan_args *a,
+                                                       void *stream) {
+  mss_status st = check_scan_args(a);
+  if (st != MSS_OK) return st;
+  Plan pl;
+  st = make_plan(a, &pl);
+  if (st != MSS_OK) return st;
+  if (pl.workspace > kNoAllocScratchBytes) return MSS_ERR_WORKSPACE;
+
+  ScanParams p{};
+  p.batch = a->batch;
+  p.dim = a->dim;
+  p.dstate = a->dstate;
+  p.seqlen = a->seqlen;
+  p.u = a->u;
+  p.delta = a->delta;
+  p.A = a->A;
+  p.B = a->B;
+  p.C = a->C;
+  p.D = a->D;
+  p.z = a->z;
+  p.delta_bias = a->delta_bias;
+  p.softplus = a->delta_softplus ? 1 : 0;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.last_state = a->last_state;
+  p.chunk = pl.chunk;
+  p.splits = pl.splits;
+  p.ch_tiles = pl.ch_tiles;
+  p.tiles = pl.tiles;
+  p.test_flags = a->test_flags;
+  p.spin_timeout_ns = a->spin_timeout_ns;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pl.splits > 1) {
+    void *ws = noalloc_scratch_address();
+    if (!ws) return MSS_ERR_CUDA;
+    scan_bind_workspace(p, ws, pl.groups);
+    // flags, ticket and status carry the previous call's values: clear them
+    if (cudaMemsetAsync(ws, 0, scan_workspace_clear_bytes(pl.tiles, pl.splits), s) !=
+        cudaSuccess)
+      return MSS_ERR_CUDA;
+  } else {
+    p.status = scan_status_word();
+    if (!p.status) return MSS_ERR_CUDA;
+  }
+  if (launch_scan_fwd(p, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16, s) !=
+      cudaSuccess)
+    return MSS_ERR_CUDA;
+  return MSS_OK;
+}
