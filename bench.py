@@ -71,6 +71,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="CPU time budget of --impl reference (default: "
+                         "3 s per step, between 20 and 120 s)")
     return ap.parse_args(argv)
 
 
@@ -422,7 +425,9 @@ def run_reference(args):
     bounded sample (a share of the channels, full length) of the workload."""
     w = workloads.BY_NAME[args.workload]
     inp = workloads.make_inputs(w, device="cpu")
-    budget = min(120.0, max(20.0, 3.0 * (args.steps + args.warmup)))
+    budget = args.ref_seconds
+    if budget is None:
+        budget = min(120.0, max(20.0, 3.0 * (args.steps + args.warmup)))
     gbs, ups, ch, threads, total = oracle_timing(inp, w, budget, steps=args.steps,
                                                  warmup=args.warmup)
     sample = (f"{ch} of {w.batch * w.dim} channels per step, full length "
@@ -451,7 +456,10 @@ def run_reference(args):
 
 
 def main(argv=None):
-    faulthandler.enable()
+    try:
+        faulthandler.enable()
+    except (AttributeError, ValueError, OSError):
+        pass  # stderr without a file descriptor (e.g. captured by a test)
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -1,0 +1,74 @@
+"""Host-side logic of bench.py (CPU only): the max-over-ranks reduction on
+two gloo ranks, the whole-job throughput arithmetic and the reference arm's
+JSON line."""
+import json
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import workloads
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}",
+                            rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        local_ms = 10.0 + 5.0 * rank          # rank 1 is the slow one
+        max_ms = bench.reduce_max(local_ms, world)
+        value = bench.whole_job_gbs(1_000_000_000, 4, world, max_ms)
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump({"max_ms": max_ms, "value": value}, f)
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_on_two_gloo_ranks(tmp_path):
+    port = _free_port()
+    mp.spawn(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(2)]
+    for r in res:
+        assert r["max_ms"] == 15.0
+        # 2 ranks x 4 steps x 1 GB in 15 ms
+        assert abs(r["value"] - 2 * 4 * 1.0 / 0.015) < 1e-6
+
+
+def test_whole_job_throughput_single_rank():
+    assert bench.reduce_max(3.5, 1) == 3.5
+    assert abs(bench.whole_job_gbs(252_817_408, 10, 1, 2.0) - 1264.08704) < 1e-6
+
+
+def test_bench_workload_bytes_match_the_roofline_table():
+    w = workloads.BY_NAME[bench.DEFAULT_WORKLOAD]
+    assert w.algorithmic_bytes() == 252_817_408
+    assert w.state_updates == 402_653_184
+
+
+def test_reference_arm_prints_the_contract_line(capsys):
+    rc = bench.main(["--impl", "reference", "--workload", "tiny-fp32",
+                     "--steps", "2", "--warmup", "1", "--ref-seconds", "0.5"])
+    assert rc == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup",
+                "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
+                "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["metric"] == bench.METRIC and line["unit"] == "GB/s"
+    assert line["config"]["workload"] == "tiny-fp32"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["value"] > 0
