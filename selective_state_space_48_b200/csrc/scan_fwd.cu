@@ -315,6 +315,110 @@ struct Scan {
     }
   }
 
+  // ---- main-pass prep/epilogue on fixed slots.  With 64 threads per role
+  // and TB/4 groups of four steps per channel row, thread ti always owns the
+  // groups ti + 64k (k < kSlots): channel row (ti + 64k) / (TB/4), steps
+  // 4 (ti % (TB/4)) .. +3 of every block.  Everything that depends only on
+  // the slot (rows, pointers, bias, D) is computed once per kernel.
+  static constexpr int QT = TB / 4;
+  static constexpr int kSlots = CH * QT / 64;
+  struct Slots {
+    int c[kSlots];
+    int t;
+    bool ok[kSlots];
+    float bias[kSlots], dk[kSlots];
+    OutT *yrow[kSlots];  // y of (b, d0 + c) at step t_begin + t
+  };
+  __device__ Slots make_slots(int ti) const {
+    Slots sl;
+    sl.t = 4 * (ti % QT);
+    OutT *y = static_cast<OutT *>(p.y);
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      const int c = (ti + 64 * k) / QT;
+      const int64_t d = d0 + c;
+      sl.c[k] = c;
+      sl.ok[k] = d < p.dim;
+      sl.bias[k] = (sl.ok[k] && p.delta_bias) ? p.delta_bias[d] : 0.f;
+      sl.dk[k] = (sl.ok[k] && p.D) ? p.D[d] : 0.f;
+      sl.yrow[k] = y + (b * p.dim + (sl.ok[k] ? d : d0)) * p.seqlen + t_begin + sl.t;
+    }
+    return sl;
+  }
+
+  __device__ void prep_slots(int stage, int set, int nt, const Slots &sl, int ti) const {
+    const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
+    float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      const int c = sl.c[k], t = sl.t;
+      const float4 u = load4_f32(ru + c * TB + t);
+      const float4 dd = load4_f32(rd + c * TB + t);
+      const float bias = sl.bias[k];
+      float4 dl = make_float4(dd.x + bias, dd.y + bias, dd.z + bias, dd.w + bias);
+      if (p.softplus) {
+        const float2 a = softplus2_f(make_float2(dl.x, dl.y));
+        const float2 a2 = softplus2_f(make_float2(dl.z, dl.w));
+        dl = make_float4(a.x, a.y, a2.x, a2.y);
+      }
+      if (t + 4 > nt) {
+        if (t >= nt) dl.x = 0.f;
+        if (t + 1 >= nt) dl.y = 0.f;
+        if (t + 2 >= nt) dl.z = 0.f;
+        if (t + 3 >= nt) dl.w = 0.f;
+      }
+      *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
+      *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
+          make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
+    }
+    const InT *rb = raw(stage, 3), *rc = raw(stage, 4);
+    float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
+#pragma unroll
+    for (int k = 0; k < (2 * NP * TB + 4 * 64 - 1) / (4 * 64); ++k) {
+      const int idx = 4 * (ti + 64 * k);
+      if (idx >= 2 * NP * TB) break;
+      if (idx < NP * TB) store4(sB + idx, load4_f32(rb + idx));
+      else store4(sC + idx - NP * TB, load4_f32(rc + idx - NP * TB));
+    }
+  }
+
+  __device__ void epilogue_slots(int stage, int set, int blk, const Slots &sl) const {
+    const int nt = nt_of(blk);
+    const int64_t toff = static_cast<int64_t>(blk) * TB;
+    const InT *ru = raw(stage, 0), *rz = raw(stage, 2);
+    const float *sPart = fpart(set);
+    const int t = sl.t;
+    if (t >= nt) return;
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      if (!sl.ok[k]) continue;
+      const int c = sl.c[k];
+      float4 s = *reinterpret_cast<const float4 *>(sPart + c * ROW + t);
+#pragma unroll
+      for (int g = 1; g < G; ++g) {
+        const float4 v = *reinterpret_cast<const float4 *>(sPart + (g * CH + c) * ROW + t);
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      const float4 u = load4_f32(ru + c * TB + t);
+      const float dk = sl.dk[k];
+      s.x = fmaf(dk, u.x, s.x); s.y = fmaf(dk, u.y, s.y);
+      s.z = fmaf(dk, u.z, s.z); s.w = fmaf(dk, u.w, s.w);
+      if (has_z) {
+        const float4 z = load4_f32(rz + c * TB + t);
+        const float2 g01 = silu2_f(make_float2(z.x, z.y));
+        const float2 g23 = silu2_f(make_float2(z.z, z.w));
+        s.x *= g01.x; s.y *= g01.y; s.z *= g23.x; s.w *= g23.y;
+      }
+      OutT *yr = sl.yrow[k] + toff;
+      if (p.y_vec && t + 4 <= nt) {
+        store4(yr, s);
+      } else {
+        const float sv[4] = {s.x, s.y, s.z, s.w};
+        for (int j = 0; j < 4 && t + j < nt; ++j) yr[j] = from_f32<OutT>(sv[j]);
+      }
+    }
+  }
+
   // The recurrence over one block for this lane's channel and 4 states:
   // h = exp(Delta A) h + Delta B u, with this warp's share of
   // y_t = sum_n C_t[n] h_t[n] written to part set `set`.  Exponents and
@@ -403,8 +507,8 @@ struct Scan {
 // through mbarriers in shared memory (one per kind and buffer set), so each
 // warp waits only for the data it needs and never for its siblings; every
 // wait is bounded.
-constexpr int kPrepWarps = 2;
-constexpr int kEpiWarps = 2;
+constexpr int kPrepWarps = 2;  // the slot layout of prep/epilogue assumes
+constexpr int kEpiWarps = 2;   // 64 threads per role
 constexpr int kAuxWarps = kPrepWarps + kEpiWarps;
 constexpr int kTilesReady = 0;  // prep -> scan: fp32 tiles of a block written
 constexpr int kTilesFree = 1;   // scan -> prep: tiles of a block consumed
@@ -507,22 +611,24 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
       mbar_arrive(sc.hand(kPartReady, s));
     }
   } else if (is_prep) {
+    const typename S::Slots sl = sc.make_slots(tp);
     for (int blk = 0; blk < nblk; ++blk) {
       if (blk >= 2) wait_hand(kTilesFree, blk & 1);
       ok &= sc.wait_raw(blk, 0, phase);
-      sc.prep(blk % STAGES, blk & 1, sc.nt_of(blk), true, tp, NPREP);
+      sc.prep_slots(blk % STAGES, blk & 1, sc.nt_of(blk), sl, tp);
       mbar_arrive(sc.hand(kTilesReady, blk & 1));
     }
     // the prep warps waited on every raw block: their phases seed the
     // correction pass
     if (tp == 0) misc[2] = static_cast<int>(phase);
   } else {
+    const typename S::Slots sl = sc.make_slots(te);
     for (int j = 0; j < STAGES; ++j) sc.produce(j, nblk, te, NEPI);
     for (int i = 0; i < nblk; ++i) {
       const int s = i & 1;
       wait_hand(kPartReady, s);
       ok &= sc.wait_raw(i, 0, phase);
-      sc.epilogue(i % STAGES, s, i, false, te, NEPI);
+      sc.epilogue_slots(i % STAGES, s, i, sl);
       if (i + 2 < nblk) mbar_arrive(sc.hand(kPartFree, s));
       // the raw stage of block i is free once every epilogue thread is done
       bar_sync(kBarEpi, NEPI);
