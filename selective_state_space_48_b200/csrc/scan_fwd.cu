@@ -104,7 +104,6 @@ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) {
 template <typename InT, typename OutT, int G, bool TMA>
 struct Scan {
   using Lay = Layout<InT, G>;
-  static constexpr int NT = 32 * G;
   static constexpr int NP = 4 * G;
 
   const ScanParams &p;
@@ -393,22 +392,25 @@ struct Scan {
     for (int k = 0; k < kSlots; ++k) {
       if (!sl.ok[k]) continue;
       const int c = sl.c[k];
+      // sum of the state-group shares, steps (t, t+1) and (t+2, t+3) paired
       float4 s = *reinterpret_cast<const float4 *>(sPart + c * ROW + t);
+      float2 s01 = make_float2(s.x, s.y), s23 = make_float2(s.z, s.w);
 #pragma unroll
       for (int g = 1; g < G; ++g) {
         const float4 v = *reinterpret_cast<const float4 *>(sPart + (g * CH + c) * ROW + t);
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        s01 = __fadd2_rn(s01, make_float2(v.x, v.y));
+        s23 = __fadd2_rn(s23, make_float2(v.z, v.w));
       }
       const float4 u = load4_f32(ru + c * TB + t);
-      const float dk = sl.dk[k];
-      s.x = fmaf(dk, u.x, s.x); s.y = fmaf(dk, u.y, s.y);
-      s.z = fmaf(dk, u.z, s.z); s.w = fmaf(dk, u.w, s.w);
+      const float2 dk = make_float2(sl.dk[k], sl.dk[k]);
+      s01 = __ffma2_rn(dk, make_float2(u.x, u.y), s01);
+      s23 = __ffma2_rn(dk, make_float2(u.z, u.w), s23);
       if (has_z) {
         const float4 z = load4_f32(rz + c * TB + t);
-        const float2 g01 = silu2_f(make_float2(z.x, z.y));
-        const float2 g23 = silu2_f(make_float2(z.z, z.w));
-        s.x *= g01.x; s.y *= g01.y; s.z *= g23.x; s.w *= g23.y;
+        s01 = __fmul2_rn(s01, make_float2(silu_f(z.x), silu_f(z.y)));
+        s23 = __fmul2_rn(s23, make_float2(silu_f(z.z), silu_f(z.w)));
       }
+      s = make_float4(s01.x, s01.y, s23.x, s23.y);
       OutT *yr = sl.yrow[k] + toff;
       if (p.y_vec && t + 4 <= nt) {
         store4(yr, s);
