@@ -321,6 +321,8 @@ struct Scan {
   // the slot (rows, pointers, bias, D) is computed once per kernel.
   static constexpr int QT = TB / 4;
   static constexpr int kSlots = CH * QT / 64;
+  static_assert(kSlots * 64 == CH * QT && 64 % QT == 0,
+                "every slot of a thread must cover the same steps");
   struct Slots {
     int c[kSlots];
     int t;
