@@ -106,7 +106,9 @@ mss_status make_plan(const mss_scan_args *a, Plan *pl) {
     if (pl->tiles >= sms) {
       want = 1;
     } else {
-      want = (target + pl->tiles - 1) / pl->tiles;
+      // as many chunks as keep every (tile, chunk) block resident at once:
+      // one block more than the chip holds would run as a second wave
+      want = std::max<int64_t>(1, target / pl->tiles);
       want = std::min<int64_t>(want, std::max<int64_t>(1, a->seqlen / kMinChunk));
     }
   }

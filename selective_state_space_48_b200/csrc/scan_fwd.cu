@@ -475,11 +475,21 @@ struct Scan {
   }
 
   // The carried-state term of the correction pass for one block:
-  // share of sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n].
+  // share of sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n].  A warp whose
+  // carried terms have all decayed (active false, warp-uniform) writes a
+  // zero share and leaves sigma as it is: with alpha <= 0 its terms only
+  // shrink further.
   __device__ void scan_carry(int set, int g, int lane, const float (&alpha)[4],
-                             const float (&h_in)[4], float &sigma) const {
+                             const float (&h_in)[4], float &sigma, bool active) const {
     const float *sDelta = fset(set, Lay::oDelta), *sC = fset(set, Lay::oC);
     float *sPart = fpart(set);
+    if (!active) {
+#pragma unroll
+      for (int q = 0; q < TB / 4; ++q)
+        *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
+            make_float4(0.f, 0.f, 0.f, 0.f);
+      return;
+    }
 #pragma unroll
     for (int q = 0; q < TB / 4; ++q) {
       const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
@@ -748,6 +758,7 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   for (int i = 0; i < 4; ++i) need |= live[i] && h_in[i] != 0.f;
   if (!__syncthreads_or(need)) return;
   float sigma = 0.f;
+  bool wactive = true;  // this scan warp still has carried terms to add
   const int base = nblk % STAGES;
   for (int j = 0; j < PREFETCH; ++j) sc.request(j, nblk, base, tid, NALL);
   for (int i = 0; i < nblk; ++i) {
@@ -759,13 +770,14 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     const int stage = (base + i) % STAGES;
     sc.prep(stage, 0, sc.nt_of(i), false, tid, NALL);
     __syncthreads();
-    if (is_scan) sc.scan_carry(0, g, lane, alpha, h_in, sigma);
+    if (is_scan) sc.scan_carry(0, g, lane, alpha, h_in, sigma, wactive);
     __syncthreads();
     sc.epilogue(stage, 0, i, true, tid, NALL);
     need = false;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       need |= live[q] && h_in[q] != 0.f && !(alpha[q] * sigma < kCutoffLog2);
+    if (is_scan) wactive = __any_sync(0xffffffffu, need);
     if (!__syncthreads_or(need)) {
       // copies already requested must land before the block exits
       bool okd = true;
