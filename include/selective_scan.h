@@ -30,8 +30,10 @@
  * out on the pages; they follow the standard Mamba parameterisation.
  *
  * Memory and ownership.  Every pointer is a device pointer owned by the
- * caller.  The library never allocates or frees device or host memory.  All
- * tensors are dense and row-major (C order) with the shapes given below.
+ * caller.  The library never allocates or frees device or host memory.
+ * Tensors are row-major (C order) with the shapes given below; the scan's
+ * (batch, rows, seqlen) tensors may carry their own batch and row strides
+ * (mss_scan_args.stride_*), everything else is dense.
  * Work is enqueued on the caller's stream (a cudaStream_t passed as void*,
  * NULL = legacy default stream) and is never synchronised, except in
  * mss_scan_status().
@@ -52,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 1
+#define MSS_ABI_VERSION 2
 
 typedef enum {
   MSS_OK = 0,
@@ -78,9 +80,22 @@ typedef enum { MSS_F32 = 0, MSS_BF16 = 1 } mss_dtype;
  *   h0, last_state   (batch, dim, dstate)   fp32
  * Optional (may be NULL): D (-> 0), z (-> no gate), delta_bias (-> 0),
  * h0 (-> zero initial state), last_state (-> not written).
+ * Strides: u, delta, z, y, B and C may be views with any batch and row
+ * (channel or state) strides, given in elements in stride_*[0] (batch) and
+ * stride_*[1] (row); the time dimension must be contiguous.  {0, 0} means
+ * packed, i.e. {rows * seqlen, seqlen}.  Input strides may be anything
+ * non-negative (a zero batch stride shares one B or C between all batch
+ * rows).  y's rows must not overlap (stride_y[1] >= seqlen when dim > 1),
+ * nor its batches (stride_y[0] >= (dim - 1) * stride_y[1] + seqlen when
+ * batch > 1), and y must not overlap any input; violations of the first two
+ * return MSS_ERR_INVALID_ARG, the last is not checked.  This covers, for
+ * instance, u and z taken as the two halves of one (batch, 2 dim, seqlen)
+ * projection.
  * Alignment: every pointer must be aligned to its element size; 16-byte
- * alignment of u, delta, z, B, C, y with seqlen * element size a multiple
- * of 16 enables the vectorised load path (otherwise a scalar path runs).
+ * alignment of u, delta, z, B, C with every stride (and seqlen) a multiple
+ * of 16 bytes enables the TMA load path (otherwise plain loads run), and y
+ * rows starting at multiples of 4 elements on a 16-byte (fp32) or 8-byte
+ * (bf16) boundary enable vector stores.
  * h0 may alias last_state. */
 typedef struct mss_scan_args {
   int64_t batch;   /* >= 1 */
@@ -110,6 +125,14 @@ typedef struct mss_scan_args {
   int plan_chunk_steps;   /* reserved, must be 0 */
   unsigned test_flags;    /* 0 in production */
   int64_t spin_timeout_ns;/* bound of each device-side wait; 0 = 1 s */
+  /* element strides {batch, row} of the (batch, rows, seqlen) tensors; time
+     is contiguous; {0, 0} = packed (see above) */
+  int64_t stride_u[2];
+  int64_t stride_delta[2];
+  int64_t stride_z[2];
+  int64_t stride_B[2];
+  int64_t stride_C[2];
+  int64_t stride_y[2];
 } mss_scan_args;
 
 /* Bytes of device workspace the scan needs for these arguments (0 when the

@@ -24,6 +24,8 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
+ABI_VERSION = 2  # MSS_ABI_VERSION of include/selective_scan.h
+
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
 MSS_ERR_UNSUPPORTED = 2
@@ -73,6 +75,12 @@ class ScanArgs(ctypes.Structure):
         ("plan_chunk_steps", ctypes.c_int),
         ("test_flags", ctypes.c_uint),
         ("spin_timeout_ns", ctypes.c_int64),
+        ("stride_u", ctypes.c_int64 * 2),
+        ("stride_delta", ctypes.c_int64 * 2),
+        ("stride_z", ctypes.c_int64 * 2),
+        ("stride_B", ctypes.c_int64 * 2),
+        ("stride_C", ctypes.c_int64 * 2),
+        ("stride_y", ctypes.c_int64 * 2),
     ]
 
 
@@ -133,6 +141,10 @@ def load_library():
             lib.mss_status_string.restype = ctypes.c_char_p
             lib.mss_abi_version.argtypes = []
             lib.mss_abi_version.restype = ctypes.c_int
+            if lib.mss_abi_version() != ABI_VERSION:
+                raise RuntimeError(
+                    f"{LIB_PATH} has ABI version {lib.mss_abi_version()}, "
+                    f"this binding expects {ABI_VERSION}; rebuild it")
             _lib = lib
     return _lib
 
@@ -153,12 +165,17 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def _check_cuda(name, t, dtype=None, shape=None):
+def _check_cuda(name, t, dtype=None, shape=None, strided=False):
+    """Type, dtype and shape checks; ``strided`` tensors may be views whose
+    last (time) dimension is contiguous, all others must be contiguous."""
     if t is None:
         return
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
+    if strided:
+        if t.dim() != 3 or (t.shape[2] > 1 and t.stride(2) != 1):
+            raise ValueError(f"{name} must be a 3-d view with a contiguous last dimension")
+    elif not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
@@ -179,18 +196,18 @@ def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     batch, dim, L = u.shape
     N = A.shape[1]
     ind = u.dtype
-    _check_cuda("u", u, ind)
-    _check_cuda("delta", delta, ind, (batch, dim, L))
+    _check_cuda("u", u, ind, strided=True)
+    _check_cuda("delta", delta, ind, (batch, dim, L), strided=True)
     _check_cuda("A", A, torch.float32, (dim, N))
-    _check_cuda("B", B, ind, (batch, N, L))
-    _check_cuda("C", C, ind, (batch, N, L))
+    _check_cuda("B", B, ind, (batch, N, L), strided=True)
+    _check_cuda("C", C, ind, (batch, N, L), strided=True)
     _check_cuda("D", D, torch.float32, (dim,))
-    _check_cuda("z", z, ind, (batch, dim, L))
+    _check_cuda("z", z, ind, (batch, dim, L), strided=True)
     _check_cuda("delta_bias", delta_bias, torch.float32, (dim,))
     _check_cuda("h0", h0, torch.float32, (batch, dim, N))
     _check_cuda("last_state", last_state, torch.float32, (batch, dim, N))
     if y is not None:
-        _check_cuda("y", y, None, (batch, dim, L))
+        _check_cuda("y", y, None, (batch, dim, L), strided=True)
     a = ScanArgs()
     a.batch, a.dim, a.dstate, a.seqlen = batch, dim, N, L
     a.in_dtype = _dtype_code(ind)
@@ -206,6 +223,10 @@ def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     a.plan_chunk_steps = 0
     a.test_flags = int(test_flags)
     a.spin_timeout_ns = int(spin_timeout_ns)
+    for name, t in (("u", u), ("delta", delta), ("z", z), ("B", B), ("C", C), ("y", y)):
+        if t is not None:
+            getattr(a, "stride_" + name)[0] = t.stride(0)
+            getattr(a, "stride_" + name)[1] = t.stride(1)
     return a
 
 

@@ -60,6 +60,40 @@ int blocks_per_sm(int dev, int in_bf16, int out_bf16, int groups) {
   return c;
 }
 
+// Element strides {batch, row} of a (batch, rows, seqlen) tensor whose
+// time dimension is contiguous: {0, 0} means packed.  Inputs may overlap
+// (a zero batch stride broadcasts one tensor to every batch row); the
+// output's rows and batches must not.  False on a negative or absurdly
+// large stride, or an overlapping output.
+bool resolve_strides(const int64_t (&in)[2], int64_t batch, int64_t rows,
+                     int64_t seqlen, bool output, int64_t (&out)[2]) {
+  if (in[0] == 0 && in[1] == 0) {
+    out[0] = rows * seqlen;
+    out[1] = seqlen;
+    return true;
+  }
+  const int64_t lim = int64_t(1) << 44;
+  if (in[0] < 0 || in[1] < 0 || in[0] > lim || in[1] > lim) return false;
+  if (output) {
+    if (rows > 1 && in[1] < seqlen) return false;
+    if (batch > 1 && in[0] < (rows - 1) * in[1] + seqlen) return false;
+  }
+  out[0] = in[0];
+  out[1] = in[1];
+  return true;
+}
+
+// All six stride pairs of a scan, resolved; false on the first bad one.
+bool resolve_scan_strides(const mss_scan_args *a, ScanParams *p) {
+  const int64_t Bt = a->batch, D = a->dim, N = a->dstate, L = a->seqlen;
+  return resolve_strides(a->stride_u, Bt, D, L, false, p->su) &&
+         resolve_strides(a->stride_delta, Bt, D, L, false, p->sdl) &&
+         resolve_strides(a->stride_z, Bt, D, L, false, p->sz) &&
+         resolve_strides(a->stride_B, Bt, N, L, false, p->sB) &&
+         resolve_strides(a->stride_C, Bt, N, L, false, p->sC) &&
+         resolve_strides(a->stride_y, Bt, D, L, true, p->sy);
+}
+
 mss_status check_scan_args(const mss_scan_args *a) {
   if (!a) return MSS_ERR_INVALID_ARG;
   if (a->batch < 1 || a->dim < 1 || a->seqlen < 1 || a->dstate < 1)
@@ -75,6 +109,10 @@ mss_status check_scan_args(const mss_scan_args *a) {
     return MSS_ERR_UNSUPPORTED;
   if (!a->u || !a->delta || !a->A || !a->B || !a->C || !a->y)
     return MSS_ERR_INVALID_ARG;
+  {
+    ScanParams probe{};
+    if (!resolve_scan_strides(a, &probe)) return MSS_ERR_INVALID_ARG;
+  }
   const size_t ei = esize(a->in_dtype), eo = esize(a->out_dtype);
   if (!aligned(a->u, ei) || !aligned(a->delta, ei) || !aligned(a->B, ei) ||
       !aligned(a->C, ei) || (a->z && !aligned(a->z, ei)) ||
@@ -122,6 +160,34 @@ mss_status make_plan(const mss_scan_args *a, Plan *pl) {
   return MSS_OK;
 }
 
+// Kernel parameters of a checked scan (everything but the status word and
+// the workspace fields).
+void fill_scan_params(const mss_scan_args *a, const Plan &pl, ScanParams *p) {
+  p->batch = a->batch;
+  p->dim = a->dim;
+  p->dstate = a->dstate;
+  p->seqlen = a->seqlen;
+  p->u = a->u;
+  p->delta = a->delta;
+  p->A = a->A;
+  p->B = a->B;
+  p->C = a->C;
+  p->D = a->D;
+  p->z = a->z;
+  p->delta_bias = a->delta_bias;
+  p->softplus = a->delta_softplus ? 1 : 0;
+  p->h0 = a->h0;
+  p->y = a->y;
+  p->last_state = a->last_state;
+  resolve_scan_strides(a, p);  // checked in check_scan_args
+  p->chunk = pl.chunk;
+  p->splits = pl.splits;
+  p->ch_tiles = pl.ch_tiles;
+  p->tiles = pl.tiles;
+  p->test_flags = a->test_flags;
+  p->spin_timeout_ns = a->spin_timeout_ns;
+}
+
 }  // namespace
 
 extern "C" {
@@ -149,28 +215,7 @@ mss_status mamba_selective_scan_fwd(const mss_scan_args *a, void *stream) {
     return MSS_ERR_WORKSPACE;
 
   ScanParams p{};
-  p.batch = a->batch;
-  p.dim = a->dim;
-  p.dstate = a->dstate;
-  p.seqlen = a->seqlen;
-  p.u = a->u;
-  p.delta = a->delta;
-  p.A = a->A;
-  p.B = a->B;
-  p.C = a->C;
-  p.D = a->D;
-  p.z = a->z;
-  p.delta_bias = a->delta_bias;
-  p.softplus = a->delta_softplus ? 1 : 0;
-  p.h0 = a->h0;
-  p.y = a->y;
-  p.last_state = a->last_state;
-  p.chunk = pl.chunk;
-  p.splits = pl.splits;
-  p.ch_tiles = pl.ch_tiles;
-  p.tiles = pl.tiles;
-  p.test_flags = a->test_flags;
-  p.spin_timeout_ns = a->spin_timeout_ns;
+  fill_scan_params(a, pl, &p);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pl.splits > 1) {
     scan_bind_workspace(p, a->workspace, pl.groups);
@@ -311,28 +356,7 @@ extern "C" mss_status mamba_selective_scan_fwd_noalloc(const mss_scan_args *a,
   if (pl.workspace > kNoAllocScratchBytes) return MSS_ERR_WORKSPACE;
 
   ScanParams p{};
-  p.batch = a->batch;
-  p.dim = a->dim;
-  p.dstate = a->dstate;
-  p.seqlen = a->seqlen;
-  p.u = a->u;
-  p.delta = a->delta;
-  p.A = a->A;
-  p.B = a->B;
-  p.C = a->C;
-  p.D = a->D;
-  p.z = a->z;
-  p.delta_bias = a->delta_bias;
-  p.softplus = a->delta_softplus ? 1 : 0;
-  p.h0 = a->h0;
-  p.y = a->y;
-  p.last_state = a->last_state;
-  p.chunk = pl.chunk;
-  p.splits = pl.splits;
-  p.ch_tiles = pl.ch_tiles;
-  p.tiles = pl.tiles;
-  p.test_flags = a->test_flags;
-  p.spin_timeout_ns = a->spin_timeout_ns;
+  fill_scan_params(a, pl, &p);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pl.splits > 1) {
     void *ws = noalloc_scratch_address();

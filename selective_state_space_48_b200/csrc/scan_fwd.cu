@@ -167,10 +167,10 @@ struct Scan {
     for (int idx = ti; idx < CH * TB; idx += nth) {
       const int c = idx / TB, t = idx % TB;
       const bool ok = d0 + c < p.dim && t < nt;
-      const int64_t off = (b * p.dim + d0 + c) * p.seqlen + t0 + t;
-      ru[idx] = ok ? gu[off] : zero;
-      rd[idx] = ok ? gd[off] : zero;
-      if (has_z) rz[idx] = ok ? gz[off] : zero;
+      const int64_t d = d0 + c, tt = t0 + t;
+      ru[idx] = ok ? gu[b * p.su[0] + d * p.su[1] + tt] : zero;
+      rd[idx] = ok ? gd[b * p.sdl[0] + d * p.sdl[1] + tt] : zero;
+      if (has_z) rz[idx] = ok ? gz[b * p.sz[0] + d * p.sz[1] + tt] : zero;
     }
     const InT *gb = static_cast<const InT *>(p.B);
     const InT *gc = static_cast<const InT *>(p.C);
@@ -178,9 +178,9 @@ struct Scan {
     for (int idx = ti; idx < NP * TB; idx += nth) {
       const int n = idx / TB, t = idx % TB;
       const bool ok = n < p.dstate && t < nt;
-      const int64_t off = (b * p.dstate + n) * p.seqlen + t0 + t;
-      rb[idx] = ok ? gb[off] : zero;
-      rc[idx] = ok ? gc[off] : zero;
+      const int64_t tt = t0 + t;
+      rb[idx] = ok ? gb[b * p.sB[0] + n * p.sB[1] + tt] : zero;
+      rc[idx] = ok ? gc[b * p.sC[0] + n * p.sC[1] + tt] : zero;
     }
   }
 
@@ -299,7 +299,7 @@ struct Scan {
         const float2 g23 = silu2_f(make_float2(z.z, z.w));
         s.x *= g01.x; s.y *= g01.y; s.z *= g23.x; s.w *= g23.y;
       }
-      OutT *yr = y + (b * p.dim + d0 + c) * p.seqlen + t0 + t;
+      OutT *yr = y + b * p.sy[0] + (d0 + c) * p.sy[1] + t0 + t;
       if (p.y_vec && t + 4 <= nt) {
         if (accumulate) {
           s.x += to_f32<OutT>(yr[0]); s.y += to_f32<OutT>(yr[1]);
@@ -342,7 +342,7 @@ struct Scan {
       sl.ok[k] = d < p.dim;
       sl.bias[k] = (sl.ok[k] && p.delta_bias) ? p.delta_bias[d] : 0.f;
       sl.dk[k] = (sl.ok[k] && p.D) ? p.D[d] : 0.f;
-      sl.yrow[k] = y + (b * p.dim + (sl.ok[k] ? d : d0)) * p.seqlen + t_begin + sl.t;
+      sl.yrow[k] = y + b * p.sy[0] + (sl.ok[k] ? d : d0) * p.sy[1] + t_begin + sl.t;
     }
     return sl;
   }
@@ -807,12 +807,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 bool encode_3d(CUtensorMap *m, const void *ptr, bool bf16, uint64_t len,
-               uint64_t rows, uint64_t batch, uint32_t box_rows) {
+               uint64_t rows, uint64_t batch, const int64_t (&st)[2], uint32_t box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const uint64_t es = bf16 ? 2 : 4;
   cuuint64_t dims[3] = {len, rows, batch};
-  cuuint64_t strides[2] = {len * es, len * rows * es};
+  cuuint64_t strides[2] = {static_cast<uint64_t>(st[1]) * es, static_cast<uint64_t>(st[0]) * es};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(TB), box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
@@ -826,6 +826,14 @@ bool tma_eligible(const ScanParams &p, int in_bf16) {
   const uint64_t es = in_bf16 ? 2 : 4;
   auto al = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
   if ((p.seqlen * es) % 16 != 0) return false;
+  // TMA strides are multiples of 16 bytes below 2^40
+  auto st_ok = [&](const int64_t (&s)[2]) {
+    return (s[0] * static_cast<int64_t>(es)) % 16 == 0 &&
+           (s[1] * static_cast<int64_t>(es)) % 16 == 0 &&
+           s[0] * static_cast<int64_t>(es) < (int64_t(1) << 40);
+  };
+  if (!st_ok(p.su) || !st_ok(p.sdl) || !st_ok(p.sB) || !st_ok(p.sC) || (p.z && !st_ok(p.sz)))
+    return false;
   if (p.seqlen >= (int64_t(1) << 31) || p.dim >= (int64_t(1) << 31) ||
       p.batch >= (int64_t(1) << 31))
     return false;
@@ -837,11 +845,11 @@ bool tma_eligible(const ScanParams &p, int in_bf16) {
 bool build_maps(const ScanParams &p, int in_bf16, int groups, TmaMaps *m) {
   const uint32_t np = 4 * groups;
   const uint64_t L = p.seqlen, D = p.dim, N = p.dstate, Bt = p.batch;
-  if (!encode_3d(&m->u, p.u, in_bf16, L, D, Bt, CH)) return false;
-  if (!encode_3d(&m->delta, p.delta, in_bf16, L, D, Bt, CH)) return false;
-  if (p.z && !encode_3d(&m->z, p.z, in_bf16, L, D, Bt, CH)) return false;
-  if (!encode_3d(&m->B, p.B, in_bf16, L, N, Bt, np)) return false;
-  if (!encode_3d(&m->C, p.C, in_bf16, L, N, Bt, np)) return false;
+  if (!encode_3d(&m->u, p.u, in_bf16, L, D, Bt, p.su, CH)) return false;
+  if (!encode_3d(&m->delta, p.delta, in_bf16, L, D, Bt, p.sdl, CH)) return false;
+  if (p.z && !encode_3d(&m->z, p.z, in_bf16, L, D, Bt, p.sz, CH)) return false;
+  if (!encode_3d(&m->B, p.B, in_bf16, L, N, Bt, p.sB, np)) return false;
+  if (!encode_3d(&m->C, p.C, in_bf16, L, N, Bt, p.sC, np)) return false;
   return true;
 }
 
@@ -951,7 +959,8 @@ cudaError_t launch_scan_fwd(const ScanParams &params, int in_bf16, int out_bf16,
   using BF = __nv_bfloat16;
   ScanParams p = params;
   const uintptr_t yv = 4 * (out_bf16 ? 2 : 4);
-  p.y_vec = (p.seqlen % 4 == 0) && (reinterpret_cast<uintptr_t>(p.y) % yv == 0);
+  p.y_vec = (p.sy[0] % 4 == 0) && (p.sy[1] % 4 == 0) &&
+            (reinterpret_cast<uintptr_t>(p.y) % yv == 0);
   TmaMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const int groups = kernel_groups(static_cast<int>((p.dstate + 3) / 4));

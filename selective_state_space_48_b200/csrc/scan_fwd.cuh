@@ -30,6 +30,9 @@ struct ScanParams {
   const float *h0;
   void *y;
   float *last_state;
+  // element strides {batch, row} of the (batch, rows, seqlen) tensors (time
+  // is contiguous); always resolved, never 0
+  int64_t su[2], sdl[2], sz[2], sB[2], sC[2], sy[2];
   int y_vec;       // rows of y allow 4-element vector stores (set at launch)
   // launch plan
   int64_t chunk;   // timesteps per sequence chunk (multiple of kTimeBlock)

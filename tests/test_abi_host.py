@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == 1
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 2
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
@@ -93,7 +93,10 @@ def _args(**kw):
     a.u = a.delta = a.A = a.B = a.C = a.y = fake
     a.plan_splits = 4
     for k, v in kw.items():
-        setattr(a, k, v)
+        if k.startswith("stride_"):
+            getattr(a, k)[0], getattr(a, k)[1] = v
+        else:
+            setattr(a, k, v)
     return a
 
 
@@ -131,6 +134,12 @@ def test_workspace_size_follows_plan(lib):
     (dict(plan_splits=-1), sss.MSS_ERR_INVALID_ARG),
     (dict(plan_chunk_steps=64), sss.MSS_ERR_INVALID_ARG),
     (dict(spin_timeout_ns=-5), sss.MSS_ERR_INVALID_ARG),
+    (dict(stride_u=(-1, 4096)), sss.MSS_ERR_INVALID_ARG),       # negative stride
+    (dict(stride_B=(0, -4096)), sss.MSS_ERR_INVALID_ARG),
+    (dict(stride_y=(40 * 4096, 4095)), sss.MSS_ERR_INVALID_ARG),  # y rows overlap
+    (dict(stride_y=(39 * 4096, 4096)), sss.MSS_ERR_INVALID_ARG),  # y batches overlap
+    (dict(stride_y=(0, 4096)), sss.MSS_ERR_INVALID_ARG),          # y batches alias
+    (dict(stride_z=(1 << 50, 4096)), sss.MSS_ERR_INVALID_ARG),    # absurd
 ])
 def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     a = _args(**kw)
@@ -138,6 +147,19 @@ def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     assert rc == code
     # the forward call applies the same checks and launches nothing
     assert lib.mamba_selective_scan_fwd(ctypes.byref(a), None) == code
+
+
+@pytest.mark.parametrize("kw", [
+    dict(stride_u=(80 * 4096, 4096)),          # u: half of a (2, 80, L) projection
+    dict(stride_z=(80 * 4096, 4096)),
+    dict(stride_B=(0, 4096)),                  # one B shared by the batch rows
+    dict(stride_C=(16 * 4096, 4096 + 8)),      # padded rows
+    dict(stride_y=(41 * 4100, 4100)),          # y inside a larger buffer
+    dict(stride_delta=(0, 0)),                 # packed
+])
+def test_valid_strides_are_accepted(lib, kw):
+    rc, n = _ws(lib, _args(plan_splits=1, **kw))
+    assert rc == sss.MSS_OK and n == 0
 
 
 def test_missing_workspace_is_reported(lib):
