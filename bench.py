@@ -67,6 +67,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=[w.name for w in workloads.WORKLOADS])
+    ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32",
+                    help="dtype of y (f32 is the metric's configuration)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work of the oracle baseline sample")
@@ -115,11 +117,16 @@ def profiled_traffic(workload: str):
     return None
 
 
-def workload_config(w) -> dict:
+def out_bytes(out_dtype: str) -> int:
+    return 2 if out_dtype == "bf16" else 4
+
+
+def workload_config(w, out_dtype="f32") -> dict:
+    nbytes = w.algorithmic_bytes(out_bytes(out_dtype))
     return {"workload": w.name, "batch": w.batch, "dim": w.dim,
             "dstate": w.dstate, "seqlen": w.seqlen, "in_dtype": w.in_dtype,
-            "out_dtype": "f32", "gate": "silu(z)" if w.has_z else "none",
-            "l2": (f"inputs+outputs {w.algorithmic_bytes() / 1e6:.0f} MB per "
+            "out_dtype": out_dtype, "gate": "silu(z)" if w.has_z else "none",
+            "l2": (f"inputs+outputs {nbytes / 1e6:.0f} MB per "
                    "step, larger than the 126 MB L2; no flush")}
 
 
@@ -282,7 +289,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = workloads.BY_NAME[args.workload]
     inp = workloads.make_inputs(w, device=dev)
-    y = torch.empty((w.batch, w.dim, w.seqlen), dtype=torch.float32, device=dev)
+    ydt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+    y = torch.empty((w.batch, w.dim, w.seqlen), dtype=ydt, device=dev)
     sargs = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"],
                                inp["C"], D=inp["D"], z=inp["z"],
                                delta_bias=inp["delta_bias"],
@@ -333,7 +341,7 @@ def run_ours(args, rank, world, local_rank):
     if lib.mss_scan_status(argp, sh) != 0:
         raise RuntimeError("device-side status error in the timed region")
 
-    bytes_step = w.algorithmic_bytes()
+    bytes_step = w.algorithmic_bytes(out_bytes(args.out_dtype))
     value = whole_job_gbs(bytes_step, K, world, max_ms)
     updates = w.state_updates * K * world / (max_ms * 1e-3)
 
@@ -391,7 +399,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w, args.out_dtype),
         "state_updates_per_s": updates,
         "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": value / world / peak,
