@@ -61,7 +61,8 @@ def _bind(lib):
     lib.oracle_silu_f64.argtypes = [ctypes.c_double]
     lib.oracle_silu_f64.restype = ctypes.c_double
     lib.oracle_selective_scan_f64.argtypes = (
-        [_I64] * 4 + [_D] * 8 + [ctypes.c_int, _D, _D, _D])
+        [_I64] * 4 + [_D] * 8 + [ctypes.c_int, _D, _D, _D,
+                                 ctypes.POINTER(ctypes.c_int32), _I64])
     lib.oracle_selective_scan_f64.restype = ctypes.c_int
     lib.oracle_selective_state_update_f64.argtypes = (
         [_I64] * 3 + [_D] * 9 + [ctypes.c_int, _D])
@@ -116,12 +117,14 @@ def silu(z, lib=None):
 
 def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                    delta_softplus=True, h0=None, return_last_state=False,
-                   lib=None):
+                   lib=None, cu_seqlens=None):
     """Sequential fp64 selective scan.
 
     u, delta, z: (batch, dim, L); B, C: (batch, N, L); A: (dim, N);
     D, delta_bias: (dim,); h0: (batch, dim, N).  Returns y (batch, dim, L)
-    float64, and the final state when ``return_last_state``.
+    float64, and the final state when ``return_last_state``.  cu_seqlens
+    (num_seqs + 1 offsets, 0 ... L) packs independent sequences into every
+    row: the state restarts from zero at each interior offset.
     """
     lib = lib or load()
     u = _f64(u)
@@ -140,10 +143,15 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     y = np.empty((batch, dim, L), dtype=np.float64)
     last = (np.empty((batch, dim, N), dtype=np.float64)
             if return_last_state else None)
+    cu, nseq = None, 0
+    if cu_seqlens is not None:
+        cu_arr = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        nseq = len(cu_arr) - 1
+        cu = cu_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
     rc = lib.oracle_selective_scan_f64(
         batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
         _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)),
-        _ptr(h0), _ptr(y), _ptr(last))
+        _ptr(h0), _ptr(y), _ptr(last), cu, nseq)
     if rc != 0:
         raise ValueError("oracle_selective_scan_f64 rejected the sizes")
     return (y, last) if return_last_state else y

@@ -67,11 +67,13 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
                               const double *D, const double *z,
                               const double *delta_bias, int delta_softplus,
                               const double *h0, double *y,
-                              double *last_state) {
+                              double *last_state, const int32_t *cu_seqlens,
+                              int64_t num_seqs) {
   /* the per-channel state lives on the stack; 256 states is far above any
    * size the tests or the bench use */
   if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256 || seqlen < 0)
     return -1;
+  if (cu_seqlens && num_seqs < 1) return -1;
   const int64_t channels = batch * dim;
 
   /* Channels (b, d) are independent recurrences; OpenMP only distributes
@@ -96,7 +98,15 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
     const double *Bb = B + b * dstate * seqlen;
     const double *Cb = C + b * dstate * seqlen;
 
+    int64_t next = 1; /* index of the next interior sequence start */
     for (int64_t t = 0; t < seqlen; ++t) {
+      /* Packed independent sequences: the state starts empty again at every
+       * interior start cu_seqlens[i], 0 < i < num_seqs. */
+      if (cu_seqlens) {
+        while (next < num_seqs && cu_seqlens[next] < t) ++next;
+        if (next < num_seqs && cu_seqlens[next] == t)
+          for (int64_t n = 0; n < dstate; ++n) hp[n] = 0.0;
+      }
       const double dt = step_size(drow[t], bias, delta_softplus);
       const double ut = urow[t];
       double acc = 0.0;

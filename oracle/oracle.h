@@ -43,7 +43,11 @@ double oracle_silu_f64(double z);
  *   h_t[n]  = exp(Delta_t * A[d,n]) * h_{t-1}[n] + Delta_t * B_t[n] * u_t
  *   y_t     = sum_n C_t[n] * h_t[n] + D[d] * u_t
  *   y_t    *= silu(z_t)                            (when z != NULL)
- * with h_{-1} = h0 (or 0).  Returns 0, or -1 on a bad size. */
+ * with h_{-1} = h0 (or 0).  Packed sequences: when cu_seqlens is not NULL
+ * (num_seqs + 1 increasing offsets, 0 ... seqlen, the same for every batch
+ * row), h is set to 0 before every step t = cu_seqlens[i], 0 < i < num_seqs,
+ * so each row holds num_seqs independent scans; h0 seeds the first and
+ * last_state is the end of the last.  Returns 0, or -1 on a bad size. */
 int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
                               int64_t seqlen, const double *u,
                               const double *delta, const double *A,
@@ -51,7 +55,8 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
                               const double *D, const double *z,
                               const double *delta_bias, int delta_softplus,
                               const double *h0, double *y,
-                              double *last_state);
+                              double *last_state, const int32_t *cu_seqlens,
+                              int64_t num_seqs);
 
 /* One decode step (the same recurrence for a single t), state updated in
  * place.  x, dt, z, y: (batch, dim); B, C: (batch, dstate);

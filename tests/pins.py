@@ -399,6 +399,52 @@ def pin_resume(lib):
     _close(s2, last, 1e-14, 1e-14, "resume state")
 
 
+# --------------------------------------------------------------------------
+# Packed sequences: a row holding several independent sequences (offsets
+# cu_seqlens) is the concatenation of their separate scans, each from an
+# empty state except the first, which starts from h0.  Checked against the
+# mpmath unrolled sums of every sequence on its own, so the reset logic is
+# pinned to the closed form, not to the oracle's recurrence.
+
+
+def pin_packed_sequences(lib):
+    rng = _rng(23)
+    bt, dm, N, L = 2, 2, 3, 11
+    # a 1-step sequence, an empty one, interior starts inside and at the end
+    cu = [0, 1, 5, 5, 9, 11]
+    u = rng.normal(size=(bt, dm, L))
+    delta = rng.normal(size=(bt, dm, L))
+    A = -rng.uniform(0.2, 2.0, size=(dm, N))
+    B = rng.normal(size=(bt, N, L))
+    C = rng.normal(size=(bt, N, L))
+    D = rng.normal(size=dm)
+    z = rng.normal(size=(bt, dm, L))
+    bias = rng.normal(size=dm) * 0.5
+    h0 = rng.normal(size=(bt, dm, N))
+    want = np.zeros((bt, dm, L))
+    want_last = None
+    for i in range(len(cu) - 1):
+        a, b = cu[i], cu[i + 1]
+        if a == b:
+            continue
+        sl = slice(a, b)
+        yi, li = _brute_force(u[..., sl], delta[..., sl], A, B[..., sl], C[..., sl],
+                              D, z[..., sl], bias, True, h0 if i == 0 else None)
+        want[..., sl] = yi
+        want_last = li
+    got, got_last = oracle.selective_scan(u, delta, A, B, C, D=D, z=z, delta_bias=bias,
+                                          h0=h0, return_last_state=True, lib=lib,
+                                          cu_seqlens=cu)
+    _close(got, want, 1e-11, 1e-12, "packed sequences y")
+    _close(got_last, want_last, 1e-11, 1e-12, "packed sequences last state")
+    # one sequence spanning the row is the plain scan
+    plain = oracle.selective_scan(u, delta, A, B, C, D=D, z=z, delta_bias=bias,
+                                  h0=h0, lib=lib)
+    one = oracle.selective_scan(u, delta, A, B, C, D=D, z=z, delta_bias=bias,
+                                h0=h0, lib=lib, cu_seqlens=[0, L])
+    _close(one, plain, 0.0, 0.0, "one packed sequence")
+
+
 ALL_PINS = [
     pin_combine_worked_example,
     pin_scan_worked_example,
@@ -412,4 +458,5 @@ ALL_PINS = [
     pin_special_cases,
     pin_softplus_silu,
     pin_resume,
+    pin_packed_sequences,
 ]

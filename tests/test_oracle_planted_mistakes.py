@@ -38,6 +38,9 @@ MUTATIONS = {
     "readout_before_update": (
         "        hp[n] = abar * hp[n] + bbar_u;\n        /* [eq]: y_t = C_t h_t, with the state after the update. */\n        acc += Cb[n * seqlen + t] * hp[n];",
         "        acc += Cb[n * seqlen + t] * hp[n];\n        hp[n] = abar * hp[n] + bbar_u;"),
+    "reset_dropped": ("          for (int64_t n = 0; n < dstate; ++n) hp[n] = 0.0;",
+                      "          ;"),
+    "reset_one_step_late": ("cu_seqlens[next] == t)", "cu_seqlens[next] == t - 1)"),
     "update_step_uses_input_twice": (
         "step * B[b * dstate + n] * x[ch];", "step * B[b * dstate + n] * x[ch] * x[ch];"),
 }
