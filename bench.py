@@ -40,6 +40,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import workloads  # noqa: E402
@@ -69,6 +70,9 @@ def parse_args(argv=None):
                     choices=[w.name for w in workloads.WORKLOADS])
     ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32",
                     help="dtype of y (f32 is the metric's configuration)")
+    ap.add_argument("--varlen", type=int, default=0,
+                    help="pack this many independent sequences into every row "
+                         "(seeded random offsets; 0 = one sequence per row)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work of the oracle baseline sample")
@@ -115,6 +119,14 @@ def profiled_traffic(workload: str):
     except Exception:
         pass
     return None
+
+
+def varlen_offsets(L: int, n: int) -> list:
+    """n sequences packed into a row of L steps: seeded random interior
+    offsets, the same for every row."""
+    rng = np.random.default_rng(48000 + n)
+    cuts = rng.choice(np.arange(1, L), size=min(n - 1, L - 1), replace=False)
+    return [0] + sorted(int(c) for c in cuts) + [L]
 
 
 def out_bytes(out_dtype: str) -> int:
@@ -291,10 +303,14 @@ def run_ours(args, rank, world, local_rank):
     inp = workloads.make_inputs(w, device=dev)
     ydt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
     y = torch.empty((w.batch, w.dim, w.seqlen), dtype=ydt, device=dev)
+    cu_t = None
+    if args.varlen > 0:
+        cu_t = torch.tensor(varlen_offsets(w.seqlen, args.varlen),
+                            dtype=torch.int32, device=dev)
     sargs = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"],
                                inp["C"], D=inp["D"], z=inp["z"],
                                delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, y=y)
+                               delta_softplus=w.softplus, y=y, cu_seqlens=cu_t)
     ws_bytes = sss.scan_workspace_size(sargs)
     ws = sss.alloc_workspace(ws_bytes, dev)
     if ws is not None:
@@ -363,7 +379,8 @@ def run_ours(args, rank, world, local_rank):
         sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"],
                                inp["C"], D=inp["D"], z=inp["z"],
                                delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, y=y, workspace=ws)
+                               delta_softplus=w.softplus, y=y, workspace=ws,
+                               cu_seqlens=cu_t)
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -399,7 +416,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": workload_config(w, args.out_dtype),
+        "config": dict(workload_config(w, args.out_dtype),
+                       **({"sequences_per_row": args.varlen} if args.varlen else {})),
         "state_updates_per_s": updates,
         "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": value / world / peak,

@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 2
+#define MSS_ABI_VERSION 3
 
 typedef enum {
   MSS_OK = 0,
@@ -133,6 +133,17 @@ typedef struct mss_scan_args {
   int64_t stride_B[2];
   int64_t stride_C[2];
   int64_t stride_y[2];
+  /* packed sequences: NULL, or num_seqs + 1 int32 offsets (device memory,
+     0 = cu_seqlens[0] <= ... <= cu_seqlens[num_seqs] = seqlen) dividing
+     every batch row into num_seqs independent sequences.  The state
+     restarts from zero at each interior offset; h0 seeds the first
+     sequence of a row and last_state receives the end of its last.
+     Requires A <= 0 (a restart is a decay of exactly zero).  The offsets
+     are read on the device and not validated there: offsets that are not
+     ordered restart the state at the wrong steps but read nothing out of
+     bounds. */
+  const int32_t *cu_seqlens;
+  int64_t num_seqs;     /* 0 when cu_seqlens is NULL */
 } mss_scan_args;
 
 /* Bytes of device workspace the scan needs for these arguments (0 when the

@@ -24,7 +24,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 2  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 3  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -81,6 +81,8 @@ class ScanArgs(ctypes.Structure):
         ("stride_B", ctypes.c_int64 * 2),
         ("stride_C", ctypes.c_int64 * 2),
         ("stride_y", ctypes.c_int64 * 2),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("num_seqs", ctypes.c_int64),
     ]
 
 
@@ -192,7 +194,7 @@ def _stream_handle(stream):
 def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                    delta_softplus=True, h0=None, y=None, last_state=None,
                    workspace=None, plan_splits=0, test_flags=0,
-                   spin_timeout_ns=0) -> ScanArgs:
+                   spin_timeout_ns=0, cu_seqlens=None) -> ScanArgs:
     batch, dim, L = u.shape
     N = A.shape[1]
     ind = u.dtype
@@ -223,6 +225,12 @@ def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     a.plan_chunk_steps = 0
     a.test_flags = int(test_flags)
     a.spin_timeout_ns = int(spin_timeout_ns)
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int32)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must hold num_seqs + 1 >= 2 offsets")
+        a.cu_seqlens = cu_seqlens.data_ptr()
+        a.num_seqs = cu_seqlens.numel() - 1
     for name, t in (("u", u), ("delta", delta), ("z", z), ("B", B), ("C", C), ("y", y)):
         if t is not None:
             getattr(a, "stride_" + name)[0] = t.stride(0)
@@ -249,13 +257,17 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                        delta_softplus=True, h0=None, return_last_state=False,
                        out_dtype=torch.float32, y=None, last_state=None,
                        workspace=None, stream=None, plan_splits=0,
-                       test_flags=0, spin_timeout_ns=0, check_status=False):
+                       test_flags=0, spin_timeout_ns=0, check_status=False,
+                       cu_seqlens=None):
     """Forward selective scan through ``mamba_selective_scan_fwd``.
 
     u, delta, z: (batch, dim, L); B, C: (batch, N, L) (float32 or bfloat16,
     all the same dtype); A: (dim, N), D, delta_bias: (dim,), h0:
-    (batch, dim, N) float32.  Returns y (batch, dim, L) in ``out_dtype``
-    (and the final state when ``return_last_state``).
+    (batch, dim, N) float32.  u, delta, z, B, C and y may be views whose
+    last dimension is contiguous.  ``cu_seqlens`` (int32 CUDA tensor of
+    num_seqs + 1 offsets, 0 ... L) packs independent sequences into every
+    row.  Returns y (batch, dim, L) in ``out_dtype`` (and the final state
+    when ``return_last_state``).
     """
     batch, dim, L = u.shape
     N = A.shape[1]
@@ -266,7 +278,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                                  device=u.device)
     args = make_scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus,
                           h0, y, last_state, None, plan_splits, test_flags,
-                          spin_timeout_ns)
+                          spin_timeout_ns, cu_seqlens)
     if workspace is None:
         workspace = alloc_workspace(scan_workspace_size(args), u.device)
     if workspace is not None:

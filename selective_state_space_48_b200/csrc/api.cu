@@ -113,6 +113,10 @@ mss_status check_scan_args(const mss_scan_args *a) {
     ScanParams probe{};
     if (!resolve_scan_strides(a, &probe)) return MSS_ERR_INVALID_ARG;
   }
+  if (a->cu_seqlens ? (a->num_seqs < 1 || a->num_seqs > INT32_MAX ||
+                       !aligned(a->cu_seqlens, 4))
+                    : a->num_seqs != 0)
+    return MSS_ERR_INVALID_ARG;
   const size_t ei = esize(a->in_dtype), eo = esize(a->out_dtype);
   if (!aligned(a->u, ei) || !aligned(a->delta, ei) || !aligned(a->B, ei) ||
       !aligned(a->C, ei) || (a->z && !aligned(a->z, ei)) ||
@@ -180,6 +184,8 @@ void fill_scan_params(const mss_scan_args *a, const Plan &pl, ScanParams *p) {
   p->y = a->y;
   p->last_state = a->last_state;
   resolve_scan_strides(a, p);  // checked in check_scan_args
+  p->cu = a->cu_seqlens;
+  p->nseq = a->cu_seqlens ? a->num_seqs : 0;
   p->chunk = pl.chunk;
   p->splits = pl.splits;
   p->ch_tiles = pl.ch_tiles;

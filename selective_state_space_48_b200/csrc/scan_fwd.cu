@@ -139,6 +139,36 @@ struct Scan {
     return static_cast<int>(min64(TB, t_end - t0_of(blk)));
   }
 
+  // ---- packed sequences.  Index of the first interior start cu[i]
+  // (1 <= i < nseq) at or after step pos, nseq when there is none.
+  __device__ int64_t first_start_from(int64_t pos) const {
+    int64_t lo = 1, hi = p.nseq;
+    while (lo < hi) {
+      const int64_t mid = lo + (hi - lo) / 2;
+      if (__ldg(p.cu + mid) < pos) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  }
+  // Bit j (j < 4) set when step pos + j (< t_end) starts a sequence; `nb`
+  // is the caller's cursor into cu, only ever moved forward.
+  __device__ uint32_t restarts4(int64_t pos, int64_t &nb) const {
+    uint32_t m = 0;
+    for (int j = 0; j < 4 && pos + j < t_end; ++j) {
+      while (nb < p.nseq && __ldg(p.cu + nb) < pos + j) ++nb;
+      if (nb < p.nseq && __ldg(p.cu + nb) == pos + j) m |= 1u << j;
+    }
+    return m;
+  }
+  // A restart is a step of infinite Delta: exp(Delta A) = 0 while the
+  // input term keeps the finite Delta (written to the Delta*u tile first).
+  static __device__ __forceinline__ void mark_restarts(float4 &dl, uint32_t m) {
+    const float inf = __int_as_float(0x7f800000);
+    if (m & 1u) dl.x = inf;
+    if (m & 2u) dl.y = inf;
+    if (m & 4u) dl.z = inf;
+    if (m & 8u) dl.w = inf;
+  }
+
   // thread 0: start the TMA copies of block `blk` into `stage`
   __device__ void issue(int stage, int blk) const {
     const uint32_t bytes = static_cast<uint32_t>(
@@ -229,7 +259,8 @@ struct Scan {
   // `set`, two timesteps per thread and iteration.  Steps past the end of
   // the chunk get Delta = 0: exp(0 * A) = 1 and no input, so they leave the
   // state unchanged.
-  __device__ void prep(int stage, int set, int nt, bool with_b, int ti, int nth) const {
+  __device__ void prep(int stage, int set, int64_t t0, int nt, bool with_b, int ti,
+                       int nth) const {
     const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
     float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
     const float *sBias = f32(Lay::bias);
@@ -252,9 +283,13 @@ struct Scan {
         if (t + 2 >= nt) dl.z = 0.f;
         if (t + 3 >= nt) dl.w = 0.f;
       }
-      *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
       *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
           make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
+      if (p.cu) {
+        int64_t nb = first_start_from(t0 + t);
+        mark_restarts(dl, restarts4(t0 + t, nb));
+      }
+      *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
     }
     const InT *rb = raw(stage, 3), *rc = raw(stage, 4);
     float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
@@ -347,7 +382,8 @@ struct Scan {
     return sl;
   }
 
-  __device__ void prep_slots(int stage, int set, int nt, const Slots &sl, int ti) const {
+  __device__ void prep_slots(int stage, int set, int nt, const Slots &sl, int ti,
+                             uint32_t restarts) const {
     const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
     float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
 #pragma unroll
@@ -368,9 +404,10 @@ struct Scan {
         if (t + 2 >= nt) dl.z = 0.f;
         if (t + 3 >= nt) dl.w = 0.f;
       }
-      *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
       *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
           make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
+      if (restarts) mark_restarts(dl, restarts);
+      *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
     }
     const InT *rb = raw(stage, 3), *rc = raw(stage, 4);
     float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
@@ -593,6 +630,9 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     const int n = 4 * g + i;
     live[i] = dvalid && n < p.dstate;
     alpha[i] = live[i] ? p.A[d * p.dstate + n] * kLog2e : 0.f;
+    // with packed sequences a restart multiplies alpha by an infinite
+    // Delta: keep A = 0 states at a decay of exactly 1 elsewhere but 0 there
+    if (p.cu && alpha[i] == 0.f) alpha[i] = -1e-30f;
     h[i] = (live[i] && k == 0 && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
   }
   float dsum = 0.f;
@@ -626,10 +666,13 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     }
   } else if (is_prep) {
     const typename S::Slots sl = sc.make_slots(tp);
+    // cursor into the sequence offsets for this thread's steps
+    int64_t nb = p.cu ? sc.first_start_from(sc.t_begin + sl.t) : 0;
     for (int blk = 0; blk < nblk; ++blk) {
       if (blk >= 2) wait_hand(kTilesFree, blk & 1);
+      const uint32_t rs = p.cu ? sc.restarts4(sc.t0_of(blk) + sl.t, nb) : 0u;
       ok &= sc.wait_raw(blk, 0, phase);
-      sc.prep_slots(blk % STAGES, blk & 1, sc.nt_of(blk), sl, tp);
+      sc.prep_slots(blk % STAGES, blk & 1, sc.nt_of(blk), sl, tp, rs);
       mbar_arrive(sc.hand(kTilesReady, blk & 1));
     }
     // the prep warps waited on every raw block: their phases seed the
@@ -768,7 +811,7 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
       return;
     }
     const int stage = (base + i) % STAGES;
-    sc.prep(stage, 0, sc.nt_of(i), false, tid, NALL);
+    sc.prep(stage, 0, sc.t0_of(i), sc.nt_of(i), false, tid, NALL);
     __syncthreads();
     if (is_scan) sc.scan_carry(0, g, lane, alpha, h_in, sigma, wactive);
     __syncthreads();

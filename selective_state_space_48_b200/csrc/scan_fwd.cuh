@@ -33,6 +33,10 @@ struct ScanParams {
   // element strides {batch, row} of the (batch, rows, seqlen) tensors (time
   // is contiguous); always resolved, never 0
   int64_t su[2], sdl[2], sz[2], sB[2], sC[2], sy[2];
+  // packed sequences (nullptr: one sequence per row): interior offsets
+  // cu[1 .. nseq-1] restart the state
+  const int32_t *cu;
+  int64_t nseq;
   int y_vec;       // rows of y allow 4-element vector stores (set at launch)
   // launch plan
   int64_t chunk;   // timesteps per sequence chunk (multiple of kTimeBlock)

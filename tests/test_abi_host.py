@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 2
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 3
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
@@ -140,6 +140,9 @@ def test_workspace_size_follows_plan(lib):
     (dict(stride_y=(39 * 4096, 4096)), sss.MSS_ERR_INVALID_ARG),  # y batches overlap
     (dict(stride_y=(0, 4096)), sss.MSS_ERR_INVALID_ARG),          # y batches alias
     (dict(stride_z=(1 << 50, 4096)), sss.MSS_ERR_INVALID_ARG),    # absurd
+    (dict(num_seqs=3), sss.MSS_ERR_INVALID_ARG),                  # offsets missing
+    (dict(cu_seqlens=0x10000, num_seqs=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(cu_seqlens=0x10002, num_seqs=2), sss.MSS_ERR_INVALID_ARG),  # misaligned
 ])
 def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     a = _args(**kw)
@@ -156,6 +159,7 @@ def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     dict(stride_C=(16 * 4096, 4096 + 8)),      # padded rows
     dict(stride_y=(41 * 4100, 4100)),          # y inside a larger buffer
     dict(stride_delta=(0, 0)),                 # packed
+    dict(cu_seqlens=0x10000, num_seqs=5),      # packed sequences
 ])
 def test_valid_strides_are_accepted(lib, kw):
     rc, n = _ws(lib, _args(plan_splits=1, **kw))
