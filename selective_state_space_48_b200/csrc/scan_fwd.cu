@@ -101,7 +101,7 @@ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) {
   return a < b ? a : b;
 }
 
-template <typename InT, typename OutT, int G, bool TMA>
+template <typename InT, typename OutT, int G, bool TMA, bool VARLEN>
 struct Scan {
   using Lay = Layout<InT, G>;
   static constexpr int NP = 4 * G;
@@ -285,7 +285,7 @@ struct Scan {
       }
       *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
           make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
-      if (p.cu) {
+      if (VARLEN && p.cu) {
         int64_t nb = first_start_from(t0 + t);
         mark_restarts(dl, restarts4(t0 + t, nb));
       }
@@ -568,10 +568,10 @@ constexpr int kPartFree = 3;    // epi -> scan: y shares of a block consumed
 constexpr int kBarEpi = 1;      // named barrier of the epilogue warps only
 constexpr uint64_t kHandoffWaitNs = 2000000000ull;
 
-template <typename InT, typename OutT, int G, bool TMA>
+template <typename InT, typename OutT, int G, bool TMA, bool VARLEN>
 __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     scan_fwd_kernel(const ScanParams p, const __grid_constant__ TmaMaps maps) {
-  using S = Scan<InT, OutT, G, TMA>;
+  using S = Scan<InT, OutT, G, TMA, VARLEN>;
   using Lay = typename S::Lay;
   constexpr int NP = 4 * G;
   constexpr int NSCAN = 32 * G;
@@ -632,7 +632,7 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     alpha[i] = live[i] ? p.A[d * p.dstate + n] * kLog2e : 0.f;
     // with packed sequences a restart multiplies alpha by an infinite
     // Delta: keep A = 0 states at a decay of exactly 1 elsewhere but 0 there
-    if (p.cu && alpha[i] == 0.f) alpha[i] = -1e-30f;
+    if (VARLEN && alpha[i] == 0.f) alpha[i] = -1e-30f;
     h[i] = (live[i] && k == 0 && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
   }
   float dsum = 0.f;
@@ -667,10 +667,10 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   } else if (is_prep) {
     const typename S::Slots sl = sc.make_slots(tp);
     // cursor into the sequence offsets for this thread's steps
-    int64_t nb = p.cu ? sc.first_start_from(sc.t_begin + sl.t) : 0;
+    int64_t nb = VARLEN ? sc.first_start_from(sc.t_begin + sl.t) : 0;
     for (int blk = 0; blk < nblk; ++blk) {
       if (blk >= 2) wait_hand(kTilesFree, blk & 1);
-      const uint32_t rs = p.cu ? sc.restarts4(sc.t0_of(blk) + sl.t, nb) : 0u;
+      const uint32_t rs = VARLEN ? sc.restarts4(sc.t0_of(blk) + sl.t, nb) : 0u;
       ok &= sc.wait_raw(blk, 0, phase);
       sc.prep_slots(blk % STAGES, blk & 1, sc.nt_of(blk), sl, tp, rs);
       mbar_arrive(sc.hand(kTilesReady, blk & 1));
@@ -896,9 +896,9 @@ bool build_maps(const ScanParams &p, int in_bf16, int groups, TmaMaps *m) {
   return true;
 }
 
-template <typename InT, typename OutT, int G, bool TMA>
+template <typename InT, typename OutT, int G, bool TMA, bool VARLEN>
 cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t s) {
-  auto kern = scan_fwd_kernel<InT, OutT, G, TMA>;
+  auto kern = scan_fwd_kernel<InT, OutT, G, TMA, VARLEN>;
   const int smem = Layout<InT, G>::bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -907,27 +907,35 @@ cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t 
   return cudaGetLastError();
 }
 
-template <typename InT, typename OutT>
-cudaError_t dispatch(const ScanParams &p, bool tma, const TmaMaps &maps, cudaStream_t s) {
+// Packed sequences get their own instantiations, so the code that finds and
+// applies restarts never touches the kernels of ordinary scans.
+template <typename InT, typename OutT, bool VARLEN>
+cudaError_t dispatch_v(const ScanParams &p, bool tma, const TmaMaps &maps, cudaStream_t s) {
   const int G = static_cast<int>((p.dstate + 3) / 4);
   if (tma) {
     switch (G) {
-      case 1: return launch_typed<InT, OutT, 1, true>(p, maps, s);
-      case 2: return launch_typed<InT, OutT, 2, true>(p, maps, s);
-      default: return launch_typed<InT, OutT, 4, true>(p, maps, s);
+      case 1: return launch_typed<InT, OutT, 1, true, VARLEN>(p, maps, s);
+      case 2: return launch_typed<InT, OutT, 2, true, VARLEN>(p, maps, s);
+      default: return launch_typed<InT, OutT, 4, true, VARLEN>(p, maps, s);
     }
   }
   switch (G) {
-    case 1: return launch_typed<InT, OutT, 1, false>(p, maps, s);
-    case 2: return launch_typed<InT, OutT, 2, false>(p, maps, s);
-    default: return launch_typed<InT, OutT, 4, false>(p, maps, s);
+    case 1: return launch_typed<InT, OutT, 1, false, VARLEN>(p, maps, s);
+    case 2: return launch_typed<InT, OutT, 2, false, VARLEN>(p, maps, s);
+    default: return launch_typed<InT, OutT, 4, false, VARLEN>(p, maps, s);
   }
+}
+
+template <typename InT, typename OutT>
+cudaError_t dispatch(const ScanParams &p, bool tma, const TmaMaps &maps, cudaStream_t s) {
+  return p.cu ? dispatch_v<InT, OutT, true>(p, tma, maps, s)
+              : dispatch_v<InT, OutT, false>(p, tma, maps, s);
 }
 
 template <typename InT, typename OutT, int G>
 int occupancy_typed() {
   int n = 0;
-  auto kern = scan_fwd_kernel<InT, OutT, G, true>;
+  auto kern = scan_fwd_kernel<InT, OutT, G, true, false>;
   const int smem = Layout<InT, G>::bytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
