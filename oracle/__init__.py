@@ -67,6 +67,9 @@ def _bind(lib):
     lib.oracle_selective_state_update_f64.argtypes = (
         [_I64] * 3 + [_D] * 9 + [ctypes.c_int, _D])
     lib.oracle_selective_state_update_f64.restype = ctypes.c_int
+    lib.oracle_selective_scan_bwd_f64.argtypes = (
+        [_I64] * 4 + [_D] * 8 + [ctypes.c_int] + [_D] * 12)
+    lib.oracle_selective_scan_bwd_f64.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -185,3 +188,33 @@ def selective_state_update(state, x, dt, A, B, C, D=None, z=None,
 def num_threads(lib=None) -> int:
     lib = lib or load()
     return int(lib.oracle_num_threads())
+
+
+def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                       delta_softplus=True, h0=None, d_last=None, lib=None):
+    """fp64 gradient of ``selective_scan`` for the loss
+    sum(dy * y) + sum(d_last * last_state).  Returns a dict with du, ddelta,
+    dA, dB, dC, dD, dz, ddelta_bias, dh0 (None where the input is absent)."""
+    lib = lib or load()
+    u, delta, A, B, C, dy = (_f64(x) for x in (u, delta, A, B, C, dy))
+    D, z, delta_bias, h0, d_last = (_f64(x) for x in (D, z, delta_bias, h0, d_last))
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    out = {
+        "du": np.empty((batch, dim, L)), "ddelta": np.empty((batch, dim, L)),
+        "dA": np.empty((dim, N)), "dB": np.empty((batch, N, L)),
+        "dC": np.empty((batch, N, L)),
+        "dD": np.empty(dim) if D is not None else None,
+        "dz": np.empty((batch, dim, L)) if z is not None else None,
+        "ddelta_bias": np.empty(dim) if delta_bias is not None else None,
+        "dh0": np.empty((batch, dim, N)),
+    }
+    rc = lib.oracle_selective_scan_bwd_f64(
+        batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+        _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)),
+        _ptr(h0), _ptr(dy), _ptr(d_last), _ptr(out["du"]), _ptr(out["ddelta"]),
+        _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]),
+        _ptr(out["dz"]), _ptr(out["ddelta_bias"]), _ptr(out["dh0"]))
+    if rc != 0:
+        raise ValueError("oracle_selective_scan_bwd_f64 rejected the sizes")
+    return out

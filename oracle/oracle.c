@@ -30,6 +30,8 @@
 
 #include <math.h>
 #include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
 
 #ifdef _OPENMP
 #include <omp.h>
@@ -160,6 +162,151 @@ int oracle_selective_state_update_f64(int64_t batch, int64_t dim,
     }
   }
   return 0;
+}
+
+/* Gradient of the full selective scan by the chain rule, sequential over t
+ * (reverse-time adjoint).  The backward pass recomputes the states it needs
+ * from the inputs instead of receiving them from the forward pass ("Mamba
+ * is attention all you really need, part 2", section "Keeping the pad on
+ * the desk"; "The State That Must Remember Everything", Part 3, "The
+ * Hardware-Aware Way Out", rematerialisation).  Here the recomputation is
+ * simply a forward sweep that keeps every state of one channel.
+ *
+ * Loss: sum(dy * y) + sum(d_last * last_state).  With s_t = sum_n C_t[n]
+ * h_t[n] + D u_t, g_t = silu(z_t) (1 without z), y_t = s_t g_t:
+ *   lam_t[n] = ds_t C_t[n] + exp(Delta_{t+1} A[n]) lam_{t+1}[n],
+ *              lam_{L-1} starting from d_last,        ds_t = dy_t g_t
+ *   dDelta_t = sum_n lam_t[n] (A[n] a_t[n] h_{t-1}[n] + B_t[n] u_t)
+ *   dA[d,n] += lam_t[n] Delta_t a_t[n] h_{t-1}[n]
+ *   dB_t[n] += lam_t[n] Delta_t u_t        dC_t[n] += ds_t h_t[n]
+ *   du_t     = ds_t D + sum_n lam_t[n] Delta_t B_t[n]
+ *   dD      += ds_t u_t                     dz_t = dy_t s_t silu'(z_t)
+ *   ddelta_t = dDelta_t sigmoid(delta_t + bias)   (dDelta_t without softplus)
+ *   dbias   += ddelta_t                     dh0 = a_0 lam_0
+ * dB, dC sum over channels, dA, dD, dbias over batch rows.  Every output
+ * is overwritten (not accumulated into).  Returns 0, or -1 on a bad size
+ * or allocation failure. */
+static double dsilu(double z) {
+  const double sg = 1.0 / (1.0 + exp(-z));
+  return sg * (1.0 + z * (1.0 - sg));
+}
+
+int oracle_selective_scan_bwd_f64(
+    int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+    const double *u, const double *delta, const double *A, const double *B,
+    const double *C, const double *D, const double *z,
+    const double *delta_bias, int delta_softplus, const double *h0,
+    const double *dy, const double *d_last, double *du, double *ddelta,
+    double *dA, double *dB, double *dC, double *dD, double *dz,
+    double *ddelta_bias, double *dh0) {
+  if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256 || seqlen < 0)
+    return -1;
+  const int64_t N = dstate, L = seqlen;
+  /* per batch row partial sums of the per-channel parameter gradients */
+  double *pA = calloc((size_t)(batch * dim * N + 1), sizeof(double));
+  double *pD = calloc((size_t)(batch * dim + 1), sizeof(double));
+  double *pb = calloc((size_t)(batch * dim + 1), sizeof(double));
+  if (!pA || !pD || !pb) {
+    free(pA); free(pD); free(pb);
+    return -1;
+  }
+  memset(dB, 0, sizeof(double) * (size_t)(batch * N * L));
+  memset(dC, 0, sizeof(double) * (size_t)(batch * N * L));
+  int failed = 0;
+
+  /* Batch rows own disjoint dB, dC slices, so they run in parallel; the
+   * channels of one row are visited in order. */
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+  for (int64_t b = 0; b < batch; ++b) {
+    double *H = malloc(sizeof(double) * (size_t)((L + 1) * N));
+    double *S = malloc(sizeof(double) * (size_t)(L + 1));
+    double *Dt = malloc(sizeof(double) * (size_t)(L + 1));
+    if (!H || !S || !Dt) {
+      free(H); free(S); free(Dt);
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+      failed = 1;
+      continue;
+    }
+    const double *Bb = B + b * N * L, *Cb = C + b * N * L;
+    double *dBb = dB + b * N * L, *dCb = dC + b * N * L;
+    for (int64_t d = 0; d < dim; ++d) {
+      const int64_t row = (b * dim + d) * L;
+      const double bias = delta_bias ? delta_bias[d] : 0.0;
+      const double dskip = D ? D[d] : 0.0;
+      /* forward sweep keeping every state: H[t + 1] = h_t, H[0] = h_{-1} */
+      for (int64_t n = 0; n < N; ++n)
+        H[n] = h0 ? h0[(b * dim + d) * N + n] : 0.0;
+      for (int64_t t = 0; t < L; ++t) {
+        const double dt = step_size(delta[row + t], bias, delta_softplus);
+        Dt[t] = dt;
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+          const double h = exp(dt * A[d * N + n]) * H[t * N + n] +
+                           dt * Bb[n * L + t] * u[row + t];
+          H[(t + 1) * N + n] = h;
+          acc += Cb[n * L + t] * h;
+        }
+        S[t] = acc + dskip * u[row + t];
+      }
+      /* reverse sweep */
+      double lam[256];
+      for (int64_t n = 0; n < N; ++n)
+        lam[n] = d_last ? d_last[(b * dim + d) * N + n] : 0.0;
+      double accD = 0.0, accb = 0.0;
+      for (int64_t t = L - 1; t >= 0; --t) {
+        const double ut = u[row + t], dt = Dt[t];
+        const double g = z ? oracle_silu_f64(z[row + t]) : 1.0;
+        const double ds = dy[row + t] * g;
+        if (z && dz) dz[row + t] = dy[row + t] * S[t] * dsilu(z[row + t]);
+        accD += ds * ut;
+        double dut = ds * dskip, dDelta = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+          const double an = A[d * N + n];
+          const double a = exp(dt * an);
+          const double hprev = H[t * N + n];
+          lam[n] += ds * Cb[n * L + t];
+          dCb[n * L + t] += ds * H[(t + 1) * N + n];
+          dDelta += lam[n] * (an * a * hprev + Bb[n * L + t] * ut);
+          pA[(b * dim + d) * N + n] += lam[n] * dt * a * hprev;
+          dBb[n * L + t] += lam[n] * dt * ut;
+          dut += lam[n] * dt * Bb[n * L + t];
+          lam[n] *= a;
+        }
+        du[row + t] = dut;
+        const double x = delta[row + t] + bias;
+        const double dd = delta_softplus ? dDelta / (1.0 + exp(-x)) : dDelta;
+        ddelta[row + t] = dd;
+        accb += dd;
+      }
+      if (dh0)
+        for (int64_t n = 0; n < N; ++n) dh0[(b * dim + d) * N + n] = lam[n];
+      pD[b * dim + d] = accD;
+      pb[b * dim + d] = accb;
+    }
+    free(H); free(S); free(Dt);
+  }
+  if (!failed) {
+    for (int64_t d = 0; d < dim; ++d) {
+      double sD = 0.0, sb = 0.0;
+      for (int64_t b = 0; b < batch; ++b) {
+        sD += pD[b * dim + d];
+        sb += pb[b * dim + d];
+      }
+      if (dD) dD[d] = sD;
+      if (ddelta_bias) ddelta_bias[d] = sb;
+      for (int64_t n = 0; n < N; ++n) {
+        double s = 0.0;
+        for (int64_t b = 0; b < batch; ++b) s += pA[(b * dim + d) * N + n];
+        dA[d * N + n] = s;
+      }
+    }
+  }
+  free(pA); free(pD); free(pb);
+  return failed ? -1 : 0;
 }
 
 int oracle_num_threads(void) {

@@ -70,6 +70,21 @@ int oracle_selective_state_update_f64(int64_t batch, int64_t dim,
                                       int dt_softplus, double *y);
 
 /* Number of OpenMP threads the scan uses (1 when built without OpenMP). */
+/* Gradient of the selective scan above (no packed sequences) for the loss
+ * sum(dy * y) + sum(d_last * last_state): du, ddelta, dz (batch, dim,
+ * seqlen), dA (dim, dstate), dB, dC (batch, dstate, seqlen), dD,
+ * ddelta_bias (dim), dh0 (batch, dim, dstate).  d_last, dz, dD,
+ * ddelta_bias and dh0 may be NULL.  Returns 0, or -1 on a bad size or an
+ * allocation failure. */
+int oracle_selective_scan_bwd_f64(
+    int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+    const double *u, const double *delta, const double *A, const double *B,
+    const double *C, const double *D, const double *z,
+    const double *delta_bias, int delta_softplus, const double *h0,
+    const double *dy, const double *d_last, double *du, double *ddelta,
+    double *dA, double *dB, double *dC, double *dD, double *dz,
+    double *ddelta_bias, double *dh0);
+
 int oracle_num_threads(void);
 
 #ifdef __cplusplus

@@ -445,6 +445,54 @@ def pin_packed_sequences(lib):
     _close(one, plain, 0.0, 0.0, "one packed sequence")
 
 
+# --------------------------------------------------------------------------
+# The backward pass: every gradient against central finite differences of
+# the forward oracle (pinned above) along a random direction, i.e.
+# <grad_X, V> = (F(X + eps V) - F(X - eps V)) / (2 eps) with
+# F = sum(dy * y) + sum(d_last * last_state).
+
+
+def _fd_check(lib, case, seed):
+    rng = _rng(seed)
+    bt, dm, N, L = case["shape"]
+    sp = case["softplus"]
+    X = dict(
+        u=rng.normal(size=(bt, dm, L)),
+        delta=rng.normal(size=(bt, dm, L)) if sp else rng.uniform(0.05, 0.6, size=(bt, dm, L)),
+        A=-rng.uniform(0.2, 2.0, size=(dm, N)),
+        B=rng.normal(size=(bt, N, L)), C=rng.normal(size=(bt, N, L)),
+        D=rng.normal(size=dm), z=rng.normal(size=(bt, dm, L)),
+        delta_bias=rng.normal(size=dm) * 0.5, h0=rng.normal(size=(bt, dm, N)))
+    dy = rng.normal(size=(bt, dm, L))
+    d_last = rng.normal(size=(bt, dm, N))
+
+    def F(X):
+        y, last = oracle.selective_scan(X["u"], X["delta"], X["A"], X["B"], X["C"],
+                                        D=X["D"], z=X["z"], delta_bias=X["delta_bias"],
+                                        delta_softplus=sp, h0=X["h0"],
+                                        return_last_state=True, lib=lib)
+        return float(np.sum(dy * y) + np.sum(d_last * last))
+
+    g = oracle.selective_scan_bwd(X["u"], X["delta"], X["A"], X["B"], X["C"], dy,
+                                  D=X["D"], z=X["z"], delta_bias=X["delta_bias"],
+                                  delta_softplus=sp, h0=X["h0"], d_last=d_last, lib=lib)
+    names = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC",
+             "D": "dD", "z": "dz", "delta_bias": "ddelta_bias", "h0": "dh0"}
+    eps = 1e-6
+    for k, gk in names.items():
+        V = rng.normal(size=X[k].shape)
+        Xp = dict(X); Xp[k] = X[k] + eps * V
+        Xm = dict(X); Xm[k] = X[k] - eps * V
+        fd = (F(Xp) - F(Xm)) / (2 * eps)
+        an = float(np.sum(g[gk] * V))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (k, fd, an, case)
+
+
+def pin_backward_finite_differences(lib):
+    _fd_check(lib, dict(shape=(2, 3, 4, 9), softplus=True), 31)
+    _fd_check(lib, dict(shape=(1, 2, 3, 13), softplus=False), 32)
+
+
 ALL_PINS = [
     pin_combine_worked_example,
     pin_scan_worked_example,
@@ -459,4 +507,5 @@ ALL_PINS = [
     pin_softplus_silu,
     pin_resume,
     pin_packed_sequences,
+    pin_backward_finite_differences,
 ]

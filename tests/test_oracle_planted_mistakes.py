@@ -41,6 +41,13 @@ MUTATIONS = {
     "reset_dropped": ("          for (int64_t n = 0; n < dstate; ++n) hp[n] = 0.0;",
                       "          ;"),
     "reset_one_step_late": ("cu_seqlens[next] == t)", "cu_seqlens[next] == t - 1)"),
+    "bwd_adjoint_not_decayed": ("          lam[n] *= a;\n", "\n"),
+    "bwd_dA_without_step": ("pA[(b * dim + d) * N + n] += lam[n] * dt * a * hprev;",
+                            "pA[(b * dim + d) * N + n] += lam[n] * a * hprev;"),
+    "bwd_dC_uses_previous_state": ("dCb[n * L + t] += ds * H[(t + 1) * N + n];",
+                                   "dCb[n * L + t] += ds * H[t * N + n];"),
+    "bwd_gate_derivative_wrong": ("return sg * (1.0 + z * (1.0 - sg));", "return sg;"),
+    "bwd_softplus_derivative_dropped": ("? dDelta / (1.0 + exp(-x)) : dDelta;", "? dDelta : dDelta;"),
     "update_step_uses_input_twice": (
         "step * B[b * dstate + n] * x[ch];", "step * B[b * dstate + n] * x[ch] * x[ch];"),
 }
