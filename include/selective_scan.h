@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 3
+#define MSS_ABI_VERSION 4
 
 typedef enum {
   MSS_OK = 0,
@@ -214,6 +214,63 @@ typedef struct mss_update_args {
 /* Single-token state update (decode): one step of the recurrence above for
  * every (batch, channel), state updated in place, y written. */
 mss_status selective_state_update(const mss_update_args *args, void *stream);
+
+/* Arguments of one backward scan: the gradients of
+ *   loss = sum(dy * y) + sum(d_last * last_state)
+ * for the forward scan with the same inputs (dense tensors, shapes as in
+ * mss_scan_args; no strides, no packed sequences).  The states are not
+ * taken from the forward pass but recomputed: a forward sweep stores the
+ * state of every channel at the start of every 16-step block in the
+ * workspace and a reverse sweep recomputes each block from it ("Mamba is
+ * attention all you really need, part 2", section "Keeping the pad on the
+ * desk"; "The State That Must Remember Everything", Part 3, "The
+ * Hardware-Aware Way Out").  Inputs: dy (batch, dim, seqlen) fp32 and
+ * d_last (batch, dim, dstate) fp32 or NULL.  Outputs, all fp32 and all
+ * overwritten: du, ddelta, dz (batch, dim, seqlen; dz NULL when z is), dA
+ * (dim, dstate), dB, dC (batch, dstate, seqlen), dD and ddelta_bias (dim;
+ * NULL when D / delta_bias are), dh0 (batch, dim, dstate) or NULL.  dA, dB,
+ * dC, dD and ddelta_bias are cleared with cudaMemsetAsync on the stream and
+ * then accumulated with atomics, so their low bits depend on the order in
+ * which blocks finish. */
+typedef struct mss_scan_bwd_args {
+  int64_t batch;
+  int64_t dim;
+  int64_t dstate;   /* 1..16 */
+  int64_t seqlen;
+  mss_dtype in_dtype; /* of u, delta, B, C, z */
+  const void *u;
+  const void *delta;
+  const float *A;
+  const void *B;
+  const void *C;
+  const float *D;
+  const void *z;
+  const float *delta_bias;
+  int delta_softplus;
+  const float *h0;
+  const float *dy;
+  const float *d_last;
+  float *du;
+  float *ddelta;
+  float *dA;
+  float *dB;
+  float *dC;
+  float *dD;
+  float *dz;
+  float *ddelta_bias;
+  float *dh0;
+  void *workspace;          /* device, >= mss_scan_bwd_workspace_size(),
+                               256-byte aligned */
+  size_t workspace_bytes;
+} mss_scan_bwd_args;
+
+/* Workspace bytes of the backward scan (the state checkpoints: 64 bytes per
+ * 16 steps of every channel, for dstate <= 16). */
+mss_status mss_scan_bwd_workspace_size(const mss_scan_bwd_args *args, size_t *bytes);
+
+/* Backward selective scan on `stream`; argument errors return before any
+ * work is enqueued. */
+mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *args, void *stream);
 
 /* Human-readable name of a status code (static string). */
 const char *mss_status_string(mss_status status);

@@ -24,7 +24,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 3  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 4  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -43,6 +43,8 @@ EXPORTED_SYMBOLS = (
     "mss_scan_status",
     "mamba_selective_scan_fwd_noalloc",
     "selective_state_update",
+    "mss_scan_bwd_workspace_size",
+    "mamba_selective_scan_bwd",
     "mss_status_string",
     "mss_abi_version",
 )
@@ -108,6 +110,24 @@ class UpdateArgs(ctypes.Structure):
     ]
 
 
+class ScanBwdArgs(ctypes.Structure):
+    """Mirror of ``mss_scan_bwd_args``."""
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("dim", ctypes.c_int64),
+        ("dstate", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("in_dtype", ctypes.c_int),
+    ] + [(name, ctypes.c_void_p) for name in (
+        "u", "delta", "A", "B", "C", "D", "z", "delta_bias")] + [
+        ("delta_softplus", ctypes.c_int),
+    ] + [(name, ctypes.c_void_p) for name in (
+        "h0", "dy", "d_last", "du", "ddelta", "dA", "dB", "dC", "dD", "dz",
+        "ddelta_bias", "dh0", "workspace")] + [
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 class MssError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
@@ -139,6 +159,10 @@ def load_library():
             lib.mamba_selective_scan_fwd_noalloc.restype = ctypes.c_int
             lib.selective_state_update.argtypes = [P(UpdateArgs), ctypes.c_void_p]
             lib.selective_state_update.restype = ctypes.c_int
+            lib.mss_scan_bwd_workspace_size.argtypes = [P(ScanBwdArgs), P(ctypes.c_size_t)]
+            lib.mss_scan_bwd_workspace_size.restype = ctypes.c_int
+            lib.mamba_selective_scan_bwd.argtypes = [P(ScanBwdArgs), ctypes.c_void_p]
+            lib.mamba_selective_scan_bwd.restype = ctypes.c_int
             lib.mss_status_string.argtypes = [ctypes.c_int]
             lib.mss_status_string.restype = ctypes.c_char_p
             lib.mss_abi_version.argtypes = []
@@ -346,3 +370,64 @@ __all__ = [
     "scan_status", "make_scan_args", "load_library", "status_string",
     "MssError", "ScanArgs", "UpdateArgs", "EXPORTED_SYMBOLS", "build",
 ]
+
+
+def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                       delta_softplus=True, h0=None, d_last=None, stream=None,
+                       workspace=None):
+    """Gradients of sum(dy * y) + sum(d_last * last_state) for the forward
+    scan on the same inputs, through ``mamba_selective_scan_bwd``.
+
+    Dense inputs as for ``selective_scan_fwd``; dy (batch, dim, L) and
+    d_last (batch, dim, N) float32.  Returns a dict of float32 tensors du,
+    ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0 (None for absent inputs).
+    """
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    ind = u.dtype
+    for name, t, dt, shape in (
+            ("u", u, ind, None), ("delta", delta, ind, (batch, dim, L)),
+            ("A", A, torch.float32, (dim, N)), ("B", B, ind, (batch, N, L)),
+            ("C", C, ind, (batch, N, L)), ("D", D, torch.float32, (dim,)),
+            ("z", z, ind, (batch, dim, L)),
+            ("delta_bias", delta_bias, torch.float32, (dim,)),
+            ("h0", h0, torch.float32, (batch, dim, N)),
+            ("dy", dy, torch.float32, (batch, dim, L)),
+            ("d_last", d_last, torch.float32, (batch, dim, N))):
+        _check_cuda(name, t, dt, shape)
+    dev = u.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {
+        "du": torch.empty((batch, dim, L), **f32),
+        "ddelta": torch.empty((batch, dim, L), **f32),
+        "dA": torch.empty((dim, N), **f32),
+        "dB": torch.empty((batch, N, L), **f32),
+        "dC": torch.empty((batch, N, L), **f32),
+        "dD": torch.empty((dim,), **f32) if D is not None else None,
+        "dz": torch.empty((batch, dim, L), **f32) if z is not None else None,
+        "ddelta_bias": torch.empty((dim,), **f32) if delta_bias is not None else None,
+        "dh0": torch.empty((batch, dim, N), **f32),
+    }
+    a = ScanBwdArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = batch, dim, N, L
+    a.in_dtype = _dtype_code(ind)
+    a.u, a.delta, a.A, a.B, a.C = _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C)
+    a.D, a.z, a.delta_bias = _ptr(D), _ptr(z), _ptr(delta_bias)
+    a.delta_softplus = 1 if delta_softplus else 0
+    a.h0, a.dy, a.d_last = _ptr(h0), _ptr(dy), _ptr(d_last)
+    for k, v in g.items():
+        setattr(a, k, _ptr(v))
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    rc = lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    if rc != MSS_OK:
+        raise MssError(rc, "mss_scan_bwd_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(int(n.value), dev)
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.mamba_selective_scan_bwd(ctypes.byref(a), _stream_handle(stream))
+    if rc != MSS_OK:
+        raise MssError(rc, "mamba_selective_scan_bwd")
+    workspace.record_stream(stream or torch.cuda.current_stream())
+    return g

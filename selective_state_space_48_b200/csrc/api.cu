@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "scan_bwd.cuh"
 #include "scan_fwd.cuh"
 #include "selective_scan.h"
 
@@ -300,6 +301,101 @@ mss_status selective_state_update(const mss_update_args *a, void *stream) {
   if (launch_state_update(p, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16,
                           static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSS_ERR_CUDA;
+  return MSS_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+mss_status check_bwd_args(const mss_scan_bwd_args *a) {
+  if (!a) return MSS_ERR_INVALID_ARG;
+  if (a->batch < 1 || a->dim < 1 || a->seqlen < 1 || a->dstate < 1)
+    return MSS_ERR_INVALID_ARG;
+  if (a->dstate > kMaxStates) return MSS_ERR_UNSUPPORTED;
+  if (!valid_dtype(a->in_dtype)) return MSS_ERR_INVALID_ARG;
+  const int64_t lim = int64_t(1) << 40;
+  if (a->batch > lim / a->dim || a->batch * a->dim > lim / a->seqlen)
+    return MSS_ERR_UNSUPPORTED;
+  if (!a->u || !a->delta || !a->A || !a->B || !a->C || !a->dy || !a->du ||
+      !a->ddelta || !a->dA || !a->dB || !a->dC)
+    return MSS_ERR_INVALID_ARG;
+  // a gradient is requested exactly for the optional inputs that are given
+  if ((a->D == nullptr) != (a->dD == nullptr) || (a->z == nullptr) != (a->dz == nullptr) ||
+      (a->delta_bias == nullptr) != (a->ddelta_bias == nullptr))
+    return MSS_ERR_INVALID_ARG;
+  const size_t ei = esize(a->in_dtype);
+  const void *in[] = {a->u, a->delta, a->B, a->C, a->z};
+  for (const void *q : in)
+    if (q && !aligned(q, ei)) return MSS_ERR_INVALID_ARG;
+  const void *f32[] = {a->A, a->D, a->delta_bias, a->h0, a->dy, a->d_last, a->du,
+                       a->ddelta, a->dA, a->dB, a->dC, a->dD, a->dz,
+                       a->ddelta_bias, a->dh0};
+  for (const void *q : f32)
+    if (q && !aligned(q, 4)) return MSS_ERR_INVALID_ARG;
+  return MSS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mss_status mss_scan_bwd_workspace_size(const mss_scan_bwd_args *a, size_t *bytes) {
+  if (!bytes) return MSS_ERR_INVALID_ARG;
+  const mss_status st = check_bwd_args(a);
+  if (st != MSS_OK) return st;
+  const int64_t tiles = a->batch * ((a->dim + kBwdChannels - 1) / kBwdChannels);
+  *bytes = scan_bwd_workspace_bytes(tiles, a->seqlen, a->dstate);
+  return MSS_OK;
+}
+
+mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
+  size_t need = 0;
+  const mss_status st = mss_scan_bwd_workspace_size(a, &need);
+  if (st != MSS_OK) return st;
+  if (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256))
+    return MSS_ERR_WORKSPACE;
+  BwdParams p{};
+  p.batch = a->batch;
+  p.dim = a->dim;
+  p.dstate = a->dstate;
+  p.seqlen = a->seqlen;
+  p.u = a->u;
+  p.delta = a->delta;
+  p.A = a->A;
+  p.B = a->B;
+  p.C = a->C;
+  p.D = a->D;
+  p.z = a->z;
+  p.delta_bias = a->delta_bias;
+  p.softplus = a->delta_softplus ? 1 : 0;
+  p.h0 = a->h0;
+  p.dy = a->dy;
+  p.d_last = a->d_last;
+  p.du = a->du;
+  p.ddelta = a->ddelta;
+  p.dA = a->dA;
+  p.dB = a->dB;
+  p.dC = a->dC;
+  p.dD = a->dD;
+  p.dz = a->dz;
+  p.ddelta_bias = a->ddelta_bias;
+  p.dh0 = a->dh0;
+  p.ckpt = static_cast<float *>(a->workspace);
+  p.ch_tiles = static_cast<int>((a->dim + kBwdChannels - 1) / kBwdChannels);
+  p.tiles = a->batch * p.ch_tiles;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the gradients that are sums over blocks are accumulated with atomics
+  const size_t f = sizeof(float);
+  const size_t nBC = static_cast<size_t>(a->batch * a->dstate * a->seqlen) * f;
+  if (cudaMemsetAsync(a->dA, 0, static_cast<size_t>(a->dim * a->dstate) * f, s) != cudaSuccess ||
+      cudaMemsetAsync(a->dB, 0, nBC, s) != cudaSuccess ||
+      cudaMemsetAsync(a->dC, 0, nBC, s) != cudaSuccess ||
+      (a->dD && cudaMemsetAsync(a->dD, 0, static_cast<size_t>(a->dim) * f, s) != cudaSuccess) ||
+      (a->ddelta_bias &&
+       cudaMemsetAsync(a->ddelta_bias, 0, static_cast<size_t>(a->dim) * f, s) != cudaSuccess))
+    return MSS_ERR_CUDA;
+  if (launch_scan_bwd(p, a->in_dtype == MSS_BF16, s) != cudaSuccess) return MSS_ERR_CUDA;
   return MSS_OK;
 }
 

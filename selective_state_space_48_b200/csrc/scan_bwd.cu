@@ -1,0 +1,360 @@
+// scan_bwd.cu -- backward pass of the selective scan (S6): gradients of
+// sum(dy * y) + sum(d_last * last_state) with respect to every input.
+//
+// The states are not kept from the forward pass; they are recomputed
+// ("Mamba is attention all you really need, part 2", section "Keeping the
+// pad on the desk"; "The State That Must Remember Everything", Part 3, "The
+// Hardware-Aware Way Out", rematerialisation).  One thread block owns 32
+// channels (one per lane) of one batch row, one warp per group of 4 states,
+// the same layout as the forward kernel:
+//
+//   forward sweep  walks the sequence in 16-step blocks and writes the state
+//                  at the start of every block to the workspace (the only
+//                  state that touches HBM: 64 B per channel and block);
+//   reverse sweep  walks the blocks backwards; for each it reloads the inputs,
+//                  recomputes the block's 16 states from the checkpoint into
+//                  registers, then runs the adjoint
+//                  lam_t = ds_t C_t + a_{t+1} lam_{t+1} step by step
+//                  (re-evaluating each decay a_t).
+//
+// With s_t = sum_n C_t[n] h_t[n] + D u_t, g_t = silu(z_t) and y_t = s_t g_t,
+// ds_t = dy_t g_t:
+//   dDelta_t = sum_n lam_t[n] (A[n] a_t[n] h_{t-1}[n] + B_t[n] u_t)
+//   dA[n]   += lam_t[n] Delta_t a_t[n] h_{t-1}[n]
+//   dB_t[n] += lam_t[n] Delta_t u_t       dC_t[n] += ds_t h_t[n]
+//   du_t     = ds_t D + sum_n lam_t[n] Delta_t B_t[n]
+//   dz_t     = dy_t s_t silu'(z_t),  ddelta_t = dDelta_t sigmoid(delta_t + bias)
+// Sums over the 16 states go through shared memory (one share per warp);
+// dB and dC, which sum over channels, are reduced across the warp's lanes
+// by a shuffle reduce-scatter every four steps and added to HBM with one
+// atomic per lane pair; dA, dD and dbias, which sum over channels of other
+// blocks and over batch rows, with one atomic per channel at the end.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "device_math.cuh"
+#include "scan_bwd.cuh"
+
+namespace sss48 {
+namespace {
+
+constexpr int CH = 32;
+constexpr int TB = 16;
+constexpr int ROW = TB + 4;  // padded fp32 row (conflict-free float4 reads)
+
+template <int G>
+struct BwdSmem {
+  static constexpr int NP = 4 * G;
+  // per (channel, step) tiles [CH][ROW]
+  float u[CH * ROW], dl[CH * ROW], du[CH * ROW], ds[CH * ROW], sg[CH * ROW],
+      z[CH * ROW], dy[CH * ROW];
+  // per (state, step) tiles [NP][TB]
+  float B[NP * TB], C[NP * TB];
+  // per warp shares [G][CH][ROW]: readout s_t, du_t, dDelta_t
+  float ps[G * CH * ROW], pu[G * CH * ROW], pd[G * CH * ROW];
+  float bias[CH], dskip[CH];
+  float accD[CH], accB[CH];  // per-channel sums of ds u and ddelta
+};
+
+template <typename T> __device__ __forceinline__ float ld_f32(const T *p, int64_t i);
+template <> __device__ __forceinline__ float ld_f32<float>(const float *p, int64_t i) {
+  return p[i];
+}
+template <> __device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16 *p,
+                                                                 int64_t i) {
+  return __bfloat162float(p[i]);
+}
+
+__device__ __forceinline__ float sigmoid_f(float x) {
+  return __fdividef(1.0f, 1.0f + ex2_mufu(-x * kLog2e));
+}
+
+// silu'(z) = sigmoid(z) (1 + z (1 - sigmoid(z)))
+__device__ __forceinline__ float dsilu_f(float z) {
+  const float s = sigmoid_f(z);
+  return s * fmaf(z, 1.0f - s, 1.0f);
+}
+
+// Sum over the 32 lanes of 16 values per lane (v[j], j = 4 i + tq): four
+// halving rounds leave lane l with the sum over the 16 lanes that share its
+// bit 0 for j = l >> 1; the last exchange completes it (both lanes of a pair
+// return the full sum of j = l >> 1).
+__device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int half = 8 >> r;
+    const int off = 16 >> r;
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const float send = upper ? v[j] : v[j + half];
+      const float keep = upper ? v[j + half] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+template <typename InT, int G>
+__global__ void __launch_bounds__(32 * G)
+    scan_bwd_kernel(const BwdParams p) {
+  using Sm = BwdSmem<G>;
+  constexpr int NP = Sm::NP;
+  constexpr int NT = 32 * G;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Sm &s = *reinterpret_cast<Sm *>(smem_raw);
+
+  const int tid = threadIdx.x, lane = tid & 31, g = tid >> 5;
+  const int64_t tile = blockIdx.x;
+  const int64_t b = tile / p.ch_tiles;
+  const int64_t d0 = (tile % p.ch_tiles) * CH;
+  const int64_t d = d0 + lane;
+  const bool dvalid = d < p.dim;
+  const int64_t L = p.seqlen;
+  const int nblk = static_cast<int>((L + TB - 1) / TB);
+
+  const InT *gu = static_cast<const InT *>(p.u);
+  const InT *gd = static_cast<const InT *>(p.delta);
+  const InT *gz = static_cast<const InT *>(p.z);
+  const InT *gB = static_cast<const InT *>(p.B);
+  const InT *gC = static_cast<const InT *>(p.C);
+
+  if (tid < CH) {
+    const bool ok = d0 + tid < p.dim;
+    s.bias[tid] = (ok && p.delta_bias) ? p.delta_bias[d0 + tid] : 0.f;
+    s.dskip[tid] = (ok && p.D) ? p.D[d0 + tid] : 0.f;
+    s.accD[tid] = 0.f;
+    s.accB[tid] = 0.f;
+  }
+
+  float alpha[4], an[4], h[4];
+  bool live[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = 4 * g + i;
+    live[i] = dvalid && n < p.dstate;
+    an[i] = live[i] ? p.A[d * p.dstate + n] : 0.f;
+    alpha[i] = an[i] * kLog2e;
+    h[i] = (live[i] && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
+  }
+  // state 4g + i of lane at the start of block k:
+  // ckpt[(k * NP + 4g + i) * CH + lane] (coalesced per warp)
+  float *ckpt = p.ckpt + tile * static_cast<int64_t>(nblk) * NP * CH;
+
+  // Block k of the inputs into the fp32 tiles with Delta and Delta*u (and,
+  // for the reverse sweep, z, dy, ds = dy silu(z), sigmoid(delta + bias)
+  // and C) -- all threads.
+  auto load_block = [&](int k, bool full) {
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+    for (int idx = tid; idx < CH * TB; idx += NT) {
+      const int c = idx / TB, t = idx % TB;
+      const int64_t dd = d0 + c;
+      const bool ok = dd < p.dim && t < nt;
+      const int64_t off = (b * p.dim + dd) * L + t0 + t;
+      const float uv = ok ? ld_f32(gu, off) : 0.f;
+      const float x = ok ? ld_f32(gd, off) + s.bias[c] : 0.f;
+      const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
+      s.u[c * ROW + t] = uv;
+      s.dl[c * ROW + t] = dl;
+      s.du[c * ROW + t] = dl * uv;
+      if (full) {
+        const float zv = (ok && gz) ? ld_f32(gz, off) : 0.f;
+        const float dyv = ok ? p.dy[off] : 0.f;
+        s.z[c * ROW + t] = zv;
+        s.dy[c * ROW + t] = dyv;
+        s.ds[c * ROW + t] = gz ? dyv * silu_f(zv) : dyv;
+        s.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
+      }
+    }
+    for (int idx = tid; idx < NP * TB; idx += NT) {
+      const int n = idx / TB, t = idx % TB;
+      const bool ok = n < p.dstate && t < nt;
+      const int64_t off = (b * p.dstate + n) * L + t0 + t;
+      s.B[idx] = ok ? ld_f32(gB, off) : 0.f;
+      if (full) s.C[idx] = ok ? ld_f32(gC, off) : 0.f;
+    }
+  };
+
+  // ------------------------------------------------------ forward sweep
+  __syncthreads();
+  for (int k = 0; k < nblk; ++k) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + i) * CH + lane] = h[i];
+    load_block(k, false);
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < TB; ++t) {
+      const float dl = s.dl[lane * ROW + t], du = s.du[lane * ROW + t];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        h[i] = fmaf(ex2_mufu(dl * alpha[i]), h[i], du * s.B[(4 * g + i) * TB + t]);
+    }
+    __syncthreads();
+  }
+
+  // ------------------------------------------------------ reverse sweep
+  float lam[4], dA[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lam[i] = (live[i] && p.d_last)
+                 ? p.d_last[(b * p.dim + d) * p.dstate + 4 * g + i] : 0.f;
+    dA[i] = 0.f;
+  }
+  for (int k = nblk - 1; k >= 0; --k) {
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+    load_block(k, true);
+    float hc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      hc[i] = ckpt[(static_cast<int64_t>(k) * NP + 4 * g + i) * CH + lane];
+    __syncthreads();
+
+    // recompute the block's states from the checkpoint; this warp's share
+    // of the readout s_t
+    float hs[4][TB];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float hh = hc[i];
+#pragma unroll
+      for (int t = 0; t < TB; ++t) {
+        hh = fmaf(ex2_mufu(s.dl[lane * ROW + t] * alpha[i]), hh,
+                  s.du[lane * ROW + t] * s.B[(4 * g + i) * TB + t]);
+        hs[i][t] = hh;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < TB; ++t) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc = fmaf(s.C[(4 * g + i) * TB + t], hs[i][t], acc);
+      s.ps[(g * CH + lane) * ROW + t] = acc;
+    }
+
+    // adjoint, four steps at a time backwards
+#pragma unroll
+    for (int q = TB / 4 - 1; q >= 0; --q) {
+      float vB[16], vC[16];
+#pragma unroll
+      for (int tq = 3; tq >= 0; --tq) {
+        const int t = 4 * q + tq;
+        const float dl = s.dl[lane * ROW + t], uu = s.u[lane * ROW + t],
+                    ds = s.ds[lane * ROW + t];
+        float pdu = 0.f, pdd = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int n = 4 * g + i;
+          const float Bv = s.B[n * TB + t], Cv = s.C[n * TB + t];
+          const float hprev = t > 0 ? hs[i][t - 1] : hc[i];
+          const float a = ex2_mufu(dl * alpha[i]);
+          lam[i] = fmaf(ds, Cv, lam[i]);
+          vC[4 * i + tq] = ds * hs[i][t];
+          const float la = lam[i] * a * hprev;
+          pdd = fmaf(lam[i], Bv * uu, fmaf(la, an[i], pdd));
+          dA[i] = fmaf(la, dl, dA[i]);
+          vB[4 * i + tq] = lam[i] * dl * uu;
+          pdu = fmaf(lam[i] * dl, Bv, pdu);
+          lam[i] *= a;
+        }
+        s.pu[(g * CH + lane) * ROW + t] = pdu;
+        s.pd[(g * CH + lane) * ROW + t] = pdd;
+      }
+      // channel sums of dB, dC for states 4g + i, steps 4q + tq: the even
+      // lane of each pair adds j = lane >> 1 = 4 i + tq
+      const float rb = reduce_scatter16(vB, lane);
+      const float rc = reduce_scatter16(vC, lane);
+      const int j = lane >> 1, n = 4 * g + j / 4, t = 4 * q + j % 4;
+      if ((lane & 1) == 0 && n < p.dstate && t < nt) {
+        const int64_t off = (b * p.dstate + n) * L + t0 + t;
+        atomicAdd(p.dB + off, rb);
+        atomicAdd(p.dC + off, rc);
+      }
+    }
+    __syncthreads();
+
+    // elementwise: du, ddelta, dz, and the per-channel sums of dD, dbias
+    for (int idx = tid; idx < CH * TB; idx += NT) {
+      const int c = idx / TB, t = idx % TB;
+      const int64_t dd = d0 + c;
+      if (dd >= p.dim || t >= nt) continue;
+      float sp = 0.f, su = 0.f, sd = 0.f;
+#pragma unroll
+      for (int w = 0; w < G; ++w) {
+        sp += s.ps[(w * CH + c) * ROW + t];
+        su += s.pu[(w * CH + c) * ROW + t];
+        sd += s.pd[(w * CH + c) * ROW + t];
+      }
+      const float uu = s.u[c * ROW + t], ds = s.ds[c * ROW + t];
+      const int64_t off = (b * p.dim + dd) * L + t0 + t;
+      p.du[off] = fmaf(ds, s.dskip[c], su);
+      const float ddl = sd * s.sg[c * ROW + t];
+      p.ddelta[off] = ddl;
+      if (p.dz) {
+        const float sv = fmaf(s.dskip[c], uu, sp);
+        p.dz[off] = s.dy[c * ROW + t] * sv * dsilu_f(s.z[c * ROW + t]);
+      }
+      atomicAdd(&s.accD[c], ds * uu);
+      atomicAdd(&s.accB[c], ddl);
+    }
+    __syncthreads();
+  }
+
+  // parameter gradients, summed over batch rows (and dh0 = lam_{-1})
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (!live[i]) continue;
+    const int n = 4 * g + i;
+    atomicAdd(p.dA + d * p.dstate + n, dA[i]);
+    if (p.dh0) p.dh0[(b * p.dim + d) * p.dstate + n] = lam[i];
+  }
+  if (tid < CH && d0 + tid < p.dim) {
+    if (p.dD) atomicAdd(p.dD + d0 + tid, s.accD[tid]);
+    if (p.ddelta_bias) atomicAdd(p.ddelta_bias + d0 + tid, s.accB[tid]);
+  }
+}
+
+template <typename InT, int G>
+cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
+  auto kern = scan_bwd_kernel<InT, G>;
+  const int smem = static_cast<int>(sizeof(BwdSmem<G>));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<static_cast<unsigned>(p.tiles), 32 * G, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename InT>
+cudaError_t dispatch(const BwdParams &p, cudaStream_t stream) {
+  switch (bwd_groups(p.dstate)) {
+    case 1: return launch_typed<InT, 1>(p, stream);
+    case 2: return launch_typed<InT, 2>(p, stream);
+    default: return launch_typed<InT, 4>(p, stream);
+  }
+}
+
+}  // namespace
+}  // namespace sss48
+
+namespace sss48 {
+
+int bwd_groups(int64_t dstate) {
+  const int g = static_cast<int>((dstate + 3) / 4);
+  return g <= 1 ? 1 : (g == 2 ? 2 : 4);
+}
+
+size_t scan_bwd_workspace_bytes(int64_t tiles, int64_t seqlen, int64_t dstate) {
+  const int64_t nblk = (seqlen + kBwdTimeBlock - 1) / kBwdTimeBlock;
+  return static_cast<size_t>(tiles) * static_cast<size_t>(nblk) *
+         static_cast<size_t>(4 * bwd_groups(dstate)) * kBwdChannels * sizeof(float);
+}
+
+cudaError_t launch_scan_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream) {
+  return in_bf16 ? dispatch<__nv_bfloat16>(p, stream) : dispatch<float>(p, stream);
+}
+
+}  // namespace sss48

@@ -1,0 +1,42 @@
+// scan_bwd.cuh -- launch interface of the backward selective-scan kernel.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace sss48 {
+
+constexpr int kBwdChannels = 32;   // channels per thread block
+constexpr int kBwdTimeBlock = 16;  // steps between state checkpoints
+
+struct BwdParams {
+  int64_t batch, dim, dstate, seqlen;
+  const void *u, *delta;
+  const float *A;
+  const void *B, *C;
+  const float *D;
+  const void *z;
+  const float *delta_bias;
+  int softplus;
+  const float *h0;
+  const float *dy;
+  const float *d_last;
+  float *du, *ddelta, *dA, *dB, *dC, *dD, *dz, *ddelta_bias, *dh0;
+  float *ckpt;      // workspace: one state per channel and 16-step block
+  int ch_tiles;     // ceil(dim / kBwdChannels)
+  int64_t tiles;    // batch * ch_tiles
+};
+
+// Warps per block (state groups of 4): 1, 2 or 4.
+int bwd_groups(int64_t dstate);
+
+// Workspace bytes of the state checkpoints.
+size_t scan_bwd_workspace_bytes(int64_t tiles, int64_t seqlen, int64_t dstate);
+
+// dA, dB, dC, dD and ddelta_bias are accumulated with atomics: the caller
+// zeroes them first.
+cudaError_t launch_scan_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream);
+
+}  // namespace sss48

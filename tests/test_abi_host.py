@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 3
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 4
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
@@ -63,15 +63,18 @@ def test_abi_version_and_status_strings(lib):
 
 
 def test_struct_layout_matches_c():
-    """Compile a C program that prints sizeof/offsetof of both structs."""
+    """Compile a C program that prints sizeof/offsetof of the structs."""
     fields_scan = [f[0] for f in sss.ScanArgs._fields_]
     fields_upd = [f[0] for f in sss.UpdateArgs._fields_]
+    fields_bwd = [f[0] for f in sss.ScanBwdArgs._fields_]
     src = ['#include <stdio.h>', '#include <stddef.h>', '#include "selective_scan.h"',
            'int main(void) {',
            'printf("%zu\\n", sizeof(mss_scan_args));']
     src += [f'printf("%zu\\n", offsetof(mss_scan_args, {f}));' for f in fields_scan]
     src += ['printf("%zu\\n", sizeof(mss_update_args));']
     src += [f'printf("%zu\\n", offsetof(mss_update_args, {f}));' for f in fields_upd]
+    src += ['printf("%zu\\n", sizeof(mss_scan_bwd_args));']
+    src += [f'printf("%zu\\n", offsetof(mss_scan_bwd_args, {f}));' for f in fields_bwd]
     src += ['return 0; }']
     with tempfile.TemporaryDirectory() as tmp:
         c = os.path.join(tmp, "layout.c")
@@ -82,6 +85,7 @@ def test_struct_layout_matches_c():
                                                check=True).stdout.split()]
     want = [ctypes.sizeof(sss.ScanArgs)] + [getattr(sss.ScanArgs, f).offset for f in fields_scan]
     want += [ctypes.sizeof(sss.UpdateArgs)] + [getattr(sss.UpdateArgs, f).offset for f in fields_upd]
+    want += [ctypes.sizeof(sss.ScanBwdArgs)] + [getattr(sss.ScanBwdArgs, f).offset for f in fields_bwd]
     assert vals == want
 
 
@@ -182,3 +186,46 @@ def test_null_args_rejected(lib):
     u = sss.UpdateArgs()
     u.batch, u.dim, u.dstate = 1, 1, 17
     assert lib.selective_state_update(ctypes.byref(u), None) == sss.MSS_ERR_UNSUPPORTED
+
+
+def _bwd_args(**kw):
+    a = sss.ScanBwdArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = 2, 40, 16, 1000
+    a.in_dtype = sss.MSS_BF16
+    fake = 0x10000
+    for f in ("u", "delta", "A", "B", "C", "dy", "du", "ddelta", "dA", "dB", "dC"):
+        setattr(a, f, fake)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_bwd_workspace_is_one_state_per_block():
+    lib = sss.load_library()
+    n = ctypes.c_size_t(0)
+    assert lib.mss_scan_bwd_workspace_size(ctypes.byref(_bwd_args()), ctypes.byref(n)) == sss.MSS_OK
+    # 2 batch rows x 2 channel tiles x 63 blocks x 16 states x 32 lanes x 4 B
+    assert n.value == 2 * 2 * 63 * 16 * 32 * 4
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(dstate=17), sss.MSS_ERR_UNSUPPORTED),
+    (dict(dy=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(dB=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(D=0x10000), sss.MSS_ERR_INVALID_ARG),        # D given without dD
+    (dict(dz=0x10000), sss.MSS_ERR_INVALID_ARG),       # dz without z
+    (dict(u=0x10001), sss.MSS_ERR_INVALID_ARG),        # misaligned bf16
+    (dict(dA=0x10002), sss.MSS_ERR_INVALID_ARG),       # misaligned fp32
+])
+def test_bwd_bad_arguments_are_rejected(kw, code):
+    lib = sss.load_library()
+    a = _bwd_args(**kw)
+    n = ctypes.c_size_t(0)
+    assert lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == code
+    assert lib.mamba_selective_scan_bwd(ctypes.byref(a), None) == code
+
+
+def test_bwd_missing_workspace_is_reported():
+    lib = sss.load_library()
+    assert lib.mamba_selective_scan_bwd(ctypes.byref(_bwd_args()), None) == sss.MSS_ERR_WORKSPACE
