@@ -73,6 +73,8 @@ def parse_args(argv=None):
     ap.add_argument("--varlen", type=int, default=0,
                     help="pack this many independent sequences into every row "
                          "(seeded random offsets; 0 = one sequence per row)")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="bwd times the backward scan (gradients of all inputs)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work of the oracle baseline sample")
@@ -295,6 +297,82 @@ def oracle_timing(inp, w, seconds: float, steps: int = 1, warmup: int = 0):
 # ------------------------------------------------------------- our arm
 
 
+def bwd_algorithmic_bytes(w) -> int:
+    """Every input of the backward pass read once (u, delta, z, B, C in the
+    input dtype, dy fp32) and every gradient written once in fp32."""
+    si = 2 if w.in_dtype == "bf16" else 4
+    bdl = w.batch * w.dim * w.seqlen
+    per_ch = 2 * si + (si + 4 if w.has_z else 0) + 4 + 2 * 4
+    bnl = w.batch * w.dstate * w.seqlen
+    return bdl * per_ch + bnl * 2 * (si + 4) + w.dim * w.dstate * 8
+
+
+def run_bwd(args, rank, world, local_rank):
+    import selective_state_space_48_b200 as sss
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.BY_NAME[args.workload]
+    inp = workloads.make_inputs(w, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(48000)
+    dy = torch.randn(w.batch, w.dim, w.seqlen, generator=g, device=dev)
+
+    def step():
+        sss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy,
+                               D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
+                               delta_softplus=w.softplus, workspace=ws)
+
+    # workspace sized once (the size depends on the shapes only)
+    nb = ctypes.c_size_t(0)
+    a = sss.ScanBwdArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = w.batch, w.dim, w.dstate, w.seqlen
+    a.in_dtype = sss.MSS_BF16 if w.in_dtype == "bf16" else sss.MSS_F32
+    for f in ("u", "delta", "A", "B", "C", "dy", "du", "ddelta", "dA", "dB", "dC"):
+        setattr(a, f, 256)  # only checked for presence and alignment here
+    if sss.load_library().mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(nb)):
+        raise RuntimeError("mss_scan_bwd_workspace_size failed")
+    ws = torch.empty(int(nb.value), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    stream = torch.cuda.current_stream(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(world)
+    max_ms = reduce_max(t0.elapsed_time(t1), world)
+    nbytes = bwd_algorithmic_bytes(w)
+    value = whole_job_gbs(nbytes, K, world, max_ms)
+    peak, src = measured_peaks()
+    line = {
+        "metric": "selective-scan backward HBM GB/s; B*D*L*N state updates/s",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": max_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(w), **{"pass": "bwd"}),
+        "state_updates_per_s": w.state_updates * K * world / (max_ms * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
+                     "unit": "GB/s", "frac": value / world / peak,
+                     "peak_source": src, "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes},
+        "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
+        "kernel_source_hash": kernel_source_hash(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, rank, world, local_rank):
     import selective_state_space_48_b200 as sss
     torch.cuda.set_device(local_rank)
@@ -500,9 +578,12 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
-        if rank == 0:
-            print(json.dumps(line), flush=True)
+        if args.pass_ == "bwd":
+            run_bwd(args, rank, world, local_rank)
+        else:
+            line = run_ours(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist
