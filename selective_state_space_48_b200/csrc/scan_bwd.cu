@@ -12,10 +12,11 @@
 //                  at the start of every block to the workspace (the only
 //                  state that touches HBM: 64 B per channel and block);
 //   reverse sweep  walks the blocks backwards; for each it reloads the inputs,
-//                  recomputes the block's 16 states from the checkpoint into
-//                  registers, then runs the adjoint
-//                  lam_t = ds_t C_t + a_{t+1} lam_{t+1} step by step
-//                  (re-evaluating each decay a_t).
+//                  recomputes the states of one half block (8 steps) from
+//                  the checkpoint into registers, runs the adjoint
+//                  lam_t = ds_t C_t + a_{t+1} lam_{t+1} backwards over them
+//                  (re-evaluating each decay a_t), then does the same for
+//                  the other half.
 //
 // With s_t = sum_n C_t[n] h_t[n] + D u_t, g_t = silu(z_t) and y_t = s_t g_t,
 // ds_t = dy_t g_t:
@@ -99,7 +100,7 @@ __device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
 }
 
 template <typename InT, int G>
-__global__ void __launch_bounds__(32 * G)
+__global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     scan_bwd_kernel(const BwdParams p) {
   using Sm = BwdSmem<G>;
   constexpr int NP = Sm::NP;
@@ -215,64 +216,74 @@ __global__ void __launch_bounds__(32 * G)
       hc[i] = ckpt[(static_cast<int64_t>(k) * NP + 4 * g + i) * CH + lane];
     __syncthreads();
 
-    // recompute the block's states from the checkpoint; this warp's share
-    // of the readout s_t
-    float hs[4][TB];
+    // Two halves of the block, the later one first.  For each: recompute
+    // the states of its 8 steps from the checkpoint into registers (with
+    // this warp's share of the readout s_t), then run the adjoint backwards
+    // over them.  Keeping 8 steps instead of 16 halves the registers the
+    // states need, for half a block of extra recomputation.
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float hh = hc[i];
+    for (int half = 1; half >= 0; --half) {
+      const int tb = 8 * half;  // first step of this half
+      float hs[4][8], hpre[4];  // states of steps tb..tb+7 and of step tb-1
 #pragma unroll
-      for (int t = 0; t < TB; ++t) {
-        hh = fmaf(ex2_mufu(s.dl[lane * ROW + t] * alpha[i]), hh,
-                  s.du[lane * ROW + t] * s.B[(4 * g + i) * TB + t]);
-        hs[i][t] = hh;
-      }
-    }
+      for (int i = 0; i < 4; ++i) {
+        float hh = hc[i];
 #pragma unroll
-    for (int t = 0; t < TB; ++t) {
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc = fmaf(s.C[(4 * g + i) * TB + t], hs[i][t], acc);
-      s.ps[(g * CH + lane) * ROW + t] = acc;
-    }
-
-    // adjoint, four steps at a time backwards
-#pragma unroll
-    for (int q = TB / 4 - 1; q >= 0; --q) {
-      float vB[16], vC[16];
-#pragma unroll
-      for (int tq = 3; tq >= 0; --tq) {
-        const int t = 4 * q + tq;
-        const float dl = s.dl[lane * ROW + t], uu = s.u[lane * ROW + t],
-                    ds = s.ds[lane * ROW + t];
-        float pdu = 0.f, pdd = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int n = 4 * g + i;
-          const float Bv = s.B[n * TB + t], Cv = s.C[n * TB + t];
-          const float hprev = t > 0 ? hs[i][t - 1] : hc[i];
-          const float a = ex2_mufu(dl * alpha[i]);
-          lam[i] = fmaf(ds, Cv, lam[i]);
-          vC[4 * i + tq] = ds * hs[i][t];
-          const float la = lam[i] * a * hprev;
-          pdd = fmaf(lam[i], Bv * uu, fmaf(la, an[i], pdd));
-          dA[i] = fmaf(la, dl, dA[i]);
-          vB[4 * i + tq] = lam[i] * dl * uu;
-          pdu = fmaf(lam[i] * dl, Bv, pdu);
-          lam[i] *= a;
+        for (int t = 0; t < tb + 8; ++t) {
+          if (t == tb) hpre[i] = hh;
+          hh = fmaf(ex2_mufu(s.dl[lane * ROW + t] * alpha[i]), hh,
+                    s.du[lane * ROW + t] * s.B[(4 * g + i) * TB + t]);
+          if (t >= tb) hs[i][t - tb] = hh;
         }
-        s.pu[(g * CH + lane) * ROW + t] = pdu;
-        s.pd[(g * CH + lane) * ROW + t] = pdd;
       }
-      // channel sums of dB, dC for states 4g + i, steps 4q + tq: the even
-      // lane of each pair adds j = lane >> 1 = 4 i + tq
-      const float rb = reduce_scatter16(vB, lane);
-      const float rc = reduce_scatter16(vC, lane);
-      const int j = lane >> 1, n = 4 * g + j / 4, t = 4 * q + j % 4;
-      if ((lane & 1) == 0 && n < p.dstate && t < nt) {
-        const int64_t off = (b * p.dstate + n) * L + t0 + t;
-        atomicAdd(p.dB + off, rb);
-        atomicAdd(p.dC + off, rc);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc = fmaf(s.C[(4 * g + i) * TB + tb + t], hs[i][t], acc);
+        s.ps[(g * CH + lane) * ROW + tb + t] = acc;
+      }
+
+      // adjoint, four steps at a time backwards
+#pragma unroll
+      for (int qq = 1; qq >= 0; --qq) {
+        const int q = 2 * half + qq;
+        float vB[16], vC[16];
+#pragma unroll
+        for (int tq = 3; tq >= 0; --tq) {
+          const int tl = 4 * qq + tq;  // step within the half
+          const int t = tb + tl;
+          const float dl = s.dl[lane * ROW + t], uu = s.u[lane * ROW + t],
+                      ds = s.ds[lane * ROW + t];
+          float pdu = 0.f, pdd = 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int n = 4 * g + i;
+            const float Bv = s.B[n * TB + t], Cv = s.C[n * TB + t];
+            const float hprev = tl > 0 ? hs[i][tl - 1] : hpre[i];
+            const float a = ex2_mufu(dl * alpha[i]);
+            lam[i] = fmaf(ds, Cv, lam[i]);
+            vC[4 * i + tq] = ds * hs[i][tl];
+            const float la = lam[i] * a * hprev;
+            pdd = fmaf(lam[i], Bv * uu, fmaf(la, an[i], pdd));
+            dA[i] = fmaf(la, dl, dA[i]);
+            vB[4 * i + tq] = lam[i] * dl * uu;
+            pdu = fmaf(lam[i] * dl, Bv, pdu);
+            lam[i] *= a;
+          }
+          s.pu[(g * CH + lane) * ROW + t] = pdu;
+          s.pd[(g * CH + lane) * ROW + t] = pdd;
+        }
+        // channel sums of dB, dC for states 4g + i, steps 4q + tq: the even
+        // lane of each pair adds j = lane >> 1 = 4 i + tq
+        const float rb = reduce_scatter16(vB, lane);
+        const float rc = reduce_scatter16(vC, lane);
+        const int j = lane >> 1, n = 4 * g + j / 4, t = 4 * q + j % 4;
+        if ((lane & 1) == 0 && n < p.dstate && t < nt) {
+          const int64_t off = (b * p.dstate + n) * L + t0 + t;
+          atomicAdd(p.dB + off, rb);
+          atomicAdd(p.dC + off, rc);
+        }
       }
     }
     __syncthreads();
