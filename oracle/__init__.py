@@ -62,7 +62,7 @@ def _bind(lib):
     lib.oracle_silu_f64.restype = ctypes.c_double
     lib.oracle_selective_scan_f64.argtypes = (
         [_I64] * 4 + [_D] * 8 + [ctypes.c_int, _D, _D, _D,
-                                 ctypes.POINTER(ctypes.c_int32), _I64])
+                                 ctypes.POINTER(ctypes.c_int32), _I64, ctypes.c_int])
     lib.oracle_selective_scan_f64.restype = ctypes.c_int
     lib.oracle_selective_state_update_f64.argtypes = (
         [_I64] * 3 + [_D] * 9 + [ctypes.c_int, _D])
@@ -120,7 +120,7 @@ def silu(z, lib=None):
 
 def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                    delta_softplus=True, h0=None, return_last_state=False,
-                   lib=None, cu_seqlens=None):
+                   lib=None, cu_seqlens=None, trapezoid=False):
     """Sequential fp64 selective scan.
 
     u, delta, z: (batch, dim, L); B, C: (batch, N, L); A: (dim, N);
@@ -128,6 +128,7 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     float64, and the final state when ``return_last_state``.  cu_seqlens
     (num_seqs + 1 offsets, 0 ... L) packs independent sequences into every
     row: the state restarts from zero at each interior offset.
+    ``trapezoid`` selects the three-term trapezoidal update.
     """
     lib = lib or load()
     u = _f64(u)
@@ -154,7 +155,7 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     rc = lib.oracle_selective_scan_f64(
         batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
         _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)),
-        _ptr(h0), _ptr(y), _ptr(last), cu, nseq)
+        _ptr(h0), _ptr(y), _ptr(last), cu, nseq, int(bool(trapezoid)))
     if rc != 0:
         raise ValueError("oracle_selective_scan_f64 rejected the sizes")
     return (y, last) if return_last_state else y

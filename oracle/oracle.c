@@ -18,6 +18,12 @@
  *           discretisation, i.e. Abar = exp(Delta A), Bbar = Delta B.
  *  [select] "State Space Models and the Post-Transformer Era", section
  *           "The Selection Mechanism": Delta, B and C are per-token inputs.
+ *  [trap]   "The State That Must Remember Everything", Part 7: Mamba-3
+ *           replaces the Euler step by a trapezoidal one with three terms,
+ *           h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1} + gamma_t B_t x_t
+ *           (alpha, beta, gamma not given there; read as the trapezoidal
+ *           rule for the same ODE: alpha = exp(Delta A), beta = alpha
+ *           Delta / 2, gamma = Delta / 2, no previous input at t = 0).
  *  The step-size nonlinearity Delta = softplus(delta + delta_bias) and the
  *  output gate y * silu(z) are not written out on the pages; this library
  *  uses the standard Mamba parameterisation for both.
@@ -70,7 +76,7 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
                               const double *delta_bias, int delta_softplus,
                               const double *h0, double *y,
                               double *last_state, const int32_t *cu_seqlens,
-                              int64_t num_seqs) {
+                              int64_t num_seqs, int trapezoid) {
   /* the per-channel state lives on the stack; 256 states is far above any
    * size the tests or the bench use */
   if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256 || seqlen < 0)
@@ -87,6 +93,9 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
     const int64_t b = ch / dim;
     const int64_t d = ch % dim;
     double hp[256];
+    /* trapezoidal rule: B_{t-1}[n] u_{t-1}, 0 before the first step */
+    double wprev[256];
+    for (int64_t n = 0; n < dstate; ++n) wprev[n] = 0.0;
     /* h_{-1} = h0, or 0 ([eq]: the state starts empty). */
     for (int64_t n = 0; n < dstate; ++n)
       hp[n] = h0 ? h0[(b * dim + d) * dstate + n] : 0.0;
@@ -107,7 +116,7 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
       if (cu_seqlens) {
         while (next < num_seqs && cu_seqlens[next] < t) ++next;
         if (next < num_seqs && cu_seqlens[next] == t)
-          for (int64_t n = 0; n < dstate; ++n) hp[n] = 0.0;
+          for (int64_t n = 0; n < dstate; ++n) hp[n] = wprev[n] = 0.0;
       }
       const double dt = step_size(drow[t], bias, delta_softplus);
       const double ut = urow[t];
@@ -115,6 +124,15 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
       for (int64_t n = 0; n < dstate; ++n) {
         /* [euler]: Abar = exp(Delta A[d,n]), Bbar u = Delta B_t[n] u_t. */
         const double abar = exp(dt * A[d * dstate + n]);
+        if (trapezoid) {
+          /* [trap]: three terms, the previous input decayed over the step
+           * and the current one, weighted by half a step each. */
+          const double w = Bb[n * seqlen + t] * ut;
+          hp[n] = abar * hp[n] + 0.5 * dt * (abar * wprev[n] + w);
+          wprev[n] = w;
+          acc += Cb[n * seqlen + t] * hp[n];
+          continue;
+        }
         const double bbar_u = dt * Bb[n * seqlen + t] * ut;
         /* [eq]: h_t = Abar h_{t-1} + Bbar u_t. */
         hp[n] = abar * hp[n] + bbar_u;

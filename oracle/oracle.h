@@ -47,7 +47,11 @@ double oracle_silu_f64(double z);
  * (num_seqs + 1 increasing offsets, 0 ... seqlen, the same for every batch
  * row), h is set to 0 before every step t = cu_seqlens[i], 0 < i < num_seqs,
  * so each row holds num_seqs independent scans; h0 seeds the first and
- * last_state is the end of the last.  Returns 0, or -1 on a bad size. */
+ * last_state is the end of the last.  With trapezoid != 0 the update is the
+ * three-term trapezoidal form
+ *   h_t = a h_{t-1} + Delta_t / 2 * (a B_{t-1}[n] u_{t-1} + B_t[n] u_t),
+ *   a = exp(Delta_t A[d,n]), no previous term at t = 0 or at a restart.
+ * Returns 0, or -1 on a bad size. */
 int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
                               int64_t seqlen, const double *u,
                               const double *delta, const double *A,
@@ -56,7 +60,7 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate,
                               const double *delta_bias, int delta_softplus,
                               const double *h0, double *y,
                               double *last_state, const int32_t *cu_seqlens,
-                              int64_t num_seqs);
+                              int64_t num_seqs, int trapezoid);
 
 /* One decode step (the same recurrence for a single t), state updated in
  * place.  x, dt, z, y: (batch, dim); B, C: (batch, dstate);

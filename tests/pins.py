@@ -493,6 +493,58 @@ def pin_backward_finite_differences(lib):
     _fd_check(lib, dict(shape=(1, 2, 3, 13), softplus=False), 32)
 
 
+# --------------------------------------------------------------------------
+# "The State That Must Remember Everything", Part 7 (Mamba-3): the update
+# gains a third term, the previous input.  Read as the trapezoidal rule for
+# dh/dt = A h + B x: two facts pin it without re-using the recurrence.
+#  * With A = 0 the state is the trapezoidal sum of B x: a cumulative sum.
+#  * Against the exact solution of dh/dt = A h + sin(t), h(0) = 0, the
+#    error at a fixed time falls 4x when the step halves (second order),
+#    where the Euler update only halves it.
+
+
+def pin_trapezoid_no_decay(lib):
+    rng = _rng(41)
+    bt, dm, N, L = 1, 2, 3, 17
+    u = rng.normal(size=(bt, dm, L))
+    delta = rng.uniform(0.05, 0.5, size=(bt, dm, L))
+    A = np.zeros((dm, N))
+    B = rng.normal(size=(bt, N, L))
+    C = rng.normal(size=(bt, N, L))
+    D = rng.normal(size=dm)
+    h0 = rng.normal(size=(bt, dm, N))
+    got, last = oracle.selective_scan(u, delta, A, B, C, D=D, delta_softplus=False,
+                                      h0=h0, return_last_state=True, lib=lib,
+                                      trapezoid=True)
+    for d in range(dm):
+        w = B[0] * u[0, d][None, :]                           # (N, L)
+        wprev = np.concatenate([np.zeros((N, 1)), w[:, :-1]], axis=1)
+        h = h0[0, d][:, None] + np.cumsum(0.5 * delta[0, d][None, :] * (wprev + w), axis=1)
+        want = np.sum(C[0] * h, axis=0) + D[d] * u[0, d]
+        _close(got[0, d], want, 1e-12, 1e-12, "trapezoid without decay")
+        _close(last[0, d], h[:, -1], 1e-12, 1e-12, "trapezoid last state")
+
+
+def _ode_error(lib, dt, trapezoid, a=-0.7, T=5.0):
+    L = int(round(T / dt)) + 1
+    t = np.arange(L) * dt
+    u = np.sin(t)[None, None, :]
+    delta = np.full((1, 1, L), dt)
+    y = oracle.selective_scan(u, delta, np.array([[a]]), np.ones((1, 1, L)),
+                              np.ones((1, 1, L)), delta_softplus=False, lib=lib,
+                              trapezoid=trapezoid)
+    exact = (-a * np.sin(T) - np.cos(T) + np.exp(a * T)) / (a * a + 1.0)
+    return abs(y[0, 0, -1] - exact)
+
+
+def pin_trapezoid_second_order(lib):
+    e1, e2 = _ode_error(lib, 0.02, True), _ode_error(lib, 0.01, True)
+    assert 3.6 < e1 / e2 < 4.4, ("trapezoid order", e1, e2)
+    f1, f2 = _ode_error(lib, 0.02, False), _ode_error(lib, 0.01, False)
+    assert 1.7 < f1 / f2 < 2.3, ("Euler order", f1, f2)
+    assert e2 < f2 / 10, ("trapezoid not more accurate than Euler", e2, f2)
+
+
 ALL_PINS = [
     pin_combine_worked_example,
     pin_scan_worked_example,
@@ -508,4 +560,6 @@ ALL_PINS = [
     pin_resume,
     pin_packed_sequences,
     pin_backward_finite_differences,
+    pin_trapezoid_no_decay,
+    pin_trapezoid_second_order,
 ]

@@ -19,8 +19,8 @@ MUTATIONS = {
     "combine_transposed": ("*b_out = a2 * b1 + b2;", "*b_out = a1 * b2 + b1;"),
     "fade_applied_to_input": ("hp[n] = abar * hp[n] + bbar_u;",
                               "hp[n] = hp[n] + abar * bbar_u;"),
-    "readout_uses_B": ("acc += Cb[n * seqlen + t] * hp[n];",
-                       "acc += Bb[n * seqlen + t] * hp[n];"),
+    "readout_uses_B": ("after the update. */\n        acc += Cb[n * seqlen + t] * hp[n];",
+                       "after the update. */\n        acc += Bb[n * seqlen + t] * hp[n];"),
     "skip_dropped": ("double yt = acc + dskip * ut;", "double yt = acc;"),
     "decay_sign": ("exp(dt * A[d * dstate + n])", "exp(-dt * A[d * dstate + n])"),
     "B_index_transposed": ("dt * Bb[n * seqlen + t] * ut",
@@ -38,7 +38,7 @@ MUTATIONS = {
     "readout_before_update": (
         "        hp[n] = abar * hp[n] + bbar_u;\n        /* [eq]: y_t = C_t h_t, with the state after the update. */\n        acc += Cb[n * seqlen + t] * hp[n];",
         "        acc += Cb[n * seqlen + t] * hp[n];\n        hp[n] = abar * hp[n] + bbar_u;"),
-    "reset_dropped": ("          for (int64_t n = 0; n < dstate; ++n) hp[n] = 0.0;",
+    "reset_dropped": ("          for (int64_t n = 0; n < dstate; ++n) hp[n] = wprev[n] = 0.0;",
                       "          ;"),
     "reset_one_step_late": ("cu_seqlens[next] == t)", "cu_seqlens[next] == t - 1)"),
     "bwd_adjoint_not_decayed": ("          lam[n] *= a;\n", "\n"),
@@ -48,6 +48,9 @@ MUTATIONS = {
                                    "dCb[n * L + t] += ds * H[t * N + n];"),
     "bwd_gate_derivative_wrong": ("return sg * (1.0 + z * (1.0 - sg));", "return sg;"),
     "bwd_softplus_derivative_dropped": ("? dDelta / (1.0 + exp(-x)) : dDelta;", "? dDelta : dDelta;"),
+    "trap_previous_input_not_decayed": ("0.5 * dt * (abar * wprev[n] + w)", "0.5 * dt * (wprev[n] + w)"),
+    "trap_full_step_weights": ("0.5 * dt * (abar * wprev[n] + w)", "dt * (abar * wprev[n] + w)"),
+    "trap_previous_input_not_kept": ("          wprev[n] = w;\n", "\n"),
     "update_step_uses_input_twice": (
         "step * B[b * dstate + n] * x[ch];", "step * B[b * dstate + n] * x[ch] * x[ch];"),
 }
