@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 4
+#define MSS_ABI_VERSION 5
 
 typedef enum {
   MSS_OK = 0,
@@ -144,6 +144,14 @@ typedef struct mss_scan_args {
      bounds. */
   const int32_t *cu_seqlens;
   int64_t num_seqs;     /* 0 when cu_seqlens is NULL */
+  /* 1: the three-term trapezoidal update of Mamba-3 ("The State That Must
+     Remember Everything", Part 7: h_t = alpha_t h_{t-1} + beta_t B_{t-1}
+     x_{t-1} + gamma_t B_t x_t), read as the trapezoidal rule for the same
+     ODE: h_t = a_t h_{t-1} + Delta_t / 2 (a_t B_{t-1} u_{t-1} + B_t u_t),
+     a_t = exp(Delta_t A), no previous input before step 0; a chunk of a
+     split sequence reads the step before it from u and B.  0: the Euler
+     update above.  Not combined with cu_seqlens (MSS_ERR_UNSUPPORTED). */
+  int trapezoid;
 } mss_scan_args;
 
 /* Bytes of device workspace the scan needs for these arguments (0 when the

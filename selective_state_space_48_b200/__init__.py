@@ -24,7 +24,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 4  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 5  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -85,6 +85,7 @@ class ScanArgs(ctypes.Structure):
         ("stride_y", ctypes.c_int64 * 2),
         ("cu_seqlens", ctypes.c_void_p),
         ("num_seqs", ctypes.c_int64),
+        ("trapezoid", ctypes.c_int),
     ]
 
 
@@ -218,7 +219,7 @@ def _stream_handle(stream):
 def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                    delta_softplus=True, h0=None, y=None, last_state=None,
                    workspace=None, plan_splits=0, test_flags=0,
-                   spin_timeout_ns=0, cu_seqlens=None) -> ScanArgs:
+                   spin_timeout_ns=0, cu_seqlens=None, trapezoid=False) -> ScanArgs:
     batch, dim, L = u.shape
     N = A.shape[1]
     ind = u.dtype
@@ -249,6 +250,7 @@ def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     a.plan_chunk_steps = 0
     a.test_flags = int(test_flags)
     a.spin_timeout_ns = int(spin_timeout_ns)
+    a.trapezoid = 1 if trapezoid else 0
     if cu_seqlens is not None:
         _check_cuda("cu_seqlens", cu_seqlens, torch.int32)
         if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
@@ -282,7 +284,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                        out_dtype=torch.float32, y=None, last_state=None,
                        workspace=None, stream=None, plan_splits=0,
                        test_flags=0, spin_timeout_ns=0, check_status=False,
-                       cu_seqlens=None):
+                       cu_seqlens=None, trapezoid=False):
     """Forward selective scan through ``mamba_selective_scan_fwd``.
 
     u, delta, z: (batch, dim, L); B, C: (batch, N, L) (float32 or bfloat16,
@@ -290,8 +292,9 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     (batch, dim, N) float32.  u, delta, z, B, C and y may be views whose
     last dimension is contiguous.  ``cu_seqlens`` (int32 CUDA tensor of
     num_seqs + 1 offsets, 0 ... L) packs independent sequences into every
-    row.  Returns y (batch, dim, L) in ``out_dtype`` (and the final state
-    when ``return_last_state``).
+    row.  ``trapezoid`` selects the three-term trapezoidal update.  Returns
+    y (batch, dim, L) in ``out_dtype`` (and the final state when
+    ``return_last_state``).
     """
     batch, dim, L = u.shape
     N = A.shape[1]
@@ -302,7 +305,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                                  device=u.device)
     args = make_scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus,
                           h0, y, last_state, None, plan_splits, test_flags,
-                          spin_timeout_ns, cu_seqlens)
+                          spin_timeout_ns, cu_seqlens, trapezoid)
     if workspace is None:
         workspace = alloc_workspace(scan_workspace_size(args), u.device)
     if workspace is not None:

@@ -118,6 +118,8 @@ mss_status check_scan_args(const mss_scan_args *a) {
                        !aligned(a->cu_seqlens, 4))
                     : a->num_seqs != 0)
     return MSS_ERR_INVALID_ARG;
+  if (a->trapezoid != 0 && a->trapezoid != 1) return MSS_ERR_INVALID_ARG;
+  if (a->trapezoid && a->cu_seqlens) return MSS_ERR_UNSUPPORTED;
   const size_t ei = esize(a->in_dtype), eo = esize(a->out_dtype);
   if (!aligned(a->u, ei) || !aligned(a->delta, ei) || !aligned(a->B, ei) ||
       !aligned(a->C, ei) || (a->z && !aligned(a->z, ei)) ||
@@ -187,6 +189,7 @@ void fill_scan_params(const mss_scan_args *a, const Plan &pl, ScanParams *p) {
   resolve_scan_strides(a, p);  // checked in check_scan_args
   p->cu = a->cu_seqlens;
   p->nseq = a->cu_seqlens ? a->num_seqs : 0;
+  p->trap = a->trapezoid;
   p->chunk = pl.chunk;
   p->splits = pl.splits;
   p->ch_tiles = pl.ch_tiles;

@@ -72,7 +72,14 @@ constexpr uint64_t kTmaWaitNs = 2000000000ull;
 
 constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 
-template <typename InT, int G>
+// Kernel variants: ordinary scans, packed sequences (restarts), and the
+// three-term trapezoidal update.  Each is its own instantiation so the
+// code of one never reaches the others.
+constexpr int kModePlain = 0;
+constexpr int kModeVarlen = 1;
+constexpr int kModeTrap = 2;
+
+template <typename InT, int G, bool TRAP = false>
 struct Layout {
   static constexpr int NP = 4 * G;
   static constexpr int tileU = align128(CH * TB * static_cast<int>(sizeof(InT)));
@@ -85,7 +92,9 @@ struct Layout {
   static constexpr int oDu = CH * ROW * 4;
   static constexpr int oB = 2 * CH * ROW * 4;
   static constexpr int oC = oB + NP * TB * 4;
-  static constexpr int set = oC + NP * TB * 4;
+  // trapezoidal update only: Delta_t u_{t-1} / 2 [CH][ROW]
+  static constexpr int oQ = oC + NP * TB * 4;
+  static constexpr int set = oQ + (TRAP ? CH * ROW * 4 : 0);
   // two sets of state-group shares of y: [G][CH][ROW]
   static constexpr int part0 = set0 + 2 * set;
   static constexpr int part = G * CH * ROW * 4;
@@ -101,9 +110,11 @@ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) {
   return a < b ? a : b;
 }
 
-template <typename InT, typename OutT, int G, bool TMA, bool VARLEN>
+template <typename InT, typename OutT, int G, bool TMA, int MODE>
 struct Scan {
-  using Lay = Layout<InT, G>;
+  static constexpr bool VARLEN = MODE == kModeVarlen;
+  static constexpr bool TRAP = MODE == kModeTrap;
+  using Lay = Layout<InT, G, TRAP>;
   static constexpr int NP = 4 * G;
 
   const ScanParams &p;
@@ -382,8 +393,10 @@ struct Scan {
     return sl;
   }
 
+  // uprev0[k]: u of the step before the block for slot k (trapezoidal
+  // update, slots starting the block only).
   __device__ void prep_slots(int stage, int set, int nt, const Slots &sl, int ti,
-                             uint32_t restarts) const {
+                             uint32_t restarts, const float (&uprev0)[kSlots]) const {
     const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
     float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
 #pragma unroll
@@ -404,8 +417,17 @@ struct Scan {
         if (t + 2 >= nt) dl.z = 0.f;
         if (t + 3 >= nt) dl.w = 0.f;
       }
-      *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
-          make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
+      if (TRAP) {
+        // half-step weights: Delta_t u_t / 2 and Delta_t u_{t-1} / 2
+        const float up = t > 0 ? to_f32<InT>(ru[c * TB + t - 1]) : uprev0[k];
+        *reinterpret_cast<float4 *>(sDu + c * ROW + t) = make_float4(
+            0.5f * dl.x * u.x, 0.5f * dl.y * u.y, 0.5f * dl.z * u.z, 0.5f * dl.w * u.w);
+        *reinterpret_cast<float4 *>(fset(set, Lay::oQ) + c * ROW + t) = make_float4(
+            0.5f * dl.x * up, 0.5f * dl.y * u.x, 0.5f * dl.z * u.y, 0.5f * dl.w * u.z);
+      } else {
+        *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
+            make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
+      }
       if (restarts) mark_restarts(dl, restarts);
       *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
     }
@@ -465,8 +487,12 @@ struct Scan {
   // y_t = sum_n C_t[n] h_t[n] written to part set `set`.  Exponents and
   // inputs of steps (t, t+1) go through one paired f32x2 instruction, as do
   // the shares of y.
+  // Trapezoidal update: the input term of step t gains the previous input,
+  // decayed over the step, e_t (Delta_t u_{t-1} / 2) B_{t-1}[n]; bprev holds
+  // B_{t-1}[n] of this lane's states across quads and blocks.
   __device__ void scan(int set, int g, int lane, float (&h)[4],
-                       const float2 (&al2)[4], float &dsum, bool split) const {
+                       const float2 (&al2)[4], float &dsum, bool split,
+                       float (&bprev)[4]) const {
     const float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
     const float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
     float *sPart = fpart(set);
@@ -476,6 +502,8 @@ struct Scan {
       const float4 du = *reinterpret_cast<const float4 *>(&sDu[lane * ROW + 4 * q]);
       const float2 dl01 = make_float2(dl.x, dl.y), dl23 = make_float2(dl.z, dl.w);
       const float2 du01 = make_float2(du.x, du.y), du23 = make_float2(du.z, du.w);
+      float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (TRAP) qv = *reinterpret_cast<const float4 *>(&fset(set, Lay::oQ)[lane * ROW + 4 * q]);
       float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -484,8 +512,8 @@ struct Scan {
         const float4 cq = *reinterpret_cast<const float4 *>(&sC[n * TB + 4 * q]);
         const float2 x01 = __fmul2_rn(dl01, al2[i]);
         const float2 x23 = __fmul2_rn(dl23, al2[i]);
-        const float2 b01 = __fmul2_rn(du01, make_float2(bq.x, bq.y));
-        const float2 b23 = __fmul2_rn(du23, make_float2(bq.z, bq.w));
+        float2 b01 = __fmul2_rn(du01, make_float2(bq.x, bq.y));
+        float2 b23 = __fmul2_rn(du23, make_float2(bq.z, bq.w));
         // the last kPolyStates states of the group take their decays from
         // the FMA-pipe polynomial, the others from the special-function unit
         float2 e01, e23;
@@ -495,6 +523,13 @@ struct Scan {
         } else {
           e01 = make_float2(ex2_mufu(x01.x), ex2_mufu(x01.y));
           e23 = make_float2(ex2_mufu(x23.x), ex2_mufu(x23.y));
+        }
+        if (TRAP) {
+          const float2 q01 = __fmul2_rn(make_float2(qv.x, qv.y), make_float2(bprev[i], bq.x));
+          const float2 q23 = __fmul2_rn(make_float2(qv.z, qv.w), make_float2(bq.y, bq.z));
+          b01 = __ffma2_rn(e01, q01, b01);
+          b23 = __ffma2_rn(e23, q23, b23);
+          bprev[i] = bq.w;
         }
         float2 h01, h23;
         h01.x = fmaf(e01.x, h[i], b01.x);
@@ -568,10 +603,12 @@ constexpr int kPartFree = 3;    // epi -> scan: y shares of a block consumed
 constexpr int kBarEpi = 1;      // named barrier of the epilogue warps only
 constexpr uint64_t kHandoffWaitNs = 2000000000ull;
 
-template <typename InT, typename OutT, int G, bool TMA, bool VARLEN>
+template <typename InT, typename OutT, int G, bool TMA, int MODE>
 __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     scan_fwd_kernel(const ScanParams p, const __grid_constant__ TmaMaps maps) {
-  using S = Scan<InT, OutT, G, TMA, VARLEN>;
+  using S = Scan<InT, OutT, G, TMA, MODE>;
+  constexpr bool VARLEN = S::VARLEN;
+  constexpr bool TRAP = S::TRAP;
   using Lay = typename S::Lay;
   constexpr int NP = 4 * G;
   constexpr int NSCAN = 32 * G;
@@ -635,6 +672,16 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     if (VARLEN && alpha[i] == 0.f) alpha[i] = -1e-30f;
     h[i] = (live[i] && k == 0 && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
   }
+  // trapezoidal update: B_{t-1}[n] of the step before this chunk (none
+  // before the sequence starts)
+  float bprev[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    bprev[i] = 0.f;
+    if (TRAP && live[i] && sc.t_begin > 0)
+      bprev[i] = to_f32<InT>(static_cast<const InT *>(p.B)[b * p.sB[0] + (4 * g + i) * p.sB[1] +
+                                                          sc.t_begin - 1]);
+  }
   float dsum = 0.f;
   float2 al2[4];
 #pragma unroll
@@ -660,7 +707,7 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
       const int s = i & 1;
       wait_hand(kTilesReady, s);
       if (i >= 2) wait_hand(kPartFree, s);
-      sc.scan(s, g, lane, h, al2, dsum, split);
+      sc.scan(s, g, lane, h, al2, dsum, split, bprev);
       if (i + 2 < nblk) mbar_arrive(sc.hand(kTilesFree, s));
       mbar_arrive(sc.hand(kPartReady, s));
     }
@@ -671,8 +718,20 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     for (int blk = 0; blk < nblk; ++blk) {
       if (blk >= 2) wait_hand(kTilesFree, blk & 1);
       const uint32_t rs = VARLEN ? sc.restarts4(sc.t0_of(blk) + sl.t, nb) : 0u;
+      // trapezoidal update: u of the step before the block, for the slots
+      // that start it (read from HBM/L2: the previous raw stage may already
+      // be refilled)
+      float up0[S::kSlots];
+#pragma unroll
+      for (int k = 0; k < S::kSlots; ++k) {
+        up0[k] = 0.f;
+        const int64_t tp0 = sc.t0_of(blk) - 1;
+        if (TRAP && sl.t == 0 && sl.ok[k] && tp0 >= 0)
+          up0[k] = to_f32<InT>(static_cast<const InT *>(p.u)[b * p.su[0] +
+                                                             (d0 + sl.c[k]) * p.su[1] + tp0]);
+      }
       ok &= sc.wait_raw(blk, 0, phase);
-      sc.prep_slots(blk % STAGES, blk & 1, sc.nt_of(blk), sl, tp, rs);
+      sc.prep_slots(blk % STAGES, blk & 1, sc.nt_of(blk), sl, tp, rs, up0);
       mbar_arrive(sc.hand(kTilesReady, blk & 1));
     }
     // the prep warps waited on every raw block: their phases seed the
@@ -896,10 +955,10 @@ bool build_maps(const ScanParams &p, int in_bf16, int groups, TmaMaps *m) {
   return true;
 }
 
-template <typename InT, typename OutT, int G, bool TMA, bool VARLEN>
+template <typename InT, typename OutT, int G, bool TMA, int MODE>
 cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t s) {
-  auto kern = scan_fwd_kernel<InT, OutT, G, TMA, VARLEN>;
-  const int smem = Layout<InT, G>::bytes;
+  auto kern = scan_fwd_kernel<InT, OutT, G, TMA, MODE>;
+  const int smem = Layout<InT, G, MODE == kModeTrap>::bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.tiles * p.splits;
@@ -907,35 +966,36 @@ cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t 
   return cudaGetLastError();
 }
 
-// Packed sequences get their own instantiations, so the code that finds and
-// applies restarts never touches the kernels of ordinary scans.
-template <typename InT, typename OutT, bool VARLEN>
+// Packed sequences and the trapezoidal update get their own instantiations,
+// so their code never touches the kernels of ordinary scans.
+template <typename InT, typename OutT, int MODE>
 cudaError_t dispatch_v(const ScanParams &p, bool tma, const TmaMaps &maps, cudaStream_t s) {
   const int G = static_cast<int>((p.dstate + 3) / 4);
   if (tma) {
     switch (G) {
-      case 1: return launch_typed<InT, OutT, 1, true, VARLEN>(p, maps, s);
-      case 2: return launch_typed<InT, OutT, 2, true, VARLEN>(p, maps, s);
-      default: return launch_typed<InT, OutT, 4, true, VARLEN>(p, maps, s);
+      case 1: return launch_typed<InT, OutT, 1, true, MODE>(p, maps, s);
+      case 2: return launch_typed<InT, OutT, 2, true, MODE>(p, maps, s);
+      default: return launch_typed<InT, OutT, 4, true, MODE>(p, maps, s);
     }
   }
   switch (G) {
-    case 1: return launch_typed<InT, OutT, 1, false, VARLEN>(p, maps, s);
-    case 2: return launch_typed<InT, OutT, 2, false, VARLEN>(p, maps, s);
-    default: return launch_typed<InT, OutT, 4, false, VARLEN>(p, maps, s);
+    case 1: return launch_typed<InT, OutT, 1, false, MODE>(p, maps, s);
+    case 2: return launch_typed<InT, OutT, 2, false, MODE>(p, maps, s);
+    default: return launch_typed<InT, OutT, 4, false, MODE>(p, maps, s);
   }
 }
 
 template <typename InT, typename OutT>
 cudaError_t dispatch(const ScanParams &p, bool tma, const TmaMaps &maps, cudaStream_t s) {
-  return p.cu ? dispatch_v<InT, OutT, true>(p, tma, maps, s)
-              : dispatch_v<InT, OutT, false>(p, tma, maps, s);
+  if (p.cu) return dispatch_v<InT, OutT, kModeVarlen>(p, tma, maps, s);
+  if (p.trap) return dispatch_v<InT, OutT, kModeTrap>(p, tma, maps, s);
+  return dispatch_v<InT, OutT, kModePlain>(p, tma, maps, s);
 }
 
 template <typename InT, typename OutT, int G>
 int occupancy_typed() {
   int n = 0;
-  auto kern = scan_fwd_kernel<InT, OutT, G, true, false>;
+  auto kern = scan_fwd_kernel<InT, OutT, G, true, kModePlain>;
   const int smem = Layout<InT, G>::bytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)

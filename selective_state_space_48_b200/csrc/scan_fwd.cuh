@@ -37,6 +37,8 @@ struct ScanParams {
   // cu[1 .. nseq-1] restart the state
   const int32_t *cu;
   int64_t nseq;
+  // three-term trapezoidal update (1) instead of the Euler one (0)
+  int trap;
   int y_vec;       // rows of y allow 4-element vector stores (set at launch)
   // launch plan
   int64_t chunk;   // timesteps per sequence chunk (multiple of kTimeBlock)

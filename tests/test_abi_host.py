@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 4
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 5
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
@@ -147,6 +147,8 @@ def test_workspace_size_follows_plan(lib):
     (dict(num_seqs=3), sss.MSS_ERR_INVALID_ARG),                  # offsets missing
     (dict(cu_seqlens=0x10000, num_seqs=0), sss.MSS_ERR_INVALID_ARG),
     (dict(cu_seqlens=0x10002, num_seqs=2), sss.MSS_ERR_INVALID_ARG),  # misaligned
+    (dict(trapezoid=2), sss.MSS_ERR_INVALID_ARG),
+    (dict(trapezoid=1, cu_seqlens=0x10000, num_seqs=2), sss.MSS_ERR_UNSUPPORTED),
 ])
 def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     a = _args(**kw)
@@ -164,6 +166,7 @@ def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     dict(stride_y=(41 * 4100, 4100)),          # y inside a larger buffer
     dict(stride_delta=(0, 0)),                 # packed
     dict(cu_seqlens=0x10000, num_seqs=5),      # packed sequences
+    dict(trapezoid=1),                         # three-term update
 ])
 def test_valid_strides_are_accepted(lib, kw):
     rc, n = _ws(lib, _args(plan_splits=1, **kw))
