@@ -73,6 +73,8 @@ def parse_args(argv=None):
     ap.add_argument("--varlen", type=int, default=0,
                     help="pack this many independent sequences into every row "
                          "(seeded random offsets; 0 = one sequence per row)")
+    ap.add_argument("--trapezoid", action="store_true",
+                    help="three-term trapezoidal update instead of the Euler one")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="bwd times the backward scan (gradients of all inputs)")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -388,7 +390,8 @@ def run_ours(args, rank, world, local_rank):
     sargs = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"],
                                inp["C"], D=inp["D"], z=inp["z"],
                                delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, y=y, cu_seqlens=cu_t)
+                               delta_softplus=w.softplus, y=y, cu_seqlens=cu_t,
+                               trapezoid=args.trapezoid)
     ws_bytes = sss.scan_workspace_size(sargs)
     ws = sss.alloc_workspace(ws_bytes, dev)
     if ws is not None:
@@ -458,7 +461,7 @@ def run_ours(args, rank, world, local_rank):
                                inp["C"], D=inp["D"], z=inp["z"],
                                delta_bias=inp["delta_bias"],
                                delta_softplus=w.softplus, y=y, workspace=ws,
-                               cu_seqlens=cu_t)
+                               cu_seqlens=cu_t, trapezoid=args.trapezoid)
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -495,7 +498,8 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "f32",
         "data": "synthetic",
         "config": dict(workload_config(w, args.out_dtype),
-                       **({"sequences_per_row": args.varlen} if args.varlen else {})),
+                       **({"sequences_per_row": args.varlen} if args.varlen else {}),
+                       **({"update": "trapezoidal"} if args.trapezoid else {})),
         "state_updates_per_s": updates,
         "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": value / world / peak,
