@@ -69,6 +69,14 @@ template <> __device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bf
   return __bfloat162float(p[i]);
 }
 
+// Component j (a compile-time constant after unrolling) of a float4.
+__device__ __forceinline__ float comp(const float4 &v, int j) {
+  return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ float4 ld4(const float *p) {
+  return *reinterpret_cast<const float4 *>(p);
+}
+
 __device__ __forceinline__ float sigmoid_f(float x) {
   return __fdividef(1.0f, 1.0f + ex2_mufu(-x * kLog2e));
 }
@@ -189,11 +197,15 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     load_block(k, false);
     __syncthreads();
 #pragma unroll
-    for (int t = 0; t < TB; ++t) {
-      const float dl = s.dl[lane * ROW + t], du = s.du[lane * ROW + t];
+    for (int q = 0; q < TB / 4; ++q) {
+      const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * q]), du4 = ld4(&s.du[lane * ROW + 4 * q]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        h[i] = fmaf(ex2_mufu(dl * alpha[i]), h[i], du * s.B[(4 * g + i) * TB + t]);
+      for (int i = 0; i < 4; ++i) {
+        const float4 b4 = ld4(&s.B[(4 * g + i) * TB + 4 * q]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          h[i] = fmaf(ex2_mufu(comp(dl4, j) * alpha[i]), h[i], comp(du4, j) * comp(b4, j));
+      }
     }
     __syncthreads();
   }
@@ -225,23 +237,34 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int half = 1; half >= 0; --half) {
       const int tb = 8 * half;  // first step of this half
       float hs[4][8], hpre[4];  // states of steps tb..tb+7 and of step tb-1
+      float hh[4] = {hc[0], hc[1], hc[2], hc[3]};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float hh = hc[i];
+      for (int q = 0; q < tb / 4 + 2; ++q) {
+        const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * q]), du4 = ld4(&s.du[lane * ROW + 4 * q]);
 #pragma unroll
-        for (int t = 0; t < tb + 8; ++t) {
-          if (t == tb) hpre[i] = hh;
-          hh = fmaf(ex2_mufu(s.dl[lane * ROW + t] * alpha[i]), hh,
-                    s.du[lane * ROW + t] * s.B[(4 * g + i) * TB + t]);
-          if (t >= tb) hs[i][t - tb] = hh;
+        for (int i = 0; i < 4; ++i) {
+          const float4 b4 = ld4(&s.B[(4 * g + i) * TB + 4 * q]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int t = 4 * q + j;
+            if (t == tb) hpre[i] = hh[i];
+            hh[i] = fmaf(ex2_mufu(comp(dl4, j) * alpha[i]), hh[i], comp(du4, j) * comp(b4, j));
+            if (t >= tb) hs[i][t - tb] = hh[i];
+          }
         }
       }
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        float acc = 0.f;
+      for (int qq = 0; qq < 2; ++qq) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc = fmaf(s.C[(4 * g + i) * TB + tb + t], hs[i][t], acc);
-        s.ps[(g * CH + lane) * ROW + tb + t] = acc;
+        for (int i = 0; i < 4; ++i) {
+          const float4 c4 = ld4(&s.C[(4 * g + i) * TB + tb + 4 * qq]);
+          acc.x = fmaf(c4.x, hs[i][4 * qq + 0], acc.x);
+          acc.y = fmaf(c4.y, hs[i][4 * qq + 1], acc.y);
+          acc.z = fmaf(c4.z, hs[i][4 * qq + 2], acc.z);
+          acc.w = fmaf(c4.w, hs[i][4 * qq + 3], acc.w);
+        }
+        *reinterpret_cast<float4 *>(&s.ps[(g * CH + lane) * ROW + tb + 4 * qq]) = acc;
       }
 
       // adjoint, four steps at a time backwards
@@ -249,17 +272,24 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       for (int qq = 1; qq >= 0; --qq) {
         const int q = 2 * half + qq;
         float vB[16], vC[16];
+        const int t4 = tb + 4 * qq;  // first step of this quad
+        const float4 dl4 = ld4(&s.dl[lane * ROW + t4]), u4 = ld4(&s.u[lane * ROW + t4]),
+                     ds4 = ld4(&s.ds[lane * ROW + t4]);
+        float4 B4[4], C4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          B4[i] = ld4(&s.B[(4 * g + i) * TB + t4]);
+          C4[i] = ld4(&s.C[(4 * g + i) * TB + t4]);
+        }
+        float4 pu4, pd4;
 #pragma unroll
         for (int tq = 3; tq >= 0; --tq) {
           const int tl = 4 * qq + tq;  // step within the half
-          const int t = tb + tl;
-          const float dl = s.dl[lane * ROW + t], uu = s.u[lane * ROW + t],
-                      ds = s.ds[lane * ROW + t];
+          const float dl = comp(dl4, tq), uu = comp(u4, tq), ds = comp(ds4, tq);
           float pdu = 0.f, pdd = 0.f;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int n = 4 * g + i;
-            const float Bv = s.B[n * TB + t], Cv = s.C[n * TB + t];
+            const float Bv = comp(B4[i], tq), Cv = comp(C4[i], tq);
             const float hprev = tl > 0 ? hs[i][tl - 1] : hpre[i];
             const float a = ex2_mufu(dl * alpha[i]);
             lam[i] = fmaf(ds, Cv, lam[i]);
@@ -271,9 +301,13 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
             pdu = fmaf(lam[i] * dl, Bv, pdu);
             lam[i] *= a;
           }
-          s.pu[(g * CH + lane) * ROW + t] = pdu;
-          s.pd[(g * CH + lane) * ROW + t] = pdd;
+          if (tq == 0) { pu4.x = pdu; pd4.x = pdd; }
+          if (tq == 1) { pu4.y = pdu; pd4.y = pdd; }
+          if (tq == 2) { pu4.z = pdu; pd4.z = pdd; }
+          if (tq == 3) { pu4.w = pdu; pd4.w = pdd; }
         }
+        *reinterpret_cast<float4 *>(&s.pu[(g * CH + lane) * ROW + t4]) = pu4;
+        *reinterpret_cast<float4 *>(&s.pd[(g * CH + lane) * ROW + t4]) = pd4;
         // channel sums of dB, dC for states 4g + i, steps 4q + tq: the even
         // lane of each pair adds j = lane >> 1 = 4 i + tq
         const float rb = reduce_scatter16(vB, lane);
