@@ -73,6 +73,9 @@ def parse_args(argv=None):
     ap.add_argument("--varlen", type=int, default=0,
                     help="pack this many independent sequences into every row "
                          "(seeded random offsets; 0 = one sequence per row)")
+    ap.add_argument("--checkpoints", action="store_true",
+                    help="forward: also write the backward's state checkpoints; "
+                         "bwd: start from checkpoints written by a forward scan")
     ap.add_argument("--trapezoid", action="store_true",
                     help="three-term trapezoidal update instead of the Euler one")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
@@ -319,10 +322,17 @@ def run_bwd(args, rank, world, local_rank):
     g.manual_seed(48000)
     dy = torch.randn(w.batch, w.dim, w.seqlen, generator=g, device=dev)
 
+    ck = None
+    if args.checkpoints:
+        ck = sss.scan_checkpoints(w.batch, w.dim, w.dstate, w.seqlen, dev)
+        sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                               D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
+                               delta_softplus=w.softplus, checkpoints=ck)
+
     def step():
         sss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy,
                                D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, workspace=ws)
+                               delta_softplus=w.softplus, workspace=ws, checkpoints=ck)
 
     # workspace sized once (the size depends on the shapes only)
     nb = ctypes.c_size_t(0)
@@ -362,7 +372,8 @@ def run_bwd(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": max_ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": dict(workload_config(w), **{"pass": "bwd"}),
+        "config": dict(workload_config(w), **{"pass": "bwd"},
+                       **({"from_checkpoints": True} if args.checkpoints else {})),
         "state_updates_per_s": w.state_updates * K * world / (max_ms * 1e-3),
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
                      "unit": "GB/s", "frac": value / world / peak,
@@ -383,6 +394,9 @@ def run_ours(args, rank, world, local_rank):
     inp = workloads.make_inputs(w, device=dev)
     ydt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
     y = torch.empty((w.batch, w.dim, w.seqlen), dtype=ydt, device=dev)
+    ck = None
+    if args.checkpoints:
+        ck = sss.scan_checkpoints(w.batch, w.dim, w.dstate, w.seqlen, dev)
     cu_t = None
     if args.varlen > 0:
         cu_t = torch.tensor(varlen_offsets(w.seqlen, args.varlen),
@@ -391,7 +405,7 @@ def run_ours(args, rank, world, local_rank):
                                inp["C"], D=inp["D"], z=inp["z"],
                                delta_bias=inp["delta_bias"],
                                delta_softplus=w.softplus, y=y, cu_seqlens=cu_t,
-                               trapezoid=args.trapezoid)
+                               trapezoid=args.trapezoid, checkpoints=ck)
     ws_bytes = sss.scan_workspace_size(sargs)
     ws = sss.alloc_workspace(ws_bytes, dev)
     if ws is not None:
@@ -461,7 +475,8 @@ def run_ours(args, rank, world, local_rank):
                                inp["C"], D=inp["D"], z=inp["z"],
                                delta_bias=inp["delta_bias"],
                                delta_softplus=w.softplus, y=y, workspace=ws,
-                               cu_seqlens=cu_t, trapezoid=args.trapezoid)
+                               cu_seqlens=cu_t, trapezoid=args.trapezoid,
+                               checkpoints=ck)
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -499,7 +514,8 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": dict(workload_config(w, args.out_dtype),
                        **({"sequences_per_row": args.varlen} if args.varlen else {}),
-                       **({"update": "trapezoidal"} if args.trapezoid else {})),
+                       **({"update": "trapezoidal"} if args.trapezoid else {}),
+                       **({"writes_checkpoints": True} if args.checkpoints else {})),
         "state_updates_per_s": updates,
         "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": value / world / peak,

@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 5
+#define MSS_ABI_VERSION 6
 
 typedef enum {
   MSS_OK = 0,
@@ -152,6 +152,14 @@ typedef struct mss_scan_args {
      split sequence reads the step before it from u and B.  0: the Euler
      update above.  Not combined with cu_seqlens (MSS_ERR_UNSUPPORTED). */
   int trapezoid;
+  /* NULL, or an output of mss_scan_bwd_workspace_size() bytes that receives
+     the state of every channel at the start of every 16-step block, in the
+     layout mamba_selective_scan_bwd reads (mss_scan_bwd_args.checkpoints):
+     fp32 [tile][block][state][lane] with tile = b * ceil(dim / 32) + d / 32,
+     block = t / 16, lane = d % 32, and states padded to 4, 8 or 16.  A scan
+     that writes checkpoints is never split into chunks; not combined with
+     cu_seqlens or trapezoid (MSS_ERR_UNSUPPORTED). */
+  float *checkpoints;
 } mss_scan_args;
 
 /* Bytes of device workspace the scan needs for these arguments (0 when the
@@ -267,8 +275,13 @@ typedef struct mss_scan_bwd_args {
   float *dz;
   float *ddelta_bias;
   float *dh0;
+  /* NULL, or the checkpoints written by the forward scan of the same
+     inputs (mss_scan_args.checkpoints): the backward then skips its own
+     forward sweep and needs no workspace. */
+  const float *checkpoints;
   void *workspace;          /* device, >= mss_scan_bwd_workspace_size(),
-                               256-byte aligned */
+                               256-byte aligned; may be NULL with
+                               checkpoints */
   size_t workspace_bytes;
 } mss_scan_bwd_args;
 

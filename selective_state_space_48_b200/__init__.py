@@ -24,7 +24,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 5  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 6  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -86,6 +86,7 @@ class ScanArgs(ctypes.Structure):
         ("cu_seqlens", ctypes.c_void_p),
         ("num_seqs", ctypes.c_int64),
         ("trapezoid", ctypes.c_int),
+        ("checkpoints", ctypes.c_void_p),
     ]
 
 
@@ -124,7 +125,7 @@ class ScanBwdArgs(ctypes.Structure):
         ("delta_softplus", ctypes.c_int),
     ] + [(name, ctypes.c_void_p) for name in (
         "h0", "dy", "d_last", "du", "ddelta", "dA", "dB", "dC", "dD", "dz",
-        "ddelta_bias", "dh0", "workspace")] + [
+        "ddelta_bias", "dh0", "checkpoints", "workspace")] + [
         ("workspace_bytes", ctypes.c_size_t),
     ]
 
@@ -219,7 +220,8 @@ def _stream_handle(stream):
 def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                    delta_softplus=True, h0=None, y=None, last_state=None,
                    workspace=None, plan_splits=0, test_flags=0,
-                   spin_timeout_ns=0, cu_seqlens=None, trapezoid=False) -> ScanArgs:
+                   spin_timeout_ns=0, cu_seqlens=None, trapezoid=False,
+                   checkpoints=None) -> ScanArgs:
     batch, dim, L = u.shape
     N = A.shape[1]
     ind = u.dtype
@@ -251,6 +253,9 @@ def make_scan_args(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     a.test_flags = int(test_flags)
     a.spin_timeout_ns = int(spin_timeout_ns)
     a.trapezoid = 1 if trapezoid else 0
+    if checkpoints is not None:
+        _check_cuda("checkpoints", checkpoints, torch.float32)
+        a.checkpoints = checkpoints.data_ptr()
     if cu_seqlens is not None:
         _check_cuda("cu_seqlens", cu_seqlens, torch.int32)
         if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
@@ -284,7 +289,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                        out_dtype=torch.float32, y=None, last_state=None,
                        workspace=None, stream=None, plan_splits=0,
                        test_flags=0, spin_timeout_ns=0, check_status=False,
-                       cu_seqlens=None, trapezoid=False):
+                       cu_seqlens=None, trapezoid=False, checkpoints=None):
     """Forward selective scan through ``mamba_selective_scan_fwd``.
 
     u, delta, z: (batch, dim, L); B, C: (batch, N, L) (float32 or bfloat16,
@@ -292,7 +297,9 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     (batch, dim, N) float32.  u, delta, z, B, C and y may be views whose
     last dimension is contiguous.  ``cu_seqlens`` (int32 CUDA tensor of
     num_seqs + 1 offsets, 0 ... L) packs independent sequences into every
-    row.  ``trapezoid`` selects the three-term trapezoidal update.  Returns
+    row.  ``trapezoid`` selects the three-term trapezoidal update.
+    ``checkpoints`` (from ``scan_checkpoints``) receives the states the
+    backward pass starts from.  Returns
     y (batch, dim, L) in ``out_dtype`` (and the final state when
     ``return_last_state``).
     """
@@ -305,7 +312,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                                  device=u.device)
     args = make_scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus,
                           h0, y, last_state, None, plan_splits, test_flags,
-                          spin_timeout_ns, cu_seqlens, trapezoid)
+                          spin_timeout_ns, cu_seqlens, trapezoid, checkpoints)
     if workspace is None:
         workspace = alloc_workspace(scan_workspace_size(args), u.device)
     if workspace is not None:
@@ -377,12 +384,13 @@ __all__ = [
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
                        delta_softplus=True, h0=None, d_last=None, stream=None,
-                       workspace=None):
+                       workspace=None, checkpoints=None):
     """Gradients of sum(dy * y) + sum(d_last * last_state) for the forward
     scan on the same inputs, through ``mamba_selective_scan_bwd``.
 
     Dense inputs as for ``selective_scan_fwd``; dy (batch, dim, L) and
-    d_last (batch, dim, N) float32.  Returns a dict of float32 tensors du,
+    d_last (batch, dim, N) float32.  ``checkpoints`` written by the forward
+    scan of the same inputs let the backward skip its forward sweep.  Returns a dict of float32 tensors du,
     ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0 (None for absent inputs).
     """
     batch, dim, L = u.shape
@@ -418,6 +426,7 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     a.D, a.z, a.delta_bias = _ptr(D), _ptr(z), _ptr(delta_bias)
     a.delta_softplus = 1 if delta_softplus else 0
     a.h0, a.dy, a.d_last = _ptr(h0), _ptr(dy), _ptr(d_last)
+    a.checkpoints = _ptr(checkpoints)
     for k, v in g.items():
         setattr(a, k, _ptr(v))
     lib = load_library()
@@ -425,12 +434,25 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     rc = lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n))
     if rc != MSS_OK:
         raise MssError(rc, "mss_scan_bwd_workspace_size")
-    if workspace is None:
+    if workspace is None and checkpoints is None:
         workspace = alloc_workspace(int(n.value), dev)
-    a.workspace = workspace.data_ptr()
-    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    if workspace is not None:
+        a.workspace = workspace.data_ptr()
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
     rc = lib.mamba_selective_scan_bwd(ctypes.byref(a), _stream_handle(stream))
     if rc != MSS_OK:
         raise MssError(rc, "mamba_selective_scan_bwd")
-    workspace.record_stream(stream or torch.cuda.current_stream())
+    if workspace is not None:
+        workspace.record_stream(stream or torch.cuda.current_stream())
     return g
+
+
+def scan_checkpoints(batch, dim, dstate, seqlen, device):
+    """A buffer for the forward scan's checkpoints (float32, the size
+    ``mss_scan_bwd_workspace_size`` reports)."""
+    groups = (dstate + 3) // 4
+    groups = 1 if groups <= 1 else (2 if groups == 2 else 4)
+    tiles = batch * ((dim + 31) // 32)
+    nblk = (seqlen + 15) // 16
+    return torch.empty(tiles * nblk * 4 * groups * 32, dtype=torch.float32,
+                       device=device)

@@ -120,6 +120,9 @@ mss_status check_scan_args(const mss_scan_args *a) {
     return MSS_ERR_INVALID_ARG;
   if (a->trapezoid != 0 && a->trapezoid != 1) return MSS_ERR_INVALID_ARG;
   if (a->trapezoid && a->cu_seqlens) return MSS_ERR_UNSUPPORTED;
+  if (a->checkpoints && (a->trapezoid || a->cu_seqlens)) return MSS_ERR_UNSUPPORTED;
+  if (a->checkpoints && (!aligned(a->checkpoints, 4) || a->plan_splits > 1))
+    return MSS_ERR_INVALID_ARG;
   const size_t ei = esize(a->in_dtype), eo = esize(a->out_dtype);
   if (!aligned(a->u, ei) || !aligned(a->delta, ei) || !aligned(a->B, ei) ||
       !aligned(a->C, ei) || (a->z && !aligned(a->z, ei)) ||
@@ -137,6 +140,9 @@ mss_status make_plan(const mss_scan_args *a, Plan *pl) {
                                   kChannelsPerBlock);
   pl->tiles = a->batch * pl->ch_tiles;
   int64_t want = a->plan_splits;
+  // checkpoints hold the true state at every block: only an unsplit scan
+  // has it before its carry correction
+  if (a->checkpoints) want = 1;
   if (want == 0) {
     // Split the sequence only when there are fewer channel tiles than SMs:
     // a chunk that does not start the sequence pays a carry correction whose
@@ -190,6 +196,7 @@ void fill_scan_params(const mss_scan_args *a, const Plan &pl, ScanParams *p) {
   p->cu = a->cu_seqlens;
   p->nseq = a->cu_seqlens ? a->num_seqs : 0;
   p->trap = a->trapezoid;
+  p->ckpt_out = a->checkpoints;
   p->chunk = pl.chunk;
   p->splits = pl.splits;
   p->ch_tiles = pl.ch_tiles;
@@ -333,7 +340,7 @@ mss_status check_bwd_args(const mss_scan_bwd_args *a) {
     if (q && !aligned(q, ei)) return MSS_ERR_INVALID_ARG;
   const void *f32[] = {a->A, a->D, a->delta_bias, a->h0, a->dy, a->d_last, a->du,
                        a->ddelta, a->dA, a->dB, a->dC, a->dD, a->dz,
-                       a->ddelta_bias, a->dh0};
+                       a->ddelta_bias, a->dh0, a->checkpoints};
   for (const void *q : f32)
     if (q && !aligned(q, 4)) return MSS_ERR_INVALID_ARG;
   return MSS_OK;
@@ -356,7 +363,8 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   size_t need = 0;
   const mss_status st = mss_scan_bwd_workspace_size(a, &need);
   if (st != MSS_OK) return st;
-  if (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256))
+  if (!a->checkpoints &&
+      (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256)))
     return MSS_ERR_WORKSPACE;
   BwdParams p{};
   p.batch = a->batch;
@@ -384,7 +392,9 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   p.dz = a->dz;
   p.ddelta_bias = a->ddelta_bias;
   p.dh0 = a->dh0;
-  p.ckpt = static_cast<float *>(a->workspace);
+  p.ckpt = a->checkpoints ? const_cast<float *>(a->checkpoints)
+                          : static_cast<float *>(a->workspace);
+  p.ckpt_given = a->checkpoints ? 1 : 0;
   p.ch_tiles = static_cast<int>((a->dim + kBwdChannels - 1) / kBwdChannels);
   p.tiles = a->batch * p.ch_tiles;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -189,8 +189,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   };
 
   // ------------------------------------------------------ forward sweep
+  // (skipped when the forward scan already wrote the checkpoints)
   __syncthreads();
-  for (int k = 0; k < nblk; ++k) {
+  for (int k = 0; k < (p.ckpt_given ? 0 : nblk); ++k) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       ckpt[(static_cast<int64_t>(k) * NP + 4 * g + i) * CH + lane] = h[i];

@@ -25,6 +25,7 @@ struct BwdParams {
   const float *d_last;
   float *du, *ddelta, *dA, *dB, *dC, *dD, *dz, *ddelta_bias, *dh0;
   float *ckpt;      // workspace: one state per channel and 16-step block
+  int ckpt_given;   // ckpt already holds the forward scan's states
   int ch_tiles;     // ceil(dim / kBwdChannels)
   int64_t tiles;    // batch * ch_tiles
 };

@@ -78,6 +78,7 @@ constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 constexpr int kModePlain = 0;
 constexpr int kModeVarlen = 1;
 constexpr int kModeTrap = 2;
+constexpr int kModeCkpt = 3;  // ordinary scan that also writes checkpoints
 
 template <typename InT, int G, bool TRAP = false>
 struct Layout {
@@ -609,6 +610,7 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   using S = Scan<InT, OutT, G, TMA, MODE>;
   constexpr bool VARLEN = S::VARLEN;
   constexpr bool TRAP = S::TRAP;
+  constexpr bool CKPT = MODE == kModeCkpt;
   using Lay = typename S::Lay;
   constexpr int NP = 4 * G;
   constexpr int NSCAN = 32 * G;
@@ -707,6 +709,12 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
       const int s = i & 1;
       wait_hand(kTilesReady, s);
       if (i >= 2) wait_hand(kPartFree, s);
+      if (CKPT) {
+        // state before block i for the backward pass (unsplit plans only)
+        float *ck = p.ckpt_out + ((item * nblk + i) * NP + 4 * g) * static_cast<int64_t>(CH) + lane;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ck[j * CH] = h[j];
+      }
       sc.scan(s, g, lane, h, al2, dsum, split, bprev);
       if (i + 2 < nblk) mbar_arrive(sc.hand(kTilesFree, s));
       mbar_arrive(sc.hand(kPartReady, s));
@@ -989,6 +997,7 @@ template <typename InT, typename OutT>
 cudaError_t dispatch(const ScanParams &p, bool tma, const TmaMaps &maps, cudaStream_t s) {
   if (p.cu) return dispatch_v<InT, OutT, kModeVarlen>(p, tma, maps, s);
   if (p.trap) return dispatch_v<InT, OutT, kModeTrap>(p, tma, maps, s);
+  if (p.ckpt_out) return dispatch_v<InT, OutT, kModeCkpt>(p, tma, maps, s);
   return dispatch_v<InT, OutT, kModePlain>(p, tma, maps, s);
 }
 

@@ -39,6 +39,8 @@ struct ScanParams {
   int64_t nseq;
   // three-term trapezoidal update (1) instead of the Euler one (0)
   int trap;
+  // optional: state at the start of every block, [tile][block][4G][CH]
+  float *ckpt_out;
   int y_vec;       // rows of y allow 4-element vector stores (set at launch)
   // launch plan
   int64_t chunk;   // timesteps per sequence chunk (multiple of kTimeBlock)

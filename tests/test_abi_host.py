@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 5
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 6
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
@@ -149,6 +149,9 @@ def test_workspace_size_follows_plan(lib):
     (dict(cu_seqlens=0x10002, num_seqs=2), sss.MSS_ERR_INVALID_ARG),  # misaligned
     (dict(trapezoid=2), sss.MSS_ERR_INVALID_ARG),
     (dict(trapezoid=1, cu_seqlens=0x10000, num_seqs=2), sss.MSS_ERR_UNSUPPORTED),
+    (dict(checkpoints=0x10000, trapezoid=1), sss.MSS_ERR_UNSUPPORTED),
+    (dict(checkpoints=0x10002), sss.MSS_ERR_INVALID_ARG),           # misaligned
+    (dict(checkpoints=0x10000, plan_splits=3), sss.MSS_ERR_INVALID_ARG),
 ])
 def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     a = _args(**kw)
@@ -167,6 +170,7 @@ def test_bad_arguments_are_rejected_before_launch(lib, kw, code):
     dict(stride_delta=(0, 0)),                 # packed
     dict(cu_seqlens=0x10000, num_seqs=5),      # packed sequences
     dict(trapezoid=1),                         # three-term update
+    dict(checkpoints=0x10000),                 # states for the backward
 ])
 def test_valid_strides_are_accepted(lib, kw):
     rc, n = _ws(lib, _args(plan_splits=1, **kw))
@@ -232,3 +236,13 @@ def test_bwd_bad_arguments_are_rejected(kw, code):
 def test_bwd_missing_workspace_is_reported():
     lib = sss.load_library()
     assert lib.mamba_selective_scan_bwd(ctypes.byref(_bwd_args()), None) == sss.MSS_ERR_WORKSPACE
+
+
+def test_checkpoint_buffer_matches_the_workspace_size():
+    lib = sss.load_library()
+    for N in (1, 4, 5, 9, 12, 16):
+        a = _bwd_args(dstate=N, seqlen=1000)
+        n = ctypes.c_size_t(0)
+        assert lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == sss.MSS_OK
+        buf = sss.scan_checkpoints(2, 40, N, 1000, "cpu")
+        assert buf.numel() * 4 == n.value, N
