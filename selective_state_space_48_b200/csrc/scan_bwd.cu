@@ -188,6 +188,66 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     }
   };
 
+  // The reverse sweep reads block k - 1 from HBM into registers while block
+  // k is computed, and writes it to the tiles at the start of the next
+  // iteration: fetch (loads only) and commit (math and shared stores).
+  constexpr int E = CH * TB / NT;             // (channel, step) elements per thread
+  constexpr int EB = (NP * TB + NT - 1) / NT; // (state, step) elements per thread
+  struct Raw {
+    float u[E], x[E], z[E], dy[E], B[EB], C[EB];
+    unsigned ok;  // bit e: element e lies inside the tensors
+  };
+  auto fetch = [&](int k, Raw &r) {
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+    r.ok = 0u;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
+      const int64_t dd = d0 + c;
+      const bool ok = dd < p.dim && t < nt;
+      const int64_t off = (b * p.dim + dd) * L + t0 + t;
+      r.u[e] = ok ? ld_f32(gu, off) : 0.f;
+      r.x[e] = ok ? ld_f32(gd, off) : 0.f;
+      r.z[e] = (ok && gz) ? ld_f32(gz, off) : 0.f;
+      r.dy[e] = ok ? p.dy[off] : 0.f;
+      if (ok) r.ok |= 1u << e;
+    }
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+      const int idx = tid + NT * e;
+      const int n = idx / TB, t = idx % TB;
+      const bool ok = idx < NP * TB && n < p.dstate && t < nt;
+      const int64_t off = (b * p.dstate + n) * L + t0 + t;
+      r.B[e] = ok ? ld_f32(gB, off) : 0.f;
+      r.C[e] = ok ? ld_f32(gC, off) : 0.f;
+    }
+  };
+  auto commit = [&](const Raw &r) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
+      const bool ok = (r.ok >> e) & 1u;
+      const float x = ok ? r.x[e] + s.bias[c] : 0.f;
+      const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
+      s.u[c * ROW + t] = r.u[e];
+      s.dl[c * ROW + t] = dl;
+      s.du[c * ROW + t] = dl * r.u[e];
+      s.z[c * ROW + t] = r.z[e];
+      s.dy[c * ROW + t] = r.dy[e];
+      s.ds[c * ROW + t] = gz ? r.dy[e] * silu_f(r.z[e]) : r.dy[e];
+      s.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
+    }
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+      const int idx = tid + NT * e;
+      if (idx < NP * TB) {
+        s.B[idx] = r.B[e];
+        s.C[idx] = r.C[e];
+      }
+    }
+  };
+
   // ------------------------------------------------------ forward sweep
   // (skipped when the forward scan already wrote the checkpoints)
   __syncthreads();
@@ -219,15 +279,25 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
                  ? p.d_last[(b * p.dim + d) * p.dstate + 4 * g + i] : 0.f;
     dA[i] = 0.f;
   }
+  // the checkpoint of the block after the current one is read a block early
+  float hnext[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    hnext[i] = ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + i) * CH + lane];
+  Raw raw;
+  fetch(nblk - 1, raw);
   for (int k = nblk - 1; k >= 0; --k) {
     const int64_t t0 = static_cast<int64_t>(k) * TB;
     const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
-    load_block(k, true);
+    commit(raw);
     float hc[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      hc[i] = ckpt[(static_cast<int64_t>(k) * NP + 4 * g + i) * CH + lane];
+    for (int i = 0; i < 4; ++i) {
+      hc[i] = hnext[i];
+      if (k > 0) hnext[i] = ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + i) * CH + lane];
+    }
     __syncthreads();
+    if (k > 0) fetch(k - 1, raw);  // in flight while block k is computed
 
     // Two halves of the block, the later one first.  For each: recompute
     // the states of its 8 steps from the checkpoint into registers (with
