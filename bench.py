@@ -78,8 +78,11 @@ def parse_args(argv=None):
                          "bwd: start from checkpoints written by a forward scan")
     ap.add_argument("--trapezoid", action="store_true",
                     help="three-term trapezoidal update instead of the Euler one")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
-                    help="bwd times the backward scan (gradients of all inputs)")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "decode"], default="fwd",
+                    help="bwd times the backward scan (gradients of all inputs); "
+                         "decode times one-token state updates")
+    ap.add_argument("--decode-batch", type=int, default=1024,
+                    help="batch rows of one decode step (the workload's dim and dstate)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work of the oracle baseline sample")
@@ -386,6 +389,77 @@ def run_bwd(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def decode_algorithmic_bytes(batch, dim, dstate, in_bytes) -> int:
+    """One decode step: the fp32 state read and written once, x, dt, z in
+    and y (fp32) out per channel, B and C per batch row, A, D, dt_bias."""
+    return (batch * dim * (8 * dstate + 3 * in_bytes + 4) + batch * dstate * 2 * in_bytes
+            + dim * dstate * 4 + dim * 8)
+
+
+def run_decode(args, rank, world, local_rank):
+    import selective_state_space_48_b200 as sss
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.BY_NAME[args.workload]
+    bt, D, N = args.decode_batch, w.dim, w.dstate
+    dt_ = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
+    g = torch.Generator(device=dev)
+    g.manual_seed(48000)
+    rnd = lambda *shape: torch.randn(*shape, generator=g, device=dev)
+    state = rnd(bt, D, N)
+    x, dtv, z = rnd(bt, D).to(dt_), rnd(bt, D).to(dt_), rnd(bt, D).to(dt_)
+    B, C = rnd(bt, N).to(dt_), rnd(bt, N).to(dt_)
+    A = -torch.arange(1, N + 1, device=dev, dtype=torch.float32).repeat(D, 1)
+    Dv = rnd(D)
+    bias = torch.log(torch.expm1(torch.rand(D, generator=g, device=dev) * 0.099 + 1e-3))
+    y = torch.empty(bt, D, device=dev)
+
+    def step():
+        sss.selective_state_update(state, x, dtv, A, B, C, D=Dv, z=z, dt_bias=bias, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    stream = torch.cuda.current_stream(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(world)
+    max_ms = reduce_max(t0.elapsed_time(t1), world)
+    nbytes = decode_algorithmic_bytes(bt, D, N, 2 if dt_ == torch.bfloat16 else 4)
+    value = whole_job_gbs(nbytes, K, world, max_ms)
+    peak, src = measured_peaks()
+    line = {
+        "metric": "selective state update (decode) HBM GB/s; tokens/s",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": max_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "pass": "decode", "batch": bt, "dim": D,
+                   "dstate": N, "in_dtype": w.in_dtype,
+                   "l2": f"{nbytes / 1e6:.0f} MB per step"},
+        "tokens_per_s": bt * K * world / (max_ms * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
+                     "unit": "GB/s", "frac": value / world / peak,
+                     "peak_source": src, "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes},
+        "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
+        "kernel_source_hash": kernel_source_hash(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, rank, world, local_rank):
     import selective_state_space_48_b200 as sss
     torch.cuda.set_device(local_rank)
@@ -600,6 +674,8 @@ def main(argv=None):
     try:
         if args.pass_ == "bwd":
             run_bwd(args, rank, world, local_rank)
+        elif args.pass_ == "decode":
+            run_decode(args, rank, world, local_rank)
         else:
             line = run_ours(args, rank, world, local_rank)
             if rank == 0:
