@@ -34,19 +34,31 @@ __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p)
   const float sx = step * x;
   float *st = p.state + ch * p.dstate;
   float acc = 0.f;
-  if (N == 16 && nst == 16 && (reinterpret_cast<uintptr_t>(st) & 15) == 0) {
+  if (N == 16 && nst == 16 && (reinterpret_cast<uintptr_t>(st) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(p.A) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(p.B) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(p.C) & 15) == 0) {
+    // 16 states: the state, A's row and the batch row's B and C move as
+    // 16-byte vectors (B, C rows are shared by the channels of a batch row)
+    const float *Ad = p.A + d * 16;
+    const InT *Bb = static_cast<const InT *>(p.B) + b * 16;
+    const InT *Cb = static_cast<const InT *>(p.C) + b * 16;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float4 hv = reinterpret_cast<float4 *>(st)[q];
-      float hs[4] = {hv.x, hv.y, hv.z, hv.w};
+      const float4 hv = reinterpret_cast<const float4 *>(st)[q];
+      const float4 av = reinterpret_cast<const float4 *>(Ad)[q];
+      const float4 bv = load4_f32(Bb + 4 * q);
+      const float4 cv = load4_f32(Cb + 4 * q);
+      const float hs[4] = {hv.x, hv.y, hv.z, hv.w}, as[4] = {av.x, av.y, av.z, av.w},
+                  bs[4] = {bv.x, bv.y, bv.z, bv.w}, cs[4] = {cv.x, cv.y, cv.z, cv.w};
+      float ho[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int n = 4 * q + j;
-        const float a = ex2_mufu(step * p.A[d * 16 + n] * kLog2e);
-        hs[j] = fmaf(a, hs[j], sx * ld<InT>(p.B, b * 16 + n));
-        acc = fmaf(ld<InT>(p.C, b * 16 + n), hs[j], acc);
+        const float a = ex2_mufu(step * as[j] * kLog2e);
+        ho[j] = fmaf(a, hs[j], sx * bs[j]);
+        acc = fmaf(cs[j], ho[j], acc);
       }
-      reinterpret_cast<float4 *>(st)[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
+      reinterpret_cast<float4 *>(st)[q] = make_float4(ho[0], ho[1], ho[2], ho[3]);
     }
   } else {
     for (int n = 0; n < nst; ++n) {

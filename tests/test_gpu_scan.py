@@ -226,3 +226,24 @@ def test_state_update_matches_oracle(dt, N):
     tol = 1e-5
     assert norm_err(y.cpu(), y_ref) <= tol
     assert norm_err(st.cpu(), st_ref) <= tol
+
+
+def test_state_update_with_unaligned_B_C_takes_the_general_path():
+    """B and C starting off a 16-byte boundary use the scalar path; the
+    result is the same as from aligned copies."""
+    batch, dim, N = 2, 64, 16
+    g = torch.Generator(device="cuda")
+    g.manual_seed(91)
+    r = lambda *s: torch.randn(*s, generator=g, device="cuda")
+    state = r(batch, dim, N)
+    x, dtv = r(batch, dim), r(batch, dim)
+    A = -torch.rand(dim, N, generator=g, device="cuda") * 3
+    flatB, flatC = r(batch * N + 1), r(batch * N + 1)
+    B_off, C_off = flatB[1:].view(batch, N), flatC[1:].view(batch, N)
+    assert B_off.data_ptr() % 16 != 0
+    s1, s2 = state.clone(), state.clone()
+    y1 = sss.selective_state_update(s1, x, dtv, A, B_off, C_off)
+    y2 = sss.selective_state_update(s2, x, dtv, A, B_off.clone(), C_off.clone())
+    torch.cuda.synchronize()
+    assert torch.allclose(y1, y2, rtol=1e-6, atol=1e-6)
+    assert torch.allclose(s1, s2, rtol=1e-6, atol=1e-6)
