@@ -41,8 +41,14 @@
  * Errors.  Argument checks happen before any launch; a failing check returns
  * MSS_ERR_INVALID_ARG or MSS_ERR_UNSUPPORTED and enqueues nothing.  A CUDA
  * launch error returns MSS_ERR_CUDA.  Errors detected on the device (a
- * bounded wait that ran out) are written to a status word inside the
- * workspace and reported by mss_scan_status().
+ * bounded wait that ran out) are written to a status word, inside the
+ * workspace for a scan split into chunks and in the library's own device
+ * memory otherwise, and reported by mss_scan_status().
+ *
+ * Besides the scan above, the library offers packed sequences, strided
+ * views, the three-term trapezoidal update and state checkpoints (fields of
+ * mss_scan_args), the backward pass (mamba_selective_scan_bwd) and the
+ * single-token decode step (selective_state_update).
  */
 #ifndef SSS48_SELECTIVE_SCAN_H
 #define SSS48_SELECTIVE_SCAN_H
@@ -172,7 +178,10 @@ mss_status mss_scan_workspace_size(const mss_scan_args *args, size_t *bytes);
 mss_status mamba_selective_scan_fwd(const mss_scan_args *args, void *stream);
 
 /* Synchronises `stream`, then reports the device-side status of the last
- * scan that used args->workspace (MSS_OK when the scan needed none). */
+ * scan with these arguments: for a split scan the status word in
+ * args->workspace, otherwise the library's own word, which is read and
+ * cleared (so it reports every unsplit scan since the previous call, on any
+ * stream of this device). */
 mss_status mss_scan_status(const mss_scan_args *args, void *stream);
 
 /* The same forward scan for callers that cannot allocate device memory:
