@@ -314,50 +314,51 @@ struct Scan {
     }
   }
 
-  // y = (sum of state-group shares + D u) * silu(z), or y += shares * silu(z);
-  // four timesteps per thread and iteration, stored with one 16-byte (fp32)
-  // or 8-byte (bf16) store when the row allows it.
-  __device__ void epilogue(int stage, int set, int blk, bool accumulate, int ti,
-                           int nth) const {
-    const int64_t t0 = t0_of(blk);
-    const int nt = nt_of(blk);
-    const InT *ru = raw(stage, 0), *rz = raw(stage, 2);
-    const float *sPart = fpart(set), *sD = f32(Lay::dskip);
-    OutT *y = static_cast<OutT *>(p.y);
+  // Correction pass, thread ti < CH * TB / 4: the y values of its quad
+  // (channel ti / (TB/4), four steps) of block `blk`, read before the
+  // block's carry term is computed so the load latency overlaps it.
+  __device__ float4 load_y_quad(int blk, int ti) const {
     constexpr int QT = TB / 4;
-    for (int idx = ti; idx < CH * QT; idx += nth) {
-      const int c = idx / QT, t = 4 * (idx % QT);
-      if (d0 + c >= p.dim || t >= nt) continue;
-      float4 s = *reinterpret_cast<const float4 *>(sPart + c * ROW + t);
+    const int c = ti / QT, t = 4 * (ti % QT);
+    const int nt = nt_of(blk);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (d0 + c >= p.dim || t >= nt) return v;
+    const OutT *yr = static_cast<const OutT *>(p.y) + b * p.sy[0] + (d0 + c) * p.sy[1] +
+                     t0_of(blk) + t;
+    if (p.y_vec && t + 4 <= nt) return load4_f32(yr);
+    float sv[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < 4 && t + j < nt; ++j) sv[j] = to_f32<OutT>(yr[j]);
+    return make_float4(sv[0], sv[1], sv[2], sv[3]);
+  }
+
+  // Correction pass: y += (sum of the state-group shares) * silu(z) for the
+  // quad of thread ti < CH * TB / 4, whose old y values are `yq`.
+  __device__ void epilogue_acc(int stage, int set, int blk, int ti, const float4 &yq) const {
+    constexpr int QT = TB / 4;
+    const int c = ti / QT, t = 4 * (ti % QT);
+    const int nt = nt_of(blk);
+    if (d0 + c >= p.dim || t >= nt) return;
+    const InT *rz = raw(stage, 2);
+    const float *sPart = fpart(set);
+    float4 s = *reinterpret_cast<const float4 *>(sPart + c * ROW + t);
 #pragma unroll
-      for (int g = 1; g < G; ++g) {
-        const float4 v = *reinterpret_cast<const float4 *>(sPart + (g * CH + c) * ROW + t);
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-      }
-      if (!accumulate) {
-        const float4 u = load4_f32(ru + c * TB + t);
-        const float dk = sD[c];
-        s.x = fmaf(dk, u.x, s.x); s.y = fmaf(dk, u.y, s.y);
-        s.z = fmaf(dk, u.z, s.z); s.w = fmaf(dk, u.w, s.w);
-      }
-      if (has_z) {
-        const float4 z = load4_f32(rz + c * TB + t);
-        const float2 g01 = silu2_f(make_float2(z.x, z.y));
-        const float2 g23 = silu2_f(make_float2(z.z, z.w));
-        s.x *= g01.x; s.y *= g01.y; s.z *= g23.x; s.w *= g23.y;
-      }
-      OutT *yr = y + b * p.sy[0] + (d0 + c) * p.sy[1] + t0 + t;
-      if (p.y_vec && t + 4 <= nt) {
-        if (accumulate) {
-          s.x += to_f32<OutT>(yr[0]); s.y += to_f32<OutT>(yr[1]);
-          s.z += to_f32<OutT>(yr[2]); s.w += to_f32<OutT>(yr[3]);
-        }
-        store4(yr, s);
-      } else {
-        const float sv[4] = {s.x, s.y, s.z, s.w};
-        for (int j = 0; j < 4 && t + j < nt; ++j)
-          yr[j] = from_f32<OutT>(accumulate ? sv[j] + to_f32<OutT>(yr[j]) : sv[j]);
-      }
+    for (int g = 1; g < G; ++g) {
+      const float4 v = *reinterpret_cast<const float4 *>(sPart + (g * CH + c) * ROW + t);
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    if (has_z) {
+      const float4 z = load4_f32(rz + c * TB + t);
+      const float2 g01 = silu2_f(make_float2(z.x, z.y));
+      const float2 g23 = silu2_f(make_float2(z.z, z.w));
+      s.x *= g01.x; s.y *= g01.y; s.z *= g23.x; s.w *= g23.y;
+    }
+    s.x += yq.x; s.y += yq.y; s.z += yq.z; s.w += yq.w;
+    OutT *yr = static_cast<OutT *>(p.y) + b * p.sy[0] + (d0 + c) * p.sy[1] + t0_of(blk) + t;
+    if (p.y_vec && t + 4 <= nt) {
+      store4(yr, s);
+    } else {
+      const float sv[4] = {s.x, s.y, s.z, s.w};
+      for (int j = 0; j < 4 && t + j < nt; ++j) yr[j] = from_f32<OutT>(sv[j]);
     }
   }
 
@@ -871,7 +872,11 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   bool wactive = true;  // this scan warp still has carried terms to add
   const int base = nblk % STAGES;
   for (int j = 0; j < PREFETCH; ++j) sc.request(j, nblk, base, tid, NALL);
+  constexpr int kQuads = CH * (TB / 4);  // y quads of a block, one per thread
   for (int i = 0; i < nblk; ++i) {
+    // this block's old y, loaded now so the latency overlaps prep and the
+    // carry term (the main pass wrote it before the last block barrier)
+    const float4 yq = tid < kQuads ? sc.load_y_quad(i, tid) : make_float4(0.f, 0.f, 0.f, 0.f);
     const bool ok = sc.land(i, nblk, base, phase);
     if (!__syncthreads_and(ok)) {
       if (tid == 0) atomicOr(p.status, kStatusTimeout);
@@ -882,7 +887,7 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     __syncthreads();
     if (is_scan) sc.scan_carry(0, g, lane, alpha, h_in, sigma, wactive);
     __syncthreads();
-    sc.epilogue(stage, 0, i, true, tid, NALL);
+    if (tid < kQuads) sc.epilogue_acc(stage, 0, i, tid, yq);
     need = false;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
