@@ -456,3 +456,41 @@ def scan_checkpoints(batch, dim, dstate, seqlen, device):
     nblk = (seqlen + 15) // 16
     return torch.empty(tiles * nblk * 4 * groups * 32, dtype=torch.float32,
                        device=device)
+
+
+class _SelectiveScanFn(torch.autograd.Function):
+    """Autograd wrapper: forward through mamba_selective_scan_fwd (writing
+    the backward's state checkpoints), backward through
+    mamba_selective_scan_bwd starting from them."""
+
+    @staticmethod
+    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0):
+        batch, dim, L = u.shape
+        ck = scan_checkpoints(batch, dim, A.shape[1], L, u.device)
+        y = selective_scan_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=delta_bias,
+                               delta_softplus=delta_softplus, h0=h0, checkpoints=ck)
+        ctx.delta_softplus = delta_softplus
+        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, h0, ck)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        u, delta, A, B, C, D, z, delta_bias, h0, ck = ctx.saved_tensors
+        g = selective_scan_bwd(u, delta, A, B, C, dy.float().contiguous(), D=D, z=z,
+                               delta_bias=delta_bias, delta_softplus=ctx.delta_softplus,
+                               h0=h0, checkpoints=ck)
+        cast = lambda t, like: None if t is None else t.to(like.dtype)
+        return (cast(g["du"], u), cast(g["ddelta"], delta), g["dA"], cast(g["dB"], B),
+                cast(g["dC"], C), g["dD"], cast(g["dz"], z) if z is not None else None,
+                g["ddelta_bias"], None, g["dh0"] if h0 is not None else None)
+
+
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                      delta_softplus=True, h0=None):
+    """Differentiable selective scan: y (batch, dim, L) float32, with
+    gradients for every tensor input through the CUDA backward pass.  Dense
+    inputs as for ``selective_scan_fwd``; gradients come back in the
+    inputs' dtypes (computed in float32)."""
+    return _SelectiveScanFn.apply(u.contiguous(), delta.contiguous(), A, B.contiguous(),
+                                  C.contiguous(), D, None if z is None else z.contiguous(),
+                                  delta_bias, delta_softplus, h0)
