@@ -70,6 +70,9 @@ def _bind(lib):
     lib.oracle_selective_scan_bwd_f64.argtypes = (
         [_I64] * 4 + [_D] * 8 + [ctypes.c_int] + [_D] * 12)
     lib.oracle_selective_scan_bwd_f64.restype = ctypes.c_int
+    lib.oracle_ssd_scan_f64.argtypes = (
+        [_I64] * 6 + [_D] * 8 + [ctypes.c_int, _D, _D, _D])
+    lib.oracle_ssd_scan_f64.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -219,3 +222,30 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     if rc != 0:
         raise ValueError("oracle_selective_scan_bwd_f64 rejected the sizes")
     return out
+
+
+def ssd_scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
+             h0=None, return_last_state=False, lib=None):
+    """Sequential fp64 Mamba-2 (SSD) scan: A is one scalar per head.
+
+    x, z: (batch, L, nheads, headdim); dt: (batch, L, nheads);
+    A, D, dt_bias: (nheads,); B, C: (batch, L, ngroups, dstate);
+    h0: (batch, nheads, headdim, dstate).  Returns y (batch, L, nheads,
+    headdim) float64, and the final state when ``return_last_state``.
+    """
+    lib = lib or load()
+    x, dt, A, B, C = (_f64(a) for a in (x, dt, A, B, C))
+    D, z, dt_bias, h0 = (_f64(a) for a in (D, z, dt_bias, h0))
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dt.shape == (batch, L, H) and A.shape == (H,)
+    assert B.shape == (batch, L, G, N) and C.shape == B.shape
+    y = np.empty((batch, L, H, P), dtype=np.float64)
+    last = np.empty((batch, H, P, N), dtype=np.float64) if return_last_state else None
+    rc = lib.oracle_ssd_scan_f64(
+        batch, L, H, P, G, N, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+        _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)), _ptr(h0),
+        _ptr(y), _ptr(last))
+    if rc != 0:
+        raise ValueError("oracle_ssd_scan_f64 rejected the sizes")
+    return (y, last) if return_last_state else y

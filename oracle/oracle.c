@@ -24,6 +24,15 @@
  *           (alpha, beta, gamma not given there; read as the trapezoidal
  *           rule for the same ODE: alpha = exp(Delta A), beta = alpha
  *           Delta / 2, gamma = Delta / 2, no previous input at t = 0).
+ *  [ssd]    "Mamba is attention all you really need, part 2", section
+ *           "The evolution", and "State Space Models and the Post-Transformer
+ *           Era", section "Mamba-2 and Structured State Space Duality":
+ *           Mamba-2 restricts A to one number times the identity; the result
+ *           is the same sequence map as attention under a 1-semiseparable
+ *           causal mask, computable by the linear scan or by the quadratic
+ *           matrix form.  Read here as: the channels of a head share Delta
+ *           and the scalar A (so a head's channels form the matrix that the
+ *           blockwise form multiplies), B and C are shared per group.
  *  The step-size nonlinearity Delta = softplus(delta + delta_bias) and the
  *  output gate y * silu(z) are not written out on the pages; this library
  *  uses the standard Mamba parameterisation for both.
@@ -324,6 +333,68 @@ int oracle_selective_scan_bwd_f64(
     }
   }
   free(pA); free(pD); free(pb);
+  return failed ? -1 : 0;
+}
+
+int oracle_ssd_scan_f64(int64_t batch, int64_t seqlen, int64_t nheads,
+                        int64_t headdim, int64_t ngroups, int64_t dstate,
+                        const double *x, const double *dt, const double *A,
+                        const double *B, const double *C, const double *D,
+                        const double *z, const double *dt_bias, int dt_softplus,
+                        const double *h0, double *y, double *last_state) {
+  if (batch < 0 || seqlen < 0 || nheads < 1 || headdim < 1 || ngroups < 1 ||
+      dstate < 1 || nheads % ngroups != 0)
+    return -1;
+  const int64_t heads_per_group = nheads / ngroups;
+  int failed = 0;
+  /* (b, h) pairs are independent; OpenMP only distributes them. */
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+  for (int64_t bh = 0; bh < batch * nheads; ++bh) {
+    const int64_t b = bh / nheads;
+    const int64_t h = bh % nheads;
+    const int64_t g = h / heads_per_group;
+    /* [ssd]: the state of one head is a headdim x dstate matrix. */
+    double *S = (double *)malloc(sizeof(double) * headdim * dstate);
+    if (!S) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+      failed = 1;
+      continue;
+    }
+    for (int64_t p = 0; p < headdim; ++p)
+      for (int64_t n = 0; n < dstate; ++n)
+        S[p * dstate + n] = h0 ? h0[((b * nheads + h) * headdim + p) * dstate + n] : 0.0;
+    const double bias = dt_bias ? dt_bias[h] : 0.0;
+    const double dskip = D ? D[h] : 0.0;
+    for (int64_t t = 0; t < seqlen; ++t) {
+      const double step = step_size(dt[(b * seqlen + t) * nheads + h], bias, dt_softplus);
+      /* [ssd] + [euler]: one fade exp(Delta A[h]) for every state entry. */
+      const double fade = exp(step * A[h]);
+      const double *Bt = B + ((b * seqlen + t) * ngroups + g) * dstate;
+      const double *Ct = C + ((b * seqlen + t) * ngroups + g) * dstate;
+      const int64_t row = ((b * seqlen + t) * nheads + h) * headdim;
+      for (int64_t p = 0; p < headdim; ++p) {
+        const double xp = x[row + p];
+        double acc = 0.0;
+        for (int64_t n = 0; n < dstate; ++n) {
+          /* [eq]: h_t = Abar h_{t-1} + Bbar x_t, per channel p. */
+          S[p * dstate + n] = fade * S[p * dstate + n] + step * Bt[n] * xp;
+          /* [eq]: read out with the state after the update. */
+          acc += Ct[n] * S[p * dstate + n];
+        }
+        double yp = acc + dskip * xp;
+        if (z) yp *= oracle_silu_f64(z[row + p]);
+        y[row + p] = yp;
+      }
+    }
+    if (last_state)
+      memcpy(last_state + (b * nheads + h) * headdim * dstate, S,
+             sizeof(double) * headdim * dstate);
+    free(S);
+  }
   return failed ? -1 : 0;
 }
 

@@ -73,7 +73,6 @@ int oracle_selective_state_update_f64(int64_t batch, int64_t dim,
                                       const double *z, const double *dt_bias,
                                       int dt_softplus, double *y);
 
-/* Number of OpenMP threads the scan uses (1 when built without OpenMP). */
 /* Gradient of the selective scan above (no packed sequences) for the loss
  * sum(dy * y) + sum(d_last * last_state): du, ddelta, dz (batch, dim,
  * seqlen), dA (dim, dstate), dB, dC (batch, dstate, seqlen), dD,
@@ -89,6 +88,28 @@ int oracle_selective_scan_bwd_f64(
     double *dA, double *dB, double *dC, double *dD, double *dz,
     double *ddelta_bias, double *dh0);
 
+/* Mamba-2 (SSD): the same recurrence with A restricted to a scalar times
+ * the identity per head, sequential over t.  headdim channels of a head
+ * share its step Delta_t and its scalar A[h]; ngroups groups of B, C are
+ * shared by nheads / ngroups consecutive heads each.  Token-major layouts:
+ *   x, z, y            (batch, seqlen, nheads, headdim)
+ *   dt                 (batch, seqlen, nheads)
+ *   A, D, dt_bias      (nheads)
+ *   B, C               (batch, seqlen, ngroups, dstate)
+ *   h0, last_state     (batch, nheads, headdim, dstate)
+ * For head h (group g = h / (nheads / ngroups)) and channel p:
+ *   Delta_t   = softplus(dt_t + dt_bias[h])  (or dt_t + dt_bias[h])
+ *   h_t[p,n]  = exp(Delta_t A[h]) h_{t-1}[p,n] + Delta_t B_t[g,n] x_t[p]
+ *   y_t[p]    = sum_n C_t[g,n] h_t[p,n] + D[h] x_t[p],  times silu(z_t[p])
+ * Returns 0, or -1 on a bad size. */
+int oracle_ssd_scan_f64(int64_t batch, int64_t seqlen, int64_t nheads,
+                        int64_t headdim, int64_t ngroups, int64_t dstate,
+                        const double *x, const double *dt, const double *A,
+                        const double *B, const double *C, const double *D,
+                        const double *z, const double *dt_bias, int dt_softplus,
+                        const double *h0, double *y, double *last_state);
+
+/* Number of OpenMP threads the scan uses (1 when built without OpenMP). */
 int oracle_num_threads(void);
 
 #ifdef __cplusplus

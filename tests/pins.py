@@ -545,6 +545,79 @@ def pin_trapezoid_second_order(lib):
     assert e2 < f2 / 10, ("trapezoid not more accurate than Euler", e2, f2)
 
 
+# --------------------------------------------------------------------------
+# Mamba-2 (SSD): A is one number times the identity per head.  The pages
+# ("State Space Models and the Post-Transformer Era", section "Mamba-2 and
+# Structured State Space Duality") state that this scan is the same map as
+# attention with a 1-semiseparable causal mask, computable either by the
+# linear recurrence or by a quadratic matrix form.  Two pins: the quadratic
+# form built with numpy matrix products, and the reduction to the S6 scan
+# (pinned above) with A[d, n] = A[h] for every channel d of head h.
+
+
+def _ssd_case(seed, softplus=True):
+    rng = _rng(seed)
+    bt, L, H, P, G, N = 2, 23, 4, 3, 2, 5
+    return dict(
+        x=rng.normal(size=(bt, L, H, P)), dt=rng.normal(size=(bt, L, H)),
+        A=-rng.uniform(0.1, 1.5, size=H), B=rng.normal(size=(bt, L, G, N)),
+        C=rng.normal(size=(bt, L, G, N)), D=rng.normal(size=H),
+        z=rng.normal(size=(bt, L, H, P)), dt_bias=rng.normal(size=H) * 0.5,
+        dt_softplus=softplus, h0=rng.normal(size=(bt, H, P, N)))
+
+
+def pin_ssd_quadratic_form(lib):
+    """y = (L o C B^T) (Delta x) plus the decayed initial state, per head:
+    L[t, s] = exp(sum_{s<k<=t} Delta_k A), zero above the diagonal."""
+    c = _ssd_case(31)
+    bt, L, H, P = c["x"].shape
+    G = c["B"].shape[2]
+    want = np.zeros_like(c["x"])
+    want_last = np.zeros_like(c["h0"])
+    for b in range(bt):
+        for h in range(H):
+            g = h // (H // G)
+            step = np.logaddexp(0.0, c["dt"][b, :, h] + c["dt_bias"][h])
+            cum = np.cumsum(step * c["A"][h])
+            mask = np.tril(np.exp(cum[:, None] - cum[None, :]))
+            Bg, Cg, X = c["B"][b, :, g], c["C"][b, :, g], c["x"][b, :, h]
+            M = (Cg @ Bg.T) * mask * step[None, :]
+            yb = M @ X + np.exp(cum)[:, None] * (Cg @ c["h0"][b, h].T) + c["D"][h] * X
+            want[b, :, h] = yb * c["z"][b, :, h] * scipy.special.expit(c["z"][b, :, h])
+            w = np.exp(cum[-1] - cum) * step
+            want_last[b, h] = np.exp(cum[-1]) * c["h0"][b, h] + (X * w[:, None]).T @ Bg
+    got, got_last = oracle.ssd_scan(c["x"], c["dt"], c["A"], c["B"], c["C"], D=c["D"],
+                                    z=c["z"], dt_bias=c["dt_bias"], h0=c["h0"],
+                                    return_last_state=True, lib=lib)
+    _close(got, want, 1e-9, 1e-12, "SSD quadratic form y")
+    _close(got_last, want_last, 1e-9, 1e-12, "SSD quadratic form last state")
+
+
+def pin_ssd_is_s6_with_scalar_A(lib):
+    for softplus in (True, False):
+        c = _ssd_case(32, softplus)
+        if not softplus:
+            c["dt"] = np.abs(c["dt"]) * 0.3 + 0.01
+        bt, L, H, P = c["x"].shape
+        G, N = c["B"].shape[2], c["B"].shape[3]
+        got, got_last = oracle.ssd_scan(c["x"], c["dt"], c["A"], c["B"], c["C"], D=c["D"],
+                                        z=c["z"], dt_bias=c["dt_bias"],
+                                        dt_softplus=softplus, h0=c["h0"],
+                                        return_last_state=True, lib=lib)
+        for h in range(H):
+            g = h // (H // G)
+            y6, l6 = oracle.selective_scan(
+                c["x"][:, :, h].transpose(0, 2, 1),
+                np.repeat(c["dt"][:, None, :, h], P, axis=1),
+                np.full((P, N), c["A"][h]),
+                c["B"][:, :, g].transpose(0, 2, 1), c["C"][:, :, g].transpose(0, 2, 1),
+                D=np.full(P, c["D"][h]), z=c["z"][:, :, h].transpose(0, 2, 1),
+                delta_bias=np.full(P, c["dt_bias"][h]), delta_softplus=softplus,
+                h0=c["h0"][:, h], return_last_state=True, lib=lib)
+            _close(got[:, :, h], y6.transpose(0, 2, 1), 1e-12, 1e-14, "SSD vs S6 y")
+            _close(got_last[:, h], l6, 1e-12, 1e-14, "SSD vs S6 last state")
+
+
 ALL_PINS = [
     pin_combine_worked_example,
     pin_scan_worked_example,
@@ -562,4 +635,6 @@ ALL_PINS = [
     pin_backward_finite_differences,
     pin_trapezoid_no_decay,
     pin_trapezoid_second_order,
+    pin_ssd_quadratic_form,
+    pin_ssd_is_s6_with_scalar_A,
 ]

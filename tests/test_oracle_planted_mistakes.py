@@ -51,6 +51,16 @@ MUTATIONS = {
     "trap_previous_input_not_decayed": ("0.5 * dt * (abar * wprev[n] + w)", "0.5 * dt * (wprev[n] + w)"),
     "trap_full_step_weights": ("0.5 * dt * (abar * wprev[n] + w)", "dt * (abar * wprev[n] + w)"),
     "trap_previous_input_not_kept": ("          wprev[n] = w;\n", "\n"),
+    "ssd_group_index": ("const int64_t g = h / heads_per_group;",
+                        "const int64_t g = h % ngroups;"),
+    "ssd_decay_sign": ("exp(step * A[h])", "exp(-step * A[h])"),
+    "ssd_readout_uses_B": ("acc += Ct[n] * S[p * dstate + n];",
+                           "acc += Bt[n] * S[p * dstate + n];"),
+    "ssd_skip_dropped": ("double yp = acc + dskip * xp;", "double yp = acc;"),
+    "ssd_input_without_step": ("step * Bt[n] * xp", "Bt[n] * xp"),
+    "ssd_h0_transposed": ("h0[((b * nheads + h) * headdim + p) * dstate + n]",
+                          "h0[((b * nheads + h) * dstate + n) * headdim + p]"),
+    "ssd_dt_of_head_zero": ("dt[(b * seqlen + t) * nheads + h]", "dt[(b * seqlen + t) * nheads]"),
     "update_step_uses_input_twice": (
         "step * B[b * dstate + n] * x[ch];", "step * B[b * dstate + n] * x[ch] * x[ch];"),
 }
