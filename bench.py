@@ -78,9 +78,13 @@ def parse_args(argv=None):
                          "bwd: start from checkpoints written by a forward scan")
     ap.add_argument("--trapezoid", action="store_true",
                     help="three-term trapezoidal update instead of the Euler one")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "decode"], default="fwd",
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "decode", "ssd"],
+                    default="fwd",
                     help="bwd times the backward scan (gradients of all inputs); "
-                         "decode times one-token state updates")
+                         "decode times one-token state updates; ssd times the "
+                         "Mamba-2 chunked scan on the tensor cores")
+    ap.add_argument("--ssd-workload", default="mamba2-2.7b-layer",
+                    choices=[w.name for w in workloads.SSD_WORKLOADS])
     ap.add_argument("--decode-batch", type=int, default=1024,
                     help="batch rows of one decode step (the workload's dim and dstate)")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -104,6 +108,18 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor peak for a kernel timed in a loop of launches: the
+    sustained cuBLAS figure of the measured peaks, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        return 1400.0, "fallback (sustained)"
 
 
 def kernel_source_hash() -> str:
@@ -667,6 +683,73 @@ def run_reference(args):
     }
 
 
+def run_ssd(args, rank, world, local_rank):
+    import selective_state_space_48_b200 as sss
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.SSD_BY_NAME[args.ssd_workload]
+    inp = workloads.make_ssd_inputs(w, seed=48100, device=dev)
+    ody = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+    y = torch.empty(w.batch, w.seqlen, w.nheads, w.headdim, dtype=ody, device=dev)
+
+    def step():
+        sss.ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                    z=inp["z"], dt_bias=inp["dt_bias"], dt_softplus=w.softplus, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    if sss.load_library().mss_ssd_status(None) != sss.MSS_OK:
+        raise RuntimeError("SSD kernel reported a timeout")
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    stream = torch.cuda.current_stream(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(world)
+    max_ms = reduce_max(t0.elapsed_time(t1), world)
+    nbytes = w.algorithmic_bytes(out_bytes(args.out_dtype))
+    flops = w.chunk_flops()
+    value = whole_job_gbs(nbytes, K, world, max_ms)
+    peak, src = measured_peaks()
+    tflops = flops * K / (max_ms * 1e-3) / 1e12
+    tpeak, tsrc = measured_tensor_peak()
+    line = {
+        "metric": "Mamba-2 SSD chunked scan HBM GB/s; tokens/s",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": max_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "pass": "ssd", "batch": w.batch,
+                   "seq_len": w.seqlen, "nheads": w.nheads, "headdim": w.headdim,
+                   "ngroups": w.ngroups, "dstate": w.dstate, "chunk": 128,
+                   "y_dtype": args.out_dtype,
+                   "l2": f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step)"},
+        "tokens_per_s": w.batch * w.seqlen * K * world / (max_ms * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
+                     "unit": "GB/s", "frac": value / world / peak,
+                     "peak_source": src, "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "tensor": {"achieved": tflops / world, "peak": tpeak,
+                                "unit": "TFLOP/s", "frac": tflops / world / tpeak,
+                                "peak_source": tsrc,
+                                "algorithmic_flops_per_launch": flops}},
+        "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
+        "kernel_source_hash": kernel_source_hash(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     try:
         faulthandler.enable()
@@ -690,6 +773,8 @@ def main(argv=None):
             run_bwd(args, rank, world, local_rank)
         elif args.pass_ == "decode":
             run_decode(args, rank, world, local_rank)
+        elif args.pass_ == "ssd":
+            run_ssd(args, rank, world, local_rank)
         else:
             line = run_ours(args, rank, world, local_rank)
             if rank == 0:

@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 6
+#define MSS_ABI_VERSION 7
 
 typedef enum {
   MSS_OK = 0,

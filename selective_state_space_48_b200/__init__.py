@@ -11,6 +11,7 @@ Functions mirror the C entry points:
   selective_state_update    -> selective_state_update(...)
   mss_scan_workspace_size   -> scan_workspace_size(...)
   mss_scan_status           -> scan_status(...)
+  mamba2_ssd_fwd            -> ssd_fwd(...)         (include/ssd.h)
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 6  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 7  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -36,7 +37,7 @@ MSS_F32 = 0
 MSS_BF16 = 1
 MSS_TESTFLAG_DROP_PUBLISH = 0x1
 
-# every symbol include/selective_scan.h declares
+# every symbol include/selective_scan.h and include/ssd.h declare
 EXPORTED_SYMBOLS = (
     "mss_scan_workspace_size",
     "mamba_selective_scan_fwd",
@@ -47,6 +48,8 @@ EXPORTED_SYMBOLS = (
     "mamba_selective_scan_bwd",
     "mss_status_string",
     "mss_abi_version",
+    "mamba2_ssd_fwd",
+    "mss_ssd_status",
 )
 
 
@@ -130,6 +133,20 @@ class ScanBwdArgs(ctypes.Structure):
     ]
 
 
+class SsdArgs(ctypes.Structure):
+    """Mirror of ``mss_ssd_args``."""
+    _fields_ = [(name, ctypes.c_int64) for name in (
+        "batch", "seqlen", "nheads", "headdim", "ngroups", "dstate")] + [
+        ("in_dtype", ctypes.c_int),
+        ("out_dtype", ctypes.c_int),
+    ] + [(name, ctypes.c_void_p) for name in (
+        "x", "dt", "A", "B", "C", "D", "z", "dt_bias")] + [
+        ("dt_softplus", ctypes.c_int),
+    ] + [(name, ctypes.c_void_p) for name in ("h0", "y", "last_state")] + [
+        ("spin_timeout_ns", ctypes.c_uint64),
+    ]
+
+
 class MssError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
@@ -167,6 +184,10 @@ def load_library():
             lib.mamba_selective_scan_bwd.restype = ctypes.c_int
             lib.mss_status_string.argtypes = [ctypes.c_int]
             lib.mss_status_string.restype = ctypes.c_char_p
+            lib.mamba2_ssd_fwd.argtypes = [P(SsdArgs), ctypes.c_void_p]
+            lib.mamba2_ssd_fwd.restype = ctypes.c_int
+            lib.mss_ssd_status.argtypes = [ctypes.c_void_p]
+            lib.mss_ssd_status.restype = ctypes.c_int
             lib.mss_abi_version.argtypes = []
             lib.mss_abi_version.restype = ctypes.c_int
             if lib.mss_abi_version() != ABI_VERSION:
@@ -371,6 +392,64 @@ def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
     return y
 
 
+def make_ssd_args(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
+                  h0=None, y=None, last_state=None, spin_timeout_ns=0) -> SsdArgs:
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    ind = x.dtype
+    _check_cuda("x", x, ind)
+    _check_cuda("dt", dt, ind, (batch, L, H))
+    _check_cuda("A", A, torch.float32, (H,))
+    _check_cuda("B", B, ind, (batch, L, G, N))
+    _check_cuda("C", C, ind, (batch, L, G, N))
+    _check_cuda("D", D, torch.float32, (H,))
+    _check_cuda("z", z, ind, (batch, L, H, P))
+    _check_cuda("dt_bias", dt_bias, torch.float32, (H,))
+    _check_cuda("h0", h0, torch.float32, (batch, H, P, N))
+    _check_cuda("last_state", last_state, torch.float32, (batch, H, P, N))
+    if y is not None:
+        _check_cuda("y", y, None, (batch, L, H, P))
+    a = SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.ngroups, a.dstate = batch, L, H, P, G, N
+    a.in_dtype = _dtype_code(ind)
+    a.out_dtype = _dtype_code(y.dtype) if y is not None else MSS_F32
+    a.x, a.dt, a.A, a.B, a.C = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C)
+    a.D, a.z, a.dt_bias = _ptr(D), _ptr(z), _ptr(dt_bias)
+    a.dt_softplus = 1 if dt_softplus else 0
+    a.h0, a.y, a.last_state = _ptr(h0), _ptr(y), _ptr(last_state)
+    a.spin_timeout_ns = int(spin_timeout_ns)
+    return a
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None,
+            return_last_state=False, out_dtype=torch.float32, y=None, last_state=None,
+            stream=None, check_status=False):
+    """Mamba-2 (SSD) chunked scan through ``mamba2_ssd_fwd``.
+
+    x, z: (batch, L, nheads, headdim); dt: (batch, L, nheads); B, C:
+    (batch, L, ngroups, dstate), all bfloat16; A, D, dt_bias: (nheads,)
+    float32; h0: (batch, nheads, headdim, dstate) float32.  Returns y
+    (batch, L, nheads, headdim) in ``out_dtype`` (and the final state when
+    ``return_last_state``).
+    """
+    batch, L, H, P = x.shape
+    N = B.shape[3]
+    if y is None:
+        y = torch.empty((batch, L, H, P), dtype=out_dtype, device=x.device)
+    if return_last_state and last_state is None:
+        last_state = torch.empty((batch, H, P, N), dtype=torch.float32, device=x.device)
+    args = make_ssd_args(x, dt, A, B, C, D, z, dt_bias, dt_softplus, h0, y, last_state)
+    lib = load_library()
+    rc = lib.mamba2_ssd_fwd(ctypes.byref(args), _stream_handle(stream))
+    if rc != MSS_OK:
+        raise MssError(rc, "mamba2_ssd_fwd")
+    if check_status:
+        rc = lib.mss_ssd_status(_stream_handle(stream))
+        if rc != MSS_OK:
+            raise MssError(rc, "mss_ssd_status")
+    return (y, last_state) if return_last_state else y
+
+
 def build(force: bool = False) -> str:
     return _build.build(force=force)
 
@@ -379,6 +458,7 @@ __all__ = [
     "selective_scan_fwd", "selective_state_update", "scan_workspace_size",
     "scan_status", "make_scan_args", "load_library", "status_string",
     "MssError", "ScanArgs", "UpdateArgs", "EXPORTED_SYMBOLS", "build",
+    "ssd_fwd", "make_ssd_args", "SsdArgs",
 ]
 
 

@@ -1,0 +1,722 @@
+// ssd_fwd.cu -- Mamba-2 (SSD) chunked scan on the sm_100a tensor cores.
+//
+// With A a scalar per head, the scan of one head over a chunk of Q = 128
+// steps is four matrix products ("State Space Models and the
+// Post-Transformer Era", section "Mamba-2 and Structured State Space
+// Duality"; "The State That Must Remember Everything", Part 4):
+//
+//   S  = C B^T                       M = t, N = s, K = n   (both K-major)
+//   Y  = S' X,   S'[t,s] = S[t,s] 2^(c_t - c_s) Delta_s  for s <= t, else 0
+//                                    M = t, N = p, K = s   (B operand MN-major)
+//   YO = C Hp,   Hp = the state before the chunk (bf16 copy)
+//                                    M = t, N = p, K = n   (B operand MN-major)
+//   H  = 2^(c_last) H + B^T X'',  X''[s,p] = X[s,p] Delta_s 2^(c_last - c_s)
+//                                    M = n, N = p, K = s   (both MN-major)
+//
+// with c_t the running sum of Delta A log2(e) inside the chunk, and the
+// output y_t = Y_t + 2^(c_t) YO_t + D x_t (times silu(z_t)).  One CTA owns
+// one (batch row, head) and walks its chunks in order, so the state H is
+// carried in tensor memory (fp32) across the whole sequence and never
+// touches HBM.  Warp roles: warp 0 issues the TMA loads of the C, B and X
+// tiles (two stages), warp 1 allocates tensor memory and issues the
+// tcgen05.mma products (one thread), warps 2-9 (256 threads, one tensor
+// memory lane quarter per pair of warps, which split the columns) compute
+// the step sizes and their running sum, build the operands S', X'' and Hp
+// in shared memory, rescale H, and write y.  The state products (YO and H)
+// are issued as soon as Hp and X'' are ready, so they run while the
+// epilogue builds the masked scores S'.
+//
+// Shared memory tiles are [128 rows][64 bf16] with the 128-byte swizzle that
+// the TMA writes and the tensor core reads: 16-byte chunk j of row r sits at
+// chunk position j ^ (r % 8).  Every wait on an mbarrier is bounded; a wait
+// that runs out records a timeout in the status word and the CTA finishes
+// its loop without waiting further, so no CTA can hang.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "device_math.cuh"
+#include "selective_scan.h"
+#include "ssd.h"
+
+namespace sss48 {
+namespace ssd {
+
+constexpr int Q = 128;   // chunk length
+constexpr int P = 64;    // headdim
+constexpr int NS = 128;  // dstate
+constexpr int kThreads = 320;  // 2 issue warps + 8 epilogue warps
+constexpr int kEpi = 256;
+constexpr int kEpiBarrier = 1;  // named barrier of the eight epilogue warps
+
+constexpr int kTile = Q * 64 * 2;      // one [128][64] bf16 tile
+constexpr int kStage = 5 * kTile;      // C (two n halves), B (two), X
+constexpr int oC = 0, oB = 2 * kTile, oX = 4 * kTile;
+constexpr int oSp = 2 * kStage;        // S' (two s halves)
+constexpr int oXpp = oSp + 2 * kTile;  // X''
+constexpr int oHp = oXpp + kTile;      // bf16 copy of the state, [n][p]
+constexpr int oCum = oHp + kTile;      // float c_s [Q]
+constexpr int oStep = oCum + Q * 4;    // float Delta_s [Q]
+constexpr int oColf = oStep + Q * 4;   // float column factors [Q]
+constexpr int oTot = oColf + Q * 4;    // float warp totals [4]
+constexpr int oBar = oTot + 16;        // 8 mbarriers
+constexpr int oTmemSlot = oBar + 8 * 8;
+constexpr int oAbort = oTmemSlot + 4;
+constexpr int kSmemUsed = oAbort + 12;
+constexpr int kSmemBytes = kSmemUsed + 1024;  // room to align the base
+static_assert(kSmemBytes <= 232448, "shared memory above the per-block limit");
+
+// tensor memory columns (fp32, lane = row)
+constexpr uint32_t kColS = 0, kColY = 128, kColYO = 192, kColH = 256;
+constexpr uint32_t kTmemCols = 512;
+
+// barrier indices: tiles landed / released (per stage), scores done,
+// state operands ready (Hp, X'', H rescaled), masked scores ready,
+// products done
+constexpr int kFull = 0, kEmpty = 2, kSFull = 4, kReadyState = 5, kReadyScores = 6,
+              kMmaDone = 7;
+
+struct Params {
+  int64_t batch, L, H, G;
+  const __nv_bfloat16 *dt;
+  const float *A, *D, *dt_bias;
+  int softplus;
+  const __nv_bfloat16 *z;
+  const float *h0;
+  void *y;
+  int y_bf16;
+  float *last;
+  unsigned *status;
+  uint64_t spin_ns;
+};
+
+struct Maps {
+  CUtensorMap x, B, C;
+};
+
+__device__ unsigned g_ssd_status;
+
+// ---------------------------------------------------------------- PTX
+
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, int c3, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// generic-proxy shared-memory writes -> visible to the tensor core
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_addr(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 in, fp32 accumulate)
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// arrive on `bar` once every tcgen05.mma issued so far by this thread is done
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+        "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+        "=r"(v[31])
+      : "r"(taddr));
+}
+
+// The loaded registers are valid only after tcgen05.wait::ld; threading
+// them through the wait keeps the compiler from using them earlier.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]),
+                 "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]),
+                 "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------ UMMA descriptors
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2),
+// version 1; addresses and offsets in 16-byte units.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFF) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32) | (uint64_t(1) << 46) |
+         (uint64_t(2) << 61);
+}
+
+// K-major operand stored as two [128 rows][64] tiles (K = 0..63, 64..127):
+// the 16-wide K slice kk starts 32 bytes into a row of tile kk / 4; rows
+// advance 128 bytes, 8-row groups 1024.
+__device__ __forceinline__ uint64_t desc_k(uint32_t tile0, int kk) {
+  return smem_desc(tile0 + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
+}
+
+// MN-major operand: rows are K, 64 MN values per 128-byte row, 16 K rows
+// per instruction (2048 bytes), a second 64-wide MN block `lbo` bytes on.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t tile, int kk, uint32_t lbo) {
+  return smem_desc(tile + kk * 2048, lbo, 1024);
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+         (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&u);
+  return __bfloat1622float2(v);
+}
+
+// byte offset of 16-byte chunk j of row r in a swizzled [128][64] tile
+__device__ __forceinline__ uint32_t swz(int r, int j) {
+  return static_cast<uint32_t>(r * 128 + ((j ^ (r & 7)) << 4));
+}
+
+// ------------------------------------------------------------- kernel
+
+struct Sync {
+  uint64_t *bar;
+  volatile int *abort;
+  unsigned *status;
+  uint64_t limit;
+  // bounded wait; after the first timeout in the CTA every wait returns at
+  // once (the results are then garbage, but nothing hangs)
+  __device__ void wait(int i, uint32_t parity) const {
+    if (*abort) return;
+    if (!mbar_wait_bounded(bar + i, parity, limit)) {
+      *abort = 1;
+      atomicOr(status, static_cast<unsigned>(MSS_ERR_TIMEOUT));
+    }
+  }
+  // bounded wait that is not skipped after a timeout: used before exit for
+  // copies and products still in flight
+  __device__ void drain(int i, uint32_t parity) const {
+    if (!mbar_wait_bounded(bar + i, parity, limit)) {
+      *abort = 1;
+      atomicOr(status, static_cast<unsigned>(MSS_ERR_TIMEOUT));
+    }
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    ssd_fwd_kernel(const __grid_constant__ Maps maps, const Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = blockIdx.x;
+  const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
+  const int g = static_cast<int>(h / (p.H / p.G));
+  const int nchunks = static_cast<int>((p.L + Q - 1) / Q);
+
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + oBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + oTmemSlot);
+  volatile int *abort = reinterpret_cast<volatile int *>(sm + oAbort);
+  float *cum_s = reinterpret_cast<float *>(sm + oCum);
+  float *step_s = reinterpret_cast<float *>(sm + oStep);
+  float *colf_s = reinterpret_cast<float *>(sm + oColf);
+  float *tot_s = reinterpret_cast<float *>(sm + oTot);
+  const Sync sy{bar, abort, p.status, p.spin_ns};
+
+  if (tid == 0) {
+    mbar_init(bar + kFull, 1);
+    mbar_init(bar + kFull + 1, 1);
+    mbar_init(bar + kEmpty, kEpi);
+    mbar_init(bar + kEmpty + 1, kEpi);
+    mbar_init(bar + kSFull, 1);
+    mbar_init(bar + kReadyState, kEpi);
+    mbar_init(bar + kReadyScores, kEpi);
+    mbar_init(bar + kMmaDone, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer
+    if (lane == 0) {
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c & 1;
+        if (c >= 2) sy.wait(kEmpty + st, ((c >> 1) - 1) & 1);
+        unsigned char *s = sm + st * kStage;
+        uint64_t *full = bar + kFull + st;
+        mbar_expect_tx(full, kStage);
+        const int t0 = c * Q;
+        tma_load_4d(s + oC, &maps.C, 0, g, t0, b, full);
+        tma_load_4d(s + oC + kTile, &maps.C, 64, g, t0, b, full);
+        tma_load_4d(s + oB, &maps.B, 0, g, t0, b, full);
+        tma_load_4d(s + oB + kTile, &maps.B, 64, g, t0, b, full);
+        tma_load_4d(s + oX, &maps.x, 0, h, t0, b, full);
+      }
+      // no copy may still be landing when the CTA exits
+      for (int c = nchunks > 2 ? nchunks - 2 : 0; c < nchunks; ++c)
+        sy.drain(kFull + (c & 1), (c >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- tensor-core issue
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idY = idesc_bf16(128, 64, 0, 1);
+      constexpr uint32_t idH = idesc_bf16(128, 64, 1, 1);
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c & 1;
+        const uint32_t s = sbase + st * kStage;
+        sy.wait(kFull + st, (c >> 1) & 1);
+        tc_fence_after();
+        if (!*abort) {
+          for (int kk = 0; kk < 8; ++kk)  // S = C B^T
+            umma_bf16(tmem + kColS, desc_k(s + oC, kk), desc_k(s + oB, kk), idS, kk > 0);
+        }
+        umma_commit(bar + kSFull);
+        sy.wait(kReadyState, c & 1);
+        tc_fence_after();
+        if (!*abort) {
+          for (int kk = 0; kk < 8; ++kk)  // YO = C Hp
+            umma_bf16(tmem + kColYO, desc_k(s + oC, kk), desc_mn(sbase + oHp, kk, kTile), idY,
+                      kk > 0);
+          for (int kk = 0; kk < 8; ++kk)  // H += B^T X''
+            umma_bf16(tmem + kColH, desc_mn(s + oB, kk, kTile), desc_mn(sbase + oXpp, kk, kTile),
+                      idH, 1);
+        }
+        sy.wait(kReadyScores, c & 1);
+        tc_fence_after();
+        if (!*abort) {
+          for (int kk = 0; kk < 8; ++kk)  // Y = S' X
+            umma_bf16(tmem + kColY, desc_k(sbase + oSp, kk), desc_mn(s + oX, kk, kTile), idY,
+                      kk > 0);
+        }
+        umma_commit(bar + kMmaDone);
+      }
+      // every product done before the tensor memory is freed
+      if (nchunks > 0) sy.drain(kMmaDone, (nchunks - 1) & 1);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------- epilogue
+    // Two warps per tensor-memory lane quarter: e = 0 / 1 split the columns.
+    const int q = warp & 3;
+    const int e = (warp - 2) >> 2;
+    const int r = 32 * q + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    const float A2 = p.A[h] * kLog2e;
+    const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
+    const float Dh = p.D ? p.D[h] : 0.0f;
+    const int64_t H = p.H;
+    const __nv_bfloat16 *dtp = p.dt + static_cast<int64_t>(b) * p.L * H + h;
+
+    // the initial state into H (row n = r, columns 32e .. 32e + 31)
+    {
+      const float *h0 = p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * P * NS : nullptr;
+      uint32_t v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        v[j] = __float_as_uint(h0 ? h0[(e * 32 + j) * NS + r] : 0.0f);
+      tmem_st32(tl + kColH + 32 * e, v);
+      tmem_wait_st();
+    }
+
+    // the raw step of row r of the next chunk, loaded one chunk ahead
+    float dt_next = 0.0f;
+    if (e == 0 && r < p.L) dt_next = __bfloat162float(dtp[static_cast<int64_t>(r) * H]);
+
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c & 1;
+      const unsigned char *s = sm + st * kStage;
+      const int64_t t = static_cast<int64_t>(c) * Q + r;
+
+      // step sizes, their running sum c_t (log2 units) and the column
+      // factors 2^(c_end - c_s) Delta_s, c_end the last step of s's
+      // 32-step block; computed by the e = 0 warps
+      float cw = 0.0f, step = 0.0f;
+      if (e == 0) {
+        if (t < p.L) {
+          const float v = dt_next + bias;
+          step = p.softplus ? softplus_f(v) : v;
+        }
+        if (t + Q < p.L) dt_next = __bfloat162float(dtp[(t + Q) * H]);
+        cw = step * A2;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, cw, o);
+          if (lane >= o) cw += u;
+        }
+        if (lane == 31) tot_s[q] = cw;
+      }
+      bar_sync(kEpiBarrier, kEpi);
+      float base = 0.0f;
+      for (int j = 0; j < q; ++j) base += tot_s[j];
+      if (e == 0) {
+        const float cum = base + cw;
+        const float cend = base + __shfl_sync(0xffffffffu, cw, 31);
+        cum_s[r] = cum;
+        step_s[r] = step;
+        colf_s[r] = ex2_mufu(cend - cum) * step;
+      }
+      bar_sync(kEpiBarrier, kEpi);
+      const float cum = cum_s[r];
+      const float cl = cum_s[Q - 1];
+
+      sy.wait(kFull + st, (c >> 1) & 1);
+
+      // Hp row n = r (columns of half e): bf16 copy of the state before
+      // this chunk; then the state decays over the chunk: H *= 2^(c_last)
+      {
+        const float gam = ex2_mufu(cl);
+        uint32_t v[32];
+        tmem_ld32(tl + kColH + 32 * e, v);
+        tmem_wait_ld(v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 o;
+          o.x = pack_bf16(__uint_as_float(v[8 * k + 0]), __uint_as_float(v[8 * k + 1]));
+          o.y = pack_bf16(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3]));
+          o.z = pack_bf16(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5]));
+          o.w = pack_bf16(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7]));
+          *reinterpret_cast<uint4 *>(sm + oHp + swz(r, e * 4 + k)) = o;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam);
+        tmem_st32(tl + kColH + 32 * e, v);
+        tmem_wait_st();
+      }
+      // X'' row s = r, four of its eight 16-byte chunks (the XOR with the
+      // row keeps the eight rows of a shared-memory phase on distinct banks)
+      {
+        const float w = step_s[r] * ex2_mufu(cl - cum);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t off = static_cast<uint32_t>(r * 128 + (((e * 4 + k) ^ (r & 7)) << 4));
+          const uint4 xv = *reinterpret_cast<const uint4 *>(s + oX + off);
+          const float2 a0 = unpack_bf16(xv.x), a1 = unpack_bf16(xv.y);
+          const float2 a2 = unpack_bf16(xv.z), a3 = unpack_bf16(xv.w);
+          *reinterpret_cast<uint4 *>(sm + oXpp + off) =
+              make_uint4(pack_bf16(a0.x * w, a0.y * w), pack_bf16(a1.x * w, a1.y * w),
+                         pack_bf16(a2.x * w, a2.y * w), pack_bf16(a3.x * w, a3.y * w));
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar + kReadyState);
+
+      // S' row t, blocks gb = e and e + 2 of 32 columns: below the diagonal
+      // S 2^(c_t - c_end(gb)) colf[s] (both factors <= 1), on the diagonal
+      // S 2^(c_t - c_s) Delta_s for s <= t, above it zero
+      sy.wait(kSFull, c & 1);
+      tc_fence_after();
+#pragma unroll 1
+      for (int gb = e; gb < 4; gb += 2) {
+        uint32_t pk[16];
+        if (gb < q) {
+          uint32_t v[32];
+          tmem_ld32(tl + kColS + 32 * gb, v);
+          const float rf = ex2_mufu(cum - cum_s[32 * gb + 31]);
+          tmem_wait_ld(v);
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int s0 = 32 * gb + j;
+            pk[j >> 1] = pack_bf16(__uint_as_float(v[j]) * rf * colf_s[s0],
+                                   __uint_as_float(v[j + 1]) * rf * colf_s[s0 + 1]);
+          }
+        } else if (gb == q) {
+          uint32_t v[32];
+          tmem_ld32(tl + kColS + 32 * gb, v);
+          tmem_wait_ld(v);
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int s0 = 32 * gb + j;
+            const float f0 = j <= lane ? __uint_as_float(v[j]) *
+                                             ex2_mufu(cum - cum_s[s0]) * step_s[s0]
+                                       : 0.0f;
+            const float f1 = j + 1 <= lane ? __uint_as_float(v[j + 1]) *
+                                                 ex2_mufu(cum - cum_s[s0 + 1]) * step_s[s0 + 1]
+                                           : 0.0f;
+            pk[j >> 1] = pack_bf16(f0, f1);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = 0u;
+        }
+        unsigned char *dst = sm + oSp + (gb >> 1) * kTile;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4 *>(dst + swz(r, (gb & 1) * 4 + k)) =
+              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar + kReadyScores);
+
+      // y row t, columns of half e: Y + 2^(c_t) YO + D x, gated
+      sy.wait(kMmaDone, c & 1);
+      tc_fence_after();
+      {
+        const float eo = ex2_mufu(cum);
+        const int64_t row = ((static_cast<int64_t>(b) * p.L + t) * H + h) * P + 32 * e;
+        uint32_t yv[32], ov[32];
+        tmem_ld32(tl + kColY + 32 * e, yv);
+        tmem_ld32(tl + kColYO + 32 * e, ov);
+        tmem_wait_ld(yv);
+        tmem_wait_ld(ov);
+        float out[32];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 xv = *reinterpret_cast<const uint4 *>(s + oX + swz(r, e * 4 + k));
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 xf = unpack_bf16(xw[i]);
+            const int j = 8 * k + 2 * i;
+            out[j] = fmaf(eo, __uint_as_float(ov[j]), __uint_as_float(yv[j])) + Dh * xf.x;
+            out[j + 1] =
+                fmaf(eo, __uint_as_float(ov[j + 1]), __uint_as_float(yv[j + 1])) + Dh * xf.y;
+          }
+        }
+        if (t < p.L) {
+          if (p.z) {
+            const uint4 *zr = reinterpret_cast<const uint4 *>(p.z + row);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint4 zv = zr[k];
+              const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 zf = unpack_bf16(zw[i]);
+                out[8 * k + 2 * i] *= silu_f(zf.x);
+                out[8 * k + 2 * i + 1] *= silu_f(zf.y);
+              }
+            }
+          }
+          if (p.y_bf16) {
+            uint4 *yr = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.y) + row);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              yr[k] = make_uint4(pack_bf16(out[8 * k], out[8 * k + 1]),
+                                 pack_bf16(out[8 * k + 2], out[8 * k + 3]),
+                                 pack_bf16(out[8 * k + 4], out[8 * k + 5]),
+                                 pack_bf16(out[8 * k + 6], out[8 * k + 7]));
+          } else {
+            float4 *yr = reinterpret_cast<float4 *>(static_cast<float *>(p.y) + row);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              yr[k] = make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar + kEmpty + st);
+    }
+
+    // the state after the last chunk (columns of half e)
+    if (p.last) {
+      float *lr = p.last + (static_cast<int64_t>(b) * H + h) * P * NS;
+      uint32_t v[32];
+      tmem_ld32(tl + kColH + 32 * e, v);
+      tmem_wait_ld(v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) lr[(e * 32 + j) * NS + r] = __uint_as_float(v[j]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor (d0 innermost, ..., d3), dense; box {64, 1, Q, 1}, 128-byte
+// swizzle, rows past the end of the sequence read as zeros
+bool encode_4d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t d3) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(Q), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool al16(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
+bool al4(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 3) == 0; }
+
+mss_status check(const mss_ssd_args *a) {
+  if (!a) return MSS_ERR_INVALID_ARG;
+  if (a->batch < 1 || a->seqlen < 1 || a->nheads < 1 || a->headdim < 1 || a->ngroups < 1 ||
+      a->dstate < 1 || a->nheads % a->ngroups != 0)
+    return MSS_ERR_INVALID_ARG;
+  if ((a->in_dtype != MSS_F32 && a->in_dtype != MSS_BF16) ||
+      (a->out_dtype != MSS_F32 && a->out_dtype != MSS_BF16))
+    return MSS_ERR_INVALID_ARG;
+  if (!a->x || !a->dt || !a->A || !a->B || !a->C || !a->y) return MSS_ERR_INVALID_ARG;
+  if (a->in_dtype != MSS_BF16 || a->headdim != P || a->dstate != NS)
+    return MSS_ERR_UNSUPPORTED;
+  if (!al16(a->x) || !al16(a->B) || !al16(a->C) || !al16(a->y) || (a->z && !al16(a->z)))
+    return MSS_ERR_INVALID_ARG;
+  if (!al4(a->A) || (a->D && !al4(a->D)) || (a->dt_bias && !al4(a->dt_bias)) ||
+      (a->h0 && !al4(a->h0)) || (a->last_state && !al4(a->last_state)) ||
+      (reinterpret_cast<uintptr_t>(a->dt) & 1))
+    return MSS_ERR_INVALID_ARG;
+  // grid of batch * nheads CTAs; TMA coordinates are 32-bit
+  if (a->batch * a->nheads >= (int64_t(1) << 31) || a->seqlen >= (int64_t(1) << 31) - Q)
+    return MSS_ERR_UNSUPPORTED;
+  return MSS_OK;
+}
+
+}  // namespace ssd
+}  // namespace sss48
+
+using namespace sss48;
+
+extern "C" mss_status mamba2_ssd_fwd(const mss_ssd_args *a, void *stream) {
+  const mss_status st = ssd::check(a);
+  if (st != MSS_OK) return st;
+  ssd::Maps maps;
+  const uint64_t L = static_cast<uint64_t>(a->seqlen), H = static_cast<uint64_t>(a->nheads),
+                 G = static_cast<uint64_t>(a->ngroups), Bt = static_cast<uint64_t>(a->batch);
+  if (!ssd::encode_4d(&maps.x, a->x, ssd::P, H, L, Bt) ||
+      !ssd::encode_4d(&maps.B, a->B, ssd::NS, G, L, Bt) ||
+      !ssd::encode_4d(&maps.C, a->C, ssd::NS, G, L, Bt))
+    return MSS_ERR_CUDA;
+  unsigned *status = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), ssd::g_ssd_status) !=
+      cudaSuccess)
+    return MSS_ERR_CUDA;
+  ssd::Params p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.H = a->nheads;
+  p.G = a->ngroups;
+  p.dt = static_cast<const __nv_bfloat16 *>(a->dt);
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.softplus = a->dt_softplus ? 1 : 0;
+  p.z = static_cast<const __nv_bfloat16 *>(a->z);
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.y_bf16 = a->out_dtype == MSS_BF16;
+  p.last = a->last_state;
+  p.status = status;
+  p.spin_ns = a->spin_timeout_ns ? a->spin_timeout_ns : 2000000000ull;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(ssd::ssd_fwd_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, ssd::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return MSS_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(a->batch * a->nheads);
+  ssd::ssd_fwd_kernel<<<grid, ssd::kThreads, ssd::kSmemBytes,
+                        static_cast<cudaStream_t>(stream)>>>(maps, p);
+  return cudaGetLastError() == cudaSuccess ? MSS_OK : MSS_ERR_CUDA;
+}
+
+extern "C" mss_status mss_ssd_status(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, ssd::g_ssd_status, sizeof(v)) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  const unsigned zero = 0;
+  if (v && cudaMemcpyToSymbol(ssd::g_ssd_status, &zero, sizeof(zero)) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  return v ? MSS_ERR_TIMEOUT : MSS_OK;
+}

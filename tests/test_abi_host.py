@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 6
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 7
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
@@ -67,7 +67,8 @@ def test_struct_layout_matches_c():
     fields_scan = [f[0] for f in sss.ScanArgs._fields_]
     fields_upd = [f[0] for f in sss.UpdateArgs._fields_]
     fields_bwd = [f[0] for f in sss.ScanBwdArgs._fields_]
-    src = ['#include <stdio.h>', '#include <stddef.h>', '#include "selective_scan.h"',
+    fields_ssd = [f[0] for f in sss.SsdArgs._fields_]
+    src = ['#include <stdio.h>', '#include <stddef.h>', '#include "ssd.h"',
            'int main(void) {',
            'printf("%zu\\n", sizeof(mss_scan_args));']
     src += [f'printf("%zu\\n", offsetof(mss_scan_args, {f}));' for f in fields_scan]
@@ -75,6 +76,8 @@ def test_struct_layout_matches_c():
     src += [f'printf("%zu\\n", offsetof(mss_update_args, {f}));' for f in fields_upd]
     src += ['printf("%zu\\n", sizeof(mss_scan_bwd_args));']
     src += [f'printf("%zu\\n", offsetof(mss_scan_bwd_args, {f}));' for f in fields_bwd]
+    src += ['printf("%zu\\n", sizeof(mss_ssd_args));']
+    src += [f'printf("%zu\\n", offsetof(mss_ssd_args, {f}));' for f in fields_ssd]
     src += ['return 0; }']
     with tempfile.TemporaryDirectory() as tmp:
         c = os.path.join(tmp, "layout.c")
@@ -86,6 +89,7 @@ def test_struct_layout_matches_c():
     want = [ctypes.sizeof(sss.ScanArgs)] + [getattr(sss.ScanArgs, f).offset for f in fields_scan]
     want += [ctypes.sizeof(sss.UpdateArgs)] + [getattr(sss.UpdateArgs, f).offset for f in fields_upd]
     want += [ctypes.sizeof(sss.ScanBwdArgs)] + [getattr(sss.ScanBwdArgs, f).offset for f in fields_bwd]
+    want += [ctypes.sizeof(sss.SsdArgs)] + [getattr(sss.SsdArgs, f).offset for f in fields_ssd]
     assert vals == want
 
 
@@ -246,3 +250,34 @@ def test_checkpoint_buffer_matches_the_workspace_size():
         assert lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == sss.MSS_OK
         buf = sss.scan_checkpoints(2, 40, N, 1000, "cpu")
         assert buf.numel() * 4 == n.value, N
+
+
+def _ssd_args(**kw):
+    a = sss.SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.ngroups, a.dstate = 2, 1000, 8, 64, 2, 128
+    a.in_dtype, a.out_dtype = sss.MSS_BF16, sss.MSS_F32
+    fake = 0x10000
+    a.x = a.dt = a.A = a.B = a.C = a.y = fake
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(headdim=32), sss.MSS_ERR_UNSUPPORTED),
+    (dict(dstate=64), sss.MSS_ERR_UNSUPPORTED),
+    (dict(in_dtype=sss.MSS_F32), sss.MSS_ERR_UNSUPPORTED),
+    (dict(ngroups=3), sss.MSS_ERR_INVALID_ARG),
+    (dict(seqlen=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(batch=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(x=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(y=0), sss.MSS_ERR_INVALID_ARG),
+    (dict(B=0x10008), sss.MSS_ERR_INVALID_ARG),
+    (dict(z=0x10004), sss.MSS_ERR_INVALID_ARG),
+    (dict(dt=0x10001), sss.MSS_ERR_INVALID_ARG),
+    (dict(h0=0x10002), sss.MSS_ERR_INVALID_ARG),
+    (dict(in_dtype=7), sss.MSS_ERR_INVALID_ARG),
+], ids=lambda v: str(v))
+def test_ssd_argument_checks(lib, kw, code):
+    """Rejected before anything is enqueued (no GPU is touched)."""
+    assert lib.mamba2_ssd_fwd(ctypes.byref(_ssd_args(**kw)), None) == code

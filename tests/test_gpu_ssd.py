@@ -1,0 +1,128 @@
+"""Mamba-2 (SSD) chunked scan on the tensor cores against the fp64 oracle
+(needs a GPU).
+
+The oracle is the sequential recurrence with a scalar A per head (pinned on
+the CPU by the quadratic masked form and by its reduction to the S6 scan).
+The CUDA path evaluates the same map by 128-step chunks of bf16 matrix
+products with fp32 accumulation, so its tolerance comes from bf16
+rounding, not fp32: the decayed scores S', the weighted inputs X'' and
+the carried state h_prev each enter one product rounded to bf16 (unit
+roundoff u = 2^-8).  Each output sums such rounded terms with independent
+rounding errors, so |y_gpu - y| stays within a small multiple of u times
+the size of y; the bound used is 2.5 u = 9.8e-3 of max |y| (and of max
+|h| for the final state), with another 2^-8 when y itself is stored in
+bf16.  Cases: chunks with a ragged tail, a single short chunk, two groups
+of B and C, no optional inputs with softplus off, an initial state, bf16
+output, a long carry chain, and outputs sampled from the full 2.7B-layer
+shape.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_48_b200 as sss
+import workloads
+from scan_checks import norm_err
+
+pytestmark = pytest.mark.gpu
+
+U_BF16 = 2.0 ** -8
+TOL = 2.5 * U_BF16
+
+
+def _oracle(inp, softplus=True, heads=None, batch=None):
+    h = workloads.to_numpy_f64(inp)
+    x, dt, A, z, h0 = h["x"], h["dt"], h["A"], h["z"], h["h0"]
+    B, C, D, bias = h["B"], h["C"], h["D"], h["dt_bias"]
+    if batch is not None:
+        sel = slice(batch, batch + 1)
+        x, dt, B, C = x[sel], dt[sel], B[sel], C[sel]
+        z = None if z is None else z[sel]
+        h0 = None if h0 is None else h0[sel]
+    if heads is not None:  # a subset of heads of a one-group input
+        assert B.shape[2] == 1
+        x, dt, A = x[:, :, heads], dt[:, :, heads], A[heads]
+        z = None if z is None else z[:, :, heads]
+        D = None if D is None else D[heads]
+        bias = None if bias is None else bias[heads]
+        h0 = None if h0 is None else h0[:, heads]
+    return oracle.ssd_scan(x, dt, A, B, C, D=D, z=z, dt_bias=bias, dt_softplus=softplus,
+                           h0=h0, return_last_state=True)
+
+
+def _run(inp, softplus=True, out_dtype=torch.float32):
+    return sss.ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                       z=inp["z"], dt_bias=inp["dt_bias"], dt_softplus=softplus,
+                       h0=inp["h0"], return_last_state=True, out_dtype=out_dtype,
+                       check_status=True)
+
+
+CASES = [
+    # name, batch, L, heads, groups, z, h0
+    ("ragged-3-chunks-2-groups", 2, 300, 4, 2, True, True),
+    ("one-short-chunk", 1, 50, 2, 1, True, False),
+    ("two-full-chunks", 1, 256, 3, 1, False, True),
+    ("long-carry", 1, 2000, 2, 1, True, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_ssd_matches_the_oracle(case):
+    name, batch, L, H, G, has_z, h0 = case
+    w = workloads.SsdWorkload(name, batch, L, H, ngroups=G, has_z=has_z)
+    inp = workloads.make_ssd_inputs(w, seed=5700 + L, device="cuda", h0=h0)
+    y, last = _run(inp)
+    torch.cuda.synchronize()
+    y_ref, last_ref = _oracle(inp)
+    assert norm_err(y.cpu().numpy(), y_ref) <= TOL, name
+    assert norm_err(last.cpu().numpy(), last_ref) <= TOL, name
+
+
+def test_ssd_without_optional_inputs_and_softplus_off():
+    w = workloads.SsdWorkload("plain", 1, 200, 2, has_z=False, has_D=False,
+                              has_dt_bias=False, softplus=False)
+    inp = workloads.make_ssd_inputs(w, seed=5750, device="cuda")
+    # positive steps without softplus
+    inp["dt"] = (inp["dt"].float().abs() * 0.05 + 0.001).to(torch.bfloat16)
+    y, last = _run(inp, softplus=False)
+    torch.cuda.synchronize()
+    y_ref, last_ref = _oracle(inp, softplus=False)
+    assert norm_err(y.cpu().numpy(), y_ref) <= TOL
+    assert norm_err(last.cpu().numpy(), last_ref) <= TOL
+
+
+def test_ssd_bf16_output():
+    w = workloads.SsdWorkload("bf16-out", 1, 300, 2, has_z=True)
+    inp = workloads.make_ssd_inputs(w, seed=5751, device="cuda", h0=True)
+    y, _ = _run(inp, out_dtype=torch.bfloat16)
+    yf, _ = _run(inp)
+    torch.cuda.synchronize()
+    assert y.dtype == torch.bfloat16
+    assert torch.equal(y, yf.to(torch.bfloat16))
+    y_ref, _ = _oracle(inp)
+    assert norm_err(y.float().cpu().numpy(), y_ref) <= TOL + U_BF16
+
+
+def test_ssd_full_layer_sampled():
+    """The 2.7B-layer shape in the launch configuration the bench times;
+    three heads of one batch row checked against the oracle."""
+    w = workloads.SSD_BY_NAME["mamba2-2.7b-layer"]
+    inp = workloads.make_ssd_inputs(w, seed=5752, device="cuda", h0=True)
+    y, last = _run(inp)
+    torch.cuda.synchronize()
+    b, heads = 5, [0, 41, w.nheads - 1]
+    y_ref, last_ref = _oracle(inp, heads=heads, batch=b)
+    got = y[b:b + 1, :, heads].cpu().numpy()
+    assert norm_err(got, y_ref) <= TOL
+    assert norm_err(last[b:b + 1, heads].cpu().numpy(), last_ref) <= TOL
+    assert torch.isfinite(y).all()
+
+
+def test_ssd_is_deterministic():
+    w = workloads.SsdWorkload("det", 2, 700, 3, has_z=True)
+    inp = workloads.make_ssd_inputs(w, seed=5753, device="cuda", h0=True)
+    y1, l1 = _run(inp)
+    y2, l2 = _run(inp)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(l1, l2)

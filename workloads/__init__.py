@@ -142,5 +142,84 @@ def describe(w: ScanWorkload) -> str:
             f"{w.in_dtype}{' +z' if w.has_z else ''}")
 
 
+# --------------------------------------------------------------------------
+# Mamba-2 (SSD) inputs: A is one scalar per head.  Shapes follow a Mamba-2
+# layer: heads of 64 channels, 128 states (eight times Mamba-1's 16), one
+# group of B, C shared by all heads.  Draw order: x, dt, B, C, z, A, D,
+# dt_bias, h0.  A[h] = -U[1, 16]; dt_bias as delta_bias above; x, dt, B,
+# C, z ~ N(0, 1) rounded to bf16; D ~ N(0, 1); h0 ~ N(0, 1) / 4.
+
+
+@dataclasses.dataclass(frozen=True)
+class SsdWorkload:
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int = 64
+    ngroups: int = 1
+    dstate: int = 128
+    has_z: bool = False
+    has_D: bool = True
+    has_dt_bias: bool = True
+    softplus: bool = True
+
+    def algorithmic_bytes(self, out_bytes: int = 4) -> int:
+        """x (and z) read and y written once per (b, t, h, p); dt once per
+        (b, t, h); B and C once per (b, t, g, n); A, D, dt_bias per head."""
+        btp = self.batch * self.seqlen * self.nheads * self.headdim
+        row = btp * (2 * (1 + int(self.has_z)) + out_bytes)
+        dt = self.batch * self.seqlen * self.nheads * 2
+        bc = 2 * self.batch * self.seqlen * self.ngroups * self.dstate * 2
+        return row + dt + bc + self.nheads * 4 * (1 + int(self.has_D) + int(self.has_dt_bias))
+
+    def chunk_flops(self, chunk: int = 128) -> int:
+        """Matrix-product FLOPs of the chunked form per full pass: per chunk
+        and group the scores C B^T (2 Q^2 N, shared by the group's heads);
+        per chunk and head the masked product with X (2 Q^2 P), the
+        carried-state readout C h (2 Q N P) and the chunk's state update
+        B^T X (2 Q N P)."""
+        Q, N, P = chunk, self.dstate, self.headdim
+        nch = -(-self.seqlen // chunk)
+        scores = self.batch * self.ngroups * nch * 2 * Q * Q * N
+        return scores + self.batch * self.nheads * nch * (2 * Q * Q * P + 4 * Q * N * P)
+
+
+SSD_WORKLOADS = [
+    SsdWorkload("ssd-small", 2, 300, 4, ngroups=2, has_z=True),
+    SsdWorkload("mamba2-2.7b-layer", 8, 2048, 80),
+]
+SSD_BY_NAME = {w.name: w for w in SSD_WORKLOADS}
+
+
+def make_ssd_inputs(w: SsdWorkload, seed: int, device: str | torch.device = "cpu",
+                    h0: bool = False) -> dict:
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    f32, bf = torch.float32, torch.bfloat16
+
+    def normal(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=f32)
+
+    bl = (w.batch, w.seqlen)
+    x = normal(*bl, w.nheads, w.headdim).to(bf)
+    dt = normal(*bl, w.nheads).to(bf)
+    B = normal(*bl, w.ngroups, w.dstate).to(bf)
+    C = normal(*bl, w.ngroups, w.dstate).to(bf)
+    z = normal(*bl, w.nheads, w.headdim).to(bf) if w.has_z else None
+    A = -(1.0 + 15.0 * torch.rand(w.nheads, generator=g, device=dev, dtype=f32))
+    D = normal(w.nheads) if w.has_D else None
+    if w.has_dt_bias:
+        v = torch.rand(w.nheads, generator=g, device=dev, dtype=torch.float64)
+        v = 1e-3 + (1e-1 - 1e-3) * v
+        dt_bias = torch.log(torch.expm1(v)).to(f32)
+    else:
+        dt_bias = None
+    hz = normal(w.batch, w.nheads, w.headdim, w.dstate) * 0.25 if h0 else None
+    return dict(x=x, dt=dt, A=A, B=B, C=C, D=D, z=z, dt_bias=dt_bias, h0=hz)
+
+
 __all__ = ["ScanWorkload", "WORKLOADS", "BY_NAME", "custom", "make_inputs",
-           "to_numpy_f64", "seed_of", "describe"]
+           "to_numpy_f64", "seed_of", "describe", "SsdWorkload", "SSD_WORKLOADS",
+           "SSD_BY_NAME", "make_ssd_inputs"]
