@@ -37,6 +37,9 @@
  *   B, C             (batch, seqlen, ngroups, dstate)   in_dtype
  *   A, D, dt_bias    (nheads)                           fp32 (D, dt_bias optional)
  *   h0, last_state   (batch, nheads, headdim, dstate)   fp32, optional
+ * A[h] is expected to be <= 0 (a decaying state, as in Mamba-2): the
+ * kernel factors the decay between two steps into per-row and per-column
+ * factors that stay below 1 only for A <= 0.
  * Supported here: in_dtype MSS_BF16, headdim 64, dstate 128 (other valid
  * sizes return MSS_ERR_UNSUPPORTED).  x, B, C, z and y must be 16-byte
  * aligned; every other pointer 4-byte aligned.  Outputs must not overlap

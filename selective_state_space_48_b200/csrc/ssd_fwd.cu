@@ -53,6 +53,7 @@ constexpr int NS = 128;  // dstate
 constexpr int kThreads = 320;  // 2 issue warps + 8 epilogue warps
 constexpr int kEpi = 256;
 constexpr int kEpiBarrier = 1;  // named barrier of the eight epilogue warps
+constexpr int kHalfBarrier = 2; // + e: named barrier of the four warps of half e
 
 constexpr int kTile = Q * 64 * 2;      // one [128][64] bf16 tile
 constexpr int kStage = 5 * kTile;      // C (two n halves), B (two), X
@@ -64,8 +65,8 @@ constexpr int oCum = oHp + kTile;      // float c_s [Q]
 constexpr int oStep = oCum + Q * 4;    // float Delta_s [Q]
 constexpr int oColf = oStep + Q * 4;   // float column factors [Q]
 constexpr int oTot = oColf + Q * 4;    // float warp totals [4]
-constexpr int oBar = oTot + 16;        // 8 mbarriers
-constexpr int oTmemSlot = oBar + 8 * 8;
+constexpr int oBar = oTot + 16;        // 9 mbarriers
+constexpr int oTmemSlot = oBar + 10 * 8;
 constexpr int oAbort = oTmemSlot + 4;
 constexpr int kSmemUsed = oAbort + 12;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // room to align the base
@@ -75,11 +76,11 @@ static_assert(kSmemBytes <= 232448, "shared memory above the per-block limit");
 constexpr uint32_t kColS = 0, kColY = 128, kColYO = 192, kColH = 256;
 constexpr uint32_t kTmemCols = 512;
 
-// barrier indices: tiles landed / released (per stage), scores done,
-// state operands ready (Hp, X'', H rescaled), masked scores ready,
-// products done
-constexpr int kFull = 0, kEmpty = 2, kSFull = 4, kReadyState = 5, kReadyScores = 6,
-              kMmaDone = 7;
+// barrier indices: tiles landed / released (per stage), scores S done,
+// masked scores S' ready, state operands ready (Hp, X'', H rescaled), the
+// output products Y and YO done, the state update done
+constexpr int kFull = 0, kEmpty = 2, kSFull = 4, kReadyScores = 5, kReadyState = 6,
+              kDoneY = 7, kDoneH = 8;
 
 struct Params {
   int64_t batch, L, H, G;
@@ -96,7 +97,7 @@ struct Params {
 };
 
 struct Maps {
-  CUtensorMap x, B, C;
+  CUtensorMap x, B, C, y;
 };
 
 __device__ unsigned g_ssd_status;
@@ -111,6 +112,26 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
       "r"(smem_addr(bar))
       : "memory");
+}
+
+// 4-D tiled TMA store of a shared-memory box (rows past the tensor's end
+// are not written), tracked by this thread's bulk group
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0,
+                                             int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared memory of this thread's bulk stores may be overwritten
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// this thread's bulk stores are complete
+__device__ __forceinline__ void tma_store_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -270,6 +291,50 @@ struct Sync {
   }
 };
 
+// Step sizes of chunk c (row r of the e = 0 warps), their running sum c_t
+// in log2 units and the column factors 2^(c_end - c_s) Delta_s, c_end the
+// last step of s's 32-step block, into shared memory.  `dt_next` holds
+// the bits of chunk c's raw bf16 step on entry and chunk c + 1's on exit
+// (converted only when used, so the load's latency is not waited for here).
+// Ends with every epilogue thread past the second barrier.
+struct StepPlan {
+  float *cum_s, *step_s, *colf_s, *tot_s;
+  const __nv_bfloat16 *dtp;
+  int64_t L, H;
+  float A2, bias;
+  int softplus;
+  __device__ void run(int c, int q, int e, int lane, int r, unsigned short &dt_next) const {
+    const int64_t t = static_cast<int64_t>(c) * Q + r;
+    float cw = 0.0f, step = 0.0f;
+    if (e == 0) {
+      if (t < L) {
+        const float v = __uint_as_float(static_cast<uint32_t>(dt_next) << 16) + bias;
+        step = softplus ? softplus_f(v) : v;
+      }
+      if (t + Q < L)
+        dt_next = *reinterpret_cast<const unsigned short *>(dtp + (t + Q) * H);
+      cw = step * A2;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, cw, o);
+        if (lane >= o) cw += u;
+      }
+      if (lane == 31) tot_s[q] = cw;
+    }
+    bar_sync(kEpiBarrier, kEpi);
+    if (e == 0) {
+      float base = 0.0f;
+      for (int j = 0; j < q; ++j) base += tot_s[j];
+      const float cum = base + cw;
+      const float cend = base + __shfl_sync(0xffffffffu, cw, 31);
+      cum_s[r] = cum;
+      step_s[r] = step;
+      colf_s[r] = ex2_mufu(cend - cum) * step;
+    }
+    bar_sync(kEpiBarrier, kEpi);
+  }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_fwd_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ unsigned char smem_raw[];
@@ -297,9 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + kEmpty, kEpi);
     mbar_init(bar + kEmpty + 1, kEpi);
     mbar_init(bar + kSFull, 1);
-    mbar_init(bar + kReadyState, kEpi);
     mbar_init(bar + kReadyScores, kEpi);
-    mbar_init(bar + kMmaDone, 1);
+    mbar_init(bar + kReadyState, kEpi);
+    mbar_init(bar + kDoneY, 1);
+    mbar_init(bar + kDoneH, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -331,41 +397,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------- tensor-core issue
+    // Descriptors of the 16-wide K slices differ from slice 0's only in the
+    // start-address field (16-byte units), by compile-time offsets.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idY = idesc_bf16(128, 64, 0, 1);
       constexpr uint32_t idH = idesc_bf16(128, 64, 1, 1);
-      for (int c = 0; c < nchunks; ++c) {
-        const int st = c & 1;
-        const uint32_t s = sbase + st * kStage;
-        sy.wait(kFull + st, (c >> 1) & 1);
+      const uint64_t dSp = desc_k(sbase + oSp, 0);
+      const uint64_t dHp = desc_mn(sbase + oHp, 0, kTile);
+      const uint64_t dXpp = desc_mn(sbase + oXpp, 0, kTile);
+      // S = C B^T of chunk c (stage c % 2), after its tiles have landed
+      auto scores = [&](int c) {
+        const uint32_t s = sbase + (c & 1) * kStage;
+        const uint64_t dC = desc_k(s + oC, 0), dBk = desc_k(s + oB, 0);
+        sy.wait(kFull + (c & 1), (c >> 1) & 1);
         tc_fence_after();
         if (!*abort) {
-          for (int kk = 0; kk < 8; ++kk)  // S = C B^T
-            umma_bf16(tmem + kColS, desc_k(s + oC, kk), desc_k(s + oB, kk), idS, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ko = (kk >> 2) * (kTile >> 4) + (kk & 3) * 2;
+            umma_bf16(tmem + kColS, dC + ko, dBk + ko, idS, kk > 0);
+          }
         }
         umma_commit(bar + kSFull);
-        sy.wait(kReadyState, c & 1);
-        tc_fence_after();
-        if (!*abort) {
-          for (int kk = 0; kk < 8; ++kk)  // YO = C Hp
-            umma_bf16(tmem + kColYO, desc_k(s + oC, kk), desc_mn(sbase + oHp, kk, kTile), idY,
-                      kk > 0);
-          for (int kk = 0; kk < 8; ++kk)  // H += B^T X''
-            umma_bf16(tmem + kColH, desc_mn(s + oB, kk, kTile), desc_mn(sbase + oXpp, kk, kTile),
-                      idH, 1);
-        }
+      };
+      // The tensor pipe runs products in issue order: the next chunk's
+      // scores go ahead of this chunk's state update, which is needed only
+      // after the next chunk's masked scores are built.
+      if (nchunks > 0) scores(0);
+      for (int c = 0; c < nchunks; ++c) {
+        const uint32_t s = sbase + (c & 1) * kStage;
+        const uint64_t dC = desc_k(s + oC, 0);
+        const uint64_t dBm = desc_mn(s + oB, 0, kTile), dX = desc_mn(s + oX, 0, kTile);
         sy.wait(kReadyScores, c & 1);
         tc_fence_after();
         if (!*abort) {
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // Y = S' X
-            umma_bf16(tmem + kColY, desc_k(sbase + oSp, kk), desc_mn(s + oX, kk, kTile), idY,
-                      kk > 0);
+            umma_bf16(tmem + kColY, dSp + (kk >> 2) * (kTile >> 4) + (kk & 3) * 2,
+                      dX + kk * 128, idY, kk > 0);
         }
-        umma_commit(bar + kMmaDone);
+        sy.wait(kReadyState, c & 1);
+        tc_fence_after();
+        if (!*abort) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // YO = C Hp
+            umma_bf16(tmem + kColYO, dC + (kk >> 2) * (kTile >> 4) + (kk & 3) * 2,
+                      dHp + kk * 128, idY, kk > 0);
+        }
+        umma_commit(bar + kDoneY);
+        if (c + 1 < nchunks) scores(c + 1);
+        if (!*abort) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // H += B^T X''
+            umma_bf16(tmem + kColH, dBm + kk * 128, dXpp + kk * 128, idH, 1);
+        }
+        umma_commit(bar + kDoneH);
       }
       // every product done before the tensor memory is freed
-      if (nchunks > 0) sy.drain(kMmaDone, (nchunks - 1) & 1);
+      if (nchunks > 0) sy.drain(kDoneH, (nchunks - 1) & 1);
     }
     __syncwarp();
   } else {
@@ -375,11 +465,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int e = (warp - 2) >> 2;
     const int r = 32 * q + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
-    const float A2 = p.A[h] * kLog2e;
-    const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
     const float Dh = p.D ? p.D[h] : 0.0f;
     const int64_t H = p.H;
-    const __nv_bfloat16 *dtp = p.dt + static_cast<int64_t>(b) * p.L * H + h;
+    // one thread per half issues the half's y stores (first lane of the
+    // half's first warp)
+    const bool writer = lane == 0 && q == 2;
+    const StepPlan plan{cum_s, step_s, colf_s, tot_s,
+                        p.dt + static_cast<int64_t>(b) * p.L * H + h, p.L, H,
+                        p.A[h] * kLog2e, p.dt_bias ? p.dt_bias[h] : 0.0f, p.softplus};
 
     // the initial state into H (row n = r, columns 32e .. 32e + 31)
     {
@@ -392,47 +485,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
     }
 
-    // the raw step of row r of the next chunk, loaded one chunk ahead
-    float dt_next = 0.0f;
-    if (e == 0 && r < p.L) dt_next = __bfloat162float(dtp[static_cast<int64_t>(r) * H]);
+    // raw steps are loaded one chunk ahead
+    unsigned short dt_next = 0;
+    if (e == 0 && r < p.L)
+      dt_next = *reinterpret_cast<const unsigned short *>(plan.dtp + static_cast<int64_t>(r) * H);
+    plan.run(0, q, e, lane, r, dt_next);
+    float cum = cum_s[r], cl = cum_s[Q - 1];
 
     for (int c = 0; c < nchunks; ++c) {
       const int st = c & 1;
-      const unsigned char *s = sm + st * kStage;
+      unsigned char *s = sm + st * kStage;
       const int64_t t = static_cast<int64_t>(c) * Q + r;
 
-      // step sizes, their running sum c_t (log2 units) and the column
-      // factors 2^(c_end - c_s) Delta_s, c_end the last step of s's
-      // 32-step block; computed by the e = 0 warps
-      float cw = 0.0f, step = 0.0f;
-      if (e == 0) {
-        if (t < p.L) {
-          const float v = dt_next + bias;
-          step = p.softplus ? softplus_f(v) : v;
-        }
-        if (t + Q < p.L) dt_next = __bfloat162float(dtp[(t + Q) * H]);
-        cw = step * A2;
+      // S' row t, blocks gb = e and e + 2 of 32 columns: below the diagonal
+      // S 2^(c_t - c_end(gb)) colf[s] (both factors <= 1); on the diagonal
+      // S 2^(c_t - c_s) Delta_s for s <= t, factored the same way when that
+      // cannot overflow; above it zero
+      sy.wait(kSFull, c & 1);
+      tc_fence_after();
+#pragma unroll 1
+      for (int gb = e; gb < 4; gb += 2) {
+        uint32_t pk[16];
+        if (gb < q) {
+          uint32_t v[32];
+          tmem_ld32(tl + kColS + 32 * gb, v);
+          const float rf = ex2_mufu(cum - cum_s[32 * gb + 31]);
+          tmem_wait_ld(v);
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float u = __shfl_up_sync(0xffffffffu, cw, o);
-          if (lane >= o) cw += u;
+          for (int j = 0; j < 32; j += 2) {
+            const int s0 = 32 * gb + j;
+            pk[j >> 1] = pack_bf16(__uint_as_float(v[j]) * rf * colf_s[s0],
+                                   __uint_as_float(v[j + 1]) * rf * colf_s[s0 + 1]);
+          }
+        } else if (gb == q) {
+          uint32_t v[32];
+          tmem_ld32(tl + kColS + 32 * gb, v);
+          const float cend = cum_s[32 * gb + 31];
+          // the same two factors when the block decays by less than 2^64
+          // (2^(c_t - c_end) <= 2^64 cannot overflow); else one 2^x each
+          const bool fact = cum_s[32 * gb] - cend < 64.0f;  // warp-uniform
+          const float rf = ex2_mufu(cum - cend);
+          tmem_wait_ld(v);
+          if (fact) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const int s0 = 32 * gb + j;
+              const float f0 = j <= lane ? __uint_as_float(v[j]) * rf * colf_s[s0] : 0.0f;
+              const float f1 =
+                  j + 1 <= lane ? __uint_as_float(v[j + 1]) * rf * colf_s[s0 + 1] : 0.0f;
+              pk[j >> 1] = pack_bf16(f0, f1);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const int s0 = 32 * gb + j;
+              const float f0 = j <= lane ? __uint_as_float(v[j]) *
+                                               ex2_mufu(cum - cum_s[s0]) * step_s[s0]
+                                         : 0.0f;
+              const float f1 = j + 1 <= lane ? __uint_as_float(v[j + 1]) *
+                                                   ex2_mufu(cum - cum_s[s0 + 1]) * step_s[s0 + 1]
+                                             : 0.0f;
+              pk[j >> 1] = pack_bf16(f0, f1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = 0u;
         }
-        if (lane == 31) tot_s[q] = cw;
+        unsigned char *dst = sm + oSp + (gb >> 1) * kTile;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4 *>(dst + swz(r, (gb & 1) * 4 + k)) =
+              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
       }
-      bar_sync(kEpiBarrier, kEpi);
-      float base = 0.0f;
-      for (int j = 0; j < q; ++j) base += tot_s[j];
-      if (e == 0) {
-        const float cum = base + cw;
-        const float cend = base + __shfl_sync(0xffffffffu, cw, 31);
-        cum_s[r] = cum;
-        step_s[r] = step;
-        colf_s[r] = ex2_mufu(cend - cum) * step;
-      }
-      bar_sync(kEpiBarrier, kEpi);
-      const float cum = cum_s[r];
-      const float cl = cum_s[Q - 1];
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar + kReadyScores);
 
+      // the previous chunk's state update is done: its tiles (B read by it,
+      // C holding the staged y) may be released once the y store has read
+      // the staging tile
+      if (c >= 1) {
+        sy.wait(kDoneH, (c - 1) & 1);
+        tc_fence_after();
+        if (writer) {
+          tma_store_wait_read();
+          mbar_arrive(bar + kEmpty + ((c - 1) & 1));
+        }
+      }
       sy.wait(kFull + st, (c >> 1) & 1);
 
       // Hp row n = r (columns of half e): bf16 copy of the state before
@@ -475,60 +615,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar + kReadyState);
 
-      // S' row t, blocks gb = e and e + 2 of 32 columns: below the diagonal
-      // S 2^(c_t - c_end(gb)) colf[s] (both factors <= 1), on the diagonal
-      // S 2^(c_t - c_s) Delta_s for s <= t, above it zero
-      sy.wait(kSFull, c & 1);
-      tc_fence_after();
-#pragma unroll 1
-      for (int gb = e; gb < 4; gb += 2) {
-        uint32_t pk[16];
-        if (gb < q) {
-          uint32_t v[32];
-          tmem_ld32(tl + kColS + 32 * gb, v);
-          const float rf = ex2_mufu(cum - cum_s[32 * gb + 31]);
-          tmem_wait_ld(v);
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int s0 = 32 * gb + j;
-            pk[j >> 1] = pack_bf16(__uint_as_float(v[j]) * rf * colf_s[s0],
-                                   __uint_as_float(v[j + 1]) * rf * colf_s[s0 + 1]);
-          }
-        } else if (gb == q) {
-          uint32_t v[32];
-          tmem_ld32(tl + kColS + 32 * gb, v);
-          tmem_wait_ld(v);
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int s0 = 32 * gb + j;
-            const float f0 = j <= lane ? __uint_as_float(v[j]) *
-                                             ex2_mufu(cum - cum_s[s0]) * step_s[s0]
-                                       : 0.0f;
-            const float f1 = j + 1 <= lane ? __uint_as_float(v[j + 1]) *
-                                                 ex2_mufu(cum - cum_s[s0 + 1]) * step_s[s0 + 1]
-                                           : 0.0f;
-            pk[j >> 1] = pack_bf16(f0, f1);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) pk[j] = 0u;
-        }
-        unsigned char *dst = sm + oSp + (gb >> 1) * kTile;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4 *>(dst + swz(r, (gb & 1) * 4 + k)) =
-              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+      // the next chunk's steps, while the output products run
+      const float cum_t = cum;
+      if (c + 1 < nchunks) {
+        plan.run(c + 1, q, e, lane, r, dt_next);
+        cum = cum_s[r];
+        cl = cum_s[Q - 1];
       }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar + kReadyScores);
 
       // y row t, columns of half e: Y + 2^(c_t) YO + D x, gated
-      sy.wait(kMmaDone, c & 1);
+      sy.wait(kDoneY, c & 1);
       tc_fence_after();
       {
-        const float eo = ex2_mufu(cum);
-        const int64_t row = ((static_cast<int64_t>(b) * p.L + t) * H + h) * P + 32 * e;
+        const float eo = ex2_mufu(cum_t);
         uint32_t yv[32], ov[32];
         tmem_ld32(tl + kColY + 32 * e, yv);
         tmem_ld32(tl + kColYO + 32 * e, ov);
@@ -548,42 +647,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fmaf(eo, __uint_as_float(ov[j + 1]), __uint_as_float(yv[j + 1])) + Dh * xf.y;
           }
         }
-        if (t < p.L) {
-          if (p.z) {
-            const uint4 *zr = reinterpret_cast<const uint4 *>(p.z + row);
+        if (p.z && t < p.L) {
+          const int64_t row = ((static_cast<int64_t>(b) * p.L + t) * H + h) * P + 32 * e;
+          const uint4 *zr = reinterpret_cast<const uint4 *>(p.z + row);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint4 zv = zr[k];
-              const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+          for (int k = 0; k < 4; ++k) {
+            const uint4 zv = zr[k];
+            const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 zf = unpack_bf16(zw[i]);
-                out[8 * k + 2 * i] *= silu_f(zf.x);
-                out[8 * k + 2 * i + 1] *= silu_f(zf.y);
-              }
+            for (int i = 0; i < 4; ++i) {
+              const float2 zf = unpack_bf16(zw[i]);
+              out[8 * k + 2 * i] *= silu_f(zf.x);
+              out[8 * k + 2 * i + 1] *= silu_f(zf.y);
             }
           }
-          if (p.y_bf16) {
-            uint4 *yr = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.y) + row);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              yr[k] = make_uint4(pack_bf16(out[8 * k], out[8 * k + 1]),
-                                 pack_bf16(out[8 * k + 2], out[8 * k + 3]),
-                                 pack_bf16(out[8 * k + 4], out[8 * k + 5]),
-                                 pack_bf16(out[8 * k + 6], out[8 * k + 7]));
-          } else {
-            float4 *yr = reinterpret_cast<float4 *>(static_cast<float *>(p.y) + row);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              yr[k] = make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
-          }
         }
+        // stage row t of half e in the stage's C tile (free once the output
+        // products are done) and store the half's 128 x 32 box with one TMA
+        // store
+        unsigned char *yt = s + oC + e * kTile;
+        if (p.y_bf16) {
+          // 64-byte rows, 64-byte swizzle: chunk k at k ^ ((t / 2) % 4)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4 *>(yt + r * 64 + ((k ^ ((r >> 1) & 3)) << 4)) =
+                make_uint4(pack_bf16(out[8 * k], out[8 * k + 1]),
+                           pack_bf16(out[8 * k + 2], out[8 * k + 3]),
+                           pack_bf16(out[8 * k + 4], out[8 * k + 5]),
+                           pack_bf16(out[8 * k + 6], out[8 * k + 7]));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4 *>(yt + swz(r, k)) =
+                make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+        }
+        fence_async_smem();
+        bar_sync(kHalfBarrier + e, kEpi / 2);
+        if (writer) tma_store_4d(&maps.y, yt, 32 * e, h, c * Q, b);
       }
       tc_fence_before();
-      mbar_arrive(bar + kEmpty + st);
+      // the writer releases the stage in the next chunk, after the state
+      // update and its store's read of the staging tile
+      if (!writer) mbar_arrive(bar + kEmpty + st);
     }
 
+    if (writer) tma_store_wait_all();
     // the state after the last chunk (columns of half e)
+    if (nchunks > 0) {
+      sy.wait(kDoneH, (nchunks - 1) & 1);
+      tc_fence_after();
+    }
     if (p.last) {
       float *lr = p.last + (static_cast<int64_t>(b) * H + h) * P * NS;
       uint32_t v[32];
@@ -634,6 +747,22 @@ bool encode_4d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64
          CUDA_SUCCESS;
 }
 
+// y: (batch, seqlen, nheads, 64) fp32 or bf16; box {32, 1, Q, 1}, the
+// swizzle matching the 128- (fp32) or 64-byte (bf16) rows of the box
+bool encode_y(CUtensorMap *m, void *ptr, bool bf16, uint64_t H, uint64_t L, uint64_t Bt) {
+  auto enc = encoder();
+  if (!enc) return false;
+  const uint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(P), H, L, Bt};
+  cuuint64_t strides[3] = {P * es, P * H * es, P * H * L * es};
+  cuuint32_t box[4] = {32, 1, static_cast<cuuint32_t>(Q), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr,
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool al16(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
 bool al4(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 3) == 0; }
 
@@ -673,7 +802,8 @@ extern "C" mss_status mamba2_ssd_fwd(const mss_ssd_args *a, void *stream) {
                  G = static_cast<uint64_t>(a->ngroups), Bt = static_cast<uint64_t>(a->batch);
   if (!ssd::encode_4d(&maps.x, a->x, ssd::P, H, L, Bt) ||
       !ssd::encode_4d(&maps.B, a->B, ssd::NS, G, L, Bt) ||
-      !ssd::encode_4d(&maps.C, a->C, ssd::NS, G, L, Bt))
+      !ssd::encode_4d(&maps.C, a->C, ssd::NS, G, L, Bt) ||
+      !ssd::encode_y(&maps.y, a->y, a->out_dtype == MSS_BF16, H, L, Bt))
     return MSS_ERR_CUDA;
   unsigned *status = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), ssd::g_ssd_status) !=
