@@ -122,25 +122,35 @@ def measured_tensor_peak():
         return 1400.0, "fallback (sustained)"
 
 
-def kernel_source_hash() -> str:
+# the sources each timed kernel is compiled from
+KERNEL_SOURCES = {
+    "fwd": ("device_math.cuh", "scan_fwd.cu", "scan_fwd.cuh"),
+    "bwd": ("device_math.cuh", "scan_bwd.cu", "scan_bwd.cuh"),
+    "decode": ("device_math.cuh", "state_update.cu"),
+    "ssd": ("device_math.cuh", "ssd_fwd.cu"),
+}
+
+
+def kernel_source_hash(kernel: str = "fwd") -> str:
+    """Hash of the source files one kernel is built from (a profile's
+    counters stay valid while it is unchanged)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_48_b200", "csrc")
-    for p in sorted(glob.glob(os.path.join(csrc, "*.cu")) +
-                    glob.glob(os.path.join(csrc, "*.cuh"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kernel: str = "fwd"):
     """DRAM bytes per launch from the committed ncu summary, or None when
-    the kernels changed since the counters were taken."""
+    the kernel changed since the counters were taken."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
         e = d.get(workload)
-        if e and e.get("kernel_source_hash") == kernel_source_hash():
+        if e and e.get("kernel_source_hash") == kernel_source_hash(kernel):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -407,7 +417,7 @@ def run_bwd(args, rank, world, local_rank):
                      "peak_source": src, "traffic": None,
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
-        "kernel_source_hash": kernel_source_hash(),
+        "kernel_source_hash": kernel_source_hash("bwd"),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -478,7 +488,7 @@ def run_decode(args, rank, world, local_rank):
                      "peak_source": src, "traffic": None,
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
-        "kernel_source_hash": kernel_source_hash(),
+        "kernel_source_hash": kernel_source_hash("decode"),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -638,7 +648,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": K,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                    "reasons": clk["reasons"], "samples": clk["samples"]},
-        "kernel_source_hash": kernel_source_hash(),
+        "kernel_source_hash": kernel_source_hash("fwd"),
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
@@ -737,14 +747,16 @@ def run_ssd(args, rank, world, local_rank):
         "tokens_per_s": w.batch * w.seqlen * K * world / (max_ms * 1e-3),
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
                      "unit": "GB/s", "frac": value / world / peak,
-                     "peak_source": src, "traffic": None,
+                     "peak_source": src,
+                     "traffic": (profiled_traffic(w.name, "ssd")
+                                 if args.out_dtype == "f32" else None),
                      "algorithmic_bytes_per_launch": nbytes,
                      "tensor": {"achieved": tflops / world, "peak": tpeak,
                                 "unit": "TFLOP/s", "frac": tflops / world / tpeak,
                                 "peak_source": tsrc,
                                 "algorithmic_flops_per_launch": flops}},
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
-        "kernel_source_hash": kernel_source_hash(),
+        "kernel_source_hash": kernel_source_hash("ssd"),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
