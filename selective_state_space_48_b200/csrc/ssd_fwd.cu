@@ -7,7 +7,8 @@
 //
 //   S  = C B^T                       M = t, N = s, K = n   (both K-major)
 //   Y  = S' X,   S'[t,s] = S[t,s] 2^(c_t - c_s) Delta_s  for s <= t, else 0
-//                                    M = t, N = p, K = s   (B operand MN-major)
+//                                    M = t, N = p, K = s   (A in tensor memory,
+//                                                         B operand MN-major)
 //   YO = C Hp,   Hp = the state before the chunk (bf16 copy)
 //                                    M = t, N = p, K = n   (B operand MN-major)
 //   H  = 2^(c_last) H + B^T X'',  X''[s,p] = X[s,p] Delta_s 2^(c_last - c_s)
@@ -21,8 +22,8 @@
 // tiles (two stages), warp 1 allocates tensor memory and issues the
 // tcgen05.mma products (one thread), warps 2-9 (256 threads, one tensor
 // memory lane quarter per pair of warps, which split the columns) compute
-// the step sizes and their running sum, build the operands S', X'' and Hp
-// in shared memory, rescale H, and write y.  The state products (YO and H)
+// the step sizes and their running sum, build the operand S' in tensor
+// memory and X'' and Hp in shared memory, rescale H, and write y.  The state products (YO and H)
 // are issued as soon as Hp and X'' are ready, so they run while the
 // epilogue builds the masked scores S'.
 //
@@ -58,8 +59,7 @@ constexpr int kHalfBarrier = 2; // + e: named barrier of the four warps of half 
 constexpr int kTile = Q * 64 * 2;      // one [128][64] bf16 tile
 constexpr int kStage = 5 * kTile;      // C (two n halves), B (two), X
 constexpr int oC = 0, oB = 2 * kTile, oX = 4 * kTile;
-constexpr int oSp = 2 * kStage;        // S' (two s halves)
-constexpr int oXpp = oSp + 2 * kTile;  // X''
+constexpr int oXpp = 2 * kStage;       // X''
 constexpr int oHp = oXpp + kTile;      // bf16 copy of the state, [n][p]
 constexpr int oCum = oHp + kTile;      // float c_s [Q]
 constexpr int oStep = oCum + Q * 4;    // float Delta_s [Q]
@@ -74,6 +74,7 @@ static_assert(kSmemBytes <= 232448, "shared memory above the per-block limit");
 
 // tensor memory columns (fp32, lane = row)
 constexpr uint32_t kColS = 0, kColY = 128, kColYO = 192, kColH = 256;
+constexpr uint32_t kColSp = 320;  // S' as bf16 pairs: 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 // barrier indices: tiles landed / released (per stage), scores S done,
@@ -167,6 +168,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]: A is M lanes of K bf16 values packed two
+// per 32-bit column (K slice kk at column offset 8 kk)
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // arrive on `bar` once every tcgen05.mma issued so far by this thread is done
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile(
@@ -213,6 +225,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
       "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
       "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's lane
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() {
@@ -403,7 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idY = idesc_bf16(128, 64, 0, 1);
       constexpr uint32_t idH = idesc_bf16(128, 64, 1, 1);
-      const uint64_t dSp = desc_k(sbase + oSp, 0);
       const uint64_t dHp = desc_mn(sbase + oHp, 0, kTile);
       const uint64_t dXpp = desc_mn(sbase + oXpp, 0, kTile);
       // S = C B^T of chunk c (stage c % 2), after its tiles have landed
@@ -433,9 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (!*abort) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // Y = S' X
-            umma_bf16(tmem + kColY, dSp + (kk >> 2) * (kTile >> 4) + (kk & 3) * 2,
-                      dX + kk * 128, idY, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)  // Y = S' X, S' from tensor memory
+            umma_bf16_ts(tmem + kColY, tmem + kColSp + 8 * kk, dX + kk * 128, idY, kk > 0);
         }
         sy.wait(kReadyState, c & 1);
         tc_fence_after();
@@ -552,13 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) pk[j] = 0u;
         }
-        unsigned char *dst = sm + oSp + (gb >> 1) * kTile;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4 *>(dst + swz(r, (gb & 1) * 4 + k)) =
-              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        tmem_st16(tl + kColSp + 16 * gb, pk);
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar + kReadyScores);
 
