@@ -65,7 +65,7 @@ constexpr int oCum = oHp + kTile;      // float c_s [Q]
 constexpr int oStep = oCum + Q * 4;    // float Delta_s [Q]
 constexpr int oColf = oStep + Q * 4;   // float column factors [Q]
 constexpr int oTot = oColf + Q * 4;    // float warp totals [4]
-constexpr int oBar = oTot + 16;        // 9 mbarriers
+constexpr int oBar = oTot + 16;        // 10 mbarriers
 constexpr int oTmemSlot = oBar + 10 * 8;
 constexpr int oAbort = oTmemSlot + 4;
 constexpr int kSmemUsed = oAbort + 12;
@@ -78,10 +78,10 @@ constexpr uint32_t kColSp = 320;  // S' as bf16 pairs: 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 // barrier indices: tiles landed / released (per stage), scores S done,
-// masked scores S' ready, state operands ready (Hp, X'', H rescaled), the
-// output products Y and YO done, the state update done
+// masked scores S' ready, Hp ready, the state update's operands ready (X'',
+// H rescaled), the output products Y and YO done, the state update done
 constexpr int kFull = 0, kEmpty = 2, kSFull = 4, kReadyScores = 5, kReadyState = 6,
-              kDoneY = 7, kDoneH = 8;
+              kDoneY = 7, kDoneH = 8, kReadyHp = 9;
 
 struct Params {
   int64_t batch, L, H, G;
@@ -386,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + kSFull, 1);
     mbar_init(bar + kReadyScores, kEpi);
     mbar_init(bar + kReadyState, kEpi);
+    mbar_init(bar + kReadyHp, kEpi);
     mbar_init(bar + kDoneY, 1);
     mbar_init(bar + kDoneH, 1);
     *abort = 0;
@@ -442,9 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(bar + kSFull);
       };
-      // The tensor pipe runs products in issue order: the next chunk's
-      // scores go ahead of this chunk's state update, which is needed only
-      // after the next chunk's masked scores are built.
+      // The tensor pipe runs products in issue order: Y, then YO as soon as
+      // Hp is written, then the next chunk's scores, then this chunk's state
+      // update, which is needed only after the next chunk's masked scores
+      // are built.
       if (nchunks > 0) scores(0);
       for (int c = 0; c < nchunks; ++c) {
         const uint32_t s = sbase + (c & 1) * kStage;
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < 8; ++kk)  // Y = S' X, S' from tensor memory
             umma_bf16_ts(tmem + kColY, tmem + kColSp + 8 * kk, dX + kk * 128, idY, kk > 0);
         }
-        sy.wait(kReadyState, c & 1);
+        sy.wait(kReadyHp, c & 1);
         tc_fence_after();
         if (!*abort) {
 #pragma unroll
@@ -467,6 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(bar + kDoneY);
         if (c + 1 < nchunks) scores(c + 1);
+        sy.wait(kReadyState, c & 1);
+        tc_fence_after();
         if (!*abort) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // H += B^T X''
@@ -607,6 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           o.w = pack_bf16(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7]));
           *reinterpret_cast<uint4 *>(sm + oHp + swz(r, e * 4 + k)) = o;
         }
+        // the carried-state readout YO = C Hp may start now
+        fence_async_smem();
+        mbar_arrive(bar + kReadyHp);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam);
         tmem_st32(tl + kColH + 32 * e, v);
