@@ -336,6 +336,54 @@ def oracle_timing(inp, w, seconds: float, steps: int = 1, warmup: int = 0):
     return gbs, ups, ch, threads, total
 
 
+def _ssd_sample(inp: dict, w, heads: int) -> list:
+    """The first `heads` (batch row, head) pairs in (b, h) order at full
+    length, as float64 host arrays grouped per batch row.  Counts are
+    whole groups of heads, so each slice keeps its heads' group of B, C."""
+    hpg = w.nheads // w.ngroups
+    heads = max(hpg, (heads // hpg) * hpg)
+    out, left, b = [], heads, 0
+    while left > 0 and b < w.batch:
+        k = min(left, w.nheads)
+        f = lambda t: t.detach().cpu().double().numpy()
+        hsel = lambda t: None if t is None else f(t[:k])
+        out.append(dict(x=f(inp["x"][b:b + 1, :, :k]), dt=f(inp["dt"][b:b + 1, :, :k]),
+                        A=hsel(inp["A"]), D=hsel(inp["D"]), dt_bias=hsel(inp["dt_bias"]),
+                        z=None if inp["z"] is None else f(inp["z"][b:b + 1, :, :k]),
+                        B=f(inp["B"][b:b + 1, :, :k // hpg]),
+                        C=f(inp["C"][b:b + 1, :, :k // hpg])))
+        left -= k
+        b += 1
+    return out
+
+
+def _run_ssd_oracle(groups, w):
+    import oracle
+    for g in groups:
+        oracle.ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                        dt_bias=g["dt_bias"], dt_softplus=w.softplus)
+
+
+def ssd_oracle_timing(inp, w, seconds: float, out_b: int = 4):
+    """Time the SSD oracle on a bounded sample of whole (batch row, head)
+    sequences; returns (GB/s, heads sampled, threads, seconds)."""
+    import oracle
+    threads = oracle.num_threads()
+    hpg = w.nheads // w.ngroups
+    probe = max(hpg, (max(1, threads) // hpg) * hpg)
+    t0 = time.perf_counter()
+    _run_ssd_oracle(_ssd_sample(inp, w, probe), w)
+    per_head = (time.perf_counter() - t0) / probe
+    heads = int(max(1, min(w.batch * w.nheads, round(seconds / max(per_head, 1e-9)))))
+    groups = _ssd_sample(inp, w, heads)
+    heads = sum(g["x"].shape[2] for g in groups)
+    t0 = time.perf_counter()
+    _run_ssd_oracle(groups, w)
+    total = time.perf_counter() - t0
+    share = heads / (w.batch * w.nheads)
+    return w.algorithmic_bytes(out_b) * share / total / 1e9, heads, threads, total
+
+
 # ------------------------------------------------------------- our arm
 
 
@@ -758,6 +806,15 @@ def run_ssd(args, rank, world, local_rank):
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
         "kernel_source_hash": kernel_source_hash("ssd"),
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, heads, threads, secs = ssd_oracle_timing(inp, w, args.cpu_seconds / 2,
+                                                      out_bytes(args.out_dtype))
+        line["cpu_baseline"] = {
+            "value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": (f"{heads} of {w.batch * w.nheads} (batch row, head) sequences at "
+                       f"full length L={w.seqlen}, one pass, {secs:.1f} s wall, fp64 C "
+                       "oracle with OpenMP over (batch row, head); GB/s = the sample's "
+                       "share of the step's algorithmic bytes / time")}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

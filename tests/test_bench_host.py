@@ -72,3 +72,31 @@ def test_reference_arm_prints_the_contract_line(capsys):
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["value"] > 0
+
+
+def test_ssd_workload_bytes_and_flops_by_hand():
+    """2.7B-shaped layer: x read and y (fp32) written per (b, t, h, p), dt per
+    (b, t, h), B and C per (b, t, n), three fp32 vectors per head; scores
+    once per (b, chunk, group), the other three products per (b, chunk, head)."""
+    w = workloads.SSD_BY_NAME["mamba2-2.7b-layer"]
+    btp = 8 * 2048 * 80 * 64
+    want = btp * (2 + 4) + 8 * 2048 * 80 * 2 + 2 * 8 * 2048 * 128 * 2 + 80 * 4 * 3
+    assert w.algorithmic_bytes(4) == want == 514327488
+    assert w.algorithmic_bytes(2) == want - btp * 2
+    chunks = 2048 // 128
+    scores = 8 * chunks * 2 * 128 * 128 * 128
+    per_head = 8 * chunks * 80 * (2 * 128 * 128 * 64 + 2 * 2 * 128 * 128 * 64)
+    assert w.chunk_flops() == scores + per_head == 64961380352
+
+
+def test_ssd_oracle_sample_timing_on_cpu():
+    """The SSD CPU baseline samples whole groups of heads and reports a
+    positive rate (inputs on the CPU here; on the GPU machine they are copied)."""
+    w = workloads.SSD_BY_NAME["ssd-small"]
+    inp = workloads.make_ssd_inputs(w, seed=3)
+    groups = bench._ssd_sample(inp, w, 3)
+    assert sum(g["x"].shape[2] for g in groups) == 2  # rounded to whole groups
+    assert all(g["B"].shape[2] * 2 == g["x"].shape[2] for g in groups)
+    gbs, heads, threads, secs = bench.ssd_oracle_timing(inp, w, 0.05)
+    assert gbs > 0 and heads % 2 == 0 and 2 <= heads <= w.batch * w.nheads
+    assert threads >= 1 and secs > 0
