@@ -849,13 +849,10 @@ extern "C" mss_status mamba2_ssd_fwd(const mss_ssd_args *a, void *stream) {
   p.last = a->last_state;
   p.status = status;
   p.spin_ns = a->spin_timeout_ns ? a->spin_timeout_ns : 2000000000ull;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(ssd::ssd_fwd_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, ssd::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return MSS_ERR_CUDA;
+  // per launch: the attribute belongs to the current device
+  if (cudaFuncSetAttribute(ssd::ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           ssd::kSmemBytes) != cudaSuccess)
+    return MSS_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(a->batch * a->nheads);
   ssd::ssd_fwd_kernel<<<grid, ssd::kThreads, ssd::kSmemBytes,
                         static_cast<cudaStream_t>(stream)>>>(maps, p);
