@@ -336,6 +336,34 @@ def oracle_timing(inp, w, seconds: float, steps: int = 1, warmup: int = 0):
     return gbs, ups, ch, threads, total
 
 
+def sample_max_norm_err(y, inp, w, channels: int) -> float:
+    """max |y - y_oracle| / max |y_oracle| over the first `channels`
+    channels of the batch (fp64 oracle on the same inputs)."""
+    import oracle
+    groups = _oracle_sample_inputs(inp, channels, w)
+    worst, scale = 0.0, 0.0
+    for b, g in enumerate(groups):
+        ref = oracle.selective_scan(g["u"], g["delta"], g["A"], g["B"], g["C"],
+                                    D=g["D"], z=g["z"], delta_bias=g["delta_bias"],
+                                    delta_softplus=w.softplus)
+        got = y[b:b + 1, :ref.shape[1]].detach().float().cpu().double().numpy()
+        worst = max(worst, float(np.abs(got - ref).max()))
+        scale = max(scale, float(np.abs(ref).max()))
+    return worst / scale if scale > 0 else worst
+
+
+def ssd_sample_max_norm_err(y, inp, w) -> float:
+    """The same for the SSD scan: the heads of batch row 0's first group."""
+    import oracle
+    g = _ssd_sample(inp, w, w.nheads // w.ngroups)[0]
+    ref = oracle.ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                          dt_bias=g["dt_bias"], dt_softplus=w.softplus)
+    got = y[0:1, :, :ref.shape[2]].detach().float().cpu().double().numpy()
+    scale = float(np.abs(ref).max())
+    err = float(np.abs(got - ref).max())
+    return err / scale if scale > 0 else err
+
+
 def _ssd_sample(inp: dict, w, heads: int) -> list:
     """The first `heads` (batch row, head) pairs in (b, h) order at full
     length, as float64 host arrays grouped per batch row.  Counts are
@@ -651,6 +679,14 @@ def run_ours(args, rank, world, local_rank):
                           "fp64 C oracle with OpenMP over channels; GB/s = the "
                           "sample's share of the step's algorithmic bytes / time")}
 
+    # ---- parity of the timed output on a sample, against the fp64 oracle
+    err = None
+    if rank == 0 and not args.varlen and not args.trapezoid:
+        try:
+            err = sample_max_norm_err(y, inp, w, 64)
+        except Exception as ex:  # reported, never fatal to the timing line
+            print(f"parity sample failed: {ex}", file=sys.stderr)
+
     peak, peak_kind = measured_peaks()
     achieved = bytes_step / (max_kernel_ms * 1e-3) / 1e9
     clk = clocks.summary()
@@ -675,6 +711,9 @@ def run_ours(args, rank, world, local_rank):
                        **({"update": "trapezoidal"} if args.trapezoid else {}),
                        **({"writes_checkpoints": True} if args.checkpoints else {})),
         "state_updates_per_s": updates,
+        "max_norm_err": err,
+        "max_norm_err_sample": ("first 64 channels, full length, vs the fp64 oracle"
+                                if err is not None else None),
         "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": value / world / peak,
         # the bound that binds: the special-function unit (one ex2 per state
@@ -806,6 +845,13 @@ def run_ssd(args, rank, world, local_rank):
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
         "kernel_source_hash": kernel_source_hash("ssd"),
     }
+    if rank == 0:
+        try:
+            line["max_norm_err"] = ssd_sample_max_norm_err(y, inp, w)
+            line["max_norm_err_sample"] = (f"batch row 0, heads 0-{w.nheads // w.ngroups - 1}, "
+                                           "full length, vs the fp64 oracle")
+        except Exception as ex:  # reported, never fatal to the timing line
+            print(f"parity sample failed: {ex}", file=sys.stderr)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, heads, threads, secs = ssd_oracle_timing(inp, w, args.cpu_seconds / 2,
                                                       out_bytes(args.out_dtype))

@@ -100,3 +100,28 @@ def test_ssd_oracle_sample_timing_on_cpu():
     gbs, heads, threads, secs = bench.ssd_oracle_timing(inp, w, 0.05)
     assert gbs > 0 and heads % 2 == 0 and 2 <= heads <= w.batch * w.nheads
     assert threads >= 1 and secs > 0
+
+
+def test_sampled_parity_helpers_on_cpu():
+    """The bench's parity samples: the oracle's own output gives only the
+    rounding of y to fp32 (the GPU's output dtype), a perturbed one the
+    perturbation relative to max |y|."""
+    import numpy as np
+    import oracle
+    w = workloads.custom(2, 8, 4, 40, in_dtype="f32", has_z=True)
+    inp = workloads.make_inputs(w, seed=4)
+    h = workloads.to_numpy_f64(inp)
+    ref = oracle.selective_scan(h["u"], h["delta"], h["A"], h["B"], h["C"], D=h["D"],
+                                z=h["z"], delta_bias=h["delta_bias"])
+    y = torch.from_numpy(ref.copy())
+    assert bench.sample_max_norm_err(y, inp, w, 12) <= 2.0 ** -24
+    y[0, 3, 7] += 0.5
+    scale = float(np.abs(ref[:1]).max())
+    assert abs(bench.sample_max_norm_err(y, inp, w, 8) - 0.5 / scale) <= 2.0 ** -23
+
+    ws = workloads.SSD_BY_NAME["ssd-small"]
+    si = workloads.make_ssd_inputs(ws, seed=5)
+    hs = workloads.to_numpy_f64(si)
+    yref = oracle.ssd_scan(hs["x"], hs["dt"], hs["A"], hs["B"], hs["C"], D=hs["D"],
+                           z=hs["z"], dt_bias=hs["dt_bias"])
+    assert bench.ssd_sample_max_norm_err(torch.from_numpy(yref.copy()), si, ws) <= 2.0 ** -24
