@@ -814,6 +814,8 @@ def run_ssd(args, rank, world, local_rank):
     clocks.stop()
     barrier(world)
     max_ms = reduce_max(t0.elapsed_time(t1), world)
+    if sss.load_library().mss_ssd_status(None) != sss.MSS_OK:
+        raise RuntimeError("SSD kernel reported a timeout in the timed region")
     nbytes = w.algorithmic_bytes(out_bytes(args.out_dtype))
     flops = w.chunk_flops()
     value = whole_job_gbs(nbytes, K, world, max_ms)
