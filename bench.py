@@ -392,9 +392,11 @@ def _run_ssd_oracle(groups, w):
                         dt_bias=g["dt_bias"], dt_softplus=w.softplus)
 
 
-def ssd_oracle_timing(inp, w, seconds: float, out_b: int = 4):
+def ssd_oracle_timing(inp, w, seconds: float, out_b: int = 4, steps: int = 1,
+                      warmup: int = 0):
     """Time the SSD oracle on a bounded sample of whole (batch row, head)
-    sequences; returns (GB/s, heads sampled, threads, seconds)."""
+    sequences, `seconds` spread over warmup + steps passes; returns (GB/s,
+    heads sampled per step, threads, seconds of the timed steps)."""
     import oracle
     threads = oracle.num_threads()
     hpg = w.nheads // w.ngroups
@@ -402,14 +404,18 @@ def ssd_oracle_timing(inp, w, seconds: float, out_b: int = 4):
     t0 = time.perf_counter()
     _run_ssd_oracle(_ssd_sample(inp, w, probe), w)
     per_head = (time.perf_counter() - t0) / probe
-    heads = int(max(1, min(w.batch * w.nheads, round(seconds / max(per_head, 1e-9)))))
+    per_step = seconds / max(1, steps + warmup)
+    heads = int(max(1, min(w.batch * w.nheads, round(per_step / max(per_head, 1e-9)))))
     groups = _ssd_sample(inp, w, heads)
     heads = sum(g["x"].shape[2] for g in groups)
+    for _ in range(warmup):
+        _run_ssd_oracle(groups, w)
     t0 = time.perf_counter()
-    _run_ssd_oracle(groups, w)
+    for _ in range(steps):
+        _run_ssd_oracle(groups, w)
     total = time.perf_counter() - t0
     share = heads / (w.batch * w.nheads)
-    return w.algorithmic_bytes(out_b) * share / total / 1e9, heads, threads, total
+    return w.algorithmic_bytes(out_b) * share * steps / total / 1e9, heads, threads, total
 
 
 # ------------------------------------------------------------- our arm
@@ -745,9 +751,45 @@ def run_ours(args, rank, world, local_rank):
 # -------------------------------------------------------- reference arm
 
 
+SSD_METRIC = "Mamba-2 SSD chunked scan HBM GB/s; tokens/s"
+
+
+def ssd_config(w, out_dtype: str) -> dict:
+    return {"workload": w.name, "pass": "ssd", "batch": w.batch, "seq_len": w.seqlen,
+            "nheads": w.nheads, "headdim": w.headdim, "ngroups": w.ngroups,
+            "dstate": w.dstate, "chunk": 128, "y_dtype": out_dtype}
+
+
+def run_reference_ssd(args):
+    """The SSD oracle as it stands, on this host's cores, each step a
+    bounded sample (whole head sequences) of the SSD workload."""
+    w = workloads.SSD_BY_NAME[args.ssd_workload]
+    inp = workloads.make_ssd_inputs(w, seed=48100)
+    budget = args.ref_seconds
+    if budget is None:
+        budget = min(120.0, max(20.0, 3.0 * (args.steps + args.warmup)))
+    gbs, heads, threads, total = ssd_oracle_timing(inp, w, budget, out_bytes(args.out_dtype),
+                                                   steps=args.steps, warmup=args.warmup)
+    sample = (f"{heads} of {w.batch * w.nheads} (batch row, head) sequences per step, full "
+              f"length L={w.seqlen}; fp64 C oracle, OpenMP over (batch row, head)")
+    return {
+        "impl": "reference", "metric": SSD_METRIC, "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": ssd_config(w, args.out_dtype),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args):
     """The fp64 oracle as it stands, on this host's cores, each step a
     bounded sample (a share of the channels, full length) of the workload."""
+    if args.pass_ == "ssd":
+        return run_reference_ssd(args)
     w = workloads.BY_NAME[args.workload]
     inp = workloads.make_inputs(w, device="cpu")
     budget = args.ref_seconds
@@ -823,16 +865,13 @@ def run_ssd(args, rank, world, local_rank):
     tflops = flops * K / (max_ms * 1e-3) / 1e12
     tpeak, tsrc = measured_tensor_peak()
     line = {
-        "metric": "Mamba-2 SSD chunked scan HBM GB/s; tokens/s",
+        "metric": SSD_METRIC,
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": max_ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "pass": "ssd", "batch": w.batch,
-                   "seq_len": w.seqlen, "nheads": w.nheads, "headdim": w.headdim,
-                   "ngroups": w.ngroups, "dstate": w.dstate, "chunk": 128,
-                   "y_dtype": args.out_dtype,
-                   "l2": f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step)"},
+        "config": dict(ssd_config(w, args.out_dtype),
+                       l2=f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step)"),
         "tokens_per_s": w.batch * w.seqlen * K * world / (max_ms * 1e-3),
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
                      "unit": "GB/s", "frac": value / world / peak,

@@ -125,3 +125,17 @@ def test_sampled_parity_helpers_on_cpu():
     yref = oracle.ssd_scan(hs["x"], hs["dt"], hs["A"], hs["B"], hs["C"], D=hs["D"],
                            z=hs["z"], dt_bias=hs["dt_bias"])
     assert bench.ssd_sample_max_norm_err(torch.from_numpy(yref.copy()), si, ws) <= 2.0 ** -24
+
+
+def test_reference_arm_for_the_ssd_pass(capsys):
+    """--impl reference --pass ssd times the SSD oracle on the SSD workload,
+    with the SSD line's metric, unit and config."""
+    rc = bench.main(["--impl", "reference", "--pass", "ssd", "--ssd-workload", "ssd-small",
+                     "--steps", "2", "--warmup", "1", "--ref-seconds", "0.3"])
+    assert rc == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.SSD_METRIC
+    assert line["unit"] == "GB/s" and line["value"] > 0
+    assert line["config"] == bench.ssd_config(workloads.SSD_BY_NAME["ssd-small"], "f32")
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
