@@ -94,7 +94,9 @@ typedef struct mss_ssd_args {
 mss_status mamba2_ssd_fwd(const mss_ssd_args *args, void *stream);
 
 /* Synchronises `stream` and returns the SSD kernels' device status word
- * (MSS_OK or MSS_ERR_TIMEOUT), clearing it. */
+ * (MSS_OK or MSS_ERR_TIMEOUT), clearing it.  The word is the library's own
+ * (one per device), so it reports every SSD call on this device since the
+ * previous read, on any stream. */
 mss_status mss_ssd_status(void *stream);
 
 #ifdef __cplusplus
