@@ -5,12 +5,18 @@
 
 One step is one full forward scan (softplus step size, discretisation,
 recurrence, C readout, D skip, silu(z) gate) over one batch of the
-Mamba-130M-shaped layer workload (batch 8, D 1536, N 16, L 2048, bf16
+Mamba-1.4B-shaped layer workload (batch 4, D 4096, N 16, L 4096, bf16
 inputs, fp32 state and output) with inputs resident in HBM.  W untimed steps,
 then exactly K steps bracketed by a barrier and a device synchronise on both
 sides, timed with CUDA events on the launching stream; the time is the max
-over ranks.  The working set (253 MB of inputs and outputs) is larger than
+over ranks.  The working set (672 MB of inputs and outputs) is larger than
 the 126 MB L2, so no step finds the previous step's data in L2.
+
+The line also carries ``per_config``: every named workload (tiny fp32,
+130M-shaped layer, 1.4B-shaped layer, long-context, audio-length) timed the
+same way for a short run, with its HBM and exponential-unit fractions and
+its error against the fp64 oracle on a sample of channels.  The default
+workload's own error is measured on every output element.
 
 Under torchrun (N > 1) every rank runs an independent replica of the
 workload on its own GPU (the scan needs no exchange between GPUs) and
@@ -47,7 +53,7 @@ import workloads  # noqa: E402
 
 METRIC = ("selective-scan HBM GB/s (fraction of B200 peak); "
           "B·D·L·N state-updates/s")
-DEFAULT_WORKLOAD = "mamba130m-layer"
+DEFAULT_WORKLOAD = "mamba1.4b-layer"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "roofline_traffic.json")
@@ -91,6 +97,11 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the short runs of the other named workloads")
+    ap.add_argument("--parity", choices=["all", "sample", "none"], default="all",
+                    help="error of the timed output against the fp64 oracle: every "
+                         "element (all), 64 channels (sample) or not at all")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="CPU time budget of --impl reference (default: "
                          "3 s per step, between 20 and 120 s)")
@@ -295,12 +306,12 @@ def _oracle_sample_inputs(inp: dict, channels: int, w):
     return groups
 
 
-def _run_oracle_groups(groups, w):
+def _run_oracle_groups(groups, w, **kw):
     import oracle
-    for g in groups:
-        oracle.selective_scan(g["u"], g["delta"], g["A"], g["B"], g["C"],
-                              D=g["D"], z=g["z"], delta_bias=g["delta_bias"],
-                              delta_softplus=w.softplus)
+    return [oracle.selective_scan(g["u"], g["delta"], g["A"], g["B"], g["C"],
+                                  D=g["D"], z=g["z"], delta_bias=g["delta_bias"],
+                                  delta_softplus=w.softplus, **kw)
+            for g in groups]
 
 
 def _calibrate_oracle(inp, w) -> float:
@@ -336,20 +347,68 @@ def oracle_timing(inp, w, seconds: float, steps: int = 1, warmup: int = 0):
     return gbs, ups, ch, threads, total
 
 
-def sample_max_norm_err(y, inp, w, channels: int) -> float:
+def sample_max_norm_err(y, inp, w, channels: int, **oracle_kw) -> float:
     """max |y - y_oracle| / max |y_oracle| over the first `channels`
-    channels of the batch (fp64 oracle on the same inputs)."""
-    import oracle
+    channels of the batch (fp64 oracle on the same inputs; ``oracle_kw``
+    passes cu_seqlens / trapezoid on)."""
     groups = _oracle_sample_inputs(inp, channels, w)
     worst, scale = 0.0, 0.0
-    for b, g in enumerate(groups):
-        ref = oracle.selective_scan(g["u"], g["delta"], g["A"], g["B"], g["C"],
-                                    D=g["D"], z=g["z"], delta_bias=g["delta_bias"],
-                                    delta_softplus=w.softplus)
+    for b, (g, ref) in enumerate(zip(groups, _run_oracle_groups(groups, w, **oracle_kw))):
         got = y[b:b + 1, :ref.shape[1]].detach().float().cpu().double().numpy()
         worst = max(worst, float(np.abs(got - ref).max()))
         scale = max(scale, float(np.abs(ref).max()))
     return worst / scale if scale > 0 else worst
+
+
+def all_elements_error(y, inp, w, block: int = 512) -> dict:
+    """Error statistics of y against the oracle on every element (the
+    oracle run a block of channels of one batch row at a time)."""
+    import oracle
+    from oracle.compare import ErrorStats
+    st = ErrorStats()
+    f = lambda t, b, d0, d1: None if t is None else \
+        t[b:b + 1, d0:d1].detach().float().cpu().double().numpy()
+    c = lambda t, d0, d1: None if t is None else t[d0:d1].detach().float().cpu().double().numpy()
+    for b in range(w.batch):
+        Bh = inp["B"][b:b + 1].detach().float().cpu().double().numpy()
+        Ch = inp["C"][b:b + 1].detach().float().cpu().double().numpy()
+        for d0 in range(0, w.dim, block):
+            d1 = min(w.dim, d0 + block)
+            ref = oracle.selective_scan(f(inp["u"], b, d0, d1), f(inp["delta"], b, d0, d1),
+                                        c(inp["A"], d0, d1), Bh, Ch, D=c(inp["D"], d0, d1),
+                                        z=f(inp["z"], b, d0, d1),
+                                        delta_bias=c(inp["delta_bias"], d0, d1),
+                                        delta_softplus=w.softplus)
+            st.add(f(y, b, d0, d1), ref)
+    return st.summary()
+
+
+def single_thread_oracle(seconds: float = 4.0) -> dict:
+    """The oracle on one core: the whole tiny fp32 workload, and a bounded
+    sample of whole channels of the 130M-shaped layer; GB/s as the sample's
+    share of the workload's algorithmic bytes per second."""
+    import oracle
+    out = {}
+    threads = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        for name in ("tiny-fp32", "mamba130m-layer"):
+            w = workloads.BY_NAME[name]
+            inp = workloads.make_inputs(w, device="cpu")
+            per_ch = _calibrate_oracle(inp, w)
+            ch = int(max(1, min(w.batch * w.dim, round(seconds / 2 / per_ch))))
+            groups = _oracle_sample_inputs(inp, ch, w)
+            t0 = time.perf_counter()
+            _run_oracle_groups(groups, w)
+            secs = time.perf_counter() - t0
+            share = ch / (w.batch * w.dim)
+            out[name] = {"value": w.algorithmic_bytes() * share / secs / 1e9, "unit": "GB/s",
+                         "state_updates_per_s": w.state_updates * share / secs,
+                         "cores": 1, "sample": f"{ch} of {w.batch * w.dim} channels, "
+                                               f"full length L={w.seqlen}, {secs:.2f} s"}
+    finally:
+        oracle.set_num_threads(threads)
+    return out
 
 
 def ssd_sample_max_norm_err(y, inp, w) -> float:
@@ -502,7 +561,37 @@ def run_bwd(args, rank, world, local_rank):
         "kernel_source_hash": kernel_source_hash("bwd"),
     }
     if rank == 0:
+        try:
+            line["max_norm_err"] = bwd_row_max_norm_err(sss, inp, dy, w, ws, ck)
+            line["max_norm_err_sample"] = ("batch row 0: du, ddelta, dz, dB, dC vs the fp64 "
+                                           "oracle backward (max over the five)")
+        except Exception as ex:  # reported, never fatal to the timing line
+            print(f"parity sample failed: {ex}", file=sys.stderr)
         print(json.dumps(line), flush=True)
+
+
+def bwd_row_max_norm_err(sss, inp, dy, w, ws, ck) -> float:
+    """The backward's per-row gradients of batch row 0 against the oracle
+    backward of that row alone (dA, dD, ddelta_bias sum over all rows and
+    are left to the tests)."""
+    import oracle
+    g = sss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy,
+                               D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
+                               delta_softplus=w.softplus, workspace=ws, checkpoints=ck)
+    torch.cuda.synchronize()
+    row = lambda t: None if t is None else t[:1].detach().float().cpu().double().numpy()
+    par = lambda t: None if t is None else t.detach().float().cpu().double().numpy()
+    ref = oracle.selective_scan_bwd(row(inp["u"]), row(inp["delta"]), par(inp["A"]),
+                                    row(inp["B"]), row(inp["C"]), row(dy), D=par(inp["D"]),
+                                    z=row(inp["z"]), delta_bias=par(inp["delta_bias"]),
+                                    delta_softplus=w.softplus)
+    worst = 0.0
+    for k in ("du", "ddelta", "dz", "dB", "dC"):
+        if ref[k] is None:
+            continue
+        got = g[k][:1].cpu().double().numpy()
+        worst = max(worst, float(np.abs(got - ref[k]).max() / np.abs(ref[k]).max()))
+    return worst
 
 
 def decode_algorithmic_bytes(batch, dim, dstate, in_bytes) -> int:
@@ -573,7 +662,143 @@ def run_decode(args, rank, world, local_rank):
         "kernel_source_hash": kernel_source_hash("decode"),
     }
     if rank == 0:
+        try:
+            import oracle
+            h = lambda t: t.detach().float().cpu().double().numpy()
+            st0 = state.clone()
+            s_ref, y_ref = oracle.selective_state_update(
+                h(st0), h(x), h(dtv), h(A), h(B), h(C), D=h(Dv), z=h(z), dt_bias=h(bias))
+            yv = sss.selective_state_update(st0, x, dtv, A, B, C, D=Dv, z=z, dt_bias=bias)
+            torch.cuda.synchronize()
+            line["max_norm_err"] = max(
+                float(np.abs(h(yv) - y_ref).max() / np.abs(y_ref).max()),
+                float(np.abs(h(st0) - s_ref).max() / np.abs(s_ref).max()))
+            line["max_norm_err_sample"] = "one more step, every y and state element"
+        except Exception as ex:  # reported, never fatal to the timing line
+            print(f"parity sample failed: {ex}", file=sys.stderr)
         print(json.dumps(line), flush=True)
+
+
+# measured on this machine's B200s with the library's own probes: results per
+# clock per SM of ex2.approx alone, and of the best mix of ex2.approx with
+# the FMA-pipe polynomial exp2 (three on the special-function unit to one
+# polynomial)
+SFU_PER_CLK_SM = 16.0
+EXP_MIX_PER_CLK_SM = 20.5
+L2_BYTES = 126 * 1024 * 1024
+
+
+def exp_unit_bound(w, kernel_ms: float, sm_mhz: float) -> dict:
+    """The special-function-unit roofline of one scan: one ex2 per state
+    update plus the softplus ex2 and the silu ex2 and reciprocal per
+    (b, d, t), against 16 per clock per SM; and the exponentials alone
+    against the measured rate of the best special-function / FMA-pipe mix
+    (the ceiling if part of the decays moved to the polynomial)."""
+    ops = sfu_ops_per_step(w)
+    clk = sm_mhz * 1e6
+    sfu_peak = SFU_PER_CLK_SM * 148 * clk / 1e12
+    mix_peak = EXP_MIX_PER_CLK_SM * 148 * clk / 1e12
+    achieved = ops / (kernel_ms * 1e-3) / 1e12
+    exps = w.state_updates / (kernel_ms * 1e-3) / 1e12
+    return {"achieved": achieved, "peak": sfu_peak, "unit": "Tops/s",
+            "frac": achieved / sfu_peak, "algorithmic_ops_per_launch": ops,
+            "peak_source": ("derived: 16 special-function results per clock per SM "
+                            "(measured) x 148 SMs x the sampled SM clock"),
+            "decay_exps_per_s": exps * 1e12,
+            "frac_of_exp_mix": exps / mix_peak,
+            "exp_mix_peak": mix_peak,
+            "exp_mix_source": ("derived: 20.5 exponentials per clock per SM measured for "
+                               "3 ex2.approx : 1 FMA-pipe polynomial, x 148 SMs x clock")}
+
+
+def _scan_setup(sss, w, inp, dev, out_dtype="f32", varlen=0, trapezoid=False,
+                checkpoints=False):
+    ydt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    y = torch.empty((w.batch, w.dim, w.seqlen), dtype=ydt, device=dev)
+    ck = sss.scan_checkpoints(w.batch, w.dim, w.dstate, w.seqlen, dev) if checkpoints else None
+    cu_t = None
+    if varlen > 0:
+        cu_t = torch.tensor(varlen_offsets(w.seqlen, varlen), dtype=torch.int32, device=dev)
+    sargs = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                               D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
+                               delta_softplus=w.softplus, y=y, cu_seqlens=cu_t,
+                               trapezoid=trapezoid, checkpoints=ck)
+    ws_bytes = sss.scan_workspace_size(sargs)
+    ws = sss.alloc_workspace(ws_bytes, dev)
+    if ws is not None:
+        sargs.workspace = ws.data_ptr()
+        sargs.workspace_bytes = ws_bytes
+    return dict(y=y, ck=ck, cu=cu_t, args=sargs, ws=ws)
+
+
+def _timed(step, stream, steps, flush=None):
+    """Per-step CUDA events around `steps` calls (an L2 flush between them,
+    outside the events, when given); returns (total ms from the first to
+    the last event, mean ms per step inside the events)."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for a, b in ev:
+        if flush is not None:
+            flush.add_(1)
+        a.record(stream)
+        step()
+        b.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    return t_start.elapsed_time(t_end), sum(a.elapsed_time(b) for a, b in ev) / steps
+
+
+def per_config(args, dev, sss, rank, sm_mhz) -> dict:
+    """Every named workload timed for a short run (inputs resident; an L2
+    flush between steps for workloads that fit in L2), with its HBM and
+    exponential-unit fractions and its error against the oracle on the
+    first 64 channels."""
+    lib = sss.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    peak, _ = measured_peaks()
+    out = {}
+    flush = None
+    for w in workloads.WORKLOADS:
+        inp = workloads.make_inputs(w, device=dev)
+        st = _scan_setup(sss, w, inp, dev)
+        argp = ctypes.byref(st["args"])
+        nbytes = w.algorithmic_bytes()
+        small = nbytes < 2 * L2_BYTES
+        if small and flush is None:
+            flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+
+        def step():
+            rc = lib.mamba_selective_scan_fwd(argp, sh)
+            if rc != 0:
+                raise sss.MssError(rc, "mamba_selective_scan_fwd")
+
+        _, warm_ms = _timed(step, stream, 3, flush if small else None)
+        steps = int(min(300, max(10, round(150.0 / max(warm_ms, 1e-3)))))
+        _, kms = _timed(step, stream, steps, flush if small else None)
+        if lib.mss_scan_status(argp, sh) != 0:
+            raise RuntimeError(f"device-side status error ({w.name})")
+        entry = {"ms_per_step": kms, "steps": steps,
+                 "value": nbytes / (kms * 1e-3) / 1e9, "unit": "GB/s",
+                 "hbm_frac": nbytes / (kms * 1e-3) / 1e9 / peak,
+                 "state_updates_per_s": w.state_updates / (kms * 1e-3),
+                 "exp_unit_frac": exp_unit_bound(w, kms, sm_mhz)["frac"],
+                 "l2": ("flushed between steps (256 MB write)" if small
+                        else "inputs+outputs larger than L2, no flush"),
+                 "sequence_split": sss.scan_workspace_size(st["args"]) > 0}
+        if rank == 0:
+            try:
+                entry["max_norm_err"] = sample_max_norm_err(st["y"], inp, w, 64)
+                entry["max_norm_err_sample"] = "first 64 channels, full length"
+            except Exception as ex:  # reported, never fatal to the timing
+                print(f"parity sample failed ({w.name}): {ex}", file=sys.stderr)
+        out[w.name] = entry
+        del inp, st
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -582,25 +807,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = workloads.BY_NAME[args.workload]
     inp = workloads.make_inputs(w, device=dev)
-    ydt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
-    y = torch.empty((w.batch, w.dim, w.seqlen), dtype=ydt, device=dev)
-    ck = None
-    if args.checkpoints:
-        ck = sss.scan_checkpoints(w.batch, w.dim, w.dstate, w.seqlen, dev)
-    cu_t = None
-    if args.varlen > 0:
-        cu_t = torch.tensor(varlen_offsets(w.seqlen, args.varlen),
-                            dtype=torch.int32, device=dev)
-    sargs = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"],
-                               inp["C"], D=inp["D"], z=inp["z"],
-                               delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, y=y, cu_seqlens=cu_t,
-                               trapezoid=args.trapezoid, checkpoints=ck)
-    ws_bytes = sss.scan_workspace_size(sargs)
-    ws = sss.alloc_workspace(ws_bytes, dev)
-    if ws is not None:
-        sargs.workspace = ws.data_ptr()
-        sargs.workspace_bytes = ws_bytes
+    st = _scan_setup(sss, w, inp, dev, args.out_dtype, args.varlen, args.trapezoid,
+                     args.checkpoints)
+    y, ck, cu_t, ws, sargs = st["y"], st["ck"], st["cu"], st["ws"], st["args"]
     lib = sss.load_library()
     stream = torch.cuda.current_stream(dev)
     sh = ctypes.c_void_p(stream.cuda_stream)
@@ -618,25 +827,13 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device-side status error during warm-up")
 
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
     barrier(world)
     torch.cuda.synchronize(dev)
     clocks.start()
-    t_start.record(stream)
-    for i in range(K):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
+    local_ms, kernel_ms = _timed(step, stream, K)
     clocks.stop()
     barrier(world)
-    local_ms = t_start.elapsed_time(t_end)
-    kernel_ms = sum(a.elapsed_time(b) for a, b in ev) / K
     max_ms = reduce_max(local_ms, world)
     max_kernel_ms = reduce_max(kernel_ms, world)
     if lib.mss_scan_status(argp, sh) != 0:
@@ -683,22 +880,38 @@ def run_ours(args, rank, world, local_rank):
                "sample": (f"{ch} of {w.batch * w.dim} channels, full length "
                           f"L={w.seqlen}, one pass, {total:.1f} s wall, "
                           "fp64 C oracle with OpenMP over channels; GB/s = the "
-                          "sample's share of the step's algorithmic bytes / time")}
+                          "sample's share of the step's algorithmic bytes / time"),
+               "single_thread": single_thread_oracle()}
 
-    # ---- parity of the timed output on a sample, against the fp64 oracle
-    err = None
-    if rank == 0 and not args.varlen and not args.trapezoid:
+    # ---- parity of the timed output against the fp64 oracle
+    err, parity = None, None
+    okw = {}
+    if args.varlen:
+        okw["cu_seqlens"] = varlen_offsets(w.seqlen, args.varlen)
+    if args.trapezoid:
+        okw["trapezoid"] = True
+    if rank == 0 and args.parity != "none":
         try:
-            err = sample_max_norm_err(y, inp, w, 64)
+            if args.parity == "all" and not okw:
+                parity = all_elements_error(y, inp, w)
+                parity["sample"] = "every output element, vs the fp64 oracle"
+                err = parity["max_norm_err"]
+            else:
+                err = sample_max_norm_err(y, inp, w, 64, **okw)
+                parity = {"max_norm_err": err,
+                          "sample": "first 64 channels, full length, vs the fp64 oracle"}
         except Exception as ex:  # reported, never fatal to the timing line
-            print(f"parity sample failed: {ex}", file=sys.stderr)
+            print(f"parity check failed: {ex}", file=sys.stderr)
+    del inp, st, host, y_host
+    torch.cuda.empty_cache()
 
     peak, peak_kind = measured_peaks()
     achieved = bytes_step / (max_kernel_ms * 1e-3) / 1e9
     clk = clocks.summary()
     sm_mhz = clk.get("sm_mhz") or 1965.0
-    sfu_ops = sfu_ops_per_step(w)
-    sfu_peak = 16 * 148 * sm_mhz * 1e6 / 1e12
+    pcfg = None
+    if not args.no_per_config and not (args.varlen or args.trapezoid or args.checkpoints):
+        pcfg = per_config(args, dev, sss, rank, sm_mhz)
     line = {
         "metric": METRIC,
         "value": value,
@@ -718,24 +931,21 @@ def run_ours(args, rank, world, local_rank):
                        **({"writes_checkpoints": True} if args.checkpoints else {})),
         "state_updates_per_s": updates,
         "max_norm_err": err,
-        "max_norm_err_sample": ("first 64 channels, full length, vs the fp64 oracle"
-                                if err is not None else None),
+        "parity": parity,
         "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": value / world / peak,
-        # the bound that binds: the special-function unit (one ex2 per state
-        # update, plus ex2 for softplus and ex2 + rcp for silu per element)
-        "roofline": {"bound": "alu", "achieved": sfu_ops / (max_kernel_ms * 1e-3) / 1e12,
-                     "peak": sfu_peak, "unit": "Tops/s",
-                     "frac": sfu_ops / (max_kernel_ms * 1e-3) / 1e12 / sfu_peak,
-                     "peak_source": ("derived: 16 special-function results per clock "
-                                     "per SM (measured) x 148 SMs x the sampled SM clock"),
-                     "traffic": profiled_traffic(w.name),
-                     "algorithmic_ops_per_launch": sfu_ops,
+        # the metric's roofline: algorithmic HBM bytes per launch over the
+        # kernel's own time (per-step events on the launching stream)
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind,
+                     "traffic": (profiled_traffic(w.name)
+                                 if not (args.varlen or args.trapezoid or args.checkpoints
+                                         or args.out_dtype != "f32") else None),
+                     "algorithmic_bytes_per_launch": bytes_step,
                      "kernel_ms": max_kernel_ms},
-        # the metric's own roofline: algorithmic HBM bytes
-        "hbm": {"achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_source": peak_kind,
-                "algorithmic_bytes_per_launch": bytes_step},
+        # the bound that binds this scan: the special-function unit (one
+        # ex2 per state update)
+        "exp_unit": exp_unit_bound(w, max_kernel_ms, sm_mhz),
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke},
         "gpu_launches": K,
@@ -743,6 +953,8 @@ def run_ours(args, rank, world, local_rank):
                    "reasons": clk["reasons"], "samples": clk["samples"]},
         "kernel_source_hash": kernel_source_hash("fwd"),
     }
+    if pcfg is not None:
+        line["per_config"] = pcfg
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line

@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 7
+#define MSS_ABI_VERSION 8
 
 typedef enum {
   MSS_OK = 0,
@@ -205,10 +205,22 @@ mss_status mss_scan_status(const mss_scan_args *args, void *stream);
  * calls share the one array and its flags are cleared on the caller's stream
  * at the start of each call: two calls whose work overlaps on the GPU (on
  * different streams, or from different threads) race and must not be
- * issued.  A bounded device-side wait that runs out is recorded inside the
- * array and not reported; results are then unspecified. */
+ * issued.  A bounded device-side wait that runs out is recorded in a status
+ * word (inside the array for a split plan) and y is then unspecified;
+ * mss_scan_noalloc_status reports it.  mss_scan_status does not apply to
+ * these calls: it reads args->workspace, which this entry point never
+ * writes. */
 mss_status mamba_selective_scan_fwd_noalloc(const mss_scan_args *args,
                                            void *stream);
+
+/* Synchronises `stream`, then reports the device-side status of
+ * mamba_selective_scan_fwd_noalloc calls with these arguments' plan:
+ * MSS_ERR_TIMEOUT if a bounded wait ran out.  For a split plan it reads the
+ * status word at the start of the library's array, which each such call
+ * clears when it starts (so call this before the next one); otherwise the
+ * library's own word, as mss_scan_status does.  The word read is cleared.
+ * Like the scan, it allocates nothing.  The pages have no counterpart. */
+mss_status mss_scan_noalloc_status(const mss_scan_args *args, void *stream);
 
 /* Arguments of one decode step.  Shapes:
  *   state            (batch, dim, dstate) fp32, updated in place

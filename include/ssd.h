@@ -42,8 +42,9 @@
  * factors that stay below 1 only for A <= 0.
  * Supported here: in_dtype MSS_BF16, headdim 64, dstate 128 (other valid
  * sizes return MSS_ERR_UNSUPPORTED).  x, B, C, z and y must be 16-byte
- * aligned; every other pointer 4-byte aligned.  Outputs must not overlap
- * inputs.
+ * aligned, dt 2-byte aligned (its bf16 elements), and the fp32 pointers
+ * (A, D, dt_bias, h0, last_state) 4-byte aligned.  Outputs must not
+ * overlap inputs.
  *
  * Ownership and streams as in selective_scan.h: device pointers owned by
  * the caller, nothing allocated, work enqueued on `stream` (a cudaStream_t
@@ -95,8 +96,11 @@ mss_status mamba2_ssd_fwd(const mss_ssd_args *args, void *stream);
 
 /* Synchronises `stream` and returns the SSD kernels' device status word
  * (MSS_OK or MSS_ERR_TIMEOUT), clearing it.  The word is the library's own
- * (one per device), so it reports every SSD call on this device since the
- * previous read, on any stream. */
+ * (one per device): it covers every SSD call on this device that has
+ * completed since the previous read.  Only `stream` is synchronised, so a
+ * call still running on another stream is covered only once it has
+ * completed (synchronise that stream, or the device, first); such a call
+ * can also record its status after this read. */
 mss_status mss_ssd_status(void *stream);
 
 #ifdef __cplusplus

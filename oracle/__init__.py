@@ -75,6 +75,8 @@ def _bind(lib):
     lib.oracle_ssd_scan_f64.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
     return lib
 
 
@@ -192,6 +194,12 @@ def selective_state_update(state, x, dt, A, B, C, D=None, z=None,
 def num_threads(lib=None) -> int:
     lib = lib or load()
     return int(lib.oracle_num_threads())
+
+
+def set_num_threads(n: int, lib=None) -> None:
+    """Threads of later oracle calls (e.g. 1 to time it on one core)."""
+    lib = lib or load()
+    lib.oracle_set_num_threads(int(n))
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,

@@ -112,6 +112,10 @@ int oracle_ssd_scan_f64(int64_t batch, int64_t seqlen, int64_t nheads,
 /* Number of OpenMP threads the scan uses (1 when built without OpenMP). */
 int oracle_num_threads(void);
 
+/* Sets the number of OpenMP threads later calls use (n >= 1; for timing
+ * the oracle on one core).  No effect when built without OpenMP. */
+void oracle_set_num_threads(int n);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,7 +25,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 7  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 8  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -43,6 +43,7 @@ EXPORTED_SYMBOLS = (
     "mamba_selective_scan_fwd",
     "mss_scan_status",
     "mamba_selective_scan_fwd_noalloc",
+    "mss_scan_noalloc_status",
     "selective_state_update",
     "mss_scan_bwd_workspace_size",
     "mamba_selective_scan_bwd",
@@ -176,6 +177,8 @@ def load_library():
             lib.mss_scan_status.restype = ctypes.c_int
             lib.mamba_selective_scan_fwd_noalloc.argtypes = [P(ScanArgs), ctypes.c_void_p]
             lib.mamba_selective_scan_fwd_noalloc.restype = ctypes.c_int
+            lib.mss_scan_noalloc_status.argtypes = [P(ScanArgs), ctypes.c_void_p]
+            lib.mss_scan_noalloc_status.restype = ctypes.c_int
             lib.selective_state_update.argtypes = [P(UpdateArgs), ctypes.c_void_p]
             lib.selective_state_update.restype = ctypes.c_int
             lib.mss_scan_bwd_workspace_size.argtypes = [P(ScanBwdArgs), P(ctypes.c_size_t)]

@@ -490,3 +490,24 @@ extern "C" mss_status mamba_selective_scan_fwd_noalloc(const mss_scan_args *a,
     return MSS_ERR_CUDA;
   return MSS_OK;
 }
+
+extern "C" mss_status mss_scan_noalloc_status(const mss_scan_args *a, void *stream) {
+  mss_status st = check_scan_args(a);
+  if (st != MSS_OK) return st;
+  Plan pl;
+  st = make_plan(a, &pl);
+  if (st != MSS_OK) return st;
+  if (pl.workspace > kNoAllocScratchBytes) return MSS_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MSS_ERR_CUDA;
+  // unsplit plans report into the library's own word, split plans into the
+  // word at the start of the array; both are read and cleared here
+  unsigned *w = pl.splits > 1 ? static_cast<unsigned *>(noalloc_scratch_address())
+                              : scan_status_word();
+  if (!w) return MSS_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, w, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(w, 0, sizeof(word)) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  return (word & kStatusTimeout) ? MSS_ERR_TIMEOUT : MSS_OK;
+}

@@ -23,8 +23,9 @@
 // The phases run in different warps at the same time: the scan warps (one
 // per group of 4 states) do nothing but the recurrence, while four auxiliary
 // warps issue the copies, prep block i+2 and finish block i.  Tiles and y
-// shares are double buffered and handed over through named barriers, so the
-// special-function work of prep and epilogue overlaps the recurrence.
+// shares are double buffered and handed over through mbarriers (every wait
+// bounded), so the special-function work of prep and epilogue overlaps the
+// recurrence.
 //
 // Long sequences with few channels are split into chunks that run in
 // parallel ("The relay": fade-and-add steps compose associatively, so a

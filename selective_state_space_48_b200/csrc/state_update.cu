@@ -1,9 +1,11 @@
 // state_update.cu -- single-token selective state update (decode).
 //
-// "Each new token is a cheap state update" (page "Mamba: The State Space
-// Models Challenging the Transformer", section "What a state space model
-// actually is"): one step of h = exp(Delta A) h + Delta B x with readout
-// y = C h + D x, gated by silu(z).  The step is bound by reading and writing
+// Decoding advances the recurrence by one token: the fixed-size state is
+// read, updated once and written back, whatever the length of the context
+// before it (page "Mamba: The State Space Models Challenging the
+// Transformer", section "What a state space model actually is").  One step
+// of h = exp(Delta A) h + Delta B x with readout y = C h + D x, gated by
+// silu(z).  The step is bound by reading and writing
 // the fp32 state (8 * dstate bytes per channel), so one thread owns one
 // channel (b, d) and moves its state with 16-byte vector loads and stores.
 #include <cuda_bf16.h>

@@ -15,6 +15,7 @@ import torch
 
 import oracle
 import selective_state_space_48_b200 as sss
+from oracle.compare import ErrorStats
 import workloads
 
 TOL_F32 = 1e-4
@@ -66,30 +67,46 @@ def run_oracle(w, inp, return_last_state=False):
         return_last_state=return_last_state)
 
 
-def sampled_channels(w, count=24, seed=0):
-    """(b, d) pairs spread over the tensor: first, last, tile edges, random."""
-    rng = np.random.default_rng(seed)
-    picks = {(0, 0), (w.batch - 1, w.dim - 1)}
-    for d in (31, 32, 63, 64):
-        if d < w.dim:
-            picks.add((0, d))
-    while len(picks) < min(count, w.batch * w.dim):
-        picks.add((int(rng.integers(w.batch)), int(rng.integers(w.dim))))
-    return sorted(picks)
+# ---------------------------------------------------------------- full size
+#
+# Full-size workloads are compared element by element: the oracle runs on
+# every channel, a block of channels of one batch row at a time (so host
+# memory stays bounded), and each block of the GPU output is compared with
+# it.  The error is normalised by the largest |y_oracle| over the whole
+# output, as everywhere else.
 
 
-def oracle_on_channels(w, inp, picks):
-    """Run the oracle only on the sampled channels (full length)."""
-    out = {}
-    for b, d in picks:
-        sl = lambda t: None if t is None else t[b:b + 1, d:d + 1].detach().cpu().double().numpy()
-        bc = lambda t: t[b:b + 1].detach().cpu().double().numpy()
-        pd = lambda t: None if t is None else t[d:d + 1].detach().cpu().double().numpy()
-        h0 = inp.get("h0")
-        y = oracle.selective_scan(
-            sl(inp["u"]), sl(inp["delta"]), pd(inp["A"]), bc(inp["B"]),
-            bc(inp["C"]), D=pd(inp["D"]), z=sl(inp["z"]),
-            delta_bias=pd(inp["delta_bias"]), delta_softplus=w.softplus,
-            h0=None if h0 is None else h0[b:b + 1, d:d + 1].cpu().double().numpy())
-        out[(b, d)] = y[0, 0]
-    return out
+def _rows(t, b, d0, d1):
+    return None if t is None else t[b:b + 1, d0:d1].detach().float().cpu().double().numpy()
+
+
+def _chan(t, d0, d1):
+    return None if t is None else t[d0:d1].detach().float().cpu().double().numpy()
+
+
+def oracle_blocks(w, inp, block=512, cu_seqlens=None, trapezoid=False):
+    """(b, d0, d1, y_oracle[1, d1-d0, L]) for every block of channels of
+    every batch row, in order."""
+    h0 = inp.get("h0")
+    for b in range(w.batch):
+        Bh = inp["B"][b:b + 1].detach().float().cpu().double().numpy()
+        Ch = inp["C"][b:b + 1].detach().float().cpu().double().numpy()
+        for d0 in range(0, w.dim, block):
+            d1 = min(w.dim, d0 + block)
+            y = oracle.selective_scan(
+                _rows(inp["u"], b, d0, d1), _rows(inp["delta"], b, d0, d1),
+                _chan(inp["A"], d0, d1), Bh, Ch, D=_chan(inp["D"], d0, d1),
+                z=_rows(inp["z"], b, d0, d1), delta_bias=_chan(inp["delta_bias"], d0, d1),
+                delta_softplus=w.softplus, h0=_rows(h0, b, d0, d1),
+                cu_seqlens=cu_seqlens, trapezoid=trapezoid)
+            yield b, d0, d1, y
+
+
+def compare_all_channels(w, inp, y, block=512, cu_seqlens=None, trapezoid=False):
+    """ErrorStats of the GPU output y (batch, dim, L) against the oracle on
+    every element."""
+    st = ErrorStats()
+    for b, d0, d1, want in oracle_blocks(w, inp, block, cu_seqlens, trapezoid):
+        got = y[b:b + 1, d0:d1].detach().float().cpu().double().numpy()
+        st.add(got, want)
+    return st

@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 7
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 8
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:

@@ -52,9 +52,54 @@ def test_whole_job_throughput_single_rank():
 
 
 def test_bench_workload_bytes_match_the_roofline_table():
+    """The default line is the 1.4B-shaped layer: u, delta, z in bf16 and y
+    in fp32 per (b, d, t), B and C in bf16 per (b, n, t), A, D, delta_bias
+    in fp32."""
     w = workloads.BY_NAME[bench.DEFAULT_WORKLOAD]
-    assert w.algorithmic_bytes() == 252_817_408
-    assert w.state_updates == 402_653_184
+    assert w.name == "mamba1.4b-layer"
+    bdl = 4 * 4096 * 4096
+    assert w.algorithmic_bytes() == bdl * (3 * 2 + 4) + 2 * 4 * 16 * 4096 * 2 + \
+        4096 * 16 * 4 + 4096 * 4 * 2 == 672_432_128
+    assert w.state_updates == bdl * 16 == 1_073_741_824
+    w1 = workloads.BY_NAME["mamba130m-layer"]
+    assert w1.algorithmic_bytes() == 252_817_408 and w1.state_updates == 402_653_184
+
+
+def test_exp_unit_bound_by_hand():
+    """One ex2 per state update plus softplus (1) and silu (2) per (b, d, t),
+    against 16 per clock per SM x 148 SMs."""
+    w = workloads.BY_NAME["mamba130m-layer"]
+    b = bench.exp_unit_bound(w, 0.1, 2000.0)
+    ops = 402_653_184 + 3 * 8 * 1536 * 2048
+    assert b["algorithmic_ops_per_launch"] == ops
+    assert abs(b["peak"] - 16 * 148 * 2e9 / 1e12) < 1e-9
+    assert abs(b["frac"] - ops / 1e-4 / (16 * 148 * 2e9)) < 1e-9
+    assert abs(b["frac_of_exp_mix"] - 402_653_184 / 1e-4 / (20.5 * 148 * 2e9)) < 1e-9
+
+
+def test_all_elements_error_on_cpu():
+    """The bench's every-element parity: the oracle's own output gives only
+    the fp32 rounding of y; one perturbed element shows up exactly."""
+    import numpy as np
+    import oracle
+    w = workloads.custom(2, 40, 4, 50, in_dtype="bf16", has_z=True)
+    inp = workloads.make_inputs(w, seed=9)
+    h = workloads.to_numpy_f64(inp)
+    ref = oracle.selective_scan(h["u"], h["delta"], h["A"], h["B"], h["C"], D=h["D"],
+                                z=h["z"], delta_bias=h["delta_bias"])
+    y = torch.from_numpy(ref.copy()).float()
+    st = bench.all_elements_error(y, inp, w, block=16)
+    assert st["elements"] == 2 * 40 * 50 and st["max_norm_err"] <= 2.0 ** -24
+    y[1, 33, 7] += 0.25
+    st = bench.all_elements_error(y, inp, w, block=16)
+    assert abs(st["max_norm_err"] - 0.25 / np.abs(ref).max()) <= 2.0 ** -22
+
+
+def test_single_thread_oracle_timing_reports_one_core():
+    res = bench.single_thread_oracle(seconds=0.2)
+    assert set(res) == {"tiny-fp32", "mamba130m-layer"}
+    for r in res.values():
+        assert r["cores"] == 1 and r["value"] > 0
 
 
 def test_reference_arm_prints_the_contract_line(capsys):

@@ -15,6 +15,7 @@ import torch
 import oracle
 import selective_state_space_48_b200 as sss
 import workloads
+from oracle.compare import ErrorStats
 from scan_checks import gpu_inputs, norm_err
 
 pytestmark = pytest.mark.gpu
@@ -87,3 +88,50 @@ def test_backward_of_the_last_state_alone():
     dy = torch.zeros(1, 32, 160, device="cuda")
     d_last = torch.randn(1, 32, 16, device="cuda")
     _compare(*_grads(w, inp, dy, d_last), "last state only")
+
+
+def _full_tolerance(terms: int) -> float:
+    """Bound for a gradient that the GPU accumulates as an fp32 sum of
+    `terms` contributions (atomics over channels or over (batch row, step)):
+    recursive summation errs by at most (terms - 1) u of the sum of the
+    magnitudes (u = 2^-24), on top of the fp32 recurrence's own 1e-4."""
+    return TOL + terms * 2.0 ** -24
+
+
+def test_backward_at_the_130m_layer_shape_every_element():
+    """The backward at the shape `bench.py --pass bwd` times (Mamba-130M
+    layer: batch 8, D 1536, N 16, L 2048, bf16 inputs): every element of
+    all gradients against the oracle backward, run one batch row at a time
+    (dA, dD, ddelta_bias summed over the rows in fp64)."""
+    w = workloads.BY_NAME["mamba130m-layer"]
+    inp = gpu_inputs(w)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(48000)
+    dy = torch.randn(w.batch, w.dim, w.seqlen, generator=g, device="cuda")
+    got = sss.selective_scan_bwd(
+        inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"],
+        z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=w.softplus)
+    torch.cuda.synchronize()
+    host = lambda t, b: None if t is None else t[b:b + 1].detach().float().cpu().double().numpy()
+    par = lambda t: None if t is None else t.detach().float().cpu().double().numpy()
+    sums = {"dA": 0.0, "dD": 0.0, "ddelta_bias": 0.0}
+    stats = {k: ErrorStats() for k in ("du", "ddelta", "dz", "dB", "dC")}
+    for b in range(w.batch):
+        ref = oracle.selective_scan_bwd(
+            host(inp["u"], b), host(inp["delta"], b), par(inp["A"]), host(inp["B"], b),
+            host(inp["C"], b), host(dy, b), D=par(inp["D"]), z=host(inp["z"], b),
+            delta_bias=par(inp["delta_bias"]), delta_softplus=w.softplus)
+        for k in stats:
+            stats[k].add(got[k][b:b + 1].cpu().numpy(), ref[k])
+        for k in sums:
+            sums[k] = sums[k] + ref[k]
+    errs = {k: st.norm_err for k, st in stats.items()}
+    for k, ref in sums.items():
+        errs[k] = norm_err(got[k].cpu().numpy(), ref)
+    bound = {"du": TOL, "ddelta": TOL, "dz": TOL,
+             "dB": _full_tolerance(w.dim), "dC": _full_tolerance(w.dim),
+             "dA": _full_tolerance(w.batch * w.seqlen),
+             "dD": _full_tolerance(w.batch * w.seqlen),
+             "ddelta_bias": _full_tolerance(w.batch * w.seqlen)}
+    bad = {k: (e, bound[k]) for k, e in errs.items() if not e <= bound[k]}
+    assert not bad, (bad, errs)

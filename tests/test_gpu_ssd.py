@@ -7,14 +7,19 @@ The CUDA path evaluates the same map by 128-step chunks of bf16 matrix
 products with fp32 accumulation, so its tolerance comes from bf16
 rounding, not fp32: the decayed scores S', the weighted inputs X'' and
 the carried state h_prev each enter one product rounded to bf16 (unit
-roundoff u = 2^-8).  Each output sums such rounded terms with independent
-rounding errors, so |y_gpu - y| stays within a small multiple of u times
-the size of y; the bound used is 2.5 u = 9.8e-3 of max |y| (and of max
-|h| for the final state), with another 2^-8 when y itself is stored in
-bf16.  Cases: chunks with a ragged tail, a single short chunk, two groups
-of B and C, no optional inputs with softplus off, an initial state, bf16
-output, a long carry chain, and outputs sampled from the full 2.7B-layer
-shape.
+roundoff u = 2^-8, relative error at most u per operand).  An output is a
+sum of such products whose rounding errors are independent and of either
+sign, so its error is a random sum of per-term errors, each within u of
+its term; for a sum of terms of random sign the error stays below
+u * max |y| except far in the tails.  The bound used is u (rounded up to
+4e-3) of max |y| (and of max |h| for the final state), with another 2^-8
+when y itself is stored in bf16.  tests/test_ssd_chunked_model.py runs the
+same decomposition with the same three roundings in fp64 on the CPU and
+stays at 1.5e-3 to 3.5e-3 on its cases.
+
+Cases: chunks with a ragged tail, a single short chunk, two groups of B
+and C, no optional inputs with softplus off, an initial state, bf16 output,
+a long carry chain, and every element of the full 2.7B-layer shape.
 """
 import numpy as np
 import pytest
@@ -23,12 +28,13 @@ import torch
 import oracle
 import selective_state_space_48_b200 as sss
 import workloads
+from oracle.compare import ErrorStats
 from scan_checks import norm_err
 
 pytestmark = pytest.mark.gpu
 
 U_BF16 = 2.0 ** -8
-TOL = 2.5 * U_BF16
+TOL = 4e-3  # u = 2^-8 = 3.9e-3, rounded up
 
 
 def _oracle(inp, softplus=True, heads=None, batch=None):
@@ -104,19 +110,23 @@ def test_ssd_bf16_output():
     assert norm_err(y.float().cpu().numpy(), y_ref) <= TOL + U_BF16
 
 
-def test_ssd_full_layer_sampled():
-    """The 2.7B-layer shape in the launch configuration the bench times;
-    three heads of one batch row checked against the oracle."""
+def test_ssd_full_layer_every_element():
+    """The 2.7B-layer shape in the launch configuration the bench times,
+    with an initial state: every element of y and of the final state
+    against the oracle (run one batch row at a time)."""
     w = workloads.SSD_BY_NAME["mamba2-2.7b-layer"]
     inp = workloads.make_ssd_inputs(w, seed=5752, device="cuda", h0=True)
     y, last = _run(inp)
     torch.cuda.synchronize()
-    b, heads = 5, [0, 41, w.nheads - 1]
-    y_ref, last_ref = _oracle(inp, heads=heads, batch=b)
-    got = y[b:b + 1, :, heads].cpu().numpy()
-    assert norm_err(got, y_ref) <= TOL
-    assert norm_err(last[b:b + 1, heads].cpu().numpy(), last_ref) <= TOL
     assert torch.isfinite(y).all()
+    sy, sl = ErrorStats(), ErrorStats()
+    for b in range(w.batch):
+        y_ref, last_ref = _oracle(inp, batch=b)
+        sy.add(y[b:b + 1].cpu().numpy(), y_ref)
+        sl.add(last[b:b + 1].cpu().numpy(), last_ref)
+    assert sy.count == y.numel() and sl.count == last.numel()
+    assert sy.norm_err <= TOL, sy.summary()
+    assert sl.norm_err <= TOL, sl.summary()
 
 
 def test_ssd_is_deterministic():

@@ -77,3 +77,15 @@ def test_trapezoid_differs_from_euler():
                                 trapezoid=True, **args)
     torch.cuda.synchronize()
     assert float((y1 - y2).abs().max()) > 1e-3 * float(y1.abs().max())
+
+
+def test_trapezoid_at_the_130m_layer_shape_every_element():
+    """The trapezoidal update at the shape `bench.py --trapezoid` times
+    (Mamba-130M layer, bf16 inputs), every output element against the
+    oracle."""
+    from scan_checks import compare_all_channels, run_gpu
+    w = workloads.BY_NAME["mamba130m-layer"]
+    inp = gpu_inputs(w)
+    y = run_gpu(w, inp, trapezoid=True, check_status=True)
+    st = compare_all_channels(w, inp, y, trapezoid=True)
+    assert st.norm_err <= tolerance(w.in_dtype), st.summary()

@@ -118,3 +118,19 @@ def test_packed_row_equals_separate_scans():
         scale = float(yp.abs().max())
         assert float((y[..., a:b] - yp).abs().max()) <= 1e-6 * scale, (a, b)
     assert float((last - lp).abs().max()) <= 1e-6 * float(lp.abs().max())
+
+
+def test_packed_sequences_at_the_130m_layer_shape_every_element():
+    """Eight packed sequences per row at the shape `bench.py --varlen 8`
+    times (Mamba-130M layer, bf16 inputs; seeded offsets shared by the
+    rows), every output element against the oracle."""
+    from scan_checks import compare_all_channels, run_gpu
+    w = workloads.BY_NAME["mamba130m-layer"]
+    inp = gpu_inputs(w)
+    rng = np.random.default_rng(48008)
+    cuts = rng.choice(np.arange(1, w.seqlen), size=7, replace=False)
+    cu = [0] + sorted(int(c) for c in cuts) + [w.seqlen]
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    y = run_gpu(w, inp, cu_seqlens=cu_t, check_status=True)
+    st = compare_all_channels(w, inp, y, cu_seqlens=cu)
+    assert st.norm_err <= tolerance(w.in_dtype), st.summary()

@@ -78,3 +78,36 @@ def test_noalloc_rejects_plans_beyond_its_array():
     a.plan_splits = 64
     assert sss.scan_workspace_size(a) > (8 << 20)
     assert _call_noalloc(a) == sss.MSS_ERR_WORKSPACE
+
+
+def _noalloc_status(args):
+    lib = sss.load_library()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.mss_scan_noalloc_status(ctypes.byref(args), stream)
+
+
+def test_noalloc_reports_a_timed_out_wait_and_recovers():
+    """A chunk that never publishes its carry (test flag): the successor's
+    bounded wait runs out, mss_scan_noalloc_status reports it from the word
+    in the library's array, and the next call is correct and reports OK."""
+    w = workloads.custom(1, 32, 16, 4096, in_dtype="f32", has_z=False)
+    inp = gpu_inputs(w, seed=2)
+    want = sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"],
+                                  inp["C"], D=inp["D"], delta_bias=inp["delta_bias"],
+                                  plan_splits=4, check_status=True)
+    y = torch.empty_like(want)
+    bad = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                             D=inp["D"], delta_bias=inp["delta_bias"], y=y,
+                             plan_splits=4, test_flags=sss.MSS_TESTFLAG_DROP_PUBLISH,
+                             spin_timeout_ns=20_000_000)
+    assert sss.scan_workspace_size(bad) > 0
+    assert _call_noalloc(bad) == sss.MSS_OK
+    assert _noalloc_status(bad) == sss.MSS_ERR_TIMEOUT
+    # the word was read and cleared
+    assert _noalloc_status(bad) == sss.MSS_OK
+    good = sss.make_scan_args(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                              D=inp["D"], delta_bias=inp["delta_bias"], y=y,
+                              plan_splits=4)
+    assert _call_noalloc(good) == sss.MSS_OK
+    assert _noalloc_status(good) == sss.MSS_OK
+    assert norm_err(y.cpu(), want.cpu()) <= tolerance("f32")
