@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "nvtx_range.cuh"
 #include "scan_bwd.cuh"
 #include "scan_fwd.cuh"
 #include "selective_scan.h"
@@ -221,6 +222,7 @@ mss_status mss_scan_workspace_size(const mss_scan_args *args, size_t *bytes) {
 }
 
 mss_status mamba_selective_scan_fwd(const mss_scan_args *a, void *stream) {
+  NvtxRange range("mamba_selective_scan_fwd");
   mss_status st = check_scan_args(a);
   if (st != MSS_OK) return st;
   Plan pl;
@@ -279,6 +281,7 @@ mss_status mss_scan_status(const mss_scan_args *a, void *stream) {
 }
 
 mss_status selective_state_update(const mss_update_args *a, void *stream) {
+  NvtxRange range("selective_state_update");
   if (!a) return MSS_ERR_INVALID_ARG;
   if (a->batch < 1 || a->dim < 1 || a->dstate < 1) return MSS_ERR_INVALID_ARG;
   if (a->dstate > kMaxStates) return MSS_ERR_UNSUPPORTED;
@@ -360,6 +363,7 @@ mss_status mss_scan_bwd_workspace_size(const mss_scan_bwd_args *a, size_t *bytes
 }
 
 mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
+  NvtxRange range("mamba_selective_scan_bwd");
   size_t need = 0;
   const mss_status st = mss_scan_bwd_workspace_size(a, &need);
   if (st != MSS_OK) return st;
@@ -463,6 +467,7 @@ void *noalloc_scratch_address() {
 
 extern "C" mss_status mamba_selective_scan_fwd_noalloc(const mss_scan_args *a,
                                                        void *stream) {
+  NvtxRange range("mamba_selective_scan_fwd_noalloc");
   mss_status st = check_scan_args(a);
   if (st != MSS_OK) return st;
   Plan pl;

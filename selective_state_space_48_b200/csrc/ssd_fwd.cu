@@ -42,6 +42,7 @@
 #include <mutex>
 
 #include "device_math.cuh"
+#include "nvtx_range.cuh"
 #include "selective_scan.h"
 #include "ssd.h"
 
@@ -818,6 +819,7 @@ mss_status check(const mss_ssd_args *a) {
 using namespace sss48;
 
 extern "C" mss_status mamba2_ssd_fwd(const mss_ssd_args *a, void *stream) {
+  sss48::NvtxRange range("mamba2_ssd_fwd");
   const mss_status st = ssd::check(a);
   if (st != MSS_OK) return st;
   ssd::Maps maps;
