@@ -77,6 +77,21 @@ typedef enum { MSS_F32 = 0, MSS_BF16 = 1 } mss_dtype;
 #define MSS_TESTFLAG_DROP_PUBLISH 0x1u /* one sequence chunk never publishes
                                           its carry, so its successor's
                                           bounded wait must run out         */
+#define MSS_TESTFLAG_DEBUG_OOB 0x2u    /* checked build only: the first y
+                                          store of the first thread block is
+                                          aimed one tensor length past y; the
+                                          bounds check must skip it and
+                                          report MSS_ERR_INVALID_ARG.  No
+                                          effect in the ordinary build.     */
+
+/* Checked build.  Compiling the library with MSS_DEBUG=1 (the builder's
+ * --debug option, libsss48_debug.so) adds a bounds check to every global
+ * access at a computed index in the forward scan, the decode step and the
+ * backward scan.  An index outside its tensor is skipped and recorded in
+ * the device status word; the status calls then return MSS_ERR_INVALID_ARG
+ * (ahead of MSS_ERR_TIMEOUT).  The checks never trap or assert.  Accesses
+ * made by the TMA engine are bounds-checked by the hardware in either
+ * build.  The ordinary build contains none of this code. */
 
 /* Arguments of one forward scan.  Shapes:
  *   u, delta, z, y   (batch, dim, seqlen)   in_dtype (y: out_dtype)
@@ -180,8 +195,10 @@ mss_status mamba_selective_scan_fwd(const mss_scan_args *args, void *stream);
 /* Synchronises `stream`, then reports the device-side status of the last
  * scan with these arguments: for a split scan the status word in
  * args->workspace, otherwise the library's own word, which is read and
- * cleared (so it reports every unsplit scan since the previous call, on any
- * stream of this device). */
+ * cleared (so it reports every unsplit scan, and in the checked build every
+ * decode step, since the previous call, on any stream of this device, once
+ * that work has completed).  MSS_ERR_TIMEOUT: a bounded wait ran out;
+ * MSS_ERR_INVALID_ARG: the checked build skipped an out-of-range access. */
 mss_status mss_scan_status(const mss_scan_args *args, void *stream);
 
 /* The same forward scan for callers that cannot allocate device memory:

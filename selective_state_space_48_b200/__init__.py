@@ -36,6 +36,7 @@ MSS_ERR_WORKSPACE = 5
 MSS_F32 = 0
 MSS_BF16 = 1
 MSS_TESTFLAG_DROP_PUBLISH = 0x1
+MSS_TESTFLAG_DEBUG_OOB = 0x2  # checked build only: one planted out-of-range y store
 
 # every symbol include/selective_scan.h and include/ssd.h declare
 EXPORTED_SYMBOLS = (
@@ -158,47 +159,69 @@ _lib = None
 _lock = threading.Lock()
 
 
+def _bind(lib):
+    P = ctypes.POINTER
+    lib.mss_scan_workspace_size.argtypes = [P(ScanArgs), P(ctypes.c_size_t)]
+    lib.mss_scan_workspace_size.restype = ctypes.c_int
+    lib.mamba_selective_scan_fwd.argtypes = [P(ScanArgs), ctypes.c_void_p]
+    lib.mamba_selective_scan_fwd.restype = ctypes.c_int
+    lib.mss_scan_status.argtypes = [P(ScanArgs), ctypes.c_void_p]
+    lib.mss_scan_status.restype = ctypes.c_int
+    lib.mamba_selective_scan_fwd_noalloc.argtypes = [P(ScanArgs), ctypes.c_void_p]
+    lib.mamba_selective_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.mss_scan_noalloc_status.argtypes = [P(ScanArgs), ctypes.c_void_p]
+    lib.mss_scan_noalloc_status.restype = ctypes.c_int
+    lib.selective_state_update.argtypes = [P(UpdateArgs), ctypes.c_void_p]
+    lib.selective_state_update.restype = ctypes.c_int
+    lib.mss_scan_bwd_workspace_size.argtypes = [P(ScanBwdArgs), P(ctypes.c_size_t)]
+    lib.mss_scan_bwd_workspace_size.restype = ctypes.c_int
+    lib.mamba_selective_scan_bwd.argtypes = [P(ScanBwdArgs), ctypes.c_void_p]
+    lib.mamba_selective_scan_bwd.restype = ctypes.c_int
+    lib.mss_status_string.argtypes = [ctypes.c_int]
+    lib.mss_status_string.restype = ctypes.c_char_p
+    lib.mamba2_ssd_fwd.argtypes = [P(SsdArgs), ctypes.c_void_p]
+    lib.mamba2_ssd_fwd.restype = ctypes.c_int
+    lib.mss_ssd_status.argtypes = [ctypes.c_void_p]
+    lib.mss_ssd_status.restype = ctypes.c_int
+    lib.mss_abi_version.argtypes = []
+    lib.mss_abi_version.restype = ctypes.c_int
+    return lib
+
+
+def _open(path: str):
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"CUDA library {path} is missing; build it with "
+            "`python -m selective_state_space_48_b200.builder`")
+    lib = _bind(ctypes.CDLL(path))
+    if lib.mss_abi_version() != ABI_VERSION:
+        raise RuntimeError(
+            f"{path} has ABI version {lib.mss_abi_version()}, "
+            f"this binding expects {ABI_VERSION}; rebuild it")
+    return lib
+
+
 def load_library():
     """Load libsss48.so (raises if it has not been built)."""
     global _lib
     with _lock:
         if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(
-                    f"CUDA library {LIB_PATH} is missing; build it with "
-                    "`python -m selective_state_space_48_b200.builder`")
-            lib = ctypes.CDLL(LIB_PATH)
-            P = ctypes.POINTER
-            lib.mss_scan_workspace_size.argtypes = [P(ScanArgs), P(ctypes.c_size_t)]
-            lib.mss_scan_workspace_size.restype = ctypes.c_int
-            lib.mamba_selective_scan_fwd.argtypes = [P(ScanArgs), ctypes.c_void_p]
-            lib.mamba_selective_scan_fwd.restype = ctypes.c_int
-            lib.mss_scan_status.argtypes = [P(ScanArgs), ctypes.c_void_p]
-            lib.mss_scan_status.restype = ctypes.c_int
-            lib.mamba_selective_scan_fwd_noalloc.argtypes = [P(ScanArgs), ctypes.c_void_p]
-            lib.mamba_selective_scan_fwd_noalloc.restype = ctypes.c_int
-            lib.mss_scan_noalloc_status.argtypes = [P(ScanArgs), ctypes.c_void_p]
-            lib.mss_scan_noalloc_status.restype = ctypes.c_int
-            lib.selective_state_update.argtypes = [P(UpdateArgs), ctypes.c_void_p]
-            lib.selective_state_update.restype = ctypes.c_int
-            lib.mss_scan_bwd_workspace_size.argtypes = [P(ScanBwdArgs), P(ctypes.c_size_t)]
-            lib.mss_scan_bwd_workspace_size.restype = ctypes.c_int
-            lib.mamba_selective_scan_bwd.argtypes = [P(ScanBwdArgs), ctypes.c_void_p]
-            lib.mamba_selective_scan_bwd.restype = ctypes.c_int
-            lib.mss_status_string.argtypes = [ctypes.c_int]
-            lib.mss_status_string.restype = ctypes.c_char_p
-            lib.mamba2_ssd_fwd.argtypes = [P(SsdArgs), ctypes.c_void_p]
-            lib.mamba2_ssd_fwd.restype = ctypes.c_int
-            lib.mss_ssd_status.argtypes = [ctypes.c_void_p]
-            lib.mss_ssd_status.restype = ctypes.c_int
-            lib.mss_abi_version.argtypes = []
-            lib.mss_abi_version.restype = ctypes.c_int
-            if lib.mss_abi_version() != ABI_VERSION:
-                raise RuntimeError(
-                    f"{LIB_PATH} has ABI version {lib.mss_abi_version()}, "
-                    f"this binding expects {ABI_VERSION}; rebuild it")
-            _lib = lib
+            _lib = _open(LIB_PATH)
     return _lib
+
+
+_debug_lib = None
+
+
+def load_debug_library():
+    """Load the checked build libsss48_debug.so (``builder --debug``): the
+    same entry points with device-side bounds checks that report an access
+    outside its tensor as MSS_ERR_INVALID_ARG through the status calls."""
+    global _debug_lib
+    with _lock:
+        if _debug_lib is None:
+            _debug_lib = _open(_build.DEBUG_LIB_PATH)
+    return _debug_lib
 
 
 def status_string(code: int) -> str:

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "device_math.cuh"
 #include "nvtx_range.cuh"
 #include "scan_bwd.cuh"
 #include "scan_fwd.cuh"
@@ -204,6 +205,19 @@ void fill_scan_params(const mss_scan_args *a, const Plan &pl, ScanParams *p) {
   p->tiles = pl.tiles;
   p->test_flags = a->test_flags;
   p->spin_timeout_ns = a->spin_timeout_ns;
+  auto ext = [&](const int64_t (&st)[2], int64_t rows) {
+    return (a->batch - 1) * st[0] + (rows - 1) * st[1] + a->seqlen;
+  };
+  p->ext_u = ext(p->su, a->dim);
+  p->ext_delta = ext(p->sdl, a->dim);
+  p->ext_z = ext(p->sz, a->dim);
+  p->ext_B = ext(p->sB, a->dstate);
+  p->ext_C = ext(p->sC, a->dstate);
+  p->ext_y = ext(p->sy, a->dim);
+  p->ext_ckpt = a->checkpoints
+                    ? static_cast<int64_t>(scan_bwd_workspace_bytes(pl.tiles, a->seqlen, a->dstate) /
+                                           sizeof(float))
+                    : 0;
 }
 
 }  // namespace
@@ -276,6 +290,7 @@ mss_status mss_scan_status(const mss_scan_args *a, void *stream) {
         cudaSuccess)
       return MSS_ERR_CUDA;
   }
+  if (word & kStatusBadIndex) return MSS_ERR_INVALID_ARG;
   if (word & kStatusTimeout) return MSS_ERR_TIMEOUT;
   return MSS_OK;
 }
@@ -311,6 +326,8 @@ mss_status selective_state_update(const mss_update_args *a, void *stream) {
   p.dt_bias = a->dt_bias;
   p.softplus = a->dt_softplus ? 1 : 0;
   p.y = a->y;
+  p.status = scan_status_word();
+  if (!p.status) return MSS_ERR_CUDA;
   if (launch_state_update(p, a->in_dtype == MSS_BF16, a->out_dtype == MSS_BF16,
                           static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSS_ERR_CUDA;
@@ -401,6 +418,8 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   p.ckpt_given = a->checkpoints ? 1 : 0;
   p.ch_tiles = static_cast<int>((a->dim + kBwdChannels - 1) / kBwdChannels);
   p.tiles = a->batch * p.ch_tiles;
+  p.status = scan_status_word();
+  if (!p.status) return MSS_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the gradients that are sums over blocks are accumulated with atomics
   const size_t f = sizeof(float);
@@ -514,5 +533,6 @@ extern "C" mss_status mss_scan_noalloc_status(const mss_scan_args *a, void *stre
   if (cudaMemcpy(&word, w, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemset(w, 0, sizeof(word)) != cudaSuccess)
     return MSS_ERR_CUDA;
+  if (word & kStatusBadIndex) return MSS_ERR_INVALID_ARG;
   return (word & kStatusTimeout) ? MSS_ERR_TIMEOUT : MSS_OK;
 }

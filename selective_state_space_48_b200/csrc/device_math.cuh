@@ -7,7 +7,34 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#ifndef MSS_DEBUG
+#define MSS_DEBUG 0
+#endif
+
 namespace sss48 {
+
+// Device status bits (read by the status entry points): a bounded wait
+// that ran out, and (checked builds only) an access outside its tensor.
+constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusBadIndex = 2u;
+
+// Bounds check of a global access at element index i of a tensor with n
+// elements.  In builds with MSS_DEBUG=1 an index outside [0, n) is
+// recorded in *status (kStatusBadIndex) and false is returned, so the
+// caller skips the access; no trap, no assert.  In ordinary builds it is
+// always true and generates no code.
+__device__ __forceinline__ bool dbg_index_ok(int64_t i, int64_t n, unsigned *status) {
+#if MSS_DEBUG
+  if (i >= 0 && i < n) return true;
+  if (status) atomicOr(status, kStatusBadIndex);
+  return false;
+#else
+  (void)i;
+  (void)n;
+  (void)status;
+  return true;
+#endif
+}
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

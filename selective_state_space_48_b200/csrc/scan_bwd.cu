@@ -11,20 +11,27 @@
 //   forward sweep  walks the sequence in 16-step blocks and writes the state
 //                  at the start of every block to the workspace (the only
 //                  state that touches HBM: 64 B per channel and block);
-//   reverse sweep  walks the blocks backwards; for each it reloads the inputs,
-//                  recomputes the states of one half block (8 steps) from
-//                  the checkpoint into registers, runs the adjoint
+//   reverse sweep  walks the blocks backwards; for each, the later half
+//                  (8 steps) first: recompute the states from the block's
+//                  checkpoint, keeping each step's state and decay a_t of the
+//                  half in registers, then run the adjoint
 //                  lam_t = ds_t C_t + a_{t+1} lam_{t+1} backwards over them
-//                  (re-evaluating each decay a_t), then does the same for
-//                  the other half.
+//                  with the kept decays (no exponential is evaluated twice
+//                  within a half); then the earlier half the same way.
+//
+// The arithmetic pairs the lane's states: two states advance together in
+// one f32x2 instruction, so B_t and C_t sit in shared memory step-major
+// ([t][n]) and a warp reads the four values of its states with one
+// warp-uniform 16-byte load.
 //
 // With s_t = sum_n C_t[n] h_t[n] + D u_t, g_t = silu(z_t) and y_t = s_t g_t,
-// ds_t = dy_t g_t:
-//   dDelta_t = sum_n lam_t[n] (A[n] a_t[n] h_{t-1}[n] + B_t[n] u_t)
-//   dA[n]   += lam_t[n] Delta_t a_t[n] h_{t-1}[n]
-//   dB_t[n] += lam_t[n] Delta_t u_t       dC_t[n] += ds_t h_t[n]
-//   du_t     = ds_t D + sum_n lam_t[n] Delta_t B_t[n]
-//   dz_t     = dy_t s_t silu'(z_t),  ddelta_t = dDelta_t sigmoid(delta_t + bias)
+// ds_t = dy_t g_t, and the per-step sums over states
+// Pb_t = sum_n lam_t[n] B_t[n], Pa_t = sum_n lam_t[n] A[n] a_t[n] h_{t-1}[n]:
+//   du_t      = Delta_t Pb_t + ds_t D
+//   dDelta_t  = Pa_t + u_t Pb_t,          ddelta_t = dDelta_t sigmoid(delta_t + bias)
+//   dA[n]    += lam_t[n] Delta_t a_t[n] h_{t-1}[n]
+//   dB_t[n]  += lam_t[n] Delta_t u_t,     dC_t[n] += ds_t h_t[n]
+//   dz_t      = dy_t s_t silu'(z_t)
 // Sums over the 16 states go through shared memory (one share per warp);
 // dB and dC, which sum over channels, are reduced across the warp's lanes
 // by a shuffle reduce-scatter every four steps and added to HBM with one
@@ -52,10 +59,10 @@ struct BwdSmem {
   // per (channel, step) tiles [CH][ROW]
   float u[CH * ROW], dl[CH * ROW], du[CH * ROW], ds[CH * ROW], sg[CH * ROW],
       z[CH * ROW], dy[CH * ROW];
-  // per (state, step) tiles [NP][TB]
-  float B[NP * TB], C[NP * TB];
-  // per warp shares [G][CH][ROW]: readout s_t, du_t, dDelta_t
-  float ps[G * CH * ROW], pu[G * CH * ROW], pd[G * CH * ROW];
+  // per (step, state) tiles [TB][NP]: a warp's four states are adjacent
+  float B[TB * NP], C[TB * NP];
+  // per warp shares [G][CH][ROW]: readout s_t, Pb_t, Pa_t
+  float ps[G * CH * ROW], pb[G * CH * ROW], pa[G * CH * ROW];
   float bias[CH], dskip[CH];
   float accD[CH], accB[CH];  // per-channel sums of ds u and ddelta
 };
@@ -75,6 +82,10 @@ __device__ __forceinline__ float comp(const float4 &v, int j) {
 }
 __device__ __forceinline__ float4 ld4(const float *p) {
   return *reinterpret_cast<const float4 *>(p);
+}
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+__device__ __forceinline__ float2 ex2_pair(float2 x) {
+  return make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
 }
 
 __device__ __forceinline__ float sigmoid_f(float x) {
@@ -125,6 +136,12 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   const int64_t L = p.seqlen;
   const int nblk = static_cast<int>((L + TB - 1) / TB);
 
+  // tensor sizes for the bounds checks of the checked build
+  const int64_t nBDL = p.batch * p.dim * L, nBNL = p.batch * p.dstate * L;
+  const int64_t nCk = p.tiles * static_cast<int64_t>(nblk) * NP * CH;
+  // the block's checkpoints (a block-uniform condition: all threads leave)
+  if (!dbg_index_ok((tile + 1) * static_cast<int64_t>(nblk) * NP * CH - 1, nCk, p.status))
+    return;
   const InT *gu = static_cast<const InT *>(p.u);
   const InT *gd = static_cast<const InT *>(p.delta);
   const InT *gz = static_cast<const InT *>(p.z);
@@ -139,15 +156,21 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     s.accB[tid] = 0.f;
   }
 
-  float alpha[4], an[4], h[4];
-  bool live[4];
+  // this lane's states 4g .. 4g+3 as two pairs (4g, 4g+1), (4g+2, 4g+3)
+  float2 al2[2], an2[2], h2[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int n = 4 * g + i;
-    live[i] = dvalid && n < p.dstate;
-    an[i] = live[i] ? p.A[d * p.dstate + n] : 0.f;
-    alpha[i] = an[i] * kLog2e;
-    h[i] = (live[i] && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
+  for (int q = 0; q < 2; ++q) {
+    float av[2], hv[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int n = 4 * g + 2 * q + e;
+      const bool live = dvalid && n < p.dstate;
+      av[e] = live ? p.A[d * p.dstate + n] : 0.f;
+      hv[e] = (live && p.h0) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.f;
+    }
+    an2[q] = make_float2(av[0], av[1]);
+    al2[q] = make_float2(av[0] * kLog2e, av[1] * kLog2e);
+    h2[q] = make_float2(hv[0], hv[1]);
   }
   // state 4g + i of lane at the start of block k:
   // ckpt[(k * NP + 4g + i) * CH + lane] (coalesced per warp)
@@ -164,15 +187,16 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       const int64_t dd = d0 + c;
       const bool ok = dd < p.dim && t < nt;
       const int64_t off = (b * p.dim + dd) * L + t0 + t;
-      const float uv = ok ? ld_f32(gu, off) : 0.f;
-      const float x = ok ? ld_f32(gd, off) + s.bias[c] : 0.f;
-      const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
+      const bool okm = ok && dbg_index_ok(off, nBDL, p.status);
+      const float uv = okm ? ld_f32(gu, off) : 0.f;
+      const float x = okm ? ld_f32(gd, off) + s.bias[c] : 0.f;
+      const float dl = okm ? (p.softplus ? softplus_f(x) : x) : 0.f;
       s.u[c * ROW + t] = uv;
       s.dl[c * ROW + t] = dl;
       s.du[c * ROW + t] = dl * uv;
       if (full) {
-        const float zv = (ok && gz) ? ld_f32(gz, off) : 0.f;
-        const float dyv = ok ? p.dy[off] : 0.f;
+        const float zv = (okm && gz) ? ld_f32(gz, off) : 0.f;
+        const float dyv = okm ? p.dy[off] : 0.f;
         s.z[c * ROW + t] = zv;
         s.dy[c * ROW + t] = dyv;
         s.ds[c * ROW + t] = gz ? dyv * silu_f(zv) : dyv;
@@ -183,8 +207,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       const int n = idx / TB, t = idx % TB;
       const bool ok = n < p.dstate && t < nt;
       const int64_t off = (b * p.dstate + n) * L + t0 + t;
-      s.B[idx] = ok ? ld_f32(gB, off) : 0.f;
-      if (full) s.C[idx] = ok ? ld_f32(gC, off) : 0.f;
+      const bool okm = ok && dbg_index_ok(off, nBNL, p.status);
+      s.B[t * NP + n] = okm ? ld_f32(gB, off) : 0.f;
+      if (full) s.C[t * NP + n] = okm ? ld_f32(gC, off) : 0.f;
     }
   };
 
@@ -205,8 +230,8 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int e = 0; e < E; ++e) {
       const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
       const int64_t dd = d0 + c;
-      const bool ok = dd < p.dim && t < nt;
       const int64_t off = (b * p.dim + dd) * L + t0 + t;
+      const bool ok = dd < p.dim && t < nt && dbg_index_ok(off, nBDL, p.status);
       r.u[e] = ok ? ld_f32(gu, off) : 0.f;
       r.x[e] = ok ? ld_f32(gd, off) : 0.f;
       r.z[e] = (ok && gz) ? ld_f32(gz, off) : 0.f;
@@ -217,8 +242,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int e = 0; e < EB; ++e) {
       const int idx = tid + NT * e;
       const int n = idx / TB, t = idx % TB;
-      const bool ok = idx < NP * TB && n < p.dstate && t < nt;
       const int64_t off = (b * p.dstate + n) * L + t0 + t;
+      const bool ok = idx < NP * TB && n < p.dstate && t < nt &&
+                      dbg_index_ok(off, nBNL, p.status);
       r.B[e] = ok ? ld_f32(gB, off) : 0.f;
       r.C[e] = ok ? ld_f32(gC, off) : 0.f;
     }
@@ -242,8 +268,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int e = 0; e < EB; ++e) {
       const int idx = tid + NT * e;
       if (idx < NP * TB) {
-        s.B[idx] = r.B[e];
-        s.C[idx] = r.C[e];
+        const int n = idx / TB, t = idx % TB;
+        s.B[t * NP + n] = r.B[e];
+        s.C[t * NP + n] = r.C[e];
       }
     }
   };
@@ -253,180 +280,227 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   __syncthreads();
   for (int k = 0; k < (p.ckpt_given ? 0 : nblk); ++k) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + i) * CH + lane] = h[i];
+    for (int q = 0; q < 2; ++q) {
+      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q) * CH + lane] = h2[q].x;
+      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q + 1) * CH + lane] = h2[q].y;
+    }
     load_block(k, false);
     __syncthreads();
 #pragma unroll
-    for (int q = 0; q < TB / 4; ++q) {
-      const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * q]), du4 = ld4(&s.du[lane * ROW + 4 * q]);
+    for (int qd = 0; qd < TB / 4; ++qd) {
+      const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * qd]), du4 = ld4(&s.du[lane * ROW + 4 * qd]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 b4 = ld4(&s.B[(4 * g + i) * TB + 4 * q]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          h[i] = fmaf(ex2_mufu(comp(dl4, j) * alpha[i]), h[i], comp(du4, j) * comp(b4, j));
+      for (int j = 0; j < 4; ++j) {
+        const float4 b4 = ld4(&s.B[(4 * qd + j) * NP + 4 * g]);
+        const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+        h2[0] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[0])), h2[0],
+                           __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+        h2[1] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[1])), h2[1],
+                           __fmul2_rn(U2, make_float2(b4.z, b4.w)));
       }
     }
     __syncthreads();
   }
 
   // ------------------------------------------------------ reverse sweep
-  float lam[4], dA[4];
+  float2 lam[2], dA2[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    lam[i] = (live[i] && p.d_last)
-                 ? p.d_last[(b * p.dim + d) * p.dstate + 4 * g + i] : 0.f;
-    dA[i] = 0.f;
+  for (int q = 0; q < 2; ++q) {
+    float lv[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int n = 4 * g + 2 * q + e;
+      lv[e] = (dvalid && n < p.dstate && p.d_last)
+                  ? p.d_last[(b * p.dim + d) * p.dstate + n] : 0.f;
+    }
+    lam[q] = make_float2(lv[0], lv[1]);
+    dA2[q] = make_float2(0.f, 0.f);
   }
   // the checkpoint of the block after the current one is read a block early
-  float hnext[4];
+  float2 hnext[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    hnext[i] = ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + i) * CH + lane];
+  for (int q = 0; q < 2; ++q)
+    hnext[q] = make_float2(
+        ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q) * CH + lane],
+        ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
   Raw raw;
   fetch(nblk - 1, raw);
+  float accD[E], accB[E];  // this thread's shares of the per-channel sums
+#pragma unroll
+  for (int e = 0; e < E; ++e) accD[e] = accB[e] = 0.f;
   for (int k = nblk - 1; k >= 0; --k) {
     const int64_t t0 = static_cast<int64_t>(k) * TB;
     const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
     commit(raw);
-    float hc[4];
+    float2 hc[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      hc[i] = hnext[i];
-      if (k > 0) hnext[i] = ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + i) * CH + lane];
+    for (int q = 0; q < 2; ++q) {
+      hc[q] = hnext[q];
+      if (k > 0)
+        hnext[q] = make_float2(
+            ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q) * CH + lane],
+            ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
     }
     __syncthreads();
     if (k > 0) fetch(k - 1, raw);  // in flight while block k is computed
 
     // Two halves of the block, the later one first.  For each: recompute
-    // the states of its 8 steps from the checkpoint into registers (with
-    // this warp's share of the readout s_t), then run the adjoint backwards
-    // over them.  Keeping 8 steps instead of 16 halves the registers the
-    // states need, for half a block of extra recomputation.
+    // the states of its 8 steps from the checkpoint, keeping every step's
+    // state and decay (with this warp's share of the readout s_t), then
+    // run the adjoint backwards over them with the kept decays.
 #pragma unroll
     for (int half = 1; half >= 0; --half) {
       const int tb = 8 * half;  // first step of this half
-      float hs[4][8], hpre[4];  // states of steps tb..tb+7 and of step tb-1
-      float hh[4] = {hc[0], hc[1], hc[2], hc[3]};
+      float2 hs[2][8], as[2][8];
+      float2 hh[2] = {hc[0], hc[1]};
 #pragma unroll
-      for (int q = 0; q < tb / 4 + 2; ++q) {
-        const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * q]), du4 = ld4(&s.du[lane * ROW + 4 * q]);
+      for (int qd = 0; qd < tb / 4 + 2; ++qd) {
+        const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * qd]), du4 = ld4(&s.du[lane * ROW + 4 * qd]);
+        float4 ds4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (4 * qd >= tb) ds4 = ld4(&s.ds[lane * ROW + 4 * qd]);
+        float4 sp4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        float vC[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 b4 = ld4(&s.B[(4 * g + i) * TB + 4 * q]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int t = 4 * q + j;
-            if (t == tb) hpre[i] = hh[i];
-            hh[i] = fmaf(ex2_mufu(comp(dl4, j) * alpha[i]), hh[i], comp(du4, j) * comp(b4, j));
-            if (t >= tb) hs[i][t - tb] = hh[i];
+        for (int j = 0; j < 4; ++j) {
+          const int t = 4 * qd + j;
+          const float4 b4 = ld4(&s.B[t * NP + 4 * g]);
+          const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+          const float2 a0 = ex2_pair(__fmul2_rn(D2, al2[0]));
+          const float2 a1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+          hh[0] = __ffma2_rn(a0, hh[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+          hh[1] = __ffma2_rn(a1, hh[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+          if (t >= tb) {
+            as[0][t - tb] = a0;
+            as[1][t - tb] = a1;
+            hs[0][t - tb] = hh[0];
+            hs[1][t - tb] = hh[1];
+            const float4 c4 = ld4(&s.C[t * NP + 4 * g]);
+            float2 r = __fmul2_rn(make_float2(c4.x, c4.y), hh[0]);
+            r = __ffma2_rn(make_float2(c4.z, c4.w), hh[1], r);
+            const float sv = r.x + r.y;
+            if (j == 0) sp4.x = sv;
+            if (j == 1) sp4.y = sv;
+            if (j == 2) sp4.z = sv;
+            if (j == 3) sp4.w = sv;
+            // dC_t[n] = sum over channels of ds_t h_t[n]
+            const float2 S2 = f2(comp(ds4, j));
+            const float2 v0 = __fmul2_rn(S2, hh[0]), v1 = __fmul2_rn(S2, hh[1]);
+            vC[0 + j] = v0.x;
+            vC[4 + j] = v0.y;
+            vC[8 + j] = v1.x;
+            vC[12 + j] = v1.y;
           }
         }
-      }
-#pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 c4 = ld4(&s.C[(4 * g + i) * TB + tb + 4 * qq]);
-          acc.x = fmaf(c4.x, hs[i][4 * qq + 0], acc.x);
-          acc.y = fmaf(c4.y, hs[i][4 * qq + 1], acc.y);
-          acc.z = fmaf(c4.z, hs[i][4 * qq + 2], acc.z);
-          acc.w = fmaf(c4.w, hs[i][4 * qq + 3], acc.w);
+        if (4 * qd >= tb) {
+          *reinterpret_cast<float4 *>(&s.ps[(g * CH + lane) * ROW + 4 * qd]) = sp4;
+          // channel sums of dC for states 4g + i, steps 4 qd + tq: the even
+          // lane of each pair adds j = lane >> 1 = 4 i + tq
+          const float rc = reduce_scatter16(vC, lane);
+          const int jj = lane >> 1, n = 4 * g + jj / 4, t = 4 * qd + jj % 4;
+          if ((lane & 1) == 0 && n < p.dstate && t < nt &&
+              dbg_index_ok((b * p.dstate + n) * L + t0 + t, nBNL, p.status))
+            atomicAdd(p.dC + (b * p.dstate + n) * L + t0 + t, rc);
         }
-        *reinterpret_cast<float4 *>(&s.ps[(g * CH + lane) * ROW + tb + 4 * qq]) = acc;
       }
 
-      // adjoint, four steps at a time backwards
+      // adjoint, four steps at a time backwards; a_t h_{t-1} = h_t - Delta_t
+      // u_t B_t needs no state of the previous step
 #pragma unroll
       for (int qq = 1; qq >= 0; --qq) {
         const int q = 2 * half + qq;
-        float vB[16], vC[16];
+        float vB[16];
         const int t4 = tb + 4 * qq;  // first step of this quad
-        const float4 dl4 = ld4(&s.dl[lane * ROW + t4]), u4 = ld4(&s.u[lane * ROW + t4]),
+        const float4 dl4 = ld4(&s.dl[lane * ROW + t4]), du4 = ld4(&s.du[lane * ROW + t4]),
                      ds4 = ld4(&s.ds[lane * ROW + t4]);
-        float4 B4[4], C4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          B4[i] = ld4(&s.B[(4 * g + i) * TB + t4]);
-          C4[i] = ld4(&s.C[(4 * g + i) * TB + t4]);
-        }
-        float4 pu4, pd4;
+        float4 pb4, pa4;
 #pragma unroll
         for (int tq = 3; tq >= 0; --tq) {
           const int tl = 4 * qq + tq;  // step within the half
-          const float dl = comp(dl4, tq), uu = comp(u4, tq), ds = comp(ds4, tq);
-          float pdu = 0.f, pdd = 0.f;
+          const float4 b4 = ld4(&s.B[(t4 + tq) * NP + 4 * g]);
+          const float4 c4 = ld4(&s.C[(t4 + tq) * NP + 4 * g]);
+          const float2 D2 = f2(comp(dl4, tq)), U2 = f2(comp(du4, tq)), S2 = f2(comp(ds4, tq));
+          const float2 nU2 = f2(-comp(du4, tq));
+          float2 qa = make_float2(0.f, 0.f), qb = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float Bv = comp(B4[i], tq), Cv = comp(C4[i], tq);
-            const float hprev = tl > 0 ? hs[i][tl - 1] : hpre[i];
-            const float a = ex2_mufu(dl * alpha[i]);
-            lam[i] = fmaf(ds, Cv, lam[i]);
-            vC[4 * i + tq] = ds * hs[i][tl];
-            const float la = lam[i] * a * hprev;
-            pdd = fmaf(lam[i], Bv * uu, fmaf(la, an[i], pdd));
-            dA[i] = fmaf(la, dl, dA[i]);
-            vB[4 * i + tq] = lam[i] * dl * uu;
-            pdu = fmaf(lam[i] * dl, Bv, pdu);
-            lam[i] *= a;
+          for (int pr = 0; pr < 2; ++pr) {
+            const float2 Bp = pr == 0 ? make_float2(b4.x, b4.y) : make_float2(b4.z, b4.w);
+            const float2 Cp = pr == 0 ? make_float2(c4.x, c4.y) : make_float2(c4.z, c4.w);
+            lam[pr] = __ffma2_rn(S2, Cp, lam[pr]);
+            const float2 la = __fmul2_rn(lam[pr], __ffma2_rn(nU2, Bp, hs[pr][tl]));
+            qa = __ffma2_rn(la, an2[pr], qa);
+            qb = __ffma2_rn(lam[pr], Bp, qb);
+            dA2[pr] = __ffma2_rn(la, D2, dA2[pr]);
+            const float2 vb = __fmul2_rn(lam[pr], U2);
+            vB[4 * (2 * pr) + tq] = vb.x;
+            vB[4 * (2 * pr + 1) + tq] = vb.y;
+            lam[pr] = __fmul2_rn(lam[pr], as[pr][tl]);
           }
-          if (tq == 0) { pu4.x = pdu; pd4.x = pdd; }
-          if (tq == 1) { pu4.y = pdu; pd4.y = pdd; }
-          if (tq == 2) { pu4.z = pdu; pd4.z = pdd; }
-          if (tq == 3) { pu4.w = pdu; pd4.w = pdd; }
+          const float sa = qa.x + qa.y, sb = qb.x + qb.y;
+          if (tq == 0) { pa4.x = sa; pb4.x = sb; }
+          if (tq == 1) { pa4.y = sa; pb4.y = sb; }
+          if (tq == 2) { pa4.z = sa; pb4.z = sb; }
+          if (tq == 3) { pa4.w = sa; pb4.w = sb; }
         }
-        *reinterpret_cast<float4 *>(&s.pu[(g * CH + lane) * ROW + t4]) = pu4;
-        *reinterpret_cast<float4 *>(&s.pd[(g * CH + lane) * ROW + t4]) = pd4;
-        // channel sums of dB, dC for states 4g + i, steps 4q + tq: the even
-        // lane of each pair adds j = lane >> 1 = 4 i + tq
+        *reinterpret_cast<float4 *>(&s.pa[(g * CH + lane) * ROW + t4]) = pa4;
+        *reinterpret_cast<float4 *>(&s.pb[(g * CH + lane) * ROW + t4]) = pb4;
+        // channel sums of dB for states 4g + i, steps 4q + tq (as for dC)
         const float rb = reduce_scatter16(vB, lane);
-        const float rc = reduce_scatter16(vC, lane);
         const int j = lane >> 1, n = 4 * g + j / 4, t = 4 * q + j % 4;
-        if ((lane & 1) == 0 && n < p.dstate && t < nt) {
-          const int64_t off = (b * p.dstate + n) * L + t0 + t;
-          atomicAdd(p.dB + off, rb);
-          atomicAdd(p.dC + off, rc);
-        }
+        if ((lane & 1) == 0 && n < p.dstate && t < nt &&
+            dbg_index_ok((b * p.dstate + n) * L + t0 + t, nBNL, p.status))
+          atomicAdd(p.dB + (b * p.dstate + n) * L + t0 + t, rb);
       }
     }
     __syncthreads();
 
     // elementwise: du, ddelta, dz, and the per-channel sums of dD, dbias
-    for (int idx = tid; idx < CH * TB; idx += NT) {
+    // (kept in registers: a thread's channels are the same in every block)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int idx = tid + NT * e;
       const int c = idx / TB, t = idx % TB;
       const int64_t dd = d0 + c;
       if (dd >= p.dim || t >= nt) continue;
-      float sp = 0.f, su = 0.f, sd = 0.f;
+      float sp = 0.f, sb = 0.f, sa = 0.f;
 #pragma unroll
       for (int w = 0; w < G; ++w) {
         sp += s.ps[(w * CH + c) * ROW + t];
-        su += s.pu[(w * CH + c) * ROW + t];
-        sd += s.pd[(w * CH + c) * ROW + t];
+        sb += s.pb[(w * CH + c) * ROW + t];
+        sa += s.pa[(w * CH + c) * ROW + t];
       }
       const float uu = s.u[c * ROW + t], ds = s.ds[c * ROW + t];
       const int64_t off = (b * p.dim + dd) * L + t0 + t;
-      p.du[off] = fmaf(ds, s.dskip[c], su);
-      const float ddl = sd * s.sg[c * ROW + t];
+      if (!dbg_index_ok(off, nBDL, p.status)) continue;
+      p.du[off] = fmaf(ds, s.dskip[c], s.dl[c * ROW + t] * sb);
+      const float ddl = fmaf(uu, sb, sa) * s.sg[c * ROW + t];
       p.ddelta[off] = ddl;
       if (p.dz) {
         const float sv = fmaf(s.dskip[c], uu, sp);
         p.dz[off] = s.dy[c * ROW + t] * sv * dsilu_f(s.z[c * ROW + t]);
       }
-      atomicAdd(&s.accD[c], ds * uu);
-      atomicAdd(&s.accB[c], ddl);
+      accD[e] = fmaf(ds, uu, accD[e]);
+      accB[e] += ddl;
     }
     __syncthreads();
   }
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int c = (tid + NT * e) / TB;
+    atomicAdd(&s.accD[c], accD[e]);
+    atomicAdd(&s.accB[c], accB[e]);
+  }
+  __syncthreads();
 
   // parameter gradients, summed over batch rows (and dh0 = lam_{-1})
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (!live[i]) continue;
-    const int n = 4 * g + i;
-    atomicAdd(p.dA + d * p.dstate + n, dA[i]);
-    if (p.dh0) p.dh0[(b * p.dim + d) * p.dstate + n] = lam[i];
+  for (int q = 0; q < 2; ++q) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int n = 4 * g + 2 * q + e;
+      if (!dvalid || n >= p.dstate) continue;
+      atomicAdd(p.dA + d * p.dstate + n, e == 0 ? dA2[q].x : dA2[q].y);
+      if (p.dh0) p.dh0[(b * p.dim + d) * p.dstate + n] = e == 0 ? lam[q].x : lam[q].y;
+    }
   }
   if (tid < CH && d0 + tid < p.dim) {
     if (p.dD) atomicAdd(p.dD + d0 + tid, s.accD[tid]);

@@ -28,6 +28,7 @@ struct BwdParams {
   int ckpt_given;   // ckpt already holds the forward scan's states
   int ch_tiles;     // ceil(dim / kBwdChannels)
   int64_t tiles;    // batch * ch_tiles
+  unsigned *status; // library status word (bounds checks of the checked build)
 };
 
 // Warps per block (state groups of 4): 1, 2 or 4.

@@ -56,6 +56,9 @@ struct ScanParams {
   float *incl;     // per item: true state at the end of the chunk
   unsigned test_flags;
   int64_t spin_timeout_ns;
+  // element extents (largest index + 1) of the streamed tensors under their
+  // strides and of the checkpoint buffer: the bounds of the checked build
+  int64_t ext_u, ext_delta, ext_z, ext_B, ext_C, ext_y, ext_ckpt;
 };
 
 // TMA descriptors of the five streamed inputs (z unused without a gate).
@@ -94,11 +97,10 @@ struct UpdateParams {
   const float *dt_bias;
   int softplus;
   void *y;
+  unsigned *status;  // library status word (bounds checks of the checked build)
 };
 
 cudaError_t launch_state_update(const UpdateParams &p, int in_bf16,
                                 int out_bf16, cudaStream_t stream);
-
-constexpr unsigned kStatusTimeout = 1u;
 
 }  // namespace sss48

@@ -26,6 +26,11 @@ template <typename InT, typename OutT, int N>
 __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p) {
   const int64_t ch = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (ch >= p.batch * p.dim) return;
+  // checked build: every computed index of this channel lies in its tensor
+  if (!dbg_index_ok((ch + 1) * p.dstate - 1, p.batch * p.dim * p.dstate, p.status) ||
+      !dbg_index_ok((ch % p.dim + 1) * p.dstate - 1, p.dim * p.dstate, p.status) ||
+      !dbg_index_ok((ch / p.dim + 1) * p.dstate - 1, p.batch * p.dstate, p.status))
+    return;
   const int64_t b = ch / p.dim;
   const int64_t d = ch % p.dim;
   const int nst = static_cast<int>(p.dstate);

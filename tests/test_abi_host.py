@@ -54,6 +54,20 @@ def test_library_exports_every_declared_symbol(lib):
         assert getattr(lib, sym) is not None
 
 
+def test_checked_build_exports_the_same_symbols():
+    """The checked build (MSS_DEBUG=1: device-side bounds checks) is the same
+    library: it loads, has this ABI version and exports every declared entry
+    point.  Built here if build() has not built it yet (nvcc, no GPU)."""
+    path = sbuild.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for sym in declared_functions():
+        assert sym in exported, sym
+    dbg = sss.load_debug_library()
+    assert dbg.mss_abi_version() == sss.ABI_VERSION
+
+
 def test_abi_version_and_status_strings(lib):
     assert lib.mss_abi_version() == sss.ABI_VERSION == 8
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
