@@ -53,14 +53,24 @@ constexpr int CH = 32;
 constexpr int TB = 16;
 constexpr int ROW = TB + 4;  // padded fp32 row (conflict-free float4 reads)
 
+// The fp32 tiles of one 16-step block.
+template <int G>
+struct BwdTiles {
+  static constexpr int NP = 4 * G;
+  // per (channel, step) tiles [CH][ROW]; gz = dy silu'(z), so that
+  // dz = gz s with s the readout (incl. D u)
+  float u[CH * ROW], dl[CH * ROW], du[CH * ROW], ds[CH * ROW], sg[CH * ROW],
+      gz[CH * ROW];
+  // per (step, state) tiles [TB][NP]: a warp's four states are adjacent
+  float B[TB * NP], C[TB * NP];
+};
+
 template <int G>
 struct BwdSmem {
   static constexpr int NP = 4 * G;
-  // per (channel, step) tiles [CH][ROW]
-  float u[CH * ROW], dl[CH * ROW], du[CH * ROW], ds[CH * ROW], sg[CH * ROW],
-      z[CH * ROW], dy[CH * ROW];
-  // per (step, state) tiles [TB][NP]: a warp's four states are adjacent
-  float B[TB * NP], C[TB * NP];
+  // two sets of tiles: block k is computed from set k & 1 while the other
+  // set still serves block k + 1's epilogue
+  BwdTiles<G> tl[2];
   // per warp shares [G][CH][ROW]: readout s_t, Pb_t, Pa_t
   float ps[G * CH * ROW], pb[G * CH * ROW], pa[G * CH * ROW];
   float bias[CH], dskip[CH];
@@ -90,12 +100,6 @@ __device__ __forceinline__ float2 ex2_pair(float2 x) {
 
 __device__ __forceinline__ float sigmoid_f(float x) {
   return __fdividef(1.0f, 1.0f + ex2_mufu(-x * kLog2e));
-}
-
-// silu'(z) = sigmoid(z) (1 + z (1 - sigmoid(z)))
-__device__ __forceinline__ float dsilu_f(float z) {
-  const float s = sigmoid_f(z);
-  return s * fmaf(z, 1.0f - s, 1.0f);
 }
 
 // Sum over the 32 lanes of 16 values per lane (v[j], j = 4 i + tq): four
@@ -176,43 +180,6 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   // ckpt[(k * NP + 4g + i) * CH + lane] (coalesced per warp)
   float *ckpt = p.ckpt + tile * static_cast<int64_t>(nblk) * NP * CH;
 
-  // Block k of the inputs into the fp32 tiles with Delta and Delta*u (and,
-  // for the reverse sweep, z, dy, ds = dy silu(z), sigmoid(delta + bias)
-  // and C) -- all threads.
-  auto load_block = [&](int k, bool full) {
-    const int64_t t0 = static_cast<int64_t>(k) * TB;
-    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
-    for (int idx = tid; idx < CH * TB; idx += NT) {
-      const int c = idx / TB, t = idx % TB;
-      const int64_t dd = d0 + c;
-      const bool ok = dd < p.dim && t < nt;
-      const int64_t off = (b * p.dim + dd) * L + t0 + t;
-      const bool okm = ok && dbg_index_ok(off, nBDL, p.status);
-      const float uv = okm ? ld_f32(gu, off) : 0.f;
-      const float x = okm ? ld_f32(gd, off) + s.bias[c] : 0.f;
-      const float dl = okm ? (p.softplus ? softplus_f(x) : x) : 0.f;
-      s.u[c * ROW + t] = uv;
-      s.dl[c * ROW + t] = dl;
-      s.du[c * ROW + t] = dl * uv;
-      if (full) {
-        const float zv = (okm && gz) ? ld_f32(gz, off) : 0.f;
-        const float dyv = okm ? p.dy[off] : 0.f;
-        s.z[c * ROW + t] = zv;
-        s.dy[c * ROW + t] = dyv;
-        s.ds[c * ROW + t] = gz ? dyv * silu_f(zv) : dyv;
-        s.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
-      }
-    }
-    for (int idx = tid; idx < NP * TB; idx += NT) {
-      const int n = idx / TB, t = idx % TB;
-      const bool ok = n < p.dstate && t < nt;
-      const int64_t off = (b * p.dstate + n) * L + t0 + t;
-      const bool okm = ok && dbg_index_ok(off, nBNL, p.status);
-      s.B[t * NP + n] = okm ? ld_f32(gB, off) : 0.f;
-      if (full) s.C[t * NP + n] = okm ? ld_f32(gC, off) : 0.f;
-    }
-  };
-
   // The reverse sweep reads block k - 1 from HBM into registers while block
   // k is computed, and writes it to the tiles at the start of the next
   // iteration: fetch (loads only) and commit (math and shared stores).
@@ -249,55 +216,113 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       r.C[e] = ok ? ld_f32(gC, off) : 0.f;
     }
   };
-  auto commit = [&](const Raw &r) {
+  auto commit = [&](const Raw &r, BwdTiles<G> &T) {
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
       const bool ok = (r.ok >> e) & 1u;
       const float x = ok ? r.x[e] + s.bias[c] : 0.f;
       const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
-      s.u[c * ROW + t] = r.u[e];
-      s.dl[c * ROW + t] = dl;
-      s.du[c * ROW + t] = dl * r.u[e];
-      s.z[c * ROW + t] = r.z[e];
-      s.dy[c * ROW + t] = r.dy[e];
-      s.ds[c * ROW + t] = gz ? r.dy[e] * silu_f(r.z[e]) : r.dy[e];
-      s.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
+      T.u[c * ROW + t] = r.u[e];
+      T.dl[c * ROW + t] = dl;
+      T.du[c * ROW + t] = dl * r.u[e];
+      // silu(z) = z sig(z) and silu'(z) = sig(z) (1 + z (1 - sig(z))) from
+      // one sigmoid
+      const float zv = r.z[e], dyv = r.dy[e];
+      const float sz = gz ? sigmoid_f(zv) : 1.f;
+      T.ds[c * ROW + t] = gz ? dyv * zv * sz : dyv;
+      T.gz[c * ROW + t] = dyv * sz * fmaf(zv, 1.0f - sz, 1.0f);
+      T.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
     }
 #pragma unroll
     for (int e = 0; e < EB; ++e) {
       const int idx = tid + NT * e;
       if (idx < NP * TB) {
         const int n = idx / TB, t = idx % TB;
-        s.B[t * NP + n] = r.B[e];
-        s.C[t * NP + n] = r.C[e];
+        T.B[t * NP + n] = r.B[e];
+        T.C[t * NP + n] = r.C[e];
       }
     }
   };
 
   // ------------------------------------------------------ forward sweep
-  // (skipped when the forward scan already wrote the checkpoints)
-  __syncthreads();
-  for (int k = 0; k < (p.ckpt_given ? 0 : nblk); ++k) {
+  // (skipped when the forward scan already wrote the checkpoints).  Block
+  // k + 1's u, delta and B are read into registers while block k is
+  // computed and committed to the other tile set next iteration, so one
+  // barrier per block separates the phases.
+  struct RawF {
+    float u[E], x[E], B[EB];
+    unsigned ok;
+  };
+  auto fetch_fwd = [&](int k, RawF &r) {
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+    r.ok = 0u;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q) * CH + lane] = h2[q].x;
-      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q + 1) * CH + lane] = h2[q].y;
+    for (int e = 0; e < E; ++e) {
+      const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
+      const int64_t dd = d0 + c;
+      const int64_t off = (b * p.dim + dd) * L + t0 + t;
+      const bool ok = dd < p.dim && t < nt && dbg_index_ok(off, nBDL, p.status);
+      r.u[e] = ok ? ld_f32(gu, off) : 0.f;
+      r.x[e] = ok ? ld_f32(gd, off) : 0.f;
+      if (ok) r.ok |= 1u << e;
     }
-    load_block(k, false);
-    __syncthreads();
 #pragma unroll
-    for (int qd = 0; qd < TB / 4; ++qd) {
-      const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * qd]), du4 = ld4(&s.du[lane * ROW + 4 * qd]);
+    for (int e = 0; e < EB; ++e) {
+      const int idx = tid + NT * e;
+      const int n = idx / TB, t = idx % TB;
+      const int64_t off = (b * p.dstate + n) * L + t0 + t;
+      const bool ok = idx < NP * TB && n < p.dstate && t < nt &&
+                      dbg_index_ok(off, nBNL, p.status);
+      r.B[e] = ok ? ld_f32(gB, off) : 0.f;
+    }
+  };
+  auto commit_fwd = [&](const RawF &r, BwdTiles<G> &T) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 b4 = ld4(&s.B[(4 * qd + j) * NP + 4 * g]);
-        const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
-        h2[0] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[0])), h2[0],
-                           __fmul2_rn(U2, make_float2(b4.x, b4.y)));
-        h2[1] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[1])), h2[1],
-                           __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+    for (int e = 0; e < E; ++e) {
+      const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
+      const bool ok = (r.ok >> e) & 1u;
+      const float x = ok ? r.x[e] + s.bias[c] : 0.f;
+      const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
+      T.dl[c * ROW + t] = dl;
+      T.du[c * ROW + t] = dl * r.u[e];
+    }
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+      const int idx = tid + NT * e;
+      if (idx < NP * TB) T.B[(idx % TB) * NP + idx / TB] = r.B[e];
+    }
+  };
+  __syncthreads();
+  if (!p.ckpt_given) {
+    RawF rf;
+    fetch_fwd(0, rf);
+    for (int k = 0; k < nblk; ++k) {
+      BwdTiles<G> &T = s.tl[k & 1];
+      commit_fwd(rf, T);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q) * CH + lane] = h2[q].x;
+        ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q + 1) * CH + lane] = h2[q].y;
       }
+      __syncthreads();
+      if (k + 1 < nblk) fetch_fwd(k + 1, rf);  // in flight while block k is computed
+#pragma unroll
+      for (int qd = 0; qd < TB / 4; ++qd) {
+        const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 b4 = ld4(&T.B[(4 * qd + j) * NP + 4 * g]);
+          const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+          h2[0] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[0])), h2[0],
+                             __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+          h2[1] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[1])), h2[1],
+                             __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+        }
+      }
+      // no barrier here: block k + 1 is committed to the other tile set, and
+      // this set is next written two blocks on, after the next barrier
     }
     __syncthreads();
   }
@@ -325,13 +350,18 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
   Raw raw;
   fetch(nblk - 1, raw);
-  float accD[E], accB[E];  // this thread's shares of the per-channel sums
+  // this thread's shares of the per-channel sums (in registers when a
+  // thread has few elements; otherwise added to shared memory per block)
+  constexpr bool kRegAcc = E <= 4;
+  constexpr int EA = kRegAcc ? E : 1;
+  float accD[EA], accB[EA];
 #pragma unroll
-  for (int e = 0; e < E; ++e) accD[e] = accB[e] = 0.f;
+  for (int e = 0; e < EA; ++e) accD[e] = accB[e] = 0.f;
   for (int k = nblk - 1; k >= 0; --k) {
     const int64_t t0 = static_cast<int64_t>(k) * TB;
     const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
-    commit(raw);
+    BwdTiles<G> &T = s.tl[k & 1];
+    commit(raw, T);
     float2 hc[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -355,15 +385,15 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       float2 hh[2] = {hc[0], hc[1]};
 #pragma unroll
       for (int qd = 0; qd < tb / 4 + 2; ++qd) {
-        const float4 dl4 = ld4(&s.dl[lane * ROW + 4 * qd]), du4 = ld4(&s.du[lane * ROW + 4 * qd]);
+        const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
         float4 ds4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (4 * qd >= tb) ds4 = ld4(&s.ds[lane * ROW + 4 * qd]);
+        if (4 * qd >= tb) ds4 = ld4(&T.ds[lane * ROW + 4 * qd]);
         float4 sp4 = make_float4(0.f, 0.f, 0.f, 0.f);
         float vC[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int t = 4 * qd + j;
-          const float4 b4 = ld4(&s.B[t * NP + 4 * g]);
+          const float4 b4 = ld4(&T.B[t * NP + 4 * g]);
           const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
           const float2 a0 = ex2_pair(__fmul2_rn(D2, al2[0]));
           const float2 a1 = ex2_pair(__fmul2_rn(D2, al2[1]));
@@ -374,7 +404,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
             as[1][t - tb] = a1;
             hs[0][t - tb] = hh[0];
             hs[1][t - tb] = hh[1];
-            const float4 c4 = ld4(&s.C[t * NP + 4 * g]);
+            const float4 c4 = ld4(&T.C[t * NP + 4 * g]);
             float2 r = __fmul2_rn(make_float2(c4.x, c4.y), hh[0]);
             r = __ffma2_rn(make_float2(c4.z, c4.w), hh[1], r);
             const float sv = r.x + r.y;
@@ -410,14 +440,14 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         const int q = 2 * half + qq;
         float vB[16];
         const int t4 = tb + 4 * qq;  // first step of this quad
-        const float4 dl4 = ld4(&s.dl[lane * ROW + t4]), du4 = ld4(&s.du[lane * ROW + t4]),
-                     ds4 = ld4(&s.ds[lane * ROW + t4]);
+        const float4 dl4 = ld4(&T.dl[lane * ROW + t4]), du4 = ld4(&T.du[lane * ROW + t4]),
+                     ds4 = ld4(&T.ds[lane * ROW + t4]);
         float4 pb4, pa4;
 #pragma unroll
         for (int tq = 3; tq >= 0; --tq) {
           const int tl = 4 * qq + tq;  // step within the half
-          const float4 b4 = ld4(&s.B[(t4 + tq) * NP + 4 * g]);
-          const float4 c4 = ld4(&s.C[(t4 + tq) * NP + 4 * g]);
+          const float4 b4 = ld4(&T.B[(t4 + tq) * NP + 4 * g]);
+          const float4 c4 = ld4(&T.C[(t4 + tq) * NP + 4 * g]);
           const float2 D2 = f2(comp(dl4, tq)), U2 = f2(comp(du4, tq)), S2 = f2(comp(ds4, tq));
           const float2 nU2 = f2(-comp(du4, tq));
           float2 qa = make_float2(0.f, 0.f), qb = make_float2(0.f, 0.f);
@@ -468,26 +498,34 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         sb += s.pb[(w * CH + c) * ROW + t];
         sa += s.pa[(w * CH + c) * ROW + t];
       }
-      const float uu = s.u[c * ROW + t], ds = s.ds[c * ROW + t];
+      const float uu = T.u[c * ROW + t], ds = T.ds[c * ROW + t];
       const int64_t off = (b * p.dim + dd) * L + t0 + t;
       if (!dbg_index_ok(off, nBDL, p.status)) continue;
-      p.du[off] = fmaf(ds, s.dskip[c], s.dl[c * ROW + t] * sb);
-      const float ddl = fmaf(uu, sb, sa) * s.sg[c * ROW + t];
+      p.du[off] = fmaf(ds, s.dskip[c], T.dl[c * ROW + t] * sb);
+      const float ddl = fmaf(uu, sb, sa) * T.sg[c * ROW + t];
       p.ddelta[off] = ddl;
       if (p.dz) {
         const float sv = fmaf(s.dskip[c], uu, sp);
-        p.dz[off] = s.dy[c * ROW + t] * sv * dsilu_f(s.z[c * ROW + t]);
+        p.dz[off] = T.gz[c * ROW + t] * sv;
       }
-      accD[e] = fmaf(ds, uu, accD[e]);
-      accB[e] += ddl;
+      if (kRegAcc) {
+        accD[e % EA] = fmaf(ds, uu, accD[e % EA]);
+        accB[e % EA] += ddl;
+      } else {
+        atomicAdd(&s.accD[c], ds * uu);
+        atomicAdd(&s.accB[c], ddl);
+      }
     }
-    __syncthreads();
+    // no barrier here: the next block is committed to the other tile set,
+    // and the shares are rewritten only after the next block's barrier,
+    // which every thread reaches after finishing this epilogue
   }
+  __syncthreads();
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
+  for (int e = 0; e < (kRegAcc ? E : 0); ++e) {
     const int c = (tid + NT * e) / TB;
-    atomicAdd(&s.accD[c], accD[e]);
-    atomicAdd(&s.accB[c], accB[e]);
+    atomicAdd(&s.accD[c], accD[e % EA]);
+    atomicAdd(&s.accB[c], accB[e % EA]);
   }
   __syncthreads();
 

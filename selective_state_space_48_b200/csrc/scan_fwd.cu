@@ -34,8 +34,11 @@
 // publishes (P, e), looks back over its predecessors' pairs to obtain the
 // true state h_in at its start (decoupled look-back, each wait bounded), and
 // then adds the missing term sum_n C_t[n] exp(A[n] sigma_t) h_in[n] to the
-// outputs it has written, until that term has decayed below 2^-64 of h_in
-// (sigma_t is the running sum of Delta from the chunk start).
+// outputs it has written, until the decay exp(A[n] sigma_t) of each of the
+// warp's states has fallen below 2^-24, fp32's unit roundoff, for every
+// channel of the warp (sigma_t is the running sum of Delta from the chunk
+// start): a term dropped there is smaller than the rounding error of the
+// carried state itself.
 //
 // Shapes whose rows TMA cannot address (a row of seqlen elements that is
 // not a multiple of 16 bytes, or unaligned pointers) take the same kernel
@@ -64,7 +67,7 @@ constexpr int ROW = TB + 4;  // padded fp32 row: float4 reads of 32 lanes at
                              // rows l spread over the bank groups
 constexpr int STAGES = 5;    // raw tile ring: blocks i-1 .. i+3 alive at once
 constexpr int PREFETCH = 3;  // block i+3 is requested while block i is scanned
-constexpr float kCutoffLog2 = -64.0f;
+constexpr float kCutoffLog2 = -24.0f;
 // States per lane (of 4) whose decay exp(Delta A) is evaluated by the
 // FMA-pipe polynomial instead of the special-function unit; balances the
 // two pipes (the unit's 16 results per clock per SM bound the scan).
