@@ -156,11 +156,13 @@ def kernel_source_hash(kernel: str = "fwd") -> str:
 
 def profiled_traffic(workload: str, kernel: str = "fwd"):
     """DRAM bytes per launch from the committed ncu summary, or None when
-    the kernel changed since the counters were taken."""
+    the kernel changed since the counters were taken.  Entries are keyed by
+    workload name, prefixed with the kernel for the passes other than the
+    forward scan and the SSD scan ("bwd:mamba130m-layer")."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
-        e = d.get(workload)
+        e = d.get(workload) if kernel in ("fwd", "ssd") else d.get(f"{kernel}:{workload}")
         if e and e.get("kernel_source_hash") == kernel_source_hash(kernel):
             return float(e["dram_bytes_per_launch"])
     except Exception:
@@ -555,7 +557,8 @@ def run_bwd(args, rank, world, local_rank):
         "state_updates_per_s": w.state_updates * K * world / (max_ms * 1e-3),
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
                      "unit": "GB/s", "frac": value / world / peak,
-                     "peak_source": src, "traffic": None,
+                     "peak_source": src,
+                     "traffic": None if args.checkpoints else profiled_traffic(w.name, "bwd"),
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
         "kernel_source_hash": kernel_source_hash("bwd"),
@@ -843,33 +846,59 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_gbs(bytes_step, K, world, max_ms)
     updates = w.state_updates * K * world / (max_ms * 1e-3)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers.  Every step
+    # uploads its inputs from pinned host memory, scans and reads y back;
+    # two sets of device buffers and three streams let step i+1's upload and
+    # step i-1's read-back run while step i is scanned (the copy engines of
+    # both directions and the SMs work at once).
     names = ["u", "delta", "z", "B", "C", "A", "D", "delta_bias"]
     host = {k: inp[k].detach().cpu().pin_memory() for k in names if inp[k] is not None}
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = y.numel() * y.element_size()
+    sets = [inp, {k: (None if v is None else torch.empty_like(v)) for k, v in inp.items()}]
+    ys = [y, torch.empty_like(y)]
+    s_up, s_cmp, s_dn = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    up_done, cmp_done, dn_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     Ke = max(1, args.e2e_steps)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(Ke):
-        for k, t in host.items():
-            inp[k].copy_(t, non_blocking=True)
-        sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"],
-                               inp["C"], D=inp["D"], z=inp["z"],
-                               delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, y=y, workspace=ws,
+    for st in (s_up, s_cmp, s_dn):
+        st.wait_stream(stream)
+    for i in range(Ke):
+        j = i % 2
+        d = sets[j]
+        if i >= 2:
+            s_up.wait_event(cmp_done[j])  # set j's scan of step i-2 is done
+        with torch.cuda.stream(s_up):
+            for k, t in host.items():
+                d[k].copy_(t, non_blocking=True)
+        up_done[j].record(s_up)
+        s_cmp.wait_event(up_done[j])
+        if i >= 2:
+            s_cmp.wait_event(dn_done[j])  # y set j was read back
+        sss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"],
+                               z=d["z"], delta_bias=d["delta_bias"],
+                               delta_softplus=w.softplus, y=ys[j], workspace=ws,
                                cu_seqlens=cu_t, trapezoid=args.trapezoid,
-                               checkpoints=ck)
-        y_host.copy_(y, non_blocking=True)
+                               checkpoints=ck, stream=s_cmp)
+        cmp_done[j].record(s_cmp)
+        s_dn.wait_event(cmp_done[j])
+        with torch.cuda.stream(s_dn):
+            y_host[j].copy_(ys[j], non_blocking=True)
+        dn_done[j].record(s_dn)
+    stream.wait_stream(s_dn)
+    stream.wait_stream(s_up)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = reduce_max(e0.elapsed_time(e1), world)
     e2e_value = whole_job_gbs(bytes_step, Ke, world, e2e_ms)
+    del sets[1], ys[1]
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
@@ -910,7 +939,10 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.summary()
     sm_mhz = clk.get("sm_mhz") or 1965.0
     pcfg = None
-    if not args.no_per_config and not (args.varlen or args.trapezoid or args.checkpoints):
+    # per-workload lines on one GPU only (each rank would time the same
+    # replicas again under torchrun)
+    if world == 1 and not args.no_per_config and not (args.varlen or args.trapezoid
+                                                      or args.checkpoints):
         pcfg = per_config(args, dev, sss, rank, sm_mhz)
     line = {
         "metric": METRIC,
@@ -947,7 +979,8 @@ def run_ours(args, rank, world, local_rank):
         # ex2 per state update)
         "exp_unit": exp_unit_bound(w, max_kernel_ms, sm_mhz),
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": Ke},
+                "d2h_bytes_per_step": d2h, "steps": Ke,
+                "overlap": "upload of step i+1 and read-back of step i-1 during the scan of step i"},
         "gpu_launches": K,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                    "reasons": clk["reasons"], "samples": clk["samples"]},
