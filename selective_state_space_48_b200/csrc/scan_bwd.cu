@@ -181,8 +181,8 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   float *ckpt = p.ckpt + tile * static_cast<int64_t>(nblk) * NP * CH;
 
   // The reverse sweep reads block k - 1 from HBM into registers while block
-  // k is computed, and writes it to the tiles at the start of the next
-  // iteration: fetch (loads only) and commit (math and shared stores).
+  // k's earlier half is computed and writes it to the other tile set right
+  // after: fetch (loads only) and commit (math and shared stores).
   constexpr int E = CH * TB / NT;             // (channel, step) elements per thread
   constexpr int EB = (NP * TB + NT - 1) / NT; // (state, step) elements per thread
   struct Raw {
@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
   Raw raw;
   fetch(nblk - 1, raw);
+  commit(raw, s.tl[(nblk - 1) & 1]);
   // this thread's shares of the per-channel sums (in registers when a
   // thread has few elements; otherwise added to shared memory per block)
   constexpr bool kRegAcc = E <= 4;
@@ -361,7 +362,6 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     const int64_t t0 = static_cast<int64_t>(k) * TB;
     const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
     BwdTiles<G> &T = s.tl[k & 1];
-    commit(raw, T);
     float2 hc[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -372,7 +372,6 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
             ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
     }
     __syncthreads();
-    if (k > 0) fetch(k - 1, raw);  // in flight while block k is computed
 
     // Two halves of the block, the later one first.  For each: recompute
     // the states of its 8 steps from the checkpoint, keeping every step's
@@ -381,6 +380,8 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
 #pragma unroll
     for (int half = 1; half >= 0; --half) {
       const int tb = 8 * half;  // first step of this half
+      // block k-1's inputs: in flight while the earlier half is computed
+      if (half == 0 && k > 0) fetch(k - 1, raw);
       float2 hs[2][8], as[2][8];
       float2 hh[2] = {hc[0], hc[1]};
 #pragma unroll
@@ -480,6 +481,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
             dbg_index_ok((b * p.dstate + n) * L + t0 + t, nBNL, p.status))
           atomicAdd(p.dB + (b * p.dstate + n) * L + t0 + t, rb);
       }
+      // block k-1 into the other tile set, which is free: block k+1's
+      // epilogue ended before this block's barrier
+      if (half == 0 && k > 0) commit(raw, s.tl[(k - 1) & 1]);
     }
     __syncthreads();
 

@@ -892,41 +892,61 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   // y_t += silu(z_t) * sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n], block by
   // block from the chunk start until every carried term has decayed.  The
   // ring continues at stage nblk so the barrier phases stay consistent.
+  // Pipelined over one barrier per block: while the scan warps add block
+  // i's carried term into share set i & 1, the other warps finish block
+  // i - 1 (old y + gate * shares), load block i's old y and turn block
+  // i + 1's raw tiles into step sizes in tile set (i + 1) & 1.
   bool need = false;
 #pragma unroll
   for (int i = 0; i < 4; ++i) need |= live[i] && h_in[i] != 0.f;
+  if (tid == 0) misc[3] = 0;  // set by a wait that runs out
   if (!__syncthreads_or(need)) return;
   float sigma = 0.f;
   bool wactive = true;  // this scan warp still has carried terms to add
   const int base = nblk % STAGES;
+  const int ta = tid - NSCAN;  // index within the other warps
+  constexpr int NAUX = NALL - NSCAN;
+  static_assert(NAUX == CH * (TB / 4), "one y quad of a block per non-scan thread");
   for (int j = 0; j < PREFETCH; ++j) sc.request(j, nblk, base, tid, NALL);
-  constexpr int kQuads = CH * (TB / 4);  // y quads of a block, one per thread
+  float4 yq = make_float4(0.f, 0.f, 0.f, 0.f);  // old y of the block in flight
+  if (!is_scan) {
+    if (!sc.land(0, nblk, base, phase)) misc[3] = 1;
+    sc.prep(base % STAGES, 0, sc.t0_of(0), sc.nt_of(0), false, ta, NAUX);
+  }
+  __syncthreads();
   for (int i = 0; i < nblk; ++i) {
-    // this block's old y, loaded now so the latency overlaps prep and the
-    // carry term (the main pass wrote it before the last block barrier)
-    const float4 yq = tid < kQuads ? sc.load_y_quad(i, tid) : make_float4(0.f, 0.f, 0.f, 0.f);
-    const bool ok = sc.land(i, nblk, base, phase);
-    if (!__syncthreads_and(ok)) {
+    if (misc[3] != 0) {
       if (tid == 0) atomicOr(p.status, kStatusTimeout);
       return;
     }
-    const int stage = (base + i) % STAGES;
-    sc.prep(stage, 0, sc.t0_of(i), sc.nt_of(i), false, tid, NALL);
-    __syncthreads();
-    if (is_scan) sc.scan_carry(0, g, lane, alpha, h_in, sigma, wactive);
-    __syncthreads();
-    if (tid < kQuads) sc.epilogue_acc(stage, 0, i, tid, yq);
-    need = false;
+    const int set = i & 1;
+    if (is_scan) {
+      sc.scan_carry(set, g, lane, alpha, h_in, sigma, wactive);
+      need = false;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      need |= live[q] && h_in[q] != 0.f && !(alpha[q] * sigma < kCutoffLog2);
-    if (is_scan) wactive = __any_sync(0xffffffffu, need);
-    if (!__syncthreads_or(need)) {
-      // copies already requested must land before the block exits
-      bool okd = true;
-      for (int j = i + 1; j < i + PREFETCH && j < nblk; ++j)
-        okd &= sc.land(j, nblk, base, phase);
-      if (!okd && tid == 0) atomicOr(p.status, kStatusTimeout);
+      for (int q = 0; q < 4; ++q)
+        need |= live[q] && h_in[q] != 0.f && !(alpha[q] * sigma < kCutoffLog2);
+      wactive = __any_sync(0xffffffffu, need);
+    } else {
+      if (i >= 1)
+        sc.epilogue_acc((base + i - 1) % STAGES, set ^ 1, i - 1, ta, yq);
+      yq = sc.load_y_quad(i, ta);
+      if (i + 1 < nblk) {
+        if (!sc.land(i + 1, nblk, base, phase)) misc[3] = 1;
+        sc.prep((base + i + 1) % STAGES, set ^ 1, sc.t0_of(i + 1), sc.nt_of(i + 1), false, ta,
+                NAUX);
+      }
+    }
+    if (!__syncthreads_or(need) || i + 1 == nblk) {
+      // block i's outputs; copies already requested must land before the
+      // block exits (blocks up to i + 1 have landed)
+      if (!is_scan) {
+        sc.epilogue_acc((base + i) % STAGES, set, i, ta, yq);
+        bool okd = true;
+        for (int j = i + 2; j < i + PREFETCH && j < nblk; ++j)
+          okd &= sc.land(j, nblk, base, phase);
+        if (!okd && ta == 0) atomicOr(p.status, kStatusTimeout);
+      }
       return;
     }
     sc.request(i + PREFETCH, nblk, base, tid, NALL);
