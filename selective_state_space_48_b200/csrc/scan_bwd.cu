@@ -65,6 +65,17 @@ struct BwdTiles {
   float B[TB * NP], C[TB * NP];
 };
 
+// The raw inputs of one 16-step block as they lie in HBM (bf16 u, delta,
+// z, B, C; fp32 dy), rows of 16 steps: the reverse sweep copies block k - 1
+// here asynchronously while block k is computed.
+template <int G>
+struct BwdStage {
+  static constexpr int NP = 4 * G;
+  __nv_bfloat16 u[CH * TB], x[CH * TB], z[CH * TB];
+  float dy[CH * TB];
+  __nv_bfloat16 B[NP * TB], C[NP * TB];
+};
+
 template <int G>
 struct BwdSmem {
   static constexpr int NP = 4 * G;
@@ -75,6 +86,7 @@ struct BwdSmem {
   float ps[G * CH * ROW], pb[G * CH * ROW], pa[G * CH * ROW];
   float bias[CH], dskip[CH];
   float accD[CH], accB[CH];  // per-channel sums of ds u and ddelta
+  alignas(16) BwdStage<G> st;  // bf16 inputs only
 };
 
 template <typename T> __device__ __forceinline__ float ld_f32(const T *p, int64_t i);
@@ -96,6 +108,22 @@ __device__ __forceinline__ float4 ld4(const float *p) {
 __device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
 __device__ __forceinline__ float2 ex2_pair(float2 x) {
   return make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
+}
+
+// 16-byte asynchronous copy global -> shared (through L2 only), tracked by
+// the thread's groups
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ bool aligned16(const void *q) {
+  return (reinterpret_cast<uintptr_t>(q) & 15) == 0;
 }
 
 __device__ __forceinline__ float sigmoid_f(float x) {
@@ -216,23 +244,26 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       r.C[e] = ok ? ld_f32(gC, off) : 0.f;
     }
   };
+  // the tiles of element (c, t) of a block from its raw values (zeros when
+  // the element lies outside the tensors)
+  auto put = [&](BwdTiles<G> &T, int c, int t, bool ok, float uu, float xr, float zv, float dyv) {
+    const float x = ok ? xr + s.bias[c] : 0.f;
+    const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
+    T.u[c * ROW + t] = uu;
+    T.dl[c * ROW + t] = dl;
+    T.du[c * ROW + t] = dl * uu;
+    // silu(z) = z sig(z) and silu'(z) = sig(z) (1 + z (1 - sig(z))) from
+    // one sigmoid
+    const float sz = gz ? sigmoid_f(zv) : 1.f;
+    T.ds[c * ROW + t] = gz ? dyv * zv * sz : dyv;
+    T.gz[c * ROW + t] = dyv * sz * fmaf(zv, 1.0f - sz, 1.0f);
+    T.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
+  };
   auto commit = [&](const Raw &r, BwdTiles<G> &T) {
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
-      const bool ok = (r.ok >> e) & 1u;
-      const float x = ok ? r.x[e] + s.bias[c] : 0.f;
-      const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
-      T.u[c * ROW + t] = r.u[e];
-      T.dl[c * ROW + t] = dl;
-      T.du[c * ROW + t] = dl * r.u[e];
-      // silu(z) = z sig(z) and silu'(z) = sig(z) (1 + z (1 - sig(z))) from
-      // one sigmoid
-      const float zv = r.z[e], dyv = r.dy[e];
-      const float sz = gz ? sigmoid_f(zv) : 1.f;
-      T.ds[c * ROW + t] = gz ? dyv * zv * sz : dyv;
-      T.gz[c * ROW + t] = dyv * sz * fmaf(zv, 1.0f - sz, 1.0f);
-      T.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
+      put(T, c, t, (r.ok >> e) & 1u, r.u[e], r.x[e], r.z[e], r.dy[e]);
     }
 #pragma unroll
     for (int e = 0; e < EB; ++e) {
@@ -241,6 +272,101 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         const int n = idx / TB, t = idx % TB;
         T.B[t * NP + n] = r.B[e];
         T.C[t * NP + n] = r.C[e];
+      }
+    }
+  };
+
+  // bf16 inputs: the reverse sweep stages block k - 1's raw inputs in
+  // shared memory by asynchronous copies (no registers held while block k
+  // is computed), 16-byte pieces of the blocks' rows where rows are whole
+  // and aligned, element loads elsewhere.
+  constexpr bool kStaged = sizeof(InT) == 2;
+  const bool rows16 = (L % 8) == 0 && aligned16(p.u) && aligned16(p.delta) &&
+                      (!gz || aligned16(p.z)) && aligned16(p.dy) && aligned16(p.B) &&
+                      aligned16(p.C);
+  auto stage_fetch = [&](int k) {
+    BwdStage<G> &st = s.st;
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+    constexpr int NR = CH * 2;                      // 8-element pieces of a bf16 tile
+    constexpr int NCH = 3 * NR + CH * 4 + 2 * NP * 2;  // + 4-element pieces of dy
+    for (int j = tid; j < NCH; j += NT) {
+      const void *src;
+      void *dst;
+      int64_t off, ext;
+      int row_ok, w, r;
+      bool f32 = false;
+      if (j < 3 * NR) {
+        const int kind = j / NR, rr = j % NR, c = rr / 2, h = rr % 2;
+        const InT *base = kind == 0 ? gu : (kind == 1 ? gd : gz);
+        off = (b * p.dim + d0 + c) * L + t0 + 8 * h;
+        ext = nBDL;
+        row_ok = d0 + c < p.dim && (kind < 2 || gz);
+        w = 8 * h;
+        src = base;
+        __nv_bfloat16 *sb = kind == 0 ? st.u : (kind == 1 ? st.x : st.z);
+        dst = sb + c * TB + 8 * h;
+      } else if (j < 3 * NR + CH * 4) {
+        r = j - 3 * NR;
+        const int c = r / 4, h = r % 4;
+        off = (b * p.dim + d0 + c) * L + t0 + 4 * h;
+        ext = nBDL;
+        row_ok = d0 + c < p.dim;
+        w = 4 * h;
+        src = p.dy;
+        dst = st.dy + c * TB + 4 * h;
+        f32 = true;
+      } else {
+        r = j - 3 * NR - CH * 4;
+        const int kind = r / (2 * NP), rr = r % (2 * NP), n = rr / 2, h = rr % 2;
+        off = (b * p.dstate + n) * L + t0 + 8 * h;
+        ext = nBNL;
+        row_ok = n < p.dstate;
+        w = 8 * h;
+        src = kind == 0 ? gB : gC;
+        dst = (kind == 0 ? st.B : st.C) + n * TB + 8 * h;
+      }
+      if (!row_ok) continue;
+      const int cnt = f32 ? 4 : 8;
+      if (rows16 && nt == TB && dbg_index_ok(off + cnt - 1, ext, p.status)) {
+        cp_async16(dst, f32 ? static_cast<const void *>(static_cast<const float *>(src) + off)
+                            : static_cast<const void *>(static_cast<const InT *>(src) + off));
+      } else {
+        for (int q = 0; q < cnt && w + q < nt; ++q) {
+          if (!dbg_index_ok(off + q, ext, p.status)) break;
+          if (f32)
+            static_cast<float *>(dst)[q] = static_cast<const float *>(src)[off + q];
+          else
+            static_cast<InT *>(dst)[q] = static_cast<const InT *>(src)[off + q];
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  // block k's tiles from the staged raw inputs (after every thread's copies
+  // have landed and a barrier)
+  auto stage_commit = [&](int k, BwdTiles<G> &T) {
+    const BwdStage<G> &st = s.st;
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
+      const bool ok = d0 + c < p.dim && t < nt;
+      const int i = c * TB + t;
+      put(T, c, t, ok, ok ? ld_f32(reinterpret_cast<const InT *>(st.u), i) : 0.f,
+          ok ? ld_f32(reinterpret_cast<const InT *>(st.x), i) : 0.f,
+          (ok && gz) ? ld_f32(reinterpret_cast<const InT *>(st.z), i) : 0.f,
+          ok ? st.dy[i] : 0.f);
+    }
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+      const int idx = tid + NT * e;
+      if (idx < NP * TB) {
+        const int n = idx / TB, t = idx % TB;
+        const bool ok = n < p.dstate && t < nt;
+        T.B[t * NP + n] = ok ? ld_f32(reinterpret_cast<const InT *>(st.B), idx) : 0.f;
+        T.C[t * NP + n] = ok ? ld_f32(reinterpret_cast<const InT *>(st.C), idx) : 0.f;
       }
     }
   };
@@ -295,32 +421,127 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     }
   };
   __syncthreads();
-  if (!p.ckpt_given) {
+  // bf16 forward sweep: block k + 2's u, delta and B are copied
+  // asynchronously into one of two areas of the staging buffer while block
+  // k is computed and block k + 1 is committed from the other area.
+  constexpr int kFArea = 2 * CH * TB * 2 + NP * TB * 2;  // bytes of one area
+  static_assert(2 * kFArea <= static_cast<int>(sizeof(BwdStage<G>)), "two areas fit");
+  auto farea = [&](int a) {
+    return reinterpret_cast<InT *>(reinterpret_cast<unsigned char *>(&s.st) + a * kFArea);
+  };
+  auto fstage_fetch = [&](int k, int a) {
+    InT *su = farea(a), *sx = su + CH * TB, *sB = sx + CH * TB;
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+    constexpr int NR = CH * 2;  // 8-element pieces of a (channel, step) tile
+    for (int j = tid; j < 2 * NR + NP * 2; j += NT) {
+      const InT *src;
+      InT *dst;
+      int64_t off, ext;
+      int w;
+      if (j < 2 * NR) {
+        const int kind = j / NR, rr = j % NR, c = rr / 2, h = rr % 2;
+        if (d0 + c >= p.dim) continue;
+        src = kind == 0 ? gu : gd;
+        dst = (kind == 0 ? su : sx) + c * TB + 8 * h;
+        off = (b * p.dim + d0 + c) * L + t0 + 8 * h;
+        ext = nBDL;
+        w = 8 * h;
+      } else {
+        const int r = j - 2 * NR, n = r / 2, h = r % 2;
+        if (n >= p.dstate) continue;
+        src = gB;
+        dst = sB + n * TB + 8 * h;
+        off = (b * p.dstate + n) * L + t0 + 8 * h;
+        ext = nBNL;
+        w = 8 * h;
+      }
+      if (rows16 && nt == TB && dbg_index_ok(off + 7, ext, p.status)) {
+        cp_async16(dst, src + off);
+      } else {
+        for (int q = 0; q < 8 && w + q < nt; ++q) {
+          if (!dbg_index_ok(off + q, ext, p.status)) break;
+          dst[q] = src[off + q];
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  auto fstage_commit = [&](int k, int a, BwdTiles<G> &T) {
+    const InT *su = farea(a), *sx = su + CH * TB, *sB = sx + CH * TB;
+    const int64_t t0 = static_cast<int64_t>(k) * TB;
+    const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
+      const bool ok = d0 + c < p.dim && t < nt;
+      const float uu = ok ? ld_f32(su, c * TB + t) : 0.f;
+      const float x = ok ? ld_f32(sx, c * TB + t) + s.bias[c] : 0.f;
+      const float dl = ok ? (p.softplus ? softplus_f(x) : x) : 0.f;
+      T.dl[c * ROW + t] = dl;
+      T.du[c * ROW + t] = dl * uu;
+    }
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+      const int idx = tid + NT * e;
+      if (idx < NP * TB) {
+        const int n = idx / TB, t = idx % TB;
+        T.B[t * NP + n] = (n < p.dstate && t < nt) ? ld_f32(sB, idx) : 0.f;
+      }
+    }
+  };
+  // block k's recurrence from tile set T, state at its start in h2
+  auto fwd_block = [&](const BwdTiles<G> &T) {
+#pragma unroll
+    for (int qd = 0; qd < TB / 4; ++qd) {
+      const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 b4 = ld4(&T.B[(4 * qd + j) * NP + 4 * g]);
+        const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+        h2[0] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[0])), h2[0],
+                           __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+        h2[1] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[1])), h2[1],
+                           __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+      }
+    }
+  };
+  auto put_ckpt = [&](int k) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q) * CH + lane] = h2[q].x;
+      ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q + 1) * CH + lane] = h2[q].y;
+    }
+  };
+  if (!p.ckpt_given && kStaged) {
+    fstage_fetch(0, 0);
+    cp_async_wait_all();
+    __syncthreads();
+    fstage_commit(0, 0, s.tl[0]);
+    if (nblk > 1) fstage_fetch(1, 1);
+    for (int k = 0; k < nblk; ++k) {
+      put_ckpt(k);
+      // block k + 1's copies (this thread's) have landed; after the barrier
+      // every thread's have, and block k's tiles are committed
+      cp_async_wait_all();
+      __syncthreads();
+      // area k & 1 held block k, committed before the barrier; tile set
+      // (k + 1) & 1 was last read by block k - 1, finished before it
+      if (k + 2 < nblk) fstage_fetch(k + 2, k & 1);
+      if (k + 1 < nblk) fstage_commit(k + 1, (k + 1) & 1, s.tl[(k + 1) & 1]);
+      fwd_block(s.tl[k & 1]);
+    }
+    __syncthreads();
+  } else if (!p.ckpt_given) {
     RawF rf;
     fetch_fwd(0, rf);
     for (int k = 0; k < nblk; ++k) {
       BwdTiles<G> &T = s.tl[k & 1];
       commit_fwd(rf, T);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q) * CH + lane] = h2[q].x;
-        ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q + 1) * CH + lane] = h2[q].y;
-      }
+      put_ckpt(k);
       __syncthreads();
       if (k + 1 < nblk) fetch_fwd(k + 1, rf);  // in flight while block k is computed
-#pragma unroll
-      for (int qd = 0; qd < TB / 4; ++qd) {
-        const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 b4 = ld4(&T.B[(4 * qd + j) * NP + 4 * g]);
-          const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
-          h2[0] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[0])), h2[0],
-                             __fmul2_rn(U2, make_float2(b4.x, b4.y)));
-          h2[1] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[1])), h2[1],
-                             __fmul2_rn(U2, make_float2(b4.z, b4.w)));
-        }
-      }
+      fwd_block(T);
       // no barrier here: block k + 1 is committed to the other tile set, and
       // this set is next written two blocks on, after the next barrier
     }
@@ -349,8 +570,15 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q) * CH + lane],
         ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
   Raw raw;
-  fetch(nblk - 1, raw);
-  commit(raw, s.tl[(nblk - 1) & 1]);
+  if (kStaged) {
+    stage_fetch(nblk - 1);
+    cp_async_wait_all();
+    __syncthreads();
+    stage_commit(nblk - 1, s.tl[(nblk - 1) & 1]);
+  } else {
+    fetch(nblk - 1, raw);
+    commit(raw, s.tl[(nblk - 1) & 1]);
+  }
   // this thread's shares of the per-channel sums (in registers when a
   // thread has few elements; otherwise added to shared memory per block)
   constexpr bool kRegAcc = E <= 4;
@@ -381,7 +609,12 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int half = 1; half >= 0; --half) {
       const int tb = 8 * half;  // first step of this half
       // block k-1's inputs: in flight while the earlier half is computed
-      if (half == 0 && k > 0) fetch(k - 1, raw);
+      if (half == 0 && k > 0) {
+        if (kStaged)
+          stage_fetch(k - 1);
+        else
+          fetch(k - 1, raw);
+      }
       float2 hs[2][8], as[2][8];
       float2 hh[2] = {hc[0], hc[1]};
 #pragma unroll
@@ -483,9 +716,13 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       }
       // block k-1 into the other tile set, which is free: block k+1's
       // epilogue ended before this block's barrier
-      if (half == 0 && k > 0) commit(raw, s.tl[(k - 1) & 1]);
+      if (!kStaged && half == 0 && k > 0) commit(raw, s.tl[(k - 1) & 1]);
     }
+    if (kStaged) cp_async_wait_all();
     __syncthreads();
+    // staged inputs: block k-1 into the other tile set once every copy has
+    // landed (the staging area is refilled only after the next barrier)
+    if (kStaged && k > 0) stage_commit(k - 1, s.tl[(k - 1) & 1]);
 
     // elementwise: du, ddelta, dz, and the per-channel sums of dD, dbias
     // (kept in registers: a thread's channels are the same in every block)
