@@ -792,6 +792,8 @@ def per_config(args, dev, sss, rank, sm_mhz) -> dict:
                  "l2": ("flushed between steps (256 MB write)" if small
                         else "inputs+outputs larger than L2, no flush"),
                  "sequence_split": sss.scan_workspace_size(st["args"]) > 0}
+        # a split scan is three kernels (chunks, prefix over the chunks, carry)
+        entry["launches_per_step"] = 3 if entry["sequence_split"] else 1
         if rank == 0:
             try:
                 entry["max_norm_err"] = sample_max_norm_err(st["y"], inp, w, 64)

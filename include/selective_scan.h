@@ -74,9 +74,11 @@ typedef enum {
 typedef enum { MSS_F32 = 0, MSS_BF16 = 1 } mss_dtype;
 
 /* Test-only flags (mss_scan_args.test_flags); 0 in production. */
-#define MSS_TESTFLAG_DROP_PUBLISH 0x1u /* one sequence chunk never publishes
-                                          its carry, so its successor's
-                                          bounded wait must run out         */
+#define MSS_TESTFLAG_DROP_PUBLISH 0x1u /* split scans: before composing the
+                                          chunks' carries, the library waits
+                                          for a publication that never
+                                          comes, so its bounded wait
+                                          (spin_timeout_ns) must run out    */
 #define MSS_TESTFLAG_DEBUG_OOB 0x2u    /* checked build only: the first y
                                           store of the first thread block is
                                           aimed one tensor length past y; the
@@ -188,8 +190,10 @@ typedef struct mss_scan_args {
 mss_status mss_scan_workspace_size(const mss_scan_args *args, size_t *bytes);
 
 /* Forward selective scan: validates, plans the launch (sequence split,
- * chunk length), clears the workspace flags with cudaMemsetAsync and
- * launches on `stream`.  Writes y and, if requested, last_state. */
+ * chunk length), clears the workspace's status word with cudaMemsetAsync
+ * and launches on `stream` (a split scan: the chunks from a zero state, the
+ * composition of their carries, then the carried terms, three kernels in
+ * stream order).  Writes y and, if requested, last_state. */
 mss_status mamba_selective_scan_fwd(const mss_scan_args *args, void *stream);
 
 /* Synchronises `stream`, then reports the device-side status of the last
@@ -219,7 +223,7 @@ mss_status mss_scan_status(const mss_scan_args *args, void *stream);
  *
  * The first call on a device looks up the array's device address (with that
  * device current); make that first call before any stream capture.  All
- * calls share the one array and its flags are cleared on the caller's stream
+ * calls share the one array and its status word is cleared on the caller's stream
  * at the start of each call: two calls whose work overlaps on the GPU (on
  * different streams, or from different threads) race and must not be
  * issued.  A bounded device-side wait that runs out is recorded in a status

@@ -171,7 +171,11 @@ mss_status make_plan(const mss_scan_args *a, Plan *pl) {
   pl->chunk = chunk;
   pl->splits = static_cast<int>((a->seqlen + chunk - 1) / chunk);
   if (pl->tiles * pl->splits > int64_t(INT32_MAX)) return MSS_ERR_UNSUPPORTED;
-  pl->workspace = scan_workspace_bytes(pl->tiles, pl->splits, pl->groups);
+  // the carry launch has one block per (tile, chunk, segment)
+  const int64_t nseg = ((chunk + kTimeBlock - 1) / kTimeBlock + kSegBlocks - 1) / kSegBlocks;
+  if (pl->splits > 1 && pl->tiles * pl->splits * nseg > int64_t(INT32_MAX))
+    return MSS_ERR_UNSUPPORTED;
+  pl->workspace = scan_workspace_bytes(pl->tiles, pl->splits, pl->chunk, pl->groups);
   return MSS_OK;
 }
 
@@ -252,9 +256,7 @@ mss_status mamba_selective_scan_fwd(const mss_scan_args *a, void *stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pl.splits > 1) {
     scan_bind_workspace(p, a->workspace, pl.groups);
-    if (cudaMemsetAsync(a->workspace, 0,
-                        scan_workspace_clear_bytes(pl.tiles, pl.splits),
-                        s) != cudaSuccess)
+    if (cudaMemsetAsync(a->workspace, 0, scan_workspace_clear_bytes(), s) != cudaSuccess)
       return MSS_ERR_CUDA;
   } else {
     p.status = scan_status_word();
@@ -501,9 +503,8 @@ extern "C" mss_status mamba_selective_scan_fwd_noalloc(const mss_scan_args *a,
     void *ws = noalloc_scratch_address();
     if (!ws) return MSS_ERR_CUDA;
     scan_bind_workspace(p, ws, pl.groups);
-    // flags, ticket and status carry the previous call's values: clear them
-    if (cudaMemsetAsync(ws, 0, scan_workspace_clear_bytes(pl.tiles, pl.splits), s) !=
-        cudaSuccess)
+    // the status word carries the previous call's value: clear it
+    if (cudaMemsetAsync(ws, 0, scan_workspace_clear_bytes(), s) != cudaSuccess)
       return MSS_ERR_CUDA;
   } else {
     p.status = scan_status_word();

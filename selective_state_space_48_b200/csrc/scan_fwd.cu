@@ -30,15 +30,26 @@
 // Long sequences with few channels are split into chunks that run in
 // parallel ("The relay": fade-and-add steps compose associatively, so a
 // chunk can be squashed into one pair (P, e) = (prod exp(Delta A), state
-// reached from zero) without knowing the state it starts from).  A chunk
-// publishes (P, e), looks back over its predecessors' pairs to obtain the
-// true state h_in at its start (decoupled look-back, each wait bounded), and
-// then adds the missing term sum_n C_t[n] exp(A[n] sigma_t) h_in[n] to the
-// outputs it has written, until the decay exp(A[n] sigma_t) of each of the
-// warp's states has fallen below 2^-24, fp32's unit roundoff, for every
-// channel of the warp (sigma_t is the running sum of Delta from the chunk
-// start): a term dropped there is smaller than the rounding error of the
-// carried state itself.
+// reached from zero) without knowing the state it starts from).  Three
+// launches on the stream, with no block ever waiting for another:
+//
+//   scan      every chunk runs from a zero state (the first from h0), writes
+//             its outputs, its pair (P, e) and the running sum of Delta at
+//             the start of every segment of 32 blocks;
+//   prefix    one thread per (tile, state, channel) composes the pairs in
+//             chunk order into the true state at the end of every chunk
+//             (and the final state);
+//   carry     one block per (tile, chunk after the first, segment) adds the
+//             missing term sum_n C_t[n] exp(A[n] sigma_t) h_in[n] to the
+//             segment's outputs (sigma_t: running sum of Delta from the
+//             chunk start, h_in: true state at the chunk start), block by
+//             block until the decay exp(A[n] sigma_t) of every state has
+//             fallen below 2^-24, fp32's unit roundoff, in every channel: a
+//             term dropped there is smaller than the rounding error of the
+//             carried state itself.  Segments whose terms have all decayed
+//             leave at once, so the work follows the states' memory and is
+//             spread over the whole chip instead of trailing behind the
+//             chunks that carry the longest.
 //
 // Shapes whose rows TMA cannot address (a row of seqlen elements that is
 // not a multiple of 16 bytes, or unaligned pointers) take the same kernel
@@ -66,7 +77,6 @@ constexpr int TB = kTimeBlock;
 constexpr int ROW = TB + 4;  // padded fp32 row: float4 reads of 32 lanes at
                              // rows l spread over the bank groups
 constexpr int STAGES = 5;    // raw tile ring: blocks i-1 .. i+3 alive at once
-constexpr int PREFETCH = 3;  // block i+3 is requested while block i is scanned
 constexpr float kCutoffLog2 = -24.0f;
 // States per lane (of 4) whose decay exp(Delta A) is evaluated by the
 // FMA-pipe polynomial instead of the special-function unit; balances the
@@ -255,121 +265,6 @@ struct Scan {
     const bool ok = mbar_wait_bounded(bar(stage), (phase >> stage) & 1u, kTmaWaitNs);
     phase ^= 1u << stage;
     return ok;
-  }
-
-  // Correction pass (all threads of the block): TMA copies or plain loads
-  // by everyone, completed by the next barrier.
-  __device__ void request(int blk, int nblk, int stage_base, int ti, int nth) const {
-    if (blk >= nblk) return;
-    const int stage = (stage_base + blk) % STAGES;
-    if (TMA) {
-      if (ti == 0) issue(stage, blk);
-    } else {
-      load_plain(stage, blk, ti, nth);
-    }
-  }
-
-  __device__ bool land(int blk, int nblk, int stage_base, uint32_t &phase) const {
-    if (!TMA || blk >= nblk) return true;
-    return wait_raw(blk, stage_base, phase);
-  }
-
-  // Delta, Delta*u (and B, C when `with_b`) of one block into fp32 set
-  // `set`, two timesteps per thread and iteration.  Steps past the end of
-  // the chunk get Delta = 0: exp(0 * A) = 1 and no input, so they leave the
-  // state unchanged.
-  __device__ void prep(int stage, int set, int64_t t0, int nt, bool with_b, int ti,
-                       int nth) const {
-    const InT *ru = raw(stage, 0), *rd = raw(stage, 1);
-    float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
-    const float *sBias = f32(Lay::bias);
-    constexpr int QT = TB / 4;
-    // four timesteps per thread: four independent softplus chains
-    for (int idx = ti; idx < CH * QT; idx += nth) {
-      const int c = idx / QT, t = 4 * (idx % QT);
-      const float4 u = load4_f32(ru + c * TB + t);
-      const float4 dd = load4_f32(rd + c * TB + t);
-      const float bias = sBias[c];
-      float4 dl = make_float4(dd.x + bias, dd.y + bias, dd.z + bias, dd.w + bias);
-      if (p.softplus) {
-        const float2 a = softplus2_f(make_float2(dl.x, dl.y));
-        const float2 b2 = softplus2_f(make_float2(dl.z, dl.w));
-        dl = make_float4(a.x, a.y, b2.x, b2.y);
-      }
-      if (t + 4 > nt) {
-        if (t >= nt) dl.x = 0.f;
-        if (t + 1 >= nt) dl.y = 0.f;
-        if (t + 2 >= nt) dl.z = 0.f;
-        if (t + 3 >= nt) dl.w = 0.f;
-      }
-      *reinterpret_cast<float4 *>(sDu + c * ROW + t) =
-          make_float4(dl.x * u.x, dl.y * u.y, dl.z * u.z, dl.w * u.w);
-      if (VARLEN && p.cu) {
-        int64_t nb = first_start_from(t0 + t);
-        mark_restarts(dl, restarts4(t0 + t, nb));
-      }
-      *reinterpret_cast<float4 *>(sDelta + c * ROW + t) = dl;
-    }
-    const InT *rb = raw(stage, 3), *rc = raw(stage, 4);
-    float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
-    for (int idx = 4 * ti; idx < 2 * NP * TB; idx += 4 * nth) {
-      if (idx < NP * TB) {
-        if (with_b) store4(sB + idx, load4_f32(rb + idx));
-      } else {
-        store4(sC + idx - NP * TB, load4_f32(rc + idx - NP * TB));
-      }
-    }
-  }
-
-  // Correction pass, thread ti < CH * TB / 4: the y values of its quad
-  // (channel ti / (TB/4), four steps) of block `blk`, read before the
-  // block's carry term is computed so the load latency overlaps it.
-  __device__ float4 load_y_quad(int blk, int ti) const {
-    constexpr int QT = TB / 4;
-    const int c = ti / QT, t = 4 * (ti % QT);
-    const int nt = nt_of(blk);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (d0 + c >= p.dim || t >= nt) return v;
-    const int64_t yi = b * p.sy[0] + (d0 + c) * p.sy[1] + t0_of(blk) + t;
-    const OutT *yr = static_cast<const OutT *>(p.y) + yi;
-    if (!dbg_index_ok(yi + min64(nt - t, 4) - 1, p.ext_y, p.status)) return v;
-    if (p.y_vec && t + 4 <= nt) return load4_f32(yr);
-    float sv[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < 4 && t + j < nt; ++j) sv[j] = to_f32<OutT>(yr[j]);
-    return make_float4(sv[0], sv[1], sv[2], sv[3]);
-  }
-
-  // Correction pass: y += (sum of the state-group shares) * silu(z) for the
-  // quad of thread ti < CH * TB / 4, whose old y values are `yq`.
-  __device__ void epilogue_acc(int stage, int set, int blk, int ti, const float4 &yq) const {
-    constexpr int QT = TB / 4;
-    const int c = ti / QT, t = 4 * (ti % QT);
-    const int nt = nt_of(blk);
-    if (d0 + c >= p.dim || t >= nt) return;
-    const InT *rz = raw(stage, 2);
-    const float *sPart = fpart(set);
-    float4 s = *reinterpret_cast<const float4 *>(sPart + c * ROW + t);
-#pragma unroll
-    for (int g = 1; g < G; ++g) {
-      const float4 v = *reinterpret_cast<const float4 *>(sPart + (g * CH + c) * ROW + t);
-      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-    }
-    if (has_z) {
-      const float4 z = load4_f32(rz + c * TB + t);
-      const float2 g01 = silu2_f(make_float2(z.x, z.y));
-      const float2 g23 = silu2_f(make_float2(z.z, z.w));
-      s.x *= g01.x; s.y *= g01.y; s.z *= g23.x; s.w *= g23.y;
-    }
-    s.x += yq.x; s.y += yq.y; s.z += yq.z; s.w += yq.w;
-    const int64_t yi = b * p.sy[0] + (d0 + c) * p.sy[1] + t0_of(blk) + t;
-    OutT *yr = static_cast<OutT *>(p.y) + yi;
-    if (!dbg_index_ok(yi + min64(nt - t, 4) - 1, p.ext_y, p.status)) return;
-    if (p.y_vec && t + 4 <= nt) {
-      store4(yr, s);
-    } else {
-      const float sv[4] = {s.x, s.y, s.z, s.w};
-      for (int j = 0; j < 4 && t + j < nt; ++j) yr[j] = from_f32<OutT>(sv[j]);
-    }
   }
 
   // ---- main-pass prep/epilogue on fixed slots.  With 64 threads per role
@@ -570,46 +465,6 @@ struct Scan {
     }
   }
 
-  // The carried-state term of the correction pass for one block:
-  // share of sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n].  A warp whose
-  // carried terms have all decayed (active false, warp-uniform) writes a
-  // zero share and leaves sigma as it is: with alpha <= 0 its terms only
-  // shrink further.
-  __device__ void scan_carry(int set, int g, int lane, const float (&alpha)[4],
-                             const float (&h_in)[4], float &sigma, bool active) const {
-    const float *sDelta = fset(set, Lay::oDelta), *sC = fset(set, Lay::oC);
-    float *sPart = fpart(set);
-    if (!active) {
-#pragma unroll
-      for (int q = 0; q < TB / 4; ++q)
-        *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
-            make_float4(0.f, 0.f, 0.f, 0.f);
-      return;
-    }
-#pragma unroll
-    for (int q = 0; q < TB / 4; ++q) {
-      const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
-      const float dls[4] = {dl.x, dl.y, dl.z, dl.w};
-      float part[4] = {0.f, 0.f, 0.f, 0.f};
-      float sig[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        sigma += dls[j];
-        sig[j] = sigma;
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int n = 4 * g + i;
-        const float4 cq = *reinterpret_cast<const float4 *>(&sC[n * TB + 4 * q]);
-        const float cs[4] = {cq.x, cq.y, cq.z, cq.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          part[j] = fmaf(cs[j] * ex2_mufu(alpha[i] * sig[j]), h_in[i], part[j]);
-      }
-      *reinterpret_cast<float4 *>(&sPart[(g * CH + lane) * ROW + 4 * q]) =
-          make_float4(part[0], part[1], part[2], part[3]);
-    }
-  }
 };
 
 // Warp roles of one block: G scan warps (one per group of 4 states), two
@@ -639,7 +494,6 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   constexpr int NSCAN = 32 * G;
   constexpr int NPREP = 32 * kPrepWarps;
   constexpr int NEPI = 32 * kEpiWarps;
-  constexpr int NALL = NSCAN + NPREP + NEPI;
   extern __shared__ __align__(128) unsigned char smem[];
   S sc(p, maps, smem);
 
@@ -651,9 +505,10 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   const int tp = tid - NSCAN;              // index within the prep warps
   const int te = tid - NSCAN - NPREP;      // index within the epilogue warps
   const bool split = p.splits > 1;
-  int *misc = reinterpret_cast<int *>(smem + Lay::misc);
 
+  int *misc = reinterpret_cast<int *>(smem + Lay::misc);
   if (tid == 0) {
+    // split scans hand out items (chunk-major) in the order blocks start
     misc[0] = split ? static_cast<int>(atomicAdd(p.ticket, 1u))
                     : static_cast<int>(blockIdx.x);
     // a raw stage completes when its TMA bytes land (one arrival) or when
@@ -752,7 +607,22 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     const typename S::Slots sl = sc.make_slots(tp);
     // cursor into the sequence offsets for this thread's steps
     int64_t nb = VARLEN ? sc.first_start_from(sc.t_begin + sl.t) : 0;
+    // split scans: this thread's share of each slot's running sum of Delta;
+    // the four threads of a channel row write the sum at every segment
+    // start for the carry launch
+    float psum[S::kSlots];
+#pragma unroll
+    for (int k = 0; k < S::kSlots; ++k) psum[k] = 0.f;
     for (int blk = 0; blk < nblk; ++blk) {
+      if (split && blk % kSegBlocks == 0) {
+#pragma unroll
+        for (int k = 0; k < S::kSlots; ++k) {
+          float v = psum[k] + __shfl_xor_sync(0xffffffffu, psum[k], 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          if (sl.t == 0 && sl.ok[k])
+            p.sig[(item * p.nseg + blk / kSegBlocks) * CH + sl.c[k]] = v;
+        }
+      }
       if (blk >= 2) wait_hand(kTilesFree, blk & 1);
       const uint32_t rs = VARLEN ? sc.restarts4(sc.t0_of(blk) + sl.t, nb) : 0u;
       // trapezoidal update: u of the step before the block, for the slots
@@ -769,11 +639,16 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
       }
       ok &= sc.wait_raw(blk, 0, phase);
       sc.prep_slots(blk % STAGES, blk & 1, sc.nt_of(blk), sl, tp, rs, up0);
+      if (split) {
+        const float *sDelta = sc.fset(blk & 1, Lay::oDelta);
+#pragma unroll
+        for (int k = 0; k < S::kSlots; ++k) {
+          const float4 dl = *reinterpret_cast<const float4 *>(sDelta + sl.c[k] * ROW + sl.t);
+          psum[k] += (dl.x + dl.y) + (dl.z + dl.w);
+        }
+      }
       mbar_arrive(sc.hand(kTilesReady, blk & 1));
     }
-    // the prep warps waited on every raw block: their phases seed the
-    // correction pass
-    if (tp == 0) misc[2] = static_cast<int>(phase);
   } else {
     const typename S::Slots sl = sc.make_slots(te);
     for (int j = 0; j < STAGES; ++j) sc.produce(j, nblk, te, NEPI);
@@ -789,8 +664,6 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     }
   }
   if (!ok) atomicOr(p.status, kStatusTimeout);
-  __syncthreads();
-  phase = static_cast<uint32_t>(misc[2]);
 
   if (!split) {
     if (p.last_state) {
@@ -801,156 +674,361 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
     return;
   }
 
-  // ---- split mode: publish, look back, publish the true end state, correct
-  const int64_t stride = static_cast<int64_t>(2) * CH * NP;
-  float *my_agg = p.agg + item * stride;
-  float *my_incl = p.incl + item * static_cast<int64_t>(CH * NP);
-  const bool drop = (p.test_flags & 1u) && k == 1 && tile == 0;
-  float P[4];
+  // ---- split mode: the chunk's pair (P, e) for the prefix launch, which
+  // also writes the final state; the carried terms are added by the carry
+  // launch
+  float *my_agg = p.agg + item * static_cast<int64_t>(2) * CH * NP;
+  if (is_scan) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) P[i] = ex2_mufu(alpha[i] * dsum);
-
-  // only the scan warps hold states; the aux warps take part in the
-  // barriers but write nothing
-  float h_in[4] = {0.f, 0.f, 0.f, 0.f};
-  if (k == 0) {
-    if (is_scan) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) my_incl[(4 * g + i) * CH + lane] = h[i];
+    for (int i = 0; i < 4; ++i) {
+      my_agg[(4 * g + i) * CH + lane] = ex2_mufu(alpha[i] * dsum);
+      my_agg[CH * NP + (4 * g + i) * CH + lane] = h[i];
     }
-  } else {
-    if (is_scan) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        my_agg[(4 * g + i) * CH + lane] = P[i];
-        my_agg[CH * NP + (4 * g + i) * CH + lane] = h[i];
+  }
+}
+
+// ------------------------------------------------------ split: prefix
+// One warp per (tile, state, channel) composes the chunks' pairs in chunk
+// order into incl_k = P_k incl_{k-1} + e_k, the true state at the end of
+// chunk k (incl_0 = e_0: the first chunk started from h0), and writes the
+// final state.  Lane l takes a run of consecutive chunks: it composes its
+// run, the warp scans the runs' pairs (composition is associative: "The
+// relay"), and the lane replays its run from the state before it.  Under
+// MSS_TESTFLAG_DROP_PUBLISH the first warp first waits for a word of the
+// workspace that nothing sets, bounded by the caller's spin timeout, and
+// records the timeout in the status word.
+__global__ void __launch_bounds__(128) scan_prefix_kernel(const ScanParams p, int np) {
+  const int lane = threadIdx.x & 31;
+  const int64_t chain = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t per_tile = static_cast<int64_t>(np) * CH;
+  if (chain >= p.tiles * per_tile) return;  // warp-uniform
+  if ((p.test_flags & 1u) && chain == 0 && lane == 0) {
+    const uint64_t limit = p.spin_timeout_ns > 0 ? static_cast<uint64_t>(p.spin_timeout_ns)
+                                                 : 1000000000ull;
+    const uint64_t start = global_timer_ns();
+    while (ld_acquire_gpu(p.status + 2) == 0u) {
+      if (global_timer_ns() - start > limit) {
+        atomicOr(p.status, kStatusTimeout);
+        break;
       }
+      __nanosleep(1000);
+    }
+  }
+  __syncwarp();
+  const int64_t tile = chain / per_tile;
+  const int r = static_cast<int>(chain % per_tile);  // state * CH + channel
+  const int64_t stride = 2 * per_tile;
+  const int run = (p.splits + 31) / 32;
+  const int k0 = min(p.splits, lane * run), k1 = min(p.splits, k0 + run);
+  auto pair = [&](int k, float &P, float &e) {
+    const int64_t item = static_cast<int64_t>(k) * p.tiles + tile;
+    P = k == 0 ? 0.f : p.agg[item * stride + r];  // nothing precedes chunk 0
+    e = p.agg[item * stride + per_tile + r];
+  };
+  // this lane's run as one pair: h -> P h + E
+  float P = 1.f, E = 0.f;
+  for (int k = k0; k < k1; ++k) {
+    float pk, ek;
+    pair(k, pk, ek);
+    E = fmaf(pk, E, ek);
+    P *= pk;
+  }
+  // inclusive scan of the runs: the earlier pair applied first
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float Po = __shfl_up_sync(0xffffffffu, P, o);
+    const float Eo = __shfl_up_sync(0xffffffffu, E, o);
+    if (lane >= o) {
+      E = fmaf(P, Eo, E);
+      P *= Po;
+    }
+  }
+  // state before this lane's run, then the run replayed
+  float h = __shfl_up_sync(0xffffffffu, E, 1);
+  if (lane == 0) h = 0.f;
+  for (int k = k0; k < k1; ++k) {
+    float pk, ek;
+    pair(k, pk, ek);
+    h = fmaf(pk, h, ek);
+    p.incl[(static_cast<int64_t>(k) * p.tiles + tile) * per_tile + r] = h;
+  }
+  if (p.last_state && k1 == p.splits && k0 < k1) {
+    const int n = r / CH, c = r % CH;
+    const int64_t b = tile / p.ch_tiles, d = (tile % p.ch_tiles) * CH + c;
+    if (d < p.dim && n < p.dstate) p.last_state[(b * p.dim + d) * p.dstate + n] = h;
+  }
+}
+
+// ------------------------------------------------------- split: carry
+// 16-byte asynchronous copy global -> shared (through L2 only), tracked by
+// the thread's groups.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// wait until at most N of this thread's committed groups are in flight
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The piece of a 16-step row that thread-level copy unit `w` (elements
+// w .. w + 16/sizeof(T) - 1) covers: one asynchronous copy when the row is
+// whole and aligned, element loads of the steps inside the chunk otherwise.
+template <typename T>
+__device__ __forceinline__ void stage_piece(T *dst, const T *row, int w, int nt, bool vec) {
+  constexpr int EL = 16 / static_cast<int>(sizeof(T));
+  if (vec && nt == TB) {
+    cp_async16(dst + w, row + w);
+  } else {
+    for (int e = 0; e < EL && w + e < nt; ++e) dst[w + e] = row[w + e];
+  }
+}
+
+// One block per (tile, chunk k >= 1, segment of kSegBlocks blocks): adds
+// silu(z_t) * sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n] to the segment's y,
+// block by block, until every term has decayed below the cutoff.  Warp g
+// takes the states g + G i (i < 4), so every warp holds slow and fast
+// states, and skips a state once its term is below the cutoff in all its
+// lanes (lane = channel).  The raw delta, z, C and old y of a block are
+// staged in shared memory two blocks ahead (three buffers).
+template <typename InT, typename OutT, int G, bool VARLEN>
+__global__ void __launch_bounds__(32 * G) scan_carry_kernel(const ScanParams p) {
+  constexpr int NP = 4 * G;
+  constexpr int NT = 32 * G;
+  constexpr int QT = TB / 4;
+  __shared__ __align__(16) InT rD[3][CH * TB];
+  __shared__ __align__(16) InT rZ[3][CH * TB];
+  __shared__ __align__(16) InT rC[3][NP * TB];
+  __shared__ __align__(16) OutT rY[3][CH * TB];
+  __shared__ __align__(16) float sDl[CH * ROW];
+  __shared__ __align__(16) float sPart[G][CH * ROW];
+  __shared__ float sBias[CH];
+
+  const int tid = threadIdx.x, lane = tid & 31, g = tid >> 5;
+  const int64_t unit = blockIdx.x;
+  const int seg = static_cast<int>(unit % p.nseg);
+  const int64_t rest = unit / p.nseg;
+  const int64_t tile = rest % p.tiles;
+  const int64_t k = rest / p.tiles + 1;
+  const int64_t item = k * p.tiles + tile;
+  const int64_t b = tile / p.ch_tiles, d0 = (tile % p.ch_tiles) * CH;
+  const int64_t t_begin = k * p.chunk;
+  const int64_t t_end = min64(t_begin + p.chunk, p.seqlen);
+  const int nblk = static_cast<int>((t_end - t_begin + TB - 1) / TB);
+  const int blk0 = seg * p.segb;
+  if (blk0 >= nblk) return;
+  const int blk1 = min(nblk, blk0 + p.segb);
+
+  // this lane's states g + G i: rate, carried state, still-active mask
+  const int64_t d = d0 + lane;
+  const bool dvalid = d < p.dim;
+  float sigma = p.sig[(item * p.nseg + seg) * CH + lane];
+  float alpha[4], hin[4];
+  unsigned act = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = g + G * i;
+    const bool live = dvalid && n < p.dstate &&
+                      dbg_index_ok(d * p.dstate + n, p.dim * p.dstate, p.status);
+    alpha[i] = live ? p.A[d * p.dstate + n] * kLog2e : 0.f;
+    if (VARLEN && alpha[i] == 0.f) alpha[i] = -1e-30f;
+    hin[i] = live ? p.incl[(item - p.tiles) * NP * CH + n * CH + lane] : 0.f;
+    if (__any_sync(0xffffffffu, hin[i] != 0.f && !(alpha[i] * sigma < kCutoffLog2)))
+      act |= 1u << i;
+  }
+  if (tid < CH) {
+    const bool ok = d0 + tid < p.dim;
+    sBias[tid] = (ok && p.delta_bias) ? p.delta_bias[d0 + tid] : 0.f;
+  }
+  if (!__syncthreads_or(act != 0u)) return;
+
+  const bool has_z = p.z != nullptr;
+  auto vec_ok = [&](const void *ptr, const int64_t (&st)[2], int es) {
+    return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0 && (st[0] * es) % 16 == 0 &&
+           (st[1] * es) % 16 == 0;
+  };
+  const bool vD = vec_ok(p.delta, p.sdl, sizeof(InT));
+  const bool vZ = has_z && vec_ok(p.z, p.sz, sizeof(InT));
+  const bool vC = vec_ok(p.C, p.sC, sizeof(InT));
+  const bool vY = vec_ok(p.y, p.sy, sizeof(OutT));
+  constexpr int PI = TB * static_cast<int>(sizeof(InT)) / 16;   // copy units per input row
+  constexpr int PO = TB * static_cast<int>(sizeof(OutT)) / 16;  // per y row
+  constexpr int EI = 16 / static_cast<int>(sizeof(InT)), EO = 16 / static_cast<int>(sizeof(OutT));
+  constexpr int NU = 2 * CH * PI + NP * PI + CH * PO;
+  auto stage = [&](int j, int buf) {
+    const int64_t t0 = t_begin + static_cast<int64_t>(j) * TB;
+    const int nt = static_cast<int>(min64(TB, t_end - t0));
+    for (int q = tid; q < NU; q += NT) {
+      if (q < CH * PI) {
+        const int c = q / PI, w = (q % PI) * EI;
+        if (d0 + c < p.dim)
+          stage_piece(rD[buf] + c * TB, static_cast<const InT *>(p.delta) + b * p.sdl[0] +
+                                            (d0 + c) * p.sdl[1] + t0,
+                      w, nt, vD);
+      } else if (q < 2 * CH * PI) {
+        const int qq = q - CH * PI, c = qq / PI, w = (qq % PI) * EI;
+        if (has_z && d0 + c < p.dim)
+          stage_piece(rZ[buf] + c * TB, static_cast<const InT *>(p.z) + b * p.sz[0] +
+                                            (d0 + c) * p.sz[1] + t0,
+                      w, nt, vZ);
+      } else if (q < 2 * CH * PI + NP * PI) {
+        const int qq = q - 2 * CH * PI, n = qq / PI, w = (qq % PI) * EI;
+        if (n < p.dstate)
+          stage_piece(rC[buf] + n * TB,
+                      static_cast<const InT *>(p.C) + b * p.sC[0] + n * p.sC[1] + t0, w, nt, vC);
+      } else {
+        const int qq = q - 2 * CH * PI - NP * PI, c = qq / PO, w = (qq % PO) * EO;
+        if (d0 + c < p.dim)
+          stage_piece(rY[buf] + c * TB, static_cast<const OutT *>(p.y) + b * p.sy[0] +
+                                            (d0 + c) * p.sy[1] + t0,
+                      w, nt, vY);
+      }
+    }
+    cp_async_commit();
+  };
+
+  stage(blk0, 0);
+  if (blk0 + 1 < blk1)
+    stage(blk0 + 1, 1);
+  else
+    cp_async_commit();
+  for (int j = blk0; j < blk1; ++j) {
+    const int buf = (j - blk0) % 3;
+    const int64_t t0 = t_begin + static_cast<int64_t>(j) * TB;
+    const int nt = static_cast<int>(min64(TB, t_end - t0));
+    // block j's copies (this thread's, then everyone's) have landed; block
+    // j - 1 is consumed, so its buffer may take block j + 2
+    cp_async_wait<1>();
+    __syncthreads();
+    if (j + 2 < blk1)
+      stage(j + 2, (j - blk0 + 2) % 3);
+    else
+      cp_async_commit();
+    // Delta = softplus(delta + bias), zero past the chunk, infinite where a
+    // packed sequence restarts
+    for (int qd = tid; qd < CH * QT; qd += NT) {
+      const int c = qd / QT, t = 4 * (qd % QT);
+      float4 dl = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (d0 + c < p.dim && t < nt) {
+        const InT *r = rD[buf] + c * TB + t;
+        const float bias = sBias[c];
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = t + e < nt ? to_f32<InT>(r[e]) + bias : 0.f;
+        if (p.softplus) {
+          const float2 a = softplus2_f(make_float2(v[0], v[1]));
+          const float2 c2 = softplus2_f(make_float2(v[2], v[3]));
+          v[0] = a.x; v[1] = a.y; v[2] = c2.x; v[3] = c2.y;
+        }
+        dl = make_float4(t < nt ? v[0] : 0.f, t + 1 < nt ? v[1] : 0.f, t + 2 < nt ? v[2] : 0.f,
+                         t + 3 < nt ? v[3] : 0.f);
+        if (VARLEN && p.cu) {
+          // binary search for the first sequence start at or after t0 + t
+          const int64_t pos = t0 + t;
+          int64_t lo = 1, hi = p.nseq;
+          while (lo < hi) {
+            const int64_t mid = lo + (hi - lo) / 2;
+            if (__ldg(p.cu + mid) < pos) lo = mid + 1; else hi = mid;
+          }
+          const float inf = __int_as_float(0x7f800000);
+          for (int64_t nb = lo; nb < p.nseq && __ldg(p.cu + nb) < pos + 4; ++nb) {
+            const int e = static_cast<int>(__ldg(p.cu + nb) - pos);
+            if (e == 0) dl.x = inf;
+            if (e == 1) dl.y = inf;
+            if (e == 2) dl.z = inf;
+            if (e == 3) dl.w = inf;
+          }
+        }
+      }
+      *reinterpret_cast<float4 *>(sDl + c * ROW + t) = dl;
     }
     __syncthreads();
-    if (tid == 0 && !drop) {
-      __threadfence();
-      st_release_gpu(&p.flags[item], 1u);
-    }
-    float pacc[4] = {1.f, 1.f, 1.f, 1.f};
-    for (int64_t j = k - 1; j >= 0; --j) {
-      const int64_t pred = j * p.tiles + tile;
-      if (tid == 0) {
-        unsigned f = ld_acquire_gpu(&p.flags[pred]);
-        const uint64_t start = global_timer_ns();
-        const uint64_t limit = p.spin_timeout_ns > 0
-                                   ? static_cast<uint64_t>(p.spin_timeout_ns)
-                                   : 1000000000ull;
-        for (uint32_t it = 0; f == 0u; ++it) {
-          if ((it > 64u && global_timer_ns() - start > limit) || it > (1u << 30)) {
-            atomicOr(p.status, kStatusTimeout);
-            break;
+    // this warp's share of the carried terms of block j
+    {
+      float *share = sPart[g];
+      if (act == 0u) {
+#pragma unroll
+        for (int q = 0; q < QT; ++q)
+          *reinterpret_cast<float4 *>(share + lane * ROW + 4 * q) = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+#pragma unroll
+        for (int q = 0; q < QT; ++q) {
+          const float4 dl = *reinterpret_cast<const float4 *>(sDl + lane * ROW + 4 * q);
+          float2 s01, s23;  // sigma after steps 4q .. 4q + 3
+          sigma += dl.x;
+          s01.x = sigma;
+          sigma += dl.y;
+          s01.y = sigma;
+          sigma += dl.z;
+          s23.x = sigma;
+          sigma += dl.w;
+          s23.y = sigma;
+          float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (!((act >> i) & 1u)) continue;
+            const float4 cq = load4_f32(rC[buf] + (g + G * i) * TB + 4 * q);
+            const float2 a2 = make_float2(alpha[i], alpha[i]), h2 = make_float2(hin[i], hin[i]);
+            const float2 x01 = __fmul2_rn(a2, s01), x23 = __fmul2_rn(a2, s23);
+            p01 = __ffma2_rn(__fmul2_rn(make_float2(cq.x, cq.y), h2),
+                             make_float2(ex2_mufu(x01.x), ex2_mufu(x01.y)), p01);
+            p23 = __ffma2_rn(__fmul2_rn(make_float2(cq.z, cq.w), h2),
+                             make_float2(ex2_mufu(x23.x), ex2_mufu(x23.y)), p23);
           }
-          __nanosleep(128);
-          f = ld_acquire_gpu(&p.flags[pred]);
+          *reinterpret_cast<float4 *>(share + lane * ROW + 4 * q) =
+              make_float4(p01.x, p01.y, p23.x, p23.y);
         }
-        misc[1] = static_cast<int>(f);
-      }
-      __syncthreads();
-      const unsigned f = static_cast<unsigned>(misc[1]);
-      bool done = true;
-      if (f == 2u) {
-        const float *pi = p.incl + pred * static_cast<int64_t>(CH * NP);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          h_in[i] = fmaf(pacc[i], __ldcg(&pi[(4 * g + i) * CH + lane]), h_in[i]);
-      } else if (f == 1u) {
-        const float *pa = p.agg + pred * stride;
+          if (!__any_sync(0xffffffffu, hin[i] != 0.f && !(alpha[i] * sigma < kCutoffLog2)))
+            act &= ~(1u << i);
+      }
+    }
+    const bool more = __syncthreads_or(act != 0u);
+    // y += silu(z) * (sum of the shares), four steps of one channel per thread
+    for (int qd = tid; qd < CH * QT; qd += NT) {
+      const int c = qd / QT, t = 4 * (qd % QT);
+      if (d0 + c >= p.dim || t >= nt) continue;
+      float4 sv = *reinterpret_cast<const float4 *>(sPart[0] + c * ROW + t);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          h_in[i] = fmaf(pacc[i], __ldcg(&pa[CH * NP + (4 * g + i) * CH + lane]), h_in[i]);
-          pacc[i] *= __ldcg(&pa[(4 * g + i) * CH + lane]);
-          if (live[i] && pacc[i] != 0.f) done = false;
+      for (int w = 1; w < G; ++w) {
+        const float4 v = *reinterpret_cast<const float4 *>(sPart[w] + c * ROW + t);
+        sv.x += v.x; sv.y += v.y; sv.z += v.z; sv.w += v.w;
+      }
+      float o[4] = {sv.x, sv.y, sv.z, sv.w};
+      const OutT *yo = rY[buf] + c * TB + t;
+      const InT *zr = rZ[buf] + c * TB + t;
+      const int64_t yi = b * p.sy[0] + (d0 + c) * p.sy[1] + t0 + t;
+      OutT *yr = static_cast<OutT *>(p.y) + yi;
+      if (!dbg_index_ok(yi + min(nt - t, 4) - 1, p.ext_y, p.status)) continue;
+      if (t + 4 <= nt) {
+        if (has_z) {
+          const float4 z = load4_f32(zr);
+          const float2 g01 = silu2_f(make_float2(z.x, z.y));
+          const float2 g23 = silu2_f(make_float2(z.z, z.w));
+          o[0] *= g01.x; o[1] *= g01.y; o[2] *= g23.x; o[3] *= g23.y;
+        }
+        const float4 old = load4_f32(yo);
+        const float4 nv = make_float4(old.x + o[0], old.y + o[1], old.z + o[2], old.w + o[3]);
+        if (p.y_vec) {
+          store4(yr, nv);
+        } else {
+          const float nvs[4] = {nv.x, nv.y, nv.z, nv.w};
+          for (int e = 0; e < 4; ++e) yr[e] = from_f32<OutT>(nvs[e]);
+        }
+      } else {
+        for (int e = 0; e < 4 && t + e < nt; ++e) {
+          const float gate = has_z ? silu_f(to_f32<InT>(zr[e])) : 1.f;
+          yr[e] = from_f32<OutT>(to_f32<OutT>(yo[e]) + o[e] * gate);
         }
       }
-      if (__syncthreads_and(done)) break;
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = fmaf(P[i], h_in[i], h[i]);
-    if (is_scan) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) my_incl[(4 * g + i) * CH + lane] = h[i];
-    }
+    if (!more) break;
   }
-  __syncthreads();
-  if (tid == 0 && !drop) {
-    __threadfence();
-    st_release_gpu(&p.flags[item], 2u);
-  }
-  if (p.last_state && sc.t_end == p.seqlen) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (live[i]) p.last_state[(b * p.dim + d) * p.dstate + 4 * g + i] = h[i];
-  }
-  if (k == 0) return;
-
-  // ------------------------------------------------------ correction pass
-  // y_t += silu(z_t) * sum_n C_t[n] 2^(alpha[n] sigma_t) h_in[n], block by
-  // block from the chunk start until every carried term has decayed.  The
-  // ring continues at stage nblk so the barrier phases stay consistent.
-  // Pipelined over one barrier per block: while the scan warps add block
-  // i's carried term into share set i & 1, the other warps finish block
-  // i - 1 (old y + gate * shares), load block i's old y and turn block
-  // i + 1's raw tiles into step sizes in tile set (i + 1) & 1.
-  bool need = false;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) need |= live[i] && h_in[i] != 0.f;
-  if (tid == 0) misc[3] = 0;  // set by a wait that runs out
-  if (!__syncthreads_or(need)) return;
-  float sigma = 0.f;
-  bool wactive = true;  // this scan warp still has carried terms to add
-  const int base = nblk % STAGES;
-  const int ta = tid - NSCAN;  // index within the other warps
-  constexpr int NAUX = NALL - NSCAN;
-  static_assert(NAUX == CH * (TB / 4), "one y quad of a block per non-scan thread");
-  for (int j = 0; j < PREFETCH; ++j) sc.request(j, nblk, base, tid, NALL);
-  float4 yq = make_float4(0.f, 0.f, 0.f, 0.f);  // old y of the block in flight
-  if (!is_scan) {
-    if (!sc.land(0, nblk, base, phase)) misc[3] = 1;
-    sc.prep(base % STAGES, 0, sc.t0_of(0), sc.nt_of(0), false, ta, NAUX);
-  }
-  __syncthreads();
-  for (int i = 0; i < nblk; ++i) {
-    if (misc[3] != 0) {
-      if (tid == 0) atomicOr(p.status, kStatusTimeout);
-      return;
-    }
-    const int set = i & 1;
-    if (is_scan) {
-      sc.scan_carry(set, g, lane, alpha, h_in, sigma, wactive);
-      need = false;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        need |= live[q] && h_in[q] != 0.f && !(alpha[q] * sigma < kCutoffLog2);
-      wactive = __any_sync(0xffffffffu, need);
-    } else {
-      if (i >= 1)
-        sc.epilogue_acc((base + i - 1) % STAGES, set ^ 1, i - 1, ta, yq);
-      yq = sc.load_y_quad(i, ta);
-      if (i + 1 < nblk) {
-        if (!sc.land(i + 1, nblk, base, phase)) misc[3] = 1;
-        sc.prep((base + i + 1) % STAGES, set ^ 1, sc.t0_of(i + 1), sc.nt_of(i + 1), false, ta,
-                NAUX);
-      }
-    }
-    if (!__syncthreads_or(need) || i + 1 == nblk) {
-      // block i's outputs; copies already requested must land before the
-      // block exits (blocks up to i + 1 have landed)
-      if (!is_scan) {
-        sc.epilogue_acc((base + i) % STAGES, set, i, ta, yq);
-        bool okd = true;
-        for (int j = i + 2; j < i + PREFETCH && j < nblk; ++j)
-          okd &= sc.land(j, nblk, base, phase);
-        if (!okd && ta == 0) atomicOr(p.status, kStatusTimeout);
-      }
-      return;
-    }
-    sc.request(i + PREFETCH, nblk, base, tid, NALL);
-  }
+  cp_async_wait<0>();  // no copy may land after the block has left
 }
 
 // ------------------------------------------------------------ host side
@@ -1024,6 +1102,16 @@ cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t 
   if (e != cudaSuccess) return e;
   const int64_t grid = p.tiles * p.splits;
   kern<<<static_cast<unsigned>(grid), 32 * (G + kAuxWarps), smem, s>>>(p, maps);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits <= 1) return e;
+  // split scans: the chunks' true start states, then the carried terms
+  const int64_t threads = p.tiles * 4 * G * CH * 32;  // one warp per chain
+  scan_prefix_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, s>>>(p, 4 * G);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t units = p.tiles * (p.splits - 1) * p.nseg;
+  scan_carry_kernel<InT, OutT, G, MODE == kModeVarlen>
+      <<<static_cast<unsigned>(units), 32 * G, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -1082,32 +1170,42 @@ int occupancy_g(int groups) {
 // groups 3 runs on the 4-group kernel (the fourth group's states are padding)
 static int kernel_groups(int groups) { return groups == 3 ? 4 : groups; }
 
-size_t scan_workspace_clear_bytes(int64_t tiles, int splits) {
-  const size_t items = static_cast<size_t>(tiles) * splits;
-  return 256 + ((items * sizeof(unsigned) + 255) / 256) * 256;
+size_t scan_workspace_clear_bytes() { return 256; }
+
+static int64_t segments_per_chunk(int64_t chunk) {
+  const int64_t nblk = (chunk + TB - 1) / TB;
+  return (nblk + kSegBlocks - 1) / kSegBlocks;
 }
 
-size_t scan_workspace_bytes(int64_t tiles, int splits, int groups) {
+static size_t round256(size_t n) { return ((n + 255) / 256) * 256; }
+
+size_t scan_workspace_bytes(int64_t tiles, int splits, int64_t chunk, int groups) {
   if (splits <= 1) return 0;
   const size_t items = static_cast<size_t>(tiles) * splits;
   const size_t np = 4 * static_cast<size_t>(kernel_groups(groups));
   const size_t agg = items * 2 * CH * np * sizeof(float);
   const size_t incl = items * CH * np * sizeof(float);
-  return scan_workspace_clear_bytes(tiles, splits) + ((agg + 255) / 256) * 256 +
-         ((incl + 255) / 256) * 256;
+  const size_t sig = items * static_cast<size_t>(segments_per_chunk(chunk)) * CH * sizeof(float);
+  return scan_workspace_clear_bytes() + round256(agg) + round256(incl) + round256(sig);
 }
 
+// Layout: status word, ticket and the word the test flag waits for in the
+// first 256 bytes, then the chunks' pairs, their true end states and the running
+// sums of Delta at the segment starts.
 void scan_bind_workspace(ScanParams &p, void *ws, int groups) {
   char *base = static_cast<char *>(ws);
   const size_t items = static_cast<size_t>(p.tiles) * p.splits;
   const size_t np = 4 * static_cast<size_t>(kernel_groups(groups));
   p.status = reinterpret_cast<unsigned *>(base);
   p.ticket = reinterpret_cast<unsigned *>(base + 4);
-  p.flags = reinterpret_cast<unsigned *>(base + 256);
-  const size_t clear = scan_workspace_clear_bytes(p.tiles, p.splits);
-  p.agg = reinterpret_cast<float *>(base + clear);
-  const size_t agg = ((items * 2 * CH * np * sizeof(float) + 255) / 256) * 256;
-  p.incl = reinterpret_cast<float *>(base + clear + agg);
+  size_t off = scan_workspace_clear_bytes();
+  p.agg = reinterpret_cast<float *>(base + off);
+  off += round256(items * 2 * CH * np * sizeof(float));
+  p.incl = reinterpret_cast<float *>(base + off);
+  off += round256(items * CH * np * sizeof(float));
+  p.sig = reinterpret_cast<float *>(base + off);
+  p.segb = kSegBlocks;
+  p.nseg = static_cast<int>(segments_per_chunk(p.chunk));
 }
 
 // The word's device address, looked up once per device (with that device

@@ -49,11 +49,14 @@ struct ScanParams {
   int64_t tiles;   // batch * ch_tiles
   // device-side status word (workspace when split, library word otherwise)
   unsigned *status;
-  // split-mode workspace
+  // split-mode workspace: next item to hand out, then per item
+  // (chunk-major: chunk * tiles + tile)
   unsigned *ticket;
-  unsigned *flags;
-  float *agg;      // per item: decay product P then local end state e
-  float *incl;     // per item: true state at the end of the chunk
+  float *agg;      // decay product P over the chunk, then local end state e
+  float *incl;     // true state at the end of the chunk
+  float *sig;      // running sum of Delta at the start of every segment
+  int segb;        // 16-step blocks per correction segment
+  int nseg;        // segments per chunk
   unsigned test_flags;
   int64_t spin_timeout_ns;
   // element extents (largest index + 1) of the streamed tensors under their
@@ -66,15 +69,19 @@ struct TmaMaps {
   CUtensorMap u, delta, z, B, C;
 };
 
-// Workspace bytes for `splits` chunks over `tiles` tiles with `groups`
-// state groups (0 when splits == 1).
-size_t scan_workspace_bytes(int64_t tiles, int splits, int groups);
+// Blocks of kTimeBlock steps per correction segment of a split scan.
+constexpr int kSegBlocks = 32;
+
+// Workspace bytes for `splits` chunks of `chunk` steps over `tiles` tiles
+// with `groups` state groups (0 when splits == 1).
+size_t scan_workspace_bytes(int64_t tiles, int splits, int64_t chunk, int groups);
 
 // Carves the workspace into the fields of `p`.
 void scan_bind_workspace(ScanParams &p, void *ws, int groups);
 
-// Bytes of the header + flag region that must be zero before a launch.
-size_t scan_workspace_clear_bytes(int64_t tiles, int splits);
+// Bytes at the start of the workspace (the status word) that must be zero
+// before a launch.
+size_t scan_workspace_clear_bytes();
 
 // Device address of the library's own status word (used when a scan has no
 // workspace); nullptr on failure.

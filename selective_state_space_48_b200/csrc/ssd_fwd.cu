@@ -20,8 +20,8 @@
 // carried in tensor memory (fp32) across the whole sequence and never
 // touches HBM.  Warp roles: warp 0 issues the TMA loads of the C, B and X
 // tiles (two stages), warp 1 allocates tensor memory and issues the
-// tcgen05.mma products (one thread), warps 2-9 (256 threads, one tensor
-// memory lane quarter per pair of warps, which split the columns) compute
+// tcgen05.mma products (one thread), warps 2-17 (512 threads, four warps
+// per tensor memory lane quarter, which split the columns) compute
 // the step sizes and their running sum, build the operand S' in tensor
 // memory and X'' and Hp in shared memory, rescale H, and write y.  The state products (YO and H)
 // are issued as soon as Hp and X'' are ready, so they run while the
@@ -52,10 +52,10 @@ namespace ssd {
 constexpr int Q = 128;   // chunk length
 constexpr int P = 64;    // headdim
 constexpr int NS = 128;  // dstate
-constexpr int kThreads = 320;  // 2 issue warps + 8 epilogue warps
-constexpr int kEpi = 256;
-constexpr int kEpiBarrier = 1;  // named barrier of the eight epilogue warps
-constexpr int kHalfBarrier = 2; // + e: named barrier of the four warps of half e
+constexpr int kThreads = 576;  // 2 issue warps + 16 epilogue warps
+constexpr int kEpi = 512;
+constexpr int kEpiBarrier = 1;  // named barrier of the sixteen epilogue warps
+constexpr int kHalfBarrier = 2; // + half: named barrier of the eight warps of a y half
 
 constexpr int kTile = Q * 64 * 2;      // one [128][64] bf16 tile
 constexpr int kStage = 5 * kTile;      // C (two n halves), B (two), X
@@ -202,6 +202,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "r"(taddr));
 }
 
+// 16 consecutive fp32 columns of this thread's lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+
 // The loaded registers are valid only after tcgen05.wait::ld; threading
 // them through the wait keeps the compiler from using them earlier.
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[32]) {
@@ -212,6 +223,14 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[32]) {
                  "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
                  "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]),
                  "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
                :
                : "memory");
 }
@@ -485,28 +504,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------- epilogue
-    // Two warps per tensor-memory lane quarter: e = 0 / 1 split the columns.
+    // Four warps per tensor-memory lane quarter: e = 0 .. 3 takes columns
+    // 16e .. 16e + 15 of the 64-wide products and score block e of the
+    // masked scores; y is written in two 32-column halves (e / 2).
     const int q = warp & 3;
     const int e = (warp - 2) >> 2;
+    const int half = e >> 1, sub = e & 1;
     const int r = 32 * q + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
     const float Dh = p.D ? p.D[h] : 0.0f;
     const int64_t H = p.H;
-    // one thread per half issues the half's y stores (first lane of the
-    // half's first warp)
-    const bool writer = lane == 0 && q == 2;
+    // one thread per half issues the half's y stores (first lane of one of
+    // the half's warps)
+    const bool writer = lane == 0 && q == 2 && sub == 0;
     const StepPlan plan{cum_s, step_s, colf_s, tot_s,
                         p.dt + static_cast<int64_t>(b) * p.L * H + h, p.L, H,
                         p.A[h] * kLog2e, p.dt_bias ? p.dt_bias[h] : 0.0f, p.softplus};
 
-    // the initial state into H (row n = r, columns 32e .. 32e + 31)
+    // the initial state into H (row n = r, columns 16e .. 16e + 15)
     {
       const float *h0 = p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * P * NS : nullptr;
-      uint32_t v[32];
+      uint32_t v[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        v[j] = __float_as_uint(h0 ? h0[(e * 32 + j) * NS + r] : 0.0f);
-      tmem_st32(tl + kColH + 32 * e, v);
+      for (int j = 0; j < 16; ++j)
+        v[j] = __float_as_uint(h0 ? h0[(e * 16 + j) * NS + r] : 0.0f);
+      tmem_st16(tl + kColH + 16 * e, v);
       tmem_wait_st();
     }
 
@@ -522,14 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       unsigned char *s = sm + st * kStage;
       const int64_t t = static_cast<int64_t>(c) * Q + r;
 
-      // S' row t, blocks gb = e and e + 2 of 32 columns: below the diagonal
+      // S' row t, block gb = e of 32 columns: below the diagonal
       // S 2^(c_t - c_end(gb)) colf[s] (both factors <= 1); on the diagonal
       // S 2^(c_t - c_s) Delta_s for s <= t, factored the same way when that
       // cannot overflow; above it zero
       sy.wait(kSFull, c & 1);
       tc_fence_after();
-#pragma unroll 1
-      for (int gb = e; gb < 4; gb += 2) {
+      {
+        const int gb = e;
         uint32_t pk[16];
         if (gb < q) {
           uint32_t v[32];
@@ -596,37 +618,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sy.wait(kFull + st, (c >> 1) & 1);
 
-      // Hp row n = r (columns of half e): bf16 copy of the state before
-      // this chunk; then the state decays over the chunk: H *= 2^(c_last)
+      // Hp row n = r (columns 16e .. 16e + 15): bf16 copy of the state
+      // before this chunk; then the state decays over the chunk:
+      // H *= 2^(c_last)
       {
         const float gam = ex2_mufu(cl);
-        uint32_t v[32];
-        tmem_ld32(tl + kColH + 32 * e, v);
+        uint32_t v[16];
+        tmem_ld16(tl + kColH + 16 * e, v);
         tmem_wait_ld(v);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 2; ++k) {
           uint4 o;
           o.x = pack_bf16(__uint_as_float(v[8 * k + 0]), __uint_as_float(v[8 * k + 1]));
           o.y = pack_bf16(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3]));
           o.z = pack_bf16(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5]));
           o.w = pack_bf16(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7]));
-          *reinterpret_cast<uint4 *>(sm + oHp + swz(r, e * 4 + k)) = o;
+          *reinterpret_cast<uint4 *>(sm + oHp + swz(r, e * 2 + k)) = o;
         }
         // the carried-state readout YO = C Hp may start now
         fence_async_smem();
         mbar_arrive(bar + kReadyHp);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam);
-        tmem_st32(tl + kColH + 32 * e, v);
+        for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam);
+        tmem_st16(tl + kColH + 16 * e, v);
         tmem_wait_st();
       }
-      // X'' row s = r, four of its eight 16-byte chunks (the XOR with the
+      // X'' row s = r, two of its eight 16-byte chunks (the XOR with the
       // row keeps the eight rows of a shared-memory phase on distinct banks)
       {
         const float w = step_s[r] * ex2_mufu(cl - cum);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t off = static_cast<uint32_t>(r * 128 + (((e * 4 + k) ^ (r & 7)) << 4));
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t off = static_cast<uint32_t>(r * 128 + (((e * 2 + k) ^ (r & 7)) << 4));
           const uint4 xv = *reinterpret_cast<const uint4 *>(s + oX + off);
           const float2 a0 = unpack_bf16(xv.x), a1 = unpack_bf16(xv.y);
           const float2 a2 = unpack_bf16(xv.z), a3 = unpack_bf16(xv.w);
@@ -647,20 +670,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         cl = cum_s[Q - 1];
       }
 
-      // y row t, columns of half e: Y + 2^(c_t) YO + D x, gated
+      // y row t, columns 16e .. 16e + 15: Y + 2^(c_t) YO + D x, gated
       sy.wait(kDoneY, c & 1);
       tc_fence_after();
       {
         const float eo = ex2_mufu(cum_t);
-        uint32_t yv[32], ov[32];
-        tmem_ld32(tl + kColY + 32 * e, yv);
-        tmem_ld32(tl + kColYO + 32 * e, ov);
+        uint32_t yv[16], ov[16];
+        tmem_ld16(tl + kColY + 16 * e, yv);
+        tmem_ld16(tl + kColYO + 16 * e, ov);
         tmem_wait_ld(yv);
         tmem_wait_ld(ov);
-        float out[32];
+        float out[16];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint4 xv = *reinterpret_cast<const uint4 *>(s + oX + swz(r, e * 4 + k));
+        for (int k = 0; k < 2; ++k) {
+          const uint4 xv = *reinterpret_cast<const uint4 *>(s + oX + swz(r, e * 2 + k));
           const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -672,10 +695,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (p.z && t < p.L) {
-          const int64_t row = ((static_cast<int64_t>(b) * p.L + t) * H + h) * P + 32 * e;
+          const int64_t row = ((static_cast<int64_t>(b) * p.L + t) * H + h) * P + 16 * e;
           const uint4 *zr = reinterpret_cast<const uint4 *>(p.z + row);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 2; ++k) {
             const uint4 zv = zr[k];
             const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
@@ -686,28 +709,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // stage row t of half e in the stage's C tile (free once the output
-        // products are done) and store the half's 128 x 32 box with one TMA
-        // store
-        unsigned char *yt = s + oC + e * kTile;
+        // stage row t of the half's 32 columns in the stage's C tile (free
+        // once the output products are done) and store the half's 128 x 32
+        // box with one TMA store
+        unsigned char *yt = s + oC + half * kTile;
         if (p.y_bf16) {
           // 64-byte rows, 64-byte swizzle: chunk k at k ^ ((t / 2) % 4)
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4 *>(yt + r * 64 + ((k ^ ((r >> 1) & 3)) << 4)) =
+          for (int k = 0; k < 2; ++k) {
+            const int j = 2 * sub + k;
+            *reinterpret_cast<uint4 *>(yt + r * 64 + ((j ^ ((r >> 1) & 3)) << 4)) =
                 make_uint4(pack_bf16(out[8 * k], out[8 * k + 1]),
                            pack_bf16(out[8 * k + 2], out[8 * k + 3]),
                            pack_bf16(out[8 * k + 4], out[8 * k + 5]),
                            pack_bf16(out[8 * k + 6], out[8 * k + 7]));
+          }
         } else {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<float4 *>(yt + swz(r, k)) =
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<float4 *>(yt + swz(r, 4 * sub + k)) =
                 make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
         }
         fence_async_smem();
-        bar_sync(kHalfBarrier + e, kEpi / 2);
-        if (writer) tma_store_4d(&maps.y, yt, 32 * e, h, c * Q, b);
+        bar_sync(kHalfBarrier + half, kEpi / 2);
+        if (writer) tma_store_4d(&maps.y, yt, 32 * half, h, c * Q, b);
       }
       tc_fence_before();
       // the writer releases the stage in the next chunk, after the state
@@ -716,18 +741,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (writer) tma_store_wait_all();
-    // the state after the last chunk (columns of half e)
+    // the state after the last chunk (columns 16e .. 16e + 15)
     if (nchunks > 0) {
       sy.wait(kDoneH, (nchunks - 1) & 1);
       tc_fence_after();
     }
     if (p.last) {
       float *lr = p.last + (static_cast<int64_t>(b) * H + h) * P * NS;
-      uint32_t v[32];
-      tmem_ld32(tl + kColH + 32 * e, v);
+      uint32_t v[16];
+      tmem_ld16(tl + kColH + 16 * e, v);
       tmem_wait_ld(v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) lr[(e * 32 + j) * NS + r] = __uint_as_float(v[j]);
+      for (int j = 0; j < 16; ++j) lr[(e * 16 + j) * NS + r] = __uint_as_float(v[j]);
     }
   }
 

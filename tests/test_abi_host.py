@@ -136,7 +136,8 @@ def test_workspace_size_follows_plan(lib):
     rc, n8 = _ws(lib, _args(plan_splits=8))
     assert rc == sss.MSS_OK and n8 > n4
     # 2 batch rows x 2 channel tiles x 8 chunks, each with (P, e) and the
-    # inclusive state for 32 channels x 16 states
+    # true end state for 32 channels x 16 states (plus the running sums of
+    # Delta at the chunk's segment starts)
     items = 2 * 2 * 8
     assert n8 >= items * 32 * 16 * 3 * 4
 

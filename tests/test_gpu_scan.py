@@ -63,7 +63,7 @@ def test_odd_shapes_match_oracle(case):
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 @pytest.mark.parametrize("N,L", [(16, 5000), (5, 4999), (2, 3001)])
 def test_sequence_split_matches_oracle(splits, dt, N, L):
-    """Chunks combined by look-back give the sequential result ("The relay":
+    """Chunks combined through their carries give the sequential result ("The relay":
     group the steps any way you like).  Odd lengths take the plain-load
     path, N < 16 the kernels with fewer state groups."""
     w = workloads.custom(2, 40, N, L, in_dtype=dt, has_z=True)
@@ -191,8 +191,9 @@ def test_unsplit_scan_is_deterministic():
 
 
 def test_dropped_publish_times_out_and_device_stays_usable():
-    """A chunk that never publishes its carry: the successor's bounded wait
-    runs out, the status word says so, and the next call works."""
+    """A publication that never comes (test flag): the bounded wait before
+    the chunks' carries are composed runs out, the status word says so, and
+    the next call works."""
     w = workloads.custom(1, 32, 16, 4096, in_dtype="f32", has_z=False)
     inp = gpu_inputs(w, seed=2)
     with pytest.raises(sss.MssError) as ei:

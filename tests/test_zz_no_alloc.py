@@ -87,9 +87,10 @@ def _noalloc_status(args):
 
 
 def test_noalloc_reports_a_timed_out_wait_and_recovers():
-    """A chunk that never publishes its carry (test flag): the successor's
-    bounded wait runs out, mss_scan_noalloc_status reports it from the word
-    in the library's array, and the next call is correct and reports OK."""
+    """A publication that never comes (test flag): the bounded wait before
+    the chunks' carries are composed runs out, mss_scan_noalloc_status
+    reports it from the word in the library's array, and the next call is
+    correct and reports OK."""
     w = workloads.custom(1, 32, 16, 4096, in_dtype="f32", has_z=False)
     inp = gpu_inputs(w, seed=2)
     want = sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"],
