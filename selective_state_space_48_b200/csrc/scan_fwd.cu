@@ -688,21 +688,22 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
 }
 
 // ------------------------------------------------------ split: prefix
-// One warp per (tile, state, channel) composes the chunks' pairs in chunk
-// order into incl_k = P_k incl_{k-1} + e_k, the true state at the end of
-// chunk k (incl_0 = e_0: the first chunk started from h0), and writes the
-// final state.  Lane l takes a run of consecutive chunks: it composes its
-// run, the warp scans the runs' pairs (composition is associative: "The
-// relay"), and the lane replays its run from the state before it.  Under
-// MSS_TESTFLAG_DROP_PUBLISH the first warp first waits for a word of the
-// workspace that nothing sets, bounded by the caller's spin timeout, and
-// records the timeout in the status word.
-__global__ void __launch_bounds__(128) scan_prefix_kernel(const ScanParams p, int np) {
-  const int lane = threadIdx.x & 31;
-  const int64_t chain = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t per_tile = static_cast<int64_t>(np) * CH;
-  if (chain >= p.tiles * per_tile) return;  // warp-uniform
-  if ((p.test_flags & 1u) && chain == 0 && lane == 0) {
+// One block of 32 x 32 threads per (tile, state) composes the chunks'
+// pairs in chunk order into incl_k = P_k incl_{k-1} + e_k, the true state at
+// the end of chunk k (incl_0 = e_0: the first chunk started from h0), and
+// writes the final state.  Thread (c, j) holds channel c (rows of the pairs
+// are read coalesced) and the j-th run of consecutive chunks: it composes
+// its run, the runs' pairs are scanned per channel through shared memory
+// (composition is associative: "The relay"), and the thread replays its
+// run from the state before it.  Under MSS_TESTFLAG_DROP_PUBLISH the first
+// thread first waits for a word of the workspace that nothing sets, bounded
+// by the caller's spin timeout, and records the timeout in the status word.
+__global__ void __launch_bounds__(1024) scan_prefix_kernel(const ScanParams p, int np) {
+  __shared__ float sP[32][33], sE[32][33];
+  const int c = threadIdx.x, j = threadIdx.y;
+  const int64_t tile = blockIdx.x / np;
+  const int n = static_cast<int>(blockIdx.x % np);
+  if ((p.test_flags & 1u) && blockIdx.x == 0 && c == 0 && j == 0) {
     const uint64_t limit = p.spin_timeout_ns > 0 ? static_cast<uint64_t>(p.spin_timeout_ns)
                                                  : 1000000000ull;
     const uint64_t start = global_timer_ns();
@@ -714,46 +715,68 @@ __global__ void __launch_bounds__(128) scan_prefix_kernel(const ScanParams p, in
       __nanosleep(1000);
     }
   }
-  __syncwarp();
-  const int64_t tile = chain / per_tile;
-  const int r = static_cast<int>(chain % per_tile);  // state * CH + channel
+  const int64_t per_tile = static_cast<int64_t>(np) * CH;
+  const int r = n * CH + c;
   const int64_t stride = 2 * per_tile;
   const int run = (p.splits + 31) / 32;
-  const int k0 = min(p.splits, lane * run), k1 = min(p.splits, k0 + run);
+  const int k0 = min(p.splits, j * run), k1 = min(p.splits, k0 + run);
   auto pair = [&](int k, float &P, float &e) {
     const int64_t item = static_cast<int64_t>(k) * p.tiles + tile;
     P = k == 0 ? 0.f : p.agg[item * stride + r];  // nothing precedes chunk 0
     e = p.agg[item * stride + per_tile + r];
   };
-  // this lane's run as one pair: h -> P h + E
+  // this thread's run as one pair: h -> P h + E (pairs read eight at a time
+  // so their loads overlap)
   float P = 1.f, E = 0.f;
-  for (int k = k0; k < k1; ++k) {
-    float pk, ek;
-    pair(k, pk, ek);
-    E = fmaf(pk, E, ek);
-    P *= pk;
-  }
-  // inclusive scan of the runs: the earlier pair applied first
+  for (int k = k0; k < k1; k += 8) {
+    float pk[8], ek[8];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const float Po = __shfl_up_sync(0xffffffffu, P, o);
-    const float Eo = __shfl_up_sync(0xffffffffu, E, o);
-    if (lane >= o) {
-      E = fmaf(P, Eo, E);
-      P *= Po;
+    for (int q = 0; q < 8; ++q) {
+      pk[q] = 1.f;
+      ek[q] = 0.f;
+      if (k + q < k1) pair(k + q, pk[q], ek[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      E = fmaf(pk[q], E, ek[q]);
+      P *= pk[q];
     }
   }
-  // state before this lane's run, then the run replayed
-  float h = __shfl_up_sync(0xffffffffu, E, 1);
-  if (lane == 0) h = 0.f;
-  for (int k = k0; k < k1; ++k) {
-    float pk, ek;
-    pair(k, pk, ek);
-    h = fmaf(pk, h, ek);
-    p.incl[(static_cast<int64_t>(k) * p.tiles + tile) * per_tile + r] = h;
+  sP[j][c] = P;
+  sE[j][c] = E;
+  __syncthreads();
+  // warp j scans channel j's runs (lane = run), the earlier pair first,
+  // and leaves the state before each run
+  {
+    float q = sP[c][j], x = sE[c][j];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float qo = __shfl_up_sync(0xffffffffu, q, o);
+      const float xo = __shfl_up_sync(0xffffffffu, x, o);
+      if (c >= o) {
+        x = fmaf(q, xo, x);
+        q *= qo;
+      }
+    }
+    const float before = __shfl_up_sync(0xffffffffu, x, 1);
+    __syncthreads();
+    sE[c][j] = c == 0 ? 0.f : before;
+  }
+  __syncthreads();
+  float h = sE[j][c];
+  for (int k = k0; k < k1; k += 8) {
+    float pk[8], ek[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (k + q < k1) pair(k + q, pk[q], ek[q]);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (k + q >= k1) break;
+      h = fmaf(pk[q], h, ek[q]);
+      p.incl[(static_cast<int64_t>(k + q) * p.tiles + tile) * per_tile + r] = h;
+    }
   }
   if (p.last_state && k1 == p.splits && k0 < k1) {
-    const int n = r / CH, c = r % CH;
     const int64_t b = tile / p.ch_tiles, d = (tile % p.ch_tiles) * CH + c;
     if (d < p.dim && n < p.dstate) p.last_state[(b * p.dim + d) * p.dstate + n] = h;
   }
@@ -1105,8 +1128,7 @@ cudaError_t launch_typed(const ScanParams &p, const TmaMaps &maps, cudaStream_t 
   e = cudaGetLastError();
   if (e != cudaSuccess || p.splits <= 1) return e;
   // split scans: the chunks' true start states, then the carried terms
-  const int64_t threads = p.tiles * 4 * G * CH * 32;  // one warp per chain
-  scan_prefix_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, s>>>(p, 4 * G);
+  scan_prefix_kernel<<<static_cast<unsigned>(p.tiles * 4 * G), dim3(32, 32), 0, s>>>(p, 4 * G);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t units = p.tiles * (p.splits - 1) * p.nseg;
