@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 8
+#define MSS_ABI_VERSION 9
 
 typedef enum {
   MSS_OK = 0,
@@ -275,8 +275,9 @@ mss_status selective_state_update(const mss_update_args *args, void *stream);
 
 /* Arguments of one backward scan: the gradients of
  *   loss = sum(dy * y) + sum(d_last * last_state)
- * for the forward scan with the same inputs (dense tensors, shapes as in
- * mss_scan_args; no strides, no packed sequences).  The states are not
+ * for the forward scan with the same inputs (shapes as in mss_scan_args;
+ * the (batch, rows, seqlen) inputs and dy may be strided, no packed
+ * sequences).  The states are not
  * taken from the forward pass but recomputed: a forward sweep stores the
  * state of every channel at the start of every 16-step block in the
  * workspace and a reverse sweep recomputes each block from it ("Mamba is
@@ -325,6 +326,15 @@ typedef struct mss_scan_bwd_args {
                                256-byte aligned; may be NULL with
                                checkpoints */
   size_t workspace_bytes;
+  /* element strides {batch, row} of u, delta, z, B, C and dy, with the
+     same meaning and rules as the input strides of mss_scan_args ({0, 0}:
+     packed); the gradients are always packed */
+  int64_t stride_u[2];
+  int64_t stride_delta[2];
+  int64_t stride_z[2];
+  int64_t stride_B[2];
+  int64_t stride_C[2];
+  int64_t stride_dy[2];
 } mss_scan_bwd_args;
 
 /* Workspace bytes of the backward scan (the state checkpoints: 64 bytes per

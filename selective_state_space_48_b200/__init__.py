@@ -25,7 +25,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 8  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 9  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -132,7 +132,8 @@ class ScanBwdArgs(ctypes.Structure):
         "h0", "dy", "d_last", "du", "ddelta", "dA", "dB", "dC", "dD", "dz",
         "ddelta_bias", "dh0", "checkpoints", "workspace")] + [
         ("workspace_bytes", ctypes.c_size_t),
-    ]
+    ] + [("stride_" + name, ctypes.c_int64 * 2) for name in (
+        "u", "delta", "z", "B", "C", "dy")]
 
 
 class SsdArgs(ctypes.Structure):
@@ -494,7 +495,8 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     """Gradients of sum(dy * y) + sum(d_last * last_state) for the forward
     scan on the same inputs, through ``mamba_selective_scan_bwd``.
 
-    Dense inputs as for ``selective_scan_fwd``; dy (batch, dim, L) and
+    Inputs as for ``selective_scan_fwd`` (u, delta, z, B, C and dy may be
+    3-d views with a contiguous last dimension); dy (batch, dim, L) and
     d_last (batch, dim, N) float32.  ``checkpoints`` written by the forward
     scan of the same inputs let the backward skip its forward sweep.  Returns a dict of float32 tensors du,
     ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0 (None for absent inputs).
@@ -502,6 +504,7 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     batch, dim, L = u.shape
     N = A.shape[1]
     ind = u.dtype
+    rows = ("u", "delta", "B", "C", "z", "dy")  # may be strided views
     for name, t, dt, shape in (
             ("u", u, ind, None), ("delta", delta, ind, (batch, dim, L)),
             ("A", A, torch.float32, (dim, N)), ("B", B, ind, (batch, N, L)),
@@ -511,7 +514,7 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
             ("h0", h0, torch.float32, (batch, dim, N)),
             ("dy", dy, torch.float32, (batch, dim, L)),
             ("d_last", d_last, torch.float32, (batch, dim, N))):
-        _check_cuda(name, t, dt, shape)
+        _check_cuda(name, t, dt, shape, strided=name in rows)
     dev = u.device
     f32 = dict(dtype=torch.float32, device=dev)
     g = {
@@ -535,6 +538,10 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     a.checkpoints = _ptr(checkpoints)
     for k, v in g.items():
         setattr(a, k, _ptr(v))
+    for name, t in (("u", u), ("delta", delta), ("z", z), ("B", B), ("C", C), ("dy", dy)):
+        if t is not None:
+            getattr(a, "stride_" + name)[0] = t.stride(0)
+            getattr(a, "stride_" + name)[1] = t.stride(1)
     lib = load_library()
     n = ctypes.c_size_t(0)
     rc = lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n))
@@ -582,7 +589,7 @@ class _SelectiveScanFn(torch.autograd.Function):
     @staticmethod
     def backward(ctx, dy):
         u, delta, A, B, C, D, z, delta_bias, h0, ck = ctx.saved_tensors
-        g = selective_scan_bwd(u, delta, A, B, C, dy.float().contiguous(), D=D, z=z,
+        g = selective_scan_bwd(u, delta, A, B, C, _rows_view(dy.float()), D=D, z=z,
                                delta_bias=delta_bias, delta_softplus=ctx.delta_softplus,
                                h0=h0, checkpoints=ck)
         cast = lambda t, like: None if t is None else t.to(like.dtype)
@@ -591,12 +598,19 @@ class _SelectiveScanFn(torch.autograd.Function):
                 g["ddelta_bias"], None, g["dh0"] if h0 is not None else None)
 
 
+def _rows_view(t):
+    """t itself when its last (time) dimension is contiguous, else a copy."""
+    return t if t.dim() == 3 and (t.shape[2] <= 1 or t.stride(2) == 1) else t.contiguous()
+
+
 def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                       delta_softplus=True, h0=None):
     """Differentiable selective scan: y (batch, dim, L) float32, with
-    gradients for every tensor input through the CUDA backward pass.  Dense
-    inputs as for ``selective_scan_fwd``; gradients come back in the
-    inputs' dtypes (computed in float32)."""
-    return _SelectiveScanFn.apply(u.contiguous(), delta.contiguous(), A, B.contiguous(),
-                                  C.contiguous(), D, None if z is None else z.contiguous(),
+    gradients for every tensor input through the CUDA backward pass.
+    Inputs as for ``selective_scan_fwd``: u, delta, B, C and z may be views
+    with a contiguous time dimension (the halves of an input projection,
+    say), which both passes read in place; gradients come back packed, in
+    the inputs' dtypes (computed in float32)."""
+    return _SelectiveScanFn.apply(_rows_view(u), _rows_view(delta), A, _rows_view(B),
+                                  _rows_view(C), D, None if z is None else _rows_view(z),
                                   delta_bias, delta_softplus, h0)

@@ -340,6 +340,18 @@ mss_status selective_state_update(const mss_update_args *a, void *stream) {
 
 namespace {
 
+// The six input stride pairs of a backward scan, resolved; false on the
+// first bad one.
+bool resolve_bwd_strides(const mss_scan_bwd_args *a, BwdParams *p) {
+  const int64_t Bt = a->batch, D = a->dim, N = a->dstate, L = a->seqlen;
+  return resolve_strides(a->stride_u, Bt, D, L, false, p->su) &&
+         resolve_strides(a->stride_delta, Bt, D, L, false, p->sdl) &&
+         resolve_strides(a->stride_z, Bt, D, L, false, p->sz) &&
+         resolve_strides(a->stride_B, Bt, N, L, false, p->sB) &&
+         resolve_strides(a->stride_C, Bt, N, L, false, p->sC) &&
+         resolve_strides(a->stride_dy, Bt, D, L, false, p->sdy);
+}
+
 mss_status check_bwd_args(const mss_scan_bwd_args *a) {
   if (!a) return MSS_ERR_INVALID_ARG;
   if (a->batch < 1 || a->dim < 1 || a->seqlen < 1 || a->dstate < 1)
@@ -352,6 +364,10 @@ mss_status check_bwd_args(const mss_scan_bwd_args *a) {
   if (!a->u || !a->delta || !a->A || !a->B || !a->C || !a->dy || !a->du ||
       !a->ddelta || !a->dA || !a->dB || !a->dC)
     return MSS_ERR_INVALID_ARG;
+  {
+    BwdParams probe{};
+    if (!resolve_bwd_strides(a, &probe)) return MSS_ERR_INVALID_ARG;
+  }
   // a gradient is requested exactly for the optional inputs that are given
   if ((a->D == nullptr) != (a->dD == nullptr) || (a->z == nullptr) != (a->dz == nullptr) ||
       (a->delta_bias == nullptr) != (a->ddelta_bias == nullptr))
@@ -420,6 +436,16 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   p.ckpt_given = a->checkpoints ? 1 : 0;
   p.ch_tiles = static_cast<int>((a->dim + kBwdChannels - 1) / kBwdChannels);
   p.tiles = a->batch * p.ch_tiles;
+  resolve_bwd_strides(a, &p);  // checked above
+  auto ext = [&](const int64_t (&st)[2], int64_t rows) {
+    return (a->batch - 1) * st[0] + (rows - 1) * st[1] + a->seqlen;
+  };
+  p.ext_u = ext(p.su, a->dim);
+  p.ext_delta = ext(p.sdl, a->dim);
+  p.ext_z = ext(p.sz, a->dim);
+  p.ext_B = ext(p.sB, a->dstate);
+  p.ext_C = ext(p.sC, a->dstate);
+  p.ext_dy = ext(p.sdy, a->dim);
   p.status = scan_status_word();
   if (!p.status) return MSS_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

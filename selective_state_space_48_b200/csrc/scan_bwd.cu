@@ -225,23 +225,30 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int e = 0; e < E; ++e) {
       const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
       const int64_t dd = d0 + c;
-      const int64_t off = (b * p.dim + dd) * L + t0 + t;
-      const bool ok = dd < p.dim && t < nt && dbg_index_ok(off, nBDL, p.status);
-      r.u[e] = ok ? ld_f32(gu, off) : 0.f;
-      r.x[e] = ok ? ld_f32(gd, off) : 0.f;
-      r.z[e] = (ok && gz) ? ld_f32(gz, off) : 0.f;
-      r.dy[e] = ok ? p.dy[off] : 0.f;
+      const int64_t ou = b * p.su[0] + dd * p.su[1] + t0 + t,
+                    ox = b * p.sdl[0] + dd * p.sdl[1] + t0 + t,
+                    oz = b * p.sz[0] + dd * p.sz[1] + t0 + t,
+                    oy = b * p.sdy[0] + dd * p.sdy[1] + t0 + t;
+      const bool ok = dd < p.dim && t < nt && dbg_index_ok(ou, p.ext_u, p.status) &&
+                      dbg_index_ok(ox, p.ext_delta, p.status) &&
+                      (!gz || dbg_index_ok(oz, p.ext_z, p.status)) &&
+                      dbg_index_ok(oy, p.ext_dy, p.status);
+      r.u[e] = ok ? ld_f32(gu, ou) : 0.f;
+      r.x[e] = ok ? ld_f32(gd, ox) : 0.f;
+      r.z[e] = (ok && gz) ? ld_f32(gz, oz) : 0.f;
+      r.dy[e] = ok ? p.dy[oy] : 0.f;
       if (ok) r.ok |= 1u << e;
     }
 #pragma unroll
     for (int e = 0; e < EB; ++e) {
       const int idx = tid + NT * e;
       const int n = idx / TB, t = idx % TB;
-      const int64_t off = (b * p.dstate + n) * L + t0 + t;
+      const int64_t ob = b * p.sB[0] + n * p.sB[1] + t0 + t,
+                    oc = b * p.sC[0] + n * p.sC[1] + t0 + t;
       const bool ok = idx < NP * TB && n < p.dstate && t < nt &&
-                      dbg_index_ok(off, nBNL, p.status);
-      r.B[e] = ok ? ld_f32(gB, off) : 0.f;
-      r.C[e] = ok ? ld_f32(gC, off) : 0.f;
+                      dbg_index_ok(ob, p.ext_B, p.status) && dbg_index_ok(oc, p.ext_C, p.status);
+      r.B[e] = ok ? ld_f32(gB, ob) : 0.f;
+      r.C[e] = ok ? ld_f32(gC, oc) : 0.f;
     }
   };
   // the tiles of element (c, t) of a block from its raw values (zeros when
@@ -281,9 +288,14 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   // is computed), 16-byte pieces of the blocks' rows where rows are whole
   // and aligned, element loads elsewhere.
   constexpr bool kStaged = sizeof(InT) == 2;
-  const bool rows16 = (L % 8) == 0 && aligned16(p.u) && aligned16(p.delta) &&
-                      (!gz || aligned16(p.z)) && aligned16(p.dy) && aligned16(p.B) &&
-                      aligned16(p.C);
+  auto st16 = [](const int64_t(&sd)[2], int es) {
+    return (sd[0] * es) % 16 == 0 && (sd[1] * es) % 16 == 0;
+  };
+  constexpr int ES = static_cast<int>(sizeof(InT));
+  const bool rows16 = aligned16(p.u) && aligned16(p.delta) && (!gz || aligned16(p.z)) &&
+                      aligned16(p.dy) && aligned16(p.B) && aligned16(p.C) &&
+                      st16(p.su, ES) && st16(p.sdl, ES) && (!gz || st16(p.sz, ES)) &&
+                      st16(p.sdy, 4) && st16(p.sB, ES) && st16(p.sC, ES);
   auto stage_fetch = [&](int k) {
     BwdStage<G> &st = s.st;
     const int64_t t0 = static_cast<int64_t>(k) * TB;
@@ -299,8 +311,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       if (j < 3 * NR) {
         const int kind = j / NR, rr = j % NR, c = rr / 2, h = rr % 2;
         const InT *base = kind == 0 ? gu : (kind == 1 ? gd : gz);
-        off = (b * p.dim + d0 + c) * L + t0 + 8 * h;
-        ext = nBDL;
+        const int64_t(&sd)[2] = kind == 0 ? p.su : (kind == 1 ? p.sdl : p.sz);
+        off = b * sd[0] + (d0 + c) * sd[1] + t0 + 8 * h;
+        ext = kind == 0 ? p.ext_u : (kind == 1 ? p.ext_delta : p.ext_z);
         row_ok = d0 + c < p.dim && (kind < 2 || gz);
         w = 8 * h;
         src = base;
@@ -309,8 +322,8 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       } else if (j < 3 * NR + CH * 4) {
         r = j - 3 * NR;
         const int c = r / 4, h = r % 4;
-        off = (b * p.dim + d0 + c) * L + t0 + 4 * h;
-        ext = nBDL;
+        off = b * p.sdy[0] + (d0 + c) * p.sdy[1] + t0 + 4 * h;
+        ext = p.ext_dy;
         row_ok = d0 + c < p.dim;
         w = 4 * h;
         src = p.dy;
@@ -319,8 +332,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       } else {
         r = j - 3 * NR - CH * 4;
         const int kind = r / (2 * NP), rr = r % (2 * NP), n = rr / 2, h = rr % 2;
-        off = (b * p.dstate + n) * L + t0 + 8 * h;
-        ext = nBNL;
+        const int64_t(&sd)[2] = kind == 0 ? p.sB : p.sC;
+        off = b * sd[0] + n * sd[1] + t0 + 8 * h;
+        ext = kind == 0 ? p.ext_B : p.ext_C;
         row_ok = n < p.dstate;
         w = 8 * h;
         src = kind == 0 ? gB : gC;
@@ -388,20 +402,22 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int e = 0; e < E; ++e) {
       const int idx = tid + NT * e, c = idx / TB, t = idx % TB;
       const int64_t dd = d0 + c;
-      const int64_t off = (b * p.dim + dd) * L + t0 + t;
-      const bool ok = dd < p.dim && t < nt && dbg_index_ok(off, nBDL, p.status);
-      r.u[e] = ok ? ld_f32(gu, off) : 0.f;
-      r.x[e] = ok ? ld_f32(gd, off) : 0.f;
+      const int64_t ou = b * p.su[0] + dd * p.su[1] + t0 + t,
+                    ox = b * p.sdl[0] + dd * p.sdl[1] + t0 + t;
+      const bool ok = dd < p.dim && t < nt && dbg_index_ok(ou, p.ext_u, p.status) &&
+                      dbg_index_ok(ox, p.ext_delta, p.status);
+      r.u[e] = ok ? ld_f32(gu, ou) : 0.f;
+      r.x[e] = ok ? ld_f32(gd, ox) : 0.f;
       if (ok) r.ok |= 1u << e;
     }
 #pragma unroll
     for (int e = 0; e < EB; ++e) {
       const int idx = tid + NT * e;
       const int n = idx / TB, t = idx % TB;
-      const int64_t off = (b * p.dstate + n) * L + t0 + t;
+      const int64_t ob = b * p.sB[0] + n * p.sB[1] + t0 + t;
       const bool ok = idx < NP * TB && n < p.dstate && t < nt &&
-                      dbg_index_ok(off, nBNL, p.status);
-      r.B[e] = ok ? ld_f32(gB, off) : 0.f;
+                      dbg_index_ok(ob, p.ext_B, p.status);
+      r.B[e] = ok ? ld_f32(gB, ob) : 0.f;
     }
   };
   auto commit_fwd = [&](const RawF &r, BwdTiles<G> &T) {
@@ -444,16 +460,17 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         if (d0 + c >= p.dim) continue;
         src = kind == 0 ? gu : gd;
         dst = (kind == 0 ? su : sx) + c * TB + 8 * h;
-        off = (b * p.dim + d0 + c) * L + t0 + 8 * h;
-        ext = nBDL;
+        const int64_t(&sd)[2] = kind == 0 ? p.su : p.sdl;
+        off = b * sd[0] + (d0 + c) * sd[1] + t0 + 8 * h;
+        ext = kind == 0 ? p.ext_u : p.ext_delta;
         w = 8 * h;
       } else {
         const int r = j - 2 * NR, n = r / 2, h = r % 2;
         if (n >= p.dstate) continue;
         src = gB;
         dst = sB + n * TB + 8 * h;
-        off = (b * p.dstate + n) * L + t0 + 8 * h;
-        ext = nBNL;
+        off = b * p.sB[0] + n * p.sB[1] + t0 + 8 * h;
+        ext = p.ext_B;
         w = 8 * h;
       }
       if (rows16 && nt == TB && dbg_index_ok(off + 7, ext, p.status)) {

@@ -29,6 +29,11 @@ struct BwdParams {
   int ch_tiles;     // ceil(dim / kBwdChannels)
   int64_t tiles;    // batch * ch_tiles
   unsigned *status; // library status word (bounds checks of the checked build)
+  // element strides {batch, row} of the (batch, rows, seqlen) inputs (time
+  // contiguous; always resolved) and their extents (largest index + 1) for
+  // the checked build; the gradients are packed
+  int64_t su[2], sdl[2], sz[2], sB[2], sC[2], sdy[2];
+  int64_t ext_u, ext_delta, ext_z, ext_B, ext_C, ext_dy;
 };
 
 // Warps per block (state groups of 4): 1, 2 or 4.

@@ -6,8 +6,11 @@
 // Transformer", section "What a state space model actually is").  One step
 // of h = exp(Delta A) h + Delta B x with readout y = C h + D x, gated by
 // silu(z).  The step is bound by reading and writing
-// the fp32 state (8 * dstate bytes per channel), so one thread owns one
-// channel (b, d) and moves its state with 16-byte vector loads and stores.
+// the fp32 state (8 * dstate bytes per channel).  With 16 states, four
+// threads share a channel, each moving 4 states as one 16-byte vector, so a
+// warp's loads and stores of its 8 channels are contiguous (512 bytes); the
+// readout is summed over the four by shuffles.  Other state sizes take one
+// thread per channel.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -22,7 +25,7 @@ __device__ __forceinline__ float ld(const void *base, int64_t i) {
   return to_f32<InT>(reinterpret_cast<const InT *>(base)[i]);
 }
 
-template <typename InT, typename OutT, int N>
+template <typename InT, typename OutT>
 __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p) {
   const int64_t ch = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (ch >= p.batch * p.dim) return;
@@ -41,53 +44,77 @@ __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p)
   const float sx = step * x;
   float *st = p.state + ch * p.dstate;
   float acc = 0.f;
-  if (N == 16 && nst == 16 && (reinterpret_cast<uintptr_t>(st) & 15) == 0 &&
-      (reinterpret_cast<uintptr_t>(p.A) & 15) == 0 &&
-      (reinterpret_cast<uintptr_t>(p.B) & 15) == 0 &&
-      (reinterpret_cast<uintptr_t>(p.C) & 15) == 0) {
-    // 16 states: the state, A's row and the batch row's B and C move as
-    // 16-byte vectors (B, C rows are shared by the channels of a batch row)
-    const float *Ad = p.A + d * 16;
-    const InT *Bb = static_cast<const InT *>(p.B) + b * 16;
-    const InT *Cb = static_cast<const InT *>(p.C) + b * 16;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 hv = reinterpret_cast<const float4 *>(st)[q];
-      const float4 av = reinterpret_cast<const float4 *>(Ad)[q];
-      const float4 bv = load4_f32(Bb + 4 * q);
-      const float4 cv = load4_f32(Cb + 4 * q);
-      const float hs[4] = {hv.x, hv.y, hv.z, hv.w}, as[4] = {av.x, av.y, av.z, av.w},
-                  bs[4] = {bv.x, bv.y, bv.z, bv.w}, cs[4] = {cv.x, cv.y, cv.z, cv.w};
-      float ho[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float a = ex2_mufu(step * as[j] * kLog2e);
-        ho[j] = fmaf(a, hs[j], sx * bs[j]);
-        acc = fmaf(cs[j], ho[j], acc);
-      }
-      reinterpret_cast<float4 *>(st)[q] = make_float4(ho[0], ho[1], ho[2], ho[3]);
-    }
-  } else {
-    for (int n = 0; n < nst; ++n) {
-      const float a = ex2_mufu(step * p.A[d * p.dstate + n] * kLog2e);
-      const float hn = fmaf(a, st[n], sx * ld<InT>(p.B, b * p.dstate + n));
-      st[n] = hn;
-      acc = fmaf(ld<InT>(p.C, b * p.dstate + n), hn, acc);
-    }
+  for (int n = 0; n < nst; ++n) {
+    const float a = ex2_mufu(step * p.A[d * p.dstate + n] * kLog2e);
+    const float hn = fmaf(a, st[n], sx * ld<InT>(p.B, b * p.dstate + n));
+    st[n] = hn;
+    acc = fmaf(ld<InT>(p.C, b * p.dstate + n), hn, acc);
   }
   float yv = acc + (p.D ? p.D[d] : 0.f) * x;
   if (p.z) yv *= silu_f(ld<InT>(p.z, ch));
   reinterpret_cast<OutT *>(p.y)[ch] = from_f32<OutT>(yv);
 }
 
+// 16 states with the state, A, B and C 16-byte aligned: thread 4 ch + qd
+// owns states 4 qd .. 4 qd + 3 of channel ch.
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(256) state_update16_kernel(const UpdateParams p) {
+  const int64_t gt = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t ch = gt >> 2;
+  const int qd = static_cast<int>(gt & 3);
+  // every thread of a channel takes part in the shuffles below
+  bool valid = ch < p.batch * p.dim;
+  if (valid && (!dbg_index_ok((ch + 1) * 16 - 1, p.batch * p.dim * 16, p.status) ||
+                !dbg_index_ok((ch % p.dim + 1) * 16 - 1, p.dim * 16, p.status) ||
+                !dbg_index_ok((ch / p.dim + 1) * 16 - 1, p.batch * 16, p.status)))
+    valid = false;
+  const int64_t c = valid ? ch : 0;
+  const int64_t b = c / p.dim, d = c % p.dim;
+  float acc = 0.f, x = 0.f;
+  if (valid) {
+    x = ld<InT>(p.x, c);
+    float s = ld<InT>(p.dt, c);
+    if (p.dt_bias) s += p.dt_bias[d];
+    const float step = p.softplus ? softplus_f(s) : s;
+    const float sx = step * x;
+    float4 *st = reinterpret_cast<float4 *>(p.state + c * 16) + qd;
+    const float4 hv = *st;
+    const float4 av = reinterpret_cast<const float4 *>(p.A + d * 16)[qd];
+    const float4 bv = load4_f32(static_cast<const InT *>(p.B) + b * 16 + 4 * qd);
+    const float4 cv = load4_f32(static_cast<const InT *>(p.C) + b * 16 + 4 * qd);
+    const float hs[4] = {hv.x, hv.y, hv.z, hv.w}, as[4] = {av.x, av.y, av.z, av.w},
+                bs[4] = {bv.x, bv.y, bv.z, bv.w}, cs[4] = {cv.x, cv.y, cv.z, cv.w};
+    float ho[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = ex2_mufu(step * as[j] * kLog2e);
+      ho[j] = fmaf(a, hs[j], sx * bs[j]);
+      acc = fmaf(cs[j], ho[j], acc);
+    }
+    *st = make_float4(ho[0], ho[1], ho[2], ho[3]);
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  if (valid && qd == 0) {
+    float yv = acc + (p.D ? p.D[d] : 0.f) * x;
+    if (p.z) yv *= silu_f(ld<InT>(p.z, c));
+    reinterpret_cast<OutT *>(p.y)[c] = from_f32<OutT>(yv);
+  }
+}
+
+bool aligned16(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
+
 template <typename InT, typename OutT>
 cudaError_t launch_typed(const UpdateParams &p, cudaStream_t s) {
   const int64_t n = p.batch * p.dim;
-  const unsigned grid = static_cast<unsigned>((n + 127) / 128);
-  if (p.dstate == 16)
-    state_update_kernel<InT, OutT, 16><<<grid, 128, 0, s>>>(p);
-  else
-    state_update_kernel<InT, OutT, 0><<<grid, 128, 0, s>>>(p);
+  if (p.dstate == 16 && aligned16(p.state) && aligned16(p.A) && aligned16(p.B) &&
+      aligned16(p.C)) {
+    const unsigned grid = static_cast<unsigned>((4 * n + 255) / 256);
+    state_update16_kernel<InT, OutT><<<grid, 256, 0, s>>>(p);
+  } else {
+    const unsigned grid = static_cast<unsigned>((n + 127) / 128);
+    state_update_kernel<InT, OutT><<<grid, 128, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

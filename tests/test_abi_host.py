@@ -69,7 +69,7 @@ def test_checked_build_exports_the_same_symbols():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 8
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 9
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:

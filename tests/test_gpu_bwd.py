@@ -135,3 +135,36 @@ def test_backward_at_the_130m_layer_shape_every_element():
              "ddelta_bias": _full_tolerance(w.batch * w.seqlen)}
     bad = {k: (e, bound[k]) for k, e in errs.items() if not e <= bound[k]}
     assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("dt,L", [("bf16", 1024), ("bf16", 777), ("f32", 512)])
+def test_backward_reads_strided_views(dt, L):
+    """u and z as the two halves of one (batch, 2 D, L) projection, B and C
+    as rows of one (batch, 2 N + 3, L) tensor and dy as a slice of a wider
+    one, read in place: every gradient matches the oracle, and the same
+    backward of packed copies.  L = 1024 stages whole aligned rows with
+    16-byte copies through the strides; L = 777 and fp32 take element
+    loads for the rows that are not whole 16-byte pieces."""
+    batch, D, N = 2, 72, 16
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    w = workloads.custom(batch, D, N, L, in_dtype=dt, has_z=True, a_noise=0.1)
+    inp = gpu_inputs(w, seed=4242 + L, h0=True)
+    proj = torch.empty(batch, 2 * D, L, dtype=tdt, device="cuda")
+    proj[:, :D], proj[:, D:] = inp["u"], inp["z"]
+    xb = torch.zeros(batch, 2 * N + 3, L, dtype=tdt, device="cuda")
+    xb[:, 1:N + 1], xb[:, N + 2:2 * N + 2] = inp["B"], inp["C"]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4343)
+    wide = torch.randn(batch, D + 5, L, generator=g, device="cuda")
+    dy = wide[:, 3:D + 3]
+    views = dict(inp, u=proj[:, :D], z=proj[:, D:], B=xb[:, 1:N + 1], C=xb[:, N + 2:2 * N + 2])
+    assert not views["u"].is_contiguous() and not dy.is_contiguous()
+    g_view, g_ref = _grads(w, views, dy, None)
+    _compare(g_view, g_ref, f"strided {dt} L={L}")
+    g_pack = sss.selective_scan_bwd(
+        inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy.contiguous(), D=inp["D"],
+        z=inp["z"], delta_bias=inp["delta_bias"], h0=inp["h0"])
+    for k in NAMES:
+        if g_pack.get(k) is None:
+            continue
+        assert norm_err(g_view[k].cpu().numpy(), g_pack[k].cpu().numpy()) <= 1e-6, k

@@ -87,6 +87,21 @@ def test_split_with_slow_decay_matches_oracle():
     assert norm_err(y.cpu(), want) <= tolerance("f32")
 
 
+@pytest.mark.parametrize("dt,out", [("f32", torch.float32), ("bf16", torch.bfloat16)])
+def test_carry_across_many_segments(dt, out):
+    """Slow decay (Delta ~ 1e-3) over chunks of 2 600 steps: the carried
+    state stays alive across several 512-step segments of the carry launch,
+    the last of them ragged; the final state comes from the chunk prefix."""
+    w = workloads.custom(2, 40, 16, 7777, in_dtype=dt, has_z=True, a_noise=0.1)
+    inp = gpu_inputs(w, seed=9, h0=True)
+    inp["delta_bias"] = torch.full_like(inp["delta_bias"], -7.0)
+    y, last = run_gpu(w, inp, out_dtype=out, plan_splits=3, return_last_state=True,
+                      check_status=True)
+    want, want_last = run_oracle(w, inp, return_last_state=True)
+    assert norm_err(y.float().cpu(), want) <= tolerance(dt, out)
+    assert norm_err(last.cpu(), want_last) <= tolerance(dt)
+
+
 @pytest.mark.parametrize("name", ["mamba130m-layer", "mamba1.4b-layer",
                                   "long-context", "audio-length"])
 def test_full_size_workload_every_element(name):

@@ -51,6 +51,9 @@ CASES = [
     ("bf16-split3", 1, 64, 16, 3000, "bf16", [1, 500, 1008, 1500, 2016, 2017, 2990], 3),
     ("bf16-split7", 1, 48, 16, 5000, "bf16", [7, 720, 721, 1440, 3000, 4999], 7),
     ("f32-many-short", 1, 32, 16, 512, "f32", list(range(0, 512, 5)), 0),
+    # two chunks of 4512 steps; restarts on and next to a 512-step segment
+    # boundary of the carry launch
+    ("bf16-split2-segments", 1, 48, 16, 9000, "bf16", [5024, 5025, 7000], 2),
 ]
 
 
