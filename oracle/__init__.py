@@ -68,7 +68,8 @@ def _bind(lib):
         [_I64] * 3 + [_D] * 9 + [ctypes.c_int, _D])
     lib.oracle_selective_state_update_f64.restype = ctypes.c_int
     lib.oracle_selective_scan_bwd_f64.argtypes = (
-        [_I64] * 4 + [_D] * 8 + [ctypes.c_int] + [_D] * 12)
+        [_I64] * 4 + [_D] * 8 + [ctypes.c_int] + [_D] * 12 +
+        [ctypes.POINTER(ctypes.c_int32), _I64])
     lib.oracle_selective_scan_bwd_f64.restype = ctypes.c_int
     lib.oracle_ssd_scan_f64.argtypes = (
         [_I64] * 6 + [_D] * 8 + [ctypes.c_int, _D, _D, _D])
@@ -203,10 +204,12 @@ def set_num_threads(n: int, lib=None) -> None:
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
-                       delta_softplus=True, h0=None, d_last=None, lib=None):
-    """fp64 gradient of ``selective_scan`` for the loss
-    sum(dy * y) + sum(d_last * last_state).  Returns a dict with du, ddelta,
-    dA, dB, dC, dD, dz, ddelta_bias, dh0 (None where the input is absent)."""
+                       delta_softplus=True, h0=None, d_last=None, lib=None,
+                       cu_seqlens=None):
+    """fp64 gradient of ``selective_scan`` (with the same ``cu_seqlens``
+    packing) for the loss sum(dy * y) + sum(d_last * last_state).  Returns a
+    dict with du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0 (None where
+    the input is absent)."""
     lib = lib or load()
     u, delta, A, B, C, dy = (_f64(x) for x in (u, delta, A, B, C, dy))
     D, z, delta_bias, h0, d_last = (_f64(x) for x in (D, z, delta_bias, h0, d_last))
@@ -221,12 +224,17 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
         "ddelta_bias": np.empty(dim) if delta_bias is not None else None,
         "dh0": np.empty((batch, dim, N)),
     }
+    cu, nseq = None, 0
+    if cu_seqlens is not None:
+        cu_arr = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        nseq = len(cu_arr) - 1
+        cu = cu_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
     rc = lib.oracle_selective_scan_bwd_f64(
         batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
         _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)),
         _ptr(h0), _ptr(dy), _ptr(d_last), _ptr(out["du"]), _ptr(out["ddelta"]),
         _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]),
-        _ptr(out["dz"]), _ptr(out["ddelta_bias"]), _ptr(out["dh0"]))
+        _ptr(out["dz"]), _ptr(out["ddelta_bias"]), _ptr(out["dh0"]), cu, nseq)
     if rc != 0:
         raise ValueError("oracle_selective_scan_bwd_f64 rejected the sizes")
     return out

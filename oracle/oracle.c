@@ -225,16 +225,26 @@ int oracle_selective_scan_bwd_f64(
     const double *delta_bias, int delta_softplus, const double *h0,
     const double *dy, const double *d_last, double *du, double *ddelta,
     double *dA, double *dB, double *dC, double *dD, double *dz,
-    double *ddelta_bias, double *dh0) {
+    double *ddelta_bias, double *dh0, const int32_t *cu_seqlens,
+    int64_t num_seqs) {
   if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256 || seqlen < 0)
     return -1;
+  if (cu_seqlens && num_seqs < 1) return -1;
   const int64_t N = dstate, L = seqlen;
+  /* Packed sequences: step t starts a sequence (the state before it is
+   * empty, as in the forward oracle) when t is an interior start
+   * cu_seqlens[i], 0 < i < num_seqs. */
+  char *starts = calloc((size_t)(L + 1), 1);
+  if (!starts) return -1;
+  if (cu_seqlens)
+    for (int64_t i = 1; i < num_seqs; ++i)
+      if (cu_seqlens[i] >= 0 && cu_seqlens[i] < L) starts[cu_seqlens[i]] = 1;
   /* per batch row partial sums of the per-channel parameter gradients */
   double *pA = calloc((size_t)(batch * dim * N + 1), sizeof(double));
   double *pD = calloc((size_t)(batch * dim + 1), sizeof(double));
   double *pb = calloc((size_t)(batch * dim + 1), sizeof(double));
   if (!pA || !pD || !pb) {
-    free(pA); free(pD); free(pb);
+    free(pA); free(pD); free(pb); free(starts);
     return -1;
   }
   memset(dB, 0, sizeof(double) * (size_t)(batch * N * L));
@@ -272,7 +282,9 @@ int oracle_selective_scan_bwd_f64(
         Dt[t] = dt;
         double acc = 0.0;
         for (int64_t n = 0; n < N; ++n) {
-          const double h = exp(dt * A[d * N + n]) * H[t * N + n] +
+          /* the state entering step t: h_{t-1}, or empty at a start */
+          const double hin = starts[t] ? 0.0 : H[t * N + n];
+          const double h = exp(dt * A[d * N + n]) * hin +
                            dt * Bb[n * L + t] * u[row + t];
           H[(t + 1) * N + n] = h;
           acc += Cb[n * L + t] * h;
@@ -293,7 +305,9 @@ int oracle_selective_scan_bwd_f64(
         double dut = ds * dskip, dDelta = 0.0;
         for (int64_t n = 0; n < N; ++n) {
           const double an = A[d * N + n];
-          const double a = exp(dt * an);
+          /* at a start nothing flows back from step t to h_{t-1} (every
+           * use of hprev below is multiplied by a) */
+          const double a = starts[t] ? 0.0 : exp(dt * an);
           const double hprev = H[t * N + n];
           lam[n] += ds * Cb[n * L + t];
           dCb[n * L + t] += ds * H[(t + 1) * N + n];
@@ -332,7 +346,7 @@ int oracle_selective_scan_bwd_f64(
       }
     }
   }
-  free(pA); free(pD); free(pb);
+  free(pA); free(pD); free(pb); free(starts);
   return failed ? -1 : 0;
 }
 

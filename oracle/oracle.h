@@ -73,7 +73,8 @@ int oracle_selective_state_update_f64(int64_t batch, int64_t dim,
                                       const double *z, const double *dt_bias,
                                       int dt_softplus, double *y);
 
-/* Gradient of the selective scan above (no packed sequences) for the loss
+/* Gradient of the selective scan above (Euler update; packed sequences as
+ * there, cu_seqlens NULL for none) for the loss
  * sum(dy * y) + sum(d_last * last_state): du, ddelta, dz (batch, dim,
  * seqlen), dA (dim, dstate), dB, dC (batch, dstate, seqlen), dD,
  * ddelta_bias (dim), dh0 (batch, dim, dstate).  d_last, dz, dD,
@@ -86,7 +87,8 @@ int oracle_selective_scan_bwd_f64(
     const double *delta_bias, int delta_softplus, const double *h0,
     const double *dy, const double *d_last, double *du, double *ddelta,
     double *dA, double *dB, double *dC, double *dD, double *dz,
-    double *ddelta_bias, double *dh0);
+    double *ddelta_bias, double *dh0, const int32_t *cu_seqlens,
+    int64_t num_seqs);
 
 /* Mamba-2 (SSD): the same recurrence with A restricted to a scalar times
  * the identity per head, sequential over t.  headdim channels of a head

@@ -466,16 +466,19 @@ def _fd_check(lib, case, seed):
     dy = rng.normal(size=(bt, dm, L))
     d_last = rng.normal(size=(bt, dm, N))
 
+    cu = case.get("cu")
+
     def F(X):
         y, last = oracle.selective_scan(X["u"], X["delta"], X["A"], X["B"], X["C"],
                                         D=X["D"], z=X["z"], delta_bias=X["delta_bias"],
                                         delta_softplus=sp, h0=X["h0"],
-                                        return_last_state=True, lib=lib)
+                                        return_last_state=True, lib=lib, cu_seqlens=cu)
         return float(np.sum(dy * y) + np.sum(d_last * last))
 
     g = oracle.selective_scan_bwd(X["u"], X["delta"], X["A"], X["B"], X["C"], dy,
                                   D=X["D"], z=X["z"], delta_bias=X["delta_bias"],
-                                  delta_softplus=sp, h0=X["h0"], d_last=d_last, lib=lib)
+                                  delta_softplus=sp, h0=X["h0"], d_last=d_last, lib=lib,
+                                  cu_seqlens=cu)
     names = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC",
              "D": "dD", "z": "dz", "delta_bias": "ddelta_bias", "h0": "dh0"}
     eps = 1e-6
@@ -491,6 +494,9 @@ def _fd_check(lib, case, seed):
 def pin_backward_finite_differences(lib):
     _fd_check(lib, dict(shape=(2, 3, 4, 9), softplus=True), 31)
     _fd_check(lib, dict(shape=(1, 2, 3, 13), softplus=False), 32)
+    # packed sequences (the forward oracle's packing, pinned above): starts
+    # at steps 1, 5 and 6 (a one-step sequence) of 13
+    _fd_check(lib, dict(shape=(2, 2, 3, 13), softplus=True, cu=[0, 1, 5, 6, 13]), 33)
 
 
 # --------------------------------------------------------------------------

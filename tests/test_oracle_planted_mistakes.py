@@ -48,6 +48,10 @@ MUTATIONS = {
                                    "dCb[n * L + t] += ds * H[t * N + n];"),
     "bwd_gate_derivative_wrong": ("return sg * (1.0 + z * (1.0 - sg));", "return sg;"),
     "bwd_softplus_derivative_dropped": ("? dDelta / (1.0 + exp(-x)) : dDelta;", "? dDelta : dDelta;"),
+    "bwd_packed_adjoint_flows_back": ("const double a = starts[t] ? 0.0 : exp(dt * an);",
+                                      "const double a = exp(dt * an);"),
+    "bwd_packed_state_not_reset": ("const double hin = starts[t] ? 0.0 : H[t * N + n];",
+                                   "const double hin = H[t * N + n];"),
     "trap_previous_input_not_decayed": ("0.5 * dt * (abar * wprev[n] + w)", "0.5 * dt * (wprev[n] + w)"),
     "trap_full_step_weights": ("0.5 * dt * (abar * wprev[n] + w)", "dt * (abar * wprev[n] + w)"),
     "trap_previous_input_not_kept": ("          wprev[n] = w;\n", "\n"),
