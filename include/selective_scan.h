@@ -276,8 +276,9 @@ mss_status selective_state_update(const mss_update_args *args, void *stream);
 /* Arguments of one backward scan: the gradients of
  *   loss = sum(dy * y) + sum(d_last * last_state)
  * for the forward scan with the same inputs (shapes as in mss_scan_args;
- * the (batch, rows, seqlen) inputs and dy may be strided, no packed
- * sequences).  The states are not
+ * the (batch, rows, seqlen) inputs and dy may be strided, and packed
+ * sequences restart the state as in the forward scan, so no gradient flows
+ * across a sequence start).  The states are not
  * taken from the forward pass but recomputed: a forward sweep stores the
  * state of every channel at the start of every 16-step block in the
  * workspace and a reverse sweep recomputes each block from it ("Mamba is
@@ -335,6 +336,10 @@ typedef struct mss_scan_bwd_args {
   int64_t stride_B[2];
   int64_t stride_C[2];
   int64_t stride_dy[2];
+  /* packed sequences as in mss_scan_args (NULL / 0: one sequence per row);
+     not combined with checkpoints */
+  const int32_t *cu_seqlens;
+  int64_t num_seqs;
 } mss_scan_bwd_args;
 
 /* Workspace bytes of the backward scan (the state checkpoints: 64 bytes per

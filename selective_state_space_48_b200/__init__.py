@@ -133,7 +133,10 @@ class ScanBwdArgs(ctypes.Structure):
         "ddelta_bias", "dh0", "checkpoints", "workspace")] + [
         ("workspace_bytes", ctypes.c_size_t),
     ] + [("stride_" + name, ctypes.c_int64 * 2) for name in (
-        "u", "delta", "z", "B", "C", "dy")]
+        "u", "delta", "z", "B", "C", "dy")] + [
+        ("cu_seqlens", ctypes.c_void_p),
+        ("num_seqs", ctypes.c_int64),
+    ]
 
 
 class SsdArgs(ctypes.Structure):
@@ -491,9 +494,10 @@ __all__ = [
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
                        delta_softplus=True, h0=None, d_last=None, stream=None,
-                       workspace=None, checkpoints=None):
+                       workspace=None, checkpoints=None, cu_seqlens=None):
     """Gradients of sum(dy * y) + sum(d_last * last_state) for the forward
-    scan on the same inputs, through ``mamba_selective_scan_bwd``.
+    scan on the same inputs (and the same ``cu_seqlens`` packing), through
+    ``mamba_selective_scan_bwd``.
 
     Inputs as for ``selective_scan_fwd`` (u, delta, z, B, C and dy may be
     3-d views with a contiguous last dimension); dy (batch, dim, L) and
@@ -542,6 +546,12 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
         if t is not None:
             getattr(a, "stride_" + name)[0] = t.stride(0)
             getattr(a, "stride_" + name)[1] = t.stride(1)
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int32)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must hold num_seqs + 1 >= 2 offsets")
+        a.cu_seqlens = cu_seqlens.data_ptr()
+        a.num_seqs = cu_seqlens.numel() - 1
     lib = load_library()
     n = ctypes.c_size_t(0)
     rc = lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n))
@@ -577,25 +587,28 @@ class _SelectiveScanFn(torch.autograd.Function):
     mamba_selective_scan_bwd starting from them."""
 
     @staticmethod
-    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0):
+    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, cu_seqlens):
         batch, dim, L = u.shape
-        ck = scan_checkpoints(batch, dim, A.shape[1], L, u.device)
+        # packed sequences: no forward checkpoints, the backward sweeps itself
+        ck = (scan_checkpoints(batch, dim, A.shape[1], L, u.device)
+              if cu_seqlens is None else None)
         y = selective_scan_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=delta_bias,
-                               delta_softplus=delta_softplus, h0=h0, checkpoints=ck)
+                               delta_softplus=delta_softplus, h0=h0, checkpoints=ck,
+                               cu_seqlens=cu_seqlens)
         ctx.delta_softplus = delta_softplus
-        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, h0, ck)
+        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, h0, ck, cu_seqlens)
         return y
 
     @staticmethod
     def backward(ctx, dy):
-        u, delta, A, B, C, D, z, delta_bias, h0, ck = ctx.saved_tensors
+        u, delta, A, B, C, D, z, delta_bias, h0, ck, cu = ctx.saved_tensors
         g = selective_scan_bwd(u, delta, A, B, C, _rows_view(dy.float()), D=D, z=z,
                                delta_bias=delta_bias, delta_softplus=ctx.delta_softplus,
-                               h0=h0, checkpoints=ck)
+                               h0=h0, checkpoints=ck, cu_seqlens=cu)
         cast = lambda t, like: None if t is None else t.to(like.dtype)
         return (cast(g["du"], u), cast(g["ddelta"], delta), g["dA"], cast(g["dB"], B),
                 cast(g["dC"], C), g["dD"], cast(g["dz"], z) if z is not None else None,
-                g["ddelta_bias"], None, g["dh0"] if h0 is not None else None)
+                g["ddelta_bias"], None, g["dh0"] if h0 is not None else None, None)
 
 
 def _rows_view(t):
@@ -604,13 +617,14 @@ def _rows_view(t):
 
 
 def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None,
-                      delta_softplus=True, h0=None):
+                      delta_softplus=True, h0=None, cu_seqlens=None):
     """Differentiable selective scan: y (batch, dim, L) float32, with
     gradients for every tensor input through the CUDA backward pass.
     Inputs as for ``selective_scan_fwd``: u, delta, B, C and z may be views
     with a contiguous time dimension (the halves of an input projection,
-    say), which both passes read in place; gradients come back packed, in
+    say), which both passes read in place; ``cu_seqlens`` packs independent
+    sequences as for ``selective_scan_fwd``.  Gradients come back packed, in
     the inputs' dtypes (computed in float32)."""
     return _SelectiveScanFn.apply(_rows_view(u), _rows_view(delta), A, _rows_view(B),
                                   _rows_view(C), D, None if z is None else _rows_view(z),
-                                  delta_bias, delta_softplus, h0)
+                                  delta_bias, delta_softplus, h0, cu_seqlens)

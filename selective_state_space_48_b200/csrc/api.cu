@@ -368,6 +368,12 @@ mss_status check_bwd_args(const mss_scan_bwd_args *a) {
     BwdParams probe{};
     if (!resolve_bwd_strides(a, &probe)) return MSS_ERR_INVALID_ARG;
   }
+  if (a->cu_seqlens ? (a->num_seqs < 1 || a->num_seqs > INT32_MAX ||
+                       !aligned(a->cu_seqlens, 4))
+                    : a->num_seqs != 0)
+    return MSS_ERR_INVALID_ARG;
+  // the forward scan writes no checkpoints for packed sequences
+  if (a->cu_seqlens && a->checkpoints) return MSS_ERR_UNSUPPORTED;
   // a gradient is requested exactly for the optional inputs that are given
   if ((a->D == nullptr) != (a->dD == nullptr) || (a->z == nullptr) != (a->dz == nullptr) ||
       (a->delta_bias == nullptr) != (a->ddelta_bias == nullptr))
@@ -446,6 +452,8 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   p.ext_B = ext(p.sB, a->dstate);
   p.ext_C = ext(p.sC, a->dstate);
   p.ext_dy = ext(p.sdy, a->dim);
+  p.cu = a->cu_seqlens;
+  p.nseq = a->cu_seqlens ? a->num_seqs : 0;
   p.status = scan_status_word();
   if (!p.status) return MSS_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -19,6 +19,12 @@
 //                  with the kept decays (no exponential is evaluated twice
 //                  within a half); then the earlier half the same way.
 //
+// Packed sequences (their own instantiation) take exp(Delta A) = 0 at every
+// sequence start, in the forward sweep and the recompute alike: the state
+// entering the start is then empty and the adjoint's lam_{t-1} = a_t lam_t
+// gets nothing across it.  The inputs may be strided views (time
+// contiguous); the gradients are packed.
+//
 // The arithmetic pairs the lane's states: two states advance together in
 // one f32x2 instruction, so B_t and C_t sit in shared memory step-major
 // ([t][n]) and a warp reads the four values of its states with one
@@ -53,9 +59,10 @@ constexpr int CH = 32;
 constexpr int TB = 16;
 constexpr int ROW = TB + 4;  // padded fp32 row (conflict-free float4 reads)
 
-// The fp32 tiles of one 16-step block.
+// The fp32 tiles of one 16-step block (16-byte aligned: the tiles are
+// read as float4, also in the second of two consecutive sets).
 template <int G>
-struct BwdTiles {
+struct alignas(16) BwdTiles {
   static constexpr int NP = 4 * G;
   // per (channel, step) tiles [CH][ROW]; gz = dy silu'(z), so that
   // dz = gz s with s the readout (incl. D u)
@@ -63,6 +70,8 @@ struct BwdTiles {
       gz[CH * ROW];
   // per (step, state) tiles [TB][NP]: a warp's four states are adjacent
   float B[TB * NP], C[TB * NP];
+  // packed sequences: bit t set when step t of the block starts a sequence
+  unsigned rmask;
 };
 
 // The raw inputs of one 16-step block as they lie in HBM (bf16 u, delta,
@@ -79,6 +88,7 @@ struct BwdStage {
 template <int G>
 struct BwdSmem {
   static constexpr int NP = 4 * G;
+  static_assert(sizeof(BwdTiles<G>) % 16 == 0, "tile sets keep 16-byte alignment");
   // two sets of tiles: block k is computed from set k & 1 while the other
   // set still serves block k + 1's epilogue
   BwdTiles<G> tl[2];
@@ -150,7 +160,23 @@ __device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
   return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
-template <typename InT, int G>
+// Bit t (t < 16) set when step t0 + t (< L) is an interior sequence start.
+__device__ unsigned restart_mask(const BwdParams &p, int64_t t0, int64_t L) {
+  int64_t lo = 1, hi = p.nseq;  // first interior start >= t0
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (__ldg(p.cu + mid) < t0) lo = mid + 1; else hi = mid;
+  }
+  unsigned m = 0u;
+  for (int64_t i = lo; i < p.nseq; ++i) {
+    const int64_t t = __ldg(p.cu + i) - t0;
+    if (t >= kBwdTimeBlock || t0 + t >= L) break;
+    m |= 1u << t;
+  }
+  return m;
+}
+
+template <typename InT, int G, bool VARLEN>
 __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     scan_bwd_kernel(const BwdParams p) {
   using Sm = BwdSmem<G>;
@@ -265,6 +291,11 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     T.ds[c * ROW + t] = gz ? dyv * zv * sz : dyv;
     T.gz[c * ROW + t] = dyv * sz * fmaf(zv, 1.0f - sz, 1.0f);
     T.sg[c * ROW + t] = p.softplus ? sigmoid_f(x) : 1.f;
+  };
+  // packed sequences: the block's restart mask, written by thread 0 with its
+  // tiles (no decay across a start: exp(Delta A) is taken as 0 there)
+  auto put_mask = [&](int k, BwdTiles<G> &T) {
+    if (VARLEN && tid == 0) T.rmask = restart_mask(p, static_cast<int64_t>(k) * TB, L);
   };
   auto commit = [&](const Raw &r, BwdTiles<G> &T) {
 #pragma unroll
@@ -516,10 +547,10 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       for (int j = 0; j < 4; ++j) {
         const float4 b4 = ld4(&T.B[(4 * qd + j) * NP + 4 * g]);
         const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
-        h2[0] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[0])), h2[0],
-                           __fmul2_rn(U2, make_float2(b4.x, b4.y)));
-        h2[1] = __ffma2_rn(ex2_pair(__fmul2_rn(D2, al2[1])), h2[1],
-                           __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+        float2 e0 = ex2_pair(__fmul2_rn(D2, al2[0])), e1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+        if (VARLEN && ((T.rmask >> (4 * qd + j)) & 1u)) e0 = e1 = make_float2(0.f, 0.f);
+        h2[0] = __ffma2_rn(e0, h2[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+        h2[1] = __ffma2_rn(e1, h2[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
       }
     }
   };
@@ -535,6 +566,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     cp_async_wait_all();
     __syncthreads();
     fstage_commit(0, 0, s.tl[0]);
+    put_mask(0, s.tl[0]);
     if (nblk > 1) fstage_fetch(1, 1);
     for (int k = 0; k < nblk; ++k) {
       put_ckpt(k);
@@ -545,7 +577,10 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       // area k & 1 held block k, committed before the barrier; tile set
       // (k + 1) & 1 was last read by block k - 1, finished before it
       if (k + 2 < nblk) fstage_fetch(k + 2, k & 1);
-      if (k + 1 < nblk) fstage_commit(k + 1, (k + 1) & 1, s.tl[(k + 1) & 1]);
+      if (k + 1 < nblk) {
+        fstage_commit(k + 1, (k + 1) & 1, s.tl[(k + 1) & 1]);
+        put_mask(k + 1, s.tl[(k + 1) & 1]);
+      }
       fwd_block(s.tl[k & 1]);
     }
     __syncthreads();
@@ -555,6 +590,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int k = 0; k < nblk; ++k) {
       BwdTiles<G> &T = s.tl[k & 1];
       commit_fwd(rf, T);
+      put_mask(k, T);
       put_ckpt(k);
       __syncthreads();
       if (k + 1 < nblk) fetch_fwd(k + 1, rf);  // in flight while block k is computed
@@ -592,9 +628,11 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     cp_async_wait_all();
     __syncthreads();
     stage_commit(nblk - 1, s.tl[(nblk - 1) & 1]);
+    put_mask(nblk - 1, s.tl[(nblk - 1) & 1]);
   } else {
     fetch(nblk - 1, raw);
     commit(raw, s.tl[(nblk - 1) & 1]);
+    put_mask(nblk - 1, s.tl[(nblk - 1) & 1]);
   }
   // this thread's shares of the per-channel sums (in registers when a
   // thread has few elements; otherwise added to shared memory per block)
@@ -646,8 +684,10 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
           const int t = 4 * qd + j;
           const float4 b4 = ld4(&T.B[t * NP + 4 * g]);
           const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
-          const float2 a0 = ex2_pair(__fmul2_rn(D2, al2[0]));
-          const float2 a1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+          float2 a0 = ex2_pair(__fmul2_rn(D2, al2[0]));
+          float2 a1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+          // a sequence start: nothing of the previous state survives it
+          if (VARLEN && ((T.rmask >> t) & 1u)) a0 = a1 = make_float2(0.f, 0.f);
           hh[0] = __ffma2_rn(a0, hh[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
           hh[1] = __ffma2_rn(a1, hh[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
           if (t >= tb) {
@@ -733,13 +773,19 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       }
       // block k-1 into the other tile set, which is free: block k+1's
       // epilogue ended before this block's barrier
-      if (!kStaged && half == 0 && k > 0) commit(raw, s.tl[(k - 1) & 1]);
+      if (!kStaged && half == 0 && k > 0) {
+        commit(raw, s.tl[(k - 1) & 1]);
+        put_mask(k - 1, s.tl[(k - 1) & 1]);
+      }
     }
     if (kStaged) cp_async_wait_all();
     __syncthreads();
     // staged inputs: block k-1 into the other tile set once every copy has
     // landed (the staging area is refilled only after the next barrier)
-    if (kStaged && k > 0) stage_commit(k - 1, s.tl[(k - 1) & 1]);
+    if (kStaged && k > 0) {
+      stage_commit(k - 1, s.tl[(k - 1) & 1]);
+      put_mask(k - 1, s.tl[(k - 1) & 1]);
+    }
 
     // elementwise: du, ddelta, dz, and the per-channel sums of dD, dbias
     // (kept in registers: a thread's channels are the same in every block)
@@ -804,9 +850,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   }
 }
 
-template <typename InT, int G>
+template <typename InT, int G, bool VARLEN>
 cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
-  auto kern = scan_bwd_kernel<InT, G>;
+  auto kern = scan_bwd_kernel<InT, G, VARLEN>;
   const int smem = static_cast<int>(sizeof(BwdSmem<G>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -814,13 +860,20 @@ cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Packed sequences get their own instantiation, so their code never
+// touches the kernel of ordinary scans.
+template <typename InT, bool VARLEN>
+cudaError_t dispatch_v(const BwdParams &p, cudaStream_t stream) {
+  switch (bwd_groups(p.dstate)) {
+    case 1: return launch_typed<InT, 1, VARLEN>(p, stream);
+    case 2: return launch_typed<InT, 2, VARLEN>(p, stream);
+    default: return launch_typed<InT, 4, VARLEN>(p, stream);
+  }
+}
+
 template <typename InT>
 cudaError_t dispatch(const BwdParams &p, cudaStream_t stream) {
-  switch (bwd_groups(p.dstate)) {
-    case 1: return launch_typed<InT, 1>(p, stream);
-    case 2: return launch_typed<InT, 2>(p, stream);
-    default: return launch_typed<InT, 4>(p, stream);
-  }
+  return p.cu ? dispatch_v<InT, true>(p, stream) : dispatch_v<InT, false>(p, stream);
 }
 
 }  // namespace

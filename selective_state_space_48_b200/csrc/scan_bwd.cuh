@@ -34,6 +34,10 @@ struct BwdParams {
   // the checked build; the gradients are packed
   int64_t su[2], sdl[2], sz[2], sB[2], sC[2], sdy[2];
   int64_t ext_u, ext_delta, ext_z, ext_B, ext_C, ext_dy;
+  // packed sequences (nullptr: one sequence per row): interior offsets
+  // cu[1 .. nseq-1] start a sequence with an empty state
+  const int32_t *cu;
+  int64_t nseq;
 };
 
 // Warps per block (state groups of 4): 1, 2 or 4.

@@ -168,3 +168,51 @@ def test_backward_reads_strided_views(dt, L):
         if g_pack.get(k) is None:
             continue
         assert norm_err(g_view[k].cpu().numpy(), g_pack[k].cpu().numpy()) <= 1e-6, k
+
+
+PACKED = [
+    # name, batch, dim, N, L, dtype, interior starts
+    ("f32-blocks", 2, 40, 16, 300, "f32", [1, 16, 17, 150, 151, 299]),
+    ("bf16-long", 1, 48, 16, 1000, "bf16", [5, 32, 33, 500, 999]),
+    ("f32-N5", 1, 33, 5, 77, "f32", [2, 3, 40]),
+]
+
+
+@pytest.mark.parametrize("case", PACKED, ids=[c[0] for c in PACKED])
+def test_backward_packed_sequences(case):
+    """Packed sequences (starts on and next to 16-step block boundaries, at
+    step 1 and at the last step, one-step sequences): every gradient against
+    the oracle backward with the same packing, where nothing flows across a
+    sequence start."""
+    name, batch, dim, N, L, dt, starts = case
+    w = workloads.custom(batch, dim, N, L, in_dtype=dt, has_z=True, a_noise=0.1)
+    inp = gpu_inputs(w, seed=5150 + L, h0=True)
+    cu = sorted(set([0, L] + starts))
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5151 + L)
+    dy = torch.randn(batch, dim, L, generator=g, device="cuda")
+    d_last = torch.randn(batch, dim, N, generator=g, device="cuda")
+    g_gpu = sss.selective_scan_bwd(
+        inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"],
+        z=inp["z"], delta_bias=inp["delta_bias"], h0=inp["h0"], d_last=d_last,
+        cu_seqlens=cu_t)
+    torch.cuda.synchronize()
+    h = workloads.to_numpy_f64(inp)
+    g_ref = oracle.selective_scan_bwd(
+        h["u"], h["delta"], h["A"], h["B"], h["C"], dy.double().cpu().numpy(),
+        D=h["D"], z=h["z"], delta_bias=h["delta_bias"], h0=h["h0"],
+        d_last=d_last.double().cpu().numpy(), cu_seqlens=cu)
+    _compare(g_gpu, g_ref, name)
+
+
+def test_packed_backward_rejects_checkpoints():
+    w = workloads.custom(1, 32, 16, 64, in_dtype="f32", has_z=False)
+    inp = gpu_inputs(w, seed=5)
+    cu_t = torch.tensor([0, 10, 64], dtype=torch.int32, device="cuda")
+    ck = sss.scan_checkpoints(1, 32, 16, 64, "cuda")
+    dy = torch.ones(1, 32, 64, device="cuda")
+    with pytest.raises(sss.MssError) as ei:
+        sss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy,
+                               cu_seqlens=cu_t, checkpoints=ck)
+    assert ei.value.code == sss.MSS_ERR_UNSUPPORTED
