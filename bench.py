@@ -503,6 +503,10 @@ def run_bwd(args, rank, world, local_rank):
     dy = torch.randn(w.batch, w.dim, w.seqlen, generator=g, device=dev)
 
     ck = None
+    cu = (torch.tensor(varlen_offsets(w.seqlen, args.varlen), dtype=torch.int32, device=dev)
+          if args.varlen else None)
+    if args.checkpoints and cu is not None:
+        raise SystemExit("--checkpoints and --varlen do not combine for the backward")
     if args.checkpoints:
         ck = sss.scan_checkpoints(w.batch, w.dim, w.dstate, w.seqlen, dev)
         sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
@@ -512,7 +516,8 @@ def run_bwd(args, rank, world, local_rank):
     def step():
         sss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy,
                                D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, workspace=ws, checkpoints=ck)
+                               delta_softplus=w.softplus, workspace=ws, checkpoints=ck,
+                               cu_seqlens=cu)
 
     # workspace sized once (the size depends on the shapes only)
     nb = ctypes.c_size_t(0)
@@ -553,19 +558,21 @@ def run_bwd(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
         "config": dict(workload_config(w), **{"pass": "bwd"},
-                       **({"from_checkpoints": True} if args.checkpoints else {})),
+                       **({"from_checkpoints": True} if args.checkpoints else {}),
+                       **({"sequences_per_row": args.varlen} if args.varlen else {})),
         "state_updates_per_s": w.state_updates * K * world / (max_ms * 1e-3),
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
                      "unit": "GB/s", "frac": value / world / peak,
                      "peak_source": src,
-                     "traffic": None if args.checkpoints else profiled_traffic(w.name, "bwd"),
+                     "traffic": (None if (args.checkpoints or args.varlen)
+                                 else profiled_traffic(w.name, "bwd")),
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
         "kernel_source_hash": kernel_source_hash("bwd"),
     }
     if rank == 0:
         try:
-            line["max_norm_err"] = bwd_row_max_norm_err(sss, inp, dy, w, ws, ck)
+            line["max_norm_err"] = bwd_row_max_norm_err(sss, inp, dy, w, ws, ck, cu)
             line["max_norm_err_sample"] = ("batch row 0: du, ddelta, dz, dB, dC vs the fp64 "
                                            "oracle backward (max over the five)")
         except Exception as ex:  # reported, never fatal to the timing line
@@ -573,21 +580,23 @@ def run_bwd(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
-def bwd_row_max_norm_err(sss, inp, dy, w, ws, ck) -> float:
+def bwd_row_max_norm_err(sss, inp, dy, w, ws, ck, cu=None) -> float:
     """The backward's per-row gradients of batch row 0 against the oracle
     backward of that row alone (dA, dD, ddelta_bias sum over all rows and
     are left to the tests)."""
     import oracle
     g = sss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy,
                                D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
-                               delta_softplus=w.softplus, workspace=ws, checkpoints=ck)
+                               delta_softplus=w.softplus, workspace=ws, checkpoints=ck,
+                               cu_seqlens=cu)
     torch.cuda.synchronize()
     row = lambda t: None if t is None else t[:1].detach().float().cpu().double().numpy()
     par = lambda t: None if t is None else t.detach().float().cpu().double().numpy()
     ref = oracle.selective_scan_bwd(row(inp["u"]), row(inp["delta"]), par(inp["A"]),
                                     row(inp["B"]), row(inp["C"]), row(dy), D=par(inp["D"]),
                                     z=row(inp["z"]), delta_bias=par(inp["delta_bias"]),
-                                    delta_softplus=w.softplus)
+                                    delta_softplus=w.softplus,
+                                    cu_seqlens=None if cu is None else cu.cpu().tolist())
     worst = 0.0
     for k in ("du", "ddelta", "dz", "dB", "dC"):
         if ref[k] is None:
