@@ -855,6 +855,9 @@ def run_ours(args, rank, world, local_rank):
 
     bytes_step = w.algorithmic_bytes(out_bytes(args.out_dtype))
     value = whole_job_gbs(bytes_step, K, world, max_ms)
+    # a split scan is three kernels per step (chunks, prefix over the chunks,
+    # carry); the roofline then covers the three together
+    launches_per_step = 3 if sss.scan_workspace_size(sargs) > 0 else 1
     updates = w.state_updates * K * world / (max_ms * 1e-3)
 
     # ---- end to end through the public API with host buffers.  Every step
@@ -985,14 +988,17 @@ def run_ours(args, rank, world, local_rank):
                                  if not (args.varlen or args.trapezoid or args.checkpoints
                                          or args.out_dtype != "f32") else None),
                      "algorithmic_bytes_per_launch": bytes_step,
-                     "kernel_ms": max_kernel_ms},
+                     "kernel_ms": max_kernel_ms,
+                     **({"covers": "the step's three launches (chunks, prefix, carry)"}
+                        if launches_per_step > 1 else {})},
         # the bound that binds this scan: the special-function unit (one
         # ex2 per state update)
         "exp_unit": exp_unit_bound(w, max_kernel_ms, sm_mhz),
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke,
                 "overlap": "upload of step i+1 and read-back of step i-1 during the scan of step i"},
-        "gpu_launches": K,
+        "gpu_launches": K * launches_per_step,
+        "launches_per_step": launches_per_step,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                    "reasons": clk["reasons"], "samples": clk["samples"]},
         "kernel_source_hash": kernel_source_hash("fwd"),

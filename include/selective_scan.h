@@ -147,7 +147,9 @@ typedef struct mss_scan_args {
                              the result does not depend on the grouping) */
   int plan_chunk_steps;   /* reserved, must be 0 */
   unsigned test_flags;    /* 0 in production */
-  int64_t spin_timeout_ns;/* bound of each device-side wait; 0 = 1 s */
+  int64_t spin_timeout_ns;/* bound of the wait MSS_TESTFLAG_DROP_PUBLISH
+                             provokes; 0 = 1 s (the pipeline's own waits
+                             are bounded at 2 s) */
   /* element strides {batch, row} of the (batch, rows, seqlen) tensors; time
      is contiguous; {0, 0} = packed (see above) */
   int64_t stride_u[2];
