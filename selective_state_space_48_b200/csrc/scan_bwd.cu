@@ -161,14 +161,14 @@ __device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
 }
 
 // Bit t (t < 16) set when step t0 + t (< L) is an interior sequence start.
-__device__ unsigned restart_mask(const BwdParams &p, int64_t t0, int64_t L) {
-  int64_t lo = 1, hi = p.nseq;  // first interior start >= t0
-  while (lo < hi) {
-    const int64_t mid = lo + (hi - lo) / 2;
-    if (__ldg(p.cu + mid) < t0) lo = mid + 1; else hi = mid;
-  }
+// `nb` is the caller's cursor into cu (1 .. nseq), moved to the first
+// interior start at or after t0: blocks are visited in order, forwards in the
+// forward sweep and backwards in the reverse sweep, so it moves a step or two.
+__device__ unsigned restart_mask(const BwdParams &p, int64_t t0, int64_t L, int64_t &nb) {
+  while (nb > 1 && __ldg(p.cu + nb - 1) >= t0) --nb;
+  while (nb < p.nseq && __ldg(p.cu + nb) < t0) ++nb;
   unsigned m = 0u;
-  for (int64_t i = lo; i < p.nseq; ++i) {
+  for (int64_t i = nb; i < p.nseq; ++i) {
     const int64_t t = __ldg(p.cu + i) - t0;
     if (t >= kBwdTimeBlock || t0 + t >= L) break;
     m |= 1u << t;
@@ -294,8 +294,10 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   };
   // packed sequences: the block's restart mask, written by thread 0 with its
   // tiles (no decay across a start: exp(Delta A) is taken as 0 there)
+  int64_t mask_cursor = 1;
   auto put_mask = [&](int k, BwdTiles<G> &T) {
-    if (VARLEN && tid == 0) T.rmask = restart_mask(p, static_cast<int64_t>(k) * TB, L);
+    if (VARLEN && tid == 0)
+      T.rmask = restart_mask(p, static_cast<int64_t>(k) * TB, L, mask_cursor);
   };
   auto commit = [&](const Raw &r, BwdTiles<G> &T) {
 #pragma unroll

@@ -175,13 +175,16 @@ struct Scan {
     }
     return lo;
   }
-  // Bit j (j < 4) set when step pos + j (< t_end) starts a sequence; `nb`
-  // is the caller's cursor into cu, only ever moved forward.
-  __device__ uint32_t restarts4(int64_t pos, int64_t &nb) const {
+  // Offset of interior start nb (nseq fits 32 bits, checked on the host).
+  __device__ int start_at(int nb) const { return nb < p.nseq ? __ldg(p.cu + nb) : 0; }
+  // Bit j (j < 4) set when step pos + j (< t_end) starts a sequence.  The
+  // caller's cursor (nb, next = start_at(nb)) only moves forward, so a
+  // window with no start in it costs one compare and no load.
+  __device__ uint32_t restarts4(int64_t pos, int &nb, int &next) const {
     uint32_t m = 0;
-    for (int j = 0; j < 4 && pos + j < t_end; ++j) {
-      while (nb < p.nseq && __ldg(p.cu + nb) < pos + j) ++nb;
-      if (nb < p.nseq && __ldg(p.cu + nb) == pos + j) m |= 1u << j;
+    while (nb < p.nseq && next < pos + 4) {
+      if (next >= pos && next < t_end) m |= 1u << (next - pos);
+      next = start_at(++nb);
     }
     return m;
   }
@@ -606,7 +609,8 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
   } else if (is_prep) {
     const typename S::Slots sl = sc.make_slots(tp);
     // cursor into the sequence offsets for this thread's steps
-    int64_t nb = VARLEN ? sc.first_start_from(sc.t_begin + sl.t) : 0;
+    int nb = VARLEN ? static_cast<int>(sc.first_start_from(sc.t_begin + sl.t)) : 0;
+    int next_start = VARLEN ? sc.start_at(nb) : 0;
     // split scans: this thread's share of each slot's running sum of Delta;
     // the four threads of a channel row write the sum at every segment
     // start for the carry launch
@@ -624,7 +628,7 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
         }
       }
       if (blk >= 2) wait_hand(kTilesFree, blk & 1);
-      const uint32_t rs = VARLEN ? sc.restarts4(sc.t0_of(blk) + sl.t, nb) : 0u;
+      const uint32_t rs = VARLEN ? sc.restarts4(sc.t0_of(blk) + sl.t, nb, next_start) : 0u;
       // trapezoidal update: u of the step before the block, for the slots
       // that start it (read from HBM/L2: the previous raw stage may already
       // be refilled)
