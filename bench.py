@@ -1092,10 +1092,23 @@ def run_ssd(args, rank, world, local_rank):
     inp = workloads.make_ssd_inputs(w, seed=48100, device=dev)
     ody = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
     y = torch.empty(w.batch, w.seqlen, w.nheads, w.headdim, dtype=ody, device=dev)
+    # workspace sized once: it lets the last wave's sequences be cut into
+    # pieces spread over the schedule (the library's rule, restated here
+    # only to report it)
+    ws_bytes = sss.ssd_workspace_size(sss.make_ssd_args(inp["x"], inp["dt"], inp["A"],
+                                                        inp["B"], inp["C"]))
+    ws = sss.alloc_workspace(ws_bytes, dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    waves, ncut = divmod(w.batch * w.nheads, sms)
+    nch = (w.seqlen + 127) // 128
+    parts = (min(max(2, (sms + ncut // 2) // ncut), waves + 1, nch, 8)
+             if ws_bytes and ncut else 0)
+    ncut = ncut if parts else 0
 
     def step():
         sss.ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"],
-                    z=inp["z"], dt_bias=inp["dt_bias"], dt_softplus=w.softplus, y=y)
+                    z=inp["z"], dt_bias=inp["dt_bias"], dt_softplus=w.softplus, y=y,
+                    workspace=ws if ws is not None else False)
 
     for _ in range(args.warmup):
         step()
@@ -1135,6 +1148,8 @@ def run_ssd(args, rank, world, local_rank):
         "config": dict(ssd_config(w, args.out_dtype),
                        l2=f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step)"),
         "tokens_per_s": w.batch * w.seqlen * K * world / (max_ms * 1e-3),
+        "schedule": {"ctas": w.batch * w.nheads + max(parts - 1, 0) * ncut,
+                     "sequences_cut": ncut, "pieces_per_cut_sequence": parts},
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
                      "unit": "GB/s", "frac": value / world / peak,
                      "peak_source": src,

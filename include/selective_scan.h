@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 9
+#define MSS_ABI_VERSION 10
 
 typedef enum {
   MSS_OK = 0,

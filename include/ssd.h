@@ -50,6 +50,18 @@
  * the caller, nothing allocated, work enqueued on `stream` (a cudaStream_t
  * as void*, NULL = legacy default stream) without synchronising.
  *
+ * Schedule.  One CTA per (batch row, head) sequence, one CTA per SM, so
+ * the sequences run in waves.  When the last wave is at most half full
+ * (r = batch * nheads mod the SM count, 0 < 2 r <= the SM count), at least
+ * one wave is full and the sequence has at least two chunks, the last r
+ * sequences are cut at chunk boundaries into min(round(SMs / r), full
+ * waves + 1, chunks, 8) pieces, and the pieces are spread over the
+ * schedule between the whole sequences, so the last wave runs short
+ * pieces.  Each piece starts from the end state of the piece before (fp32,
+ * in the workspace); the output is bit-identical to the uncut schedule.
+ * Cutting needs the workspace below (mss_ssd_workspace_size() bytes);
+ * without one (workspace NULL) every sequence runs whole.
+ *
  * Errors.  Argument errors return MSS_ERR_INVALID_ARG / MSS_ERR_UNSUPPORTED
  * and enqueue nothing; a failed launch returns MSS_ERR_CUDA.  The kernel's
  * waits are bounded (spin_timeout_ns, 0 = 2 s); one that runs out records
@@ -89,7 +101,19 @@ typedef struct mss_ssd_args {
   void *y;
   float *last_state;    /* NULL: not written */
   uint64_t spin_timeout_ns;
+  /* NULL (every sequence runs whole), or device memory of at least
+     mss_ssd_workspace_size() bytes, 16-byte aligned, not shared with a call
+     in flight: a work-item counter and flags (cleared by cudaMemsetAsync on
+     `stream` at every call) and the end states of the pieces.
+     Smaller than required: MSS_ERR_WORKSPACE. */
+  void *workspace;
+  size_t workspace_bytes;
 } mss_ssd_args;
+
+/* Workspace bytes that let mamba2_ssd_fwd cut the last wave's sequences
+ * into pieces on the current device (0 when its schedule cuts nothing).  Reads only
+ * batch, nheads and seqlen, and the current device's SM count. */
+mss_status mss_ssd_workspace_size(const mss_ssd_args *args, size_t *bytes);
 
 /* Chunked SSD forward: y (and last_state) for the arguments above. */
 mss_status mamba2_ssd_fwd(const mss_ssd_args *args, void *stream);

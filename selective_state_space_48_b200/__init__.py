@@ -12,6 +12,7 @@ Functions mirror the C entry points:
   mss_scan_workspace_size   -> scan_workspace_size(...)
   mss_scan_status           -> scan_status(...)
   mamba2_ssd_fwd            -> ssd_fwd(...)         (include/ssd.h)
+  mss_ssd_workspace_size    -> ssd_workspace_size(...)
 """
 from __future__ import annotations
 
@@ -25,7 +26,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 9  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 10  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -50,6 +51,7 @@ EXPORTED_SYMBOLS = (
     "mamba_selective_scan_bwd",
     "mss_status_string",
     "mss_abi_version",
+    "mss_ssd_workspace_size",
     "mamba2_ssd_fwd",
     "mss_ssd_status",
 )
@@ -150,6 +152,8 @@ class SsdArgs(ctypes.Structure):
         ("dt_softplus", ctypes.c_int),
     ] + [(name, ctypes.c_void_p) for name in ("h0", "y", "last_state")] + [
         ("spin_timeout_ns", ctypes.c_uint64),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -183,6 +187,8 @@ def _bind(lib):
     lib.mamba_selective_scan_bwd.restype = ctypes.c_int
     lib.mss_status_string.argtypes = [ctypes.c_int]
     lib.mss_status_string.restype = ctypes.c_char_p
+    lib.mss_ssd_workspace_size.argtypes = [P(SsdArgs), P(ctypes.c_size_t)]
+    lib.mss_ssd_workspace_size.restype = ctypes.c_int
     lib.mamba2_ssd_fwd.argtypes = [P(SsdArgs), ctypes.c_void_p]
     lib.mamba2_ssd_fwd.restype = ctypes.c_int
     lib.mss_ssd_status.argtypes = [ctypes.c_void_p]
@@ -451,16 +457,28 @@ def make_ssd_args(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True
     return a
 
 
+def ssd_workspace_size(args: SsdArgs) -> int:
+    """``mss_ssd_workspace_size``: bytes that let the SSD scan cut the last
+    wave's sequences in two on the current device (0: nothing to cut)."""
+    n = ctypes.c_size_t(0)
+    rc = load_library().mss_ssd_workspace_size(ctypes.byref(args), ctypes.byref(n))
+    if rc != MSS_OK:
+        raise MssError(rc, "mss_ssd_workspace_size")
+    return int(n.value)
+
+
 def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None,
             return_last_state=False, out_dtype=torch.float32, y=None, last_state=None,
-            stream=None, check_status=False):
+            stream=None, check_status=False, workspace=None):
     """Mamba-2 (SSD) chunked scan through ``mamba2_ssd_fwd``.
 
     x, z: (batch, L, nheads, headdim); dt: (batch, L, nheads); B, C:
     (batch, L, ngroups, dstate), all bfloat16; A, D, dt_bias: (nheads,)
     float32; h0: (batch, nheads, headdim, dstate) float32.  Returns y
     (batch, L, nheads, headdim) in ``out_dtype`` (and the final state when
-    ``return_last_state``).
+    ``return_last_state``).  ``workspace``: None allocates what
+    ``ssd_workspace_size`` asks for; False runs every sequence whole; a
+    uint8 CUDA tensor is used as given.
     """
     batch, L, H, P = x.shape
     N = B.shape[3]
@@ -469,10 +487,18 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=N
     if return_last_state and last_state is None:
         last_state = torch.empty((batch, H, P, N), dtype=torch.float32, device=x.device)
     args = make_ssd_args(x, dt, A, B, C, D, z, dt_bias, dt_softplus, h0, y, last_state)
+    if workspace is None:
+        workspace = alloc_workspace(ssd_workspace_size(args), x.device)
+    if workspace is not None and workspace is not False:
+        args.workspace = workspace.data_ptr()
+        args.workspace_bytes = workspace.numel() * workspace.element_size()
     lib = load_library()
     rc = lib.mamba2_ssd_fwd(ctypes.byref(args), _stream_handle(stream))
     if rc != MSS_OK:
         raise MssError(rc, "mamba2_ssd_fwd")
+    # keep the workspace alive until the stream has used it
+    if workspace is not None and workspace is not False:
+        workspace.record_stream(stream or torch.cuda.current_stream())
     if check_status:
         rc = lib.mss_ssd_status(_stream_handle(stream))
         if rc != MSS_OK:
@@ -488,7 +514,7 @@ __all__ = [
     "selective_scan_fwd", "selective_state_update", "scan_workspace_size",
     "scan_status", "make_scan_args", "load_library", "status_string",
     "MssError", "ScanArgs", "UpdateArgs", "EXPORTED_SYMBOLS", "build",
-    "ssd_fwd", "make_ssd_args", "SsdArgs",
+    "ssd_fwd", "make_ssd_args", "SsdArgs", "ssd_workspace_size",
 ]
 
 

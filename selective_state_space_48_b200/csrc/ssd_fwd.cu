@@ -27,6 +27,20 @@
 // are issued as soon as Hp and X'' are ready, so they run while the
 // epilogue builds the masked scores S'.
 //
+// The grid has one CTA per sequence, so batch * nheads CTAs fill the SMs in
+// waves.  When the last wave is at most half full (r sequences), those r
+// sequences are cut at chunk boundaries into `parts` pieces (about SMs / r,
+// at most the number of full waves + 1) and the pieces are spread over the
+// schedule: CTAs take work items in ticket order, and the order is piece 0
+// of the r sequences, a share of the whole sequences, piece 1, another
+// share, ..., the last piece.  A piece therefore starts only after the
+// piece before it was taken by a running CTA, normally long after that one
+// ended, and the last wave holds short pieces instead of whole sequences.
+// A piece publishes its end state (fp32, in the caller's workspace) with a
+// release flag; the next piece loads it as its initial state.  Every piece
+// runs exactly the per-chunk arithmetic of the whole sequence, so the output
+// is the same bit for bit.
+//
 // Shared memory tiles are [128 rows][64 bf16] with the 128-byte swizzle that
 // the TMA writes and the tensor core reads: 16-byte chunk j of row r sits at
 // chunk position j ^ (r % 8).  Every wait on an mbarrier is bounded; a wait
@@ -38,6 +52,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -69,6 +84,7 @@ constexpr int oTot = oColf + Q * 4;    // float warp totals [4]
 constexpr int oBar = oTot + 16;        // 10 mbarriers
 constexpr int oTmemSlot = oBar + 10 * 8;
 constexpr int oAbort = oTmemSlot + 4;
+constexpr int oItem = oAbort + 4;      // this CTA's work item
 constexpr int kSmemUsed = oAbort + 12;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // room to align the base
 static_assert(kSmemBytes <= 232448, "shared memory above the per-block limit");
@@ -96,6 +112,14 @@ struct Params {
   float *last;
   unsigned *status;
   uint64_t spin_ns;
+  // cut sequences: the last ncut of the batch * nheads order, in `parts`
+  // pieces, with gfull whole sequences between two pieces (the rest before
+  // the last piece); ticket, flags and end states in the workspace
+  int ncut, parts;
+  int64_t gfull;
+  unsigned *ticket;
+  unsigned *flag;  // [(parts - 1) * ncut]: 1 once the piece's end state is written
+  float *mid;      // [(parts - 1) * ncut][P][NS]: end states of all but the last pieces
 };
 
 struct Maps {
@@ -377,6 +401,44 @@ struct StepPlan {
   }
 };
 
+// Work item -> sequence bh and its chunks [c0, c0 + nc), and the state
+// slots of a piece: `in` holds its initial state, `out` receives its end
+// state (-1: the caller's h0 / last_state).  Items in ticket order: piece 0
+// of the cut sequences, gfull whole sequences, piece 1, gfull more, ...,
+// the remaining whole sequences, the last piece.
+struct Work {
+  int64_t bh;
+  int c0, nc, in, out;
+  static __device__ Work of(int item, const Params &p, int nchunks) {
+    Work w{item, 0, nchunks, -1, -1};
+    if (!p.ncut) return w;
+    const int64_t F = p.batch * p.H - p.ncut;  // whole sequences
+    int64_t pos = item, full = 0;
+    for (int j = 0; j < p.parts; ++j) {
+      if (pos < p.ncut) {  // piece j of cut sequence si
+        const int si = static_cast<int>(pos);
+        w.bh = F + si;
+        w.c0 = static_cast<int>(static_cast<int64_t>(j) * nchunks / p.parts);
+        w.nc = static_cast<int>(static_cast<int64_t>(j + 1) * nchunks / p.parts) - w.c0;
+        w.in = j > 0 ? (j - 1) * p.ncut + si : -1;
+        w.out = j < p.parts - 1 ? j * p.ncut + si : -1;
+        return w;
+      }
+      pos -= p.ncut;
+      if (j < p.parts - 1) {
+        const int64_t gs = j < p.parts - 2 ? p.gfull : F - p.gfull * (p.parts - 2);
+        if (pos < gs) {
+          w.bh = full + pos;
+          return w;
+        }
+        pos -= gs;
+        full += gs;
+      }
+    }
+    return w;  // not reached: the grid has F + parts * ncut items
+  }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_fwd_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ unsigned char smem_raw[];
@@ -384,9 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t bh = blockIdx.x;
-  const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
-  const int g = static_cast<int>(h / (p.H / p.G));
   const int nchunks = static_cast<int>((p.L + Q - 1) / Q);
 
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + oBar);
@@ -410,6 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + kDoneY, 1);
     mbar_init(bar + kDoneH, 1);
     *abort = 0;
+    *reinterpret_cast<int *>(sm + oItem) =
+        p.ncut ? static_cast<int>(atomicAdd(p.ticket, 1u)) : static_cast<int>(blockIdx.x);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -418,16 +479,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  const Work wk = Work::of(*reinterpret_cast<const int *>(sm + oItem), p, nchunks);
+  const int c0 = wk.c0, nc = wk.nc;
+  const int b = static_cast<int>(wk.bh / p.H), h = static_cast<int>(wk.bh % p.H);
+  const int g = static_cast<int>(h / (p.H / p.G));
+
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer
     if (lane == 0) {
-      for (int c = 0; c < nchunks; ++c) {
-        const int st = c & 1;
-        if (c >= 2) sy.wait(kEmpty + st, ((c >> 1) - 1) & 1);
+      for (int i = 0; i < nc; ++i) {
+        const int st = i & 1;
+        if (i >= 2) sy.wait(kEmpty + st, ((i >> 1) - 1) & 1);
         unsigned char *s = sm + st * kStage;
         uint64_t *full = bar + kFull + st;
         mbar_expect_tx(full, kStage);
-        const int t0 = c * Q;
+        const int t0 = (c0 + i) * Q;
         tma_load_4d(s + oC, &maps.C, 0, g, t0, b, full);
         tma_load_4d(s + oC + kTile, &maps.C, 64, g, t0, b, full);
         tma_load_4d(s + oB, &maps.B, 0, g, t0, b, full);
@@ -435,8 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(s + oX, &maps.x, 0, h, t0, b, full);
       }
       // no copy may still be landing when the CTA exits
-      for (int c = nchunks > 2 ? nchunks - 2 : 0; c < nchunks; ++c)
-        sy.drain(kFull + (c & 1), (c >> 1) & 1);
+      for (int i = nc > 2 ? nc - 2 : 0; i < nc; ++i) sy.drain(kFull + (i & 1), (i >> 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------- tensor-core issue
@@ -448,11 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idH = idesc_bf16(128, 64, 1, 1);
       const uint64_t dHp = desc_mn(sbase + oHp, 0, kTile);
       const uint64_t dXpp = desc_mn(sbase + oXpp, 0, kTile);
-      // S = C B^T of chunk c (stage c % 2), after its tiles have landed
-      auto scores = [&](int c) {
-        const uint32_t s = sbase + (c & 1) * kStage;
+      // S = C B^T of this CTA's i-th chunk (stage i % 2), after its tiles
+      // have landed
+      auto scores = [&](int i) {
+        const uint32_t s = sbase + (i & 1) * kStage;
         const uint64_t dC = desc_k(s + oC, 0), dBk = desc_k(s + oB, 0);
-        sy.wait(kFull + (c & 1), (c >> 1) & 1);
+        sy.wait(kFull + (i & 1), (i >> 1) & 1);
         tc_fence_after();
         if (!*abort) {
 #pragma unroll
@@ -467,19 +533,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Hp is written, then the next chunk's scores, then this chunk's state
       // update, which is needed only after the next chunk's masked scores
       // are built.
-      if (nchunks > 0) scores(0);
-      for (int c = 0; c < nchunks; ++c) {
-        const uint32_t s = sbase + (c & 1) * kStage;
+      if (nc > 0) scores(0);
+      for (int i = 0; i < nc; ++i) {
+        const uint32_t s = sbase + (i & 1) * kStage;
         const uint64_t dC = desc_k(s + oC, 0);
         const uint64_t dBm = desc_mn(s + oB, 0, kTile), dX = desc_mn(s + oX, 0, kTile);
-        sy.wait(kReadyScores, c & 1);
+        sy.wait(kReadyScores, i & 1);
         tc_fence_after();
         if (!*abort) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // Y = S' X, S' from tensor memory
             umma_bf16_ts(tmem + kColY, tmem + kColSp + 8 * kk, dX + kk * 128, idY, kk > 0);
         }
-        sy.wait(kReadyHp, c & 1);
+        sy.wait(kReadyHp, i & 1);
         tc_fence_after();
         if (!*abort) {
 #pragma unroll
@@ -488,8 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       dHp + kk * 128, idY, kk > 0);
         }
         umma_commit(bar + kDoneY);
-        if (c + 1 < nchunks) scores(c + 1);
-        sy.wait(kReadyState, c & 1);
+        if (i + 1 < nc) scores(i + 1);
+        sy.wait(kReadyState, i & 1);
         tc_fence_after();
         if (!*abort) {
 #pragma unroll
@@ -499,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(bar + kDoneH);
       }
       // every product done before the tensor memory is freed
-      if (nchunks > 0) sy.drain(kDoneH, (nchunks - 1) & 1);
+      if (nc > 0) sy.drain(kDoneH, (nc - 1) & 1);
     }
     __syncwarp();
   } else {
@@ -521,26 +587,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                         p.dt + static_cast<int64_t>(b) * p.L * H + h, p.L, H,
                         p.A[h] * kLog2e, p.dt_bias ? p.dt_bias[h] : 0.0f, p.softplus};
 
-    // the initial state into H (row n = r, columns 16e .. 16e + 15)
+    // the initial state into H (row n = r, columns 16e .. 16e + 15): the
+    // caller's h0, or for a later piece the end state of the piece before,
+    // once published (one thread waits, bounded; the barrier passes it on)
     {
       const float *h0 = p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * P * NS : nullptr;
+      if (wk.in >= 0) {
+        if (tid == 64) {
+          const uint64_t start = global_timer_ns();
+          while (ld_acquire_gpu(p.flag + wk.in) == 0u) {
+            if (global_timer_ns() - start > p.spin_ns) {
+              *abort = 1;
+              atomicOr(p.status, static_cast<unsigned>(MSS_ERR_TIMEOUT));
+              break;
+            }
+            __nanosleep(256);
+          }
+          __threadfence();
+        }
+        bar_sync(kEpiBarrier, kEpi);
+        h0 = p.mid + static_cast<int64_t>(wk.in) * P * NS;
+      }
       uint32_t v[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        v[j] = __float_as_uint(h0 ? h0[(e * 16 + j) * NS + r] : 0.0f);
+        v[j] = __float_as_uint(h0 ? __ldcg(h0 + (e * 16 + j) * NS + r) : 0.0f);
       tmem_st16(tl + kColH + 16 * e, v);
       tmem_wait_st();
     }
 
     // raw steps are loaded one chunk ahead
     unsigned short dt_next = 0;
-    if (e == 0 && r < p.L)
-      dt_next = *reinterpret_cast<const unsigned short *>(plan.dtp + static_cast<int64_t>(r) * H);
-    plan.run(0, q, e, lane, r, dt_next);
+    const int64_t tfirst = static_cast<int64_t>(c0) * Q + r;
+    if (e == 0 && tfirst < p.L)
+      dt_next = *reinterpret_cast<const unsigned short *>(plan.dtp + tfirst * H);
+    plan.run(c0, q, e, lane, r, dt_next);
     float cum = cum_s[r], cl = cum_s[Q - 1];
 
-    for (int c = 0; c < nchunks; ++c) {
-      const int st = c & 1;
+    // chunk c = c0 + i of the sequence; barrier phases and stages follow i
+    for (int i = 0; i < nc; ++i) {
+      const int c = c0 + i;
+      const int st = i & 1;
       unsigned char *s = sm + st * kStage;
       const int64_t t = static_cast<int64_t>(c) * Q + r;
 
@@ -548,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // S 2^(c_t - c_end(gb)) colf[s] (both factors <= 1); on the diagonal
       // S 2^(c_t - c_s) Delta_s for s <= t, factored the same way when that
       // cannot overflow; above it zero
-      sy.wait(kSFull, c & 1);
+      sy.wait(kSFull, i & 1);
       tc_fence_after();
       {
         const int gb = e;
@@ -608,15 +695,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the previous chunk's state update is done: its tiles (B read by it,
       // C holding the staged y) may be released once the y store has read
       // the staging tile
-      if (c >= 1) {
-        sy.wait(kDoneH, (c - 1) & 1);
+      if (i >= 1) {
+        sy.wait(kDoneH, (i - 1) & 1);
         tc_fence_after();
         if (writer) {
           tma_store_wait_read();
-          mbar_arrive(bar + kEmpty + ((c - 1) & 1));
+          mbar_arrive(bar + kEmpty + ((i - 1) & 1));
         }
       }
-      sy.wait(kFull + st, (c >> 1) & 1);
+      sy.wait(kFull + st, (i >> 1) & 1);
 
       // Hp row n = r (columns 16e .. 16e + 15): bf16 copy of the state
       // before this chunk; then the state decays over the chunk:
@@ -664,14 +751,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // the next chunk's steps, while the output products run
       const float cum_t = cum;
-      if (c + 1 < nchunks) {
+      if (i + 1 < nc) {
         plan.run(c + 1, q, e, lane, r, dt_next);
         cum = cum_s[r];
         cl = cum_s[Q - 1];
       }
 
       // y row t, columns 16e .. 16e + 15: Y + 2^(c_t) YO + D x, gated
-      sy.wait(kDoneY, c & 1);
+      sy.wait(kDoneY, i & 1);
       tc_fence_after();
       {
         const float eo = ex2_mufu(cum_t);
@@ -741,18 +828,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (writer) tma_store_wait_all();
-    // the state after the last chunk (columns 16e .. 16e + 15)
-    if (nchunks > 0) {
-      sy.wait(kDoneH, (nchunks - 1) & 1);
+    // the state after the last chunk (columns 16e .. 16e + 15): the
+    // caller's last_state, or a piece's end state for the next piece
+    if (nc > 0) {
+      sy.wait(kDoneH, (nc - 1) & 1);
       tc_fence_after();
     }
-    if (p.last) {
-      float *lr = p.last + (static_cast<int64_t>(b) * H + h) * P * NS;
+    // (the work item is decoded again: nothing of it stays live in the loop)
+    const Work we = Work::of(*reinterpret_cast<volatile int *>(sm + oItem), p, nchunks);
+    float *lr = we.out >= 0 ? p.mid + static_cast<int64_t>(we.out) * P * NS
+                            : (p.last ? p.last + we.bh * P * NS : nullptr);
+    if (lr) {
       uint32_t v[16];
       tmem_ld16(tl + kColH + 16 * e, v);
       tmem_wait_ld(v);
 #pragma unroll
       for (int j = 0; j < 16; ++j) lr[(e * 16 + j) * NS + r] = __uint_as_float(v[j]);
+    }
+    if (we.out >= 0) {
+      // every epilogue thread's stores are visible before the flag is set
+      // (published after a timeout too, so the next piece never waits for
+      // nothing)
+      __threadfence();
+      bar_sync(kEpiBarrier, kEpi);
+      if (tid == 64) st_release_gpu(p.flag + we.out, 1u);
     }
   }
 
@@ -833,8 +932,44 @@ mss_status check(const mss_ssd_args *a) {
       (reinterpret_cast<uintptr_t>(a->dt) & 1))
     return MSS_ERR_INVALID_ARG;
   // grid of batch * nheads CTAs; TMA coordinates are 32-bit
-  if (a->batch * a->nheads >= (int64_t(1) << 31) || a->seqlen >= (int64_t(1) << 31) - Q)
+  if (a->batch * a->nheads >= (int64_t(1) << 31) - 65536 || a->seqlen >= (int64_t(1) << 31) - Q)
     return MSS_ERR_UNSUPPORTED;
+  return MSS_OK;
+}
+
+// The cut schedule (one CTA per SM: a CTA's shared memory is above half an
+// SM's).  With W full waves and r sequences left over (0 < 2 r <= SMs,
+// W >= 1: the pieces need whole sequences to run between them), the r
+// sequences are cut into min(round(SMs / r), W + 1, chunks, 8) >= 2
+// pieces.  Workspace: the work-item counter at byte 0, the flags from byte
+// 256, the end states after them; the first `clear` bytes are cleared per
+// call.
+struct Plan {
+  int ncut = 0, parts = 0;
+  int64_t gfull = 0;
+  size_t clear = 0, bytes = 0;
+};
+
+mss_status plan_of(const mss_ssd_args *a, Plan *pl) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  *pl = Plan();
+  if (sms < 1) return MSS_OK;
+  const int64_t BH = a->batch * a->nheads;
+  const int64_t nchunks = (a->seqlen + Q - 1) / Q;
+  const int64_t W = BH / sms, r = BH % sms;
+  if (W < 1 || r < 1 || 2 * r > sms || nchunks < 2) return MSS_OK;
+  int64_t parts = (sms + r / 2) / r;  // round(SMs / r) >= 2
+  parts = std::min<int64_t>(std::min<int64_t>(parts, W + 1), std::min<int64_t>(nchunks, 8));
+  if (parts < 2) return MSS_OK;
+  const size_t slots = static_cast<size_t>(r) * static_cast<size_t>(parts - 1);
+  pl->ncut = static_cast<int>(r);
+  pl->parts = static_cast<int>(parts);
+  pl->gfull = (BH - r) / (parts - 1);
+  pl->clear = 256 + ((4 * slots + 255) / 256) * 256;
+  pl->bytes = pl->clear + slots * P * NS * sizeof(float);
   return MSS_OK;
 }
 
@@ -855,6 +990,12 @@ extern "C" mss_status mamba2_ssd_fwd(const mss_ssd_args *a, void *stream) {
       !ssd::encode_4d(&maps.C, a->C, ssd::NS, G, L, Bt) ||
       !ssd::encode_y(&maps.y, a->y, a->out_dtype == MSS_BF16, H, L, Bt))
     return MSS_ERR_CUDA;
+  ssd::Plan plan;
+  const mss_status pst = ssd::plan_of(a, &plan);
+  if (pst != MSS_OK) return pst;
+  if (!a->workspace) plan = ssd::Plan();  // no workspace: every sequence whole
+  if (plan.ncut && (a->workspace_bytes < plan.bytes)) return MSS_ERR_WORKSPACE;
+  if (plan.ncut && !ssd::al16(a->workspace)) return MSS_ERR_INVALID_ARG;
   unsigned *status = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), ssd::g_ssd_status) !=
       cudaSuccess)
@@ -876,14 +1017,34 @@ extern "C" mss_status mamba2_ssd_fwd(const mss_ssd_args *a, void *stream) {
   p.last = a->last_state;
   p.status = status;
   p.spin_ns = a->spin_timeout_ns ? a->spin_timeout_ns : 2000000000ull;
+  unsigned char *ws = static_cast<unsigned char *>(a->workspace);
+  p.ncut = plan.ncut;
+  p.parts = plan.parts;
+  p.gfull = plan.gfull;
+  p.ticket = plan.ncut ? reinterpret_cast<unsigned *>(ws) : nullptr;
+  p.flag = plan.ncut ? reinterpret_cast<unsigned *>(ws + 256) : nullptr;
+  p.mid = plan.ncut ? reinterpret_cast<float *>(ws + plan.clear) : nullptr;
   // per launch: the attribute belongs to the current device
   if (cudaFuncSetAttribute(ssd::ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            ssd::kSmemBytes) != cudaSuccess)
     return MSS_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(a->batch * a->nheads);
+  if (plan.ncut &&
+      cudaMemsetAsync(ws, 0, plan.clear, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSS_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(a->batch * a->nheads +
+                                              static_cast<int64_t>(plan.parts - 1) * plan.ncut);
   ssd::ssd_fwd_kernel<<<grid, ssd::kThreads, ssd::kSmemBytes,
                         static_cast<cudaStream_t>(stream)>>>(maps, p);
   return cudaGetLastError() == cudaSuccess ? MSS_OK : MSS_ERR_CUDA;
+}
+
+extern "C" mss_status mss_ssd_workspace_size(const mss_ssd_args *a, size_t *bytes) {
+  if (!a || !bytes || a->batch < 1 || a->seqlen < 1 || a->nheads < 1) return MSS_ERR_INVALID_ARG;
+  ssd::Plan plan;
+  const mss_status st = ssd::plan_of(a, &plan);
+  if (st != MSS_OK) return st;
+  *bytes = plan.bytes;
+  return MSS_OK;
 }
 
 extern "C" mss_status mss_ssd_status(void *stream) {

@@ -69,7 +69,7 @@ def test_checked_build_exports_the_same_symbols():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mss_abi_version() == sss.ABI_VERSION == 9
+    assert lib.mss_abi_version() == sss.ABI_VERSION == 10
     for code, name in [(0, "MSS_OK"), (1, "MSS_ERR_INVALID_ARG"),
                        (2, "MSS_ERR_UNSUPPORTED"), (3, "MSS_ERR_CUDA"),
                        (4, "MSS_ERR_TIMEOUT"), (5, "MSS_ERR_WORKSPACE")]:
@@ -296,3 +296,13 @@ def _ssd_args(**kw):
 def test_ssd_argument_checks(lib, kw, code):
     """Rejected before anything is enqueued (no GPU is touched)."""
     assert lib.mamba2_ssd_fwd(ctypes.byref(_ssd_args(**kw)), None) == code
+
+
+@pytest.mark.parametrize("kw", [dict(batch=0), dict(seqlen=0), dict(nheads=0)],
+                         ids=lambda v: str(v))
+def test_ssd_workspace_size_checks_sizes_first(lib, kw):
+    """Bad sizes are rejected before the device is asked for its SM count."""
+    n = ctypes.c_size_t(7)
+    assert lib.mss_ssd_workspace_size(ctypes.byref(_ssd_args(**kw)), ctypes.byref(n)) == \
+        sss.MSS_ERR_INVALID_ARG
+    assert lib.mss_ssd_workspace_size(None, ctypes.byref(n)) == sss.MSS_ERR_INVALID_ARG

@@ -136,3 +136,70 @@ def test_ssd_is_deterministic():
     y2, l2 = _run(inp)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2) and torch.equal(l1, l2)
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+CUT_CASES = [
+    # name, batch, L, heads, groups: with 148 SMs, the sequences of the last
+    # wave are cut into pieces spread over the schedule
+    ("three-pieces-ragged", 2, 657, 160, 2),   # 320: 2 waves + 24, 3 pieces of 2 chunks
+    ("halves-of-two-chunks", 1, 129, 160, 1),  # 160: 1 wave + 12, 2 pieces of 1 chunk
+    ("halves-of-five-chunks", 1, 640, 200, 1), # 200: 1 wave + 52, pieces of 2 and 3 chunks
+    ("four-pieces-of-one-chunk", 4, 385, 112, 1),  # 448: 3 waves + 4, 4 pieces
+]
+
+
+@pytest.mark.parametrize("case", CUT_CASES, ids=[c[0] for c in CUT_CASES])
+def test_ssd_cut_sequences_equal_the_whole_schedule(case):
+    """Sequences cut into pieces at chunk boundaries (each piece starting
+    from the fp32 end state of the piece before) run the same per-chunk
+    arithmetic as the whole sequence, so y and the final state are
+    bit-identical to the schedule without a workspace; and they match the
+    oracle."""
+    name, batch, L, H, G = case
+    w = workloads.SsdWorkload(name, batch, L, H, ngroups=G, has_z=True)
+    inp = workloads.make_ssd_inputs(w, seed=5760 + L, device="cuda", h0=True)
+    args = sss.make_ssd_args(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"])
+    assert sss.ssd_workspace_size(args) > 0 or _sms() != 148
+    y_cut, last_cut = _run(inp)
+    y_whole, last_whole = sss.ssd_fwd(
+        inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], z=inp["z"],
+        dt_bias=inp["dt_bias"], h0=inp["h0"], return_last_state=True, check_status=True,
+        workspace=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y_cut, y_whole)
+    assert torch.equal(last_cut, last_whole)
+    y_ref, last_ref = _oracle(inp)
+    assert norm_err(y_cut.cpu().numpy(), y_ref) <= TOL
+    assert norm_err(last_cut.cpu().numpy(), last_ref) <= TOL
+
+
+def test_ssd_workspace_plan():
+    """What is cut, and the workspace it takes: nothing without a whole wave
+    to run between the pieces, for one chunk, or when the last wave is more
+    than half full; r sequences in min(round(SMs / r), waves + 1, chunks, 8)
+    pieces otherwise.  A workspace smaller than asked for is rejected before
+    launch."""
+    sms = _sms()
+
+    def need(batch, H, L):
+        w = workloads.SsdWorkload("plan", batch, L, H, has_z=False)
+        inp = workloads.make_ssd_inputs(w, seed=5770, device="cuda")
+        args = sss.make_ssd_args(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"])
+        return sss.ssd_workspace_size(args), inp
+
+    state = 64 * 128 * 4
+    assert need(1, 4, 300)[0] == 0               # less than one wave
+    assert need(1, sms + 6, 128)[0] == 0         # one chunk
+    assert need(1, sms, 300)[0] == 0             # whole waves
+    assert need(1, 2 * sms - 1, 300)[0] == 0     # last wave more than half full
+    assert need(1, 2 * sms + 24, 640)[0] == 512 + 2 * 24 * state  # 3 pieces
+    n, inp = need(1, sms + 6, 300)
+    assert n == 512 + 6 * state                  # 2 pieces: counter, flags, 6 states
+    small = torch.empty(n - 4, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sss.MssError) as ex:
+        sss.ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], workspace=small)
+    assert ex.value.code == sss.MSS_ERR_WORKSPACE
