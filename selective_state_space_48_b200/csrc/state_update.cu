@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p)
   const int nst = static_cast<int>(p.dstate);
   float x = ld<InT>(p.x, ch);
   float s = ld<InT>(p.dt, ch);
+  const float gate = p.z ? ld<InT>(p.z, ch) : 1.f;
+  const float skip = p.D ? p.D[d] : 0.f;
   if (p.dt_bias) s += p.dt_bias[d];
   const float step = p.softplus ? softplus_f(s) : s;
   const float sx = step * x;
@@ -46,12 +48,12 @@ __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p)
   float acc = 0.f;
   for (int n = 0; n < nst; ++n) {
     const float a = ex2_mufu(step * p.A[d * p.dstate + n] * kLog2e);
-    const float hn = fmaf(a, st[n], sx * ld<InT>(p.B, b * p.dstate + n));
-    st[n] = hn;
+    const float hn = fmaf(a, __ldcs(st + n), sx * ld<InT>(p.B, b * p.dstate + n));
+    __stcs(st + n, hn);
     acc = fmaf(ld<InT>(p.C, b * p.dstate + n), hn, acc);
   }
-  float yv = acc + (p.D ? p.D[d] : 0.f) * x;
-  if (p.z) yv *= silu_f(ld<InT>(p.z, ch));
+  float yv = fmaf(skip, x, acc);
+  if (p.z) yv *= silu_f(gate);
   reinterpret_cast<OutT *>(p.y)[ch] = from_f32<OutT>(yv);
 }
 
@@ -70,15 +72,22 @@ __global__ void __launch_bounds__(256) state_update16_kernel(const UpdateParams 
     valid = false;
   const int64_t c = valid ? ch : 0;
   const int64_t b = c / p.dim, d = c % p.dim;
-  float acc = 0.f, x = 0.f;
+  float acc = 0.f, x = 0.f, gate = 1.f, skip = 0.f;
   if (valid) {
+    // every load is issued before the arithmetic (the gate and skip inputs
+    // too, by all four threads of the channel), so no thread waits on
+    // memory twice
     x = ld<InT>(p.x, c);
     float s = ld<InT>(p.dt, c);
+    if (p.z) gate = ld<InT>(p.z, c);
+    if (p.D) skip = p.D[d];
     if (p.dt_bias) s += p.dt_bias[d];
     const float step = p.softplus ? softplus_f(s) : s;
     const float sx = step * x;
     float4 *st = reinterpret_cast<float4 *>(p.state + c * 16) + qd;
-    const float4 hv = *st;
+    // the state is read once and written once: streaming (evict-first)
+    // accesses keep it from displacing A, B and C in the caches
+    const float4 hv = __ldcs(st);
     const float4 av = reinterpret_cast<const float4 *>(p.A + d * 16)[qd];
     const float4 bv = load4_f32(static_cast<const InT *>(p.B) + b * 16 + 4 * qd);
     const float4 cv = load4_f32(static_cast<const InT *>(p.C) + b * 16 + 4 * qd);
@@ -91,13 +100,13 @@ __global__ void __launch_bounds__(256) state_update16_kernel(const UpdateParams 
       ho[j] = fmaf(a, hs[j], sx * bs[j]);
       acc = fmaf(cs[j], ho[j], acc);
     }
-    *st = make_float4(ho[0], ho[1], ho[2], ho[3]);
+    __stcs(st, make_float4(ho[0], ho[1], ho[2], ho[3]));
   }
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   if (valid && qd == 0) {
-    float yv = acc + (p.D ? p.D[d] : 0.f) * x;
-    if (p.z) yv *= silu_f(ld<InT>(p.z, c));
+    float yv = fmaf(skip, x, acc);
+    if (p.z) yv *= silu_f(gate);
     reinterpret_cast<OutT *>(p.y)[c] = from_f32<OutT>(yv);
   }
 }
