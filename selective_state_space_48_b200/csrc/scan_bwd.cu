@@ -48,6 +48,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "scan_bwd.cuh"
@@ -540,19 +541,46 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       }
     }
   };
-  // block k's recurrence from tile set T, state at its start in h2
+  // block k's recurrence from tile set T, state at its start in h2.  With
+  // packed sequences only a block with a start in it takes the masked loop
+  // (the test is uniform over the block); the ordinary kernel keeps its own
+  // copy of the loop, whose register allocation a shared generic lambda
+  // changed (0.7 % slower).
   auto fwd_block = [&](const BwdTiles<G> &T) {
+    if constexpr (VARLEN) {
+      auto run = [&](auto masked) {
 #pragma unroll
-    for (int qd = 0; qd < TB / 4; ++qd) {
-      const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
+        for (int qd = 0; qd < TB / 4; ++qd) {
+          const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]);
+          const float4 du4 = ld4(&T.du[lane * ROW + 4 * qd]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 b4 = ld4(&T.B[(4 * qd + j) * NP + 4 * g]);
-        const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
-        float2 e0 = ex2_pair(__fmul2_rn(D2, al2[0])), e1 = ex2_pair(__fmul2_rn(D2, al2[1]));
-        if (VARLEN && ((T.rmask >> (4 * qd + j)) & 1u)) e0 = e1 = make_float2(0.f, 0.f);
-        h2[0] = __ffma2_rn(e0, h2[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
-        h2[1] = __ffma2_rn(e1, h2[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+          for (int j = 0; j < 4; ++j) {
+            const float4 b4 = ld4(&T.B[(4 * qd + j) * NP + 4 * g]);
+            const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+            float2 e0 = ex2_pair(__fmul2_rn(D2, al2[0])), e1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+            if (decltype(masked)::value && ((T.rmask >> (4 * qd + j)) & 1u))
+              e0 = e1 = make_float2(0.f, 0.f);
+            h2[0] = __ffma2_rn(e0, h2[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+            h2[1] = __ffma2_rn(e1, h2[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+          }
+        }
+      };
+      if (T.rmask != 0u)
+        run(std::true_type{});
+      else
+        run(std::false_type{});
+    } else {
+#pragma unroll
+      for (int qd = 0; qd < TB / 4; ++qd) {
+        const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 b4 = ld4(&T.B[(4 * qd + j) * NP + 4 * g]);
+          const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+          float2 e0 = ex2_pair(__fmul2_rn(D2, al2[0])), e1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+          h2[0] = __ffma2_rn(e0, h2[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+          h2[1] = __ffma2_rn(e1, h2[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+        }
       }
     }
   };
@@ -674,55 +702,116 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       }
       float2 hs[2][8], as[2][8];
       float2 hh[2] = {hc[0], hc[1]};
+      if constexpr (VARLEN) {
+        // packed sequences: the masked loop only when this pass has a start
+        auto recompute = [&](auto masked) {
 #pragma unroll
-      for (int qd = 0; qd < tb / 4 + 2; ++qd) {
-        const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
-        float4 ds4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (4 * qd >= tb) ds4 = ld4(&T.ds[lane * ROW + 4 * qd]);
-        float4 sp4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        float vC[16];
+          for (int qd = 0; qd < tb / 4 + 2; ++qd) {
+            const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]);
+            const float4 du4 = ld4(&T.du[lane * ROW + 4 * qd]);
+            float4 ds4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (4 * qd >= tb) ds4 = ld4(&T.ds[lane * ROW + 4 * qd]);
+            float4 sp4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            float vC[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int t = 4 * qd + j;
-          const float4 b4 = ld4(&T.B[t * NP + 4 * g]);
-          const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
-          float2 a0 = ex2_pair(__fmul2_rn(D2, al2[0]));
-          float2 a1 = ex2_pair(__fmul2_rn(D2, al2[1]));
-          // a sequence start: nothing of the previous state survives it
-          if (VARLEN && ((T.rmask >> t) & 1u)) a0 = a1 = make_float2(0.f, 0.f);
-          hh[0] = __ffma2_rn(a0, hh[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
-          hh[1] = __ffma2_rn(a1, hh[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
-          if (t >= tb) {
-            as[0][t - tb] = a0;
-            as[1][t - tb] = a1;
-            hs[0][t - tb] = hh[0];
-            hs[1][t - tb] = hh[1];
-            const float4 c4 = ld4(&T.C[t * NP + 4 * g]);
-            float2 r = __fmul2_rn(make_float2(c4.x, c4.y), hh[0]);
-            r = __ffma2_rn(make_float2(c4.z, c4.w), hh[1], r);
-            const float sv = r.x + r.y;
-            if (j == 0) sp4.x = sv;
-            if (j == 1) sp4.y = sv;
-            if (j == 2) sp4.z = sv;
-            if (j == 3) sp4.w = sv;
-            // dC_t[n] = sum over channels of ds_t h_t[n]
-            const float2 S2 = f2(comp(ds4, j));
-            const float2 v0 = __fmul2_rn(S2, hh[0]), v1 = __fmul2_rn(S2, hh[1]);
-            vC[0 + j] = v0.x;
-            vC[4 + j] = v0.y;
-            vC[8 + j] = v1.x;
-            vC[12 + j] = v1.y;
+            for (int j = 0; j < 4; ++j) {
+              const int t = 4 * qd + j;
+              const float4 b4 = ld4(&T.B[t * NP + 4 * g]);
+              const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+              float2 a0 = ex2_pair(__fmul2_rn(D2, al2[0]));
+              float2 a1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+              // a sequence start: nothing of the previous state survives it
+              if (decltype(masked)::value && ((T.rmask >> t) & 1u))
+                a0 = a1 = make_float2(0.f, 0.f);
+              hh[0] = __ffma2_rn(a0, hh[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+              hh[1] = __ffma2_rn(a1, hh[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+              if (t >= tb) {
+                as[0][t - tb] = a0;
+                as[1][t - tb] = a1;
+                hs[0][t - tb] = hh[0];
+                hs[1][t - tb] = hh[1];
+                const float4 c4 = ld4(&T.C[t * NP + 4 * g]);
+                float2 r = __fmul2_rn(make_float2(c4.x, c4.y), hh[0]);
+                r = __ffma2_rn(make_float2(c4.z, c4.w), hh[1], r);
+                const float sv = r.x + r.y;
+                if (j == 0) sp4.x = sv;
+                if (j == 1) sp4.y = sv;
+                if (j == 2) sp4.z = sv;
+                if (j == 3) sp4.w = sv;
+                // dC_t[n] = sum over channels of ds_t h_t[n]
+                const float2 S2 = f2(comp(ds4, j));
+                const float2 v0 = __fmul2_rn(S2, hh[0]), v1 = __fmul2_rn(S2, hh[1]);
+                vC[0 + j] = v0.x;
+                vC[4 + j] = v0.y;
+                vC[8 + j] = v1.x;
+                vC[12 + j] = v1.y;
+              }
+            }
+            if (4 * qd >= tb) {
+              *reinterpret_cast<float4 *>(&s.ps[(g * CH + lane) * ROW + 4 * qd]) = sp4;
+              // channel sums of dC for states 4g + i, steps 4 qd + tq: the even
+              // lane of each pair adds j = lane >> 1 = 4 i + tq
+              const float rc = reduce_scatter16(vC, lane);
+              const int jj = lane >> 1, n = 4 * g + jj / 4, t = 4 * qd + jj % 4;
+              if ((lane & 1) == 0 && n < p.dstate && t < nt &&
+                  dbg_index_ok((b * p.dstate + n) * L + t0 + t, nBNL, p.status))
+                atomicAdd(p.dC + (b * p.dstate + n) * L + t0 + t, rc);
+            }
           }
-        }
-        if (4 * qd >= tb) {
-          *reinterpret_cast<float4 *>(&s.ps[(g * CH + lane) * ROW + 4 * qd]) = sp4;
-          // channel sums of dC for states 4g + i, steps 4 qd + tq: the even
-          // lane of each pair adds j = lane >> 1 = 4 i + tq
-          const float rc = reduce_scatter16(vC, lane);
-          const int jj = lane >> 1, n = 4 * g + jj / 4, t = 4 * qd + jj % 4;
-          if ((lane & 1) == 0 && n < p.dstate && t < nt &&
-              dbg_index_ok((b * p.dstate + n) * L + t0 + t, nBNL, p.status))
-            atomicAdd(p.dC + (b * p.dstate + n) * L + t0 + t, rc);
+        };
+        if ((T.rmask & (half ? 0xFFFFu : 0x00FFu)) != 0u)
+          recompute(std::true_type{});
+        else
+          recompute(std::false_type{});
+      } else {
+#pragma unroll
+        for (int qd = 0; qd < tb / 4 + 2; ++qd) {
+          const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
+          float4 ds4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (4 * qd >= tb) ds4 = ld4(&T.ds[lane * ROW + 4 * qd]);
+          float4 sp4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          float vC[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int t = 4 * qd + j;
+            const float4 b4 = ld4(&T.B[t * NP + 4 * g]);
+            const float2 D2 = f2(comp(dl4, j)), U2 = f2(comp(du4, j));
+            float2 a0 = ex2_pair(__fmul2_rn(D2, al2[0]));
+            float2 a1 = ex2_pair(__fmul2_rn(D2, al2[1]));
+            hh[0] = __ffma2_rn(a0, hh[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
+            hh[1] = __ffma2_rn(a1, hh[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
+            if (t >= tb) {
+              as[0][t - tb] = a0;
+              as[1][t - tb] = a1;
+              hs[0][t - tb] = hh[0];
+              hs[1][t - tb] = hh[1];
+              const float4 c4 = ld4(&T.C[t * NP + 4 * g]);
+              float2 r = __fmul2_rn(make_float2(c4.x, c4.y), hh[0]);
+              r = __ffma2_rn(make_float2(c4.z, c4.w), hh[1], r);
+              const float sv = r.x + r.y;
+              if (j == 0) sp4.x = sv;
+              if (j == 1) sp4.y = sv;
+              if (j == 2) sp4.z = sv;
+              if (j == 3) sp4.w = sv;
+              // dC_t[n] = sum over channels of ds_t h_t[n]
+              const float2 S2 = f2(comp(ds4, j));
+              const float2 v0 = __fmul2_rn(S2, hh[0]), v1 = __fmul2_rn(S2, hh[1]);
+              vC[0 + j] = v0.x;
+              vC[4 + j] = v0.y;
+              vC[8 + j] = v1.x;
+              vC[12 + j] = v1.y;
+            }
+          }
+          if (4 * qd >= tb) {
+            *reinterpret_cast<float4 *>(&s.ps[(g * CH + lane) * ROW + 4 * qd]) = sp4;
+            // channel sums of dC for states 4g + i, steps 4 qd + tq: the even
+            // lane of each pair adds j = lane >> 1 = 4 i + tq
+            const float rc = reduce_scatter16(vC, lane);
+            const int jj = lane >> 1, n = 4 * g + jj / 4, t = 4 * qd + jj % 4;
+            if ((lane & 1) == 0 && n < p.dstate && t < nt &&
+                dbg_index_ok((b * p.dstate + n) * L + t0 + t, nBNL, p.status))
+              atomicAdd(p.dC + (b * p.dstate + n) * L + t0 + t, rc);
+          }
         }
       }
 
