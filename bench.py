@@ -93,7 +93,7 @@ def parse_args(argv=None):
                     choices=[w.name for w in workloads.SSD_WORKLOADS])
     ap.add_argument("--decode-batch", type=int, default=1024,
                     help="batch rows of one decode step (the workload's dim and dstate)")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -912,6 +912,27 @@ def run_ours(args, rank, world, local_rank):
     barrier(world)
     e2e_ms = reduce_max(e0.elapsed_time(e1), world)
     e2e_value = whole_job_gbs(bytes_step, Ke, world, e2e_ms)
+    # the link's own bound for the same bytes: the step's uploads and its
+    # read-back as plain copies, both directions at once, no scan
+    def copies_only():
+        s_up.wait_stream(stream)
+        s_dn.wait_stream(stream)
+        with torch.cuda.stream(s_up):
+            for k, t in host.items():
+                sets[1][k].copy_(t, non_blocking=True)
+        with torch.cuda.stream(s_dn):
+            y_host[1].copy_(ys[1], non_blocking=True)
+        stream.wait_stream(s_up)
+        stream.wait_stream(s_dn)
+    copies_only()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(3):
+        copies_only()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    link_ms = reduce_max(e0.elapsed_time(e1), world) / 3
+    link_value = whole_job_gbs(bytes_step, 1, world, link_ms)
     del sets[1], ys[1]
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
@@ -996,7 +1017,10 @@ def run_ours(args, rank, world, local_rank):
         "exp_unit": exp_unit_bound(w, max_kernel_ms, sm_mhz),
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke,
-                "overlap": "upload of step i+1 and read-back of step i-1 during the scan of step i"},
+                "overlap": "upload of step i+1 and read-back of step i-1 during the scan of step i",
+                "link_bound": {"value": link_value, "unit": "GB/s",
+                               "what": "the same uploads and read-back as plain pinned copies, "
+                                       "both directions at once, no scan"}},
         "gpu_launches": K * launches_per_step,
         "launches_per_step": launches_per_step,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
