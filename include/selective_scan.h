@@ -326,8 +326,9 @@ typedef struct mss_scan_bwd_args {
      forward sweep and needs no workspace. */
   const float *checkpoints;
   void *workspace;          /* device, >= mss_scan_bwd_workspace_size(),
-                               256-byte aligned; may be NULL with
-                               checkpoints */
+                               256-byte aligned, not shared with a call in
+                               flight; may be NULL with checkpoints (no
+                               cut schedule then) */
   size_t workspace_bytes;
   /* element strides {batch, row} of u, delta, z, B, C and dy, with the
      same meaning and rules as the input strides of mss_scan_args ({0, 0}:
@@ -344,8 +345,17 @@ typedef struct mss_scan_bwd_args {
   int64_t num_seqs;
 } mss_scan_bwd_args;
 
-/* Workspace bytes of the backward scan (the state checkpoints: 64 bytes per
- * 16 steps of every channel, for dstate <= 16). */
+/* Workspace bytes of the backward scan: the state checkpoints (64 bytes per
+ * 16 steps of every channel, for dstate <= 16; none when `checkpoints` is
+ * given), then the area of the cut schedule when it applies on the current
+ * device.  A launch of batch * ceil(dim / 32) blocks whose last wave of
+ * resident blocks is at most half full cuts the tiles of that wave in two
+ * at their middle 16-step block: the first part's forward sweep, the second
+ * part's sweeps and the first part's reverse sweep run as separate work
+ * items (taken by ticket, spread over the schedule), handing the state and
+ * the adjoint over through the workspace; du, ddelta and dz are
+ * bit-identical to the uncut schedule.  A workspace with the checkpoints
+ * but not that area runs every tile whole.  Packed sequences are not cut. */
 mss_status mss_scan_bwd_workspace_size(const mss_scan_bwd_args *args, size_t *bytes);
 
 /* Backward selective scan on `stream`; argument errors return before any

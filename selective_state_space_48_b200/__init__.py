@@ -583,8 +583,11 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     rc = lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n))
     if rc != MSS_OK:
         raise MssError(rc, "mss_scan_bwd_workspace_size")
-    if workspace is None and checkpoints is None:
+    if workspace is None:
+        # the checkpoints (without given ones) and the cut schedule's area
         workspace = alloc_workspace(int(n.value), dev)
+    if workspace is False:  # no workspace (valid with checkpoints): no cut
+        workspace = None
     if workspace is not None:
         a.workspace = workspace.data_ptr()
         a.workspace_bytes = workspace.numel() * workspace.element_size()

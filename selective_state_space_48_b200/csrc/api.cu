@@ -394,23 +394,42 @@ mss_status check_bwd_args(const mss_scan_bwd_args *a) {
 
 extern "C" {
 
+// The backward's cut schedule for these arguments on the current device.
+static BwdCut bwd_cut_of(const mss_scan_bwd_args *a) {
+  BwdParams q{};
+  q.seqlen = a->seqlen;
+  q.dstate = a->dstate;
+  q.tiles = a->batch * ((a->dim + kBwdChannels - 1) / kBwdChannels);
+  q.ckpt_given = a->checkpoints ? 1 : 0;
+  q.cu = a->cu_seqlens;
+  return plan_bwd_cut(q, a->in_dtype == MSS_BF16);
+}
+
 mss_status mss_scan_bwd_workspace_size(const mss_scan_bwd_args *a, size_t *bytes) {
   if (!bytes) return MSS_ERR_INVALID_ARG;
   const mss_status st = check_bwd_args(a);
   if (st != MSS_OK) return st;
   const int64_t tiles = a->batch * ((a->dim + kBwdChannels - 1) / kBwdChannels);
-  *bytes = scan_bwd_workspace_bytes(tiles, a->seqlen, a->dstate);
+  *bytes = (a->checkpoints ? 0 : scan_bwd_workspace_bytes(tiles, a->seqlen, a->dstate)) +
+           bwd_cut_of(a).bytes;
   return MSS_OK;
 }
 
 mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   NvtxRange range("mamba_selective_scan_bwd");
-  size_t need = 0;
-  const mss_status st = mss_scan_bwd_workspace_size(a, &need);
+  const mss_status st = check_bwd_args(a);
   if (st != MSS_OK) return st;
+  const int64_t ntiles = a->batch * ((a->dim + kBwdChannels - 1) / kBwdChannels);
+  const size_t ck_bytes =
+      a->checkpoints ? 0 : scan_bwd_workspace_bytes(ntiles, a->seqlen, a->dstate);
   if (!a->checkpoints &&
-      (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256)))
+      (!a->workspace || a->workspace_bytes < ck_bytes || !aligned(a->workspace, 256)))
     return MSS_ERR_WORKSPACE;
+  // the cut schedule runs when the workspace also holds its area (after the
+  // checkpoints); otherwise every tile runs whole
+  BwdCut cut = bwd_cut_of(a);
+  if (!a->workspace || !aligned(a->workspace, 256) || a->workspace_bytes < ck_bytes + cut.bytes)
+    cut = BwdCut();
   BwdParams p{};
   p.batch = a->batch;
   p.dim = a->dim;
@@ -457,6 +476,21 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   p.status = scan_status_word();
   if (!p.status) return MSS_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  p.ncut = cut.ncut;
+  p.kcut = cut.kcut;
+  p.gap0 = cut.gap0;
+  p.gap1 = cut.gap1;
+  if (cut.ncut) {
+    unsigned char *area = static_cast<unsigned char *>(a->workspace) + ck_bytes;
+    p.ticket = reinterpret_cast<unsigned *>(area);
+    p.flag = reinterpret_cast<unsigned *>(area + 256);
+    p.lam = reinterpret_cast<float *>(area + 256 + ((8 * static_cast<size_t>(cut.ncut) + 255) /
+                                                    256) * 256);
+    // the ticket and the flags start at zero on every call
+    if (cudaMemsetAsync(area, 0, reinterpret_cast<unsigned char *>(p.lam) - area, s) !=
+        cudaSuccess)
+      return MSS_ERR_CUDA;
+  }
   // the gradients that are sums over blocks are accumulated with atomics
   const size_t f = sizeof(float);
   const size_t nBC = static_cast<size_t>(a->batch * a->dstate * a->seqlen) * f;

@@ -177,7 +177,59 @@ __device__ unsigned restart_mask(const BwdParams &p, int64_t t0, int64_t L, int6
   return m;
 }
 
-template <typename InT, int G, bool VARLEN>
+// Work item of a block under the cut schedule: tile and blocks [kb0, kb1),
+// piece -1 (a whole tile), 0 (the first part's forward sweep), 1 (the
+// second part: its forward sweep unless the checkpoints are given, and its
+// reverse sweep) or 2 (the first part's reverse sweep), of cut tile si.
+// Items in ticket order: the first pieces of the cut tiles, gap0 whole
+// tiles, the next pieces, gap1 whole tiles, the last pieces.
+struct BwdWork {
+  int64_t tile;
+  int kb0, kb1, piece, si;
+};
+
+__device__ BwdWork bwd_work(int64_t item, const BwdParams &p, int nblk) {
+  BwdWork w{item, 0, nblk, -1, 0};
+  const int64_t F = p.tiles - p.ncut;  // whole tiles
+  const int first = p.ckpt_given ? 1 : 0;
+  int64_t pos = item, full = 0;
+  for (int j = first; j < 3; ++j) {
+    if (pos < p.ncut) {
+      w.si = static_cast<int>(pos);
+      w.tile = F + w.si;
+      w.piece = j;
+      w.kb0 = j == 1 ? p.kcut : 0;
+      w.kb1 = j == 1 ? nblk : p.kcut;
+      return w;
+    }
+    pos -= p.ncut;
+    if (j < 2) {
+      const int64_t gs = j == first ? p.gap0 : p.gap1;
+      if (pos < gs) {
+        w.tile = full + pos;
+        return w;
+      }
+      pos -= gs;
+      full += gs;
+    }
+  }
+  return w;  // not reached: the grid has F + (3 - first) * ncut items
+}
+
+// one thread waits (bounded) for a flag another block releases
+__device__ void wait_flag(const unsigned *f, unsigned *status) {
+  const uint64_t start = global_timer_ns();
+  while (ld_acquire_gpu(f) == 0u) {
+    if (global_timer_ns() - start > 2000000000ull) {
+      atomicOr(status, kStatusTimeout);
+      break;
+    }
+    __nanosleep(256);
+  }
+  __threadfence();
+}
+
+template <typename InT, int G, bool VARLEN, bool CUT>
 __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     scan_bwd_kernel(const BwdParams p) {
   using Sm = BwdSmem<G>;
@@ -187,13 +239,21 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   Sm &s = *reinterpret_cast<Sm *>(smem_raw);
 
   const int tid = threadIdx.x, lane = tid & 31, g = tid >> 5;
-  const int64_t tile = blockIdx.x;
+  const int64_t L = p.seqlen;
+  const int nblk = static_cast<int>((L + TB - 1) / TB);
+  // the block's work: a whole tile, or with the cut schedule a ticket's item
+  __shared__ int64_t s_item;
+  if (CUT) {
+    if (tid == 0) s_item = atomicAdd(p.ticket, 1u);
+    __syncthreads();
+  }
+  const BwdWork wk = CUT ? bwd_work(s_item, p, nblk) : BwdWork{blockIdx.x, 0, nblk, -1, 0};
+  const int kb0 = wk.kb0, kb1 = wk.kb1;
+  const int64_t tile = wk.tile;
   const int64_t b = tile / p.ch_tiles;
   const int64_t d0 = (tile % p.ch_tiles) * CH;
   const int64_t d = d0 + lane;
   const bool dvalid = d < p.dim;
-  const int64_t L = p.seqlen;
-  const int nblk = static_cast<int>((L + TB - 1) / TB);
 
   // tensor sizes for the bounds checks of the checked build
   const int64_t nBDL = p.batch * p.dim * L, nBNL = p.batch * p.dstate * L;
@@ -234,6 +294,16 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   // state 4g + i of lane at the start of block k:
   // ckpt[(k * NP + 4g + i) * CH + lane] (coalesced per warp)
   float *ckpt = p.ckpt + tile * static_cast<int64_t>(nblk) * NP * CH;
+  // a second part with its own forward sweep starts from the state the
+  // first part's sweep left at block kb0
+  if (CUT && wk.piece == 1 && !p.ckpt_given) {
+    if (tid == 0) wait_flag(p.flag + wk.si, p.status);
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      h2[q] = make_float2(__ldcg(&ckpt[(static_cast<int64_t>(kb0) * NP + 4 * g + 2 * q) * CH + lane]),
+                          __ldcg(&ckpt[(static_cast<int64_t>(kb0) * NP + 4 * g + 2 * q + 1) * CH + lane]));
+  }
 
   // The reverse sweep reads block k - 1 from HBM into registers while block
   // k's earlier half is computed and writes it to the other tile set right
@@ -591,14 +661,15 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       ckpt[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q + 1) * CH + lane] = h2[q].y;
     }
   };
-  if (!p.ckpt_given && kStaged) {
-    fstage_fetch(0, 0);
+  const bool sweep = !p.ckpt_given && wk.piece != 2;
+  if (sweep && kStaged) {
+    fstage_fetch(kb0, kb0 & 1);
     cp_async_wait_all();
     __syncthreads();
-    fstage_commit(0, 0, s.tl[0]);
-    put_mask(0, s.tl[0]);
-    if (nblk > 1) fstage_fetch(1, 1);
-    for (int k = 0; k < nblk; ++k) {
+    fstage_commit(kb0, kb0 & 1, s.tl[kb0 & 1]);
+    put_mask(kb0, s.tl[kb0 & 1]);
+    if (kb0 + 1 < kb1) fstage_fetch(kb0 + 1, (kb0 + 1) & 1);
+    for (int k = kb0; k < kb1; ++k) {
       put_ckpt(k);
       // block k + 1's copies (this thread's) have landed; after the barrier
       // every thread's have, and block k's tiles are committed
@@ -606,29 +677,38 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       __syncthreads();
       // area k & 1 held block k, committed before the barrier; tile set
       // (k + 1) & 1 was last read by block k - 1, finished before it
-      if (k + 2 < nblk) fstage_fetch(k + 2, k & 1);
-      if (k + 1 < nblk) {
+      if (k + 2 < kb1) fstage_fetch(k + 2, k & 1);
+      if (k + 1 < kb1) {
         fstage_commit(k + 1, (k + 1) & 1, s.tl[(k + 1) & 1]);
         put_mask(k + 1, s.tl[(k + 1) & 1]);
       }
       fwd_block(s.tl[k & 1]);
     }
     __syncthreads();
-  } else if (!p.ckpt_given) {
+  } else if (sweep) {
     RawF rf;
-    fetch_fwd(0, rf);
-    for (int k = 0; k < nblk; ++k) {
+    fetch_fwd(kb0, rf);
+    for (int k = kb0; k < kb1; ++k) {
       BwdTiles<G> &T = s.tl[k & 1];
       commit_fwd(rf, T);
       put_mask(k, T);
       put_ckpt(k);
       __syncthreads();
-      if (k + 1 < nblk) fetch_fwd(k + 1, rf);  // in flight while block k is computed
+      if (k + 1 < kb1) fetch_fwd(k + 1, rf);  // in flight while block k is computed
       fwd_block(T);
       // no barrier here: block k + 1 is committed to the other tile set, and
       // this set is next written two blocks on, after the next barrier
     }
     __syncthreads();
+  }
+  if (CUT && wk.piece == 0) {
+    // the first part's sweep ends here: its end state is the checkpoint of
+    // block kb1, published for the second part
+    put_ckpt(kb1);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release_gpu(p.flag + wk.si, 1u);
+    return;
   }
 
   // ------------------------------------------------------ reverse sweep
@@ -645,24 +725,41 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     lam[q] = make_float2(lv[0], lv[1]);
     dA2[q] = make_float2(0.f, 0.f);
   }
+  // the first part's reverse sweep starts from the adjoint the second part
+  // left at its first block
+  if (CUT && wk.piece == 2) {
+    if (tid == 0) wait_flag(p.flag + p.ncut + wk.si, p.status);
+    __syncthreads();
+    const float *lr = p.lam + static_cast<int64_t>(wk.si) * NP * CH;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float lv[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {  // written only for live (channel, state)
+        const int n = 4 * g + 2 * q + e;
+        lv[e] = (dvalid && n < p.dstate) ? __ldcg(&lr[n * CH + lane]) : 0.f;
+      }
+      lam[q] = make_float2(lv[0], lv[1]);
+    }
+  }
   // the checkpoint of the block after the current one is read a block early
   float2 hnext[2];
 #pragma unroll
   for (int q = 0; q < 2; ++q)
     hnext[q] = make_float2(
-        ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q) * CH + lane],
-        ckpt[(static_cast<int64_t>(nblk - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
+        ckpt[(static_cast<int64_t>(kb1 - 1) * NP + 4 * g + 2 * q) * CH + lane],
+        ckpt[(static_cast<int64_t>(kb1 - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
   Raw raw;
   if (kStaged) {
-    stage_fetch(nblk - 1);
+    stage_fetch(kb1 - 1);
     cp_async_wait_all();
     __syncthreads();
-    stage_commit(nblk - 1, s.tl[(nblk - 1) & 1]);
-    put_mask(nblk - 1, s.tl[(nblk - 1) & 1]);
+    stage_commit(kb1 - 1, s.tl[(kb1 - 1) & 1]);
+    put_mask(kb1 - 1, s.tl[(kb1 - 1) & 1]);
   } else {
-    fetch(nblk - 1, raw);
-    commit(raw, s.tl[(nblk - 1) & 1]);
-    put_mask(nblk - 1, s.tl[(nblk - 1) & 1]);
+    fetch(kb1 - 1, raw);
+    commit(raw, s.tl[(kb1 - 1) & 1]);
+    put_mask(kb1 - 1, s.tl[(kb1 - 1) & 1]);
   }
   // this thread's shares of the per-channel sums (in registers when a
   // thread has few elements; otherwise added to shared memory per block)
@@ -671,7 +768,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   float accD[EA], accB[EA];
 #pragma unroll
   for (int e = 0; e < EA; ++e) accD[e] = accB[e] = 0.f;
-  for (int k = nblk - 1; k >= 0; --k) {
+  for (int k = kb1 - 1; k >= kb0; --k) {
     const int64_t t0 = static_cast<int64_t>(k) * TB;
     const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
     BwdTiles<G> &T = s.tl[k & 1];
@@ -679,7 +776,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       hc[q] = hnext[q];
-      if (k > 0)
+      if (k > kb0)
         hnext[q] = make_float2(
             ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q) * CH + lane],
             ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
@@ -694,7 +791,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     for (int half = 1; half >= 0; --half) {
       const int tb = 8 * half;  // first step of this half
       // block k-1's inputs: in flight while the earlier half is computed
-      if (half == 0 && k > 0) {
+      if (half == 0 && k > kb0) {
         if (kStaged)
           stage_fetch(k - 1);
         else
@@ -864,7 +961,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       }
       // block k-1 into the other tile set, which is free: block k+1's
       // epilogue ended before this block's barrier
-      if (!kStaged && half == 0 && k > 0) {
+      if (!kStaged && half == 0 && k > kb0) {
         commit(raw, s.tl[(k - 1) & 1]);
         put_mask(k - 1, s.tl[(k - 1) & 1]);
       }
@@ -873,7 +970,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     __syncthreads();
     // staged inputs: block k-1 into the other tile set once every copy has
     // landed (the staging area is refilled only after the next barrier)
-    if (kStaged && k > 0) {
+    if (kStaged && k > kb0) {
       stage_commit(k - 1, s.tl[(k - 1) & 1]);
       put_mask(k - 1, s.tl[(k - 1) & 1]);
     }
@@ -932,8 +1029,17 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       const int n = 4 * g + 2 * q + e;
       if (!dvalid || n >= p.dstate) continue;
       atomicAdd(p.dA + d * p.dstate + n, e == 0 ? dA2[q].x : dA2[q].y);
-      if (p.dh0) p.dh0[(b * p.dim + d) * p.dstate + n] = e == 0 ? lam[q].x : lam[q].y;
+      if (CUT && wk.piece == 1)  // the adjoint handed to the first part
+        p.lam[static_cast<int64_t>(wk.si) * NP * CH + (4 * g + 2 * q + e) * CH + lane] =
+            e == 0 ? lam[q].x : lam[q].y;
+      else if (p.dh0)
+        p.dh0[(b * p.dim + d) * p.dstate + n] = e == 0 ? lam[q].x : lam[q].y;
     }
+  }
+  if (CUT && wk.piece == 1) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release_gpu(p.flag + p.ncut + wk.si, 1u);
   }
   if (tid < CH && d0 + tid < p.dim) {
     if (p.dD) atomicAdd(p.dD + d0 + tid, s.accD[tid]);
@@ -941,14 +1047,47 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   }
 }
 
-template <typename InT, int G, bool VARLEN>
-cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
-  auto kern = scan_bwd_kernel<InT, G, VARLEN>;
+template <typename InT, int G, bool VARLEN, bool CUT>
+cudaError_t launch_kernel(const BwdParams &p, cudaStream_t stream) {
+  auto kern = scan_bwd_kernel<InT, G, VARLEN, CUT>;
   const int smem = static_cast<int>(sizeof(BwdSmem<G>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(p.tiles), 32 * G, smem, stream>>>(p);
+  // items: the whole tiles, and two or three pieces of every cut tile
+  const int64_t items = p.tiles + (CUT ? (p.ckpt_given ? 1 : 2) * static_cast<int64_t>(p.ncut) : 0);
+  kern<<<static_cast<unsigned>(items), 32 * G, smem, stream>>>(p);
   return cudaGetLastError();
+}
+
+// The cut schedule has its own instantiation (ordinary scans only), so the
+// kernel of whole tiles keeps its code.
+template <typename InT, int G, bool VARLEN>
+cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
+  if constexpr (!VARLEN) {
+    if (p.ncut) return launch_kernel<InT, G, false, true>(p, stream);
+  }
+  return launch_kernel<InT, G, VARLEN, false>(p, stream);
+}
+
+template <typename InT, int G>
+int blocks_per_sm() {
+  int n = 0;
+  const int smem = static_cast<int>(sizeof(BwdSmem<G>));
+  auto kern = scan_bwd_kernel<InT, G, false, false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * G, smem) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+template <typename InT>
+int blocks_per_sm_g(int groups) {
+  switch (groups) {
+    case 1: return blocks_per_sm<InT, 1>();
+    case 2: return blocks_per_sm<InT, 2>();
+    default: return blocks_per_sm<InT, 4>();
+  }
 }
 
 // Packed sequences get their own instantiation, so their code never
@@ -985,6 +1124,41 @@ size_t scan_bwd_workspace_bytes(int64_t tiles, int64_t seqlen, int64_t dstate) {
 
 cudaError_t launch_scan_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream) {
   return in_bf16 ? dispatch<__nv_bfloat16>(p, stream) : dispatch<float>(p, stream);
+}
+
+// A launch of `tiles` blocks fills W full waves of the resident slots and a
+// last wave of r blocks.  When that wave is at most half full (and a tile
+// has two 16-step blocks or more), the last r tiles are cut in two at their
+// middle block: the first part's forward sweep, the second part's sweeps
+// and the first part's reverse sweep become separate work items, with half
+// of the whole tiles between the first two and the rest between the last
+// two (with checkpoints: the second part, every whole tile, the first
+// part).  Packed sequences are not cut.
+BwdCut plan_bwd_cut(const BwdParams &p, int in_bf16) {
+  BwdCut c;
+  const int nblk = static_cast<int>((p.seqlen + kBwdTimeBlock - 1) / kBwdTimeBlock);
+  if (p.cu || nblk < 2) return c;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();  // no device: nothing is cut
+    return c;
+  }
+  const int G = bwd_groups(p.dstate);
+  const int per_sm = in_bf16 ? blocks_per_sm_g<__nv_bfloat16>(G) : blocks_per_sm_g<float>(G);
+  const int64_t slots = static_cast<int64_t>(sms) * per_sm;
+  if (slots < 1) return c;
+  const int64_t W = p.tiles / slots, r = p.tiles % slots;
+  if (W < 1 || r < 1 || 2 * r > slots) return c;
+  c.ncut = static_cast<int>(r);
+  c.kcut = nblk / 2;
+  const int64_t F = p.tiles - r;
+  c.gap0 = p.ckpt_given ? F : F / 2;
+  c.gap1 = p.ckpt_given ? 0 : F - F / 2;
+  const size_t NPc = static_cast<size_t>(4 * G);
+  c.bytes = 256 + ((8 * static_cast<size_t>(r) + 255) / 256) * 256 +
+            static_cast<size_t>(r) * NPc * kBwdChannels * sizeof(float);
+  return c;
 }
 
 }  // namespace sss48

@@ -38,7 +38,26 @@ struct BwdParams {
   // cu[1 .. nseq-1] start a sequence with an empty state
   const int32_t *cu;
   int64_t nseq;
+  // cut schedule (ncut == 0: one block per tile in blockIdx order).  The
+  // last ncut tiles are cut after block kcut into work items taken by
+  // ticket: the first part's forward sweep (no item when the checkpoints
+  // are given), the second part's sweeps, the first part's reverse sweep,
+  // with gap0 whole tiles after the first of them and gap1 after the second
+  int ncut, kcut;
+  int64_t gap0, gap1;
+  unsigned *ticket;
+  unsigned *flag;  // [2][ncut]: first part's states written, second part's adjoint written
+  float *lam;      // [ncut][4 * groups][32]: the adjoint entering the second part
 };
+
+// The cut schedule of a launch: how many tiles are cut, where, and the
+// workspace it needs beyond the checkpoints (0 bytes: nothing is cut).
+struct BwdCut {
+  int ncut = 0, kcut = 0;
+  int64_t gap0 = 0, gap1 = 0;
+  size_t bytes = 0;
+};
+BwdCut plan_bwd_cut(const BwdParams &p, int in_bf16);
 
 // Warps per block (state groups of 4): 1, 2 or 4.
 int bwd_groups(int64_t dstate);

@@ -216,3 +216,69 @@ def test_packed_backward_rejects_checkpoints():
         sss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy,
                                cu_seqlens=cu_t, checkpoints=ck)
     assert ei.value.code == sss.MSS_ERR_UNSUPPORTED
+
+
+def _bwd_ws(inp, dy, d_last, workspace, checkpoints=None):
+    g = sss.selective_scan_bwd(
+        inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"],
+        z=inp["z"], delta_bias=inp["delta_bias"], h0=inp["h0"], d_last=d_last,
+        workspace=workspace, checkpoints=checkpoints)
+    torch.cuda.synchronize()
+    return g
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_backward_cut_schedule(dt):
+    """More tiles than one wave of resident blocks and a last wave at most
+    half full: the last wave's tiles are cut at their middle block into work
+    items that hand the state and the adjoint over through the workspace.
+    du, ddelta, dz and dh0 are bit-identical to the run with every tile
+    whole (a workspace of the checkpoints only), from the backward's own
+    forward sweep and from the forward scan's checkpoints; the atomic sums
+    agree to fp32 rounding; and a row of the cut tiles matches the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # 3 resident blocks per SM (4 warps, 168 registers): one wave of slots
+    # plus 16 more 32-channel tiles, in one batch row
+    dim = 32 * (3 * sms + 16)
+    w = workloads.custom(1, dim, 16, 100, in_dtype=dt, has_z=True, a_noise=0.1)
+    inp = workloads.make_inputs(w, seed=5900, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5901)
+    inp["h0"] = torch.randn(1, dim, 16, generator=gen, device="cuda")
+    dy = torch.randn(1, dim, 100, generator=gen, device="cuda")
+    d_last = torch.randn(1, dim, 16, generator=gen, device="cuda")
+    ck_bytes = sss.scan_checkpoints(1, dim, 16, 100, "cpu").numel() * 4
+    whole_ws = torch.empty(ck_bytes, dtype=torch.uint8, device="cuda")
+    g_whole = _bwd_ws(inp, dy, d_last, whole_ws)
+    g_cut = _bwd_ws(inp, dy, d_last, None)   # allocates checkpoints + cut area
+    exact = ("du", "ddelta", "dz", "dh0")
+    for k in exact:
+        assert torch.equal(g_cut[k], g_whole[k]), k
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        assert norm_err(g_cut[k].cpu().numpy(), g_whole[k].double().cpu().numpy()) <= 1e-5, k
+    # from the forward scan's checkpoints: cut (workspace) against whole (none)
+    ck = sss.scan_checkpoints(1, dim, 16, 100, "cuda")
+    sss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                           z=inp["z"], delta_bias=inp["delta_bias"], h0=inp["h0"],
+                           checkpoints=ck)
+    g_ck_whole = _bwd_ws(inp, dy, d_last, False, checkpoints=ck)
+    g_ck_cut = _bwd_ws(inp, dy, d_last, None, checkpoints=ck)
+    for k in exact:
+        assert torch.equal(g_ck_cut[k], g_ck_whole[k]), k
+        assert torch.equal(g_ck_cut[k], g_whole[k]), k
+    # the cut tiles (the last 16) against the oracle: their channels only
+    c0 = dim - 32 * 16
+    sub = {k: (v[:, c0:] if v is not None and v.dim() == 3 else v) for k, v in inp.items()}
+    sub["A"] = inp["A"][c0:]
+    for k in ("D", "delta_bias"):
+        sub[k] = inp[k][c0:] if inp[k] is not None else None
+    sub["B"], sub["C"] = inp["B"], inp["C"]
+    h = workloads.to_numpy_f64(sub)
+    g_ref = oracle.selective_scan_bwd(
+        h["u"], h["delta"], h["A"], h["B"], h["C"], dy[:, c0:].double().cpu().numpy(),
+        D=h["D"], z=h["z"], delta_bias=h["delta_bias"], delta_softplus=True, h0=h["h0"],
+        d_last=d_last[:, c0:].double().cpu().numpy())
+    for k in ("du", "ddelta", "dz", "dh0"):
+        assert norm_err(g_cut[k][:, c0:].cpu().numpy(), g_ref[k]) <= TOL, k
+    for k in ("dA", "dD", "ddelta_bias"):
+        assert norm_err(g_cut[k][c0:].cpu().numpy(), g_ref[k]) <= TOL, k
