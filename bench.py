@@ -668,7 +668,9 @@ def run_decode(args, rank, world, local_rank):
         "tokens_per_s": bt * K * world / (max_ms * 1e-3),
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak,
                      "unit": "GB/s", "frac": value / world / peak,
-                     "peak_source": src, "traffic": None,
+                     "peak_source": src,
+                     "traffic": (profiled_traffic(f"{w.name}-{bt}rows", "decode")
+                                 if bt == 1024 else None),
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": None, "gpu_launches": K, "clocks": clocks.summary(),
         "kernel_source_hash": kernel_source_hash("decode"),

@@ -58,20 +58,23 @@ __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p)
 }
 
 // 16 states with the state, A, B and C 16-byte aligned: thread 4 ch + qd
-// owns states 4 qd .. 4 qd + 3 of channel ch.
-template <typename InT, typename OutT>
+// owns states 4 qd .. 4 qd + 3 of channel ch.  Idx is the index type: 32
+// bits when every state index fits (a 64-bit division per thread is a long
+// instruction sequence; the kernel is bound by issue, not by DRAM).
+template <typename InT, typename OutT, typename Idx>
 __global__ void __launch_bounds__(256) state_update16_kernel(const UpdateParams p) {
-  const int64_t gt = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  const int64_t ch = gt >> 2;
+  const Idx gt = static_cast<Idx>(blockIdx.x) * static_cast<Idx>(blockDim.x) + threadIdx.x;
+  const Idx ch = gt >> 2;
   const int qd = static_cast<int>(gt & 3);
+  const Idx dim = static_cast<Idx>(p.dim);
   // every thread of a channel takes part in the shuffles below
-  bool valid = ch < p.batch * p.dim;
+  bool valid = static_cast<int64_t>(ch) < p.batch * p.dim;
   if (valid && (!dbg_index_ok((ch + 1) * 16 - 1, p.batch * p.dim * 16, p.status) ||
                 !dbg_index_ok((ch % p.dim + 1) * 16 - 1, p.dim * 16, p.status) ||
                 !dbg_index_ok((ch / p.dim + 1) * 16 - 1, p.batch * 16, p.status)))
     valid = false;
-  const int64_t c = valid ? ch : 0;
-  const int64_t b = c / p.dim, d = c % p.dim;
+  const Idx c = valid ? ch : 0;
+  const Idx b = c / dim, d = c - b * dim;
   float acc = 0.f, x = 0.f, gate = 1.f, skip = 0.f;
   if (valid) {
     // every load is issued before the arithmetic (the gate and skip inputs
@@ -119,7 +122,12 @@ cudaError_t launch_typed(const UpdateParams &p, cudaStream_t s) {
   if (p.dstate == 16 && aligned16(p.state) && aligned16(p.A) && aligned16(p.B) &&
       aligned16(p.C)) {
     const unsigned grid = static_cast<unsigned>((4 * n + 255) / 256);
-    state_update16_kernel<InT, OutT><<<grid, 256, 0, s>>>(p);
+    // 32-bit indices when the largest state index (16 n) and the thread
+    // count (4 n, rounded up to the block) fit
+    if (16 * n + 256 <= static_cast<int64_t>(UINT32_MAX))
+      state_update16_kernel<InT, OutT, uint32_t><<<grid, 256, 0, s>>>(p);
+    else
+      state_update16_kernel<InT, OutT, int64_t><<<grid, 256, 0, s>>>(p);
   } else {
     const unsigned grid = static_cast<unsigned>((n + 127) / 128);
     state_update_kernel<InT, OutT><<<grid, 128, 0, s>>>(p);
