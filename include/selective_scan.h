@@ -355,7 +355,10 @@ typedef struct mss_scan_bwd_args {
  * items (taken by ticket, spread over the schedule), handing the state and
  * the adjoint over through the workspace; du, ddelta and dz are
  * bit-identical to the uncut schedule.  A workspace with the checkpoints
- * but not that area runs every tile whole.  Packed sequences are not cut. */
+ * but not that area runs every tile whole.  Packed sequences are not cut.
+ * A hand-over wait is bounded (2 s); one that runs out records a timeout in
+ * the library's own status word (reported by mss_scan_status for an
+ * unsplit scan's arguments). */
 mss_status mss_scan_bwd_workspace_size(const mss_scan_bwd_args *args, size_t *bytes);
 
 /* Backward selective scan on `stream`; argument errors return before any

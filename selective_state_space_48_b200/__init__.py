@@ -528,8 +528,12 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     Inputs as for ``selective_scan_fwd`` (u, delta, z, B, C and dy may be
     3-d views with a contiguous last dimension); dy (batch, dim, L) and
     d_last (batch, dim, N) float32.  ``checkpoints`` written by the forward
-    scan of the same inputs let the backward skip its forward sweep.  Returns a dict of float32 tensors du,
-    ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0 (None for absent inputs).
+    scan of the same inputs let the backward skip its forward sweep.
+    ``workspace``: None allocates what ``mss_scan_bwd_workspace_size`` asks
+    for (the checkpoints and the cut schedule's area); False passes none
+    (valid with ``checkpoints``; every tile then runs whole); a uint8 CUDA
+    tensor is used as given.  Returns a dict of float32 tensors du, ddelta,
+    dA, dB, dC, dD, dz, ddelta_bias, dh0 (None for absent inputs).
     """
     batch, dim, L = u.shape
     N = A.shape[1]
