@@ -8,6 +8,8 @@ as max |g_gpu - g_ref| / max |g_ref| per tensor.  Both sides do the same
 arithmetic; the GPU does it in fp32 with atomic sums over channels and
 batch rows, hence the fp32-level bound.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -282,3 +284,39 @@ def test_backward_cut_schedule(dt):
         assert norm_err(g_cut[k][:, c0:].cpu().numpy(), g_ref[k]) <= TOL, k
     for k in ("dA", "dD", "ddelta_bias"):
         assert norm_err(g_cut[k][c0:].cpu().numpy(), g_ref[k]) <= TOL, k
+
+
+def test_backward_cut_schedule_with_eight_states():
+    """The cut schedule with 8 states (two warps per block, so more blocks
+    per SM): the smallest whole number of 32-channel tiles for which the
+    workspace size asks for the cut area, then the cut run against the whole
+    run (bit-identical du, ddelta, dz, dh0)."""
+    lib = sss.load_library()
+    ck_bytes = lambda dim: sss.scan_checkpoints(1, dim, 8, 48, "cpu").numel() * 4
+
+    def need(dim):
+        a = sss.ScanBwdArgs()
+        a.batch, a.dim, a.dstate, a.seqlen = 1, dim, 8, 48
+        a.in_dtype = sss.MSS_BF16
+        for f in ("u", "delta", "A", "B", "C", "dy", "du", "ddelta", "dA", "dB", "dC"):
+            setattr(a, f, 256)
+        n = ctypes.c_size_t(0)
+        assert lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == sss.MSS_OK
+        return n.value
+
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    dim = next(32 * k for k in range(sms, 32 * sms) if need(32 * k) > ck_bytes(32 * k))
+    w = workloads.custom(1, dim, 8, 48, in_dtype="bf16", has_z=True, a_noise=0.1)
+    inp = workloads.make_inputs(w, seed=5910, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5911)
+    inp["h0"] = torch.randn(1, dim, 8, generator=gen, device="cuda")
+    dy = torch.randn(1, dim, 48, generator=gen, device="cuda")
+    d_last = torch.randn(1, dim, 8, generator=gen, device="cuda")
+    whole_ws = torch.empty(ck_bytes(dim), dtype=torch.uint8, device="cuda")
+    g_whole = _bwd_ws(inp, dy, d_last, whole_ws)
+    g_cut = _bwd_ws(inp, dy, d_last, None)
+    for k in ("du", "ddelta", "dz", "dh0"):
+        assert torch.equal(g_cut[k], g_whole[k]), k
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        assert norm_err(g_cut[k].cpu().numpy(), g_whole[k].double().cpu().numpy()) <= 1e-5, k
