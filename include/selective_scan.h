@@ -352,7 +352,8 @@ typedef struct mss_scan_bwd_args {
  * resident blocks is at most half full cuts the tiles of that wave in two
  * at their middle 16-step block: the first part's forward sweep, the second
  * part's sweeps and the first part's reverse sweep run as separate work
- * items (taken by ticket, spread over the schedule), handing the state and
+ * items (taken by ticket: the first pieces, every whole tile, the other
+ * pieces), handing the state and
  * the adjoint over through the workspace; du, ddelta and dz are
  * bit-identical to the uncut schedule.  A workspace with the checkpoints
  * but not that area runs every tile whole.  Packed sequences are not cut.
