@@ -177,7 +177,9 @@ typedef struct mss_scan_args {
      split sequence reads the step before it from u and B.  0: the Euler
      update above.  Not combined with cu_seqlens (MSS_ERR_UNSUPPORTED). */
   int trapezoid;
-  /* NULL, or an output of mss_scan_bwd_workspace_size() bytes that receives
+  /* NULL, or an output of 64 bytes per 16 steps of every channel (for
+     dstate <= 16: tiles * ceil(seqlen / 16) * 4 * groups * 32 floats, the
+     checkpoint part of mss_scan_bwd_workspace_size()) that receives
      the state of every channel at the start of every 16-step block, in the
      layout mamba_selective_scan_bwd reads (mss_scan_bwd_args.checkpoints):
      fp32 [tile][block][state][lane] with tile = b * ceil(dim / 32) + d / 32,

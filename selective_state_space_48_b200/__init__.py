@@ -604,8 +604,8 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
 
 
 def scan_checkpoints(batch, dim, dstate, seqlen, device):
-    """A buffer for the forward scan's checkpoints (float32, the size
-    ``mss_scan_bwd_workspace_size`` reports)."""
+    """A buffer for the forward scan's checkpoints (float32, the checkpoint
+    part of what ``mss_scan_bwd_workspace_size`` reports)."""
     groups = (dstate + 3) // 4
     groups = 1 if groups <= 1 else (2 if groups == 2 else 4)
     tiles = batch * ((dim + 31) // 32)
