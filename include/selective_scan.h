@@ -347,9 +347,10 @@ typedef struct mss_scan_bwd_args {
   int64_t num_seqs;
 } mss_scan_bwd_args;
 
-/* Workspace bytes of the backward scan: the state checkpoints (64 bytes per
- * 16 steps of every channel, for dstate <= 16; none when `checkpoints` is
- * given), then the area of the cut schedule when it applies on the current
+/* Workspace bytes of the backward scan: the states of its own forward sweep
+ * (64 bytes per 16 steps of every channel, for dstate <= 16, twice over --
+ * block starts and mid-block -- without cu_seqlens; none when `checkpoints`
+ * is given), then the area of the cut schedule when it applies on the current
  * device.  A launch of batch * ceil(dim / 32) blocks whose last wave of
  * resident blocks is at most half full cuts the tiles of that wave in two
  * at their middle 16-step block: the first part's forward sweep, the second

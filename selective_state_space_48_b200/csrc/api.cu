@@ -410,8 +410,10 @@ mss_status mss_scan_bwd_workspace_size(const mss_scan_bwd_args *a, size_t *bytes
   const mss_status st = check_bwd_args(a);
   if (st != MSS_OK) return st;
   const int64_t tiles = a->batch * ((a->dim + kBwdChannels - 1) / kBwdChannels);
-  *bytes = (a->checkpoints ? 0 : scan_bwd_workspace_bytes(tiles, a->seqlen, a->dstate)) +
-           bwd_cut_of(a).bytes;
+  // the own sweep of ordinary sequences keeps a second array of states at
+  // mid-block
+  const size_t arrays = a->checkpoints ? 0 : (a->cu_seqlens ? 1 : 2);
+  *bytes = arrays * scan_bwd_workspace_bytes(tiles, a->seqlen, a->dstate) + bwd_cut_of(a).bytes;
   return MSS_OK;
 }
 
@@ -420,8 +422,8 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   const mss_status st = check_bwd_args(a);
   if (st != MSS_OK) return st;
   const int64_t ntiles = a->batch * ((a->dim + kBwdChannels - 1) / kBwdChannels);
-  const size_t ck_bytes =
-      a->checkpoints ? 0 : scan_bwd_workspace_bytes(ntiles, a->seqlen, a->dstate);
+  const size_t ck_array = scan_bwd_workspace_bytes(ntiles, a->seqlen, a->dstate);
+  const size_t ck_bytes = a->checkpoints ? 0 : (a->cu_seqlens ? 1 : 2) * ck_array;
   if (!a->checkpoints &&
       (!a->workspace || a->workspace_bytes < ck_bytes || !aligned(a->workspace, 256)))
     return MSS_ERR_WORKSPACE;
@@ -458,6 +460,10 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   p.dh0 = a->dh0;
   p.ckpt = a->checkpoints ? const_cast<float *>(a->checkpoints)
                           : static_cast<float *>(a->workspace);
+  p.ckpt_mid = (a->checkpoints || a->cu_seqlens)
+                   ? nullptr
+                   : reinterpret_cast<float *>(static_cast<unsigned char *>(a->workspace) +
+                                               ck_array);
   p.ckpt_given = a->checkpoints ? 1 : 0;
   p.ch_tiles = static_cast<int>((a->dim + kBwdChannels - 1) / kBwdChannels);
   p.tiles = a->batch * p.ch_tiles;

@@ -229,7 +229,7 @@ __device__ void wait_flag(const unsigned *f, unsigned *status) {
   __threadfence();
 }
 
-template <typename InT, int G, bool VARLEN, bool CUT>
+template <typename InT, int G, bool VARLEN, bool CUT, bool MID>
 __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     scan_bwd_kernel(const BwdParams p) {
   using Sm = BwdSmem<G>;
@@ -294,6 +294,10 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   // state 4g + i of lane at the start of block k:
   // ckpt[(k * NP + 4g + i) * CH + lane] (coalesced per warp)
   float *ckpt = p.ckpt + tile * static_cast<int64_t>(nblk) * NP * CH;
+  // with its own forward sweep the kernel also keeps the state after the
+  // 8th step of every block, so the reverse sweep recomputes each half of a
+  // block from its own start
+  float *ckmid = MID ? p.ckpt_mid + tile * static_cast<int64_t>(nblk) * NP * CH : nullptr;
   // a second part with its own forward sweep starts from the state the
   // first part's sweep left at block kb0
   if (CUT && wk.piece == 1 && !p.ckpt_given) {
@@ -616,7 +620,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   // (the test is uniform over the block); the ordinary kernel keeps its own
   // copy of the loop, whose register allocation a shared generic lambda
   // changed (0.7 % slower).
-  auto fwd_block = [&](const BwdTiles<G> &T) {
+  auto fwd_block = [&](const BwdTiles<G> &T, int k) {
     if constexpr (VARLEN) {
       auto run = [&](auto masked) {
 #pragma unroll
@@ -651,6 +655,15 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
           h2[0] = __ffma2_rn(e0, h2[0], __fmul2_rn(U2, make_float2(b4.x, b4.y)));
           h2[1] = __ffma2_rn(e1, h2[1], __fmul2_rn(U2, make_float2(b4.z, b4.w)));
         }
+        if constexpr (MID) {
+          if (qd == 1) {  // the state entering step 8 of block k
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              ckmid[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q) * CH + lane] = h2[q].x;
+              ckmid[(static_cast<int64_t>(k) * NP + 4 * g + 2 * q + 1) * CH + lane] = h2[q].y;
+            }
+          }
+        }
       }
     }
   };
@@ -682,7 +695,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         fstage_commit(k + 1, (k + 1) & 1, s.tl[(k + 1) & 1]);
         put_mask(k + 1, s.tl[(k + 1) & 1]);
       }
-      fwd_block(s.tl[k & 1]);
+      fwd_block(s.tl[k & 1], k);
     }
     __syncthreads();
   } else if (sweep) {
@@ -695,7 +708,7 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
       put_ckpt(k);
       __syncthreads();
       if (k + 1 < kb1) fetch_fwd(k + 1, rf);  // in flight while block k is computed
-      fwd_block(T);
+      fwd_block(T, k);
       // no barrier here: block k + 1 is committed to the other tile set, and
       // this set is next written two blocks on, after the next barrier
     }
@@ -743,12 +756,17 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     }
   }
   // the checkpoint of the block after the current one is read a block early
-  float2 hnext[2];
+  float2 hnext[2], hnextm[2];
 #pragma unroll
-  for (int q = 0; q < 2; ++q)
+  for (int q = 0; q < 2; ++q) {
     hnext[q] = make_float2(
         ckpt[(static_cast<int64_t>(kb1 - 1) * NP + 4 * g + 2 * q) * CH + lane],
         ckpt[(static_cast<int64_t>(kb1 - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
+    if constexpr (MID)
+      hnextm[q] = make_float2(
+          ckmid[(static_cast<int64_t>(kb1 - 1) * NP + 4 * g + 2 * q) * CH + lane],
+          ckmid[(static_cast<int64_t>(kb1 - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
+  }
   Raw raw;
   if (kStaged) {
     stage_fetch(kb1 - 1);
@@ -772,14 +790,20 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
     const int64_t t0 = static_cast<int64_t>(k) * TB;
     const int nt = static_cast<int>(min(static_cast<int64_t>(TB), L - t0));
     BwdTiles<G> &T = s.tl[k & 1];
-    float2 hc[2];
+    float2 hc[2], hcm[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       hc[q] = hnext[q];
-      if (k > kb0)
+      if constexpr (MID) hcm[q] = hnextm[q];
+      if (k > kb0) {
         hnext[q] = make_float2(
             ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q) * CH + lane],
             ckpt[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
+        if constexpr (MID)
+          hnextm[q] = make_float2(
+              ckmid[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q) * CH + lane],
+              ckmid[(static_cast<int64_t>(k - 1) * NP + 4 * g + 2 * q + 1) * CH + lane]);
+      }
     }
     __syncthreads();
 
@@ -861,8 +885,15 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
         else
           recompute(std::false_type{});
       } else {
+        // with the mid-block states, the later half starts at step 8
+        if constexpr (MID) {
+          if (half == 1) {
+            hh[0] = hcm[0];
+            hh[1] = hcm[1];
+          }
+        }
 #pragma unroll
-        for (int qd = 0; qd < tb / 4 + 2; ++qd) {
+        for (int qd = MID ? tb / 4 : 0; qd < tb / 4 + 2; ++qd) {
           const float4 dl4 = ld4(&T.dl[lane * ROW + 4 * qd]), du4 = ld4(&T.du[lane * ROW + 4 * qd]);
           float4 ds4 = make_float4(0.f, 0.f, 0.f, 0.f);
           if (4 * qd >= tb) ds4 = ld4(&T.ds[lane * ROW + 4 * qd]);
@@ -1047,9 +1078,9 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   }
 }
 
-template <typename InT, int G, bool VARLEN, bool CUT>
+template <typename InT, int G, bool VARLEN, bool CUT, bool MID>
 cudaError_t launch_kernel(const BwdParams &p, cudaStream_t stream) {
-  auto kern = scan_bwd_kernel<InT, G, VARLEN, CUT>;
+  auto kern = scan_bwd_kernel<InT, G, VARLEN, CUT, MID>;
   const int smem = static_cast<int>(sizeof(BwdSmem<G>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1059,21 +1090,25 @@ cudaError_t launch_kernel(const BwdParams &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// The cut schedule has its own instantiation (ordinary scans only), so the
-// kernel of whole tiles keeps its code.
+// The cut schedule and the mid-block checkpoints of the backward's own
+// sweep have their own instantiations (ordinary scans only), so the kernel
+// that starts from the forward's checkpoints keeps its code.
 template <typename InT, int G, bool VARLEN>
 cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
   if constexpr (!VARLEN) {
-    if (p.ncut) return launch_kernel<InT, G, false, true>(p, stream);
+    if (p.ckpt_mid)
+      return p.ncut ? launch_kernel<InT, G, false, true, true>(p, stream)
+                    : launch_kernel<InT, G, false, false, true>(p, stream);
+    if (p.ncut) return launch_kernel<InT, G, false, true, false>(p, stream);
   }
-  return launch_kernel<InT, G, VARLEN, false>(p, stream);
+  return launch_kernel<InT, G, VARLEN, false, false>(p, stream);
 }
 
 template <typename InT, int G>
 int blocks_per_sm() {
   int n = 0;
   const int smem = static_cast<int>(sizeof(BwdSmem<G>));
-  auto kern = scan_bwd_kernel<InT, G, false, false>;
+  auto kern = scan_bwd_kernel<InT, G, false, false, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * G, smem) != cudaSuccess)

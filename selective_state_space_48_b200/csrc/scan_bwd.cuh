@@ -25,6 +25,8 @@ struct BwdParams {
   const float *d_last;
   float *du, *ddelta, *dA, *dB, *dC, *dD, *dz, *ddelta_bias, *dh0;
   float *ckpt;      // workspace: one state per channel and 16-step block
+  float *ckpt_mid;  // own forward sweep of ordinary sequences: the state
+                    // entering step 8 of every block (same layout), else null
   int ckpt_given;   // ckpt already holds the forward scan's states
   int ch_tiles;     // ceil(dim / kBwdChannels)
   int64_t tiles;    // batch * ch_tiles
@@ -62,7 +64,8 @@ BwdCut plan_bwd_cut(const BwdParams &p, int in_bf16);
 // Warps per block (state groups of 4): 1, 2 or 4.
 int bwd_groups(int64_t dstate);
 
-// Workspace bytes of the state checkpoints.
+// Workspace bytes of the state checkpoints (one array; the backward's own
+// sweep of ordinary sequences keeps two, the second at mid-block).
 size_t scan_bwd_workspace_bytes(int64_t tiles, int64_t seqlen, int64_t dstate);
 
 // dA, dB, dC, dD and ddelta_bias are accumulated with atomics: the caller

@@ -226,11 +226,16 @@ def _bwd_args(**kw):
     return a
 
 
-def test_bwd_workspace_is_one_state_per_block():
+def test_bwd_workspace_is_two_states_per_block():
     lib = sss.load_library()
     n = ctypes.c_size_t(0)
     assert lib.mss_scan_bwd_workspace_size(ctypes.byref(_bwd_args()), ctypes.byref(n)) == sss.MSS_OK
-    # 2 batch rows x 2 channel tiles x 63 blocks x 16 states x 32 lanes x 4 B
+    # (block start, mid-block) x 2 batch rows x 2 channel tiles x 63 blocks
+    # x 16 states x 32 lanes x 4 B
+    assert n.value == 2 * 2 * 2 * 63 * 16 * 32 * 4
+    # packed sequences keep the block starts only
+    a = _bwd_args(cu_seqlens=0x10000, num_seqs=2)
+    assert lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == sss.MSS_OK
     assert n.value == 2 * 2 * 63 * 16 * 32 * 4
 
 
@@ -258,13 +263,20 @@ def test_bwd_missing_workspace_is_reported():
 
 
 def test_checkpoint_buffer_matches_the_workspace_size():
+    """The backward's own sweep keeps two arrays of states in the shape of
+    the forward's checkpoint buffer (block starts and mid-block); with the
+    forward's checkpoints it needs no workspace here (no device to plan a
+    cut schedule for)."""
     lib = sss.load_library()
     for N in (1, 4, 5, 9, 12, 16):
         a = _bwd_args(dstate=N, seqlen=1000)
         n = ctypes.c_size_t(0)
         assert lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == sss.MSS_OK
         buf = sss.scan_checkpoints(2, 40, N, 1000, "cpu")
-        assert buf.numel() * 4 == n.value, N
+        assert 2 * buf.numel() * 4 == n.value, N
+        a.checkpoints = 256
+        assert lib.mss_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == sss.MSS_OK
+        assert n.value == 0, N
 
 
 def _ssd_args(**kw):
