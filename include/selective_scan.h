@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MSS_ABI_VERSION 10
+#define MSS_ABI_VERSION 11
 
 typedef enum {
   MSS_OK = 0,
@@ -177,13 +177,15 @@ typedef struct mss_scan_args {
      split sequence reads the step before it from u and B.  0: the Euler
      update above.  Not combined with cu_seqlens (MSS_ERR_UNSUPPORTED). */
   int trapezoid;
-  /* NULL, or an output of 64 bytes per 16 steps of every channel (for
-     dstate <= 16: tiles * ceil(seqlen / 16) * 4 * groups * 32 floats, the
-     checkpoint part of mss_scan_bwd_workspace_size()) that receives
-     the state of every channel at the start of every 16-step block, in the
-     layout mamba_selective_scan_bwd reads (mss_scan_bwd_args.checkpoints):
-     fp32 [tile][block][state][lane] with tile = b * ceil(dim / 32) + d / 32,
-     block = t / 16, lane = d % 32, and states padded to 4, 8 or 16.  A scan
+  /* NULL, or an output of 128 bytes per 16 steps of every channel (for
+     dstate <= 16: 2 * tiles * ceil(seqlen / 16) * 4 * groups * 32 floats,
+     the checkpoint part of mss_scan_bwd_workspace_size()) that receives two
+     arrays of states in the layout mamba_selective_scan_bwd reads
+     (mss_scan_bwd_args.checkpoints): the state of every channel at the
+     start of every 16-step block, then the state entering its 9th step,
+     each fp32 [tile][block][state][lane] with tile = b * ceil(dim / 32) +
+     d / 32, block = t / 16, lane = d % 32, and states padded to 4, 8 or
+     16.  A scan
      that writes checkpoints is never split into chunks; not combined with
      cu_seqlens or trapezoid (MSS_ERR_UNSUPPORTED). */
   float *checkpoints;
@@ -349,8 +351,8 @@ typedef struct mss_scan_bwd_args {
 
 /* Workspace bytes of the backward scan: the states of its own forward sweep
  * (64 bytes per 16 steps of every channel, for dstate <= 16, twice over --
- * block starts and mid-block -- without cu_seqlens; none when `checkpoints`
- * is given), then the area of the cut schedule when it applies on the current
+ * block starts and mid-block -- without cu_seqlens, once with; none when
+ * `checkpoints` is given), then the area of the cut schedule when it applies on the current
  * device.  A launch of batch * ceil(dim / 32) blocks whose last wave of
  * resident blocks is at most half full cuts the tiles of that wave in two
  * at their middle 16-step block: the first part's forward sweep, the second

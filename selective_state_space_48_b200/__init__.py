@@ -26,7 +26,7 @@ from . import builder as _build
 
 LIB_PATH = _build.LIB_PATH
 
-ABI_VERSION = 10  # MSS_ABI_VERSION of include/selective_scan.h
+ABI_VERSION = 11  # MSS_ABI_VERSION of include/selective_scan.h
 
 MSS_OK = 0
 MSS_ERR_INVALID_ARG = 1
@@ -610,7 +610,8 @@ def scan_checkpoints(batch, dim, dstate, seqlen, device):
     groups = 1 if groups <= 1 else (2 if groups == 2 else 4)
     tiles = batch * ((dim + 31) // 32)
     nblk = (seqlen + 15) // 16
-    return torch.empty(tiles * nblk * 4 * groups * 32, dtype=torch.float32,
+    # two arrays: the states at every block's start and entering its step 8
+    return torch.empty(2 * tiles * nblk * 4 * groups * 32, dtype=torch.float32,
                        device=device)
 
 

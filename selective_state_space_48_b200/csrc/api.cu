@@ -218,10 +218,9 @@ void fill_scan_params(const mss_scan_args *a, const Plan &pl, ScanParams *p) {
   p->ext_B = ext(p->sB, a->dstate);
   p->ext_C = ext(p->sC, a->dstate);
   p->ext_y = ext(p->sy, a->dim);
-  p->ext_ckpt = a->checkpoints
-                    ? static_cast<int64_t>(scan_bwd_workspace_bytes(pl.tiles, a->seqlen, a->dstate) /
-                                           sizeof(float))
-                    : 0;
+  // two arrays: block starts and mid-block states
+  const size_t ck = scan_bwd_workspace_bytes(pl.tiles, a->seqlen, a->dstate);
+  p->ext_ckpt = a->checkpoints ? static_cast<int64_t>(2 * ck / sizeof(float)) : 0;
 }
 
 }  // namespace
@@ -460,10 +459,11 @@ mss_status mamba_selective_scan_bwd(const mss_scan_bwd_args *a, void *stream) {
   p.dh0 = a->dh0;
   p.ckpt = a->checkpoints ? const_cast<float *>(a->checkpoints)
                           : static_cast<float *>(a->workspace);
-  p.ckpt_mid = (a->checkpoints || a->cu_seqlens)
-                   ? nullptr
-                   : reinterpret_cast<float *>(static_cast<unsigned char *>(a->workspace) +
-                                               ck_array);
+  // the second array: the states entering step 8 of every block (written
+  // by the backward's own sweep, or by the forward scan with its checkpoints)
+  p.ckpt_mid = a->cu_seqlens ? nullptr
+                             : reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(p.ckpt) +
+                                                         ck_array);
   p.ckpt_given = a->checkpoints ? 1 : 0;
   p.ch_tiles = static_cast<int>((a->dim + kBwdChannels - 1) / kBwdChannels);
   p.tiles = a->batch * p.ch_tiles;

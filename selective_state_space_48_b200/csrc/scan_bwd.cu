@@ -294,9 +294,10 @@ __global__ void __launch_bounds__(32 * G, 12 / G)  // 3 blocks of 4 warps per SM
   // state 4g + i of lane at the start of block k:
   // ckpt[(k * NP + 4g + i) * CH + lane] (coalesced per warp)
   float *ckpt = p.ckpt + tile * static_cast<int64_t>(nblk) * NP * CH;
-  // with its own forward sweep the kernel also keeps the state after the
-  // 8th step of every block, so the reverse sweep recomputes each half of a
-  // block from its own start
+  // ordinary scans also have the state after the 8th step of every block
+  // (kept by the own forward sweep, or written by the forward scan with its
+  // checkpoints), so the reverse sweep recomputes each half of a block from
+  // its own start
   float *ckmid = MID ? p.ckpt_mid + tile * static_cast<int64_t>(nblk) * NP * CH : nullptr;
   // a second part with its own forward sweep starts from the state the
   // first part's sweep left at block kb0
@@ -1090,25 +1091,24 @@ cudaError_t launch_kernel(const BwdParams &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// The cut schedule and the mid-block checkpoints of the backward's own
-// sweep have their own instantiations (ordinary scans only), so the kernel
-// that starts from the forward's checkpoints keeps its code.
+// Ordinary scans read the mid-block states (from the backward's own sweep
+// or the forward's checkpoints), and the cut schedule has its own
+// instantiation; packed sequences keep block starts only and are not cut.
 template <typename InT, int G, bool VARLEN>
 cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
   if constexpr (!VARLEN) {
-    if (p.ckpt_mid)
-      return p.ncut ? launch_kernel<InT, G, false, true, true>(p, stream)
-                    : launch_kernel<InT, G, false, false, true>(p, stream);
-    if (p.ncut) return launch_kernel<InT, G, false, true, false>(p, stream);
+    return p.ncut ? launch_kernel<InT, G, false, true, true>(p, stream)
+                  : launch_kernel<InT, G, false, false, true>(p, stream);
+  } else {
+    return launch_kernel<InT, G, true, false, false>(p, stream);
   }
-  return launch_kernel<InT, G, VARLEN, false, false>(p, stream);
 }
 
 template <typename InT, int G>
 int blocks_per_sm() {
   int n = 0;
   const int smem = static_cast<int>(sizeof(BwdSmem<G>));
-  auto kern = scan_bwd_kernel<InT, G, false, false, false>;
+  auto kern = scan_bwd_kernel<InT, G, false, false, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * G, smem) != cudaSuccess)

@@ -25,8 +25,8 @@ struct BwdParams {
   const float *d_last;
   float *du, *ddelta, *dA, *dB, *dC, *dD, *dz, *ddelta_bias, *dh0;
   float *ckpt;      // workspace: one state per channel and 16-step block
-  float *ckpt_mid;  // own forward sweep of ordinary sequences: the state
-                    // entering step 8 of every block (same layout), else null
+  float *ckpt_mid;  // ordinary sequences: the state entering step 8 of
+                    // every block (same layout); null with packed sequences
   int ckpt_given;   // ckpt already holds the forward scan's states
   int ch_tiles;     // ceil(dim / kBwdChannels)
   int64_t tiles;    // batch * ch_tiles

@@ -412,14 +412,15 @@ struct Scan {
   // Trapezoidal update: the input term of step t gains the previous input,
   // decayed over the step, e_t (Delta_t u_{t-1} / 2) B_{t-1}[n]; bprev holds
   // B_{t-1}[n] of this lane's states across quads and blocks.
+  // steps 4 q0 .. 4 q1 - 1 of the block (the whole block: 0, TB / 4)
   __device__ void scan(int set, int g, int lane, float (&h)[4],
                        const float2 (&al2)[4], float &dsum, bool split,
-                       float (&bprev)[4]) const {
+                       float (&bprev)[4], int q0 = 0, int q1 = TB / 4) const {
     const float *sDelta = fset(set, Lay::oDelta), *sDu = fset(set, Lay::oDu);
     const float *sB = fset(set, Lay::oB), *sC = fset(set, Lay::oC);
     float *sPart = fpart(set);
 #pragma unroll
-    for (int q = 0; q < TB / 4; ++q) {
+    for (int q = q0; q < q1; ++q) {
       const float4 dl = *reinterpret_cast<const float4 *>(&sDelta[lane * ROW + 4 * q]);
       const float4 du = *reinterpret_cast<const float4 *>(&sDu[lane * ROW + 4 * q]);
       const float2 dl01 = make_float2(dl.x, dl.y), dl23 = make_float2(dl.z, dl.w);
@@ -485,8 +486,11 @@ constexpr int kPartFree = 3;    // epi -> scan: y shares of a block consumed
 constexpr int kBarEpi = 1;      // named barrier of the epilogue warps only
 constexpr uint64_t kHandoffWaitNs = 2000000000ull;
 
+// (checkpoint mode: 4 blocks per SM asked for, so the extra stores of the
+// mid-block states do not cost a resident block; the other modes give ptxas
+// no minimum, which keeps their register allocation)
 template <typename InT, typename OutT, int G, bool TMA, int MODE>
-__global__ void __launch_bounds__(32 * (G + kAuxWarps))
+__global__ void __launch_bounds__(32 * (G + kAuxWarps), MODE == kModeCkpt ? 4 : 0)
     scan_fwd_kernel(const ScanParams p, const __grid_constant__ TmaMaps maps) {
   using S = Scan<InT, OutT, G, TMA, MODE>;
   constexpr bool VARLEN = S::VARLEN;
@@ -594,15 +598,26 @@ __global__ void __launch_bounds__(32 * (G + kAuxWarps))
       wait_hand(kTilesReady, s);
       if (i >= 2) wait_hand(kPartFree, s);
       if (CKPT) {
-        // state before block i for the backward pass (unsplit plans only)
+        // state before block i for the backward pass (unsplit plans only),
+        // and in the second array the state entering its step 8
         const int64_t ci = ((item * nblk + i) * NP + 4 * g) * static_cast<int64_t>(CH) + lane;
+        const int64_t arr = p.tiles * static_cast<int64_t>(nblk) * NP * CH;
         float *ck = p.ckpt_out + ci;
-        if (dbg_index_ok(ci + 3 * CH, p.ext_ckpt, p.status)) {
+        const bool ok = dbg_index_ok(ci + 3 * CH, p.ext_ckpt, p.status) &&
+                        dbg_index_ok(arr + ci + 3 * CH, p.ext_ckpt, p.status);
+        if (ok) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) ck[j * CH] = h[j];
         }
+        sc.scan(s, g, lane, h, al2, dsum, split, bprev, 0, TB / 8);
+        if (ok) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ck[arr + j * CH] = h[j];
+        }
+        sc.scan(s, g, lane, h, al2, dsum, split, bprev, TB / 8, TB / 4);
+      } else {
+        sc.scan(s, g, lane, h, al2, dsum, split, bprev);
       }
-      sc.scan(s, g, lane, h, al2, dsum, split, bprev);
       if (i + 2 < nblk) mbar_arrive(sc.hand(kTilesFree, s));
       mbar_arrive(sc.hand(kPartReady, s));
     }

@@ -250,7 +250,7 @@ def test_backward_cut_schedule(dt):
     dy = torch.randn(1, dim, 100, generator=gen, device="cuda")
     d_last = torch.randn(1, dim, 16, generator=gen, device="cuda")
     # the own sweep's two arrays of states, without the cut schedule's area
-    ck_bytes = 2 * sss.scan_checkpoints(1, dim, 16, 100, "cpu").numel() * 4
+    ck_bytes = sss.scan_checkpoints(1, dim, 16, 100, "cpu").numel() * 4
     whole_ws = torch.empty(ck_bytes, dtype=torch.uint8, device="cuda")
     g_whole = _bwd_ws(inp, dy, d_last, whole_ws)
     g_cut = _bwd_ws(inp, dy, d_last, None)   # allocates checkpoints + cut area
@@ -293,7 +293,7 @@ def test_backward_cut_schedule_with_eight_states():
     workspace size asks for the cut area, then the cut run against the whole
     run (bit-identical du, ddelta, dz, dh0)."""
     lib = sss.load_library()
-    ck_bytes = lambda dim: 2 * sss.scan_checkpoints(1, dim, 8, 48, "cpu").numel() * 4
+    ck_bytes = lambda dim: sss.scan_checkpoints(1, dim, 8, 48, "cpu").numel() * 4
 
     def need(dim):
         a = sss.ScanBwdArgs()

@@ -1,11 +1,12 @@
 """Forward-scan checkpoints for the backward pass (needs a GPU).
 
 With mss_scan_args.checkpoints the forward scan also writes the state of
-every channel at the start of every 16-step block, and the backward pass
-starts from them instead of its own forward sweep.  Checked: the
-checkpoints are the oracle's state after the first 16 k steps (its last
-state of the prefix); y does not change; the backward from checkpoints
-matches the backward without them and the oracle.
+every channel at the start of every 16-step block and, in a second array,
+the state entering its 9th step; the backward pass starts from them
+instead of its own forward sweep.  Checked: the checkpoints are the
+oracle's state after the first 16 k (and 16 k + 8) steps (its last state
+of the prefix); y does not change; the backward from checkpoints matches
+the backward without them and the oracle.
 """
 import numpy as np
 import pytest
@@ -33,10 +34,11 @@ def test_checkpoints_are_the_prefix_states(N, dt):
     assert torch.equal(y1, y0)
     NP = 4 * {1: 1, 2: 2}.get((N + 3) // 4, 4)
     tiles, nblk = batch * ((dim + 31) // 32), (L + 15) // 16
-    c = ck.view(tiles, nblk, NP, 32).cpu().numpy()
+    c2 = ck.view(2, tiles, nblk, NP, 32).cpu().numpy()
     h = workloads.to_numpy_f64(inp)
-    for k in (0, 1, 5, nblk - 1):
-        t = 16 * k
+    for k, arr in ((0, 0), (1, 0), (5, 0), (nblk - 1, 0), (0, 1), (3, 1), (nblk - 2, 1)):
+        c = c2[arr]
+        t = 16 * k + 8 * arr
         if t == 0:
             want = h["h0"]
         else:
@@ -49,7 +51,7 @@ def test_checkpoints_are_the_prefix_states(N, dt):
             for d in range(dim):
                 tile = b * ((dim + 31) // 32) + d // 32
                 got[b, d] = c[tile, k, :N, d % 32]
-        assert norm_err(got, want) <= 2e-3, k
+        assert norm_err(got, want) <= 2e-3, (k, arr)
 
 
 def test_backward_from_checkpoints():
