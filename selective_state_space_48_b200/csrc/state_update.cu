@@ -60,21 +60,39 @@ __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p)
 // 16 states with the state, A, B and C 16-byte aligned: thread 4 ch + qd
 // owns states 4 qd .. 4 qd + 3 of channel ch.  Idx is the index type: 32
 // bits when every state index fits (a 64-bit division per thread is a long
-// instruction sequence; the kernel is bound by issue, not by DRAM).
-template <typename InT, typename OutT, typename Idx>
+// instruction sequence; the kernel is bound by issue, not by DRAM).  With
+// ROWS the grid is (channel blocks, batch): the row is blockIdx.y and no
+// thread divides at all.
+template <typename InT, typename OutT, typename Idx, bool ROWS>
 __global__ void __launch_bounds__(256) state_update16_kernel(const UpdateParams p) {
-  const Idx gt = static_cast<Idx>(blockIdx.x) * static_cast<Idx>(blockDim.x) + threadIdx.x;
-  const Idx ch = gt >> 2;
-  const int qd = static_cast<int>(gt & 3);
   const Idx dim = static_cast<Idx>(p.dim);
-  // every thread of a channel takes part in the shuffles below
-  bool valid = static_cast<int64_t>(ch) < p.batch * p.dim;
+  Idx ch;
+  int qd;
+  bool valid;  // every thread of a channel takes part in the shuffles below
+  if constexpr (ROWS) {
+    const Idx dl = static_cast<Idx>(blockIdx.x) * 64 + (threadIdx.x >> 2);
+    qd = static_cast<int>(threadIdx.x & 3);
+    valid = dl < dim;
+    ch = static_cast<Idx>(blockIdx.y) * dim + dl;
+  } else {
+    const Idx gt = static_cast<Idx>(blockIdx.x) * static_cast<Idx>(blockDim.x) + threadIdx.x;
+    ch = gt >> 2;
+    qd = static_cast<int>(gt & 3);
+    valid = static_cast<int64_t>(ch) < p.batch * p.dim;
+  }
   if (valid && (!dbg_index_ok((ch + 1) * 16 - 1, p.batch * p.dim * 16, p.status) ||
                 !dbg_index_ok((ch % p.dim + 1) * 16 - 1, p.dim * 16, p.status) ||
                 !dbg_index_ok((ch / p.dim + 1) * 16 - 1, p.batch * 16, p.status)))
     valid = false;
   const Idx c = valid ? ch : 0;
-  const Idx b = c / dim, d = c - b * dim;
+  Idx b, d;
+  if constexpr (ROWS) {
+    b = valid ? static_cast<Idx>(blockIdx.y) : 0;
+    d = c - b * dim;
+  } else {
+    b = c / dim;
+    d = c - b * dim;
+  }
   float acc = 0.f, x = 0.f, gate = 1.f, skip = 0.f;
   if (valid) {
     // every load is issued before the arithmetic (the gate and skip inputs
@@ -123,11 +141,17 @@ cudaError_t launch_typed(const UpdateParams &p, cudaStream_t s) {
       aligned16(p.C)) {
     const unsigned grid = static_cast<unsigned>((4 * n + 255) / 256);
     // 32-bit indices when the largest state index (16 n) and the thread
-    // count (4 n, rounded up to the block) fit
-    if (16 * n + 256 <= static_cast<int64_t>(UINT32_MAX))
-      state_update16_kernel<InT, OutT, uint32_t><<<grid, 256, 0, s>>>(p);
-    else
-      state_update16_kernel<InT, OutT, int64_t><<<grid, 256, 0, s>>>(p);
+    // count (4 n, rounded up to the block) fit; a grid row per batch row
+    // when the batch fits the grid's y extent
+    const bool fits32 = 16 * n + 256 <= static_cast<int64_t>(UINT32_MAX);
+    if (fits32 && p.batch <= 65535) {
+      const dim3 g2(static_cast<unsigned>((p.dim + 63) / 64), static_cast<unsigned>(p.batch));
+      state_update16_kernel<InT, OutT, uint32_t, true><<<g2, 256, 0, s>>>(p);
+    } else if (fits32) {
+      state_update16_kernel<InT, OutT, uint32_t, false><<<grid, 256, 0, s>>>(p);
+    } else {
+      state_update16_kernel<InT, OutT, int64_t, false><<<grid, 256, 0, s>>>(p);
+    }
   } else {
     const unsigned grid = static_cast<unsigned>((n + 127) / 128);
     state_update_kernel<InT, OutT><<<grid, 128, 0, s>>>(p);

@@ -255,6 +255,30 @@ def test_state_update_matches_oracle(dt, N):
     assert norm_err(st.cpu(), st_ref) <= tol
 
 
+def test_state_update_past_the_grid_row_limit():
+    """More than 65535 batch rows: the 16-state kernel runs on a flat grid
+    of channels instead of one grid row per batch row; the result still
+    matches the oracle."""
+    batch, dim, N = 65537, 3, 16
+    g = torch.Generator(device="cuda")
+    g.manual_seed(93)
+    r = lambda *s: torch.randn(*s, generator=g, device="cuda")
+    state = r(batch, dim, N)
+    x, dtv, z = r(batch, dim), r(batch, dim), r(batch, dim)
+    A = -torch.rand(dim, N, generator=g, device="cuda") * 3
+    B, C = r(batch, N), r(batch, N)
+    D, bias = r(dim), r(dim) * 0.5
+    st_ref, y_ref = oracle.selective_state_update(
+        state.cpu().double().numpy(), x.cpu().double().numpy(), dtv.cpu().double().numpy(),
+        A.cpu().double().numpy(), B.cpu().double().numpy(), C.cpu().double().numpy(),
+        D=D.cpu().double().numpy(), z=z.cpu().double().numpy(),
+        dt_bias=bias.cpu().double().numpy())
+    st = state.clone()
+    y = sss.selective_state_update(st, x, dtv, A, B, C, D=D, z=z, dt_bias=bias)
+    assert norm_err(y.cpu(), y_ref) <= 1e-5
+    assert norm_err(st.cpu(), st_ref) <= 1e-5
+
+
 def test_state_update_with_unaligned_B_C_takes_the_general_path():
     """B and C starting off a 16-byte boundary use the scalar path; the
     result is the same as from aligned copies."""
