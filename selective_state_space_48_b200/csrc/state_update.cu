@@ -63,14 +63,15 @@ __global__ void __launch_bounds__(128) state_update_kernel(const UpdateParams p)
 // instruction sequence; the kernel is bound by issue, not by DRAM).  With
 // ROWS the grid is (channel blocks, batch): the row is blockIdx.y and no
 // thread divides at all.
+constexpr int kRowsThreads = 128;  // threads of a block on the (channel blocks, rows) grid
 template <typename InT, typename OutT, typename Idx, bool ROWS>
-__global__ void __launch_bounds__(256) state_update16_kernel(const UpdateParams p) {
+__global__ void __launch_bounds__(ROWS ? kRowsThreads : 256) state_update16_kernel(const UpdateParams p) {
   const Idx dim = static_cast<Idx>(p.dim);
   Idx ch;
   int qd;
   bool valid;  // every thread of a channel takes part in the shuffles below
   if constexpr (ROWS) {
-    const Idx dl = static_cast<Idx>(blockIdx.x) * 64 + (threadIdx.x >> 2);
+    const Idx dl = static_cast<Idx>(blockIdx.x) * (kRowsThreads / 4) + (threadIdx.x >> 2);
     qd = static_cast<int>(threadIdx.x & 3);
     valid = dl < dim;
     ch = static_cast<Idx>(blockIdx.y) * dim + dl;
@@ -145,8 +146,9 @@ cudaError_t launch_typed(const UpdateParams &p, cudaStream_t s) {
     // when the batch fits the grid's y extent
     const bool fits32 = 16 * n + 256 <= static_cast<int64_t>(UINT32_MAX);
     if (fits32 && p.batch <= 65535) {
-      const dim3 g2(static_cast<unsigned>((p.dim + 63) / 64), static_cast<unsigned>(p.batch));
-      state_update16_kernel<InT, OutT, uint32_t, true><<<g2, 256, 0, s>>>(p);
+      constexpr int cpb = kRowsThreads / 4;  // channels per block
+      const dim3 g2(static_cast<unsigned>((p.dim + cpb - 1) / cpb), static_cast<unsigned>(p.batch));
+      state_update16_kernel<InT, OutT, uint32_t, true><<<g2, kRowsThreads, 0, s>>>(p);
     } else if (fits32) {
       state_update16_kernel<InT, OutT, uint32_t, false><<<grid, 256, 0, s>>>(p);
     } else {
